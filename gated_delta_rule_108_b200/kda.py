@@ -1,0 +1,177 @@
+"""Thin ctypes binding of libkda_b200.so (declared in include/kda.h).
+
+Argument marshalling only: shapes and dtypes are read off torch tensors, output
+and workspace buffers are allocated with torch on the tensors' device, and the
+C entry points do all of the work on the current (or given) CUDA stream.  There
+is no CPU path: if the library is missing, every call raises :class:`KDAError`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libkda_b200.so"
+
+KDA_OK = 0
+_STATUS = {
+    0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA",
+    4: "KDA_ERR_TIMEOUT", 5: "KDA_ERR_WORKSPACE", 6: "KDA_ERR_BAD_SEQLENS",
+}
+KDA_F32, KDA_BF16 = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+class KDAError(RuntimeError):
+    """A libkda_b200 call returned a status other than KDA_OK."""
+
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+
+
+def library_path() -> str:
+    """Path of the in-tree CUDA library (built by ``__graft_entry__.build()``)."""
+    return os.environ.get("KDA_B200_LIB", os.path.join(_HERE, _LIB_NAME))
+
+
+def _declare(lib):
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    fp = ctypes.POINTER(f)
+    lib.kda_chunk_fwd_workspace_size.restype = sz
+    lib.kda_chunk_fwd_workspace_size.argtypes = [i, i, i, i, i, i, i, i]
+    lib.kda_chunk_fwd.restype = i
+    lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
+                                  vp, vp, vp, sz, vp]
+    lib.kda_recurrent_step.restype = i
+    lib.kda_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp]
+    lib.kda_workspace_status.restype = i
+    lib.kda_workspace_status.argtypes = [vp, sz, vp]
+    lib.kda_last_error.restype = ctypes.c_char_p
+    lib.kda_last_error.argtypes = []
+    lib.kda_version.restype = ctypes.c_char_p
+    lib.kda_version.argtypes = []
+    del fp
+    return lib
+
+
+def lib():
+    """Load (once) and return the ctypes handle of libkda_b200.so."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise KDAError(3, f"CUDA library not found at {path}; build it with "
+                                  "`python -c 'import __graft_entry__ as g; g.build()'`")
+            _lib = _declare(ctypes.CDLL(path))
+    return _lib
+
+
+def _check(status: int):
+    if status != KDA_OK:
+        raise KDAError(status, lib().kda_last_error().decode(errors="replace"))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KDA_F32
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream], device) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
+                             num_seqs: int, varlen: bool, dtype: torch.dtype) -> int:
+    """Workspace bytes ``chunk_fwd`` needs (``kda_chunk_fwd_workspace_size``)."""
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(lib().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs,
+                                                  int(bool(varlen)), code))
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
+              output_final_state: bool = True, o=None, final_state=None,
+              workspace=None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise KDA forward (``kda_chunk_fwd``).
+
+    q, k, log_alpha [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H];
+    initial_state [N, H, dk, dv] fp32 or None; cu_seqlens int32 [N+1] or None.
+    Returns (o [B, T, H, dv], final_state [N, H, dk, dv] or None).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    _need(log_alpha, "log_alpha", torch.float32)
+    _need(beta, "beta", torch.float32)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if initial_state is not None:
+        _need(initial_state, "initial_state", torch.float32)
+    if o is None:
+        o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    ws_bytes = chunk_fwd_workspace_size(B, T, H, dk, dv, N, cu_seqlens is not None, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    _check(lib().kda_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+        _ptr(cu_seqlens), B, T, H, dk, dv, N, _dtype_code(q), _ptr(o), _ptr(final_state),
+        _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream_ptr(stream, q.device)))
+    return o, final_state
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise and return the device status code left in ``workspace``."""
+    return int(lib().kda_workspace_status(_ptr(workspace), workspace.numel(),
+                                          _stream_ptr(stream, workspace.device)))
+
+
+def recurrent_step(q, k, v, log_alpha, beta, state, o=None, stream=None) -> torch.Tensor:
+    """One decoding step (``kda_recurrent_step``); ``state`` is updated in place.
+
+    q, k, log_alpha [B, H, dk]; v [B, H, dv]; beta [B, H]; state [B, H, dk, dv] fp32.
+    Returns o [B, H, dv] in q's dtype.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    _need(log_alpha, "log_alpha", torch.float32)
+    _need(beta, "beta", torch.float32)
+    _need(state, "state", torch.float32)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+    _check(lib().kda_recurrent_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state),
+        B, H, dk, dv, _dtype_code(q), _ptr(o), _stream_ptr(stream, q.device)))
+    return o

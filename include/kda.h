@@ -1,0 +1,133 @@
+/*
+ * kda.h -- C ABI of libkda_b200.so, the B200 (sm_100a) Kimi Delta Attention
+ * recurrence.
+ *
+ * The operation (daiw.net "Kimi Delta Attention", section "KDA 的更新式"), per
+ * sequence and head, with S in R^{d_k x d_v}:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = d_k^{-1/2} S_t^T q_t
+ *
+ * alpha_t in (0,1]^{d_k} is one decay per key channel (section
+ * "一、Diag(alpha_t)：通道级遗忘"), passed as log_alpha = log(alpha_t) <= 0;
+ * beta_t is a scalar write strength (section "二、I - beta k k^T：delta 规则").
+ * The step order -- forget per channel, predict on the decayed state, correct,
+ * write, read with d_k^{-1/2} -- is the one in news.bugfactory.tech/news/3610
+ * (KDA paragraph), which also names the two modes exposed here: a chunkwise
+ * mode for training and long prefill, and a token-by-token recurrent mode for
+ * decoding.  Keys and queries are used as given (the library does not
+ * normalise them).
+ *
+ * Conventions shared by every call:
+ *  - All tensor pointers are DEVICE pointers to contiguous row-major tensors,
+ *    16-byte aligned, owned by the caller.  The library allocates nothing and
+ *    never synchronises the stream (except kda_workspace_status).
+ *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream.  All work is enqueued asynchronously on it.
+ *  - Supported head sizes: d_k, d_v in {64, 128}.
+ *  - q, k, v and o have the element type `dtype` (fp32 or bf16); log_alpha,
+ *    beta and every state tensor are fp32.
+ *  - On any status other than KDA_OK nothing was enqueued, except for
+ *    KDA_ERR_CUDA (a launch failed) -- kda_last_error() has the message.
+ *  - Calls are thread-safe; the last-error message is per host thread.
+ */
+#ifndef KDA_B200_KDA_H
+#define KDA_B200_KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, B != 1 with cu_seqlens */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d_k = 96) */
+    KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = 4,       /* device status: a bounded wait inside a kernel gave up */
+    KDA_ERR_WORKSPACE = 5,     /* workspace missing, too small or misaligned */
+    KDA_ERR_BAD_SEQLENS = 6    /* device status: cu_seqlens not 0 .. T non-decreasing */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/*
+ * Bytes of device workspace kda_chunk_fwd needs for these sizes.  `varlen` is
+ * non-zero when cu_seqlens will be passed (then B must be 1 and num_seqs is
+ * the number of packed sequences); otherwise num_seqs is ignored (= B).
+ * Returns 0 for invalid sizes.
+ */
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
+                                    int num_seqs, int varlen, kda_dtype dtype);
+
+/*
+ * Chunkwise forward over whole sequences ("chunkwise" mode, news.bugfactory.tech
+ * /news/3610, KDA paragraph; chunks of 64 tokens as in the chunk-wise parallel
+ * scheme on the kongchang.com page, section "硬件效率的优化策略").  Inside a
+ * chunk the tokens are combined with matrix products (the WY/UT form of the
+ * product of transitions D_t - beta_t D_t k_t k_t^T); between chunks the state
+ * is carried.  The result equals the token-by-token recurrence above up to
+ * rounding.
+ *
+ *  q, k        [B, T, H, dk]   dtype
+ *  v           [B, T, H, dv]   dtype
+ *  log_alpha   [B, T, H, dk]   fp32, <= 0 (finite)
+ *  beta        [B, T, H]       fp32
+ *  initial_state [N, H, dk, dv] fp32, or NULL for zeros
+ *  cu_seqlens  [N + 1] int32 device array, or NULL.  With it, B must be 1 and
+ *              the T tokens hold N = num_seqs packed sequences,
+ *              cu_seqlens[0] = 0 <= ... <= cu_seqlens[N] = T (empty sequences
+ *              allowed).  Without it, N = B sequences of T tokens each.
+ *              The device checks the array; a bad one sets KDA_ERR_BAD_SEQLENS
+ *              in the workspace status and leaves o / final_state unwritten.
+ *  o           [B, T, H, dv]   dtype, written
+ *  final_state [N, H, dk, dv]  fp32, written, or NULL.  May alias
+ *              initial_state exactly (each state is read before it is written).
+ *  workspace   device scratch of at least kda_chunk_fwd_workspace_size(...)
+ *              bytes, 256-byte aligned; its contents on entry do not matter.
+ *              Calls that share one workspace must be ordered on one stream.
+ */
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         int B, int T, int H, int dk, int dv, int num_seqs,
+                         kda_dtype dtype, void* o, float* final_state,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One decoding step for B sequences ("fused recurrent" mode,
+ * news.bugfactory.tech/news/3610, KDA paragraph): each (sequence, head) state
+ * is read once, updated by one token and written back in place.
+ *
+ *  q, k        [B, H, dk]  dtype       v [B, H, dv] dtype
+ *  log_alpha   [B, H, dk]  fp32        beta [B, H] fp32
+ *  state_inout [B, H, dk, dv] fp32, updated in place
+ *  o           [B, H, dv]  dtype, written (must not alias the state)
+ */
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
+                              const float* log_alpha, const float* beta,
+                              float* state_inout, int B, int H, int dk, int dv,
+                              kda_dtype dtype, void* o, void* stream);
+
+/*
+ * Waits for `stream`, then reads the device status word that the last
+ * kda_chunk_fwd on this workspace left: KDA_OK, KDA_ERR_BAD_SEQLENS or
+ * KDA_ERR_TIMEOUT (or KDA_ERR_CUDA if the copy fails).  This is the only call
+ * that synchronises.
+ */
+kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char* kda_last_error(void);
+
+/* Library version string, e.g. "kda-b200 0.1.0 sm_100a". */
+const char* kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_KDA_H */
