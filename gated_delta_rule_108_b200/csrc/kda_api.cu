@@ -1,0 +1,213 @@
+// kda_api.cu -- the C ABI of libkda_b200 (declared in include/kda.h).
+//
+// Validates arguments, carves the caller's workspace, and enqueues the
+// kernels on the caller's stream.  Nothing here allocates device memory or
+// synchronises, except kda_workspace_status.
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/kda.h"
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local cudaEvent_t g_stage_events[4] = {nullptr, nullptr, nullptr, nullptr};
+thread_local bool g_stage_events_on = false;
+
+cudaError_t mark_stage(int i, cudaStream_t s) {
+    return g_stage_events_on ? cudaEventRecord(g_stage_events[i], s) : cudaSuccess;
+}
+
+kda_status fail(kda_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+kda_status ok() {
+    g_last_error.clear();
+    return KDA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool supported_dim(int d) { return d == 64 || d == 128; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace carve-up: [header 256 B][chunk_offsets (N+1) int32, 256-aligned][records].
+struct WsLayout {
+    size_t offsets_off, records_off, total;
+    size_t max_chunks;
+    int chunks_per_seq;
+};
+
+bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, kda_dtype dtype,
+               WsLayout& L) {
+    if (B < 0 || T < 0 || H <= 0 || !supported_dim(dk) || !supported_dim(dv)) return false;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return false;
+    const int N = varlen ? num_seqs : B;
+    if (N < 0 || (varlen && B != 1)) return false;
+    L.chunks_per_seq = (T + kda::kChunk - 1) / kda::kChunk;
+    if (varlen) {
+        // each sequence of length l holds ceil(l/64) <= (l + 63)/64 chunks
+        L.max_chunks = ((size_t)T + 63u * (size_t)N) / kda::kChunk;
+    } else {
+        L.max_chunks = (size_t)B * L.chunks_per_seq;
+    }
+    const size_t rec = kda::simt_record_bytes(dk, dv);
+    L.offsets_off = kda::kHeaderBytes;
+    L.records_off = round_up(L.offsets_off + sizeof(int32_t) * ((size_t)N + 1), 256);
+    L.total = L.records_off + rec * (size_t)H * L.max_chunks;
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int varlen,
+                                    kda_dtype dtype) {
+    WsLayout L;
+    if (!ws_layout(B, T, H, dk, dv, num_seqs, varlen != 0, dtype, L)) return 0;
+    return L.total;
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                         const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                         int B, int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype,
+                         void* o, float* final_state, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B < 0 || T < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d", B, T, H);
+    if (dk <= 0 || dv <= 0) return fail(KDA_ERR_INVALID_ARG, "bad head sizes dk=%d dv=%d", dk, dv);
+    if (!supported_dim(dk) || !supported_dim(dv))
+        return fail(KDA_ERR_UNSUPPORTED, "head sizes dk=%d dv=%d not in {64, 128}", dk, dv);
+    const bool varlen = cu_seqlens != nullptr;
+    if (varlen && B != 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (got B=%d)", B);
+    if (varlen && num_seqs < 0) return fail(KDA_ERR_INVALID_ARG, "num_seqs=%d < 0", num_seqs);
+    const int N = varlen ? num_seqs : B;
+    const size_t tokens = varlen ? (size_t)T : (size_t)B * T;
+    if (tokens * (size_t)H * (size_t)(dk > dv ? dk : dv) >= (size_t)1 << 31)
+        return fail(KDA_ERR_UNSUPPORTED, "B*T*H*d = %zu elements exceeds 2^31", tokens * H * (dk > dv ? dk : dv));
+    if (tokens > 0) {
+        if (!q || !k || !v || !log_alpha || !beta || !o)
+            return fail(KDA_ERR_INVALID_ARG, "null input/output pointer");
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o))
+            return fail(KDA_ERR_INVALID_ARG, "q/k/v/log_alpha/o must be 16-byte aligned");
+    }
+    if (initial_state && !aligned16(initial_state)) return fail(KDA_ERR_INVALID_ARG, "initial_state misaligned");
+    if (final_state && !aligned16(final_state)) return fail(KDA_ERR_INVALID_ARG, "final_state misaligned");
+    if (initial_state && final_state && initial_state != final_state) {
+        const char* a0 = (const char*)initial_state;
+        const char* b0 = (const char*)final_state;
+        const size_t bytes = (size_t)N * H * dk * dv * sizeof(float);
+        if (a0 < b0 + bytes && b0 < a0 + bytes)
+            return fail(KDA_ERR_INVALID_ARG, "initial_state and final_state overlap without being equal");
+    }
+    WsLayout L;
+    if (!ws_layout(B, T, H, dk, dv, num_seqs, varlen, dtype, L))
+        return fail(KDA_ERR_INVALID_ARG, "invalid sizes for the workspace layout");
+    if (!workspace) return fail(KDA_ERR_WORKSPACE, "workspace is null (need %zu bytes)", L.total);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(KDA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (workspace_bytes < L.total)
+        return fail(KDA_ERR_WORKSPACE, "workspace has %zu bytes, need %zu", workspace_bytes, L.total);
+
+    kda::ChunkArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
+    a.o = o; a.final_state = final_state;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.num_seqs = N;
+    a.bf16 = dtype == KDA_BF16;
+    a.scale = 1.0f / sqrtf((float)dk);
+    a.ws_header = workspace;
+    a.chunk_offsets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + L.offsets_off);
+    a.records = static_cast<char*>(workspace) + L.records_off;
+    a.max_chunks = L.max_chunks;
+    a.fixed_chunks_per_seq = L.chunks_per_seq;
+    a.stream = static_cast<cudaStream_t>(stream);
+
+    cudaError_t e = mark_stage(0, a.stream);
+    if (e == cudaSuccess) e = kda::launch_chunk_prep(a);
+    if (e == cudaSuccess) e = mark_stage(1, a.stream);
+    if (e == cudaSuccess) e = kda::launch_chunk_intra(a);
+    if (e == cudaSuccess) e = mark_stage(2, a.stream);
+    if (e == cudaSuccess) e = kda::launch_chunk_inter(a);
+    if (e == cudaSuccess) e = mark_stage(3, a.stream);
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_chunk_fwd launch failed: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* log_alpha,
+                              const float* beta, float* state_inout, int B, int H, int dk, int dv,
+                              kda_dtype dtype, void* o, void* stream) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B < 0 || H <= 0 || dk <= 0 || dv <= 0)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d H=%d dk=%d dv=%d", B, H, dk, dv);
+    if (!supported_dim(dk) || !supported_dim(dv))
+        return fail(KDA_ERR_UNSUPPORTED, "head sizes dk=%d dv=%d not in {64, 128}", dk, dv);
+    if ((size_t)B * H * dk * dv >= (size_t)1 << 40)
+        return fail(KDA_ERR_UNSUPPORTED, "state too large");
+    if (B > 0) {
+        if (!q || !k || !v || !log_alpha || !beta || !state_inout || !o)
+            return fail(KDA_ERR_INVALID_ARG, "null pointer");
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) ||
+            !aligned16(state_inout) || !aligned16(o))
+            return fail(KDA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+        const char* s0 = (const char*)state_inout;
+        const char* o0 = (const char*)o;
+        const size_t sb = (size_t)B * H * dk * dv * sizeof(float);
+        const size_t ob = (size_t)B * H * dv * (dtype == KDA_BF16 ? 2 : 4);
+        if (o0 < s0 + sb && s0 < o0 + ob) return fail(KDA_ERR_INVALID_ARG, "o aliases state_inout");
+    }
+    kda::DecodeArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.state = state_inout; a.o = o;
+    a.B = B; a.H = H; a.dk = dk; a.dv = dv;
+    a.bf16 = dtype == KDA_BF16;
+    a.scale = 1.0f / sqrtf((float)dk);
+    a.stream = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = kda::launch_decode(a);
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_recurrent_step launch failed: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace || workspace_bytes < (size_t)kda::kHeaderBytes)
+        return fail(KDA_ERR_WORKSPACE, "workspace missing or smaller than its header");
+    int st = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&st, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "reading workspace status: %s", cudaGetErrorString(e));
+    if (st == kda::kStatusOk) return ok();
+    if (st == kda::kStatusBadSeqlens) return fail(KDA_ERR_BAD_SEQLENS, "cu_seqlens rejected on the device");
+    if (st == kda::kStatusTimeout) return fail(KDA_ERR_TIMEOUT, "a bounded wait inside a kernel gave up");
+    return fail(KDA_ERR_CUDA, "unknown device status %d", st);
+}
+
+kda_status kda_set_stage_events(void* const* events, int count) {
+    if (!events) {
+        g_stage_events_on = false;
+        return ok();
+    }
+    if (count < 4) return fail(KDA_ERR_INVALID_ARG, "need at least 4 events, got %d", count);
+    for (int i = 0; i < 4; ++i) {
+        if (!events[i]) return fail(KDA_ERR_INVALID_ARG, "event %d is null", i);
+        g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+    }
+    g_stage_events_on = true;
+    return ok();
+}
+
+const char* kda_last_error(void) { return g_last_error.c_str(); }
+
+const char* kda_version(void) { return "kda-b200 0.1.0 sm_100a"; }
+
+}  // extern "C"

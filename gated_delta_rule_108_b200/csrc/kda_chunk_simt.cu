@@ -1,0 +1,486 @@
+// kda_chunk_simt.cu -- chunkwise KDA forward on CUDA cores in fp32 (sm_100a).
+//
+// This is the fp32 path of kda_chunk_fwd: every product is an fp32 FMA, so it
+// meets a 1e-4 relative error bound on fp32 inputs.  It implements the same
+// chunk algebra as the tensor-core path, in three launches:
+//
+//   K0 chunk_prep   -- resets the workspace status; for packed sequences it
+//                      checks cu_seqlens and builds the chunk table.
+//   K1 intra_chunk  -- one CTA per (chunk, head), all chunks in parallel.
+//   K2 inter_chunk  -- one CTA per (sequence, head, 32-wide value slice),
+//                      serial over the sequence's chunks, state in shared memory.
+//
+// Chunk algebra (derived by unrolling the update equation of the daiw.net page,
+// section "KDA 的更新式", over one chunk of L <= 64 tokens; S is the state
+// entering the chunk, g_r = sum_{i<=r} log_alpha_i per key channel):
+//
+//   Q~_r = q_r e^{g_r}   K~_r = k_r e^{g_r}   K^_r = k_r e^{g_{L-1} - g_r}
+//   A_{ri} = beta_r <k_r e^{g_r - g_m}, k_i e^{g_m - g_i}>   (i < r)
+//   P_{ri} =        <q_r e^{g_r - g_m}, k_i e^{g_m - g_i}>   (i <= r)
+//   T = (I + A)^{-1},  W = T diag(beta) K~,  U0 = T diag(beta) V
+//   U = U0 - W S,  O = dk^{-1/2} (Q~ S + P U),  S' = Diag(e^{g_{L-1}}) S + K^^T U
+//
+// g_m is the value at the middle token of the chunk; splitting the decay of
+// A and P there halves the largest exponent that is formed (products are
+// unchanged).  T is formed by forward substitution, one column per thread.
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace kda {
+namespace {
+
+// ---------------------------------------------------------------- K0 ------
+__global__ void __launch_bounds__(1024)
+chunk_prep_kernel(WsHeader* hdr, int32_t* chunk_offsets, const int32_t* __restrict__ cu,
+                  int N, int T, int fixed_num_chunks)
+{
+    __shared__ int warp_sums[32];
+    __shared__ int s_carry, s_bad;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (cu == nullptr) {
+        if (tid == 0) { hdr->status = kStatusOk; hdr->num_chunks = fixed_num_chunks; }
+        return;
+    }
+    if (tid == 0) { s_carry = 0; s_bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0; }
+    __syncthreads();
+    for (int base = 0; base < N; base += 1024) {
+        const int s = base + tid;
+        int cnt = 0;
+        if (s < N) {
+            const int len = cu[s + 1] - cu[s];
+            if (len < 0) atomicOr(&s_bad, 1);
+            cnt = len > 0 ? (len + kChunk - 1) / kChunk : 0;
+        }
+        int incl = cnt;  // inclusive warp scan
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (lane == 31) warp_sums[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int w = warp_sums[lane];
+            int wi = w;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, wi, off);
+                if (lane >= off) wi += y;
+            }
+            warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
+        }
+        __syncthreads();
+        const int excl = s_carry + warp_sums[warp] + incl - cnt;
+        if (s < N) chunk_offsets[s] = excl;
+        __syncthreads();
+        if (tid == 1023) s_carry = excl + cnt;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        chunk_offsets[N] = s_carry;
+        const bool bad = s_bad != 0;
+        hdr->status = bad ? kStatusBadSeqlens : kStatusOk;
+        hdr->num_chunks = bad ? 0 : s_carry;
+    }
+}
+
+// Record of one (head, chunk), fp32: W [64][DK] | U0 [64][DV] | Qt [64][DK] |
+// Kh [64][DK] | P [64][64] | gC [DK].  Rows >= L are zero.
+template <int DK, int DV>
+struct SimtRec {
+    static constexpr size_t W = 0;
+    static constexpr size_t U0 = W + kChunk * DK;
+    static constexpr size_t QT = U0 + kChunk * DV;
+    static constexpr size_t KH = QT + kChunk * DK;
+    static constexpr size_t P = KH + kChunk * DK;
+    static constexpr size_t GC = P + kChunk * kChunk;
+    static constexpr size_t FLOATS_RAW = GC + DK;
+    static constexpr size_t FLOATS = (FLOATS_RAW + 63) / 64 * 64;  // 256-byte multiple
+};
+
+// ---------------------------------------------------------------- K1 ------
+template <typename T, int DK, int DV>
+struct IntraSmem {
+    static constexpr int LDK = DK + 4;   // padded row strides (float4-aligned)
+    static constexpr int LDN = (DK > DV ? DK : DV) + 4;
+    static constexpr int LDA = kChunk + 1;
+    float g[kChunk][DK];
+    float bufA[kChunk][LDK];   // K~ with mid reference, later K~ (chunk-start reference)
+    float bufB[kChunk][LDK];   // K- (k e^{g_m - g})
+    float bufC[kChunk][LDN];   // Q~ with mid reference, later V
+    float Am[kChunk][LDA];     // A, later T diag(beta)
+    float Pm[kChunk][LDA];
+    float beta[kChunk];
+    float gref[DK], gend[DK];
+};
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(256)
+intra_chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                        const float* __restrict__ log_alpha, const float* __restrict__ beta,
+                        ChunkMap map, const WsHeader* __restrict__ hdr, float* __restrict__ records,
+                        int H, size_t max_chunks)
+{
+    using R = SimtRec<DK, DV>;
+    using Sm = IntraSmem<T, DK, DV>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    Sm& sm = *reinterpret_cast<Sm*>(smem_raw);
+
+    if (hdr->status != kStatusOk) return;
+    const int c = blockIdx.x, h = blockIdx.y;
+    if (c >= hdr->num_chunks) return;
+    int s, tok0, L;
+    map.locate(c, s, tok0, L);
+    float* rec = records + ((size_t)h * max_chunks + c) * R::FLOATS;
+    const int tid = threadIdx.x;
+    const size_t rowk = (size_t)H * DK, rowv = (size_t)H * DV;
+
+    // a. in-chunk cumulative log-decay per key channel; padded rows add 0
+    if (tid < DK) {
+        float acc = 0.f;
+        const float* la = log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid;
+#pragma unroll 8
+        for (int r = 0; r < kChunk; ++r) {
+            acc += (r < L) ? la[(size_t)r * rowk] : 0.f;
+            sm.g[r][tid] = acc;
+        }
+    } else if (tid >= 128 && tid < 128 + kChunk) {
+        const int r = tid - 128;
+        sm.beta[r] = (r < L) ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
+    }
+    __syncthreads();
+    if (tid < DK) {
+        sm.gref[tid] = sm.g[(L - 1) >> 1][tid];
+        sm.gend[tid] = sm.g[L - 1][tid];
+    }
+    __syncthreads();
+
+    // b. decayed operands; Q~ and K^ go straight to the record
+    for (int idx = tid; idx < kChunk * DK; idx += 256) {
+        const int r = idx / DK, ch = idx - r * DK;
+        float kk = 0.f, qq = 0.f;
+        if (r < L) {
+            const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
+            kk = to_f32(k[off]);
+            qq = to_f32(q[off]);
+        }
+        const float gg = sm.g[r][ch];
+        const float em = expf(gg - sm.gref[ch]);
+        sm.bufA[r][ch] = kk * em;
+        sm.bufB[r][ch] = kk * expf(sm.gref[ch] - gg);
+        sm.bufC[r][ch] = qq * em;
+        rec[R::QT + (size_t)r * DK + ch] = qq * expf(gg);
+        rec[R::KH + (size_t)r * DK + ch] = kk * expf(sm.gend[ch] - gg);
+    }
+    __syncthreads();
+
+    // c. A (strictly lower, beta-weighted) and P (lower incl. diagonal)
+    {
+        const int ty = tid >> 4, tx = tid & 15;
+        float acc_a[4][4], acc_p[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) { acc_a[a][b] = 0.f; acc_p[a][b] = 0.f; }
+        for (int ch = 0; ch < DK; ch += 4) {
+            float4 kr[4], qr[4], kc[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                kr[a] = *reinterpret_cast<const float4*>(&sm.bufA[ty + 16 * a][ch]);
+                qr[a] = *reinterpret_cast<const float4*>(&sm.bufC[ty + 16 * a][ch]);
+                kc[a] = *reinterpret_cast<const float4*>(&sm.bufB[tx + 16 * a][ch]);
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    acc_a[a][b] += kr[a].x * kc[b].x + kr[a].y * kc[b].y + kr[a].z * kc[b].z + kr[a].w * kc[b].w;
+                    acc_p[a][b] += qr[a].x * kc[b].x + qr[a].y * kc[b].y + qr[a].z * kc[b].z + qr[a].w * kc[b].w;
+                }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int r = ty + 16 * a, i = tx + 16 * b;
+                sm.Am[r][i] = (i < r) ? sm.beta[r] * acc_a[a][b] : 0.f;
+                sm.Pm[r][i] = (i <= r) ? acc_p[a][b] : 0.f;
+            }
+    }
+    __syncthreads();
+
+    // d. T = (I + A)^{-1} by forward substitution (threads 0..63, one column
+    //    each); meanwhile the other threads stage K~ (chunk-start reference)
+    //    and V for the W / U0 products.
+    float x[kChunk];
+    if (tid < kChunk) {
+#pragma unroll
+        for (int r = 0; r < kChunk; ++r) {
+            float a0 = (r == tid) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+            for (int i = 0; i + 3 < r; i += 4) {
+                a0 -= sm.Am[r][i] * x[i];
+                a1 -= sm.Am[r][i + 1] * x[i + 1];
+                a2 -= sm.Am[r][i + 2] * x[i + 2];
+                a3 -= sm.Am[r][i + 3] * x[i + 3];
+            }
+#pragma unroll
+            for (int i = r & ~3; i < r; ++i) a0 -= sm.Am[r][i] * x[i];
+            x[r] = (a0 + a1) + (a2 + a3);
+        }
+    } else {
+        for (int idx = tid - kChunk; idx < kChunk * DK; idx += 256 - kChunk) {
+            const int r = idx / DK, ch = idx - r * DK;
+            float kk = 0.f;
+            if (r < L) kk = to_f32(k[(size_t)(tok0 + r) * rowk + (size_t)h * DK + ch]);
+            sm.bufA[r][ch] = kk * expf(sm.g[r][ch]);
+        }
+        for (int idx = tid - kChunk; idx < kChunk * DV; idx += 256 - kChunk) {
+            const int r = idx / DV, ch = idx - r * DV;
+            sm.bufC[r][ch] = (r < L) ? to_f32(v[(size_t)(tok0 + r) * rowv + (size_t)h * DV + ch]) : 0.f;
+        }
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        const float bt = sm.beta[tid];
+#pragma unroll
+        for (int r = 0; r < kChunk; ++r) sm.Am[r][tid] = x[r] * bt;  // T diag(beta)
+    }
+    __syncthreads();
+
+    // e. W = T diag(beta) K~ and U0 = T diag(beta) V (columns [0,DK) | [DK,DK+DV))
+    {
+        constexpr int NCOL = (DK + DV) / 16;
+        const int ty = tid >> 4, tx = tid & 15;
+        float acc[4][NCOL];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < NCOL; ++b) acc[a][b] = 0.f;
+        for (int i = 0; i < kChunk; ++i) {
+            float t[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) t[a] = sm.Am[ty + 16 * a][i];
+#pragma unroll
+            for (int b = 0; b < NCOL; ++b) {
+                const int n = tx + 16 * b;
+                const float y = (n < DK) ? sm.bufA[i][n] : sm.bufC[i][n - DK];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) acc[a][b] = fmaf(t[a], y, acc[a][b]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < NCOL; ++b) {
+                const int r = ty + 16 * a, n = tx + 16 * b;
+                if (n < DK) rec[R::W + (size_t)r * DK + n] = acc[a][b];
+                else rec[R::U0 + (size_t)r * DV + (n - DK)] = acc[a][b];
+            }
+    }
+
+    // f. P and the chunk's total decay
+    for (int idx = tid; idx < kChunk * kChunk; idx += 256)
+        rec[R::P + idx] = sm.Pm[idx >> 6][idx & 63];
+    if (tid < DK) rec[R::GC + tid] = expf(sm.gend[tid]);
+}
+
+// ---------------------------------------------------------------- K2 ------
+constexpr int kSlice = 32;  // value columns per inter-chunk CTA
+
+template <int DK>
+struct InterSmem {
+    static constexpr int LDK = DK + 4;
+    float S[DK][kSlice + 1];
+    float W[kChunk][LDK];
+    float Qt[kChunk][LDK];
+    float Kh[kChunk][LDK];
+    float P[kChunk][kChunk + 4];
+    float U0[kChunk][kSlice + 1];
+    float U[kChunk][kSlice + 4];
+    float gC[DK];
+};
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(128)
+inter_chunk_simt_kernel(const float* __restrict__ initial_state, float* __restrict__ final_state,
+                        T* __restrict__ o, ChunkMap map, const WsHeader* __restrict__ hdr,
+                        const float* __restrict__ records, int H, size_t max_chunks, float scale)
+{
+    using R = SimtRec<DK, DV>;
+    using Sm = InterSmem<DK>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    Sm& sm = *reinterpret_cast<Sm*>(smem_raw);
+
+    if (hdr->status != kStatusOk) return;
+    const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSlice;
+    const int tid = threadIdx.x;
+    const size_t state_off = ((size_t)s * H + h) * DK * DV;
+
+    for (int idx = tid; idx < DK * kSlice; idx += 128) {
+        const int r = idx / kSlice, j = idx - r * kSlice;
+        sm.S[r][j] = initial_state ? initial_state[state_off + (size_t)r * DV + j0 + j] : 0.f;
+    }
+
+    const int first = map.seq_first_chunk(s);
+    const int nch = map.seq_num_chunks(s);
+    const int tok_begin = map.seq_token_begin(s), tok_end = map.seq_token_end(s);
+
+    for (int n = 0; n < nch; ++n) {
+        const float* rec = records + ((size_t)h * max_chunks + first + n) * R::FLOATS;
+        __syncthreads();  // previous chunk done with shared buffers
+        for (int idx = tid; idx < kChunk * DK / 4; idx += 128) {
+            const int r = idx / (DK / 4), c4 = (idx - r * (DK / 4)) * 4;
+            *reinterpret_cast<float4*>(&sm.W[r][c4]) = *reinterpret_cast<const float4*>(rec + R::W + (size_t)r * DK + c4);
+            *reinterpret_cast<float4*>(&sm.Qt[r][c4]) = *reinterpret_cast<const float4*>(rec + R::QT + (size_t)r * DK + c4);
+            *reinterpret_cast<float4*>(&sm.Kh[r][c4]) = *reinterpret_cast<const float4*>(rec + R::KH + (size_t)r * DK + c4);
+        }
+        for (int idx = tid; idx < kChunk * kChunk / 4; idx += 128) {
+            const int r = idx >> 4, c4 = (idx & 15) * 4;
+            *reinterpret_cast<float4*>(&sm.P[r][c4]) = *reinterpret_cast<const float4*>(rec + R::P + (size_t)r * kChunk + c4);
+        }
+        for (int idx = tid; idx < kChunk * kSlice; idx += 128) {
+            const int r = idx / kSlice, j = idx - r * kSlice;
+            sm.U0[r][j] = rec[R::U0 + (size_t)r * DV + j0 + j];
+        }
+        for (int idx = tid; idx < DK; idx += 128) sm.gC[idx] = rec[R::GC + idx];
+        __syncthreads();
+
+        // 1. W S and Q~ S for rows r = ry + 4a, column j = lane
+        const int lane = tid & 31, ry = tid >> 5;
+        float ws[16], qs[16];
+#pragma unroll
+        for (int a = 0; a < 16; ++a) { ws[a] = 0.f; qs[a] = 0.f; }
+        for (int c = 0; c < DK; c += 4) {
+            const float s0 = sm.S[c][lane], s1 = sm.S[c + 1][lane];
+            const float s2 = sm.S[c + 2][lane], s3 = sm.S[c + 3][lane];
+#pragma unroll
+            for (int a = 0; a < 16; ++a) {
+                const float4 w = *reinterpret_cast<const float4*>(&sm.W[ry + 4 * a][c]);
+                const float4 qv = *reinterpret_cast<const float4*>(&sm.Qt[ry + 4 * a][c]);
+                ws[a] += w.x * s0 + w.y * s1 + w.z * s2 + w.w * s3;
+                qs[a] += qv.x * s0 + qv.y * s1 + qv.z * s2 + qv.w * s3;
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 16; ++a) sm.U[ry + 4 * a][lane] = sm.U0[ry + 4 * a][lane] - ws[a];
+        __syncthreads();
+
+        // 2. O = scale (Q~ S + P U)
+        for (int i = 0; i < kChunk; i += 4) {
+            const float u0 = sm.U[i][lane], u1 = sm.U[i + 1][lane];
+            const float u2 = sm.U[i + 2][lane], u3 = sm.U[i + 3][lane];
+#pragma unroll
+            for (int a = 0; a < 16; ++a) {
+                const float4 p = *reinterpret_cast<const float4*>(&sm.P[ry + 4 * a][i]);
+                qs[a] += p.x * u0 + p.y * u1 + p.z * u2 + p.w * u3;
+            }
+        }
+        const int chunk_tok0 = tok_begin + n * kChunk;
+#pragma unroll
+        for (int a = 0; a < 16; ++a) {
+            const int tok = chunk_tok0 + ry + 4 * a;
+            if (tok < tok_end)
+                o[((size_t)tok * H + h) * DV + j0 + lane] = from_f32<T>(scale * qs[a]);
+        }
+
+        // 3. S' = Diag(gC) S + K^^T U, one key row per thread
+        if (tid < DK) {
+            float acc[kSlice];
+            const float gc = sm.gC[tid];
+#pragma unroll
+            for (int j = 0; j < kSlice; ++j) acc[j] = gc * sm.S[tid][j];
+            for (int r = 0; r < kChunk; ++r) {
+                const float kh = sm.Kh[r][tid];
+#pragma unroll
+                for (int j = 0; j < kSlice; j += 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(&sm.U[r][j]);
+                    acc[j] += kh * u.x; acc[j + 1] += kh * u.y;
+                    acc[j + 2] += kh * u.z; acc[j + 3] += kh * u.w;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kSlice; ++j) sm.S[tid][j] = acc[j];
+        }
+    }
+    __syncthreads();
+    if (final_state) {
+        for (int idx = tid; idx < DK * kSlice; idx += 128) {
+            const int r = idx / kSlice, j = idx - r * kSlice;
+            final_state[state_off + (size_t)r * DV + j0 + j] = sm.S[r][j];
+        }
+    }
+}
+
+template <typename T, int DK, int DV>
+cudaError_t launch_intra_t(const ChunkArgs& a) {
+    if (a.max_chunks == 0) return cudaSuccess;
+    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
+    auto k1 = intra_chunk_simt_kernel<T, DK, DV>;
+    const int smem = (int)sizeof(IntraSmem<T, DK, DV>);
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)a.max_chunks, (unsigned)a.H);
+    k1<<<grid, 256, smem, a.stream>>>(
+        static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
+        a.log_alpha, a.beta, map, static_cast<const WsHeader*>(a.ws_header),
+        static_cast<float*>(a.records), a.H, a.max_chunks);
+    return cudaGetLastError();
+}
+
+template <typename T, int DK, int DV>
+cudaError_t launch_inter_t(const ChunkArgs& a) {
+    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
+    auto k2 = inter_chunk_simt_kernel<T, DK, DV>;
+    const int smem = (int)sizeof(InterSmem<DK>);
+    cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)a.num_seqs, (unsigned)a.H, (unsigned)(DV / kSlice));
+    k2<<<grid, 128, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<T*>(a.o), map,
+                                       static_cast<const WsHeader*>(a.ws_header),
+                                       static_cast<const float*>(a.records), a.H, a.max_chunks,
+                                       a.scale);
+    return cudaGetLastError();
+}
+
+#define KDA_DISPATCH(FN, a)                                                         \
+    do {                                                                            \
+        if ((a).bf16) {                                                             \
+            if ((a).dk == 128 && (a).dv == 128) return FN<__nv_bfloat16, 128, 128>(a); \
+            if ((a).dk == 128 && (a).dv == 64) return FN<__nv_bfloat16, 128, 64>(a);   \
+            if ((a).dk == 64 && (a).dv == 128) return FN<__nv_bfloat16, 64, 128>(a);   \
+            if ((a).dk == 64 && (a).dv == 64) return FN<__nv_bfloat16, 64, 64>(a);     \
+        } else {                                                                    \
+            if ((a).dk == 128 && (a).dv == 128) return FN<float, 128, 128>(a);         \
+            if ((a).dk == 128 && (a).dv == 64) return FN<float, 128, 64>(a);           \
+            if ((a).dk == 64 && (a).dv == 128) return FN<float, 64, 128>(a);           \
+            if ((a).dk == 64 && (a).dv == 64) return FN<float, 64, 64>(a);             \
+        }                                                                           \
+        return cudaErrorInvalidValue;                                               \
+    } while (0)
+
+}  // namespace
+
+size_t simt_record_bytes(int dk, int dv) {
+    if (dk == 128 && dv == 128) return SimtRec<128, 128>::FLOATS * sizeof(float);
+    if (dk == 128 && dv == 64) return SimtRec<128, 64>::FLOATS * sizeof(float);
+    if (dk == 64 && dv == 128) return SimtRec<64, 128>::FLOATS * sizeof(float);
+    if (dk == 64 && dv == 64) return SimtRec<64, 64>::FLOATS * sizeof(float);
+    return 0;
+}
+
+cudaError_t launch_chunk_prep(const ChunkArgs& a) {
+    const int fixed_chunks = a.cu_seqlens ? 0 : a.num_seqs * a.fixed_chunks_per_seq;
+    chunk_prep_kernel<<<1, 1024, 0, a.stream>>>(static_cast<WsHeader*>(a.ws_header), a.chunk_offsets,
+                                               a.cu_seqlens, a.num_seqs, a.T, fixed_chunks);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_intra(const ChunkArgs& a) { KDA_DISPATCH(launch_intra_t, a); }
+
+cudaError_t launch_chunk_inter(const ChunkArgs& a) {
+    if (a.num_seqs == 0) return cudaSuccess;
+    KDA_DISPATCH(launch_inter_t, a);
+}
+
+}  // namespace kda

@@ -1,0 +1,82 @@
+// kda_common.cuh -- shared device/host helpers of libkda_b200 (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kda {
+
+constexpr int kChunk = 64;          // tokens per chunk in the chunkwise form
+constexpr int kHeaderBytes = 256;   // workspace header (status word, counts)
+
+// Device status codes written into the workspace header (same values as
+// kda_status in include/kda.h).
+constexpr int kStatusOk = 0;
+constexpr int kStatusTimeout = 4;
+constexpr int kStatusBadSeqlens = 6;
+
+// Workspace header, at offset 0 of the caller's workspace.
+struct WsHeader {
+    int status;       // first error a kernel of the last call hit (0 = none)
+    int num_chunks;   // chunks per head in this call
+    int reserved[62];
+};
+static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
+
+// Element loads/stores for the two input dtypes.
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Where the tokens of one chunk live.  Sequences are either B rows of T
+// tokens (fixed) or packed by cu_seqlens (varlen); chunks never cross a
+// sequence boundary and the last chunk of a sequence may be short.
+struct ChunkMap {
+    const int32_t* cu_seqlens;     // varlen: [N+1]; nullptr for fixed length
+    const int32_t* chunk_offsets;  // varlen: [N+1] first chunk of each sequence
+    int num_seqs;                  // N
+    int T;                         // fixed: tokens per sequence; varlen: total
+    int chunks_per_seq;            // fixed: ceil(T / 64)
+
+    __device__ __forceinline__ int seq_first_chunk(int s) const {
+        return cu_seqlens ? chunk_offsets[s] : s * chunks_per_seq;
+    }
+    __device__ __forceinline__ int seq_num_chunks(int s) const {
+        return cu_seqlens ? chunk_offsets[s + 1] - chunk_offsets[s] : chunks_per_seq;
+    }
+    __device__ __forceinline__ int seq_token_begin(int s) const {
+        return cu_seqlens ? cu_seqlens[s] : s * T;
+    }
+    __device__ __forceinline__ int seq_token_end(int s) const {
+        return cu_seqlens ? cu_seqlens[s + 1] : (s + 1) * T;
+    }
+    // Global chunk index -> (sequence, first token, length).
+    __device__ __forceinline__ void locate(int c, int& s, int& tok0, int& len) const {
+        if (!cu_seqlens) {
+            s = c / chunks_per_seq;
+            const int j = c - s * chunks_per_seq;
+            tok0 = s * T + j * kChunk;
+            len = min(kChunk, T - j * kChunk);
+            return;
+        }
+        // largest s with chunk_offsets[s] <= c (skips empty sequences)
+        int lo = 0, hi = num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (chunk_offsets[mid] <= c) lo = mid; else hi = mid - 1;
+        }
+        s = lo;
+        tok0 = cu_seqlens[s] + (c - chunk_offsets[s]) * kChunk;
+        len = min(kChunk, cu_seqlens[s + 1] - tok0);
+    }
+};
+
+}  // namespace kda

@@ -53,6 +53,8 @@ def _declare(lib):
     lib.kda_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp]
     lib.kda_workspace_status.restype = i
     lib.kda_workspace_status.argtypes = [vp, sz, vp]
+    lib.kda_set_stage_events.restype = i
+    lib.kda_set_stage_events.argtypes = [ctypes.POINTER(vp), i]
     lib.kda_last_error.restype = ctypes.c_char_p
     lib.kda_last_error.argtypes = []
     lib.kda_version.restype = ctypes.c_char_p
@@ -154,6 +156,16 @@ def workspace_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise and return the device status code left in ``workspace``."""
     return int(lib().kda_workspace_status(_ptr(workspace), workspace.numel(),
                                           _stream_ptr(stream, workspace.device)))
+
+
+def set_stage_events(events) -> None:
+    """Record ``events`` (4 ``torch.cuda.Event``s) at the stage boundaries of
+    the following ``chunk_fwd`` calls on this thread; ``None`` stops it."""
+    if events is None:
+        _check(lib().kda_set_stage_events(None, 0))
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(lib().kda_set_stage_events(arr, len(events)))
 
 
 def recurrent_step(q, k, v, log_alpha, beta, state, o=None, stream=None) -> torch.Tensor:

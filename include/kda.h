@@ -120,6 +120,17 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes,
                                 void* stream);
 
+/*
+ * Measurement hook for benchmarks.  When `events` is non-NULL, each later
+ * kda_chunk_fwd on this host thread records the caller-created CUDA events
+ * (cudaEvent_t passed as void*) on its stream at the stage boundaries:
+ * events[0] before the first kernel, events[1] after the chunk-table/status
+ * kernel, events[2] after the intra-chunk stage, events[3] after the
+ * inter-chunk stage.  `count` must be >= 4.  Pass NULL to stop.  Recording an
+ * event costs a few microseconds of stream time and changes no result.
+ */
+kda_status kda_set_stage_events(void* const* events, int count);
+
 /* Message of the last failing call on this host thread ("" if none). */
 const char* kda_last_error(void);
 

@@ -1,0 +1,97 @@
+"""The C-ABI library: it loads, exports every symbol include/kda.h declares, and
+rejects bad arguments on the host (no GPU needed: nothing is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_108_b200 import build, kda
+    build.build()
+    return kda.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_chunk_fwd_workspace_size",
+              "kda_workspace_status", "kda_last_error", "kda_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in kda.h but not exported"
+
+
+def test_version(lib):
+    assert b"sm_100a" in lib.kda_version()
+
+
+def test_workspace_size(lib):
+    from gated_delta_rule_108_b200 import kda
+    f32, bf16 = 0, 1
+    s1 = lib.kda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 4, 0, bf16)
+    assert s1 > 4 * 64 * 16 * 128 * 128  # at least the per-chunk records
+    # varlen bound covers the fixed-length count for the same tokens
+    s2 = lib.kda_chunk_fwd_workspace_size(1, 4 * 4096, 16, 128, 128, 4, 1, bf16)
+    assert s2 >= s1
+    assert lib.kda_chunk_fwd_workspace_size(1, 100, 2, 96, 64, 1, 0, f32) == 0  # unsupported dk
+    assert lib.kda_chunk_fwd_workspace_size(2, 100, 2, 64, 64, 2, 1, f32) == 0  # varlen needs B=1
+    assert kda.KDA_OK == 0
+
+
+def _chunk(lib, **over):
+    args = dict(q=1 << 20, k=1 << 20, v=1 << 20, la=1 << 20, beta=1 << 20, s0=None, cu=None,
+                B=1, T=64, H=1, dk=64, dv=64, N=1, dtype=0, o=1 << 20, sf=None,
+                ws=1 << 20, wsb=1 << 30, stream=None)
+    args.update(over)
+    a = args
+    return lib.kda_chunk_fwd(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["cu"],
+                             a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"], a["dtype"],
+                             a["o"], a["sf"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(dk=96), 2),                 # unsupported head size
+    (dict(dtype=7), 1),               # unknown dtype
+    (dict(q=None), 1),                # null input
+    (dict(k=(1 << 20) + 4), 1),       # misaligned
+    (dict(B=2, cu=1 << 20), 1),       # varlen with B != 1
+    (dict(ws=None), 5),               # missing workspace
+    (dict(ws=(1 << 20) + 16), 5),     # workspace not 256-aligned
+    (dict(wsb=16), 5),                # workspace too small
+    (dict(H=0), 1),
+    (dict(s0=1 << 20, sf=(1 << 20) + 64), 1),  # partially overlapping states
+])
+def test_chunk_fwd_rejects(lib, over, status):
+    assert _chunk(lib, **over) == status
+    assert lib.kda_last_error()  # a message is set
+
+
+def test_recurrent_step_rejects(lib):
+    p = 1 << 20
+    assert lib.kda_recurrent_step(p, p, p, p, p, p, 2, 2, 80, 64, 1, p + (1 << 24), None) == 2
+    assert lib.kda_recurrent_step(None, p, p, p, p, p, 2, 2, 64, 64, 1, p + (1 << 24), None) == 1
+    # o aliasing the state
+    assert lib.kda_recurrent_step(p, p, p, p, p, p, 2, 2, 64, 64, 1, p, None) == 1
+
+
+def test_python_binding_has_no_cpu_path(monkeypatch, tmp_path):
+    """The binding raises when the library is missing instead of computing on the CPU."""
+    from gated_delta_rule_108_b200 import kda
+    monkeypatch.setenv("KDA_B200_LIB", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(kda, "_lib", None)
+    with pytest.raises(kda.KDAError):
+        kda.lib()

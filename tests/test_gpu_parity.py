@@ -1,0 +1,287 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Tolerances (the accuracy bar of the workloads): fp32 inputs -> max relative
+error ||g - r||_inf / ||r||_inf <= 1e-4; bf16 inputs -> relative L2 error
+||g - r||_2 / ||r||_2 <= 5e-3, on o and on the final state, with the oracle run
+in fp64 on the bf16-rounded inputs.  Full-size workloads are checked on sampled
+(sequence, head) pairs, each pair against its own oracle run.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_108_b200 import inputs as I
+from gated_delta_rule_108_b200 import kda
+from oracle import oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32_MAXREL = 1e-4
+TOL_BF16_RELL2 = 5e-3
+
+
+def rel_l2(g, r):
+    g = np.asarray(g, dtype=np.float64)
+    r = np.asarray(r, dtype=np.float64)
+    return float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-300))
+
+
+def max_rel(g, r):
+    g = np.asarray(g, dtype=np.float64)
+    r = np.asarray(r, dtype=np.float64)
+    return float(np.max(np.abs(g - r)) / max(np.max(np.abs(r)), 1e-300))
+
+
+def check(g, r, dtype, what):
+    g = g.float().cpu().numpy() if hasattr(g, "cpu") else g
+    assert np.all(np.isfinite(g)), f"{what}: non-finite values"
+    if dtype == torch.float32:
+        e = max_rel(g, r)
+        assert e <= TOL_F32_MAXREL, f"{what}: max rel error {e:.3e}"
+    else:
+        e = rel_l2(g, r)
+        assert e <= TOL_BF16_RELL2, f"{what}: rel L2 error {e:.3e}"
+    return e
+
+
+def to_dev(x):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+def run_chunk(x, **kw):
+    g = to_dev(x)
+    o, S = kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], g["initial_state"],
+                         g["cu_seqlens"], **kw)
+    torch.cuda.synchronize()
+    return o, S
+
+
+def oracle_chunk(x):
+    return orc.kda_forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                           x["initial_state"], x["cu_seqlens"])
+
+
+# ----------------------------------------------------------------- small ---
+SHAPES = [(64, 64), (64, 128), (128, 64), (128, 128)]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", SHAPES, ids=[f"dk{a}dv{b}" for a, b in SHAPES])
+def test_chunk_fwd_small(cuda_device, dtype, dk, dv):
+    # 3 full chunks and a ragged tail of 17 tokens, 2 sequences, 3 heads
+    w = I.ChunkWorkload("small", B=2, T=209, H=3, dk=dk, dv=dv, dtype=dtype, s0_std=0.05, seed=21)
+    x = I.chunk_inputs(w)
+    o, S = run_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check(o, o_ref, dtype, "o")
+    check(S, S_ref, dtype, "final_state")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", SHAPES, ids=[f"dk{a}dv{b}" for a, b in SHAPES])
+def test_recurrent_step_small(cuda_device, dtype, dk, dv):
+    w = I.DecodeWorkload("small", B=5, H=3, dk=dk, dv=dv, steps=8, dtype=dtype, s0_std=0.1)
+    d = I.decode_inputs(w, pool=8)
+    st = d["state0"].cuda().clone()
+    S_ref = d["state0"].double().numpy()
+    for n in range(8):
+        o = kda.recurrent_step(d["q"][n].cuda(), d["k"][n].cuda(), d["v"][n].cuda(),
+                               d["log_alpha"][n].cuda(), d["beta"][n].cuda(), st)
+        torch.cuda.synchronize()
+        o_ref, S_ref = orc.kda_decode_step(d["q"][n], d["k"][n], d["v"][n], d["log_alpha"][n],
+                                           d["beta"][n], S_ref)
+        check(o, o_ref, dtype, f"o step {n}")
+    check(st, S_ref, dtype, "state after 8 steps")
+
+
+# ------------------------------------------------------------ full size ---
+def test_c0_full(cuda_device):
+    """fp32, B=1, H=2, T=256, d=64, zero initial state, seed 0: max rel <= 1e-4."""
+    w = I.workload("C0")
+    x = I.chunk_inputs(w)
+    o, S = run_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check(o, o_ref, torch.float32, "C0 o")
+    check(S, S_ref, torch.float32, "C0 final_state")
+
+
+def _sampled_chunk_check(name, pairs):
+    w = I.workload(name)
+    x = I.chunk_inputs(w)
+    o, S = run_chunk(x)
+    o, S = o.cpu(), S.cpu()
+    cu = x["cu_seqlens"]
+    for (s, h) in pairs:
+        if cu is None:
+            sl = (slice(s, s + 1), slice(None))
+            xs = {k: x[k][sl[0], :, h:h + 1] for k in ("q", "k", "v", "log_alpha", "beta")}
+            o_g = o[s:s + 1, :, h:h + 1]
+        else:
+            a, b = int(cu[s]), int(cu[s + 1])
+            xs = {k: x[k][:, a:b, h:h + 1] for k in ("q", "k", "v", "log_alpha", "beta")}
+            o_g = o[:, a:b, h:h + 1]
+        S0 = None if x["initial_state"] is None else x["initial_state"][s:s + 1, h:h + 1]
+        o_ref, S_ref = orc.kda_forward(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["beta"], S0)
+        check(o_g, o_ref, w.dtype, f"{name} o (seq {s}, head {h})")
+        check(S[s:s + 1, h:h + 1], S_ref, w.dtype, f"{name} final_state (seq {s}, head {h})")
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
+
+
+def test_c1_full_sampled(cuda_device):
+    _sampled_chunk_check("C1", [(0, 0), (1, 7), (3, 15)])
+
+
+def test_c2_full_sampled(cuda_device):
+    _sampled_chunk_check("C2", [(0, 0), (0, 31)])
+
+
+def test_c4_varlen_full_sampled(cuda_device):
+    _sampled_chunk_check("C4", [(0, 0), (7, 13), (15, 31)])
+
+
+def test_c3_decode_full_sampled(cuda_device):
+    """1024 steps, B=256, H=32; inputs cycle through a pool of 32 seeded draws."""
+    w = I.workload("C3")
+    P = 32
+    d = I.decode_inputs(w, pool=P)
+    g = {k: v.cuda() for k, v in d.items()}
+    st = g["state0"].clone()
+    o_last = None
+    pairs = [(0, 0), (100, 17), (255, 31)]
+    outs = {p: [] for p in pairs}
+    for n in range(w.steps):
+        j = n % P
+        o_last = kda.recurrent_step(g["q"][j], g["k"][j], g["v"][j], g["log_alpha"][j],
+                                    g["beta"][j], st)
+        if n % 97 == 0 or n == w.steps - 1:
+            oc = o_last.cpu()
+            for (b, h) in pairs:
+                outs[(b, h)].append((n, oc[b, h].clone()))
+    torch.cuda.synchronize()
+    S = st.cpu()
+    idx = [n % P for n in range(w.steps)]
+    for (b, h) in pairs:
+        seq = {k: d[k][idx, b, h][None, :, None] for k in ("q", "k", "v", "log_alpha", "beta")}
+        o_ref, S_ref = orc.kda_forward(seq["q"], seq["k"], seq["v"], seq["log_alpha"], seq["beta"],
+                                       d["state0"][b:b + 1, h:h + 1])
+        got = torch.stack([t for _, t in outs[(b, h)]]).float().numpy()
+        ref = np.stack([o_ref[0, n, 0] for n, _ in outs[(b, h)]])
+        check(got, ref, w.dtype, f"C3 o (b {b}, h {h})")
+        check(S[b:b + 1, h:h + 1], S_ref, w.dtype, f"C3 state (b {b}, h {h})")
+
+
+# ----------------------------------------------------------- consistency ---
+def test_chunk_equals_decode_steps(cuda_device):
+    """The chunkwise and the recurrent modes agree on one sequence set."""
+    w = I.ChunkWorkload("cons", B=3, T=130, H=2, dk=128, dv=128, dtype=torch.bfloat16,
+                        s0_std=0.05, seed=22)
+    x = I.chunk_inputs(w)
+    o, S = run_chunk(x)
+    st = x["initial_state"].cuda().clone()
+    g = to_dev(x)
+    od = []
+    for t in range(w.T):
+        od.append(kda.recurrent_step(g["q"][:, t].contiguous(), g["k"][:, t].contiguous(),
+                                     g["v"][:, t].contiguous(), g["log_alpha"][:, t].contiguous(),
+                                     g["beta"][:, t].contiguous(), st))
+    torch.cuda.synchronize()
+    od = torch.stack(od, dim=1)
+    assert rel_l2(od.float().cpu(), o.float().cpu()) < 5e-3
+    assert rel_l2(st.cpu(), S.cpu()) < 5e-3
+    o_ref, S_ref = oracle_chunk(x)
+    check(od, o_ref, torch.bfloat16, "decode loop o")
+
+
+def test_split_sequence_carries_state(cuda_device):
+    w = I.ChunkWorkload("split", B=2, T=300, H=2, dk=64, dv=128, dtype=torch.float32,
+                        s0_std=0.05, seed=23)
+    x = I.chunk_inputs(w)
+    o, S = run_chunk(x)
+    c = 100  # not a multiple of the chunk size
+    xa = {k: (v[:, :c].contiguous() if k in ("q", "k", "v", "log_alpha", "beta") else v) for k, v in x.items()}
+    oa, Sa = run_chunk(xa)
+    xb = {k: (v[:, c:].contiguous() if k in ("q", "k", "v", "log_alpha", "beta") else v) for k, v in x.items()}
+    xb["initial_state"] = Sa.cpu()
+    ob, Sb = run_chunk(xb)
+    assert max_rel(torch.cat([oa, ob], 1).cpu().numpy(), o.cpu().numpy()) < 1e-5
+    assert max_rel(Sb.cpu().numpy(), S.cpu().numpy()) < 1e-5
+
+
+def test_varlen_equals_separate_calls(cuda_device):
+    lens = (1, 63, 64, 65, 0, 130, 200)
+    w = I.ChunkWorkload("vl", B=1, T=sum(lens), H=2, dk=128, dv=64, dtype=torch.bfloat16,
+                        s0_std=0.05, lengths=lens, beta_edge_frac=0.1, seed=24)
+    x = I.chunk_inputs(w)
+    o, S = run_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check(o, o_ref, torch.bfloat16, "varlen o")
+    check(S, S_ref, torch.bfloat16, "varlen final_state")
+    cu = x["cu_seqlens"].tolist()
+    for s in range(len(lens)):
+        a, b = cu[s], cu[s + 1]
+        xs = {k: x[k][:, a:b].contiguous() for k in ("q", "k", "v", "log_alpha", "beta")}
+        xs["initial_state"] = x["initial_state"][s:s + 1]
+        xs["cu_seqlens"] = None
+        os_, Ss = run_chunk(xs)
+        assert torch.equal(os_.cpu(), o[:, a:b].cpu()), f"seq {s} o differs from the packed call"
+        assert torch.equal(Ss.cpu(), S[s:s + 1].cpu()), f"seq {s} state differs from the packed call"
+
+
+# ------------------------------------------------------------ edge cases ---
+def test_empty_input_passes_state_through(cuda_device):
+    S0 = torch.randn(2, 3, 64, 64).cuda()
+    e = lambda *s: torch.empty(*s, device="cuda")
+    q = e(2, 0, 3, 64).bfloat16()
+    o, S = kda.chunk_fwd(q, q, e(2, 0, 3, 64).bfloat16(), e(2, 0, 3, 64), e(2, 0, 3), S0)
+    torch.cuda.synchronize()
+    assert o.shape == (2, 0, 3, 64) and torch.equal(S, S0)
+    o, S = kda.chunk_fwd(q, q, e(2, 0, 3, 64).bfloat16(), e(2, 0, 3, 64), e(2, 0, 3), None)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(S) == 0
+
+
+@pytest.mark.parametrize("case", ["beta0", "beta1", "nodecay"])
+def test_degenerate_gates(cuda_device, case):
+    w = I.ChunkWorkload("deg", B=1, T=150, H=2, dk=128, dv=128, dtype=torch.float32, s0_std=0.1, seed=25)
+    x = I.chunk_inputs(w)
+    if case == "beta0":
+        x["beta"].zero_()
+    elif case == "beta1":
+        x["beta"].fill_(1.0)
+    else:
+        x["log_alpha"].zero_()
+    o, S = run_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check(o, o_ref, torch.float32, f"{case} o")
+    check(S, S_ref, torch.float32, f"{case} final_state")
+
+
+def test_state_alias_in_place(cuda_device):
+    w = I.ChunkWorkload("alias", B=2, T=100, H=2, dk=64, dv=64, dtype=torch.bfloat16, s0_std=0.05, seed=26)
+    x = I.chunk_inputs(w)
+    o_ref, S_ref = oracle_chunk(x)
+    g = to_dev(x)
+    st = g["initial_state"].clone()
+    o, S = kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], st, final_state=st)
+    torch.cuda.synchronize()
+    assert S.data_ptr() == st.data_ptr()
+    check(st, S_ref, torch.bfloat16, "aliased final_state")
+
+
+def test_bad_cu_seqlens_reported(cuda_device):
+    w = I.ChunkWorkload("bad", B=1, T=100, H=2, dk=64, dv=64, dtype=torch.bfloat16, seed=27)
+    x = I.chunk_inputs(w)
+    g = to_dev(x)
+    cu = torch.tensor([0, 60, 40, 100], dtype=torch.int32, device="cuda")  # decreasing
+    o = torch.full((1, 100, 2, 64), 7.0, device="cuda").bfloat16()
+    ws = torch.empty(kda.chunk_fwd_workspace_size(1, 100, 2, 64, 64, 3, True, torch.bfloat16),
+                     dtype=torch.uint8, device="cuda")
+    kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], None, cu, o=o, workspace=ws)
+    with pytest.raises(kda.KDAError) as ei:
+        kda._check(kda.workspace_status(ws))
+    assert ei.value.status == 6
+    assert bool((o.float() == 7.0).all()), "o must be left unwritten"
+    # a good call on the same workspace clears the status
+    cu_ok = torch.tensor([0, 40, 60, 100], dtype=torch.int32, device="cuda")
+    kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], None, cu_ok, workspace=ws)
+    assert kda.workspace_status(ws) == 0
