@@ -69,6 +69,18 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
 
 }  // namespace
 
+namespace kda {
+int set_error(int status, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return status;
+}
+}  // namespace kda
+
 extern "C" {
 
 size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int varlen,

@@ -40,6 +40,10 @@ struct ChunkArgs {
 // Bytes of per-(head, chunk) intermediates for the SIMT fp32 path.
 size_t simt_record_bytes(int dk, int dv);
 
+// Sets the calling thread's kda_last_error() message and returns `status`
+// (status is a kda_status value).
+int set_error(int status, const char* fmt, ...);
+
 cudaError_t launch_decode(const DecodeArgs& a);
 cudaError_t launch_chunk_prep(const ChunkArgs& a);     // K0: status reset + varlen chunk table
 cudaError_t launch_chunk_intra(const ChunkArgs& a);    // K1: all chunks in parallel

@@ -121,6 +121,34 @@ kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes,
                                 void* stream);
 
 /*
+ * kda_chunk_fwd without a caller-provided workspace.  The paper has no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory -- a plugin whose host framework owns all device memory and forbids
+ * other allocations, a latency-critical loop that cannot afford cudaMalloc's
+ * implicit synchronisation, or a tool with a fixed memory budget.
+ *
+ * The scratch space comes from one fixed array of KDA_STATIC_WORKSPACE_BYTES
+ * in the library's device image, present on every GPU that loads the library
+ * until the process exits.  Arguments and results are those of kda_chunk_fwd
+ * minus the workspace.  Sizes whose workspace (kda_chunk_fwd_workspace_size)
+ * exceeds KDA_STATIC_WORKSPACE_BYTES are rejected with KDA_ERR_WORKSPACE and
+ * nothing is launched.  Nothing is allocated: no cudaMalloc or cudaFree.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call uses the same array, so calls that
+ * overlap on one GPU (e.g. on two streams) race; order them on one stream.
+ * kda_workspace_status cannot read this workspace (use kda_chunk_fwd when the
+ * device status is needed).
+ */
+#define KDA_STATIC_WORKSPACE_BYTES (64u << 20)
+kda_status kda_chunk_fwd_static(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta,
+                                const float* initial_state, const int32_t* cu_seqlens,
+                                int B, int T, int H, int dk, int dv, int num_seqs,
+                                kda_dtype dtype, void* o, float* final_state, void* stream);
+
+/*
  * Measurement hook for benchmarks.  When `events` is non-NULL, each later
  * kda_chunk_fwd on this host thread records the caller-created CUDA events
  * (cudaEvent_t passed as void*) on its stream at the stage boundaries:
