@@ -1,0 +1,46 @@
+"""Run one small, fixed case of a kernel of the library (for profilers).
+
+    python -m gated_delta_rule_108_b200.profile_case decode --B 96 --H 32 --launches 3
+    python -m gated_delta_rule_108_b200.profile_case chunk --B 1 --T 8192 --H 16 --launches 3
+
+Inputs are seeded synthetic data (gated_delta_rule_108_b200.inputs); each
+launch is one library call; the process synchronises and exits 0 on success.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import inputs as I
+from . import kda
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("what", choices=["decode", "chunk"])
+    ap.add_argument("--B", type=int, default=96)
+    ap.add_argument("--T", type=int, default=8192)
+    ap.add_argument("--H", type=int, default=32)
+    ap.add_argument("--d", type=int, default=128)
+    ap.add_argument("--dtype", choices=["bf16", "f32"], default="bf16")
+    ap.add_argument("--launches", type=int, default=3)
+    a = ap.parse_args()
+    dt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
+    if a.what == "decode":
+        w = I.DecodeWorkload("profile", B=a.B, H=a.H, dk=a.d, dv=a.d, steps=a.launches, dtype=dt)
+        x = {k: v.cuda() for k, v in I.decode_inputs(w, pool=1).items()}
+        st = x["state0"].clone()
+        for _ in range(a.launches):
+            kda.recurrent_step(x["q"][0], x["k"][0], x["v"][0], x["log_alpha"][0], x["beta"][0], st)
+    else:
+        w = I.ChunkWorkload("profile", B=a.B, T=a.T, H=a.H, dk=a.d, dv=a.d, dtype=dt, s0_std=0.01, seed=7)
+        x = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in I.chunk_inputs(w).items()}
+        for _ in range(a.launches):
+            kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
+    torch.cuda.synchronize()
+    print(f"{a.what}: {a.launches} launches ok")
+
+
+if __name__ == "__main__":
+    main()
