@@ -60,7 +60,9 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
     } else {
         L.max_chunks = (size_t)B * L.chunks_per_seq;
     }
-    const size_t rec = kda::simt_record_bytes(dk, dv);
+    // bf16 inputs run on the tensor cores with fp16 records; fp32 inputs on
+    // CUDA cores with fp32 records.
+    const size_t rec = dtype == KDA_BF16 ? kda::tc_record_bytes(dk, dv) : kda::simt_record_bytes(dk, dv);
     L.offsets_off = kda::kHeaderBytes;
     L.records_off = round_up(L.offsets_off + sizeof(int32_t) * ((size_t)N + 1), 256);
     L.total = L.records_off + rec * (size_t)H * L.max_chunks;
@@ -148,9 +150,9 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
     cudaError_t e = mark_stage(0, a.stream);
     if (e == cudaSuccess) e = kda::launch_chunk_prep(a);
     if (e == cudaSuccess) e = mark_stage(1, a.stream);
-    if (e == cudaSuccess) e = kda::launch_chunk_intra(a);
+    if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_intra_tc(a) : kda::launch_chunk_intra(a);
     if (e == cudaSuccess) e = mark_stage(2, a.stream);
-    if (e == cudaSuccess) e = kda::launch_chunk_inter(a);
+    if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_inter_tc(a) : kda::launch_chunk_inter(a);
     if (e == cudaSuccess) e = mark_stage(3, a.stream);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_chunk_fwd launch failed: %s", cudaGetErrorString(e));
     return ok();
@@ -193,14 +195,17 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {
     if (!workspace || workspace_bytes < (size_t)kda::kHeaderBytes)
         return fail(KDA_ERR_WORKSPACE, "workspace missing or smaller than its header");
-    int st = 0;
+    int words[3] = {0, 0, 0};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(&st, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
+    cudaError_t e = cudaMemcpyAsync(words, workspace, sizeof(words), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "reading workspace status: %s", cudaGetErrorString(e));
+    const int st = words[0] != 0 ? words[0] : words[2];
     if (st == kda::kStatusOk) return ok();
     if (st == kda::kStatusBadSeqlens) return fail(KDA_ERR_BAD_SEQLENS, "cu_seqlens rejected on the device");
     if (st == kda::kStatusTimeout) return fail(KDA_ERR_TIMEOUT, "a bounded wait inside a kernel gave up");
+    if (st == kda::kStatusRange)
+        return fail(KDA_ERR_RANGE, "an intermediate exceeded the fp16 range of the bf16 path (use fp32 inputs)");
     return fail(KDA_ERR_CUDA, "unknown device status %d", st);
 }
 

@@ -38,7 +38,7 @@ chunk_prep_kernel(WsHeader* hdr, int32_t* chunk_offsets, const int32_t* __restri
     __shared__ int s_carry, s_bad;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (cu == nullptr) {
-        if (tid == 0) { hdr->status = kStatusOk; hdr->num_chunks = fixed_num_chunks; }
+        if (tid == 0) { hdr->status = kStatusOk; hdr->num_chunks = fixed_num_chunks; hdr->runtime_err = 0; }
         return;
     }
     if (tid == 0) { s_carry = 0; s_bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0; }
@@ -81,6 +81,7 @@ chunk_prep_kernel(WsHeader* hdr, int32_t* chunk_offsets, const int32_t* __restri
         const bool bad = s_bad != 0;
         hdr->status = bad ? kStatusBadSeqlens : kStatusOk;
         hdr->num_chunks = bad ? 0 : s_carry;
+        hdr->runtime_err = 0;
     }
 }
 

@@ -15,12 +15,14 @@ constexpr int kHeaderBytes = 256;   // workspace header (status word, counts)
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 4;
 constexpr int kStatusBadSeqlens = 6;
+constexpr int kStatusRange = 7;
 
 // Workspace header, at offset 0 of the caller's workspace.
 struct WsHeader {
-    int status;       // first error a kernel of the last call hit (0 = none)
+    int status;       // argument check of the last call (0 = ok): kernels skip work if set
     int num_chunks;   // chunks per head in this call
-    int reserved[62];
+    int runtime_err;  // first error a kernel hit while working (0 = none), e.g. a timeout
+    int reserved[61];
 };
 static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
 

@@ -37,8 +37,9 @@ struct ChunkArgs {
     cudaStream_t stream;
 };
 
-// Bytes of per-(head, chunk) intermediates for the SIMT fp32 path.
+// Bytes of per-(head, chunk) intermediates: fp32 CUDA-core path / bf16 tensor-core path.
 size_t simt_record_bytes(int dk, int dv);
+size_t tc_record_bytes(int dk, int dv);
 
 // Sets the calling thread's kda_last_error() message and returns `status`
 // (status is a kda_status value).
@@ -48,5 +49,7 @@ cudaError_t launch_decode(const DecodeArgs& a);
 cudaError_t launch_chunk_prep(const ChunkArgs& a);     // K0: status reset + varlen chunk table
 cudaError_t launch_chunk_intra(const ChunkArgs& a);    // K1: all chunks in parallel
 cudaError_t launch_chunk_inter(const ChunkArgs& a);    // K2: serial over each sequence's chunks
+cudaError_t launch_chunk_intra_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K1
+cudaError_t launch_chunk_inter_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K2
 
 }  // namespace kda

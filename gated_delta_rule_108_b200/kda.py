@@ -20,7 +20,7 @@ _LIB_NAME = "libkda_b200.so"
 KDA_OK = 0
 _STATUS = {
     0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA",
-    4: "KDA_ERR_TIMEOUT", 5: "KDA_ERR_WORKSPACE", 6: "KDA_ERR_BAD_SEQLENS",
+    4: "KDA_ERR_TIMEOUT", 5: "KDA_ERR_WORKSPACE", 6: "KDA_ERR_BAD_SEQLENS", 7: "KDA_ERR_RANGE",
 }
 KDA_F32, KDA_BF16 = 0, 1
 

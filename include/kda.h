@@ -48,7 +48,8 @@ typedef enum {
     KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
     KDA_ERR_TIMEOUT = 4,       /* device status: a bounded wait inside a kernel gave up */
     KDA_ERR_WORKSPACE = 5,     /* workspace missing, too small or misaligned */
-    KDA_ERR_BAD_SEQLENS = 6    /* device status: cu_seqlens not 0 .. T non-decreasing */
+    KDA_ERR_BAD_SEQLENS = 6,   /* device status: cu_seqlens not 0 .. T non-decreasing */
+    KDA_ERR_RANGE = 7          /* device status: a bf16-path intermediate left the fp16 range */
 } kda_status;
 
 typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
@@ -112,10 +113,13 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
                               kda_dtype dtype, void* o, void* stream);
 
 /*
- * Waits for `stream`, then reads the device status word that the last
- * kda_chunk_fwd on this workspace left: KDA_OK, KDA_ERR_BAD_SEQLENS or
- * KDA_ERR_TIMEOUT (or KDA_ERR_CUDA if the copy fails).  This is the only call
- * that synchronises.
+ * Waits for `stream`, then reads the device status that the last
+ * kda_chunk_fwd on this workspace left: KDA_OK, KDA_ERR_BAD_SEQLENS,
+ * KDA_ERR_TIMEOUT or KDA_ERR_RANGE (or KDA_ERR_CUDA if the copy fails).
+ * KDA_ERR_RANGE means a value-side quantity (|v|, the state, the per-token
+ * errors u) exceeded 65000 in magnitude: the bf16 path keeps its chunk
+ * intermediates in fp16, so such inputs need the fp32 path.  This is the only
+ * call that synchronises.
  */
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes,
                                 void* stream);
