@@ -204,6 +204,7 @@ kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes, v
     if (st == kda::kStatusOk) return ok();
     if (st == kda::kStatusBadSeqlens) return fail(KDA_ERR_BAD_SEQLENS, "cu_seqlens rejected on the device");
     if (st == kda::kStatusTimeout) return fail(KDA_ERR_TIMEOUT, "a bounded wait inside a kernel gave up");
+    if (st == kda::kStatusInternal) return fail(KDA_ERR_CUDA, "a kernel found its shared memory misaligned");
     if (st == kda::kStatusRange)
         return fail(KDA_ERR_RANGE, "an intermediate exceeded the fp16 range of the bf16 path (use fp32 inputs)");
     return fail(KDA_ERR_CUDA, "unknown device status %d", st);

@@ -81,20 +81,48 @@ struct TcRec {
 };
 
 // ---------------------------------------------------------------- K1 ----
+// Persistent: one CTA per SM walks the (chunk, head) work items.  The k, v, q
+// tiles of the next item are TMA-loaded into the other half of a double
+// buffer, and its log_alpha / beta are loaded into registers, while the
+// current item is being computed.
 template <int DK, int DV>
 struct K1Smem {
-    static constexpr uint32_t KS = 0;                           // k tiles (bf16 -> fp16 K~ in place)
-    static constexpr uint32_t VS = KS + (DK / 64) * 8192;       // v tiles (bf16 -> fp16 in place)
-    static constexpr uint32_t QS = VS + (DV / 64) * 8192;       // q tiles (bf16)
-    static constexpr uint32_t LAS = QS + (DK / 64) * 8192;      // log_alpha [64][DK] fp32, dense
-    static constexpr uint32_t OPA = LAS + 64 * DK * 4;          // tf32 [K~m; Q~m]: DK/32 tiles of 16 KB
-    static constexpr uint32_t OPB = OPA + (DK / 32) * 16384;    // tf32 K-m: DK/32 tiles of 8 KB
-    static constexpr uint32_t END = OPB + (DK / 32) * 8192;
-    static constexpr uint32_t AM = QS;   // after the decay pass: A in fp32 [64][65]
-    static constexpr uint32_t TP = OPB;  // after MMA1: T diag(beta) fp16, K-major 128 x 64 tokens
-    static constexpr uint32_t TX_BYTES = (2 * (DK / 64) + DV / 64) * 8192 + 64 * DK * 4;
-    static_assert(QS + 64 * 65 * 4 <= OPA, "A matrix alias");
-    static_assert(TP + 16384 <= END, "T alias");
+    static constexpr uint32_t TILE = 8192;                          // 64 tokens x 128 bytes
+    static constexpr uint32_t STAGE = (2 * (DK / 64) + DV / 64) * TILE;
+    static constexpr uint32_t KS = 0;                               // + stage * STAGE: k tiles (-> fp16 K~)
+    static constexpr uint32_t VS = (DK / 64) * TILE;                //                  v tiles (-> fp16 V)
+    static constexpr uint32_t QS = VS + (DV / 64) * TILE;           //                  q tiles (-> fp16 Q~)
+    static constexpr uint32_t G = 2 * STAGE;                        // cumulative log-decay [64][DK] fp32
+    static constexpr uint32_t OPA = G + 64 * DK * 4;                // tf32 [K~m; Q~m]: DK/32 tiles of 16 KB
+    static constexpr uint32_t OPB = OPA + (DK / 32) * 16384;        // tf32 K-m: DK/32 tiles of 8 KB
+    static constexpr uint32_t OPB_END = OPB + (DK / 32) * 8192;
+    // after MMA1 (OPA/OPB dead): A, T (fp32, 64 x 68) and the E blocks (6 x 16 x 17)
+    // in OPA when it is large enough, else in an extra region
+    static constexpr uint32_t SCR_BYTES = 2 * 64 * 68 * 4 + 6 * 16 * 17 * 4;
+    static constexpr bool SCR_IN_OPA = (DK / 32) * 16384 >= SCR_BYTES;
+    static constexpr uint32_t AM = SCR_IN_OPA ? OPA : OPB_END;
+    static constexpr uint32_t TM = AM + 64 * 68 * 4;
+    static constexpr uint32_t YM = TM + 64 * 68 * 4;
+    static constexpr uint32_t END = SCR_IN_OPA ? OPB_END : OPB_END + SCR_BYTES;
+    // after MMA1: T diag(beta) fp16, K-major 128 rows x 64 tokens, in OPB
+    static constexpr uint32_t TP = OPB;
+    static constexpr uint32_t TX_BYTES = STAGE;
+    static constexpr uint32_t LA_BYTES = 64 * DK * 4;               // log_alpha tile into G
+    // small per-item arrays after END (no static shared memory, so the
+    // dynamic window starts 1024-byte aligned)
+    static constexpr uint32_t BAR = END;                            // 4 mbarriers
+    static constexpr uint32_t TMEMADDR = BAR + 32;   // after bar_load[2], bar_mma, bar_la
+    static constexpr uint32_t BETA = TMEMADDR + 16;                 // [64]
+    static constexpr uint32_t GM = BETA + 256;                      // [DK] g_m, e^{g_m}, e^{g_{L-1}-g_m}
+    static constexpr uint32_t EGM = GM + DK * 4;
+    static constexpr uint32_t EGLM = EGM + DK * 4;
+    static constexpr uint32_t TOTAL = EGLM + DK * 4;
+    // cumulative-sum partials live in the (then unused) T-solve scratch
+    static constexpr uint32_t PART = YM;
+    static_assert(YM + 6 * 16 * 17 * 4 <= END, "T-solve scratch");
+    static_assert(PART + (256 / DK) * DK * 4 <= END, "partials alias");
+    static_assert((DK / 32) * 8192 >= 16384, "T diag(beta) in OPB");
+    static_assert(TOTAL <= 232448, "shared memory");
 };
 
 template <int DK, int DV>
@@ -106,111 +134,212 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
 {
     using Sm = K1Smem<DK, DV>;
     using R = TcRec<DK, DV>;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar_load, bar_mma;
-    __shared__ uint32_t s_tmem;
-    __shared__ float s_beta[kChunk];
+    constexpr int NPART = 256 / DK;       // threads per key channel in the cumulative sum
+    constexpr int TPP = kChunk / NPART;   // tokens per such thread
+    constexpr int NCH8 = DK / 8;          // 8-channel (16-byte bf16) groups per token row
+    extern __shared__ __align__(1024) unsigned char sm[];
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + Sm::BAR);   // [2]
+    uint64_t& bar_mma = bar_load[2];
+    uint64_t& bar_la = bar_load[3];
+    uint32_t& s_tmem = *reinterpret_cast<uint32_t*>(sm + Sm::TMEMADDR);
+    float* s_beta = reinterpret_cast<float*>(sm + Sm::BETA);
+    float* s_gm = reinterpret_cast<float*>(sm + Sm::GM);
+    float* s_egm = reinterpret_cast<float*>(sm + Sm::EGM);
+    float* s_eglm = reinterpret_cast<float*>(sm + Sm::EGLM);
+    float* s_part = reinterpret_cast<float*>(sm + Sm::PART);        // [NPART][DK]
 
     if (hdr->status != kStatusOk) return;
-    const int c = blockIdx.x, h = blockIdx.y;
-    if (c >= hdr->num_chunks) return;
-    int seq, tok0, L;
-    map.locate(c, seq, tok0, L);
+    const int total = hdr->num_chunks * H;
+    if ((int)blockIdx.x >= total) return;
+    if ((smem_u32(sm) & 1023u) != 0) {   // the swizzled layouts need 1024-byte alignment
+        if (threadIdx.x == 0) flag_error(hdr, kStatusInternal);
+        return;
+    }
     const int tid = threadIdx.x, warp = tid >> 5;
-    unsigned char* rec = records + ((size_t)h * max_chunks + c) * R::BYTES;
+    const int ch = tid % DK, part = tid / DK, r0 = part * TPP;   // cumulative-sum mapping
 
     if (tid == 0) {
-        mbar_init(&bar_load, 1);
+        mbar_init(&bar_load[0], 1);
+        mbar_init(&bar_load[1], 1);
         mbar_init(&bar_mma, 1);
+        mbar_init(&bar_la, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(&s_tmem, 512);
+        tmem_alloc(&s_tmem, 256);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    const uint32_t R1 = tmem;         // [A; P]      128 lanes x 64 columns (fp32)
-    const uint32_t R2 = tmem + 128;   // [W | U0]    128 lanes x (DK + DV) columns
+    const uint32_t R1 = tmem;   // [A; P] 128 lanes x 64 columns, then [W | U0] 128 x (DK + DV)
+    const uint32_t R2 = tmem;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const int wg = warp >> 2;
+
+    // work item w -> (chunk, head); consecutive items are heads of one chunk
+    auto locate = [&](int w, int& c, int& h, int& tok0, int& L) {
+        c = w / H;
+        h = w - c * H;
+        int seq;
+        map.locate(c, seq, tok0, L);
+    };
+    auto issue_tma = [&](int w, int stage) {
+        int c, h, tok0, L;
+        locate(w, c, h, tok0, L);
+        unsigned char* st = sm + stage * Sm::STAGE;
+        mbar_arrive_expect_tx(&bar_load[stage], Sm::TX_BYTES);
+#pragma unroll
+        for (int b = 0; b < DK / 64; ++b) tma_load_3d(st + Sm::KS + b * Sm::TILE, &tm_k, &bar_load[stage], b * 64, h, tok0);
+#pragma unroll
+        for (int b = 0; b < DV / 64; ++b) tma_load_3d(st + Sm::VS + b * Sm::TILE, &tm_v, &bar_load[stage], b * 64, h, tok0);
+#pragma unroll
+        for (int b = 0; b < DK / 64; ++b) tma_load_3d(st + Sm::QS + b * Sm::TILE, &tm_q, &bar_load[stage], b * 64, h, tok0);
+    };
+    // log_alpha tile of item w into G (when G is free), by TMA
+    auto issue_la = [&](int w) {
+        int c, h, tok0, L;
+        locate(w, c, h, tok0, L);
+        mbar_arrive_expect_tx(&bar_la, Sm::LA_BYTES);
+        tma_load_3d(sm + Sm::G, &tm_la, &bar_la, 0, h, tok0);
+    };
+    // beta of item w into a register (threads 192..255, one token each)
+    float beta_next = 0.f;
+    auto load_beta = [&](int w) {
+        if (tid >= 192) {
+            int c, h, tok0, L;
+            locate(w, c, h, tok0, L);
+            const int r = tid - 192;
+            beta_next = (r < L) ? ld_prefetch_f32(beta + (size_t)(tok0 + r) * H + h) : 0.f;
+        }
+    };
 
     if (tid == 0) {
-        mbar_arrive_expect_tx(&bar_load, Sm::TX_BYTES);
-#pragma unroll
-        for (int b = 0; b < DK / 64; ++b) tma_load_3d(sm + Sm::KS + b * 8192, &tm_k, &bar_load, b * 64, h, tok0);
-#pragma unroll
-        for (int b = 0; b < DV / 64; ++b) tma_load_3d(sm + Sm::VS + b * 8192, &tm_v, &bar_load, b * 64, h, tok0);
-#pragma unroll
-        for (int b = 0; b < DK / 64; ++b) tma_load_3d(sm + Sm::QS + b * 8192, &tm_q, &bar_load, b * 64, h, tok0);
-        tma_load_3d(sm + Sm::LAS, &tm_la, &bar_load, 0, h, tok0);
+        issue_tma(blockIdx.x, 0);
+        issue_la(blockIdx.x);
     }
-    if (tid >= 192) {
-        const int r = tid - 192;
-        s_beta[r] = (r < L) ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
-    }
-    bool ok = mbar_wait_cycles(&bar_load, 0, kWaitCycles);
-    bool aborted = __syncthreads_or(!ok);
-    int mma_issued = 0;   // commits issued on bar_mma (uniform across the CTA)
+    load_beta(blockIdx.x);
+    bool aborted = false;
+    uint32_t mma_phase = 0;
+    int mma_pending = 0;      // commits issued on bar_mma not yet waited for
+    bool stored = false;      // thread 0 has bulk stores in flight
     float range_max = 0.f;
 
-    if (!aborted) {
-        // ---- decay pass: one thread per key channel ------------------------
-        if (tid < DK) {
-            const int ch = tid;
-            const float* las = reinterpret_cast<const float*>(sm + Sm::LAS);
-            float g[kChunk];
+    int it = 0;
+    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x, ++it) {
+        const int stage = it & 1;
+        unsigned char* st = sm + stage * Sm::STAGE;
+        int c, h, tok0, L;
+        locate(w, c, h, tok0, L);
+        unsigned char* rec = records + ((size_t)h * max_chunks + c) * R::BYTES;
+        if (tid >= 192) s_beta[tid - 192] = beta_next;
+
+        const int wn = w + gridDim.x;   // this CTA's next item
+        if (wn < total) load_beta(wn);
+
+        // ---- cumulative log-decay, in place over the log_alpha tile in G -------
+        float* g = reinterpret_cast<float*>(sm + Sm::G);   // [64][DK]
+        const bool ok_la = mbar_wait_cycles(&bar_la, it & 1, kWaitCycles);
+        const bool ok_load = mbar_wait_cycles(&bar_load[stage], (it >> 1) & 1, kWaitCycles);
+        if (__syncthreads_or(!(ok_la && ok_load))) { aborted = true; break; }
+        {
+            float la_cur[TPP];
             float acc = 0.f;
 #pragma unroll
-            for (int r = 0; r < kChunk; ++r) {
-                acc += (r < L) ? las[r * DK + ch] : 0.f;
-                g[r] = acc;
+            for (int i = 0; i < TPP; ++i) {
+                la_cur[i] = (r0 + i < L) ? g[(r0 + i) * DK + ch] : 0.f;
+                acc += la_cur[i];
             }
-            float gm = g[0], gl = g[0];
+            s_part[part * DK + ch] = acc;
+            __syncthreads();
+            acc = 0.f;
+            for (int p = 0; p < part; ++p) acc += s_part[p * DK + ch];
 #pragma unroll
-            for (int r = 0; r < kChunk; ++r) {
-                if (r == ((L - 1) >> 1)) gm = g[r];
-                if (r == L - 1) gl = g[r];
+            for (int i = 0; i < TPP; ++i) {
+                acc += la_cur[i];
+                g[(r0 + i) * DK + ch] = acc;
             }
-            const float egm = __expf(gm), eglm = __expf(gl - gm);
+        }
+        __syncthreads();
+        if (tid < DK) {
+            const float gm = g[((L - 1) >> 1) * DK + tid], gl = g[(L - 1) * DK + tid];
+            s_gm[tid] = gm;
+            s_egm[tid] = __expf(gm);
+            s_eglm[tid] = __expf(gl - gm);
+            reinterpret_cast<float*>(rec + R::GC)[tid] = expf(gl);
+        }
+        __syncthreads();
+
+        // ---- decayed operands: thread -> token row r = tid / 4, 8-channel groups
+        //      c8 = 8 (tid % 4) + 32 k; two neighbouring rows share an 8-thread
+        //      store phase and their swizzles differ, so the fp32 stores are
+        //      bank-conflict free
+        {
+            const int r = tid >> 2;
+            const bool live = r < L;
 #pragma unroll
-            for (int r = 0; r < kChunk; ++r) {
-                const uint32_t ho = h_off(r, ch, 8192);
-                float kk = 0.f, qq = 0.f;
-                if (r < L) {
-                    kk = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Sm::KS + ho));
-                    qq = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + Sm::QS + ho));
+            for (int k = 0; k < DK / 32; ++k) {
+                const int c8 = 8 * (tid & 3) + 32 * k;
+                const uint32_t ho = (c8 >> 6) * Sm::TILE + sw128_offset(r, (c8 & 63) * 2);   // 16-byte chunk
+                uint4 kraw = *reinterpret_cast<const uint4*>(st + Sm::KS + ho);
+                uint4 qraw = *reinterpret_cast<const uint4*>(st + Sm::QS + ho);
+                if (!live) { kraw = make_uint4(0, 0, 0, 0); qraw = kraw; }
+                const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(&kraw);
+                const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(&qraw);
+                const float4 g0 = *reinterpret_cast<const float4*>(g + r * DK + c8);
+                const float4 g1 = *reinterpret_cast<const float4*>(g + r * DK + c8 + 4);
+                const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                __align__(16) float ka[8], qa[8], kbm[8];
+                __align__(16) __half k0[8], q0[8], kh[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float kk = __bfloat162float(kb[e]), qq = __bfloat162float(qb[e]);
+                    const float gm = s_gm[c8 + e];
+                    const float em = __expf(gv[e] - gm);   // e^{g_r - g_m}
+                    const float eb = __expf(gm - gv[e]);   // e^{g_m - g_r}
+                    const float e0 = s_egm[c8 + e] * em;   // e^{g_r}
+                    const float eh = s_eglm[c8 + e] * eb;  // e^{g_{L-1} - g_r}
+                    ka[e] = round_tf32(kk * em);
+                    qa[e] = round_tf32(qq * em);
+                    kbm[e] = round_tf32(kk * eb);
+                    k0[e] = __float2half_rn(kk * e0);
+                    q0[e] = __float2half_rn(qq * e0);
+                    kh[e] = __float2half_rn(kk * eh);
                 }
-                const float em = __expf(g[r] - gm);   // e^{g_r - g_m}
-                const float eb = __expf(gm - g[r]);   // e^{g_m - g_r}
-                const float e0 = egm * em;            // e^{g_r}
-                const float eh = eglm * eb;           // e^{g_{L-1} - g_r}
-                *reinterpret_cast<float*>(sm + Sm::OPA + f_off(r, ch, 16384)) = round_tf32(kk * em);
-                *reinterpret_cast<float*>(sm + Sm::OPA + f_off(64 + r, ch, 16384)) = round_tf32(qq * em);
-                *reinterpret_cast<float*>(sm + Sm::OPB + f_off(r, ch, 8192)) = round_tf32(kk * eb);
-                *reinterpret_cast<__half*>(sm + Sm::KS + ho) = __float2half_rn(kk * e0);
-                const float qt = qq * e0, kh = kk * eh;
-                *reinterpret_cast<__half*>(rec + R::WQ + h_off(64 + r, ch, 16384)) = __float2half_rn(qt);
-                *reinterpret_cast<__half*>(rec + R::KH + ho) = __float2half_rn(kh);
-            }
-            reinterpret_cast<float*>(rec + R::GC)[ch] = expf(gl);
-        } else {
-            // v: bf16 -> fp16 in place (same swizzled slot), zero beyond the chunk
-            for (int idx = tid - DK; idx < kChunk * DV; idx += 256 - DK) {
-                const int r = idx / DV, j = idx - r * DV;
-                const uint32_t o = Sm::VS + h_off(r, j, 8192);
-                const float x = (r < L) ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + o)) : 0.f;
-                range_max = fmaxf(range_max, fabsf(x));
-                *reinterpret_cast<__half*>(sm + o) = __float2half_rn(x);
+                // tf32 operands: 8 fp32 = two 16-byte chunks of a 128-byte row
+                const uint32_t fo = (c8 >> 5) * 16384u, fob = (c8 >> 5) * 8192u;
+                const uint32_t fb = (c8 & 31) * 4;
+                *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(r, fb)) = *reinterpret_cast<const float4*>(ka);
+                *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(r, fb + 16)) = *reinterpret_cast<const float4*>(ka + 4);
+                *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(64 + r, fb)) = *reinterpret_cast<const float4*>(qa);
+                *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(64 + r, fb + 16)) = *reinterpret_cast<const float4*>(qa + 4);
+                *reinterpret_cast<float4*>(sm + Sm::OPB + fob + sw128_offset(r, fb)) = *reinterpret_cast<const float4*>(kbm);
+                *reinterpret_cast<float4*>(sm + Sm::OPB + fob + sw128_offset(r, fb + 16)) = *reinterpret_cast<const float4*>(kbm + 4);
+                *reinterpret_cast<uint4*>(st + Sm::KS + ho) = *reinterpret_cast<const uint4*>(k0);   // K~ (MMA2 operand)
+                *reinterpret_cast<uint4*>(st + Sm::QS + ho) = *reinterpret_cast<const uint4*>(q0);   // Q~ (record)
+                *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(kh);  // K^ (record)
             }
         }
         fence_proxy_async_smem();
+        tc_fence_before();
         __syncthreads();
-
-        // ---- MMA1 (tf32): [K~m; Q~m] K-m^T -> R1 ---------------------------
+        if (tid == 0 && wn < total) {
+            // prefetch the next item: log_alpha into G (free now) and its k, v, q
+            // tiles into the other stage (free once the bulk stores of the item
+            // that used it have read their tiles)
+            issue_la(wn);
+            if (stored) bulk_store_wait_read();
+            issue_tma(wn, stage ^ 1);
+        }
         if (tid == 0) {
+            // Q~ tiles are the lower halves (rows 64..127) of the record's WQ tiles
+#pragma unroll
+            for (int b = 0; b < DK / 64; ++b)
+                bulk_store(rec + R::WQ + b * 16384 + 8192, st + Sm::QS + b * Sm::TILE, 8192);
+            bulk_store_commit();
+            stored = true;
+            // ---- MMA1 (tf32): [K~m; Q~m] K-m^T -> R1 (overlaps the v conversion)
             tc_fence_after();
             constexpr uint32_t idesc = instr_desc(kFmtTF32, 128, 64);
             const uint32_t a0 = smem_u32(sm + Sm::OPA), b0 = smem_u32(sm + Sm::OPB);
@@ -223,92 +352,186 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                              (kb | ks) != 0);
             mma_commit(&bar_mma);
         }
-        mma_issued = 1;
-        ok = mbar_wait_cycles(&bar_mma, 0, kWaitCycles);
-        aborted = __syncthreads_or(!ok);
-    }
-    if (!aborted) {
+        mma_pending = 1;
+        // v: bf16 -> fp16 in place, 8 values per thread and step
+        for (int item = tid; item < kChunk * (DV / 8); item += 256) {
+            const int r = item / (DV / 8), j8 = (item - r * (DV / 8)) * 8;
+            const uint32_t o = Sm::VS + (j8 >> 6) * Sm::TILE + sw128_offset(r, (j8 & 63) * 2);
+            uint4 raw = *reinterpret_cast<const uint4*>(st + o);
+            if (r >= L) raw = make_uint4(0, 0, 0, 0);
+            const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(&raw);
+            __align__(16) __half vh[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float x = __bfloat162float(vb[e]);
+                range_max = fmaxf(range_max, fabsf(x));
+                vh[e] = __float2half_rn(x);
+            }
+            *reinterpret_cast<uint4*>(st + o) = *reinterpret_cast<const uint4*>(vh);
+        }
+        fence_proxy_async_smem();   // fp16 v (MMA2 operand)
+        bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        mma_phase ^= 1;
+        mma_pending = 0;
         tc_fence_after();
-        // ---- A to shared memory (rows 0..63), P to the record (rows 64..127)
-        float* am = reinterpret_cast<float*>(sm + Sm::AM);  // [64][65]
-        if (tid < 128) {
+
+        // ---- A (rows 0..63, beta-scaled, strictly lower) to smem; P (rows
+        //      64..127, lower incl. diagonal) to the record
+        float* am = reinterpret_cast<float*>(sm + Sm::AM);   // [64][68]
+        float* tmx = reinterpret_cast<float*>(sm + Sm::TM);  // [64][68]
+        float* ym = reinterpret_cast<float*>(sm + Sm::YM);   // [6][16][17]
+        {
             float v[32];
-            const int row = tid;   // TMEM lane = MMA row
+            const int row = (warp & 3) * 32 + (tid & 31);
+            tmem_ld32_sync(R1 + lane_base + 32 * wg, v);
+            if (row < 64) {
+                const float b = s_beta[row];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32_sync(R1 + lane_base + 32 * half, v);
-                if (row < 64) {
-                    const float b = s_beta[row];
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    float4 a4;
+                    const int col = 32 * wg + 4 * i4;
+                    a4.x = (col + 0 < row) ? b * v[4 * i4 + 0] : 0.f;
+                    a4.y = (col + 1 < row) ? b * v[4 * i4 + 1] : 0.f;
+                    a4.z = (col + 2 < row) ? b * v[4 * i4 + 2] : 0.f;
+                    a4.w = (col + 3 < row) ? b * v[4 * i4 + 3] : 0.f;
+                    *reinterpret_cast<float4*>(am + row * 68 + col) = a4;
+                }
+            } else {
+                const int r = row - 64;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int col = 32 * half + i;
-                        am[row * 65 + col] = (col < row) ? b * v[i] : 0.f;
+                for (int i8 = 0; i8 < 4; ++i8) {
+                    __align__(16) __half hv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int col = 32 * wg + 8 * i8 + e;
+                        hv[e] = __float2half_rn(col <= r ? v[8 * i8 + e] : 0.f);
                     }
-                } else {
-                    const int r = row - 64;
-#pragma unroll
-                    for (int i8 = 0; i8 < 4; ++i8) {
-                        __align__(16) __half hv[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int col = 32 * half + 8 * i8 + e;
-                            hv[e] = __float2half_rn(col <= r ? v[8 * i8 + e] : 0.f);
-                        }
-                        *reinterpret_cast<uint4*>(rec + R::P + sw128_offset(r, (32 * half + 8 * i8) * 2)) =
-                            *reinterpret_cast<const uint4*>(hv);
-                    }
+                    *reinterpret_cast<uint4*>(rec + R::P + sw128_offset(r, (32 * wg + 8 * i8) * 2)) =
+                        *reinterpret_cast<const uint4*>(hv);
                 }
             }
         }
         __syncthreads();
 
-        // ---- T = (I + A)^{-1}: column tid by forward substitution ----------
-        if (tid < kChunk) {
-            float x[kChunk];
+        // ---- T = (I + A)^{-1} in 16 x 16 blocks, written as fp16 T diag(beta)
+        //      (K-major, rows 0..63) as soon as each block is final.
+        //      D_b = (I + A_bb)^{-1};  E_im = D_i A_im (i > m);
+        //      T_{b+l,b} = -sum_{m=b}^{b+l-1} E_{b+l,m} T_{m,b}
+        auto put_t = [&](int row, int col, float t) {
+            *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(row, col * 2)) = __float2half_rn(t * s_beta[col]);
+        };
+        float* em_ = ym;   // E blocks: 6 x 16 x 17 fp32
+        if (tid < 64) {    // diagonal blocks, one column per thread
+            const int b = tid >> 4, cc = tid & 15, base = 16 * b;
+            float x[16];
 #pragma unroll
-            for (int r = 0; r < kChunk; ++r) {
-                float a0 = (r == tid) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            for (int j = 0; j < 16; ++j) {
+                const float* arow = am + (base + j) * 68 + base;
+                float av[16];
 #pragma unroll
-                for (int i = 0; i + 3 < r; i += 4) {
-                    a0 -= am[r * 65 + i] * x[i];
-                    a1 -= am[r * 65 + i + 1] * x[i + 1];
-                    a2 -= am[r * 65 + i + 2] * x[i + 2];
-                    a3 -= am[r * 65 + i + 3] * x[i + 3];
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(arow + 4 * k4);
+                    av[4 * k4] = t4.x; av[4 * k4 + 1] = t4.y; av[4 * k4 + 2] = t4.z; av[4 * k4 + 3] = t4.w;
                 }
+                float a0 = (j == cc) ? 1.f : 0.f, a1 = 0.f;
 #pragma unroll
-                for (int i = r & ~3; i < r; ++i) a0 -= am[r * 65 + i] * x[i];
-                x[r] = (a0 + a1) + (a2 + a3);
+                for (int k = 0; k + 1 < j; k += 2) {
+                    a0 -= av[k] * x[k];
+                    a1 -= av[k + 1] * x[k + 1];
+                }
+                if (j & 1) a0 -= av[j - 1] * x[j - 1];
+                x[j] = a0 + a1;
+                tmx[(base + j) * 68 + base + cc] = x[j];
+                put_t(base + j, base + cc, x[j]);
             }
-            const float bt = s_beta[tid];
+        } else {           // zeros above the diagonal blocks
+            for (int o = tid - 64; o < 6 * 256; o += 192) {
+                const int pair = o >> 8, p = (o >> 4) & 15, q = o & 15;
+                const int i = pair < 3 ? 0 : (pair < 5 ? 1 : 2);
+                const int j = pair < 3 ? pair + 1 : (pair < 5 ? pair - 1 : 3);
+                *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(16 * i + p, (16 * j + q) * 2)) = __float2half_rn(0.f);
+            }
+        }
+        __syncthreads();
+        // E_im = D_i A_im for the 6 pairs i > m (pair index: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)),
+        // 2 x 2 outputs per thread
+        for (int o = tid; o < 6 * 64; o += 256) {
+            const int pair = o >> 6, p0 = ((o >> 3) & 7) * 2, q0 = (o & 7) * 2;
+            const int i = pair == 0 ? 1 : (pair < 3 ? 2 : 3);
+            const int m = pair == 0 ? 0 : (pair == 1 ? 0 : (pair == 2 ? 1 : pair - 3));
+            const float* d0 = tmx + (16 * i + p0) * 68 + 16 * i;
+            const float* d1 = d0 + 68;
+            float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
 #pragma unroll
-            for (int r = 0; r < kChunk; ++r)   // T diag(beta), K-major row r, column tid
-                *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(r, tid * 2)) = __float2half_rn(x[r] * bt);
+            for (int k = 0; k < 16; ++k) {
+                const float2 a = *reinterpret_cast<const float2*>(am + (16 * i + k) * 68 + 16 * m + q0);
+                const float e0 = d0[k], e1 = d1[k];
+                c00 += e0 * a.x; c01 += e0 * a.y; c10 += e1 * a.x; c11 += e1 * a.y;
+            }
+            float* out = em_ + (pair * 16 + p0) * 17 + q0;
+            out[0] = c00; out[1] = c01; out[17] = c10; out[18] = c11;
+        }
+        __syncthreads();
+        // T_{b+l,b} = -sum_{m=b}^{b+l-1} E_{b+l,m} T_{m,b}, 2 x 2 outputs per thread
+#pragma unroll 1
+        for (int l = 1; l < 4; ++l) {
+            for (int o = tid; o < (4 - l) * 64; o += 256) {
+                const int b = o >> 6, p0 = ((o >> 3) & 7) * 2, q0 = (o & 7) * 2;
+                const int i = b + l, j = b;
+                float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
+                for (int m = j; m < i; ++m) {
+                    const int pair = i == 1 ? 0 : (i == 2 ? 1 + m : 3 + m);
+                    const float* e0p = em_ + (pair * 16 + p0) * 17;
+                    const float* e1p = e0p + 17;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float2 t = *reinterpret_cast<const float2*>(tmx + (16 * m + k) * 68 + 16 * j + q0);
+                        const float e0 = e0p[k], e1 = e1p[k];
+                        c00 += e0 * t.x; c01 += e0 * t.y; c10 += e1 * t.x; c11 += e1 * t.y;
+                    }
+                }
+                const int r = 16 * i + p0, cidx = 16 * j + q0;
+                tmx[r * 68 + cidx] = -c00;
+                tmx[r * 68 + cidx + 1] = -c01;
+                tmx[(r + 1) * 68 + cidx] = -c10;
+                tmx[(r + 1) * 68 + cidx + 1] = -c11;
+                put_t(r, cidx, -c00);
+                put_t(r, cidx + 1, -c01);
+                put_t(r + 1, cidx, -c10);
+                put_t(r + 1, cidx + 1, -c11);
+            }
+            __syncthreads();
         }
         fence_proxy_async_smem();
+        tc_fence_before();
         __syncthreads();
 
         // ---- MMA2 (fp16): [T diag(beta); *] [K~ | V] -> R2 -----------------
         if (tid == 0) {
             tc_fence_after();
             constexpr uint32_t idesc = instr_desc(kFmtF16, 128, DK + DV, false, true);
-            const uint32_t a0 = smem_u32(sm + Sm::TP), b0 = smem_u32(sm + Sm::KS);
+            const uint32_t a0 = smem_u32(sm + Sm::TP), b0 = smem_u32(st + Sm::KS);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_f16(R2, smem_desc(a0 + ks * 32, 16, 1024, kLayoutSW128),
-                        smem_desc(b0 + ks * 2048, 8192, 1024, kLayoutSW128), idesc, ks != 0);
+                        smem_desc(b0 + ks * 2048, Sm::TILE, 1024, kLayoutSW128), idesc, ks != 0);
             mma_commit(&bar_mma);
         }
-        mma_issued = 2;
-        ok = mbar_wait_cycles(&bar_mma, 1, kWaitCycles);
-        aborted = __syncthreads_or(!ok);
-    }
-    if (!aborted) {
+        mma_pending = 1;
+        ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        mma_phase ^= 1;
+        mma_pending = 0;
         tc_fence_after();
-        // ---- W and U0 (rows 0..63) to the record ---------------------------
-        if (tid < 64) {
-            const int r = tid;
+
+        // ---- W and U0 (rows 0..63): fp16 into the stage's k/v tiles (free after
+        //      MMA2; same 64-row swizzled tile layout as the record), then one
+        //      bulk store per tile.  The two warpgroups take alternate 32-column chunks.
+        if ((warp & 3) < 2) {
+            const int r = (warp & 3) * 32 + (tid & 31);
 #pragma unroll
-            for (int cb = 0; cb < (DK + DV) / 32; ++cb) {
+            for (int cb = wg; cb < (DK + DV) / 32; cb += 2) {
                 float v[32];
                 tmem_ld32_sync(R2 + lane_base + 32 * cb, v);
 #pragma unroll
@@ -319,23 +542,36 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                         range_max = fmaxf(range_max, fabsf(v[8 * i8 + e]));
                         hv[e] = __float2half_rn(v[8 * i8 + e]);
                     }
-                    const int col = 32 * cb + 8 * i8;
-                    unsigned char* dst = (col < DK) ? rec + R::WQ + h_off(r, col, 16384)
-                                                    : rec + R::U0 + h_off(r, col - DK, 8192);
-                    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(hv);
+                    const int col = 32 * cb + 8 * i8;   // k tiles then v tiles, 64 columns each
+                    *reinterpret_cast<uint4*>(st + Sm::KS + h_off(r, col, Sm::TILE)) = *reinterpret_cast<const uint4*>(hv);
                 }
             }
         }
-    } else {
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+#pragma unroll
+            for (int b = 0; b < DK / 64; ++b)   // W: rows 0..63 of each WQ tile
+                bulk_store(rec + R::WQ + b * 16384, st + Sm::KS + b * Sm::TILE, Sm::TILE);
+            bulk_store(rec + R::U0, st + Sm::VS, (DV / 64) * Sm::TILE);
+            bulk_store_commit();
+        }
+        tc_fence_before();
+        __syncthreads();   // R1/R2, TP and the stage are free for the next item
+    }
+
+    if (aborted) {
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         // let this CTA's own copies and MMAs finish (bounded) before freeing
-        (void)mbar_wait_cycles(&bar_load, 0, kWaitCycles);
-        if (mma_issued > 0) (void)mbar_wait_cycles(&bar_mma, (uint32_t)(mma_issued - 1), kWaitCycles);
+        for (int s2 = 0; s2 < 2; ++s2) (void)mbar_wait_cycles(&bar_load[s2], 0, kWaitCycles / 4);
+        (void)mbar_wait_cycles(&bar_la, 0, kWaitCycles / 4);
+        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
     }
+    if (stored) bulk_store_wait_all();
     if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // ---------------------------------------------------------------- K2 ----
@@ -642,10 +878,14 @@ cudaError_t launch_intra_tc_t(const ChunkArgs& a) {
         return cudaErrorInvalidValue;
     ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
     auto kern = intra_chunk_tc_kernel<DK, DV>;
-    const int smem = (int)K1Smem<DK, DV>::END + 1024;
+    const int smem = (int)K1Smem<DK, DV>::TOTAL;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)a.max_chunks, (unsigned)a.H);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const size_t items = a.max_chunks * (size_t)a.H;   // upper bound; the kernel reads the exact count
+    const unsigned grid = (unsigned)(items < (size_t)sms ? items : (size_t)sms);
     kern<<<grid, 256, smem, a.stream>>>(mk, mv, mq, mla, a.beta, map, static_cast<WsHeader*>(a.ws_header),
                                         static_cast<unsigned char*>(a.records), a.H, a.max_chunks);
     return cudaGetLastError();

@@ -13,6 +13,7 @@ constexpr int kHeaderBytes = 256;   // workspace header (status word, counts)
 // Device status codes written into the workspace header (same values as
 // kda_status in include/kda.h).
 constexpr int kStatusOk = 0;
+constexpr int kStatusInternal = 3;   // reported as KDA_ERR_CUDA
 constexpr int kStatusTimeout = 4;
 constexpr int kStatusBadSeqlens = 6;
 constexpr int kStatusRange = 7;

@@ -64,6 +64,14 @@ __device__ __forceinline__ bool mbar_wait_cycles(uint64_t* bar, uint32_t parity,
     return true;
 }
 
+// Global load that the compiler may not move (a prefetch into registers
+// that is consumed much later, e.g. in the next loop iteration).
+__device__ __forceinline__ float ld_prefetch_f32(const float* p) {
+    float v;
+    asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
 // --------------------------------------------------------------- fences ---
 // Generic-proxy writes to shared memory -> visible to the async proxy.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -112,6 +120,17 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+
+// Contiguous shared -> global copy (bulk async group); the source may be
+// reused only after bulk_store_wait_read().
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(smem_u32(src)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Wait only until the shared-memory sources of all committed bulk stores have been read.
+__device__ __forceinline__ void bulk_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // ------------------------------------------------------------- tcgen05 ----
 // Allocate `ncols` (power of two, >= 32) TMEM columns; one full warp calls
