@@ -289,23 +289,39 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                 const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(&qraw);
                 const float4 g0 = *reinterpret_cast<const float4*>(g + r * DK + c8);
                 const float4 g1 = *reinterpret_cast<const float4*>(g + r * DK + c8 + 4);
+                const float4 m0 = *reinterpret_cast<const float4*>(s_gm + c8);
+                const float4 m1 = *reinterpret_cast<const float4*>(s_gm + c8 + 4);
+                const float4 x0 = *reinterpret_cast<const float4*>(s_egm + c8);
+                const float4 x1 = *reinterpret_cast<const float4*>(s_egm + c8 + 4);
+                const float4 y0 = *reinterpret_cast<const float4*>(s_eglm + c8);
+                const float4 y1 = *reinterpret_cast<const float4*>(s_eglm + c8 + 4);
                 const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                const float gmv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                const float egmv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                const float eglmv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
                 __align__(16) float ka[8], qa[8], kbm[8];
-                __align__(16) __half k0[8], q0[8], kh[8];
+                __align__(16) __half2 k0[4], q0[4], kh[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float kk = __bfloat162float(kb[e]), qq = __bfloat162float(qb[e]);
-                    const float gm = s_gm[c8 + e];
-                    const float em = __expf(gv[e] - gm);   // e^{g_r - g_m}
-                    const float eb = __expf(gm - gv[e]);   // e^{g_m - g_r}
-                    const float e0 = s_egm[c8 + e] * em;   // e^{g_r}
-                    const float eh = s_eglm[c8 + e] * eb;  // e^{g_{L-1} - g_r}
-                    ka[e] = round_tf32(kk * em);
-                    qa[e] = round_tf32(qq * em);
-                    kbm[e] = round_tf32(kk * eb);
-                    k0[e] = __float2half_rn(kk * e0);
-                    q0[e] = __float2half_rn(qq * e0);
-                    kh[e] = __float2half_rn(kk * eh);
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    float k0v[2], q0v[2], khv[2];
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int e = 2 * e2 + h2;
+                        const float kk = __bfloat162float(kb[e]), qq = __bfloat162float(qb[e]);
+                        const float em = __expf(gv[e] - gmv[e]);   // e^{g_r - g_m}
+                        const float eb = __expf(gmv[e] - gv[e]);   // e^{g_m - g_r}
+                        const float e0 = egmv[e] * em;             // e^{g_r}
+                        const float eh = eglmv[e] * eb;            // e^{g_{L-1} - g_r}
+                        ka[e] = round_tf32_alu(kk * em);
+                        qa[e] = round_tf32_alu(qq * em);
+                        kbm[e] = round_tf32_alu(kk * eb);
+                        k0v[h2] = kk * e0;
+                        q0v[h2] = qq * e0;
+                        khv[h2] = kk * eh;
+                    }
+                    k0[e2] = __floats2half2_rn(k0v[0], k0v[1]);
+                    q0[e2] = __floats2half2_rn(q0v[0], q0v[1]);
+                    kh[e2] = __floats2half2_rn(khv[0], khv[1]);
                 }
                 // tf32 operands: 8 fp32 = two 16-byte chunks of a 128-byte row
                 const uint32_t fo = (c8 >> 5) * 16384u, fob = (c8 >> 5) * 8192u;
@@ -359,13 +375,13 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             const uint32_t o = Sm::VS + (j8 >> 6) * Sm::TILE + sw128_offset(r, (j8 & 63) * 2);
             uint4 raw = *reinterpret_cast<const uint4*>(st + o);
             if (r >= L) raw = make_uint4(0, 0, 0, 0);
-            const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(&raw);
-            __align__(16) __half vh[8];
+            const __nv_bfloat162* vb = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            __align__(16) __half2 vh[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float x = __bfloat162float(vb[e]);
-                range_max = fmaxf(range_max, fabsf(x));
-                vh[e] = __float2half_rn(x);
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = __bfloat1622float2(vb[e]);
+                range_max = fmaxf(range_max, fmaxf(fabsf(x.x), fabsf(x.y)));
+                vh[e] = __floats2half2_rn(x.x, x.y);
             }
             *reinterpret_cast<uint4*>(st + o) = *reinterpret_cast<const uint4*>(vh);
         }
@@ -434,14 +450,10 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                     const float4 t4 = *reinterpret_cast<const float4*>(arow + 4 * k4);
                     av[4 * k4] = t4.x; av[4 * k4 + 1] = t4.y; av[4 * k4 + 2] = t4.z; av[4 * k4 + 3] = t4.w;
                 }
-                float a0 = (j == cc) ? 1.f : 0.f, a1 = 0.f;
+                float acc4[4] = {(j == cc) ? 1.f : 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int k = 0; k + 1 < j; k += 2) {
-                    a0 -= av[k] * x[k];
-                    a1 -= av[k + 1] * x[k + 1];
-                }
-                if (j & 1) a0 -= av[j - 1] * x[j - 1];
-                x[j] = a0 + a1;
+                for (int k = 0; k < j; ++k) acc4[k & 3] -= av[k] * x[k];
+                x[j] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
                 tmx[(base + j) * 68 + base + cc] = x[j];
                 put_t(base + j, base + cc, x[j]);
             }
@@ -595,7 +607,7 @@ struct K2Smem {
 };
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict__ final_state,
                       __nv_bfloat16* __restrict__ o, ChunkMap map, WsHeader* hdr,
                       const unsigned char* __restrict__ records, int H, size_t max_chunks, float scale)
@@ -610,6 +622,8 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
     if (hdr->status != kStatusOk) return;
     const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSliceTc;
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int lane_row = (warp & 3) * 32 + (tid & 31);   // TMEM lane = MMA row
+    const int wg = warp >> 2;                            // warpgroup: columns [32 wg, 32 wg + 32)
     const int first = map.seq_first_chunk(s), nch = map.seq_num_chunks(s);
     const int tok_begin = map.seq_token_begin(s), tok_end = map.seq_token_end(s);
     const size_t state_off = ((size_t)s * H + h) * DK * DV;
@@ -621,15 +635,16 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(&s_tmem, 128);
+        tmem_alloc(&s_tmem, 256);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    const uint32_t R3 = tmem;        // [W S; Q~ S + P U]   128 lanes x 64
-    const uint32_t SACC = tmem + 64; // state slice (fp32)  lanes = key channel
+    // [W S; Q~ S + P U] of chunk n at columns 64 (n & 1) (128 lanes x 64), then the state slice
+    auto r3 = [&](int n) -> uint32_t { return tmem + 64u * (uint32_t)(n & 1); };
+    const uint32_t SACC = tmem + 128;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     float range_max = 0.f;
 
@@ -645,32 +660,52 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
         bulk_load(st + Sm::U0, rec + R::U0 + (j0 / 64) * 8192, 8192, bar);
         bulk_load(st + Sm::GC, rec + R::GC, DK * 4, bar);
     };
-
-    // initial state slice -> TMEM accumulator and fp16 operand copy
-    if (tid < DK) {
-        float v[32];
+    // fp16 copy of 32 state columns of this thread's key channel (row of S16)
+    auto put_s16 = [&](const float (&v)[32]) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int i8 = 0; i8 < 4; ++i8) {
+            __align__(16) __half2 hv[4];
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (initial_state)
-                    x = *reinterpret_cast<const float4*>(initial_state + state_off + (size_t)tid * DV + j0 + 32 * half + i);
-                v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+            for (int e = 0; e < 4; ++e) {
+                const float a = v[8 * i8 + 2 * e], b = v[8 * i8 + 2 * e + 1];
+                range_max = fmaxf(range_max, fmaxf(fabsf(a), fabsf(b)));
+                hv[e] = __floats2half2_rn(a, b);
             }
-            tmem_st32_sync(SACC + lane_base + 32 * half, v);
+            *reinterpret_cast<uint4*>(sm + Sm::S16 + sw128_offset(lane_row, (32 * wg + 8 * i8) * 2)) =
+                *reinterpret_cast<const uint4*>(hv);
+        }
+    };
+    // output rows (lanes 64..127) of chunk n from R3[n & 1]: warps 2, 3, 6, 7
+    auto write_o = [&](int n) {
+        const int r = lane_row - 64;
+        const int tok = tok_begin + n * kChunk + r;
+        float v[32];
+        tmem_ld32_sync(r3(n) + lane_base + 32 * wg, v);
+        if (tok < tok_end) {
+            __nv_bfloat16* dst = o + ((size_t)tok * H + h) * DV + j0 + 32 * wg;
 #pragma unroll
             for (int i8 = 0; i8 < 4; ++i8) {
-                __align__(16) __half hv[8];
+                __align__(16) __nv_bfloat162 bv[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    range_max = fmaxf(range_max, fabsf(v[8 * i8 + e]));
-                    hv[e] = __float2half_rn(v[8 * i8 + e]);
-                }
-                *reinterpret_cast<uint4*>(sm + Sm::S16 + sw128_offset(tid, (32 * half + 8 * i8) * 2)) =
-                    *reinterpret_cast<const uint4*>(hv);
+                for (int e = 0; e < 4; ++e)
+                    bv[e] = __floats2bfloat162_rn(scale * v[8 * i8 + 2 * e], scale * v[8 * i8 + 2 * e + 1]);
+                *reinterpret_cast<uint4*>(dst + 8 * i8) = *reinterpret_cast<const uint4*>(bv);
             }
         }
+    };
+
+    // initial state slice -> TMEM accumulator and fp16 operand copy
+    if (lane_row < DK) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (initial_state)
+                x = *reinterpret_cast<const float4*>(initial_state + state_off + (size_t)lane_row * DV + j0 + 32 * wg + i);
+            v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+        }
+        tmem_st32_sync(SACC + lane_base + 32 * wg, v);
+        put_s16(v);
     }
     if (tid == 0) {
         issue(0);
@@ -683,12 +718,14 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
 
     bool aborted = false;
     uint32_t mma_phase = 0;
-    for (int n = 0; n < nch && !aborted; ++n) {
+    int n = 0;
+    for (; n < nch; ++n) {
         const int b = n & 1;
         unsigned char* st = sm + b * Sm::STAGE;
         bool ok = mbar_wait_cycles(&bar_full[b], (n >> 1) & 1, kWaitCycles);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
 
+        const uint32_t R3 = r3(n);
         // MMA3: [W; Q~] S -> R3
         if (tid == 0) {
             tc_fence_after();
@@ -703,44 +740,41 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
                             (kb | ks) != 0);
             mma_commit(&bar_mma);
         }
-        // meanwhile: S_acc <- Diag(gC) S_acc (MMA3 reads the fp16 copy, not S_acc)
-        if (tid < DK) {
-            const float gc = reinterpret_cast<const float*>(st + Sm::GC)[tid];
+        // meanwhile: S_acc <- Diag(gC) S_acc (MMA3 reads the fp16 copy, not S_acc),
+        // and the previous chunk's output rows
+        if (lane_row < DK) {
+            const float gc = reinterpret_cast<const float*>(st + Sm::GC)[lane_row];
             float v[32];
+            tmem_ld32_sync(SACC + lane_base + 32 * wg, v);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32_sync(SACC + lane_base + 32 * half, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= gc;
-                tmem_st32_sync(SACC + lane_base + 32 * half, v);
-            }
+            for (int i = 0; i < 32; ++i) v[i] *= gc;
+            tmem_st32_sync(SACC + lane_base + 32 * wg, v);
         }
+        if (n > 0 && lane_row >= 64) write_o(n - 1);
         ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
         mma_phase ^= 1;
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         tc_fence_after();
 
         // U = U0 - W S  (rows 0..63 = tokens), fp16 -> U16
-        if (tid < 64) {
-            const int r = tid;
+        if (lane_row < 64) {
+            const int r = lane_row;
+            float v[32];
+            tmem_ld32_sync(R3 + lane_base + 32 * wg, v);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float v[32];
-                tmem_ld32_sync(R3 + lane_base + 32 * half, v);
+            for (int i8 = 0; i8 < 4; ++i8) {
+                const uint32_t off = sw128_offset(r, (32 * wg + 8 * i8) * 2);
+                const uint4 u0raw = *reinterpret_cast<const uint4*>(st + Sm::U0 + off);
+                const __half2* u0 = reinterpret_cast<const __half2*>(&u0raw);
+                __align__(16) __half2 hv[4];
 #pragma unroll
-                for (int i8 = 0; i8 < 4; ++i8) {
-                    const uint32_t off = sw128_offset(r, (32 * half + 8 * i8) * 2);
-                    const uint4 u0raw = *reinterpret_cast<const uint4*>(st + Sm::U0 + off);
-                    const __half* u0 = reinterpret_cast<const __half*>(&u0raw);
-                    __align__(16) __half hv[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float u = __half2float(u0[e]) - v[8 * i8 + e];
-                        range_max = fmaxf(range_max, fabsf(u));
-                        hv[e] = __float2half_rn(u);
-                    }
-                    *reinterpret_cast<uint4*>(sm + Sm::U16 + off) = *reinterpret_cast<const uint4*>(hv);
+                for (int e = 0; e < 4; ++e) {
+                    const float2 u0f = __half22float2(u0[e]);
+                    const float ua = u0f.x - v[8 * i8 + 2 * e], ub = u0f.y - v[8 * i8 + 2 * e + 1];
+                    range_max = fmaxf(range_max, fmaxf(fabsf(ua), fabsf(ub)));
+                    hv[e] = __floats2half2_rn(ua, ub);
                 }
+                *reinterpret_cast<uint4*>(sm + Sm::U16 + off) = *reinterpret_cast<const uint4*>(hv);
             }
         }
         fence_proxy_async_smem();
@@ -772,45 +806,12 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
             fence_proxy_async_smem();
             issue(n + 2);   // this stage is no longer read
         }
-
-        // O = scale (Q~ S + P U): rows 64..127
-        if (tid >= 64) {
-            const int r = tid - 64;
-            const int tok = tok_begin + n * kChunk + r;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float v[32];
-                tmem_ld32_sync(R3 + lane_base + 32 * half, v);
-                if (tok < tok_end) {
-                    __nv_bfloat16* dst = o + ((size_t)tok * H + h) * DV + j0 + 32 * half;
-#pragma unroll
-                    for (int i8 = 0; i8 < 4; ++i8) {
-                        __align__(16) __nv_bfloat16 bv[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) bv[e] = __float2bfloat16_rn(scale * v[8 * i8 + e]);
-                        *reinterpret_cast<uint4*>(dst + 8 * i8) = *reinterpret_cast<const uint4*>(bv);
-                    }
-                }
-            }
-        }
-        // next state's fp16 operand copy
-        if (tid < DK) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float v[32];
-                tmem_ld32_sync(SACC + lane_base + 32 * half, v);
-#pragma unroll
-                for (int i8 = 0; i8 < 4; ++i8) {
-                    __align__(16) __half hv[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        range_max = fmaxf(range_max, fabsf(v[8 * i8 + e]));
-                        hv[e] = __float2half_rn(v[8 * i8 + e]);
-                    }
-                    *reinterpret_cast<uint4*>(sm + Sm::S16 + sw128_offset(tid, (32 * half + 8 * i8) * 2)) =
-                        *reinterpret_cast<const uint4*>(hv);
-                }
-            }
+        // next state's fp16 operand copy (the serial path); the output rows of
+        // this chunk are written during the next chunk's MMA3
+        if (lane_row < DK) {
+            float v[32];
+            tmem_ld32_sync(SACC + lane_base + 32 * wg, v);
+            put_s16(v);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -823,12 +824,12 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
         // let MMAs and copies this CTA issued finish before its memory goes away
         (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
         for (int b = 0; b < 2; ++b) (void)mbar_wait_cycles(&bar_full[b], 0, kWaitCycles / 8);
-    } else if (final_state && tid < DK) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+    } else {
+        if (nch > 0 && lane_row >= 64) write_o(nch - 1);
+        if (final_state && lane_row < DK) {
             float v[32];
-            tmem_ld32_sync(SACC + lane_base + 32 * half, v);
-            float* dst = final_state + state_off + (size_t)tid * DV + j0 + 32 * half;
+            tmem_ld32_sync(SACC + lane_base + 32 * wg, v);
+            float* dst = final_state + state_off + (size_t)lane_row * DV + j0 + 32 * wg;
 #pragma unroll
             for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
         }
@@ -836,7 +837,7 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
     if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 128);
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // ------------------------------------------------------------- host -----
@@ -899,7 +900,7 @@ cudaError_t launch_inter_tc_t(const ChunkArgs& a) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.num_seqs, (unsigned)a.H, (unsigned)(DV / kSliceTc));
-    kern<<<grid, 128, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<__nv_bfloat16*>(a.o), map,
+    kern<<<grid, 256, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<__nv_bfloat16*>(a.o), map,
                                         static_cast<WsHeader*>(a.ws_header),
                                         static_cast<const unsigned char*>(a.records), a.H, a.max_chunks, a.scale);
     return cudaGetLastError();

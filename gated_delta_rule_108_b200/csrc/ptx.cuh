@@ -276,6 +276,14 @@ __device__ __forceinline__ float round_tf32(float x) {
     return __uint_as_float(r);
 }
 
+// The same rounding (to the nearest value with a 10-bit mantissa, ties away
+// from zero) done with integer operations on the bit pattern: add half a unit
+// of the 11th mantissa bit, then clear the low 13 bits.  Keeps the conversion
+// off the special-function pipe.  Finite inputs only (inf/NaN are not used).
+__device__ __forceinline__ float round_tf32_alu(float x) {
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+}
+
 // Byte offset of element (row, byte b) inside a K-major, 128-byte-swizzled
 // operand tile whose rows are 128 bytes long: 8-row atoms of 1024 bytes, the
 // 16-byte chunk index XOR-ed with (row mod 8).
