@@ -318,7 +318,12 @@ def run_ours(args):
     out_bytes = w.dv * eb                                          # o
     state_bytes = 2 * w.num_seqs * w.H * w.dk * w.dv * 4           # S0 read + final write
     n_chunks = w.num_seqs * ((w.T + 63) // 64) * w.H
-    rec_bytes = 4 * (64 * (3 * w.dk + w.dv + 64) + w.dk)           # fp32 intermediates per chunk-head
+    # chunk intermediates written by the intra-chunk kernel and read by the
+    # inter-chunk kernel, per chunk and head: W, Q~, K^ [64 x dk], P [64 x 64],
+    # U0 [64 x dv] (fp16 on the bf16 tensor-core path, fp32 on the fp32 path)
+    # and gC [dk] fp32
+    rec_eb = 2 if w.dtype == torch.bfloat16 else 4
+    rec_bytes = rec_eb * 64 * (3 * w.dk + w.dv + 64) + 4 * w.dk
     kernels = {
         "intra_chunk": (th * in_bytes + n_chunks * rec_bytes, res["stages"]["intra_chunk"]),
         "inter_chunk": (n_chunks * rec_bytes + th * out_bytes + state_bytes, res["stages"]["inter_chunk"]),
