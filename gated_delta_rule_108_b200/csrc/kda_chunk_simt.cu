@@ -150,11 +150,15 @@ intra_chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const 
         sm.beta[r] = (r < L) ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
     }
     __syncthreads();
+    bool wide = false;
     if (tid < DK) {
         sm.gref[tid] = sm.g[(L - 1) >> 1][tid];
         sm.gend[tid] = sm.g[L - 1][tid];
+        wide = fmaxf(sm.g[0][tid] - sm.gref[tid], sm.gref[tid] - sm.gend[tid]) > 60.f;
     }
-    __syncthreads();
+    // Strong decay: the split factors e^{+-(g - g_m)} could overflow, so this
+    // chunk forms A and P exactly (every exponent <= 0) from the raw k and q.
+    const bool strong = __syncthreads_or(wide);
 
     // b. decayed operands; Q~ and K^ go straight to the record
     for (int idx = tid; idx < kChunk * DK; idx += 256) {
@@ -166,17 +170,44 @@ intra_chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const 
             qq = to_f32(q[off]);
         }
         const float gg = sm.g[r][ch];
-        const float em = expf(gg - sm.gref[ch]);
-        sm.bufA[r][ch] = kk * em;
-        sm.bufB[r][ch] = kk * expf(sm.gref[ch] - gg);
-        sm.bufC[r][ch] = qq * em;
+        if (!strong) {
+            const float em = expf(gg - sm.gref[ch]);
+            sm.bufA[r][ch] = kk * em;
+            sm.bufB[r][ch] = kk * expf(sm.gref[ch] - gg);
+            sm.bufC[r][ch] = qq * em;
+        } else {
+            sm.bufA[r][ch] = kk;
+            sm.bufC[r][ch] = qq;
+        }
         rec[R::QT + (size_t)r * DK + ch] = qq * expf(gg);
         rec[R::KH + (size_t)r * DK + ch] = kk * expf(sm.gend[ch] - gg);
     }
     __syncthreads();
 
     // c. A (strictly lower, beta-weighted) and P (lower incl. diagonal)
-    {
+    if (strong) {   // exact: one warp per (r, i), lanes over channels
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int pr = warp; pr < kChunk * kChunk; pr += 8) {
+            const int r = pr >> 6, i = pr & 63;
+            float sa = 0.f, sp = 0.f;
+            if (i <= r) {
+                for (int c = lane; c < DK; c += 32) {
+                    const float w = expf(sm.g[r][c] - sm.g[i][c]);
+                    sa += sm.bufA[r][c] * sm.bufA[i][c] * w;
+                    sp += sm.bufC[r][c] * sm.bufA[i][c] * w;
+                }
+#pragma unroll
+                for (int off = 16; off; off >>= 1) {
+                    sa += __shfl_xor_sync(0xffffffffu, sa, off);
+                    sp += __shfl_xor_sync(0xffffffffu, sp, off);
+                }
+            }
+            if (lane == 0) {
+                sm.Am[r][i] = (i < r) ? sm.beta[r] * sa : 0.f;
+                sm.Pm[r][i] = (i <= r) ? sp : 0.f;
+            }
+        }
+    } else {
         const int ty = tid >> 4, tx = tid & 15;
         float acc_a[4][4], acc_p[4][4];
 #pragma unroll
@@ -207,7 +238,7 @@ intra_chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const 
                 sm.Am[r][i] = (i < r) ? sm.beta[r] * acc_a[a][b] : 0.f;
                 sm.Pm[r][i] = (i <= r) ? acc_p[a][b] : 0.f;
             }
-    }
+    }  // !strong
     __syncthreads();
 
     // d. T = (I + A)^{-1} by forward substitution (threads 0..63, one column

@@ -36,6 +36,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "kda_common.cuh"
 #include "kda_launch.h"
@@ -79,6 +80,48 @@ struct TcRec {
     static constexpr uint32_t GC = U0 + U0_BYTES, GC_BYTES = DK * 4;
     static constexpr uint32_t BYTES = (GC + GC_BYTES + 1023) / 1024 * 1024;
 };
+
+
+constexpr float kMaxSplitExponent = 60.f;   // e^60 ~ 1e26: far inside the fp32 range
+
+// Exact A and P of one chunk, used when its decay is too strong for the split
+// factors: A_ri = beta_r sum_c k_rc k_ic e^{g_rc - g_ic} (i < r) into am
+// [64][68] (zero on and above the diagonal) and P_ri = sum_c q_rc k_ic e^{g_rc - g_ic}
+// (i <= r) as fp16 into the record's P tile.  Every exponent is <= 0.  One warp
+// per (r, i) pair, lanes over channels; k and q are the bf16 tiles as loaded.
+template <int DK>
+__device__ __forceinline__ void exact_a_p(const float* g, const unsigned char* ks, const unsigned char* qs,
+                                          const float* s_beta, int L, float* am, unsigned char* prec)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int pr = warp; pr < 64 * 64; pr += 8) {
+        const int r = pr >> 6, i = pr & 63;
+        float sa = 0.f, sp = 0.f;
+        if (i <= r && r < L) {
+#pragma unroll
+            for (int c0 = 0; c0 < DK; c0 += 32) {
+                const int c = c0 + lane;
+                const uint32_t hr = (c >> 6) * 8192u + sw128_offset(r, (c & 63) * 2);
+                const uint32_t hi = (c >> 6) * 8192u + sw128_offset(i, (c & 63) * 2);
+                const float w = __expf(g[r * DK + c] - g[i * DK + c]);
+                const float ki = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ks + hi));
+                const float kr = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ks + hr));
+                const float qr = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qs + hr));
+                sa += kr * ki * w;
+                sp += qr * ki * w;
+            }
+#pragma unroll
+            for (int off = 16; off; off >>= 1) {
+                sa += __shfl_xor_sync(0xffffffffu, sa, off);
+                sp += __shfl_xor_sync(0xffffffffu, sp, off);
+            }
+        }
+        if (lane == 0) {
+            am[r * 68 + i] = (i < r) ? s_beta[r] * sa : 0.f;
+            *reinterpret_cast<__half*>(prec + sw128_offset(r, i * 2)) = __float2half_rn(sp);
+        }
+    }
+}
 
 // ---------------------------------------------------------------- K1 ----
 // Persistent: one CTA per SM walks the (chunk, head) work items.  The k, v, q
@@ -262,19 +305,30 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             }
         }
         __syncthreads();
+        bool wide = false;   // this channel's decay within the chunk too strong for the split factors
         if (tid < DK) {
             const float gm = g[((L - 1) >> 1) * DK + tid], gl = g[(L - 1) * DK + tid];
             s_gm[tid] = gm;
             s_egm[tid] = __expf(gm);
             s_eglm[tid] = __expf(gl - gm);
             reinterpret_cast<float*>(rec + R::GC)[tid] = expf(gl);
+            wide = fmaxf(g[tid] - gm, gm - gl) > kMaxSplitExponent;
         }
-        __syncthreads();
+        // Strong decay: the factors e^{+-(g - g_m)} of A and P could overflow, so
+        // this chunk forms A and P exactly (slow path, no MMA1).
+        const bool strong = __syncthreads_or(wide);
+        if (strong) {
+            float* am = reinterpret_cast<float*>(sm + Sm::AM);
+            exact_a_p<DK>(g, st + Sm::KS, st + Sm::QS, s_beta, L, am, rec + R::P);
+            __syncthreads();   // the k, q tiles are converted in place next
+        }
 
         // ---- decayed operands: thread -> token row r = tid / 4, 8-channel groups
         //      c8 = 8 (tid % 4) + 32 k; two neighbouring rows share an 8-thread
         //      store phase and their swizzles differ, so the fp32 stores are
         //      bank-conflict free
+        auto element_pass = [&](auto strong_tag) {
+            constexpr bool STRONG = decltype(strong_tag)::value;
         {
             const int r = tid >> 2;
             const bool live = r < L;
@@ -308,10 +362,17 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                     for (int h2 = 0; h2 < 2; ++h2) {
                         const int e = 2 * e2 + h2;
                         const float kk = __bfloat162float(kb[e]), qq = __bfloat162float(qb[e]);
-                        const float em = __expf(gv[e] - gmv[e]);   // e^{g_r - g_m}
-                        const float eb = __expf(gmv[e] - gv[e]);   // e^{g_m - g_r}
-                        const float e0 = egmv[e] * em;             // e^{g_r}
-                        const float eh = eglmv[e] * eb;            // e^{g_{L-1} - g_r}
+                        float em, eb, e0, eh;
+                        if constexpr (!STRONG) {
+                            em = __expf(gv[e] - gmv[e]);   // e^{g_r - g_m}
+                            eb = __expf(gmv[e] - gv[e]);   // e^{g_m - g_r}
+                            e0 = egmv[e] * em;             // e^{g_r}
+                            eh = eglmv[e] * eb;            // e^{g_{L-1} - g_r}
+                        } else {                           // unsplit, every exponent <= 0
+                            em = eb = 0.f;
+                            e0 = __expf(gv[e]);
+                            eh = __expf(g[(L - 1) * DK + c8 + e] - gv[e]);
+                        }
                         ka[e] = round_tf32_alu(kk * em);
                         qa[e] = round_tf32_alu(qq * em);
                         kbm[e] = round_tf32_alu(kk * eb);
@@ -326,17 +387,22 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                 // tf32 operands: 8 fp32 = two 16-byte chunks of a 128-byte row
                 const uint32_t fo = (c8 >> 5) * 16384u, fob = (c8 >> 5) * 8192u;
                 const uint32_t fb = (c8 & 31) * 4;
+                if constexpr (!STRONG) {
                 *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(r, fb)) = *reinterpret_cast<const float4*>(ka);
                 *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(r, fb + 16)) = *reinterpret_cast<const float4*>(ka + 4);
                 *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(64 + r, fb)) = *reinterpret_cast<const float4*>(qa);
                 *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(64 + r, fb + 16)) = *reinterpret_cast<const float4*>(qa + 4);
                 *reinterpret_cast<float4*>(sm + Sm::OPB + fob + sw128_offset(r, fb)) = *reinterpret_cast<const float4*>(kbm);
                 *reinterpret_cast<float4*>(sm + Sm::OPB + fob + sw128_offset(r, fb + 16)) = *reinterpret_cast<const float4*>(kbm + 4);
+                }
                 *reinterpret_cast<uint4*>(st + Sm::KS + ho) = *reinterpret_cast<const uint4*>(k0);   // K~ (MMA2 operand)
                 *reinterpret_cast<uint4*>(st + Sm::QS + ho) = *reinterpret_cast<const uint4*>(q0);   // Q~ (record)
                 *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(kh);  // K^ (record)
             }
         }
+        };
+        if (strong) element_pass(std::true_type{});
+        else element_pass(std::false_type{});
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -355,6 +421,8 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                 bulk_store(rec + R::WQ + b * 16384 + 8192, st + Sm::QS + b * Sm::TILE, 8192);
             bulk_store_commit();
             stored = true;
+        }
+        if (tid == 0 && !strong) {
             // ---- MMA1 (tf32): [K~m; Q~m] K-m^T -> R1 (overlaps the v conversion)
             tc_fence_after();
             constexpr uint32_t idesc = instr_desc(kFmtTF32, 128, 64);
@@ -368,7 +436,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                              (kb | ks) != 0);
             mma_commit(&bar_mma);
         }
-        mma_pending = 1;
+        mma_pending = strong ? 0 : 1;
         // v: bf16 -> fp16 in place, 8 values per thread and step
         for (int item = tid; item < kChunk * (DV / 8); item += 256) {
             const int r = item / (DV / 8), j8 = (item - r * (DV / 8)) * 8;
@@ -386,7 +454,12 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             *reinterpret_cast<uint4*>(st + o) = *reinterpret_cast<const uint4*>(vh);
         }
         fence_proxy_async_smem();   // fp16 v (MMA2 operand)
-        bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        float* am = reinterpret_cast<float*>(sm + Sm::AM);   // [64][68]
+        float* tmx = reinterpret_cast<float*>(sm + Sm::TM);  // [64][68]
+        float* ym = reinterpret_cast<float*>(sm + Sm::YM);   // [6][16][17]
+        bool ok = true;
+        if (!strong) {
+        ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         mma_phase ^= 1;
         mma_pending = 0;
@@ -394,9 +467,6 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
 
         // ---- A (rows 0..63, beta-scaled, strictly lower) to smem; P (rows
         //      64..127, lower incl. diagonal) to the record
-        float* am = reinterpret_cast<float*>(sm + Sm::AM);   // [64][68]
-        float* tmx = reinterpret_cast<float*>(sm + Sm::TM);  // [64][68]
-        float* ym = reinterpret_cast<float*>(sm + Sm::YM);   // [6][16][17]
         {
             float v[32];
             const int row = (warp & 3) * 32 + (tid & 31);
@@ -428,6 +498,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                 }
             }
         }
+        }   // !strong
         __syncthreads();
 
         // ---- T = (I + A)^{-1} in 16 x 16 blocks, written as fp16 T diag(beta)

@@ -285,3 +285,34 @@ def test_bad_cu_seqlens_reported(cuda_device):
     cu_ok = torch.tensor([0, 40, 60, 100], dtype=torch.int32, device="cuda")
     kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], None, cu_ok, workspace=ws)
     assert kda.workspace_status(ws) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("where", ["all_channels", "few_channels"])
+def test_strong_decay(cuda_device, dtype, where):
+    """Chunks whose log-decay over half a chunk exceeds the split-factor range
+    take the exact slow path for A and P; results still match the oracle."""
+    w = I.ChunkWorkload("strong", B=2, T=200, H=2, dk=128, dv=64, dtype=dtype, s0_std=0.05, seed=28)
+    x = I.chunk_inputs(w)
+    g = torch.Generator().manual_seed(281)
+    strong = -4.0 * torch.exp(0.2 * torch.randn(x["log_alpha"].shape, generator=g))
+    if where == "all_channels":
+        x["log_alpha"] = strong
+    else:   # channels 5 and 77 of head 1 only
+        x["log_alpha"][:, :, 1, [5, 77]] = strong[:, :, 1, [5, 77]]
+    o, S = run_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check(o, o_ref, dtype, f"{where} o")
+    check(S, S_ref, dtype, f"{where} final_state")
+
+
+def test_value_range_reported(cuda_device):
+    """bf16 path: a value beyond the fp16 range of the intermediates is reported."""
+    w = I.ChunkWorkload("range", B=1, T=70, H=1, dk=64, dv=64, dtype=torch.bfloat16, seed=29)
+    x = I.chunk_inputs(w)
+    x["v"] = (x["v"].float() * 1e5).to(torch.bfloat16)
+    g = to_dev(x)
+    ws = torch.empty(kda.chunk_fwd_workspace_size(1, 70, 1, 64, 64, 1, False, torch.bfloat16),
+                     dtype=torch.uint8, device="cuda")
+    kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], None, None, workspace=ws)
+    assert kda.workspace_status(ws) == 7
