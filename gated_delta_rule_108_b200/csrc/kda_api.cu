@@ -92,12 +92,14 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
     return L.total;
 }
 
-kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
-                         const float* beta, const float* initial_state, const int32_t* cu_seqlens,
-                         int B, int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype,
-                         void* o, float* final_state, void* workspace, size_t workspace_bytes,
-                         void* stream) {
+static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const float* log_alpha,
+                                 const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                                 int B, int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype,
+                                 kda_gate gate, void* o, float* final_state, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE)
+        return fail(KDA_ERR_INVALID_ARG, "unknown gate kind %d", (int)gate);
     if (B < 0 || T < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d", B, T, H);
     if (dk <= 0 || dv <= 0) return fail(KDA_ERR_INVALID_ARG, "bad head sizes dk=%d dv=%d", dk, dv);
     if (!supported_dim(dk) || !supported_dim(dv))
@@ -110,9 +112,10 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
     if (tokens * (size_t)H * (size_t)(dk > dv ? dk : dv) >= (size_t)1 << 31)
         return fail(KDA_ERR_UNSUPPORTED, "B*T*H*d = %zu elements exceeds 2^31", tokens * H * (dk > dv ? dk : dv));
     if (tokens > 0) {
-        if (!q || !k || !v || !log_alpha || !beta || !o)
+        if (!q || !k || !v || !beta || !o || (gate != KDA_GATE_NONE && !log_alpha))
             return fail(KDA_ERR_INVALID_ARG, "null input/output pointer");
-        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o))
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+            (gate == KDA_GATE_CHANNEL && !aligned16(log_alpha)))
             return fail(KDA_ERR_INVALID_ARG, "q/k/v/log_alpha/o must be 16-byte aligned");
     }
     if (initial_state && !aligned16(initial_state)) return fail(KDA_ERR_INVALID_ARG, "initial_state misaligned");
@@ -138,6 +141,7 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
     a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
     a.o = o; a.final_state = final_state;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.num_seqs = N;
+    a.gate = (int)gate;
     a.bf16 = dtype == KDA_BF16;
     a.scale = 1.0f / sqrtf((float)dk);
     a.ws_header = workspace;
@@ -158,10 +162,12 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const floa
     return ok();
 }
 
-kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* log_alpha,
-                              const float* beta, float* state_inout, int B, int H, int dk, int dv,
-                              kda_dtype dtype, void* o, void* stream) {
+static kda_status recurrent_step_impl(const void* q, const void* k, const void* v, const float* log_alpha,
+                                      const float* beta, float* state_inout, int B, int H, int dk, int dv,
+                                      kda_dtype dtype, kda_gate gate, void* o, void* stream) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE)
+        return fail(KDA_ERR_INVALID_ARG, "unknown gate kind %d", (int)gate);
     if (B < 0 || H <= 0 || dk <= 0 || dv <= 0)
         return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d H=%d dk=%d dv=%d", B, H, dk, dv);
     if (!supported_dim(dk) || !supported_dim(dv))
@@ -169,10 +175,10 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
     if ((size_t)B * H * dk * dv >= (size_t)1 << 40)
         return fail(KDA_ERR_UNSUPPORTED, "state too large");
     if (B > 0) {
-        if (!q || !k || !v || !log_alpha || !beta || !state_inout || !o)
+        if (!q || !k || !v || !beta || !state_inout || !o || (gate != KDA_GATE_NONE && !log_alpha))
             return fail(KDA_ERR_INVALID_ARG, "null pointer");
-        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) ||
-            !aligned16(state_inout) || !aligned16(o))
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state_inout) || !aligned16(o) ||
+            (gate == KDA_GATE_CHANNEL && !aligned16(log_alpha)))
             return fail(KDA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
         const char* s0 = (const char*)state_inout;
         const char* o0 = (const char*)o;
@@ -184,12 +190,44 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
     a.state = state_inout; a.o = o;
     a.B = B; a.H = H; a.dk = dk; a.dv = dv;
+    a.gate = (int)gate;
     a.bf16 = dtype == KDA_BF16;
     a.scale = 1.0f / sqrtf((float)dk);
     a.stream = static_cast<cudaStream_t>(stream);
     const cudaError_t e = kda::launch_decode(a);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_recurrent_step launch failed: %s", cudaGetErrorString(e));
     return ok();
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                         const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                         int B, int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype,
+                         void* o, float* final_state, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, initial_state, cu_seqlens, B, T, H, dk, dv, num_seqs,
+                          dtype, KDA_GATE_CHANNEL, o, final_state, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* log_alpha,
+                               const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                               int B, int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype,
+                               kda_gate gate, void* o, float* final_state, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, initial_state, cu_seqlens, B, T, H, dk, dv, num_seqs,
+                          dtype, gate, o, final_state, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_recurrent_step(const void* q, const void* k, const void* v, const float* log_alpha,
+                              const float* beta, float* state_inout, int B, int H, int dk, int dv,
+                              kda_dtype dtype, void* o, void* stream) {
+    return recurrent_step_impl(q, k, v, log_alpha, beta, state_inout, B, H, dk, dv, dtype, KDA_GATE_CHANNEL,
+                               o, stream);
+}
+
+kda_status kda_recurrent_step_gated(const void* q, const void* k, const void* v, const float* log_alpha,
+                                    const float* beta, float* state_inout, int B, int H, int dk, int dv,
+                                    kda_dtype dtype, kda_gate gate, void* o, void* stream) {
+    return recurrent_step_impl(q, k, v, log_alpha, beta, state_inout, B, H, dk, dv, dtype, gate, o, stream);
 }
 
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256)
 intra_chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                         const float* __restrict__ log_alpha, const float* __restrict__ beta,
                         ChunkMap map, const WsHeader* __restrict__ hdr, float* __restrict__ records,
-                        int H, size_t max_chunks)
+                        int H, size_t max_chunks, int gate)
 {
     using R = SimtRec<DK, DV>;
     using Sm = IntraSmem<T, DK, DV>;
@@ -138,11 +138,15 @@ intra_chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const 
 
     // a. in-chunk cumulative log-decay per key channel; padded rows add 0
     if (tid < DK) {
+        // per-channel gate: [.., H, DK]; per-head gate: [.., H] (the same value
+        // for every channel); no gate: log-decay 0
+        const size_t rstride = gate == kGateChannel ? rowk : (size_t)H;
+        const float* la = gate == kGateChannel ? log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid
+                                               : log_alpha + (size_t)tok0 * H + h;
         float acc = 0.f;
-        const float* la = log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid;
 #pragma unroll 8
         for (int r = 0; r < kChunk; ++r) {
-            acc += (r < L) ? la[(size_t)r * rowk] : 0.f;
+            acc += (r < L && gate != kGateNone) ? la[(size_t)r * rstride] : 0.f;
             sm.g[r][tid] = acc;
         }
     } else if (tid >= 128 && tid < 128 + kChunk) {
@@ -456,7 +460,7 @@ cudaError_t launch_intra_t(const ChunkArgs& a) {
     k1<<<grid, 256, smem, a.stream>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
         a.log_alpha, a.beta, map, static_cast<const WsHeader*>(a.ws_header),
-        static_cast<float*>(a.records), a.H, a.max_chunks);
+        static_cast<float*>(a.records), a.H, a.max_chunks, a.gate);
     return cudaGetLastError();
 }
 

@@ -35,6 +35,7 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 #include <type_traits>
 
@@ -159,7 +160,8 @@ struct K1Smem {
     static constexpr uint32_t GM = BETA + 256;                      // [DK] g_m, e^{g_m}, e^{g_{L-1}-g_m}
     static constexpr uint32_t EGM = GM + DK * 4;
     static constexpr uint32_t EGLM = EGM + DK * 4;
-    static constexpr uint32_t TOTAL = EGLM + DK * 4;
+    static constexpr uint32_t LAH = EGLM + DK * 4;                  // [64] per-head log-decay
+    static constexpr uint32_t TOTAL = LAH + 256;
     // cumulative-sum partials live in the (then unused) T-solve scratch
     static constexpr uint32_t PART = YM;
     static_assert(YM + 6 * 16 * 17 * 4 <= END, "T-solve scratch");
@@ -168,12 +170,13 @@ struct K1Smem {
     static_assert(TOTAL <= 232448, "shared memory");
 };
 
-template <int DK, int DV>
+template <int DK, int DV, int GATE>
 __global__ void __launch_bounds__(256, 1)
 intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_la,
-                      const float* __restrict__ beta, ChunkMap map, WsHeader* hdr,
-                      unsigned char* __restrict__ records, int H, size_t max_chunks)
+                      const float* __restrict__ log_alpha_head, const float* __restrict__ beta,
+                      ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
+                      size_t max_chunks)
 {
     using Sm = K1Smem<DK, DV>;
     using R = TcRec<DK, DV>;
@@ -189,6 +192,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
     float* s_gm = reinterpret_cast<float*>(sm + Sm::GM);
     float* s_egm = reinterpret_cast<float*>(sm + Sm::EGM);
     float* s_eglm = reinterpret_cast<float*>(sm + Sm::EGLM);
+    float* s_lah = reinterpret_cast<float*>(sm + Sm::LAH);
     float* s_part = reinterpret_cast<float*>(sm + Sm::PART);        // [NPART][DK]
 
     if (hdr->status != kStatusOk) return;
@@ -240,21 +244,25 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
 #pragma unroll
         for (int b = 0; b < DK / 64; ++b) tma_load_3d(st + Sm::QS + b * Sm::TILE, &tm_q, &bar_load[stage], b * 64, h, tok0);
     };
-    // log_alpha tile of item w into G (when G is free), by TMA
+    // per-channel gate: log_alpha tile of item w into G (when G is free), by TMA
+    constexpr bool channel_gate = GATE == kGateChannel;
     auto issue_la = [&](int w) {
+        if constexpr (!channel_gate) return;
         int c, h, tok0, L;
         locate(w, c, h, tok0, L);
         mbar_arrive_expect_tx(&bar_la, Sm::LA_BYTES);
         tma_load_3d(sm + Sm::G, &tm_la, &bar_la, 0, h, tok0);
     };
-    // beta of item w into a register (threads 192..255, one token each)
-    float beta_next = 0.f;
+    // beta (and a per-head log-decay) of item w into registers, threads
+    // 192..255, one token each
+    float beta_next = 0.f, lah_next = 0.f;
     auto load_beta = [&](int w) {
         if (tid >= 192) {
             int c, h, tok0, L;
             locate(w, c, h, tok0, L);
             const int r = tid - 192;
             beta_next = (r < L) ? ld_prefetch_f32(beta + (size_t)(tok0 + r) * H + h) : 0.f;
+            lah_next = (GATE == kGateHead && r < L) ? ld_prefetch_f32(log_alpha_head + (size_t)(tok0 + r) * H + h) : 0.f;
         }
     };
 
@@ -276,14 +284,17 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         int c, h, tok0, L;
         locate(w, c, h, tok0, L);
         unsigned char* rec = records + ((size_t)h * max_chunks + c) * R::BYTES;
-        if (tid >= 192) s_beta[tid - 192] = beta_next;
+        if (tid >= 192) {
+            s_beta[tid - 192] = beta_next;
+            if constexpr (GATE == kGateHead) s_lah[tid - 192] = lah_next;
+        }
 
         const int wn = w + gridDim.x;   // this CTA's next item
         if (wn < total) load_beta(wn);
 
         // ---- cumulative log-decay, in place over the log_alpha tile in G -------
         float* g = reinterpret_cast<float*>(sm + Sm::G);   // [64][DK]
-        const bool ok_la = mbar_wait_cycles(&bar_la, it & 1, kWaitCycles);
+        const bool ok_la = !channel_gate || mbar_wait_cycles(&bar_la, it & 1, kWaitCycles);
         const bool ok_load = mbar_wait_cycles(&bar_load[stage], (it >> 1) & 1, kWaitCycles);
         if (__syncthreads_or(!(ok_la && ok_load))) { aborted = true; break; }
         {
@@ -291,7 +302,9 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             float acc = 0.f;
 #pragma unroll
             for (int i = 0; i < TPP; ++i) {
-                la_cur[i] = (r0 + i < L) ? g[(r0 + i) * DK + ch] : 0.f;
+                if constexpr (channel_gate) la_cur[i] = (r0 + i < L) ? g[(r0 + i) * DK + ch] : 0.f;
+                else if constexpr (GATE == kGateHead) la_cur[i] = (r0 + i < L) ? s_lah[r0 + i] : 0.f;
+                else la_cur[i] = 0.f;   // no gate: alpha = 1
                 acc += la_cur[i];
             }
             s_part[part * DK + ch] = acc;
@@ -332,7 +345,8 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         {
             const int r = tid >> 2;
             const bool live = r < L;
-#pragma unroll
+            constexpr int KUNROLL = STRONG ? 1 : DK / 32;   // keep the rare path small
+#pragma unroll KUNROLL
             for (int k = 0; k < DK / 32; ++k) {
                 const int c8 = 8 * (tid & 3) + 32 * k;
                 const uint32_t ho = (c8 >> 6) * Sm::TILE + sw128_offset(r, (c8 & 63) * 2);   // 16-byte chunk
@@ -647,7 +661,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         // let this CTA's own copies and MMAs finish (bounded) before freeing
         for (int s2 = 0; s2 < 2; ++s2) (void)mbar_wait_cycles(&bar_load[s2], 0, kWaitCycles / 4);
-        (void)mbar_wait_cycles(&bar_la, 0, kWaitCycles / 4);
+        if constexpr (channel_gate) (void)mbar_wait_cycles(&bar_la, 0, kWaitCycles / 4);
         if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
     }
     if (stored) bulk_store_wait_all();
@@ -946,10 +960,14 @@ cudaError_t launch_intra_tc_t(const ChunkArgs& a) {
     if (!make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, ntok, DK, CU_TENSOR_MAP_SWIZZLE_NONE))
+        (a.gate == kGateChannel &&
+         !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, ntok, DK, CU_TENSOR_MAP_SWIZZLE_NONE)))
         return cudaErrorInvalidValue;
+    if (a.gate != kGateChannel) memset(&mla, 0, sizeof(mla));   // unused
     ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
-    auto kern = intra_chunk_tc_kernel<DK, DV>;
+    auto kern = a.gate == kGateChannel ? intra_chunk_tc_kernel<DK, DV, kGateChannel>
+              : a.gate == kGateHead    ? intra_chunk_tc_kernel<DK, DV, kGateHead>
+                                       : intra_chunk_tc_kernel<DK, DV, kGateNone>;
     const int smem = (int)K1Smem<DK, DV>::TOTAL;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -958,7 +976,8 @@ cudaError_t launch_intra_tc_t(const ChunkArgs& a) {
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const size_t items = a.max_chunks * (size_t)a.H;   // upper bound; the kernel reads the exact count
     const unsigned grid = (unsigned)(items < (size_t)sms ? items : (size_t)sms);
-    kern<<<grid, 256, smem, a.stream>>>(mk, mv, mq, mla, a.beta, map, static_cast<WsHeader*>(a.ws_header),
+    kern<<<grid, 256, smem, a.stream>>>(mk, mv, mq, mla, a.log_alpha, a.beta, map,
+                                        static_cast<WsHeader*>(a.ws_header),
                                         static_cast<unsigned char*>(a.records), a.H, a.max_chunks);
     return cudaGetLastError();
 }

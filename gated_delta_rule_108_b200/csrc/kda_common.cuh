@@ -18,6 +18,12 @@ constexpr int kStatusTimeout = 4;
 constexpr int kStatusBadSeqlens = 6;
 constexpr int kStatusRange = 7;
 
+// Decay gate kinds (same values as kda_gate in include/kda.h): one log-decay
+// per key channel (KDA), one per head (Gated DeltaNet), or none (DeltaNet).
+constexpr int kGateChannel = 0;
+constexpr int kGateHead = 1;
+constexpr int kGateNone = 2;
+
 // Workspace header, at offset 0 of the caller's workspace.
 struct WsHeader {
     int status;       // argument check of the last call (0 = ok): kernels skip work if set

@@ -10,7 +10,9 @@
 //   S' = S~ + k u^T             o = dk^{-1/2} S'^T q = dk^{-1/2} (S~^T q + u <k, q>)
 //
 // The last identity lets the read share the pass over S~ with the predict, so
-// S is touched by exactly one load and one store per element.
+// S is touched by exactly one load and one store per element.  With a per-head
+// gate (Gated DeltaNet) every channel decays by the same alpha; without a gate
+// (DeltaNet) alpha = 1.
 //
 // Layout: one CTA per (b, h); warp w owns key rows [w*DK/NW, (w+1)*DK/NW), lane
 // l owns value columns [l*DV/32, (l+1)*DV/32) -- a warp reads one 512-byte row
@@ -51,7 +53,7 @@ template <typename T, int DK, int DV, int NW>
 __global__ void __launch_bounds__(NW * 32)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                   float* __restrict__ state, T* __restrict__ o, float scale)
+                   float* __restrict__ state, T* __restrict__ o, float scale, int gate)
 {
     constexpr int NT = NW * 32;
     constexpr int ROWS = DK / NW;   // key rows per warp
@@ -72,10 +74,11 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     for (int r = 0; r < ROWS; ++r)
         load_vec<VEC>(S + (size_t)(warp * ROWS + r) * DV + lane * VEC, s[r]);
 
+    const float a_head = (gate == kGateHead) ? expf(log_alpha[bh]) : 1.f;
     for (int i = tid; i < DK; i += NT) {
         sk[i] = to_f32(k[(size_t)bh * DK + i]);
         sq[i] = to_f32(q[(size_t)bh * DK + i]);
-        sa[i] = expf(log_alpha[(size_t)bh * DK + i]);
+        sa[i] = (gate == kGateChannel) ? expf(log_alpha[(size_t)bh * DK + i]) : a_head;
     }
     for (int j = tid; j < DV; j += NT) sv[j] = to_f32(v[(size_t)bh * DV + j]);
     __syncthreads();
@@ -141,7 +144,7 @@ cudaError_t launch_decode_t(const DecodeArgs& a) {
     const int grid = a.B * a.H;
     decode_step_kernel<T, DK, DV, NW><<<grid, NW * 32, 0, a.stream>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
-        a.log_alpha, a.beta, a.state, static_cast<T*>(a.o), a.scale);
+        a.log_alpha, a.beta, a.state, static_cast<T*>(a.o), a.scale, a.gate);
     return cudaGetLastError();
 }
 

@@ -13,6 +13,7 @@ struct DecodeArgs {
     const float* log_alpha; const float* beta;
     float* state; void* o;
     int B, H, dk, dv;
+    int gate;                     // kGateChannel: log_alpha [B,H,dk]; kGateHead: [B,H]; kGateNone: unused
     bool bf16;
     float scale;
     cudaStream_t stream;
@@ -26,6 +27,7 @@ struct ChunkArgs {
     const int32_t* cu_seqlens;    // nullable
     void* o; float* final_state;  // final_state nullable
     int B, T, H, dk, dv, num_seqs;
+    int gate;                     // kGateChannel: log_alpha [.., H, dk]; kGateHead: [.., H]; kGateNone: unused
     bool bf16;
     float scale;
     // workspace carve-up (computed by the ABI layer)

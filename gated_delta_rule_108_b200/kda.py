@@ -23,6 +23,7 @@ _STATUS = {
     4: "KDA_ERR_TIMEOUT", 5: "KDA_ERR_WORKSPACE", 6: "KDA_ERR_BAD_SEQLENS", 7: "KDA_ERR_RANGE",
 }
 KDA_F32, KDA_BF16 = 0, 1
+KDA_GATE_CHANNEL, KDA_GATE_HEAD, KDA_GATE_NONE = 0, 1, 2
 
 _lock = threading.Lock()
 _lib = None
@@ -51,6 +52,11 @@ def _declare(lib):
                                   vp, vp, vp, sz, vp]
     lib.kda_recurrent_step.restype = i
     lib.kda_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp]
+    lib.kda_chunk_fwd_gated.restype = i
+    lib.kda_chunk_fwd_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
+                                        vp, vp, vp, sz, vp]
+    lib.kda_recurrent_step_gated.restype = i
+    lib.kda_recurrent_step_gated.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp]
     lib.kda_workspace_status.restype = i
     lib.kda_workspace_status.argtypes = [vp, sz, vp]
     lib.kda_set_stage_events.restype = i
@@ -115,20 +121,35 @@ def chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
                                                   int(bool(varlen)), code))
 
 
+def _gate_of(log_alpha, channel_ndim: int, shape_channel, shape_head) -> int:
+    """Gate kind from log_alpha's shape: None -> no gate (DeltaNet), one value
+    per head -> Gated DeltaNet, one value per key channel -> KDA."""
+    if log_alpha is None:
+        return KDA_GATE_NONE
+    _need(log_alpha, "log_alpha", torch.float32)
+    if tuple(log_alpha.shape) == tuple(shape_channel):
+        return KDA_GATE_CHANNEL
+    if tuple(log_alpha.shape) == tuple(shape_head):
+        return KDA_GATE_HEAD
+    raise ValueError(f"log_alpha must be {tuple(shape_channel)} (per channel), {tuple(shape_head)} "
+                     f"(per head) or None, got {tuple(log_alpha.shape)}")
+
+
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
               output_final_state: bool = True, o=None, final_state=None,
               workspace=None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Chunkwise KDA forward (``kda_chunk_fwd``).
+    """Chunkwise forward (``kda_chunk_fwd_gated``).
 
-    q, k, log_alpha [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H];
+    q, k [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H];
+    log_alpha [B, T, H, dk] (KDA), [B, T, H] (Gated DeltaNet) or None (DeltaNet);
     initial_state [N, H, dk, dv] fp32 or None; cu_seqlens int32 [N+1] or None.
     Returns (o [B, T, H, dv], final_state [N, H, dk, dv] or None).
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype)
-    _need(log_alpha, "log_alpha", torch.float32)
     _need(beta, "beta", torch.float32)
     B, T, H, dk = q.shape
+    gate = _gate_of(log_alpha, 4, (B, T, H, dk), (B, T, H))
     dv = v.shape[-1]
     if cu_seqlens is not None:
         _need(cu_seqlens, "cu_seqlens", torch.int32)
@@ -144,9 +165,9 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     ws_bytes = chunk_fwd_workspace_size(B, T, H, dk, dv, N, cu_seqlens is not None, q.dtype)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
-    _check(lib().kda_chunk_fwd(
+    _check(lib().kda_chunk_fwd_gated(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
-        _ptr(cu_seqlens), B, T, H, dk, dv, N, _dtype_code(q), _ptr(o), _ptr(final_state),
+        _ptr(cu_seqlens), B, T, H, dk, dv, N, _dtype_code(q), gate, _ptr(o), _ptr(final_state),
         _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream_ptr(stream, q.device)))
     return o, final_state
@@ -169,21 +190,22 @@ def set_stage_events(events) -> None:
 
 
 def recurrent_step(q, k, v, log_alpha, beta, state, o=None, stream=None) -> torch.Tensor:
-    """One decoding step (``kda_recurrent_step``); ``state`` is updated in place.
+    """One decoding step (``kda_recurrent_step_gated``); ``state`` is updated in place.
 
-    q, k, log_alpha [B, H, dk]; v [B, H, dv]; beta [B, H]; state [B, H, dk, dv] fp32.
+    q, k [B, H, dk]; v [B, H, dv]; beta [B, H]; state [B, H, dk, dv] fp32;
+    log_alpha [B, H, dk] (KDA), [B, H] (Gated DeltaNet) or None (DeltaNet).
     Returns o [B, H, dv] in q's dtype.
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, q.dtype)
-    _need(log_alpha, "log_alpha", torch.float32)
     _need(beta, "beta", torch.float32)
     _need(state, "state", torch.float32)
     B, H, dk = q.shape
     dv = v.shape[-1]
+    gate = _gate_of(log_alpha, 3, (B, H, dk), (B, H))
     if o is None:
         o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
-    _check(lib().kda_recurrent_step(
+    _check(lib().kda_recurrent_step_gated(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state),
-        B, H, dk, dv, _dtype_code(q), _ptr(o), _stream_ptr(stream, q.device)))
+        B, H, dk, dv, _dtype_code(q), gate, _ptr(o), _stream_ptr(stream, q.device)))
     return o

@@ -55,6 +55,18 @@ typedef enum {
 typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
 
 /*
+ * Shape of the decay gate.  KDA_GATE_CHANNEL is Kimi Delta Attention: one
+ * log-decay per key channel, log_alpha [.., H, dk] (daiw.net "Kimi Delta
+ * Attention", section "一、Diag(alpha_t)：通道级遗忘").  KDA_GATE_HEAD is Gated
+ * DeltaNet: one scalar log-decay per token and head, log_alpha [.., H], applied
+ * to the whole state before the prediction (news.bugfactory.tech/news/3610,
+ * Gated DeltaNet paragraph).  KDA_GATE_NONE is DeltaNet: no decay (alpha = 1,
+ * log_alpha unused, may be NULL) (same page, DeltaNet paragraph).  The three
+ * are the same recurrence with log_alpha broadcast to [.., H, dk].
+ */
+typedef enum { KDA_GATE_CHANNEL = 0, KDA_GATE_HEAD = 1, KDA_GATE_NONE = 2 } kda_gate;
+
+/*
  * Bytes of device workspace kda_chunk_fwd needs for these sizes.  `varlen` is
  * non-zero when cu_seqlens will be passed (then B must be 1 and num_seqs is
  * the number of packed sequences); otherwise num_seqs is ignored (= B).
@@ -123,6 +135,29 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
  */
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes,
                                 void* stream);
+
+/*
+ * kda_chunk_fwd with the gate shape chosen by `gate` (see kda_gate): log_alpha
+ * is [B, T, H, dk] for KDA_GATE_CHANNEL (16-byte aligned), [B, T, H] for
+ * KDA_GATE_HEAD, and unused for KDA_GATE_NONE.  Everything else as kda_chunk_fwd;
+ * the workspace size does not depend on the gate.
+ */
+kda_status kda_chunk_fwd_gated(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta,
+                               const float* initial_state, const int32_t* cu_seqlens,
+                               int B, int T, int H, int dk, int dv, int num_seqs,
+                               kda_dtype dtype, kda_gate gate, void* o, float* final_state,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * kda_recurrent_step with the gate shape chosen by `gate`: log_alpha is
+ * [B, H, dk] for KDA_GATE_CHANNEL, [B, H] for KDA_GATE_HEAD, unused for
+ * KDA_GATE_NONE.
+ */
+kda_status kda_recurrent_step_gated(const void* q, const void* k, const void* v,
+                                    const float* log_alpha, const float* beta,
+                                    float* state_inout, int B, int H, int dk, int dv,
+                                    kda_dtype dtype, kda_gate gate, void* o, void* stream);
 
 /*
  * kda_chunk_fwd without a caller-provided workspace.  The paper has no

@@ -95,3 +95,20 @@ def test_python_binding_has_no_cpu_path(monkeypatch, tmp_path):
     monkeypatch.setattr(kda, "_lib", None)
     with pytest.raises(kda.KDAError):
         kda.lib()
+
+
+def test_gated_entry_points_validate(lib):
+    p = 1 << 20
+    f = lib.kda_chunk_fwd_gated
+    # unknown gate kind
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 64, 64, 1, 0, 9, p, None, p, 1 << 30, None) == 1
+    # a gate that needs log_alpha, given none
+    assert f(p, p, p, None, p, None, None, 1, 64, 1, 64, 64, 1, 0, 0, p, None, p, 1 << 30, None) == 1
+    assert f(p, p, p, None, p, None, None, 1, 64, 1, 64, 64, 1, 0, 1, p, None, p, 1 << 30, None) == 1
+    # no gate: log_alpha may be NULL (fails later, on the missing workspace)
+    assert f(p, p, p, None, p, None, None, 1, 64, 1, 64, 64, 1, 0, 2, p, None, None, 0, None) == 5
+    # per-head gate: log_alpha only needs 4-byte alignment (fails on the workspace)
+    assert f(p, p, p, p + 4, p, None, None, 1, 64, 1, 64, 64, 1, 0, 1, p, None, None, 0, None) == 5
+    d = lib.kda_recurrent_step_gated
+    assert d(p, p, p, None, p, p, 2, 2, 64, 64, 1, 0, p + (1 << 24), None) == 1
+    assert d(p, p, p, p, p, p, 2, 2, 64, 64, 1, 7, p + (1 << 24), None) == 1
