@@ -53,6 +53,12 @@ def load_library(path: str):
         dp, dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, dp, dp,
     ]
+    lib.oracle_kda_backward.restype = ctypes.c_int
+    lib.oracle_kda_backward.argtypes = [
+        dp, dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, dp, dp,
+        dp, dp, dp, dp, dp, dp,
+    ]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     return lib
@@ -86,6 +92,19 @@ def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
 
+def _seqlens(cu_seqlens, B, T):
+    if cu_seqlens is None:
+        return np.arange(B + 1, dtype=np.int64) * T
+    if B != 1:
+        raise ValueError("cu_seqlens requires B == 1")
+    if hasattr(cu_seqlens, "detach"):
+        cu_seqlens = cu_seqlens.detach().cpu().numpy()
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    if cu[0] != 0 or cu[-1] != T or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must start at 0, be non-decreasing, end at T")
+    return cu
+
+
 def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, lib=None):
     """Token-by-token fp64 KDA forward.
 
@@ -104,16 +123,7 @@ def kda_forward(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, l
         raise ValueError("q, k and log_alpha must share one shape")
     if v.shape[:3] != (B, T, H) or b.shape != (B, T, H):
         raise ValueError("v / beta shapes do not match q")
-    if cu_seqlens is None:
-        cu = np.arange(B + 1, dtype=np.int64) * T
-    else:
-        if B != 1:
-            raise ValueError("cu_seqlens requires B == 1")
-        if hasattr(cu_seqlens, "detach"):
-            cu_seqlens = cu_seqlens.detach().cpu().numpy()
-        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
-        if cu[0] != 0 or cu[-1] != T or np.any(np.diff(cu) < 0):
-            raise ValueError("cu_seqlens must start at 0, be non-decreasing, end at T")
+    cu = _seqlens(cu_seqlens, B, T)
     N = cu.shape[0] - 1
     S0 = _f64(initial_state)
     if S0 is not None and S0.shape != (N, H, dk, dv):
@@ -143,3 +153,39 @@ def kda_decode_step(q, k, v, log_alpha, beta, state):
     o, S = kda_forward(q[None], k[None], v[None], la[None], b[None],
                        initial_state=state, cu_seqlens=cu)
     return o[0], S
+
+
+def kda_backward(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=None,
+                 cu_seqlens=None, lib=None):
+    """Gradients of L = <d_o, o> + <d_final_state, final_state> in fp64.
+
+    Reverse-mode derivative of the token loop of ``kda_forward`` (same shapes and
+    sequence rules; ``d_o`` like o, ``d_final_state`` like the final state, None
+    for zeros).  Returns a dict with ``dq, dk, dv, dlog_alpha, dbeta`` (shaped like
+    their inputs) and ``dS0`` [N, H, dk, dv], as fp64 numpy arrays.
+    """
+    q, k, v, la, b, do = (_f64(x) for x in (q, k, v, log_alpha, beta, d_o))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or la.shape != q.shape:
+        raise ValueError("q, k and log_alpha must share one shape")
+    if v.shape[:3] != (B, T, H) or b.shape != (B, T, H) or do.shape != v.shape:
+        raise ValueError("v / beta / d_o shapes do not match q")
+    cu = _seqlens(cu_seqlens, B, T)
+    N = cu.shape[0] - 1
+    S0, dSf = _f64(initial_state), _f64(d_final_state)
+    for name, x in (("initial_state", S0), ("d_final_state", dSf)):
+        if x is not None and x.shape != (N, H, dk, dv):
+            raise ValueError(f"{name} must be {(N, H, dk, dv)}, got {x.shape}")
+    g = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v),
+         "dlog_alpha": np.zeros_like(la), "dbeta": np.zeros_like(b),
+         "dS0": np.zeros((N, H, dk, dv), dtype=np.float64)}
+    rc = (lib or _load()).oracle_kda_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(S0),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), N, H, dk, dv,
+        _ptr(do), _ptr(dSf), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+        _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dS0"]),
+    )
+    if rc != 0:
+        raise RuntimeError(f"oracle_kda_backward failed with code {rc}")
+    return g
