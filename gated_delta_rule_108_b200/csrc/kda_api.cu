@@ -69,6 +69,29 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
     return true;
 }
 
+// Backward workspace: [header][chunk_offsets][fp32 records][T][chunk-start
+// states][dS at chunk ends][dU][per-CTA scratch], each 256-byte aligned.
+struct BwdLayout {
+    WsLayout base;   // header, offsets (records re-sized below)
+    size_t tmat_off, states_off, dS_off, dU_off, scratch_off, total;
+    int ctas;        // CTAs the scratch holds
+};
+
+bool bwd_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, kda_dtype dtype,
+                BwdLayout& L) {
+    if (!ws_layout(B, T, H, dk, dv, num_seqs, varlen, dtype, L.base)) return false;
+    const size_t units = (size_t)H * L.base.max_chunks;   // (head, chunk) pairs
+    const size_t rec = kda::simt_record_bytes(dk, dv);
+    L.tmat_off = round_up(L.base.records_off + rec * units, 256);
+    L.states_off = round_up(L.tmat_off + sizeof(float) * kda::kChunk * kda::kChunk * units, 256);
+    L.dS_off = round_up(L.states_off + sizeof(float) * (size_t)dk * dv * units, 256);
+    L.dU_off = round_up(L.dS_off + sizeof(float) * (size_t)dk * dv * units, 256);
+    L.scratch_off = round_up(L.dU_off + sizeof(float) * kda::kChunk * (size_t)dv * units, 256);
+    L.ctas = (int)(units < (size_t)kda::kBwdMaxCtas ? units : (size_t)kda::kBwdMaxCtas);
+    L.total = L.scratch_off + kda::bwd_scratch_bytes_per_cta(dk, dv) * (size_t)L.ctas;
+    return true;
+}
+
 }  // namespace
 
 namespace kda {
@@ -228,6 +251,85 @@ kda_status kda_recurrent_step_gated(const void* q, const void* k, const void* v,
                                     const float* beta, float* state_inout, int B, int H, int dk, int dv,
                                     kda_dtype dtype, kda_gate gate, void* o, void* stream) {
     return recurrent_step_impl(q, k, v, log_alpha, beta, state_inout, B, H, dk, dv, dtype, gate, o, stream);
+}
+
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int varlen,
+                                    kda_dtype dtype) {
+    BwdLayout L;
+    if (!bwd_layout(B, T, H, dk, dv, num_seqs, varlen != 0, dtype, L)) return 0;
+    return L.total;
+}
+
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                         const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                         const void* d_o, const float* d_final_state, int B, int T, int H, int dk, int dv,
+                         int num_seqs, kda_dtype dtype, void* dq, void* dk_out, void* dv_out,
+                         float* dlog_alpha, float* dbeta, float* d_initial_state, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (B < 0 || T < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d", B, T, H);
+    if (dk <= 0 || dv <= 0) return fail(KDA_ERR_INVALID_ARG, "bad head sizes dk=%d dv=%d", dk, dv);
+    if (!supported_dim(dk) || !supported_dim(dv))
+        return fail(KDA_ERR_UNSUPPORTED, "head sizes dk=%d dv=%d not in {64, 128}", dk, dv);
+    const bool varlen = cu_seqlens != nullptr;
+    if (varlen && B != 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (got B=%d)", B);
+    if (varlen && num_seqs < 0) return fail(KDA_ERR_INVALID_ARG, "num_seqs=%d < 0", num_seqs);
+    const int N = varlen ? num_seqs : B;
+    const size_t tokens = varlen ? (size_t)T : (size_t)B * T;
+    if (tokens * (size_t)H * (size_t)(dk > dv ? dk : dv) >= (size_t)1 << 31)
+        return fail(KDA_ERR_UNSUPPORTED, "B*T*H*d = %zu elements exceeds 2^31", tokens * H * (dk > dv ? dk : dv));
+    if (tokens > 0) {
+        if (!q || !k || !v || !log_alpha || !beta || !d_o || !dq || !dk_out || !dv_out || !dlog_alpha || !dbeta)
+            return fail(KDA_ERR_INVALID_ARG, "null input/output pointer");
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) || !aligned16(log_alpha))
+            return fail(KDA_ERR_INVALID_ARG, "q/k/v/log_alpha/d_o must be 16-byte aligned");
+    }
+    BwdLayout L;
+    if (!bwd_layout(B, T, H, dk, dv, num_seqs, varlen, dtype, L))
+        return fail(KDA_ERR_INVALID_ARG, "invalid sizes for the workspace layout");
+    if (!workspace) return fail(KDA_ERR_WORKSPACE, "workspace is null (need %zu bytes)", L.total);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(KDA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (workspace_bytes < L.total)
+        return fail(KDA_ERR_WORKSPACE, "workspace has %zu bytes, need %zu", workspace_bytes, L.total);
+
+    char* ws = static_cast<char*>(workspace);
+    kda::ChunkArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.num_seqs = N;
+    a.gate = kda::kGateChannel;
+    a.bf16 = dtype == KDA_BF16;
+    a.scale = 1.0f / sqrtf((float)dk);
+    a.ws_header = workspace;
+    a.chunk_offsets = reinterpret_cast<int32_t*>(ws + L.base.offsets_off);
+    a.records = ws + L.base.records_off;
+    a.max_chunks = L.base.max_chunks;
+    a.fixed_chunks_per_seq = L.base.chunks_per_seq;
+    a.stream = static_cast<cudaStream_t>(stream);
+    a.tmat = reinterpret_cast<float*>(ws + L.tmat_off);
+    a.states = reinterpret_cast<float*>(ws + L.states_off);
+    a.d_o = d_o; a.d_final_state = d_final_state;
+    a.dq = dq; a.dk_out = dk_out; a.dv_out = dv_out;
+    a.dlog_alpha = dlog_alpha; a.dbeta = dbeta; a.d_initial_state = d_initial_state;
+    a.dS_end = reinterpret_cast<float*>(ws + L.dS_off);
+    a.dU = reinterpret_cast<float*>(ws + L.dU_off);
+    a.scratch = reinterpret_cast<float*>(ws + L.scratch_off);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "device query failed: %s", cudaGetErrorString(e));
+    a.bwd_ctas = L.ctas < 2 * sms ? L.ctas : 2 * sms;
+
+    // forward recomputation (fp32 records + T + chunk-start states), then the
+    // reversed pass over chunks, then the per-chunk gradients
+    e = kda::launch_chunk_prep(a);
+    if (e == cudaSuccess) e = kda::launch_chunk_intra(a);
+    if (e == cudaSuccess) e = kda::launch_chunk_inter(a);
+    if (e == cudaSuccess) e = kda::launch_chunk_bwd_inter(a);
+    if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_chunk_bwd launch failed: %s", cudaGetErrorString(e));
+    return ok();
 }
 
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {

@@ -1,0 +1,656 @@
+// kda_chunk_bwd.cu -- chunkwise KDA backward on CUDA cores in fp32 (sm_100a).
+//
+// The chunkwise form is the training mode of news.bugfactory.tech/news/3610
+// (KDA paragraph); this file differentiates it.  The forward chunk algebra
+// (unrolling the update equation of the daiw.net page, section "KDA 的更新式",
+// over a chunk of L <= 64 tokens; g_r = sum_{i<=r} log_alpha_i per channel):
+//
+//   Kl = k e^{g-g_m}  Kr = k e^{g_m-g}  Ql = q e^{g-g_m}     (split at the middle token)
+//   M = Kl Kr^T,  A = diag(beta) M (strictly lower),  P = Ql Kr^T (lower incl. diagonal)
+//   T = (I + A)^{-1},  K~ = k e^{g},  Q~ = q e^{g},  K^ = k e^{g_{L-1}-g},  gamma = e^{g_{L-1}}
+//   W = T diag(beta) K~,  U0 = T diag(beta) V
+//   U = U0 - W S,  O = c (Q~ S + P U),  S' = Diag(gamma) S + K^^T U       (c = dk^{-1/2})
+//
+// Reverse, with D = c dO and dS' the cotangent of the state leaving the chunk:
+//
+//   across chunks (serial, reversed; KB3):
+//     dU = P^T D + K^ dS'               dS = Diag(gamma) dS' + Q~^T D - W^T dU
+//   within a chunk (all chunks in parallel; KB4):
+//     dQ~ = D S^T   dK^ = U dS'^T   dW = -dU S^T   dP = D U^T (lower)   dgamma = rowsum(dS' * S)
+//     Z = T^T dU  -> dv = beta Z,  dbeta += <Z, v>
+//     Y = T^T dW  -> dK~ = beta Y, dbeta += <Y, K~>
+//     dT = (dW K~^T + dU V^T) diag(beta);   dA = -T^T dT T^T (strictly lower)
+//     dbeta += rowsum(dA * M);  dM = diag(beta) dA
+//     dKl = dM Kr,  dQl = dP Kr,  dKr = dM^T Kl + dP^T Ql
+//     dk = dKl e^{g-g_m} + dKr e^{g_m-g} + dK~ e^{g} + dK^ e^{g_{L-1}-g}
+//     dq = dQl e^{g-g_m} + dQ~ e^{g}
+//     dg = k (dKl e^{g-g_m} - dKr e^{g_m-g} + dK~ e^{g} - dK^ e^{g_{L-1}-g}) + q (dQl e^{g-g_m} + dQ~ e^{g})
+//     dg_{L-1} += sum_r dK^_r K^_r + dgamma gamma;   dlog_alpha_s = sum_{r>=s} dg_r
+//
+// (The split point g_m cancels in M and P, so it carries no gradient.)  Chunks
+// whose decay is too strong for the split factors use the exact pairwise form
+// e^{g_r - g_i} <= 1 instead, as the forward does.
+//
+// The forward quantities come from the forward kernels run again with two
+// extra outputs: T from K1 and the state entering every chunk from K2.
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace kda {
+namespace {
+
+constexpr float kMaxSplitExponent = 60.f;   // same split guard as the forward
+
+// fp32 record of the CUDA-core forward (same layout as kda_chunk_simt.cu)
+template <int DK, int DV>
+struct Rec {
+    static constexpr size_t W = 0;
+    static constexpr size_t U0 = W + kChunk * DK;
+    static constexpr size_t QT = U0 + kChunk * DV;
+    static constexpr size_t KH = QT + kChunk * DK;
+    static constexpr size_t P = KH + kChunk * DK;
+    static constexpr size_t GC = P + kChunk * kChunk;
+    static constexpr size_t FLOATS = (GC + DK + 63) / 64 * 64;
+};
+
+// ------------------------------------------------------------------ KB3 ----
+constexpr int kSlice = 32;   // value columns per CTA
+
+template <int DK>
+struct BwdInterSmem {
+    static constexpr int LDK = DK + 4;
+    float dS[DK][kSlice + 1];
+    float W[kChunk][LDK];
+    float Qt[kChunk][LDK];
+    float Kh[kChunk][LDK];
+    float P[kChunk][kChunk + 4];
+    float D[kChunk][kSlice + 4];
+    float dU[kChunk][kSlice + 4];
+    float gC[DK];
+};
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(128)
+bwd_inter_kernel(const T* __restrict__ d_o, const float* __restrict__ d_final_state,
+                 float* __restrict__ d_initial_state, float* __restrict__ dS_end, float* __restrict__ dU_all,
+                 ChunkMap map, const WsHeader* __restrict__ hdr, const float* __restrict__ records,
+                 int H, size_t max_chunks, float scale)
+{
+    using R = Rec<DK, DV>;
+    using Sm = BwdInterSmem<DK>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    Sm& sm = *reinterpret_cast<Sm*>(smem_raw);
+
+    if (hdr->status != kStatusOk) return;
+    const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSlice;
+    const int tid = threadIdx.x, lane = tid & 31, ry = tid >> 5;
+    const size_t state_off = ((size_t)s * H + h) * DK * DV;
+
+    for (int idx = tid; idx < DK * kSlice; idx += 128) {
+        const int r = idx / kSlice, j = idx - r * kSlice;
+        sm.dS[r][j] = d_final_state ? d_final_state[state_off + (size_t)r * DV + j0 + j] : 0.f;
+    }
+    const int first = map.seq_first_chunk(s);
+    const int nch = map.seq_num_chunks(s);
+    const int tok_begin = map.seq_token_begin(s), tok_end = map.seq_token_end(s);
+
+    for (int n = nch - 1; n >= 0; --n) {
+        const size_t item = (size_t)h * max_chunks + first + n;
+        const float* rec = records + item * R::FLOATS;
+        __syncthreads();   // dS of the chunk after this one is complete
+        {
+            float* out = dS_end + item * DK * DV;
+            for (int idx = tid; idx < DK * kSlice; idx += 128) {
+                const int r = idx / kSlice, j = idx - r * kSlice;
+                out[(size_t)r * DV + j0 + j] = sm.dS[r][j];
+            }
+        }
+        for (int idx = tid; idx < kChunk * DK / 4; idx += 128) {
+            const int r = idx / (DK / 4), c4 = (idx - r * (DK / 4)) * 4;
+            *reinterpret_cast<float4*>(&sm.W[r][c4]) = *reinterpret_cast<const float4*>(rec + R::W + (size_t)r * DK + c4);
+            *reinterpret_cast<float4*>(&sm.Qt[r][c4]) = *reinterpret_cast<const float4*>(rec + R::QT + (size_t)r * DK + c4);
+            *reinterpret_cast<float4*>(&sm.Kh[r][c4]) = *reinterpret_cast<const float4*>(rec + R::KH + (size_t)r * DK + c4);
+        }
+        for (int idx = tid; idx < kChunk * kChunk / 4; idx += 128) {
+            const int r = idx >> 4, c4 = (idx & 15) * 4;
+            *reinterpret_cast<float4*>(&sm.P[r][c4]) = *reinterpret_cast<const float4*>(rec + R::P + (size_t)r * kChunk + c4);
+        }
+        const int tok0 = tok_begin + n * kChunk;
+        for (int idx = tid; idx < kChunk * kSlice; idx += 128) {
+            const int r = idx / kSlice, j = idx - r * kSlice;
+            const int tok = tok0 + r;
+            sm.D[r][j] = tok < tok_end ? scale * to_f32(d_o[((size_t)tok * H + h) * DV + j0 + j]) : 0.f;
+        }
+        for (int idx = tid; idx < DK; idx += 128) sm.gC[idx] = rec[R::GC + idx];
+        __syncthreads();
+
+        // 1. dU = P^T D + K^ dS' for rows r = ry + 4a, column j = lane
+        float acc[16];
+#pragma unroll
+        for (int a = 0; a < 16; ++a) acc[a] = 0.f;
+        for (int c = 0; c < DK; c += 4) {
+            const float s0 = sm.dS[c][lane], s1 = sm.dS[c + 1][lane];
+            const float s2 = sm.dS[c + 2][lane], s3 = sm.dS[c + 3][lane];
+#pragma unroll
+            for (int a = 0; a < 16; ++a) {
+                const float4 kh = *reinterpret_cast<const float4*>(&sm.Kh[ry + 4 * a][c]);
+                acc[a] += kh.x * s0 + kh.y * s1 + kh.z * s2 + kh.w * s3;
+            }
+        }
+        for (int i = 0; i < kChunk; ++i) {
+            const float d = sm.D[i][lane];
+#pragma unroll
+            for (int a = 0; a < 16; ++a) acc[a] = fmaf(sm.P[i][ry + 4 * a], d, acc[a]);
+        }
+        {
+            float* out = dU_all + item * kChunk * DV;
+#pragma unroll
+            for (int a = 0; a < 16; ++a) {
+                sm.dU[ry + 4 * a][lane] = acc[a];
+                out[(size_t)(ry + 4 * a) * DV + j0 + lane] = acc[a];
+            }
+        }
+        __syncthreads();
+
+        // 2. dS = Diag(gamma) dS' + Q~^T D - W^T dU, one key row per thread
+        for (int c = tid; c < DK; c += 128) {
+            float x[kSlice];
+            const float gc = sm.gC[c];
+#pragma unroll
+            for (int j = 0; j < kSlice; ++j) x[j] = gc * sm.dS[c][j];
+            for (int r = 0; r < kChunk; ++r) {
+                const float qt = sm.Qt[r][c], w = sm.W[r][c];
+#pragma unroll
+                for (int j = 0; j < kSlice; j += 4) {
+                    const float4 d = *reinterpret_cast<const float4*>(&sm.D[r][j]);
+                    const float4 u = *reinterpret_cast<const float4*>(&sm.dU[r][j]);
+                    x[j] += qt * d.x - w * u.x;
+                    x[j + 1] += qt * d.y - w * u.y;
+                    x[j + 2] += qt * d.z - w * u.z;
+                    x[j + 3] += qt * d.w - w * u.w;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kSlice; ++j) sm.dS[c][j] = x[j];
+        }
+    }
+    __syncthreads();
+    if (d_initial_state) {
+        for (int idx = tid; idx < DK * kSlice; idx += 128) {
+            const int r = idx / kSlice, j = idx - r * kSlice;
+            d_initial_state[state_off + (size_t)r * DV + j0 + j] = sm.dS[r][j];
+        }
+    }
+}
+
+// ------------------------------------------------------------------ KB4 ----
+// A 64 x N product for the whole CTA (256 threads): thread (ty, tx) = (tid/16,
+// tid%16) owns rows 4 ty .. 4 ty + 3 and columns 64 h + 4 tx .. + 3 (h < N/64).
+// Operands are fp32 matrices in global memory (L2-resident scratch or inputs),
+// read in K-slabs of 32 through shared memory.  Element (r, c) of a Mat is
+// p[r * ld + c], or p[c * ld + r] when t is set (the stored matrix transposed).
+struct Mat {
+    const float* p;
+    int ld;
+    bool t;
+    __device__ __forceinline__ float at(int r, int c) const {
+        return t ? p[(size_t)c * ld + r] : p[(size_t)r * ld + c];
+    }
+};
+
+constexpr int kSlab = 32;
+constexpr int kMaxN = 128;
+
+struct GemmStage {
+    float a[kSlab][64 + 4];
+    float b[kSlab][kMaxN + 4];
+};
+
+template <int N>
+__device__ __forceinline__ void zero_acc(float (&acc)[4][N / 16]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < N / 16; ++j) acc[i][j] = 0.f;
+}
+
+// acc += A(64 x K) B(K x N)
+template <int N>
+__device__ void gemm64(float (&acc)[4][N / 16], Mat A, Mat B, int K, GemmStage& st) {
+    const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+    for (int k0 = 0; k0 < K; k0 += kSlab) {
+        __syncthreads();   // earlier readers of the stage / writers of the operands are done
+        for (int e = tid; e < 64 * kSlab; e += 256) {
+            int m, kk;
+            if (A.t) { kk = e >> 6; m = e & 63; } else { m = e / kSlab; kk = e % kSlab; }
+            st.a[kk][m] = A.at(m, k0 + kk);
+        }
+        for (int e = tid; e < N * kSlab; e += 256) {
+            int n, kk;
+            if (B.t) { n = e / kSlab; kk = e % kSlab; } else { kk = e / N; n = e % N; }
+            st.b[kk][n] = B.at(k0 + kk, n);
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int kk = 0; kk < kSlab; ++kk) {
+            const float4 av = *reinterpret_cast<const float4*>(&st.a[kk][ty * 4]);
+            const float ar[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+            for (int hh = 0; hh < N / 64; ++hh) {
+                const float4 bv = *reinterpret_cast<const float4*>(&st.b[kk][hh * 64 + tx * 4]);
+                const float br[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][hh * 4 + j] = fmaf(ar[i], br[j], acc[i][hh * 4 + j]);
+            }
+        }
+    }
+}
+
+// f(row, col, value) over the thread's accumulators
+template <int N, typename F>
+__device__ __forceinline__ void for_acc(float (&acc)[4][N / 16], F f) {
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int hh = 0; hh < N / 64; ++hh)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) f(ty * 4 + i, hh * 64 + tx * 4 + j, acc[i][hh * 4 + j]);
+}
+
+// Sum over the 16 threads that share a row (one half-warp).
+__device__ __forceinline__ float row_sum16(float x) {
+#pragma unroll
+    for (int off = 8; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+// Per-CTA fp32 scratch (global memory), offsets in floats.
+template <int DK, int DV>
+struct Scr {
+    static constexpr size_t KL = 0;                     // k e^{g-g_m} (strong chunk: raw k)
+    static constexpr size_t KR = KL + kChunk * DK;      // k e^{g_m-g}
+    static constexpr size_t QL = KR + kChunk * DK;      // q e^{g-g_m} (strong chunk: raw q)
+    static constexpr size_t KT = QL + kChunk * DK;      // K~ = k e^{g}
+    static constexpr size_t VV = KT + kChunk * DK;      // v
+    static constexpr size_t DO = VV + kChunk * DV;      // c dO
+    static constexpr size_t U = DO + kChunk * DV;
+    static constexpr size_t DQT = U + kChunk * DV;
+    static constexpr size_t DKH = DQT + kChunk * DK;
+    static constexpr size_t DW = DKH + kChunk * DK;
+    static constexpr size_t DKT = DW + kChunk * DK;
+    static constexpr size_t DP = DKT + kChunk * DK;
+    static constexpr size_t DT = DP + kChunk * kChunk;
+    static constexpr size_t X1 = DT + kChunk * kChunk;
+    static constexpr size_t DM = X1 + kChunk * kChunk;
+    static constexpr size_t M = DM + kChunk * kChunk;
+    static constexpr size_t DKL = M + kChunk * kChunk;  // dKl e^{g-g_m}
+    static constexpr size_t DQL = DKL + kChunk * DK;    // dQl e^{g-g_m}
+    static constexpr size_t DKR = DQL + kChunk * DK;    // dKr e^{g_m-g}
+    static constexpr size_t FLOATS = DKR + kChunk * DK;
+};
+
+template <int DK>
+struct BwdIntraSmem {
+    GemmStage st;
+    float g[kChunk][DK];   // cumulative log-decay, later dg
+    float gm[DK], gl[DK], dgam[DK], dgl[DK];
+    float beta[kChunk], dbeta[kChunk];
+};
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(256, 2)
+bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                 const float* __restrict__ log_alpha, const float* __restrict__ beta, const T* __restrict__ d_o,
+                 ChunkMap map, const WsHeader* __restrict__ hdr, const float* __restrict__ records,
+                 const float* __restrict__ tmat, const float* __restrict__ states,
+                 const float* __restrict__ dS_end, const float* __restrict__ dU_all, float* scratch,
+                 T* __restrict__ dq, T* __restrict__ dk, T* __restrict__ dv, float* __restrict__ dla,
+                 float* __restrict__ dbeta, int H, size_t max_chunks, float scale)
+{
+    using R = Rec<DK, DV>;
+    using C = Scr<DK, DV>;
+    using Sm = BwdIntraSmem<DK>;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    Sm& sm = *reinterpret_cast<Sm*>(smem_raw);
+
+    if (hdr->status != kStatusOk) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t rowk = (size_t)H * DK, rowv = (size_t)H * DV;
+    const long total = (long)hdr->num_chunks * H;
+    float* scr = scratch + (size_t)blockIdx.x * C::FLOATS;
+
+    for (long item = blockIdx.x; item < total; item += gridDim.x) {
+        const int c = (int)(item / H), h = (int)(item % H);
+        int s, tok0, L;
+        map.locate(c, s, tok0, L);
+        const size_t it = (size_t)h * max_chunks + c;
+        const float* rec = records + it * R::FLOATS;
+        const float* Tm = tmat + it * kChunk * kChunk;
+        const float* Sn = states + it * DK * DV;
+        const float* dSe = dS_end + it * DK * DV;
+        const float* dUc = dU_all + it * kChunk * DV;
+
+        __syncthreads();   // the previous item is done with shared memory and scratch
+        // ---- cumulative log-decay, beta --------------------------------------
+        if (tid < DK) {
+            const float* la = log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid;
+            float acc = 0.f;
+            for (int r = 0; r < kChunk; ++r) {
+                acc += (r < L) ? la[(size_t)r * rowk] : 0.f;
+                sm.g[r][tid] = acc;
+            }
+            sm.dgl[tid] = 0.f;
+        } else if (tid >= 128 && tid < 128 + kChunk) {
+            const int r = tid - 128;
+            sm.beta[r] = (r < L) ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
+            sm.dbeta[r] = 0.f;
+        }
+        __syncthreads();
+        bool wide = false;
+        if (tid < DK) {
+            sm.gm[tid] = sm.g[(L - 1) >> 1][tid];
+            sm.gl[tid] = sm.g[L - 1][tid];
+            wide = fmaxf(sm.g[0][tid] - sm.gm[tid], sm.gm[tid] - sm.gl[tid]) > kMaxSplitExponent;
+        }
+        const bool strong = __syncthreads_or(wide);
+
+        // ---- operands into scratch ------------------------------------------
+        for (int idx = tid; idx < kChunk * DK; idx += 256) {
+            const int r = idx / DK, ch = idx - r * DK;
+            float kk = 0.f, qq = 0.f;
+            if (r < L) {
+                const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
+                kk = to_f32(k[off]);
+                qq = to_f32(q[off]);
+            }
+            const float gg = sm.g[r][ch];
+            if (!strong) {
+                const float em = expf(gg - sm.gm[ch]);
+                scr[C::KL + idx] = kk * em;
+                scr[C::KR + idx] = kk * expf(sm.gm[ch] - gg);
+                scr[C::QL + idx] = qq * em;
+            } else {
+                scr[C::KL + idx] = kk;
+                scr[C::QL + idx] = qq;
+            }
+            scr[C::KT + idx] = kk * expf(gg);
+        }
+        for (int idx = tid; idx < kChunk * DV; idx += 256) {
+            const int r = idx / DV, j = idx - r * DV;
+            const size_t off = (size_t)(tok0 + r) * rowv + (size_t)h * DV + j;
+            scr[C::VV + idx] = (r < L) ? to_f32(v[off]) : 0.f;
+            scr[C::DO + idx] = (r < L) ? scale * to_f32(d_o[off]) : 0.f;
+        }
+        // dgamma_c = sum_j dS'_cj S_cj: one warp per key row
+        for (int ch = warp; ch < DK; ch += 8) {
+            float acc = 0.f;
+            for (int j = lane; j < DV; j += 32) acc += dSe[(size_t)ch * DV + j] * Sn[(size_t)ch * DV + j];
+#pragma unroll
+            for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (lane == 0) sm.dgam[ch] = acc;
+        }
+
+        // ---- products over the value dimension ---------------------------------
+        {   // U = U0 - W S
+            float acc[4][DV / 16];
+            zero_acc<DV>(acc);
+            gemm64<DV>(acc, Mat{rec + R::W, DK, false}, Mat{Sn, DV, false}, DK, sm.st);
+            for_acc<DV>(acc, [&](int r, int n, float x) { scr[C::U + r * DV + n] = rec[R::U0 + r * DV + n] - x; });
+        }
+        {   // dQ~ = D S^T
+            float acc[4][DK / 16];
+            zero_acc<DK>(acc);
+            gemm64<DK>(acc, Mat{scr + C::DO, DV, false}, Mat{Sn, DV, true}, DV, sm.st);
+            for_acc<DK>(acc, [&](int r, int n, float x) { scr[C::DQT + r * DK + n] = x; });
+        }
+        {   // dW = -dU S^T
+            float acc[4][DK / 16];
+            zero_acc<DK>(acc);
+            gemm64<DK>(acc, Mat{dUc, DV, false}, Mat{Sn, DV, true}, DV, sm.st);
+            for_acc<DK>(acc, [&](int r, int n, float x) { scr[C::DW + r * DK + n] = -x; });
+        }
+        {   // dK^ = U dS'^T
+            float acc[4][DK / 16];
+            zero_acc<DK>(acc);
+            gemm64<DK>(acc, Mat{scr + C::U, DV, false}, Mat{dSe, DV, true}, DV, sm.st);
+            for_acc<DK>(acc, [&](int r, int n, float x) { scr[C::DKH + r * DK + n] = x; });
+        }
+        {   // dP = D U^T, lower triangle with the diagonal
+            float acc[4][kChunk / 16];
+            zero_acc<kChunk>(acc);
+            gemm64<kChunk>(acc, Mat{scr + C::DO, DV, false}, Mat{scr + C::U, DV, true}, DV, sm.st);
+            for_acc<kChunk>(acc, [&](int r, int i, float x) { scr[C::DP + r * kChunk + i] = (i <= r) ? x : 0.f; });
+        }
+        // ---- through W = T diag(beta) K~ and U0 = T diag(beta) V -------------
+        {   // Z = T^T dU: dv = beta Z, dbeta += <Z, v>
+            float acc[4][DV / 16];
+            zero_acc<DV>(acc);
+            gemm64<DV>(acc, Mat{Tm, kChunk, true}, Mat{dUc, DV, false}, kChunk, sm.st);
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
+            for_acc<DV>(acc, [&](int r, int n, float x) {
+                part[r & 3] += x * scr[C::VV + r * DV + n];
+                if (r < L) dv[(size_t)(tok0 + r) * rowv + (size_t)h * DV + n] = from_f32<T>(sm.beta[r] * x);
+            });
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float t = row_sum16(part[i]);
+                if ((tid & 15) == 0) sm.dbeta[(tid >> 4) * 4 + i] += t;
+            }
+        }
+        {   // Y = T^T dW: dK~ = beta Y, dbeta += <Y, K~>
+            float acc[4][DK / 16];
+            zero_acc<DK>(acc);
+            gemm64<DK>(acc, Mat{Tm, kChunk, true}, Mat{scr + C::DW, DK, false}, kChunk, sm.st);
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
+            for_acc<DK>(acc, [&](int r, int n, float x) {
+                part[r & 3] += x * scr[C::KT + r * DK + n];
+                scr[C::DKT + r * DK + n] = sm.beta[r] * x;
+            });
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float t = row_sum16(part[i]);
+                if ((tid & 15) == 0) sm.dbeta[(tid >> 4) * 4 + i] += t;
+            }
+        }
+        {   // dT = (dW K~^T + dU V^T) diag(beta)
+            float acc[4][kChunk / 16];
+            zero_acc<kChunk>(acc);
+            gemm64<kChunk>(acc, Mat{scr + C::DW, DK, false}, Mat{scr + C::KT, DK, true}, DK, sm.st);
+            gemm64<kChunk>(acc, Mat{dUc, DV, false}, Mat{scr + C::VV, DV, true}, DV, sm.st);
+            for_acc<kChunk>(acc, [&](int r, int i, float x) { scr[C::DT + r * kChunk + i] = x * sm.beta[i]; });
+        }
+        {   // X1 = dT T^T
+            float acc[4][kChunk / 16];
+            zero_acc<kChunk>(acc);
+            gemm64<kChunk>(acc, Mat{scr + C::DT, kChunk, false}, Mat{Tm, kChunk, true}, kChunk, sm.st);
+            for_acc<kChunk>(acc, [&](int r, int i, float x) { scr[C::X1 + r * kChunk + i] = x; });
+        }
+        // ---- M = Kl Kr^T (the unweighted A), strictly lower -------------------
+        if (!strong) {
+            float acc[4][kChunk / 16];
+            zero_acc<kChunk>(acc);
+            gemm64<kChunk>(acc, Mat{scr + C::KL, DK, false}, Mat{scr + C::KR, DK, true}, DK, sm.st);
+            for_acc<kChunk>(acc, [&](int r, int i, float x) { scr[C::M + r * kChunk + i] = (i < r) ? x : 0.f; });
+        } else {   // exact: one warp per (r, i), every exponent <= 0
+            __syncthreads();
+            for (int pr = warp; pr < kChunk * kChunk; pr += 8) {
+                const int r = pr >> 6, i = pr & 63;
+                float acc = 0.f;
+                if (i < r)
+                    for (int ch = lane; ch < DK; ch += 32)
+                        acc += scr[C::KL + r * DK + ch] * scr[C::KL + i * DK + ch] * expf(sm.g[r][ch] - sm.g[i][ch]);
+#pragma unroll
+                for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                if (lane == 0) scr[C::M + pr] = acc;
+            }
+        }
+        {   // dA = -T^T X1 (strictly lower); dbeta += rowsum(dA M); dM = diag(beta) dA
+            float acc[4][kChunk / 16];
+            zero_acc<kChunk>(acc);
+            gemm64<kChunk>(acc, Mat{Tm, kChunk, true}, Mat{scr + C::X1, kChunk, false}, kChunk, sm.st);
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
+            for_acc<kChunk>(acc, [&](int r, int i, float x) {
+                const float da = (i < r) ? -x : 0.f;
+                part[r & 3] += da * scr[C::M + r * kChunk + i];
+                scr[C::DM + r * kChunk + i] = sm.beta[r] * da;
+            });
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float t = row_sum16(part[i]);
+                if ((tid & 15) == 0) sm.dbeta[(tid >> 4) * 4 + i] += t;
+            }
+        }
+        // ---- through M and P to the (decayed) keys and queries ---------------
+        if (!strong) {
+            {   // dKl = dM Kr, dQl = dP Kr (times e^{g-g_m})
+                float acc[4][DK / 16];
+                zero_acc<DK>(acc);
+                gemm64<DK>(acc, Mat{scr + C::DM, kChunk, false}, Mat{scr + C::KR, DK, false}, kChunk, sm.st);
+                for_acc<DK>(acc, [&](int r, int n, float x) {
+                    scr[C::DKL + r * DK + n] = x * expf(sm.g[r][n] - sm.gm[n]);
+                });
+                zero_acc<DK>(acc);
+                gemm64<DK>(acc, Mat{scr + C::DP, kChunk, false}, Mat{scr + C::KR, DK, false}, kChunk, sm.st);
+                for_acc<DK>(acc, [&](int r, int n, float x) {
+                    scr[C::DQL + r * DK + n] = x * expf(sm.g[r][n] - sm.gm[n]);
+                });
+            }
+            {   // dKr = dM^T Kl + dP^T Ql (times e^{g_m-g})
+                float acc[4][DK / 16];
+                zero_acc<DK>(acc);
+                gemm64<DK>(acc, Mat{scr + C::DM, kChunk, true}, Mat{scr + C::KL, DK, false}, kChunk, sm.st);
+                gemm64<DK>(acc, Mat{scr + C::DP, kChunk, true}, Mat{scr + C::QL, DK, false}, kChunk, sm.st);
+                for_acc<DK>(acc, [&](int r, int n, float x) {
+                    scr[C::DKR + r * DK + n] = x * expf(sm.gm[n] - sm.g[r][n]);
+                });
+            }
+        } else {   // exact pairwise form; KL / QL hold the raw k / q
+            __syncthreads();
+            for (int idx = tid; idx < kChunk * DK; idx += 256) {
+                const int r = idx / DK, ch = idx - r * DK;
+                const float gr = sm.g[r][ch];
+                const float kr = scr[C::KL + idx], qr = scr[C::QL + idx];
+                float dkl = 0.f, dql = 0.f, dkr = 0.f;
+                for (int i = 0; i <= r; ++i) {   // r is the later token
+                    const float e = expf(gr - sm.g[i][ch]);
+                    const float ki = scr[C::KL + i * DK + ch];
+                    dql += scr[C::DP + r * kChunk + i] * ki * e;
+                    if (i < r) dkl += scr[C::DM + r * kChunk + i] * ki * e;
+                }
+                for (int j = r; j < kChunk; ++j) {   // r is the earlier token
+                    const float e = expf(sm.g[j][ch] - gr);
+                    dkr += scr[C::DP + j * kChunk + r] * scr[C::QL + j * DK + ch] * e;
+                    if (j > r) dkr += scr[C::DM + j * kChunk + r] * scr[C::KL + j * DK + ch] * e;
+                }
+                (void)kr; (void)qr;
+                scr[C::DKL + idx] = dkl;
+                scr[C::DQL + idx] = dql;
+                scr[C::DKR + idx] = dkr;
+            }
+        }
+        __syncthreads();
+
+        // ---- dq, dk, dg -------------------------------------------------------
+        for (int idx = tid; idx < kChunk * DK; idx += 256) {
+            const int r = idx / DK, ch = idx - r * DK;
+            float kk = 0.f, qq = 0.f;
+            const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
+            if (r < L) {
+                kk = to_f32(k[off]);
+                qq = to_f32(q[off]);
+            }
+            const float gg = sm.g[r][ch];
+            const float eg = expf(gg), eh = expf(sm.gl[ch] - gg);
+            const float dkl = scr[C::DKL + idx], dkr = scr[C::DKR + idx], dql = scr[C::DQL + idx];
+            const float dkt = scr[C::DKT + idx], dkh = scr[C::DKH + idx], dqt = scr[C::DQT + idx];
+            if (r < L) {
+                dk[off] = from_f32<T>(dkl + dkr + dkt * eg + dkh * eh);
+                dq[off] = from_f32<T>(dql + dqt * eg);
+            }
+            const float kh = kk * eh;
+            atomicAdd(&sm.dgl[ch], dkh * kh);
+            sm.g[r][ch] = kk * (dkl - dkr + dkt * eg) - dkh * kh + qq * (dql + dqt * eg);   // dg
+        }
+        __syncthreads();
+        // dlog_alpha_s = sum_{r >= s} dg_r, with g_{L-1}'s own cotangent added at L-1
+        if (tid < DK) {
+            float run = sm.dgl[tid] + sm.dgam[tid] * expf(sm.gl[tid]);
+            for (int r = L - 1; r >= 0; --r) {
+                run += sm.g[r][tid];
+                dla[(size_t)(tok0 + r) * rowk + (size_t)h * DK + tid] = run;
+            }
+        } else if (tid >= 128 && tid < 128 + kChunk) {
+            const int r = tid - 128;
+            if (r < L) dbeta[(size_t)(tok0 + r) * H + h] = sm.dbeta[r];
+        }
+    }
+}
+
+template <typename T, int DK, int DV>
+cudaError_t launch_bwd_inter_t(const ChunkArgs& a) {
+    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
+    auto kern = bwd_inter_kernel<T, DK, DV>;
+    const int smem = (int)sizeof(BwdInterSmem<DK>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)a.num_seqs, (unsigned)a.H, (unsigned)(DV / kSlice));
+    kern<<<grid, 128, smem, a.stream>>>(static_cast<const T*>(a.d_o), a.d_final_state, a.d_initial_state,
+                                         a.dS_end, a.dU, map, static_cast<const WsHeader*>(a.ws_header),
+                                         static_cast<const float*>(a.records), a.H, a.max_chunks, a.scale);
+    return cudaGetLastError();
+}
+
+template <typename T, int DK, int DV>
+cudaError_t launch_bwd_intra_t(const ChunkArgs& a) {
+    if (a.max_chunks == 0 || a.bwd_ctas <= 0) return cudaSuccess;
+    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
+    auto kern = bwd_intra_kernel<T, DK, DV>;
+    const int smem = (int)sizeof(BwdIntraSmem<DK>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<a.bwd_ctas, 256, smem, a.stream>>>(
+        static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.log_alpha, a.beta,
+        static_cast<const T*>(a.d_o), map, static_cast<const WsHeader*>(a.ws_header),
+        static_cast<const float*>(a.records), a.tmat, a.states, a.dS_end, a.dU, a.scratch,
+        static_cast<T*>(a.dq), static_cast<T*>(a.dk_out), static_cast<T*>(a.dv_out), a.dlog_alpha, a.dbeta,
+        a.H, a.max_chunks, a.scale);
+    return cudaGetLastError();
+}
+
+#define KDA_BWD_DISPATCH(FN, a)                                                     \
+    do {                                                                            \
+        if ((a).bf16) {                                                             \
+            if ((a).dk == 128 && (a).dv == 128) return FN<__nv_bfloat16, 128, 128>(a); \
+            if ((a).dk == 128 && (a).dv == 64) return FN<__nv_bfloat16, 128, 64>(a);   \
+            if ((a).dk == 64 && (a).dv == 128) return FN<__nv_bfloat16, 64, 128>(a);   \
+            if ((a).dk == 64 && (a).dv == 64) return FN<__nv_bfloat16, 64, 64>(a);     \
+        } else {                                                                    \
+            if ((a).dk == 128 && (a).dv == 128) return FN<float, 128, 128>(a);         \
+            if ((a).dk == 128 && (a).dv == 64) return FN<float, 128, 64>(a);           \
+            if ((a).dk == 64 && (a).dv == 128) return FN<float, 64, 128>(a);           \
+            if ((a).dk == 64 && (a).dv == 64) return FN<float, 64, 64>(a);             \
+        }                                                                           \
+        return cudaErrorInvalidValue;                                               \
+    } while (0)
+
+}  // namespace
+
+size_t bwd_scratch_bytes_per_cta(int dk, int dv) {
+    if (dk == 128 && dv == 128) return Scr<128, 128>::FLOATS * sizeof(float);
+    if (dk == 128 && dv == 64) return Scr<128, 64>::FLOATS * sizeof(float);
+    if (dk == 64 && dv == 128) return Scr<64, 128>::FLOATS * sizeof(float);
+    if (dk == 64 && dv == 64) return Scr<64, 64>::FLOATS * sizeof(float);
+    return 0;
+}
+
+cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a) {
+    if (a.num_seqs == 0) return cudaSuccess;
+    KDA_BWD_DISPATCH(launch_bwd_inter_t, a);
+}
+
+cudaError_t launch_chunk_bwd_intra(const ChunkArgs& a) { KDA_BWD_DISPATCH(launch_bwd_intra_t, a); }
+
+}  // namespace kda

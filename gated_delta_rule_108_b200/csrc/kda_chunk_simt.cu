@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256)
 intra_chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                         const float* __restrict__ log_alpha, const float* __restrict__ beta,
                         ChunkMap map, const WsHeader* __restrict__ hdr, float* __restrict__ records,
-                        int H, size_t max_chunks, int gate)
+                        float* __restrict__ tmat, int H, size_t max_chunks, int gate)
 {
     using R = SimtRec<DK, DV>;
     using Sm = IntraSmem<T, DK, DV>;
@@ -264,6 +264,11 @@ intra_chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const 
             for (int i = r & ~3; i < r; ++i) a0 -= sm.Am[r][i] * x[i];
             x[r] = (a0 + a1) + (a2 + a3);
         }
+        if (tmat) {   // T itself, for the backward pass
+            float* tm = tmat + ((size_t)h * max_chunks + c) * kChunk * kChunk;
+#pragma unroll
+            for (int r = 0; r < kChunk; ++r) tm[r * kChunk + tid] = x[r];
+        }
     } else {
         for (int idx = tid - kChunk; idx < kChunk * DK; idx += 256 - kChunk) {
             const int r = idx / DK, ch = idx - r * DK;
@@ -340,8 +345,9 @@ struct InterSmem {
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(128)
 inter_chunk_simt_kernel(const float* __restrict__ initial_state, float* __restrict__ final_state,
-                        T* __restrict__ o, ChunkMap map, const WsHeader* __restrict__ hdr,
-                        const float* __restrict__ records, int H, size_t max_chunks, float scale)
+                        T* __restrict__ o, float* __restrict__ states, ChunkMap map,
+                        const WsHeader* __restrict__ hdr, const float* __restrict__ records, int H,
+                        size_t max_chunks, float scale)
 {
     using R = SimtRec<DK, DV>;
     using Sm = InterSmem<DK>;
@@ -380,6 +386,13 @@ inter_chunk_simt_kernel(const float* __restrict__ initial_state, float* __restri
             sm.U0[r][j] = rec[R::U0 + (size_t)r * DV + j0 + j];
         }
         for (int idx = tid; idx < DK; idx += 128) sm.gC[idx] = rec[R::GC + idx];
+        if (states) {   // the state entering this chunk, for the backward pass
+            float* st = states + ((size_t)h * max_chunks + first + n) * DK * DV;
+            for (int idx = tid; idx < DK * kSlice; idx += 128) {
+                const int r = idx / kSlice, j = idx - r * kSlice;
+                st[(size_t)r * DV + j0 + j] = sm.S[r][j];
+            }
+        }
         __syncthreads();
 
         // 1. W S and Q~ S for rows r = ry + 4a, column j = lane
@@ -403,6 +416,7 @@ inter_chunk_simt_kernel(const float* __restrict__ initial_state, float* __restri
         __syncthreads();
 
         // 2. O = scale (Q~ S + P U)
+        if (o) {
         for (int i = 0; i < kChunk; i += 4) {
             const float u0 = sm.U[i][lane], u1 = sm.U[i + 1][lane];
             const float u2 = sm.U[i + 2][lane], u3 = sm.U[i + 3][lane];
@@ -419,6 +433,7 @@ inter_chunk_simt_kernel(const float* __restrict__ initial_state, float* __restri
             if (tok < tok_end)
                 o[((size_t)tok * H + h) * DV + j0 + lane] = from_f32<T>(scale * qs[a]);
         }
+        }  // o
 
         // 3. S' = Diag(gC) S + K^^T U, one key row per thread
         if (tid < DK) {
@@ -460,7 +475,7 @@ cudaError_t launch_intra_t(const ChunkArgs& a) {
     k1<<<grid, 256, smem, a.stream>>>(
         static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v),
         a.log_alpha, a.beta, map, static_cast<const WsHeader*>(a.ws_header),
-        static_cast<float*>(a.records), a.H, a.max_chunks, a.gate);
+        static_cast<float*>(a.records), a.tmat, a.H, a.max_chunks, a.gate);
     return cudaGetLastError();
 }
 
@@ -472,7 +487,7 @@ cudaError_t launch_inter_t(const ChunkArgs& a) {
     cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.num_seqs, (unsigned)a.H, (unsigned)(DV / kSlice));
-    k2<<<grid, 128, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<T*>(a.o), map,
+    k2<<<grid, 128, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<T*>(a.o), a.states, map,
                                        static_cast<const WsHeader*>(a.ws_header),
                                        static_cast<const float*>(a.records), a.H, a.max_chunks,
                                        a.scale);

@@ -37,6 +37,18 @@ struct ChunkArgs {
     size_t max_chunks;            // chunks per head the records can hold
     int fixed_chunks_per_seq;     // ceil(T / 64) for fixed length
     cudaStream_t stream;
+    // backward pass only (all null in the forward)
+    float* tmat;                  // [H][max_chunks][64][64]: K1 also writes T = (I + A)^{-1}
+    float* states;                // [H][max_chunks][dk][dv]: K2 also writes the state entering each chunk
+    const void* d_o;              // [.., H, dv], input dtype
+    const float* d_final_state;   // [N, H, dk, dv], nullable (zeros)
+    void* dq; void* dk_out; void* dv_out;   // input dtype
+    float* dlog_alpha; float* dbeta;
+    float* d_initial_state;       // [N, H, dk, dv], nullable (not written)
+    float* dS_end;                // [H][max_chunks][dk][dv]: dL/d(state leaving each chunk)
+    float* dU;                    // [H][max_chunks][64][dv]: dL/dU of each chunk
+    float* scratch;               // per-CTA fp32 scratch of the per-chunk gradient kernel
+    int bwd_ctas;                 // CTAs of that kernel (its scratch holds this many)
 };
 
 // Bytes of per-(head, chunk) intermediates: fp32 CUDA-core path / bf16 tensor-core path.
@@ -53,5 +65,9 @@ cudaError_t launch_chunk_intra(const ChunkArgs& a);    // K1: all chunks in para
 cudaError_t launch_chunk_inter(const ChunkArgs& a);    // K2: serial over each sequence's chunks
 cudaError_t launch_chunk_intra_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K1
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K2
+cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a);  // backward: serial over chunks, reversed
+cudaError_t launch_chunk_bwd_intra(const ChunkArgs& a);  // backward: all chunks in parallel
+size_t bwd_scratch_bytes_per_cta(int dk, int dv);
+constexpr int kBwdMaxCtas = 512;   // scratch is sized for at most this many CTAs
 
 }  // namespace kda

@@ -126,7 +126,7 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
 
 /*
  * Waits for `stream`, then reads the device status that the last
- * kda_chunk_fwd on this workspace left: KDA_OK, KDA_ERR_BAD_SEQLENS,
+ * kda_chunk_fwd or kda_chunk_bwd on this workspace left: KDA_OK, KDA_ERR_BAD_SEQLENS,
  * KDA_ERR_TIMEOUT or KDA_ERR_RANGE (or KDA_ERR_CUDA if the copy fails).
  * KDA_ERR_RANGE means a value-side quantity (|v|, the state, the per-token
  * errors u) exceeded 65000 in magnitude: the bf16 path keeps its chunk
@@ -186,6 +186,45 @@ kda_status kda_chunk_fwd_static(const void* q, const void* k, const void* v,
                                 const float* initial_state, const int32_t* cu_seqlens,
                                 int B, int T, int H, int dk, int dv, int num_seqs,
                                 kda_dtype dtype, void* o, float* final_state, void* stream);
+
+/*
+ * Bytes of device workspace kda_chunk_bwd needs for these sizes (arguments as
+ * kda_chunk_fwd_workspace_size).  Returns 0 for invalid sizes.
+ */
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv,
+                                    int num_seqs, int varlen, kda_dtype dtype);
+
+/*
+ * Gradients of the chunkwise forward (the chunkwise mode is the training mode
+ * of news.bugfactory.tech/news/3610, KDA paragraph).  For the loss
+ *     L = sum <d_o, o> + sum <d_final_state, final_state>
+ * of the kda_chunk_fwd call with the same inputs, it writes dL/dq, dL/dk,
+ * dL/dv, dL/dlog_alpha, dL/dbeta and dL/dinitial_state.  The forward
+ * quantities are recomputed from the inputs (no forward output is needed).
+ * All arithmetic is fp32 on CUDA cores for both dtypes.
+ *
+ *  q, k, v, log_alpha, beta, initial_state, cu_seqlens, sizes, dtype:
+ *              as kda_chunk_fwd (per-channel gate)
+ *  d_o         [B, T, H, dv]   dtype, cotangent of o
+ *  d_final_state [N, H, dk, dv] fp32, cotangent of the final state, or NULL
+ *              for zeros
+ *  dq, dk      [B, T, H, dk]   dtype, written
+ *  dv          [B, T, H, dv]   dtype, written
+ *  dlog_alpha  [B, T, H, dk]   fp32, written
+ *  dbeta       [B, T, H]       fp32, written
+ *  d_initial_state [N, H, dk, dv] fp32, written, or NULL (not computed)
+ *  workspace   device scratch of at least kda_chunk_bwd_workspace_size(...)
+ *              bytes, 256-byte aligned; kda_workspace_status reads its status.
+ * Outputs must not alias inputs.  Nothing is allocated or synchronised.
+ */
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
+                         const float* log_alpha, const float* beta,
+                         const float* initial_state, const int32_t* cu_seqlens,
+                         const void* d_o, const float* d_final_state,
+                         int B, int T, int H, int dk, int dv, int num_seqs,
+                         kda_dtype dtype, void* dq, void* dk_out, void* dv_out,
+                         float* dlog_alpha, float* dbeta, float* d_initial_state,
+                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Measurement hook for benchmarks.  When `events` is non-NULL, each later

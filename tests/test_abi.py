@@ -112,3 +112,45 @@ def test_gated_entry_points_validate(lib):
     d = lib.kda_recurrent_step_gated
     assert d(p, p, p, None, p, p, 2, 2, 64, 64, 1, 0, p + (1 << 24), None) == 1
     assert d(p, p, p, p, p, p, 2, 2, 64, 64, 1, 7, p + (1 << 24), None) == 1
+
+
+def _bwd(lib, **over):
+    P = 1 << 20
+    args = dict(q=P, k=P, v=P, la=P, beta=P, s0=None, cu=None, do=P, dsf=None,
+                B=1, T=64, H=1, dk=64, dv=64, N=1, dtype=0, dq=P, dk_=P, dv_=P, dla=P, db=P,
+                ds0=None, ws=P, wsb=1 << 30, stream=None)
+    args.update(over)
+    a = args
+    return lib.kda_chunk_bwd(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["cu"], a["do"],
+                             a["dsf"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["N"], a["dtype"],
+                             a["dq"], a["dk_"], a["dv_"], a["dla"], a["db"], a["ds0"], a["ws"],
+                             a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(dk=96), 2),                 # unsupported head size
+    (dict(dtype=7), 1),               # unknown dtype
+    (dict(do=None), 1),               # null cotangent
+    (dict(la=None), 1),               # the backward takes the per-channel gate
+    (dict(dla=None), 1),              # null gradient output
+    (dict(v=(1 << 20) + 4), 1),       # misaligned
+    (dict(B=2, cu=1 << 20), 1),       # varlen with B != 1
+    (dict(ws=None), 5),               # missing workspace
+    (dict(wsb=16), 5),                # workspace too small
+    (dict(H=0), 1),
+])
+def test_chunk_bwd_rejects(lib, over, status):
+    assert _bwd(lib, **over) == status
+    assert lib.kda_last_error()
+
+
+def test_bwd_workspace_size(lib):
+    f32, bf16 = 0, 1
+    fwd = lib.kda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 4, 0, f32)
+    bwd = lib.kda_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 4, 0, f32)
+    units = 4 * 64 * 16
+    # records + T + two state-sized buffers per (head, chunk) + dU
+    assert bwd >= fwd + units * 4 * (64 * 64 + 2 * 128 * 128 + 64 * 128)
+    # bf16 inputs recompute fp32 records too: same size
+    assert lib.kda_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 4, 0, bf16) == bwd
+    assert lib.kda_chunk_bwd_workspace_size(1, 100, 2, 96, 64, 1, 0, f32) == 0
