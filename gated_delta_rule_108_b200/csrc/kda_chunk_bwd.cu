@@ -35,6 +35,7 @@
 // extra outputs: T from K1 and the state entering every chunk from K2.
 #include "kda_common.cuh"
 #include "kda_launch.h"
+#include "ptx.cuh"
 
 namespace kda {
 namespace {
@@ -54,39 +55,60 @@ struct Rec {
 };
 
 // ------------------------------------------------------------------ KB3 ----
-constexpr int kSlice = 32;   // value columns per CTA
+constexpr int kSlice = 64;   // value columns per CTA
+constexpr int kInterThreads = 256;
 
-template <int DK>
+// Shared memory of KB3.  The record tiles are unpadded copies of the record
+// rows (every access below is a broadcast or along consecutive columns).
+template <typename T, int DK>
 struct BwdInterSmem {
-    static constexpr int LDK = DK + 4;
     float dS[DK][kSlice + 1];
-    float W[kChunk][LDK];
-    float Qt[kChunk][LDK];
-    float Kh[kChunk][LDK];
-    float P[kChunk][kChunk + 4];
-    float D[kChunk][kSlice + 4];
+    float W[kChunk][DK];
+    float Qt[kChunk][DK];
+    float Kh[kChunk][DK];
+    float P[kChunk][kChunk];
     float dU[kChunk][kSlice + 4];
     float gC[DK];
+    T D[2][kChunk][kSlice];   // raw cotangent slice of o, double-buffered
 };
 
+template <typename T>
+__device__ __forceinline__ float4 load4f(const T* p);
+template <>
+__device__ __forceinline__ float4 load4f<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
+template <>
+__device__ __forceinline__ float4 load4f<__nv_bfloat16>(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+// One CTA (8 warps) per (sequence, head, 64-wide value slice), serial over the
+// chunks in reverse.  The loads of chunk n-1 are software-pipelined with the
+// work of chunk n: K^, P and the cotangent slice are fetched (cp.async) as soon
+// as step 1 of chunk n is done with them, Q~, W and gamma as soon as step 2 is.
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kInterThreads, 1)
 bwd_inter_kernel(const T* __restrict__ d_o, const float* __restrict__ d_final_state,
                  float* __restrict__ d_initial_state, float* __restrict__ dS_end, float* __restrict__ dU_all,
                  ChunkMap map, const WsHeader* __restrict__ hdr, const float* __restrict__ records,
                  int H, size_t max_chunks, float scale)
 {
     using R = Rec<DK, DV>;
-    using Sm = BwdInterSmem<DK>;
+    using Sm = BwdInterSmem<T, DK>;
+    constexpr int NT = kInterThreads;
+    constexpr int CPT = kSlice * DK / NT;   // step-2 columns per thread
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Sm& sm = *reinterpret_cast<Sm*>(smem_raw);
 
     if (hdr->status != kStatusOk) return;
     const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSlice;
-    const int tid = threadIdx.x, lane = tid & 31, ry = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
     const size_t state_off = ((size_t)s * H + h) * DK * DV;
 
-    for (int idx = tid; idx < DK * kSlice; idx += 128) {
+    for (int idx = tid; idx < DK * kSlice; idx += NT) {
         const int r = idx / kSlice, j = idx - r * kSlice;
         sm.dS[r][j] = d_final_state ? d_final_state[state_off + (size_t)r * DV + j0 + j] : 0.f;
     }
@@ -94,76 +116,107 @@ bwd_inter_kernel(const T* __restrict__ d_o, const float* __restrict__ d_final_st
     const int nch = map.seq_num_chunks(s);
     const int tok_begin = map.seq_token_begin(s), tok_end = map.seq_token_end(s);
 
+    auto issue_a = [&](int n) {   // K^, P, cotangent slice of chunk n
+        const float* rec = records + ((size_t)h * max_chunks + first + n) * R::FLOATS;
+        for (int e = tid; e < kChunk * DK / 4; e += NT) ptx::cp_async16(&sm.Kh[0][0] + 4 * e, rec + R::KH + 4 * e);
+        for (int e = tid; e < kChunk * kChunk / 4; e += NT) ptx::cp_async16(&sm.P[0][0] + 4 * e, rec + R::P + 4 * e);
+        constexpr int EPP = 16 / (int)sizeof(T);   // elements per 16-byte piece
+        constexpr int PPR = kSlice / EPP;          // pieces per row
+        const int tok0 = tok_begin + n * kChunk;
+        for (int e = tid; e < kChunk * PPR; e += NT) {
+            const int r = e / PPR, pc = e - r * PPR;
+            const bool live = tok0 + r < tok_end;   // rows past the sequence are zero-filled
+            const T* src = d_o + ((size_t)(live ? tok0 + r : tok0) * H + h) * DV + j0 + pc * EPP;
+            ptx::cp_async16(&sm.D[n & 1][r][pc * EPP], src, live ? 16u : 0u);
+        }
+    };
+    auto issue_b = [&](int n) {   // Q~, W, gamma of chunk n
+        const float* rec = records + ((size_t)h * max_chunks + first + n) * R::FLOATS;
+        for (int e = tid; e < kChunk * DK / 4; e += NT) {
+            ptx::cp_async16(&sm.Qt[0][0] + 4 * e, rec + R::QT + 4 * e);
+            ptx::cp_async16(&sm.W[0][0] + 4 * e, rec + R::W + 4 * e);
+        }
+        for (int e = tid; e < DK / 4; e += NT) ptx::cp_async16(&sm.gC[0] + 4 * e, rec + R::GC + 4 * e);
+    };
+
+    if (nch > 0) {
+        issue_a(nch - 1);
+        ptx::cp_async_commit();
+        issue_b(nch - 1);
+        ptx::cp_async_commit();
+    }
     for (int n = nch - 1; n >= 0; --n) {
         const size_t item = (size_t)h * max_chunks + first + n;
-        const float* rec = records + item * R::FLOATS;
-        __syncthreads();   // dS of the chunk after this one is complete
+        const int buf = n & 1;
+        ptx::cp_async_wait<1>();   // this thread's part of K^, P, D of chunk n has landed
+        __syncthreads();           // everyone's; dS of the chunk after this one is complete
         {
             float* out = dS_end + item * DK * DV;
-            for (int idx = tid; idx < DK * kSlice; idx += 128) {
+            for (int idx = tid; idx < DK * kSlice; idx += NT) {
                 const int r = idx / kSlice, j = idx - r * kSlice;
                 out[(size_t)r * DV + j0 + j] = sm.dS[r][j];
             }
         }
-        for (int idx = tid; idx < kChunk * DK / 4; idx += 128) {
-            const int r = idx / (DK / 4), c4 = (idx - r * (DK / 4)) * 4;
-            *reinterpret_cast<float4*>(&sm.W[r][c4]) = *reinterpret_cast<const float4*>(rec + R::W + (size_t)r * DK + c4);
-            *reinterpret_cast<float4*>(&sm.Qt[r][c4]) = *reinterpret_cast<const float4*>(rec + R::QT + (size_t)r * DK + c4);
-            *reinterpret_cast<float4*>(&sm.Kh[r][c4]) = *reinterpret_cast<const float4*>(rec + R::KH + (size_t)r * DK + c4);
-        }
-        for (int idx = tid; idx < kChunk * kChunk / 4; idx += 128) {
-            const int r = idx >> 4, c4 = (idx & 15) * 4;
-            *reinterpret_cast<float4*>(&sm.P[r][c4]) = *reinterpret_cast<const float4*>(rec + R::P + (size_t)r * kChunk + c4);
-        }
-        const int tok0 = tok_begin + n * kChunk;
-        for (int idx = tid; idx < kChunk * kSlice; idx += 128) {
-            const int r = idx / kSlice, j = idx - r * kSlice;
-            const int tok = tok0 + r;
-            sm.D[r][j] = tok < tok_end ? scale * to_f32(d_o[((size_t)tok * H + h) * DV + j0 + j]) : 0.f;
-        }
-        for (int idx = tid; idx < DK; idx += 128) sm.gC[idx] = rec[R::GC + idx];
-        __syncthreads();
 
-        // 1. dU = P^T D + K^ dS' for rows r = ry + 4a, column j = lane
-        float acc[16];
+        // 1. dU = P^T D + K^ dS' for rows r = wp + 8a, columns lane and lane + 32
+        float acc[8][2];
 #pragma unroll
-        for (int a = 0; a < 16; ++a) acc[a] = 0.f;
+        for (int a = 0; a < 8; ++a) { acc[a][0] = 0.f; acc[a][1] = 0.f; }
         for (int c = 0; c < DK; c += 4) {
-            const float s0 = sm.dS[c][lane], s1 = sm.dS[c + 1][lane];
-            const float s2 = sm.dS[c + 2][lane], s3 = sm.dS[c + 3][lane];
+            float s0[4], s1[4];
 #pragma unroll
-            for (int a = 0; a < 16; ++a) {
-                const float4 kh = *reinterpret_cast<const float4*>(&sm.Kh[ry + 4 * a][c]);
-                acc[a] += kh.x * s0 + kh.y * s1 + kh.z * s2 + kh.w * s3;
+            for (int t = 0; t < 4; ++t) { s0[t] = sm.dS[c + t][lane]; s1[t] = sm.dS[c + t][lane + 32]; }
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const float4 kh = *reinterpret_cast<const float4*>(&sm.Kh[wp + 8 * a][c]);
+                acc[a][0] += kh.x * s0[0] + kh.y * s0[1] + kh.z * s0[2] + kh.w * s0[3];
+                acc[a][1] += kh.x * s1[0] + kh.y * s1[1] + kh.z * s1[2] + kh.w * s1[3];
             }
         }
         for (int i = 0; i < kChunk; ++i) {
-            const float d = sm.D[i][lane];
+            const float d0 = scale * to_f32(sm.D[buf][i][lane]);
+            const float d1 = scale * to_f32(sm.D[buf][i][lane + 32]);
 #pragma unroll
-            for (int a = 0; a < 16; ++a) acc[a] = fmaf(sm.P[i][ry + 4 * a], d, acc[a]);
+            for (int a = 0; a < 8; ++a) {
+                const float p = sm.P[i][wp + 8 * a];
+                acc[a][0] = fmaf(p, d0, acc[a][0]);
+                acc[a][1] = fmaf(p, d1, acc[a][1]);
+            }
         }
         {
             float* out = dU_all + item * kChunk * DV;
 #pragma unroll
-            for (int a = 0; a < 16; ++a) {
-                sm.dU[ry + 4 * a][lane] = acc[a];
-                out[(size_t)(ry + 4 * a) * DV + j0 + lane] = acc[a];
+            for (int a = 0; a < 8; ++a) {
+                const int r = wp + 8 * a;
+                sm.dU[r][lane] = acc[a][0];
+                sm.dU[r][lane + 32] = acc[a][1];
+                out[(size_t)r * DV + j0 + lane] = acc[a][0];
+                out[(size_t)r * DV + j0 + lane + 32] = acc[a][1];
             }
+        }
+        __syncthreads();   // K^ and P are free, dU is complete
+        if (n > 0) {
+            issue_a(n - 1);
+            ptx::cp_async_commit();
+            ptx::cp_async_wait<1>();   // Q~, W, gamma of chunk n have landed
+        } else {
+            ptx::cp_async_wait<0>();
         }
         __syncthreads();
 
-        // 2. dS = Diag(gamma) dS' + Q~^T D - W^T dU, one key row per thread
-        for (int c = tid; c < DK; c += 128) {
-            float x[kSlice];
+        // 2. dS = Diag(gamma) dS' + Q~^T D - W^T dU: key row c, CPT columns from jb
+        {
+            const int c = tid % DK, jb = (tid / DK) * CPT;
+            float x[CPT];
             const float gc = sm.gC[c];
 #pragma unroll
-            for (int j = 0; j < kSlice; ++j) x[j] = gc * sm.dS[c][j];
+            for (int j = 0; j < CPT; ++j) x[j] = gc * sm.dS[c][jb + j];
             for (int r = 0; r < kChunk; ++r) {
-                const float qt = sm.Qt[r][c], w = sm.W[r][c];
+                const float qt = scale * sm.Qt[r][c], w = sm.W[r][c];
 #pragma unroll
-                for (int j = 0; j < kSlice; j += 4) {
-                    const float4 d = *reinterpret_cast<const float4*>(&sm.D[r][j]);
-                    const float4 u = *reinterpret_cast<const float4*>(&sm.dU[r][j]);
+                for (int j = 0; j < CPT; j += 4) {
+                    const float4 d = load4f<T>(&sm.D[buf][r][jb + j]);
+                    const float4 u = *reinterpret_cast<const float4*>(&sm.dU[r][jb + j]);
                     x[j] += qt * d.x - w * u.x;
                     x[j + 1] += qt * d.y - w * u.y;
                     x[j + 2] += qt * d.z - w * u.z;
@@ -171,12 +224,17 @@ bwd_inter_kernel(const T* __restrict__ d_o, const float* __restrict__ d_final_st
                 }
             }
 #pragma unroll
-            for (int j = 0; j < kSlice; ++j) sm.dS[c][j] = x[j];
+            for (int j = 0; j < CPT; ++j) sm.dS[c][jb + j] = x[j];   // this thread's own segment
+        }
+        __syncthreads();   // Q~, W and this chunk's D are free
+        if (n > 0) {
+            issue_b(n - 1);
+            ptx::cp_async_commit();
         }
     }
     __syncthreads();
     if (d_initial_state) {
-        for (int idx = tid; idx < DK * kSlice; idx += 128) {
+        for (int idx = tid; idx < DK * kSlice; idx += NT) {
             const int r = idx / kSlice, j = idx - r * kSlice;
             d_initial_state[state_off + (size_t)r * DV + j0 + j] = sm.dS[r][j];
         }
@@ -214,23 +272,61 @@ __device__ __forceinline__ void zero_acc(float (&acc)[4][N / 16]) {
         for (int j = 0; j < N / 16; ++j) acc[i][j] = 0.f;
 }
 
-// acc += A(64 x K) B(K x N)
+// acc += A(64 x K) B(K x N).  Each K-slab is read with 16-byte loads along the
+// stored matrix's contiguous dimension into registers one slab ahead, so the
+// L2 latency of slab s+1 overlaps the products of slab s; the stage holds the
+// slab as a[k][m] and b[k][n] whatever the stored orientation.
 template <int N>
 __device__ void gemm64(float (&acc)[4][N / 16], Mat A, Mat B, int K, GemmStage& st) {
+    constexpr int A4 = 64 * kSlab / 4 / 256;   // float4s of the A slab per thread
+    constexpr int B4 = N * kSlab / 4 / 256;
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+    float4 ra[A4], rb[B4];
+    auto load = [&](int k0) {
+#pragma unroll
+        for (int i = 0; i < A4; ++i) {
+            const int e = tid + 256 * i;
+            ra[i] = A.t ? *reinterpret_cast<const float4*>(A.p + (size_t)(k0 + (e >> 4)) * A.ld + (e & 15) * 4)
+                        : *reinterpret_cast<const float4*>(A.p + (size_t)(e >> 3) * A.ld + k0 + (e & 7) * 4);
+        }
+#pragma unroll
+        for (int i = 0; i < B4; ++i) {
+            const int e = tid + 256 * i;
+            rb[i] = B.t ? *reinterpret_cast<const float4*>(B.p + (size_t)(e >> 3) * B.ld + k0 + (e & 7) * 4)
+                        : *reinterpret_cast<const float4*>(B.p + (size_t)(k0 + e / (N / 4)) * B.ld + (e % (N / 4)) * 4);
+        }
+    };
+    auto store = [&]() {
+#pragma unroll
+        for (int i = 0; i < A4; ++i) {
+            const int e = tid + 256 * i;
+            if (A.t) {
+                *reinterpret_cast<float4*>(&st.a[e >> 4][(e & 15) * 4]) = ra[i];
+            } else {
+                const int m = e >> 3, k4 = (e & 7) * 4;
+                st.a[k4][m] = ra[i].x; st.a[k4 + 1][m] = ra[i].y;
+                st.a[k4 + 2][m] = ra[i].z; st.a[k4 + 3][m] = ra[i].w;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < B4; ++i) {
+            const int e = tid + 256 * i;
+            if (B.t) {
+                const int n = e >> 3, k4 = (e & 7) * 4;
+                st.b[k4][n] = rb[i].x; st.b[k4 + 1][n] = rb[i].y;
+                st.b[k4 + 2][n] = rb[i].z; st.b[k4 + 3][n] = rb[i].w;
+            } else {
+                *reinterpret_cast<float4*>(&st.b[e / (N / 4)][(e % (N / 4)) * 4]) = rb[i];
+            }
+        }
+    };
+    __syncthreads();   // operands written by earlier epilogues are complete
+    load(0);
     for (int k0 = 0; k0 < K; k0 += kSlab) {
-        __syncthreads();   // earlier readers of the stage / writers of the operands are done
-        for (int e = tid; e < 64 * kSlab; e += 256) {
-            int m, kk;
-            if (A.t) { kk = e >> 6; m = e & 63; } else { m = e / kSlab; kk = e % kSlab; }
-            st.a[kk][m] = A.at(m, k0 + kk);
-        }
-        for (int e = tid; e < N * kSlab; e += 256) {
-            int n, kk;
-            if (B.t) { n = e / kSlab; kk = e % kSlab; } else { kk = e / N; n = e % N; }
-            st.b[kk][n] = B.at(k0 + kk, n);
-        }
+        __syncthreads();   // earlier readers of the stage are done
+        store();
         __syncthreads();
+        if (k0 + kSlab < K) load(k0 + kSlab);
 #pragma unroll 4
         for (int kk = 0; kk < kSlab; ++kk) {
             const float4 av = *reinterpret_cast<const float4*>(&st.a[kk][ty * 4]);
@@ -358,6 +454,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         const bool strong = __syncthreads_or(wide);
 
         // ---- operands into scratch ------------------------------------------
+#pragma unroll 4
         for (int idx = tid; idx < kChunk * DK; idx += 256) {
             const int r = idx / DK, ch = idx - r * DK;
             float kk = 0.f, qq = 0.f;
@@ -378,6 +475,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             }
             scr[C::KT + idx] = kk * expf(gg);
         }
+#pragma unroll 4
         for (int idx = tid; idx < kChunk * DV; idx += 256) {
             const int r = idx / DV, j = idx - r * DV;
             const size_t off = (size_t)(tok0 + r) * rowv + (size_t)h * DV + j;
@@ -554,6 +652,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         __syncthreads();
 
         // ---- dq, dk, dg -------------------------------------------------------
+#pragma unroll 4
         for (int idx = tid; idx < kChunk * DK; idx += 256) {
             const int r = idx / DK, ch = idx - r * DK;
             float kk = 0.f, qq = 0.f;
@@ -593,11 +692,11 @@ template <typename T, int DK, int DV>
 cudaError_t launch_bwd_inter_t(const ChunkArgs& a) {
     ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
     auto kern = bwd_inter_kernel<T, DK, DV>;
-    const int smem = (int)sizeof(BwdInterSmem<DK>);
+    const int smem = (int)sizeof(BwdInterSmem<T, DK>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.num_seqs, (unsigned)a.H, (unsigned)(DV / kSlice));
-    kern<<<grid, 128, smem, a.stream>>>(static_cast<const T*>(a.d_o), a.d_final_state, a.d_initial_state,
+    kern<<<grid, kInterThreads, smem, a.stream>>>(static_cast<const T*>(a.d_o), a.d_final_state, a.d_initial_state,
                                          a.dS_end, a.dU, map, static_cast<const WsHeader*>(a.ws_header),
                                          static_cast<const float*>(a.records), a.H, a.max_chunks, a.scale);
     return cudaGetLastError();

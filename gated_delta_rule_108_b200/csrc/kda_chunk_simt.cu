@@ -7,7 +7,7 @@
 //   K0 chunk_prep   -- resets the workspace status; for packed sequences it
 //                      checks cu_seqlens and builds the chunk table.
 //   K1 intra_chunk  -- one CTA per (chunk, head), all chunks in parallel.
-//   K2 inter_chunk  -- one CTA per (sequence, head, 32-wide value slice),
+//   K2 inter_chunk  -- one CTA per (sequence, head, 64-wide value slice),
 //                      serial over the sequence's chunks, state in shared memory.
 //
 // Chunk algebra (derived by unrolling the update equation of the daiw.net page,
@@ -25,6 +25,7 @@
 // unchanged).  T is formed by forward substitution, one column per thread.
 #include "kda_common.cuh"
 #include "kda_launch.h"
+#include "ptx.cuh"
 
 namespace kda {
 namespace {
@@ -327,23 +328,29 @@ intra_chunk_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const 
 }
 
 // ---------------------------------------------------------------- K2 ------
-constexpr int kSlice = 32;  // value columns per inter-chunk CTA
+constexpr int kSlice = 64;  // value columns per inter-chunk CTA
+constexpr int kInterThreads = 256;
 
+// Shared memory of K2.  The record tiles are unpadded copies of the record
+// rows: every access below is a warp broadcast or along consecutive columns.
 template <int DK>
 struct InterSmem {
-    static constexpr int LDK = DK + 4;
     float S[DK][kSlice + 1];
-    float W[kChunk][LDK];
-    float Qt[kChunk][LDK];
-    float Kh[kChunk][LDK];
-    float P[kChunk][kChunk + 4];
-    float U0[kChunk][kSlice + 1];
+    float W[kChunk][DK];
+    float Qt[kChunk][DK];
+    float Kh[kChunk][DK];
+    float P[kChunk][kChunk];
+    float U0[kChunk][kSlice];
     float U[kChunk][kSlice + 4];
     float gC[DK];
 };
 
+// One CTA (8 warps) per (sequence, head, 64-wide value slice), serial over the
+// chunks.  The loads of chunk n+1 are software-pipelined with the work of
+// chunk n: W, Q~ and the U0 slice are fetched (cp.async) once step 1 of chunk n
+// is done with them, P, K^ and gamma once steps 2 and 3 are.
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kInterThreads, 1)
 inter_chunk_simt_kernel(const float* __restrict__ initial_state, float* __restrict__ final_state,
                         T* __restrict__ o, float* __restrict__ states, ChunkMap map,
                         const WsHeader* __restrict__ hdr, const float* __restrict__ records, int H,
@@ -351,15 +358,17 @@ inter_chunk_simt_kernel(const float* __restrict__ initial_state, float* __restri
 {
     using R = SimtRec<DK, DV>;
     using Sm = InterSmem<DK>;
+    constexpr int NT = kInterThreads;
+    constexpr int CPT = kSlice * DK / NT;   // step-3 columns per thread
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Sm& sm = *reinterpret_cast<Sm*>(smem_raw);
 
     if (hdr->status != kStatusOk) return;
     const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSlice;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
     const size_t state_off = ((size_t)s * H + h) * DK * DV;
 
-    for (int idx = tid; idx < DK * kSlice; idx += 128) {
+    for (int idx = tid; idx < DK * kSlice; idx += NT) {
         const int r = idx / kSlice, j = idx - r * kSlice;
         sm.S[r][j] = initial_state ? initial_state[state_off + (size_t)r * DV + j0 + j] : 0.f;
     }
@@ -368,95 +377,128 @@ inter_chunk_simt_kernel(const float* __restrict__ initial_state, float* __restri
     const int nch = map.seq_num_chunks(s);
     const int tok_begin = map.seq_token_begin(s), tok_end = map.seq_token_end(s);
 
-    for (int n = 0; n < nch; ++n) {
+    auto issue_a = [&](int n) {   // W, Q~, U0 slice of chunk n
         const float* rec = records + ((size_t)h * max_chunks + first + n) * R::FLOATS;
-        __syncthreads();  // previous chunk done with shared buffers
-        for (int idx = tid; idx < kChunk * DK / 4; idx += 128) {
-            const int r = idx / (DK / 4), c4 = (idx - r * (DK / 4)) * 4;
-            *reinterpret_cast<float4*>(&sm.W[r][c4]) = *reinterpret_cast<const float4*>(rec + R::W + (size_t)r * DK + c4);
-            *reinterpret_cast<float4*>(&sm.Qt[r][c4]) = *reinterpret_cast<const float4*>(rec + R::QT + (size_t)r * DK + c4);
-            *reinterpret_cast<float4*>(&sm.Kh[r][c4]) = *reinterpret_cast<const float4*>(rec + R::KH + (size_t)r * DK + c4);
+        for (int e = tid; e < kChunk * DK / 4; e += NT) {
+            ptx::cp_async16(&sm.W[0][0] + 4 * e, rec + R::W + 4 * e);
+            ptx::cp_async16(&sm.Qt[0][0] + 4 * e, rec + R::QT + 4 * e);
         }
-        for (int idx = tid; idx < kChunk * kChunk / 4; idx += 128) {
-            const int r = idx >> 4, c4 = (idx & 15) * 4;
-            *reinterpret_cast<float4*>(&sm.P[r][c4]) = *reinterpret_cast<const float4*>(rec + R::P + (size_t)r * kChunk + c4);
+        for (int e = tid; e < kChunk * kSlice / 4; e += NT) {
+            const int r = e / (kSlice / 4), c4 = (e - r * (kSlice / 4)) * 4;
+            ptx::cp_async16(&sm.U0[r][c4], rec + R::U0 + (size_t)r * DV + j0 + c4);
         }
-        for (int idx = tid; idx < kChunk * kSlice; idx += 128) {
-            const int r = idx / kSlice, j = idx - r * kSlice;
-            sm.U0[r][j] = rec[R::U0 + (size_t)r * DV + j0 + j];
-        }
-        for (int idx = tid; idx < DK; idx += 128) sm.gC[idx] = rec[R::GC + idx];
+    };
+    auto issue_b = [&](int n) {   // P, K^, gamma of chunk n
+        const float* rec = records + ((size_t)h * max_chunks + first + n) * R::FLOATS;
+        for (int e = tid; e < kChunk * DK / 4; e += NT) ptx::cp_async16(&sm.Kh[0][0] + 4 * e, rec + R::KH + 4 * e);
+        for (int e = tid; e < kChunk * kChunk / 4; e += NT) ptx::cp_async16(&sm.P[0][0] + 4 * e, rec + R::P + 4 * e);
+        for (int e = tid; e < DK / 4; e += NT) ptx::cp_async16(&sm.gC[0] + 4 * e, rec + R::GC + 4 * e);
+    };
+
+    if (nch > 0) {
+        issue_a(0);
+        ptx::cp_async_commit();
+        issue_b(0);
+        ptx::cp_async_commit();
+    }
+    for (int n = 0; n < nch; ++n) {
+        ptx::cp_async_wait<1>();   // this thread's part of W, Q~, U0 of chunk n has landed
+        __syncthreads();           // everyone's; S of the previous chunk is complete
         if (states) {   // the state entering this chunk, for the backward pass
             float* st = states + ((size_t)h * max_chunks + first + n) * DK * DV;
-            for (int idx = tid; idx < DK * kSlice; idx += 128) {
+            for (int idx = tid; idx < DK * kSlice; idx += NT) {
                 const int r = idx / kSlice, j = idx - r * kSlice;
                 st[(size_t)r * DV + j0 + j] = sm.S[r][j];
             }
         }
-        __syncthreads();
 
-        // 1. W S and Q~ S for rows r = ry + 4a, column j = lane
-        const int lane = tid & 31, ry = tid >> 5;
-        float ws[16], qs[16];
+        // 1. W S and Q~ S for rows r = wp + 8a, columns lane and lane + 32
+        float ws[8][2], qs[8][2];
 #pragma unroll
-        for (int a = 0; a < 16; ++a) { ws[a] = 0.f; qs[a] = 0.f; }
+        for (int a = 0; a < 8; ++a) { ws[a][0] = ws[a][1] = qs[a][0] = qs[a][1] = 0.f; }
         for (int c = 0; c < DK; c += 4) {
-            const float s0 = sm.S[c][lane], s1 = sm.S[c + 1][lane];
-            const float s2 = sm.S[c + 2][lane], s3 = sm.S[c + 3][lane];
+            float s0[4], s1[4];
 #pragma unroll
-            for (int a = 0; a < 16; ++a) {
-                const float4 w = *reinterpret_cast<const float4*>(&sm.W[ry + 4 * a][c]);
-                const float4 qv = *reinterpret_cast<const float4*>(&sm.Qt[ry + 4 * a][c]);
-                ws[a] += w.x * s0 + w.y * s1 + w.z * s2 + w.w * s3;
-                qs[a] += qv.x * s0 + qv.y * s1 + qv.z * s2 + qv.w * s3;
+            for (int t = 0; t < 4; ++t) { s0[t] = sm.S[c + t][lane]; s1[t] = sm.S[c + t][lane + 32]; }
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const float4 w = *reinterpret_cast<const float4*>(&sm.W[wp + 8 * a][c]);
+                const float4 qv = *reinterpret_cast<const float4*>(&sm.Qt[wp + 8 * a][c]);
+                ws[a][0] += w.x * s0[0] + w.y * s0[1] + w.z * s0[2] + w.w * s0[3];
+                ws[a][1] += w.x * s1[0] + w.y * s1[1] + w.z * s1[2] + w.w * s1[3];
+                qs[a][0] += qv.x * s0[0] + qv.y * s0[1] + qv.z * s0[2] + qv.w * s0[3];
+                qs[a][1] += qv.x * s1[0] + qv.y * s1[1] + qv.z * s1[2] + qv.w * s1[3];
             }
         }
 #pragma unroll
-        for (int a = 0; a < 16; ++a) sm.U[ry + 4 * a][lane] = sm.U0[ry + 4 * a][lane] - ws[a];
+        for (int a = 0; a < 8; ++a) {
+            const int r = wp + 8 * a;
+            sm.U[r][lane] = sm.U0[r][lane] - ws[a][0];
+            sm.U[r][lane + 32] = sm.U0[r][lane + 32] - ws[a][1];
+        }
+        __syncthreads();   // W, Q~, U0 are free; U is complete
+        if (n + 1 < nch) {
+            issue_a(n + 1);
+            ptx::cp_async_commit();
+            ptx::cp_async_wait<1>();   // P, K^, gamma of chunk n have landed
+        } else {
+            ptx::cp_async_wait<0>();
+        }
         __syncthreads();
 
         // 2. O = scale (Q~ S + P U)
         if (o) {
-        for (int i = 0; i < kChunk; i += 4) {
-            const float u0 = sm.U[i][lane], u1 = sm.U[i + 1][lane];
-            const float u2 = sm.U[i + 2][lane], u3 = sm.U[i + 3][lane];
+            for (int i = 0; i < kChunk; i += 4) {
+                float u0[4], u1[4];
 #pragma unroll
-            for (int a = 0; a < 16; ++a) {
-                const float4 p = *reinterpret_cast<const float4*>(&sm.P[ry + 4 * a][i]);
-                qs[a] += p.x * u0 + p.y * u1 + p.z * u2 + p.w * u3;
+                for (int t = 0; t < 4; ++t) { u0[t] = sm.U[i + t][lane]; u1[t] = sm.U[i + t][lane + 32]; }
+#pragma unroll
+                for (int a = 0; a < 8; ++a) {
+                    const float4 p = *reinterpret_cast<const float4*>(&sm.P[wp + 8 * a][i]);
+                    qs[a][0] += p.x * u0[0] + p.y * u0[1] + p.z * u0[2] + p.w * u0[3];
+                    qs[a][1] += p.x * u1[0] + p.y * u1[1] + p.z * u1[2] + p.w * u1[3];
+                }
+            }
+            const int chunk_tok0 = tok_begin + n * kChunk;
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const int tok = chunk_tok0 + wp + 8 * a;
+                if (tok < tok_end) {
+                    T* orow = o + ((size_t)tok * H + h) * DV + j0;
+                    orow[lane] = from_f32<T>(scale * qs[a][0]);
+                    orow[lane + 32] = from_f32<T>(scale * qs[a][1]);
+                }
             }
         }
-        const int chunk_tok0 = tok_begin + n * kChunk;
-#pragma unroll
-        for (int a = 0; a < 16; ++a) {
-            const int tok = chunk_tok0 + ry + 4 * a;
-            if (tok < tok_end)
-                o[((size_t)tok * H + h) * DV + j0 + lane] = from_f32<T>(scale * qs[a]);
-        }
-        }  // o
 
-        // 3. S' = Diag(gC) S + K^^T U, one key row per thread
-        if (tid < DK) {
-            float acc[kSlice];
-            const float gc = sm.gC[tid];
+        // 3. S' = Diag(gC) S + K^^T U: key row c, CPT columns from jb
+        {
+            const int c = tid % DK, jb = (tid / DK) * CPT;
+            float acc[CPT];
+            const float gc = sm.gC[c];
 #pragma unroll
-            for (int j = 0; j < kSlice; ++j) acc[j] = gc * sm.S[tid][j];
+            for (int j = 0; j < CPT; ++j) acc[j] = gc * sm.S[c][jb + j];
             for (int r = 0; r < kChunk; ++r) {
-                const float kh = sm.Kh[r][tid];
+                const float kh = sm.Kh[r][c];
 #pragma unroll
-                for (int j = 0; j < kSlice; j += 4) {
-                    const float4 u = *reinterpret_cast<const float4*>(&sm.U[r][j]);
+                for (int j = 0; j < CPT; j += 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(&sm.U[r][jb + j]);
                     acc[j] += kh * u.x; acc[j + 1] += kh * u.y;
                     acc[j + 2] += kh * u.z; acc[j + 3] += kh * u.w;
                 }
             }
 #pragma unroll
-            for (int j = 0; j < kSlice; ++j) sm.S[tid][j] = acc[j];
+            for (int j = 0; j < CPT; ++j) sm.S[c][jb + j] = acc[j];   // this thread's own segment
+        }
+        __syncthreads();   // P, K^, gamma are free
+        if (n + 1 < nch) {
+            issue_b(n + 1);
+            ptx::cp_async_commit();
         }
     }
     __syncthreads();
     if (final_state) {
-        for (int idx = tid; idx < DK * kSlice; idx += 128) {
+        for (int idx = tid; idx < DK * kSlice; idx += NT) {
             const int r = idx / kSlice, j = idx - r * kSlice;
             final_state[state_off + (size_t)r * DV + j0 + j] = sm.S[r][j];
         }
@@ -487,7 +529,7 @@ cudaError_t launch_inter_t(const ChunkArgs& a) {
     cudaError_t e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.num_seqs, (unsigned)a.H, (unsigned)(DV / kSlice));
-    k2<<<grid, 128, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<T*>(a.o), a.states, map,
+    k2<<<grid, kInterThreads, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<T*>(a.o), a.states, map,
                                        static_cast<const WsHeader*>(a.ws_header),
                                        static_cast<const float*>(a.records), a.H, a.max_chunks,
                                        a.scale);

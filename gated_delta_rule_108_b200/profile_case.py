@@ -2,6 +2,7 @@
 
     python -m gated_delta_rule_108_b200.profile_case decode --B 96 --H 32 --launches 3
     python -m gated_delta_rule_108_b200.profile_case chunk --B 1 --T 8192 --H 16 --launches 3
+    python -m gated_delta_rule_108_b200.profile_case chunk_bwd --B 4 --T 4096 --H 16 --launches 2
 
 Inputs are seeded synthetic data (gated_delta_rule_108_b200.inputs); each
 launch is one library call; the process synchronises and exits 0 on success.
@@ -18,7 +19,7 @@ from . import kda
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["decode", "chunk"])
+    ap.add_argument("what", choices=["decode", "chunk", "chunk_bwd"])
     ap.add_argument("--B", type=int, default=96)
     ap.add_argument("--T", type=int, default=8192)
     ap.add_argument("--H", type=int, default=32)
@@ -36,8 +37,14 @@ def main():
     else:
         w = I.ChunkWorkload("profile", B=a.B, T=a.T, H=a.H, dk=a.d, dv=a.d, dtype=dt, s0_std=0.01, seed=7)
         x = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in I.chunk_inputs(w).items()}
-        for _ in range(a.launches):
-            kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
+        if a.what == "chunk":
+            for _ in range(a.launches):
+                kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
+        else:
+            g = torch.Generator().manual_seed(8)
+            d_o = torch.randn(x["v"].shape, generator=g).to(dt).cuda()
+            for _ in range(a.launches):
+                kda.chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], d_o, x["initial_state"])
     torch.cuda.synchronize()
     print(f"{a.what}: {a.launches} launches ok")
 
