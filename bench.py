@@ -44,6 +44,9 @@ if ROOT not in sys.path:
 import torch  # noqa: E402
 
 METRIC = "KDA tokens/s (chunk fwd & decode) at 1 B200; % bf16 TC peak / % HBM BW"
+# fp32 CUDA-core peak of one B200 from its unit counts and clock: 148 SMs x 128
+# fp32 lanes x 2 flops per FMA x 1.965 GHz (clocks.max.sm)
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # FLOPs per token and head of the chunk forward at MMA tile granularity
 # (d_k = d_v = d, chunk C = 64): 2C(3d_k + 2d_v) + 6 d_k d_v.
@@ -212,6 +215,59 @@ def bench_chunk(args, dev, world, rank):
                 x=x, o=o, S=S, ws=ws)
 
 
+def chunk_bwd_flops_per_chunk_head(dk, dv, C=64):
+    """Multiply-adds of the per-chunk gradient kernel, x2: the value-side
+    products U, dQ~, dW, dK^ (C dk dv each), dP, Z (C C dv), Y, M, dKl, dQl
+    (C C dk), dT (C C (dk + dv)), dKr (2 C C dk), dT T^T and T^T X (C^3)."""
+    return 2 * (4 * C * dk * dv + C * C * (3 * dv + 7 * dk) + 2 * C ** 3)
+
+
+def bench_backward(args, dev, world, rank):
+    """kda_chunk_bwd on the forward's workload, a seeded d_o and d_final_state."""
+    from gated_delta_rule_108_b200 import inputs as I
+    from gated_delta_rule_108_b200 import kda
+
+    w = I.workload(args.workload)
+    wr = I.ChunkWorkload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    x = I.chunk_inputs(wr)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    gen = torch.Generator().manual_seed(5000 + rank)
+    d_o = torch.randn(w.B, w.T, w.H, w.dv, generator=gen).to(w.dtype).to(dev)
+    dSf = torch.randn(w.B, w.H, w.dk, w.dv, generator=gen).to(dev)
+    ws = torch.empty(kda.chunk_bwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.B, False, w.dtype),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.chunk_bwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], d_o, g["initial_state"], dSf,
+                      workspace=ws)
+
+    steps = args.bwd_steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    for evs in ev:
+        for e in evs:
+            e.record()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if kda.workspace_status(ws) != 0:
+        raise RuntimeError("device status set after the backward warm-up")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(steps):
+        kda.set_stage_events(ev[i])
+        step()
+    end.record()
+    kda.set_stage_events(None)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end), world, dev) / steps
+    names = ("chunk_prep", "fwd_intra_chunk", "fwd_inter_chunk", "bwd_inter_chunk", "bwd_intra_chunk")
+    stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i, n in enumerate(names)}
+    return dict(w=w, ms_per_step=ms, stages=stages, launches=5 * steps)
+
+
 def bench_decode(args, dev, world, rank):
     from gated_delta_rule_108_b200 import inputs as I
     from gated_delta_rule_108_b200 import kda
@@ -305,6 +361,7 @@ def run_ours(args):
     clocks.start()
     res = bench_chunk(args, dev, world, rank)
     dec = None if args.no_decode else bench_decode(args, dev, world, rank)
+    bwd = None if args.no_bwd else bench_backward(args, dev, world, rank)
     clk = clocks.stop()
     e2e = None if args.no_e2e else bench_e2e(args, dev, world, res)
 
@@ -384,6 +441,24 @@ def run_ours(args):
                          "unit": "GB/s", "frac": dgbs / hbm, "traffic": traffic_for("decode_step"),
                          "algorithmic_bytes_per_launch": dbytes},
         }
+    if bwd is not None:
+        bw = bwd["w"]
+        n_ch = bw.num_seqs * ((bw.T + 63) // 64) * bw.H
+        bflops = chunk_bwd_flops_per_chunk_head(bw.dk, bw.dv) * n_ch
+        bms = bwd["stages"]["bwd_intra_chunk"]
+        btf = bflops / (bms / 1e3) / 1e12
+        alu_peak = FP32_SIMT_TFLOPS
+        line["chunk_bwd"] = {
+            "workload": f"{bw.name}: kda_chunk_bwd (dq, dk, dv, dlog_alpha, dbeta, dS0), B={bw.B}, T={bw.T}, "
+                        f"H={bw.H}, d_k=d_v={bw.dk}, bf16 q/k/v/d_o, fp32 arithmetic on CUDA cores",
+            "value": bw.tokens * world / (bwd["ms_per_step"] / 1e3), "unit": "tokens/s",
+            "ms_per_step": bwd["ms_per_step"], "steps": args.bwd_steps, "kernels_ms": bwd["stages"],
+            "gpu_launches": bwd["launches"],
+            "roofline": {"kernel": "bwd_intra_chunk", "bound": "alu", "achieved": btf, "peak": alu_peak,
+                         "unit": "TFLOP/s", "frac": btf / alu_peak, "traffic": traffic_for("bwd_intra_chunk"),
+                         "peak_source": "derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1.965 GHz",
+                         "algorithmic_flops_per_launch": bflops, "ms_per_launch": bms},
+        }
     if e2e is not None:
         ms_e, h2d, d2h = e2e
         line["e2e"] = {"value": res["tokens"] * world / (ms_e / 1e3), "unit": "tokens/s",
@@ -452,6 +527,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--reference-tokens", type=int, default=1024)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward (kda_chunk_bwd) measurement")
+    ap.add_argument("--bwd-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

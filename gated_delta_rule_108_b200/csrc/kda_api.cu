@@ -14,11 +14,12 @@
 namespace {
 
 thread_local std::string g_last_error;
-thread_local cudaEvent_t g_stage_events[4] = {nullptr, nullptr, nullptr, nullptr};
-thread_local bool g_stage_events_on = false;
+constexpr int kMaxStageEvents = 6;
+thread_local cudaEvent_t g_stage_events[kMaxStageEvents] = {};
+thread_local int g_stage_event_count = 0;   // 0: off
 
 cudaError_t mark_stage(int i, cudaStream_t s) {
-    return g_stage_events_on ? cudaEventRecord(g_stage_events[i], s) : cudaSuccess;
+    return i < g_stage_event_count ? cudaEventRecord(g_stage_events[i], s) : cudaSuccess;
 }
 
 kda_status fail(kda_status st, const char* fmt, ...) {
@@ -319,15 +320,23 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const floa
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "device query failed: %s", cudaGetErrorString(e));
-    a.bwd_ctas = L.ctas < 2 * sms ? L.ctas : 2 * sms;
+    a.bwd_ctas = L.ctas < 2 * sms ? L.ctas : 2 * sms;   // two resident per SM
 
     // forward recomputation (fp32 records + T + chunk-start states), then the
     // reversed pass over chunks, then the per-chunk gradients
-    e = kda::launch_chunk_prep(a);
+    const bool marks = g_stage_event_count >= 6;   // the backward records all six or none
+    auto mark = [&](int i) { return marks ? mark_stage(i, a.stream) : cudaSuccess; };
+    e = mark(0);
+    if (e == cudaSuccess) e = kda::launch_chunk_prep(a);
+    if (e == cudaSuccess) e = mark(1);
     if (e == cudaSuccess) e = kda::launch_chunk_intra(a);
+    if (e == cudaSuccess) e = mark(2);
     if (e == cudaSuccess) e = kda::launch_chunk_inter(a);
+    if (e == cudaSuccess) e = mark(3);
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_inter(a);
+    if (e == cudaSuccess) e = mark(4);
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);
+    if (e == cudaSuccess) e = mark(5);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_chunk_bwd launch failed: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -352,15 +361,15 @@ kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes, v
 
 kda_status kda_set_stage_events(void* const* events, int count) {
     if (!events) {
-        g_stage_events_on = false;
+        g_stage_event_count = 0;
         return ok();
     }
     if (count < 4) return fail(KDA_ERR_INVALID_ARG, "need at least 4 events, got %d", count);
-    for (int i = 0; i < 4; ++i) {
+    const int n = count < kMaxStageEvents ? count : kMaxStageEvents;
+    for (int i = 0; i < n; ++i)
         if (!events[i]) return fail(KDA_ERR_INVALID_ARG, "event %d is null", i);
-        g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
-    }
-    g_stage_events_on = true;
+    for (int i = 0; i < n; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+    g_stage_event_count = n;
     return ok();
 }
 

@@ -370,22 +370,25 @@ struct Scr {
     static constexpr size_t KR = KL + kChunk * DK;      // k e^{g_m-g}
     static constexpr size_t QL = KR + kChunk * DK;      // q e^{g-g_m} (strong chunk: raw q)
     static constexpr size_t KT = QL + kChunk * DK;      // K~ = k e^{g}
+    static constexpr int DX = DK > DV ? DK : DV;       // value-side buffers are reused for 64 x DK
     static constexpr size_t VV = KT + kChunk * DK;      // v
-    static constexpr size_t DO = VV + kChunk * DV;      // c dO
-    static constexpr size_t U = DO + kChunk * DV;
-    static constexpr size_t DQT = U + kChunk * DV;
+    static constexpr size_t DO = VV + kChunk * DX;      // c dO
+    static constexpr size_t U = DO + kChunk * DX;
+    static constexpr size_t DQT = U + kChunk * DX;
     static constexpr size_t DKH = DQT + kChunk * DK;
     static constexpr size_t DW = DKH + kChunk * DK;
     static constexpr size_t DKT = DW + kChunk * DK;
     static constexpr size_t DP = DKT + kChunk * DK;
     static constexpr size_t DT = DP + kChunk * kChunk;
-    static constexpr size_t X1 = DT + kChunk * kChunk;
-    static constexpr size_t DM = X1 + kChunk * kChunk;
+    static constexpr size_t X1 = DT;                    // dT T^T overwrites dT (read in full first)
+    static constexpr size_t DM = DT + kChunk * kChunk;
     static constexpr size_t M = DM + kChunk * kChunk;
-    static constexpr size_t DKL = M + kChunk * kChunk;  // dKl e^{g-g_m}
-    static constexpr size_t DQL = DKL + kChunk * DK;    // dQl e^{g-g_m}
-    static constexpr size_t DKR = DQL + kChunk * DK;    // dKr e^{g_m-g}
-    static constexpr size_t FLOATS = DKR + kChunk * DK;
+    static constexpr size_t FLOATS = M + kChunk * kChunk;
+    // the last products reuse buffers that are dead by then (v, D and U are
+    // last read by the dT and dP products)
+    static constexpr size_t DKL = VV;                   // dKl e^{g-g_m}
+    static constexpr size_t DQL = DO;                   // dQl e^{g-g_m}
+    static constexpr size_t DKR = U;                    // dKr e^{g_m-g}
 };
 
 template <int DK>

@@ -232,8 +232,12 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
  * (cudaEvent_t passed as void*) on its stream at the stage boundaries:
  * events[0] before the first kernel, events[1] after the chunk-table/status
  * kernel, events[2] after the intra-chunk stage, events[3] after the
- * inter-chunk stage.  `count` must be >= 4.  Pass NULL to stop.  Recording an
- * event costs a few microseconds of stream time and changes no result.
+ * inter-chunk stage.  With `count` >= 6, each later kda_chunk_bwd records
+ * events[0] before its first kernel and events[1..5] after the chunk-table,
+ * forward intra-chunk, forward inter-chunk, reversed inter-chunk and per-chunk
+ * gradient kernels.  `count` must be >= 4 (only the first 6 are used).  Pass
+ * NULL to stop.  Recording an event costs a few microseconds of stream time
+ * and changes no result.
  */
 kda_status kda_set_stage_events(void* const* events, int count);
 
