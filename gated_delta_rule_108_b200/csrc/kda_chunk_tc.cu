@@ -84,9 +84,14 @@ struct TcRec {
 
 
 constexpr float kMaxSplitExponent = 60.f;   // e^60 ~ 1e26: far inside the fp32 range
+// The intra-chunk kernel keeps the cumulative log-decay in base 2 (g log2(e)),
+// so each factor e^{x} is one hardware 2^{x}.
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kMaxSplitExponent2 = kMaxSplitExponent * kLog2e;
+constexpr int kCopyThread = 32;   // the intra-chunk kernel's TMA / bulk-copy thread (warp 1)
 
 // Exact A and P of one chunk, used when its decay is too strong for the split
-// factors: A_ri = beta_r sum_c k_rc k_ic e^{g_rc - g_ic} (i < r) into am
+// factors (g in base 2): A_ri = beta_r sum_c k_rc k_ic e^{g_rc - g_ic} (i < r) into am
 // [64][68] (zero on and above the diagonal) and P_ri = sum_c q_rc k_ic e^{g_rc - g_ic}
 // (i <= r) as fp16 into the record's P tile.  Every exponent is <= 0.  One warp
 // per (r, i) pair, lanes over channels; k and q are the bf16 tiles as loaded.
@@ -104,7 +109,7 @@ __device__ __forceinline__ void exact_a_p(const float* g, const unsigned char* k
                 const int c = c0 + lane;
                 const uint32_t hr = (c >> 6) * 8192u + sw128_offset(r, (c & 63) * 2);
                 const uint32_t hi = (c >> 6) * 8192u + sw128_offset(i, (c & 63) * 2);
-                const float w = __expf(g[r * DK + c] - g[i * DK + c]);
+                const float w = ex2_approx(g[r * DK + c] - g[i * DK + c]);
                 const float ki = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ks + hi));
                 const float kr = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ks + hr));
                 const float qr = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qs + hr));
@@ -274,7 +279,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
     bool aborted = false;
     uint32_t mma_phase = 0;
     int mma_pending = 0;      // commits issued on bar_mma not yet waited for
-    bool stored = false;      // thread 0 has bulk stores in flight
+    bool stored = false;      // the copy thread has bulk stores in flight
     float range_max = 0.f;
 
     int it = 0;
@@ -314,18 +319,18 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
 #pragma unroll
             for (int i = 0; i < TPP; ++i) {
                 acc += la_cur[i];
-                g[(r0 + i) * DK + ch] = acc;
+                g[(r0 + i) * DK + ch] = acc * kLog2e;   // base 2
             }
         }
         __syncthreads();
         bool wide = false;   // this channel's decay within the chunk too strong for the split factors
         if (tid < DK) {
-            const float gm = g[((L - 1) >> 1) * DK + tid], gl = g[(L - 1) * DK + tid];
+            const float gm = g[((L - 1) >> 1) * DK + tid], gl = g[(L - 1) * DK + tid];   // base 2
             s_gm[tid] = gm;
-            s_egm[tid] = __expf(gm);
-            s_eglm[tid] = __expf(gl - gm);
-            reinterpret_cast<float*>(rec + R::GC)[tid] = expf(gl);
-            wide = fmaxf(g[tid] - gm, gm - gl) > kMaxSplitExponent;
+            s_egm[tid] = ex2_approx(gm);
+            s_eglm[tid] = ex2_approx(gl - gm);
+            reinterpret_cast<float*>(rec + R::GC)[tid] = exp2f(gl);
+            wide = fmaxf(g[tid] - gm, gm - gl) > kMaxSplitExponent2;
         }
         // Strong decay: the factors e^{+-(g - g_m)} of A and P could overflow, so
         // this chunk forms A and P exactly (slow path, no MMA1).
@@ -376,23 +381,24 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                     for (int h2 = 0; h2 < 2; ++h2) {
                         const int e = 2 * e2 + h2;
                         const float kk = __bfloat162float(kb[e]), qq = __bfloat162float(qb[e]);
-                        float em, eb, e0, eh;
                         if constexpr (!STRONG) {
-                            em = __expf(gv[e] - gmv[e]);   // e^{g_r - g_m}
-                            eb = __expf(gmv[e] - gv[e]);   // e^{g_m - g_r}
-                            e0 = egmv[e] * em;             // e^{g_r}
-                            eh = eglmv[e] * eb;            // e^{g_{L-1} - g_r}
-                        } else {                           // unsplit, every exponent <= 0
-                            em = eb = 0.f;
-                            e0 = __expf(gv[e]);
-                            eh = __expf(g[(L - 1) * DK + c8 + e] - gv[e]);
+                            const float d = gv[e] - gmv[e];
+                            const float em = ex2_approx(d);          // e^{g_r - g_m}
+                            const float kem = kk * em, qem = qq * em;
+                            const float keb = kk * ex2_approx(-d);   // k e^{g_m - g_r}
+                            ka[e] = round_tf32_alu(kem);
+                            qa[e] = round_tf32_alu(qem);
+                            kbm[e] = round_tf32_alu(keb);
+                            k0v[h2] = kem * egmv[e];                 // k e^{g_r}
+                            q0v[h2] = qem * egmv[e];                 // q e^{g_r}
+                            khv[h2] = keb * eglmv[e];                // k e^{g_{L-1} - g_r}
+                        } else {                                     // unsplit, every exponent <= 0
+                            const float e0 = ex2_approx(gv[e]);
+                            k0v[h2] = kk * e0;
+                            q0v[h2] = qq * e0;
+                            khv[h2] = kk * ex2_approx(g[(L - 1) * DK + c8 + e] - gv[e]);
+                            ka[e] = qa[e] = kbm[e] = 0.f;
                         }
-                        ka[e] = round_tf32_alu(kk * em);
-                        qa[e] = round_tf32_alu(qq * em);
-                        kbm[e] = round_tf32_alu(kk * eb);
-                        k0v[h2] = kk * e0;
-                        q0v[h2] = qq * e0;
-                        khv[h2] = kk * eh;
                     }
                     k0[e2] = __floats2half2_rn(k0v[0], k0v[1]);
                     q0[e2] = __floats2half2_rn(q0v[0], q0v[1]);
@@ -420,22 +426,6 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0 && wn < total) {
-            // prefetch the next item: log_alpha into G (free now) and its k, v, q
-            // tiles into the other stage (free once the bulk stores of the item
-            // that used it have read their tiles)
-            issue_la(wn);
-            if (stored) bulk_store_wait_read();
-            issue_tma(wn, stage ^ 1);
-        }
-        if (tid == 0) {
-            // Q~ tiles are the lower halves (rows 64..127) of the record's WQ tiles
-#pragma unroll
-            for (int b = 0; b < DK / 64; ++b)
-                bulk_store(rec + R::WQ + b * 16384 + 8192, st + Sm::QS + b * Sm::TILE, 8192);
-            bulk_store_commit();
-            stored = true;
-        }
         if (tid == 0 && !strong) {
             // ---- MMA1 (tf32): [K~m; Q~m] K-m^T -> R1 (overlaps the v conversion)
             tc_fence_after();
@@ -450,9 +440,27 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                              (kb | ks) != 0);
             mma_commit(&bar_mma);
         }
+        // The copy thread (warp 1) prefetches the next item and stores this
+        // item's Q~ while warp 0 issues MMA1 and warps 2..7 convert v.  It
+        // issues every bulk store of the kernel, so its wait covers them all.
+        if (tid == kCopyThread) {
+            if (wn < total) {
+                // log_alpha into G (free now); k, v, q tiles into the other
+                // stage once the bulk stores of the item that used it have read it
+                issue_la(wn);
+                if (stored) bulk_store_wait_read();
+                issue_tma(wn, stage ^ 1);
+            }
+            // Q~ tiles are the lower halves (rows 64..127) of the record's WQ tiles
+#pragma unroll
+            for (int b = 0; b < DK / 64; ++b)
+                bulk_store(rec + R::WQ + b * 16384 + 8192, st + Sm::QS + b * Sm::TILE, 8192);
+            bulk_store_commit();
+            stored = true;
+        }
         mma_pending = strong ? 0 : 1;
-        // v: bf16 -> fp16 in place, 8 values per thread and step
-        for (int item = tid; item < kChunk * (DV / 8); item += 256) {
+        // v: bf16 -> fp16 in place, 8 values per thread and step (warps 2..7)
+        for (int item = tid - 64; tid >= 64 && item < kChunk * (DV / 8); item += 192) {
             const int r = item / (DV / 8), j8 = (item - r * (DV / 8)) * 8;
             const uint32_t o = Sm::VS + (j8 >> 6) * Sm::TILE + sw128_offset(r, (j8 & 63) * 2);
             uint4 raw = *reinterpret_cast<const uint4*>(st + o);
@@ -646,7 +654,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         }
         fence_proxy_async_smem();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == kCopyThread) {
 #pragma unroll
             for (int b = 0; b < DK / 64; ++b)   // W: rows 0..63 of each WQ tile
                 bulk_store(rec + R::WQ + b * 16384, st + Sm::KS + b * Sm::TILE, Sm::TILE);
