@@ -14,6 +14,7 @@
 namespace {
 
 thread_local std::string g_last_error;
+thread_local long long g_debug_drop_cap = 0;   // armed by kda_debug_drop_copy (one call)
 constexpr int kMaxStageEvents = 6;
 thread_local cudaEvent_t g_stage_events[kMaxStageEvents] = {};
 thread_local int g_stage_event_count = 0;   // 0: off
@@ -174,6 +175,11 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
     a.max_chunks = L.max_chunks;
     a.fixed_chunks_per_seq = L.chunks_per_seq;
     a.stream = static_cast<cudaStream_t>(stream);
+    if (g_debug_drop_cap > 0 && a.bf16 && gate == KDA_GATE_CHANNEL) {   // one-shot test hook
+        a.debug_drop_copy = 1;
+        a.wait_cap = g_debug_drop_cap;
+        g_debug_drop_cap = 0;
+    }
 
     cudaError_t e = mark_stage(0, a.stream);
     if (e == cudaSuccess) e = kda::launch_chunk_prep(a);
@@ -370,6 +376,12 @@ kda_status kda_set_stage_events(void* const* events, int count) {
         if (!events[i]) return fail(KDA_ERR_INVALID_ARG, "event %d is null", i);
     for (int i = 0; i < n; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
     g_stage_event_count = n;
+    return ok();
+}
+
+kda_status kda_debug_drop_copy(long long wait_cycles) {
+    if (wait_cycles < 0) return fail(KDA_ERR_INVALID_ARG, "wait_cycles=%lld < 0", wait_cycles);
+    g_debug_drop_cap = wait_cycles;
     return ok();
 }
 

@@ -181,7 +181,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                       const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_la,
                       const float* __restrict__ log_alpha_head, const float* __restrict__ beta,
                       ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
-                      size_t max_chunks)
+                      size_t max_chunks, long long wait_cap, int drop_first_la)
 {
     using Sm = K1Smem<DK, DV>;
     using R = TcRec<DK, DV>;
@@ -273,7 +273,9 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
 
     if (tid == 0) {
         issue_tma(blockIdx.x, 0);
-        issue_la(blockIdx.x);
+        // test hook: CTA 0 can leave out its first log-decay copy, so that the
+        // bounded wait on it gives up (nothing else is in flight at that wait)
+        if (!(drop_first_la && blockIdx.x == 0)) issue_la(blockIdx.x);
     }
     load_beta(blockIdx.x);
     bool aborted = false;
@@ -299,8 +301,8 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
 
         // ---- cumulative log-decay, in place over the log_alpha tile in G -------
         float* g = reinterpret_cast<float*>(sm + Sm::G);   // [64][DK]
-        const bool ok_la = !channel_gate || mbar_wait_cycles(&bar_la, it & 1, kWaitCycles);
-        const bool ok_load = mbar_wait_cycles(&bar_load[stage], (it >> 1) & 1, kWaitCycles);
+        const bool ok_la = !channel_gate || mbar_wait_cycles(&bar_la, it & 1, wait_cap);
+        const bool ok_load = mbar_wait_cycles(&bar_load[stage], (it >> 1) & 1, wait_cap);
         if (__syncthreads_or(!(ok_la && ok_load))) { aborted = true; break; }
         {
             float la_cur[TPP];
@@ -481,7 +483,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         float* ym = reinterpret_cast<float*>(sm + Sm::YM);   // [6][16][17]
         bool ok = true;
         if (!strong) {
-        ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         mma_phase ^= 1;
         mma_pending = 0;
@@ -624,7 +626,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             mma_commit(&bar_mma);
         }
         mma_pending = 1;
-        ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         mma_phase ^= 1;
         mma_pending = 0;
@@ -668,9 +670,9 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
     if (aborted) {
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         // let this CTA's own copies and MMAs finish (bounded) before freeing
-        for (int s2 = 0; s2 < 2; ++s2) (void)mbar_wait_cycles(&bar_load[s2], 0, kWaitCycles / 4);
-        if constexpr (channel_gate) (void)mbar_wait_cycles(&bar_la, 0, kWaitCycles / 4);
-        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        for (int s2 = 0; s2 < 2; ++s2) (void)mbar_wait_cycles(&bar_load[s2], 0, wait_cap / 4);
+        if constexpr (channel_gate) (void)mbar_wait_cycles(&bar_la, 0, wait_cap / 4);
+        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
     }
     if (stored) bulk_store_wait_all();
     if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
@@ -986,7 +988,8 @@ cudaError_t launch_intra_tc_t(const ChunkArgs& a) {
     const unsigned grid = (unsigned)(items < (size_t)sms ? items : (size_t)sms);
     kern<<<grid, 256, smem, a.stream>>>(mk, mv, mq, mla, a.log_alpha, a.beta, map,
                                         static_cast<WsHeader*>(a.ws_header),
-                                        static_cast<unsigned char*>(a.records), a.H, a.max_chunks);
+                                        static_cast<unsigned char*>(a.records), a.H, a.max_chunks,
+                                        a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy);
     return cudaGetLastError();
 }
 

@@ -49,6 +49,10 @@ struct ChunkArgs {
     float* dU;                    // [H][max_chunks][64][dv]: dL/dU of each chunk
     float* scratch;               // per-CTA fp32 scratch of the per-chunk gradient kernel
     int bwd_ctas;                 // CTAs of that kernel (its scratch holds this many)
+    // test hook (kda_debug_drop_copy): the tensor-core intra-chunk kernel leaves
+    // out one copy and caps its waits at wait_cap cycles (0: the default cap)
+    int debug_drop_copy;
+    long long wait_cap;
 };
 
 // Bytes of per-(head, chunk) intermediates: fp32 CUDA-core path / bf16 tensor-core path.

@@ -66,6 +66,8 @@ def _declare(lib):
     lib.kda_workspace_status.argtypes = [vp, sz, vp]
     lib.kda_set_stage_events.restype = i
     lib.kda_set_stage_events.argtypes = [ctypes.POINTER(vp), i]
+    lib.kda_debug_drop_copy.restype = i
+    lib.kda_debug_drop_copy.argtypes = [ctypes.c_longlong]
     lib.kda_last_error.restype = ctypes.c_char_p
     lib.kda_last_error.argtypes = []
     lib.kda_version.restype = ctypes.c_char_p
@@ -226,6 +228,11 @@ def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=N
         _ptr(g["dS0"]), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream_ptr(stream, q.device)))
     return g
+
+
+def debug_drop_copy(wait_cycles: int) -> None:
+    """Arm the one-shot failure-path test hook (``kda_debug_drop_copy``)."""
+    _check(lib().kda_debug_drop_copy(int(wait_cycles)))
 
 
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:

@@ -241,6 +241,18 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
  */
 kda_status kda_set_stage_events(void* const* events, int count);
 
+/*
+ * Test hook for the failure path (no counterpart in the pages).  Arms the next
+ * kda_chunk_fwd with bf16 inputs and the per-channel gate on this host thread
+ * (one call only): its intra-chunk kernel leaves out one asynchronous copy
+ * (the log-decay tile of the first work item of its first CTA) and caps each
+ * of its waits at `wait_cycles` SM clock cycles.  The wait on the missing copy
+ * gives up, the kernel records KDA_ERR_TIMEOUT in the workspace status
+ * (kda_workspace_status) and returns; that call's outputs are not meaningful.
+ * Nothing faults or hangs, and later calls run normally.  0 disarms.
+ */
+kda_status kda_debug_drop_copy(long long wait_cycles);
+
 /* Message of the last failing call on this host thread ("" if none). */
 const char* kda_last_error(void);
 

@@ -154,3 +154,11 @@ def test_bwd_workspace_size(lib):
     # bf16 inputs recompute fp32 records too: same size
     assert lib.kda_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 4, 0, bf16) == bwd
     assert lib.kda_chunk_bwd_workspace_size(1, 100, 2, 96, 64, 1, 0, f32) == 0
+
+
+def test_debug_drop_copy_arms_and_disarms(lib):
+    """The failure-path test hook: negative caps are rejected; arming and
+    disarming need no GPU (the hook only takes effect in a bf16 chunk call)."""
+    assert lib.kda_debug_drop_copy(-1) == 1
+    assert lib.kda_debug_drop_copy(1000) == 0
+    assert lib.kda_debug_drop_copy(0) == 0
