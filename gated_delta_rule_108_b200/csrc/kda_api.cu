@@ -267,13 +267,15 @@ size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num
     return L.total;
 }
 
-kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
-                         const float* beta, const float* initial_state, const int32_t* cu_seqlens,
-                         const void* d_o, const float* d_final_state, int B, int T, int H, int dk, int dv,
-                         int num_seqs, kda_dtype dtype, void* dq, void* dk_out, void* dv_out,
-                         float* dlog_alpha, float* dbeta, float* d_initial_state, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, const float* log_alpha,
+                                 const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                                 const void* d_o, const float* d_final_state, int B, int T, int H, int dk,
+                                 int dv, int num_seqs, kda_dtype dtype, kda_gate gate, void* dq, void* dk_out,
+                                 void* dv_out, float* dlog_alpha, float* dbeta, float* d_initial_state,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE)
+        return fail(KDA_ERR_INVALID_ARG, "unknown gate kind %d", (int)gate);
     if (B < 0 || T < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d", B, T, H);
     if (dk <= 0 || dv <= 0) return fail(KDA_ERR_INVALID_ARG, "bad head sizes dk=%d dv=%d", dk, dv);
     if (!supported_dim(dk) || !supported_dim(dv))
@@ -286,9 +288,11 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const floa
     if (tokens * (size_t)H * (size_t)(dk > dv ? dk : dv) >= (size_t)1 << 31)
         return fail(KDA_ERR_UNSUPPORTED, "B*T*H*d = %zu elements exceeds 2^31", tokens * H * (dk > dv ? dk : dv));
     if (tokens > 0) {
-        if (!q || !k || !v || !log_alpha || !beta || !d_o || !dq || !dk_out || !dv_out || !dlog_alpha || !dbeta)
+        if (!q || !k || !v || !beta || !d_o || !dq || !dk_out || !dv_out || !dbeta ||
+            (gate != KDA_GATE_NONE && (!log_alpha || !dlog_alpha)))
             return fail(KDA_ERR_INVALID_ARG, "null input/output pointer");
-        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) || !aligned16(log_alpha))
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) ||
+            (gate == KDA_GATE_CHANNEL && !aligned16(log_alpha)))
             return fail(KDA_ERR_INVALID_ARG, "q/k/v/log_alpha/d_o must be 16-byte aligned");
     }
     BwdLayout L;
@@ -305,7 +309,7 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const floa
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
     a.initial_state = initial_state; a.cu_seqlens = cu_seqlens;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.num_seqs = N;
-    a.gate = kda::kGateChannel;
+    a.gate = (int)gate;
     a.bf16 = dtype == KDA_BF16;
     a.scale = 1.0f / sqrtf((float)dk);
     a.ws_header = workspace;
@@ -345,6 +349,28 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const floa
     if (e == cudaSuccess) e = mark(5);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_chunk_bwd launch failed: %s", cudaGetErrorString(e));
     return ok();
+}
+
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                         const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                         const void* d_o, const float* d_final_state, int B, int T, int H, int dk, int dv,
+                         int num_seqs, kda_dtype dtype, void* dq, void* dk_out, void* dv_out,
+                         float* dlog_alpha, float* dbeta, float* d_initial_state, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    return chunk_bwd_impl(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_o, d_final_state, B, T, H, dk,
+                          dv, num_seqs, dtype, KDA_GATE_CHANNEL, dq, dk_out, dv_out, dlog_alpha, dbeta,
+                          d_initial_state, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_chunk_bwd_gated(const void* q, const void* k, const void* v, const float* log_alpha,
+                               const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                               const void* d_o, const float* d_final_state, int B, int T, int H, int dk,
+                               int dv, int num_seqs, kda_dtype dtype, kda_gate gate, void* dq, void* dk_out,
+                               void* dv_out, float* dlog_alpha, float* dbeta, float* d_initial_state,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+    return chunk_bwd_impl(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_o, d_final_state, B, T, H, dk,
+                          dv, num_seqs, dtype, gate, dq, dk_out, dv_out, dlog_alpha, dbeta, d_initial_state,
+                          workspace, workspace_bytes, stream);
 }
 
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {

@@ -407,7 +407,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                  const float* __restrict__ tmat, const float* __restrict__ states,
                  const float* __restrict__ dS_end, const float* __restrict__ dU_all, float* scratch,
                  T* __restrict__ dq, T* __restrict__ dk, T* __restrict__ dv, float* __restrict__ dla,
-                 float* __restrict__ dbeta, int H, size_t max_chunks, float scale)
+                 float* __restrict__ dbeta, int H, size_t max_chunks, float scale, int gate)
 {
     using R = Rec<DK, DV>;
     using C = Scr<DK, DV>;
@@ -435,11 +435,20 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         __syncthreads();   // the previous item is done with shared memory and scratch
         // ---- cumulative log-decay, beta --------------------------------------
         if (tid < DK) {
-            const float* la = log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid;
+            // per-channel gate [.., H, DK]; per-head gate [.., H] (the same value
+            // for every channel); no gate: log-decay 0
             float acc = 0.f;
-            for (int r = 0; r < kChunk; ++r) {
-                acc += (r < L) ? la[(size_t)r * rowk] : 0.f;
-                sm.g[r][tid] = acc;
+            if (gate == kGateNone) {
+                for (int r = 0; r < kChunk; ++r) sm.g[r][tid] = 0.f;
+            } else {
+                const bool chan = gate == kGateChannel;
+                const size_t rstride = chan ? rowk : (size_t)H;
+                const float* la = chan ? log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid
+                                       : log_alpha + (size_t)tok0 * H + h;
+                for (int r = 0; r < kChunk; ++r) {
+                    acc += (r < L) ? la[(size_t)r * rstride] : 0.f;
+                    sm.g[r][tid] = acc;
+                }
             }
             sm.dgl[tid] = 0.f;
         } else if (tid >= 128 && tid < 128 + kChunk) {
@@ -677,16 +686,28 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             sm.g[r][ch] = kk * (dkl - dkr + dkt * eg) - dkh * kh + qq * (dql + dqt * eg);   // dg
         }
         __syncthreads();
-        // dlog_alpha_s = sum_{r >= s} dg_r, with g_{L-1}'s own cotangent added at L-1
-        if (tid < DK) {
+        // dlog_alpha_s = sum_{r >= s} dg_r, with g_{L-1}'s own cotangent added at
+        // L-1; a per-head gate is shared by all channels, so its cotangent is
+        // the sum over channels
+        if (gate != kGateNone && tid < DK) {
             float run = sm.dgl[tid] + sm.dgam[tid] * expf(sm.gl[tid]);
             for (int r = L - 1; r >= 0; --r) {
                 run += sm.g[r][tid];
-                dla[(size_t)(tok0 + r) * rowk + (size_t)h * DK + tid] = run;
+                if (gate == kGateChannel) dla[(size_t)(tok0 + r) * rowk + (size_t)h * DK + tid] = run;
+                else sm.g[r][tid] = run;
             }
-        } else if (tid >= 128 && tid < 128 + kChunk) {
+        }
+        if (tid >= 128 && tid < 128 + kChunk) {
             const int r = tid - 128;
             if (r < L) dbeta[(size_t)(tok0 + r) * H + h] = sm.dbeta[r];
+        }
+        if (gate == kGateHead) {
+            __syncthreads();
+            if (tid < L) {
+                float acc = 0.f;
+                for (int c = 0; c < DK; ++c) acc += sm.g[tid][(c + tid) % DK];   // rotated: no bank conflicts
+                dla[(size_t)(tok0 + tid) * H + h] = acc;
+            }
         }
     }
 }
@@ -718,7 +739,7 @@ cudaError_t launch_bwd_intra_t(const ChunkArgs& a) {
         static_cast<const T*>(a.d_o), map, static_cast<const WsHeader*>(a.ws_header),
         static_cast<const float*>(a.records), a.tmat, a.states, a.dS_end, a.dU, a.scratch,
         static_cast<T*>(a.dq), static_cast<T*>(a.dk_out), static_cast<T*>(a.dv_out), a.dlog_alpha, a.dbeta,
-        a.H, a.max_chunks, a.scale);
+        a.H, a.max_chunks, a.scale, a.gate);
     return cudaGetLastError();
 }
 

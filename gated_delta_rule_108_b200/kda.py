@@ -62,6 +62,9 @@ def _declare(lib):
     lib.kda_chunk_bwd.restype = i
     lib.kda_chunk_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
                                   vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.kda_chunk_bwd_gated.restype = i
+    lib.kda_chunk_bwd_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
+                                        vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.kda_workspace_status.restype = i
     lib.kda_workspace_status.argtypes = [vp, sz, vp]
     lib.kda_set_stage_events.restype = i
@@ -191,21 +194,20 @@ def chunk_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
 def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=None,
               cu_seqlens=None, output_d_initial_state: bool = True, workspace=None,
               stream=None) -> Dict[str, Optional[torch.Tensor]]:
-    """Gradients of the chunkwise forward (``kda_chunk_bwd``).
+    """Gradients of the chunkwise forward (``kda_chunk_bwd_gated``).
 
-    Inputs as ``chunk_fwd`` (per-channel log_alpha [B, T, H, dk]); d_o like o;
-    d_final_state [N, H, dk, dv] fp32 or None.  Returns a dict with dq, dk, dv
-    (input dtype), dlog_alpha, dbeta (fp32) and dS0 [N, H, dk, dv] (fp32, or
-    None when ``output_d_initial_state`` is false).
+    Inputs as ``chunk_fwd``: log_alpha [B, T, H, dk] (KDA), [B, T, H] (Gated
+    DeltaNet) or None (DeltaNet); d_o like o; d_final_state [N, H, dk, dv] fp32
+    or None.  Returns a dict with dq, dk, dv (input dtype), dlog_alpha (shaped
+    like log_alpha, None without a gate), dbeta (fp32) and dS0 [N, H, dk, dv]
+    (fp32, or None when ``output_d_initial_state`` is false).
     """
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o")):
         _need(t, n, q.dtype)
     _need(beta, "beta", torch.float32)
-    _need(log_alpha, "log_alpha", torch.float32)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    if tuple(log_alpha.shape) != (B, T, H, dk):
-        raise KDAError(1, f"log_alpha must be {(B, T, H, dk)}, got {tuple(log_alpha.shape)}")
+    gate = _gate_of(log_alpha, 4, (B, T, H, dk), (B, T, H))
     if cu_seqlens is not None:
         _need(cu_seqlens, "cu_seqlens", torch.int32)
         N = cu_seqlens.numel() - 1
@@ -215,15 +217,16 @@ def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=N
         if t is not None:
             _need(t, n, torch.float32)
     g = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
-         "dlog_alpha": torch.empty_like(log_alpha), "dbeta": torch.empty_like(beta),
+         "dlog_alpha": None if log_alpha is None else torch.empty_like(log_alpha),
+         "dbeta": torch.empty_like(beta),
          "dS0": (torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
                  if output_d_initial_state else None)}
     ws_bytes = chunk_bwd_workspace_size(B, T, H, dk, dv, N, cu_seqlens is not None, q.dtype)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
-    _check(lib().kda_chunk_bwd(
+    _check(lib().kda_chunk_bwd_gated(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
-        _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state), B, T, H, dk, dv, N, _dtype_code(q),
+        _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state), B, T, H, dk, dv, N, _dtype_code(q), gate,
         _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]),
         _ptr(g["dS0"]), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream_ptr(stream, q.device)))

@@ -227,6 +227,23 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * kda_chunk_bwd with the gate shape chosen by `gate` (see kda_gate): log_alpha
+ * and dlog_alpha are [B, T, H, dk] for KDA_GATE_CHANNEL, [B, T, H] for
+ * KDA_GATE_HEAD (the cotangent of a per-head log-decay is the sum over the key
+ * channels it decays), and unused (may be NULL) for KDA_GATE_NONE.  Everything
+ * else as kda_chunk_bwd; the workspace size does not depend on the gate.
+ */
+kda_status kda_chunk_bwd_gated(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta,
+                               const float* initial_state, const int32_t* cu_seqlens,
+                               const void* d_o, const float* d_final_state,
+                               int B, int T, int H, int dk, int dv, int num_seqs,
+                               kda_dtype dtype, kda_gate gate, void* dq, void* dk_out,
+                               void* dv_out, float* dlog_alpha, float* dbeta,
+                               float* d_initial_state, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
  * Measurement hook for benchmarks.  When `events` is non-NULL, each later
  * kda_chunk_fwd on this host thread records the caller-created CUDA events
  * (cudaEvent_t passed as void*) on its stream at the stage boundaries:

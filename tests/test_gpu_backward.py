@@ -40,7 +40,7 @@ def run_bwd(x, d_o, dSf):
                         d_final_state=None if dSf is None else dSf.cuda(),
                         cu_seqlens=g["cu_seqlens"])
     torch.cuda.synchronize()
-    return {k: v.cpu() for k, v in out.items()}
+    return {k: (None if v is None else v.cpu()) for k, v in out.items()}
 
 
 def oracle_bwd(x, d_o, dSf):
@@ -122,3 +122,30 @@ def test_chunk_bwd_c1_sampled(cuda_device):
         part = {n: (got[n][s:s + 1, :, h:h + 1] if n != "dS0" else got[n][s:s + 1, h:h + 1])
                 for n in GRADS}
         check_all(part, ref, torch.bfloat16, f"C1 seq {s} head {h}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("gate", ["head", "none"])
+def test_chunk_bwd_gates(cuda_device, dtype, gate):
+    """Gated DeltaNet (one log-decay per head) and DeltaNet (none) through the
+    backward.  The oracle takes the gate broadcast to every channel; a per-head
+    log-decay's cotangent is the sum of the per-channel ones (chain rule)."""
+    w = I.ChunkWorkload("bgate", B=2, T=150, H=2, dk=128, dv=64, dtype=dtype, s0_std=0.05, seed=56)
+    x = I.chunk_inputs(w)
+    B, T, H, dk = x["q"].shape
+    if gate == "head":
+        gen = torch.Generator().manual_seed(561)
+        la = -torch.exp(torch.randn(B, T, H, generator=gen)) / 16
+        la_full = la[..., None].expand(B, T, H, dk).contiguous()
+    else:
+        la, la_full = None, torch.zeros(B, T, H, dk)
+    d_o, dSf = cotangents(x, 562)
+    got = run_bwd(dict(x, log_alpha=la), d_o, dSf)
+    ref = oracle_bwd(dict(x, log_alpha=la_full), d_o, dSf)
+    for n in ("dq", "dk", "dv", "dbeta", "dS0"):
+        check(got[n], ref[n], dtype, f"{gate} {n}")
+    if gate == "head":
+        assert got["dlog_alpha"].shape == (B, T, H)
+        check(got["dlog_alpha"], ref["dlog_alpha"].sum(-1), dtype, "head dlog_alpha")
+    else:
+        assert got["dlog_alpha"] is None
