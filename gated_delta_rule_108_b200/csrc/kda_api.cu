@@ -71,10 +71,12 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
     return true;
 }
 
-// Backward workspace: [header][chunk_offsets][fp32 records][T][chunk-start
-// states][dS at chunk ends][dU][per-CTA scratch], each 256-byte aligned.
+// Backward workspace: [header][chunk_offsets][the forward's records][bf16
+// inputs: fp32 records][T][chunk-start states][dS at chunk ends][dU][per-CTA
+// scratch], each 256-byte aligned.
 struct BwdLayout {
-    WsLayout base;   // header, offsets (records re-sized below)
+    WsLayout base;   // header, offsets, the forward's records for this dtype
+    size_t xrec_off; // bf16: fp32 records written by the tensor-core K1 (0 for fp32)
     size_t tmat_off, states_off, dS_off, dU_off, scratch_off, total;
     int ctas;        // CTAs the scratch holds
 };
@@ -83,8 +85,13 @@ bool bwd_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, 
                 BwdLayout& L) {
     if (!ws_layout(B, T, H, dk, dv, num_seqs, varlen, dtype, L.base)) return false;
     const size_t units = (size_t)H * L.base.max_chunks;   // (head, chunk) pairs
-    const size_t rec = kda::simt_record_bytes(dk, dv);
-    L.tmat_off = round_up(L.base.records_off + rec * units, 256);
+    size_t off = round_up(L.base.total, 256);
+    L.xrec_off = 0;
+    if (dtype == KDA_BF16) {
+        L.xrec_off = off;
+        off = round_up(off + kda::simt_record_bytes(dk, dv) * units, 256);
+    }
+    L.tmat_off = off;
     L.states_off = round_up(L.tmat_off + sizeof(float) * kda::kChunk * kda::kChunk * units, 256);
     L.dS_off = round_up(L.states_off + sizeof(float) * (size_t)dk * dv * units, 256);
     L.dU_off = round_up(L.dS_off + sizeof(float) * (size_t)dk * dv * units, 256);
@@ -332,17 +339,21 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "device query failed: %s", cudaGetErrorString(e));
     a.bwd_ctas = L.ctas < 2 * sms ? L.ctas : 2 * sms;   // two resident per SM
 
-    // forward recomputation (fp32 records + T + chunk-start states), then the
-    // reversed pass over chunks, then the per-chunk gradients
+    // forward recomputation (fp32 records + T + chunk-start states: on the
+    // tensor cores for bf16 inputs, which also write their own fp16 records
+    // for their inter-chunk kernel), then the reversed pass over chunks, then
+    // the per-chunk gradients
     const bool marks = g_stage_event_count >= 6;   // the backward records all six or none
     auto mark = [&](int i) { return marks ? mark_stage(i, a.stream) : cudaSuccess; };
+    if (a.bf16) a.xrecords = reinterpret_cast<float*>(ws + L.xrec_off);
     e = mark(0);
     if (e == cudaSuccess) e = kda::launch_chunk_prep(a);
     if (e == cudaSuccess) e = mark(1);
-    if (e == cudaSuccess) e = kda::launch_chunk_intra(a);
+    if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_intra_tc(a) : kda::launch_chunk_intra(a);
     if (e == cudaSuccess) e = mark(2);
-    if (e == cudaSuccess) e = kda::launch_chunk_inter(a);
+    if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_inter_tc(a) : kda::launch_chunk_inter(a);
     if (e == cudaSuccess) e = mark(3);
+    if (a.bf16) a.records = a.xrecords;   // the backward kernels read the fp32 records
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_inter(a);
     if (e == cudaSuccess) e = mark(4);
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);

@@ -42,17 +42,8 @@ namespace {
 
 constexpr float kMaxSplitExponent = 60.f;   // same split guard as the forward
 
-// fp32 record of the CUDA-core forward (same layout as kda_chunk_simt.cu)
 template <int DK, int DV>
-struct Rec {
-    static constexpr size_t W = 0;
-    static constexpr size_t U0 = W + kChunk * DK;
-    static constexpr size_t QT = U0 + kChunk * DV;
-    static constexpr size_t KH = QT + kChunk * DK;
-    static constexpr size_t P = KH + kChunk * DK;
-    static constexpr size_t GC = P + kChunk * kChunk;
-    static constexpr size_t FLOATS = (GC + DK + 63) / 64 * 64;
-};
+using Rec = F32Rec<DK, DV>;
 
 // ------------------------------------------------------------------ KB3 ----
 constexpr int kSlice = 64;   // value columns per CTA

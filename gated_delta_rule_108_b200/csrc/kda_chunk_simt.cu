@@ -86,19 +86,8 @@ chunk_prep_kernel(WsHeader* hdr, int32_t* chunk_offsets, const int32_t* __restri
     }
 }
 
-// Record of one (head, chunk), fp32: W [64][DK] | U0 [64][DV] | Qt [64][DK] |
-// Kh [64][DK] | P [64][64] | gC [DK].  Rows >= L are zero.
 template <int DK, int DV>
-struct SimtRec {
-    static constexpr size_t W = 0;
-    static constexpr size_t U0 = W + kChunk * DK;
-    static constexpr size_t QT = U0 + kChunk * DV;
-    static constexpr size_t KH = QT + kChunk * DK;
-    static constexpr size_t P = KH + kChunk * DK;
-    static constexpr size_t GC = P + kChunk * kChunk;
-    static constexpr size_t FLOATS_RAW = GC + DK;
-    static constexpr size_t FLOATS = (FLOATS_RAW + 63) / 64 * 64;  // 256-byte multiple
-};
+using SimtRec = F32Rec<DK, DV>;
 
 // ---------------------------------------------------------------- K1 ------
 template <typename T, int DK, int DV>

@@ -33,6 +33,22 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
 
+// fp32 record of one (head, chunk), row-major: W [64][DK] | U0 [64][DV] |
+// Q~ [64][DK] | K^ [64][DK] | P [64][64] | gamma [DK].  Rows past the chunk's
+// tokens are zero.  Written by the CUDA-core intra-chunk kernel (fp32 inputs)
+// or by the tensor-core one in its backward mode; read by the CUDA-core
+// inter-chunk kernel and the backward kernels.
+template <int DK, int DV>
+struct F32Rec {
+    static constexpr size_t W = 0;
+    static constexpr size_t U0 = W + kChunk * DK;
+    static constexpr size_t QT = U0 + kChunk * DV;
+    static constexpr size_t KH = QT + kChunk * DK;
+    static constexpr size_t P = KH + kChunk * DK;
+    static constexpr size_t GC = P + kChunk * kChunk;
+    static constexpr size_t FLOATS = (GC + DK + 63) / 64 * 64;   // 256-byte multiple
+};
+
 // Element loads/stores for the two input dtypes.
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
