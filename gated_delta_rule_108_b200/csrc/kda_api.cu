@@ -353,8 +353,10 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
     if (e == cudaSuccess) e = mark(2);
     if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_inter_tc(a) : kda::launch_chunk_inter(a);
     if (e == cudaSuccess) e = mark(3);
-    if (a.bf16) a.records = a.xrecords;   // the backward kernels read the fp32 records
-    if (e == cudaSuccess) e = kda::launch_chunk_bwd_inter(a);
+    // the reversed chain reads the fp16 tensor-core records (bf16) or the fp32
+    // ones; the per-chunk gradient kernel reads the fp32 records
+    if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_bwd_inter_tc(a) : kda::launch_chunk_bwd_inter(a);
+    if (a.bf16) a.records = a.xrecords;
     if (e == cudaSuccess) e = mark(4);
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);
     if (e == cudaSuccess) e = mark(5);

@@ -977,6 +977,272 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// --------------------------------------------------- backward KB3 (bf16) ----
+// The backward's reversed chunk chain on the tensor cores (bf16 inputs), one
+// CTA (8 warps) per (sequence, head, 64-wide value slice).  With D = c dO and
+// dS' the cotangent of the state leaving chunk n:
+//     dU = K^ dS' + P^T D        dS = Diag(gamma) dS' + Q~^T D + W^T (-dU)
+// dS lives in TMEM (fp32) for the whole sequence with an fp16 copy in smem as
+// the MMA operand, as the forward's state does; the records are the forward
+// intra-chunk kernel's fp16 tiles and D is TMA-loaded from d_o (bf16) and
+// converted in place.  dU and dS' of every chunk go out in fp32 for the
+// per-chunk gradient kernel.
+template <int DK, int DV>
+struct B3Smem {
+    using K2 = K2Smem<DK, DV>;                                  // record layout of a stage
+    static constexpr uint32_t D = K2::STAGE;                    // cotangent tile: 64 tokens x 64 columns
+    static constexpr uint32_t STAGE = K2::STAGE + 8192;
+    static constexpr uint32_t DS16 = 2 * STAGE;                 // fp16 dS', rows = key channel
+    static constexpr uint32_t DU16 = DS16 + 128 * 128;          // fp16 -dU, rows = token
+    static constexpr uint32_t END = DU16 + 8192;
+    static constexpr uint32_t TX_BYTES = TcRec<DK, DV>::WQ_BYTES + TcRec<DK, DV>::KH_BYTES + 8192 + DK * 4 + 8192;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(256, 1)
+bwd_inter_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const float* __restrict__ d_final_state,
+                    float* __restrict__ d_initial_state, float* __restrict__ dS_end, float* __restrict__ dU_all,
+                    ChunkMap map, WsHeader* hdr, const unsigned char* __restrict__ records, int H,
+                    size_t max_chunks, float scale)
+{
+    using Sm = B3Smem<DK, DV>;
+    using K2 = K2Smem<DK, DV>;
+    using R = TcRec<DK, DV>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t bar_full[2], bar_mma;
+    __shared__ uint32_t s_tmem;
+
+    if (hdr->status != kStatusOk) return;
+    const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSliceTc;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int lane_row = (warp & 3) * 32 + (tid & 31);   // TMEM lane = MMA row
+    const int wg = warp >> 2;                            // warpgroup: columns [32 wg, 32 wg + 32)
+    const int first = map.seq_first_chunk(s), nch = map.seq_num_chunks(s);
+    const int tok_begin = map.seq_token_begin(s), tok_end = map.seq_token_end(s);
+    const size_t state_off = ((size_t)s * H + h) * DK * DV;
+
+    if (tid == 0) {
+        mbar_init(&bar_full[0], 1);
+        mbar_init(&bar_full[1], 1);
+        mbar_init(&bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const uint32_t RDU = tmem;          // [dU; *] 128 lanes x 64 columns
+    const uint32_t SACC = tmem + 64;    // dS slice: lane = key channel
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    float range_max = 0.f;
+
+    auto issue = [&](int n) {   // chunk n's records and cotangent tile into stage n & 1
+        if (n < 0) return;
+        unsigned char* st = sm + (n & 1) * Sm::STAGE;
+        const unsigned char* rec = records + ((size_t)h * max_chunks + first + n) * R::BYTES;
+        uint64_t* bar = &bar_full[n & 1];
+        mbar_arrive_expect_tx(bar, Sm::TX_BYTES);
+        bulk_load(st + K2::WQ, rec + R::WQ, R::WQ_BYTES, bar);
+        bulk_load(st + K2::KH, rec + R::KH, R::KH_BYTES, bar);
+        bulk_load(st + K2::P, rec + R::P, 8192, bar);
+        bulk_load(st + K2::GC, rec + R::GC, DK * 4, bar);
+        tma_load_3d(st + Sm::D, &tm_do, bar, j0, h, tok_begin + n * kChunk);
+    };
+    // fp16 copy of 32 columns of this thread's key channel of dS (row of DS16)
+    auto put_ds16 = [&](const float (&v)[32]) {
+#pragma unroll
+        for (int i8 = 0; i8 < 4; ++i8) {
+            __align__(16) __half2 hv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float a = v[8 * i8 + 2 * e], b = v[8 * i8 + 2 * e + 1];
+                range_max = fmaxf(range_max, fmaxf(fabsf(a), fabsf(b)));
+                hv[e] = __floats2half2_rn(a, b);
+            }
+            *reinterpret_cast<uint4*>(sm + Sm::DS16 + sw128_offset(lane_row, (32 * wg + 8 * i8) * 2)) =
+                *reinterpret_cast<const uint4*>(hv);
+        }
+    };
+
+    // cotangent of the final state -> TMEM and its fp16 copy
+    if (lane_row < DK) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (d_final_state)
+                x = *reinterpret_cast<const float4*>(d_final_state + state_off + (size_t)lane_row * DV + j0 + 32 * wg + i);
+            v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+        }
+        tmem_st32_sync(SACC + lane_base + 32 * wg, v);
+        put_ds16(v);
+    }
+    if (tid == 0) {
+        issue(nch - 1);
+        issue(nch - 2);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    bool aborted = false;
+    uint32_t mma_phase = 0;
+    int mma_pending = 0;
+    for (int n = nch - 1; n >= 0; --n) {
+        const int b = n & 1, m = nch - 1 - n;   // m-th chunk processed; stage b's (m >> 1)-th use
+        unsigned char* st = sm + b * Sm::STAGE;
+        const size_t item = (size_t)h * max_chunks + first + n;
+        const int tok0 = tok_begin + n * kChunk;
+        bool ok = mbar_wait_cycles(&bar_full[b], (m >> 1) & 1, kWaitCycles);
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+
+        // D = c dO: bf16 -> fp16 in place; rows past the sequence are zero
+        for (int it = tid; it < kChunk * 8; it += 256) {
+            const int r = it >> 3, j8 = (it & 7) * 8;
+            const uint32_t o = Sm::D + sw128_offset(r, j8 * 2);
+            uint4 raw = *reinterpret_cast<const uint4*>(st + o);
+            if (tok0 + r >= tok_end) raw = make_uint4(0, 0, 0, 0);
+            const __nv_bfloat162* db = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            __align__(16) __half2 dh[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = __bfloat1622float2(db[e]);
+                const float a = scale * x.x, c2 = scale * x.y;
+                range_max = fmaxf(range_max, fmaxf(fabsf(a), fabsf(c2)));
+                dh[e] = __floats2half2_rn(a, c2);
+            }
+            *reinterpret_cast<uint4*>(st + o) = *reinterpret_cast<const uint4*>(dh);
+        }
+        // dS' of this chunk out in fp32; then S_acc <- Diag(gamma) dS' (MMA-a reads the fp16 copy)
+        if (lane_row < DK) {
+            const float gc = reinterpret_cast<const float*>(st + K2::GC)[lane_row];
+            float v[32];
+            tmem_ld32_sync(SACC + lane_base + 32 * wg, v);
+            float* dst = dS_end + (item * DK + lane_row) * DV + j0 + 32 * wg;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                v[i] *= gc; v[i + 1] *= gc; v[i + 2] *= gc; v[i + 3] *= gc;
+            }
+            tmem_st32_sync(SACC + lane_base + 32 * wg, v);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // MMA-a: [K^; *] dS' + [P^T; *] D -> RDU
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc_k = instr_desc(kFmtF16, 128, kSliceTc, false, true);   // A K-major
+            constexpr uint32_t idesc_m = instr_desc(kFmtF16, 128, kSliceTc, true, true);    // A MN-major
+            const uint32_t kh = smem_u32(st + K2::KH), ds = smem_u32(sm + Sm::DS16);
+            const uint32_t pa = smem_u32(st + K2::P), da = smem_u32(st + Sm::D);
+#pragma unroll
+            for (int kb = 0; kb < DK / 64; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(RDU, smem_desc(kh + kb * 8192 + ks * 32, 16, 1024, kLayoutSW128),
+                            smem_desc(ds + kb * 8192 + ks * 2048, 8192, 1024, kLayoutSW128), idesc_k,
+                            (kb | ks) != 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(RDU, smem_desc(pa + ks * 2048, 8192, 1024, kLayoutSW128),
+                        smem_desc(da + ks * 2048, 8192, 1024, kLayoutSW128), idesc_m, true);
+            mma_commit(&bar_mma);
+        }
+        mma_pending = 1;
+        ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        mma_phase ^= 1;
+        mma_pending = 0;
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        tc_fence_after();
+
+        // dU (rows 0..63): fp32 out; -dU as the fp16 operand of MMA-b
+        if (lane_row < 64) {
+            float v[32];
+            tmem_ld32_sync(RDU + lane_base + 32 * wg, v);
+            float* dst = dU_all + (item * kChunk + lane_row) * DV + j0 + 32 * wg;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+#pragma unroll
+            for (int i8 = 0; i8 < 4; ++i8) {
+                __align__(16) __half2 hv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float a = v[8 * i8 + 2 * e], c2 = v[8 * i8 + 2 * e + 1];
+                    range_max = fmaxf(range_max, fmaxf(fabsf(a), fabsf(c2)));
+                    hv[e] = __floats2half2_rn(-a, -c2);
+                }
+                *reinterpret_cast<uint4*>(sm + Sm::DU16 + sw128_offset(lane_row, (32 * wg + 8 * i8) * 2)) =
+                    *reinterpret_cast<const uint4*>(hv);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // MMA-b: S_acc += Q~^T D + W^T (-dU)
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc_m = instr_desc(kFmtF16, 128, kSliceTc, true, true);
+            const uint32_t wq = smem_u32(st + K2::WQ), da = smem_u32(st + Sm::D), du = smem_u32(sm + Sm::DU16);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // Q~: rows 64..127 of each WQ tile
+                mma_f16(SACC, smem_desc(wq + 8192 + ks * 2048, 16384, 1024, kLayoutSW128),
+                        smem_desc(da + ks * 2048, 8192, 1024, kLayoutSW128), idesc_m, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // W: rows 0..63 of each WQ tile
+                mma_f16(SACC, smem_desc(wq + ks * 2048, 16384, 1024, kLayoutSW128),
+                        smem_desc(du + ks * 2048, 8192, 1024, kLayoutSW128), idesc_m, true);
+            mma_commit(&bar_mma);
+        }
+        mma_pending = 1;
+        ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        mma_phase ^= 1;
+        mma_pending = 0;
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        tc_fence_after();
+        if (tid == 0) {
+            fence_proxy_async_smem();
+            issue(n - 2);   // this stage is no longer read
+        }
+        // the fp16 copy of dS for the previous chunk
+        if (lane_row < DK) {
+            float v[32];
+            tmem_ld32_sync(SACC + lane_base + 32 * wg, v);
+            put_ds16(v);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    if (aborted) {
+        if (tid == 0) flag_error(hdr, kStatusTimeout);
+        // let MMAs and copies this CTA issued finish before its memory goes away
+        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        for (int b = 0; b < 2; ++b) (void)mbar_wait_cycles(&bar_full[b], 0, kWaitCycles / 8);
+    } else if (d_initial_state && lane_row < DK) {
+        float v[32];
+        tmem_ld32_sync(SACC + lane_base + 32 * wg, v);
+        float* dst = d_initial_state + state_off + (size_t)lane_row * DV + j0 + 32 * wg;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    }
+    if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
 // ------------------------------------------------------------- host -----
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1051,6 +1317,25 @@ cudaError_t launch_inter_tc_t(const ChunkArgs& a) {
     return cudaGetLastError();
 }
 
+template <int DK, int DV>
+cudaError_t launch_bwd_inter_tc_t(const ChunkArgs& a) {
+    if (a.num_seqs == 0) return cudaSuccess;
+    const int ntok = a.cu_seqlens ? a.T : a.B * a.T;
+    CUtensorMap mdo;
+    if (!make_map(&mdo, a.d_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
+    auto kern = bwd_inter_tc_kernel<DK, DV>;
+    const int smem = (int)B3Smem<DK, DV>::END + 1024;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)a.num_seqs, (unsigned)a.H, (unsigned)(DV / kSliceTc));
+    kern<<<grid, 256, smem, a.stream>>>(mdo, a.d_final_state, a.d_initial_state, a.dS_end, a.dU, map,
+                                        static_cast<WsHeader*>(a.ws_header),
+                                        static_cast<const unsigned char*>(a.records), a.H, a.max_chunks, a.scale);
+    return cudaGetLastError();
+}
+
 #define KDA_TC_DISPATCH(FN, a)                                                  \
     do {                                                                       \
         if ((a).dk == 128 && (a).dv == 128) return FN<128, 128>(a);            \
@@ -1076,5 +1361,7 @@ cudaError_t launch_chunk_inter_tc(const ChunkArgs& a) {
     if (a.num_seqs == 0) return cudaSuccess;
     KDA_TC_DISPATCH(launch_inter_tc_t, a);
 }
+
+cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_inter_tc_t, a); }
 
 }  // namespace kda

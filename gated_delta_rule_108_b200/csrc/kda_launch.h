@@ -71,6 +71,7 @@ cudaError_t launch_chunk_inter(const ChunkArgs& a);    // K2: serial over each s
 cudaError_t launch_chunk_intra_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K1
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K2
 cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a);  // backward: serial over chunks, reversed
+cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a); // the same on the tensor cores (bf16 inputs)
 cudaError_t launch_chunk_bwd_intra(const ChunkArgs& a);  // backward: all chunks in parallel
 size_t bwd_scratch_bytes_per_cta(int dk, int dv);
 constexpr int kBwdMaxCtas = 512;   // scratch is sized for at most this many CTAs
