@@ -77,6 +77,7 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
 struct BwdLayout {
     WsLayout base;   // header, offsets, the forward's records for this dtype
     size_t xrec_off; // bf16: fp32 records written by the tensor-core K1 (0 for fp32)
+    size_t vside_off;// bf16: the value-side products per (head, chunk) (0 for fp32)
     size_t tmat_off, states_off, dS_off, dU_off, scratch_off, total;
     int ctas;        // CTAs the scratch holds
 };
@@ -87,9 +88,13 @@ bool bwd_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, 
     const size_t units = (size_t)H * L.base.max_chunks;   // (head, chunk) pairs
     size_t off = round_up(L.base.total, 256);
     L.xrec_off = 0;
+    L.vside_off = 0;
     if (dtype == KDA_BF16) {
         L.xrec_off = off;
         off = round_up(off + kda::simt_record_bytes(dk, dv) * units, 256);
+        L.vside_off = off;
+        const size_t vs_floats = dk == 128 ? kda::VSide<128>::FLOATS : kda::VSide<64>::FLOATS;
+        off = round_up(off + sizeof(float) * vs_floats * units, 256);
     }
     L.tmat_off = off;
     L.states_off = round_up(L.tmat_off + sizeof(float) * kda::kChunk * kda::kChunk * units, 256);
@@ -354,10 +359,15 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
     if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_inter_tc(a) : kda::launch_chunk_inter(a);
     if (e == cudaSuccess) e = mark(3);
     // the reversed chain reads the fp16 tensor-core records (bf16) or the fp32
-    // ones; the per-chunk gradient kernel reads the fp32 records
+    // ones; for bf16 the products over the value dimension are formed on the
+    // tensor cores too; the per-chunk gradient kernel reads the fp32 records
     if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_bwd_inter_tc(a) : kda::launch_chunk_bwd_inter(a);
-    if (a.bf16) a.records = a.xrecords;
     if (e == cudaSuccess) e = mark(4);
+    if (a.bf16) {
+        a.vside = reinterpret_cast<float*>(ws + L.vside_off);
+        if (e == cudaSuccess) e = kda::launch_chunk_bwd_vside_tc(a);
+        a.records = a.xrecords;
+    }
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);
     if (e == cudaSuccess) e = mark(5);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_chunk_bwd launch failed: %s", cudaGetErrorString(e));

@@ -398,7 +398,8 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                  const float* __restrict__ tmat, const float* __restrict__ states,
                  const float* __restrict__ dS_end, const float* __restrict__ dU_all, float* scratch,
                  T* __restrict__ dq, T* __restrict__ dk, T* __restrict__ dv, float* __restrict__ dla,
-                 float* __restrict__ dbeta, int H, size_t max_chunks, float scale, int gate)
+                 float* __restrict__ dbeta, int H, size_t max_chunks, float scale, int gate,
+                 const float* __restrict__ vside)
 {
     using R = Rec<DK, DV>;
     using C = Scr<DK, DV>;
@@ -422,6 +423,12 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         const float* Sn = states + it * DK * DV;
         const float* dSe = dS_end + it * DK * DV;
         const float* dUc = dU_all + it * kChunk * DV;
+        // the products over the value dimension: precomputed (bf16 inputs) or formed here
+        const float* vs = vside ? vside + it * VSide<DK>::FLOATS : nullptr;
+        const float* pDQT = vs ? vs + VSide<DK>::DQT : scr + C::DQT;
+        const float* pDW = vs ? vs + VSide<DK>::DW : scr + C::DW;
+        const float* pDKH = vs ? vs + VSide<DK>::DKH : scr + C::DKH;
+        const float* pDP = vs ? vs + VSide<DK>::DP : scr + C::DP;
 
         __syncthreads();   // the previous item is done with shared memory and scratch
         // ---- cumulative log-decay, beta --------------------------------------
@@ -483,9 +490,12 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             const int r = idx / DV, j = idx - r * DV;
             const size_t off = (size_t)(tok0 + r) * rowv + (size_t)h * DV + j;
             scr[C::VV + idx] = (r < L) ? to_f32(v[off]) : 0.f;
-            scr[C::DO + idx] = (r < L) ? scale * to_f32(d_o[off]) : 0.f;
+            if (!vs) scr[C::DO + idx] = (r < L) ? scale * to_f32(d_o[off]) : 0.f;
         }
         // dgamma_c = sum_j dS'_cj S_cj: one warp per key row
+        if (vs) {
+            if (tid < DK) sm.dgam[tid] = vs[VSide<DK>::DGAM + tid];
+        } else
         for (int ch = warp; ch < DK; ch += 8) {
             float acc = 0.f;
             for (int j = lane; j < DV; j += 32) acc += dSe[(size_t)ch * DV + j] * Sn[(size_t)ch * DV + j];
@@ -495,6 +505,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         }
 
         // ---- products over the value dimension ---------------------------------
+        if (!vs) {
         {   // U = U0 - W S
             float acc[4][DV / 16];
             zero_acc<DV>(acc);
@@ -525,6 +536,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             gemm64<kChunk>(acc, Mat{scr + C::DO, DV, false}, Mat{scr + C::U, DV, true}, DV, sm.st);
             for_acc<kChunk>(acc, [&](int r, int i, float x) { scr[C::DP + r * kChunk + i] = (i <= r) ? x : 0.f; });
         }
+        }   // !vs
         // ---- through W = T diag(beta) K~ and U0 = T diag(beta) V -------------
         {   // Z = T^T dU: dv = beta Z, dbeta += <Z, v>
             float acc[4][DV / 16];
@@ -544,7 +556,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         {   // Y = T^T dW: dK~ = beta Y, dbeta += <Y, K~>
             float acc[4][DK / 16];
             zero_acc<DK>(acc);
-            gemm64<DK>(acc, Mat{Tm, kChunk, true}, Mat{scr + C::DW, DK, false}, kChunk, sm.st);
+            gemm64<DK>(acc, Mat{Tm, kChunk, true}, Mat{pDW, DK, false}, kChunk, sm.st);
             float part[4] = {0.f, 0.f, 0.f, 0.f};
             for_acc<DK>(acc, [&](int r, int n, float x) {
                 part[r & 3] += x * scr[C::KT + r * DK + n];
@@ -559,7 +571,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         {   // dT = (dW K~^T + dU V^T) diag(beta)
             float acc[4][kChunk / 16];
             zero_acc<kChunk>(acc);
-            gemm64<kChunk>(acc, Mat{scr + C::DW, DK, false}, Mat{scr + C::KT, DK, true}, DK, sm.st);
+            gemm64<kChunk>(acc, Mat{pDW, DK, false}, Mat{scr + C::KT, DK, true}, DK, sm.st);
             gemm64<kChunk>(acc, Mat{dUc, DV, false}, Mat{scr + C::VV, DV, true}, DV, sm.st);
             for_acc<kChunk>(acc, [&](int r, int i, float x) { scr[C::DT + r * kChunk + i] = x * sm.beta[i]; });
         }
@@ -614,7 +626,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                     scr[C::DKL + r * DK + n] = x * expf(sm.g[r][n] - sm.gm[n]);
                 });
                 zero_acc<DK>(acc);
-                gemm64<DK>(acc, Mat{scr + C::DP, kChunk, false}, Mat{scr + C::KR, DK, false}, kChunk, sm.st);
+                gemm64<DK>(acc, Mat{pDP, kChunk, false}, Mat{scr + C::KR, DK, false}, kChunk, sm.st);
                 for_acc<DK>(acc, [&](int r, int n, float x) {
                     scr[C::DQL + r * DK + n] = x * expf(sm.g[r][n] - sm.gm[n]);
                 });
@@ -623,7 +635,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                 float acc[4][DK / 16];
                 zero_acc<DK>(acc);
                 gemm64<DK>(acc, Mat{scr + C::DM, kChunk, true}, Mat{scr + C::KL, DK, false}, kChunk, sm.st);
-                gemm64<DK>(acc, Mat{scr + C::DP, kChunk, true}, Mat{scr + C::QL, DK, false}, kChunk, sm.st);
+                gemm64<DK>(acc, Mat{pDP, kChunk, true}, Mat{scr + C::QL, DK, false}, kChunk, sm.st);
                 for_acc<DK>(acc, [&](int r, int n, float x) {
                     scr[C::DKR + r * DK + n] = x * expf(sm.gm[n] - sm.g[r][n]);
                 });
@@ -638,12 +650,12 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                 for (int i = 0; i <= r; ++i) {   // r is the later token
                     const float e = expf(gr - sm.g[i][ch]);
                     const float ki = scr[C::KL + i * DK + ch];
-                    dql += scr[C::DP + r * kChunk + i] * ki * e;
+                    dql += pDP[r * kChunk + i] * ki * e;
                     if (i < r) dkl += scr[C::DM + r * kChunk + i] * ki * e;
                 }
                 for (int j = r; j < kChunk; ++j) {   // r is the earlier token
                     const float e = expf(sm.g[j][ch] - gr);
-                    dkr += scr[C::DP + j * kChunk + r] * scr[C::QL + j * DK + ch] * e;
+                    dkr += pDP[j * kChunk + r] * scr[C::QL + j * DK + ch] * e;
                     if (j > r) dkr += scr[C::DM + j * kChunk + r] * scr[C::KL + j * DK + ch] * e;
                 }
                 (void)kr; (void)qr;
@@ -667,7 +679,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             const float gg = sm.g[r][ch];
             const float eg = expf(gg), eh = expf(sm.gl[ch] - gg);
             const float dkl = scr[C::DKL + idx], dkr = scr[C::DKR + idx], dql = scr[C::DQL + idx];
-            const float dkt = scr[C::DKT + idx], dkh = scr[C::DKH + idx], dqt = scr[C::DQT + idx];
+            const float dkt = scr[C::DKT + idx], dkh = pDKH[idx], dqt = pDQT[idx];
             if (r < L) {
                 dk[off] = from_f32<T>(dkl + dkr + dkt * eg + dkh * eh);
                 dq[off] = from_f32<T>(dql + dqt * eg);
@@ -730,7 +742,7 @@ cudaError_t launch_bwd_intra_t(const ChunkArgs& a) {
         static_cast<const T*>(a.d_o), map, static_cast<const WsHeader*>(a.ws_header),
         static_cast<const float*>(a.records), a.tmat, a.states, a.dS_end, a.dU, a.scratch,
         static_cast<T*>(a.dq), static_cast<T*>(a.dk_out), static_cast<T*>(a.dv_out), a.dlog_alpha, a.dbeta,
-        a.H, a.max_chunks, a.scale, a.gate);
+        a.H, a.max_chunks, a.scale, a.gate, a.vside);
     return cudaGetLastError();
 }
 

@@ -1243,6 +1243,288 @@ bwd_inter_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const float* __re
     if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
+// ------------------------------------------- backward value-side (bf16) ----
+// The backward's products over the value dimension on the tensor cores (bf16
+// inputs), one (chunk, head) at a time per CTA:
+//     [W; Q~] S -> U = U0 - W S          [D; -dU] S^T -> [dQ~; dW]
+//     [U; *] dS'^T -> dK^                 [D; -dU] U^T -> dP (lower)
+// and dgamma = rowsum(dS' * S).  S, dS', dU (fp32) are converted to fp16
+// 128-byte-swizzled tiles, D = c dO is TMA-loaded (bf16) and converted in
+// place, W, Q~, U0 are the forward's fp16 record tiles; the products are
+// fp32 in TMEM and go out in fp32 (VSide layout).
+template <int DK, int DV>
+struct VsSmem {
+    static constexpr uint32_t NJ = DV / 64;                       // 64-column value blocks
+    static constexpr uint32_t AB = 0;                             // [D; -dU]: NJ tiles of 128 rows
+    static constexpr uint32_t S16 = AB + NJ * 16384;              // S: NJ tiles of DK rows (key channel)
+    static constexpr uint32_t DS16 = S16 + NJ * DK * 128;         // dS': same
+    static constexpr uint32_t U16 = DS16 + NJ * DK * 128;         // U: NJ tiles of 64 rows (+ one spare tile)
+    static constexpr uint32_t WQ = U16 + NJ * 8192 + 8192;        // record tiles [W; Q~]
+    static constexpr uint32_t U0 = WQ + (DK / 64) * 16384;        // record tiles U0
+    static constexpr uint32_t END = U0 + NJ * 8192;
+    static constexpr uint32_t TX_BYTES = (DK / 64) * 16384 + NJ * 8192 + NJ * 8192;
+    static_assert(END + 1024 <= 232448, "shared memory");
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(256, 1)
+bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsHeader* hdr,
+                    const unsigned char* __restrict__ records, const float* __restrict__ states,
+                    const float* __restrict__ dS_end, const float* __restrict__ dU_all,
+                    float* __restrict__ vside, int H, size_t max_chunks, float scale)
+{
+    using Sm = VsSmem<DK, DV>;
+    using R = TcRec<DK, DV>;
+    using VS = VSide<DK>;
+    constexpr int NJ = DV / 64;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t bar_load, bar_mma;
+    __shared__ uint32_t s_tmem;
+    __shared__ float s_dgam[DK];
+
+    if (hdr->status != kStatusOk) return;
+    const int total = hdr->num_chunks * H;
+    if ((int)blockIdx.x >= total) return;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int lane_row = (warp & 3) * 32 + (tid & 31);   // TMEM lane = MMA row
+    const int wg = warp >> 2;
+    if (tid == 0) {
+        mbar_init(&bar_load, 1);
+        mbar_init(&bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const uint32_t TA = tmem;                 // [W S; Q~ S]: DV columns
+    const uint32_t TB = tmem + DV;            // [dQ~; dW]: DK columns
+    const uint32_t TC = tmem + DV + DK;       // [dK^; *]: DK columns
+    const uint32_t TD = tmem + DV + 2 * DK;   // [dP; *]: 64 columns
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    float range_max = 0.f;
+    uint32_t load_phase = 0, mma_phase = 0;
+    bool aborted = false;
+    int mma_pending = 0;
+
+    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x) {
+        const int c = w / H, h = w - c * H;
+        int seq, tok0, L;
+        map.locate(c, seq, tok0, L);
+        const size_t it = (size_t)h * max_chunks + c;
+        const unsigned char* rec = records + it * R::BYTES;
+        const float* Sn = states + it * DK * DV;
+        const float* dSe = dS_end + it * DK * DV;
+        const float* dUc = dU_all + it * kChunk * DV;
+        float* out = vside + it * VS::FLOATS;
+
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&bar_load, Sm::TX_BYTES);
+            bulk_load(sm + Sm::WQ, rec + R::WQ, R::WQ_BYTES, &bar_load);
+            bulk_load(sm + Sm::U0, rec + R::U0, R::U0_BYTES, &bar_load);
+#pragma unroll
+            for (int b = 0; b < NJ; ++b) tma_load_3d(sm + Sm::AB + b * 16384, &tm_do, &bar_load, b * 64, h, tok0);
+        }
+        if (tid < DK) s_dgam[tid] = 0.f;
+        __syncthreads();
+        // fp16 operands: S and dS' (rows = key channel), -dU (rows 64..127 of [D; -dU]); dgamma
+#pragma unroll 2
+        for (int idx = tid; idx < DK * DV / 8; idx += 256) {
+            const int ch = idx / (DV / 8), j8 = (idx - ch * (DV / 8)) * 8;
+            const float4 s0 = *reinterpret_cast<const float4*>(Sn + (size_t)ch * DV + j8);
+            const float4 s1 = *reinterpret_cast<const float4*>(Sn + (size_t)ch * DV + j8 + 4);
+            const float4 d0 = *reinterpret_cast<const float4*>(dSe + (size_t)ch * DV + j8);
+            const float4 d1 = *reinterpret_cast<const float4*>(dSe + (size_t)ch * DV + j8 + 4);
+            atomicAdd(&s_dgam[ch], s0.x * d0.x + s0.y * d0.y + s0.z * d0.z + s0.w * d0.w +
+                                   s1.x * d1.x + s1.y * d1.y + s1.z * d1.z + s1.w * d1.w);
+            __align__(16) __half2 hs[4] = {__floats2half2_rn(s0.x, s0.y), __floats2half2_rn(s0.z, s0.w),
+                                           __floats2half2_rn(s1.x, s1.y), __floats2half2_rn(s1.z, s1.w)};
+            __align__(16) __half2 hd[4] = {__floats2half2_rn(d0.x, d0.y), __floats2half2_rn(d0.z, d0.w),
+                                           __floats2half2_rn(d1.x, d1.y), __floats2half2_rn(d1.z, d1.w)};
+            range_max = fmaxf(range_max, fmaxf(fmaxf(fabsf(s0.x), fabsf(s0.y)), fmaxf(fabsf(s0.z), fabsf(s0.w))));
+            range_max = fmaxf(range_max, fmaxf(fmaxf(fabsf(s1.x), fabsf(s1.y)), fmaxf(fabsf(s1.z), fabsf(s1.w))));
+            range_max = fmaxf(range_max, fmaxf(fmaxf(fabsf(d0.x), fabsf(d0.y)), fmaxf(fabsf(d0.z), fabsf(d0.w))));
+            range_max = fmaxf(range_max, fmaxf(fmaxf(fabsf(d1.x), fabsf(d1.y)), fmaxf(fabsf(d1.z), fabsf(d1.w))));
+            const uint32_t o = (j8 >> 6) * (DK * 128) + sw128_offset(ch, (j8 & 63) * 2);
+            *reinterpret_cast<uint4*>(sm + Sm::S16 + o) = *reinterpret_cast<const uint4*>(hs);
+            *reinterpret_cast<uint4*>(sm + Sm::DS16 + o) = *reinterpret_cast<const uint4*>(hd);
+        }
+        for (int idx = tid; idx < kChunk * DV / 8; idx += 256) {
+            const int r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
+            const float4 u0 = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8);
+            const float4 u1 = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8 + 4);
+            __align__(16) __half2 hu[4] = {__floats2half2_rn(-u0.x, -u0.y), __floats2half2_rn(-u0.z, -u0.w),
+                                           __floats2half2_rn(-u1.x, -u1.y), __floats2half2_rn(-u1.z, -u1.w)};
+            range_max = fmaxf(range_max, fmaxf(fmaxf(fabsf(u0.x), fabsf(u0.y)), fmaxf(fabsf(u0.z), fabsf(u0.w))));
+            range_max = fmaxf(range_max, fmaxf(fmaxf(fabsf(u1.x), fabsf(u1.y)), fmaxf(fabsf(u1.z), fabsf(u1.w))));
+            *reinterpret_cast<uint4*>(sm + Sm::AB + (j8 >> 6) * 16384 + sw128_offset(64 + r, (j8 & 63) * 2)) =
+                *reinterpret_cast<const uint4*>(hu);
+        }
+        // D = c dO: bf16 -> fp16 in place (rows 0..63 of [D; -dU]); rows past the chunk are zero
+        const bool ok_load = mbar_wait_cycles(&bar_load, load_phase, kWaitCycles);
+        load_phase ^= 1;
+        if (__syncthreads_or(!ok_load)) { aborted = true; break; }
+        for (int idx = tid; idx < kChunk * DV / 8; idx += 256) {
+            const int r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
+            const uint32_t o = Sm::AB + (j8 >> 6) * 16384 + sw128_offset(r, (j8 & 63) * 2);
+            uint4 raw = *reinterpret_cast<const uint4*>(sm + o);
+            if (r >= L) raw = make_uint4(0, 0, 0, 0);
+            const __nv_bfloat162* db = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            __align__(16) __half2 dh[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = __bfloat1622float2(db[e]);
+                range_max = fmaxf(range_max, fmaxf(fabsf(scale * x.x), fabsf(scale * x.y)));
+                dh[e] = __floats2half2_rn(scale * x.x, scale * x.y);
+            }
+            *reinterpret_cast<uint4*>(sm + o) = *reinterpret_cast<const uint4*>(dh);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // [W; Q~] S -> TA and [D; -dU] S^T -> TB
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc_a = instr_desc(kFmtF16, 128, DV, false, true);   // B MN-major
+            constexpr uint32_t idesc_b = instr_desc(kFmtF16, 128, DK, false, false);  // both K-major
+            const uint32_t wq = smem_u32(sm + Sm::WQ), s16 = smem_u32(sm + Sm::S16), ab = smem_u32(sm + Sm::AB);
+#pragma unroll
+            for (int kb = 0; kb < DK / 64; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(TA, smem_desc(wq + kb * 16384 + ks * 32, 16, 1024, kLayoutSW128),
+                            smem_desc(s16 + kb * 8192 + ks * 2048, DK * 128, 1024, kLayoutSW128), idesc_a,
+                            (kb | ks) != 0);
+#pragma unroll
+            for (int kb = 0; kb < NJ; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(TB, smem_desc(ab + kb * 16384 + ks * 32, 16, 1024, kLayoutSW128),
+                            smem_desc(s16 + kb * (DK * 128) + ks * 32, 16, 1024, kLayoutSW128), idesc_b,
+                            (kb | ks) != 0);
+            mma_commit(&bar_mma);
+        }
+        mma_pending = 1;
+        bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        mma_phase ^= 1;
+        mma_pending = 0;
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        tc_fence_after();
+
+        // U = U0 - W S (rows 0..63) -> fp16 U tiles
+        if (lane_row < 64) {
+#pragma unroll 1
+            for (int cb = wg; cb < DV / 32; cb += 2) {
+                float v[32];
+                tmem_ld32_sync(TA + lane_base + 32 * cb, v);
+#pragma unroll
+                for (int i8 = 0; i8 < 4; ++i8) {
+                    const int col = 32 * cb + 8 * i8;
+                    const uint32_t o = (col >> 6) * 8192 + sw128_offset(lane_row, (col & 63) * 2);
+                    const uint4 u0raw = *reinterpret_cast<const uint4*>(sm + Sm::U0 + o);
+                    const __half2* u0 = reinterpret_cast<const __half2*>(&u0raw);
+                    __align__(16) __half2 hv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 u0f = __half22float2(u0[e]);
+                        const float a = u0f.x - v[8 * i8 + 2 * e], b2 = u0f.y - v[8 * i8 + 2 * e + 1];
+                        range_max = fmaxf(range_max, fmaxf(fabsf(a), fabsf(b2)));
+                        hv[e] = __floats2half2_rn(a, b2);
+                    }
+                    *reinterpret_cast<uint4*>(sm + Sm::U16 + o) = *reinterpret_cast<const uint4*>(hv);
+                }
+            }
+        }
+        // [dQ~; dW] out (all 128 lanes)
+#pragma unroll 1
+        for (int cb = wg; cb < DK / 32; cb += 2) {
+            float v[32];
+            tmem_ld32_sync(TB + lane_base + 32 * cb, v);
+            float* dst = lane_row < 64 ? out + VS::DQT + (size_t)lane_row * DK + 32 * cb
+                                       : out + VS::DW + (size_t)(lane_row - 64) * DK + 32 * cb;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // [U; *] dS'^T -> TC and [D; -dU] U^T -> TD
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc_c = instr_desc(kFmtF16, 128, DK, false, false);
+            constexpr uint32_t idesc_d = instr_desc(kFmtF16, 128, 64, false, false);
+            const uint32_t u16 = smem_u32(sm + Sm::U16), ds16 = smem_u32(sm + Sm::DS16), ab = smem_u32(sm + Sm::AB);
+#pragma unroll
+            for (int kb = 0; kb < NJ; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(TC, smem_desc(u16 + kb * 8192 + ks * 32, 16, 1024, kLayoutSW128),
+                            smem_desc(ds16 + kb * (DK * 128) + ks * 32, 16, 1024, kLayoutSW128), idesc_c,
+                            (kb | ks) != 0);
+#pragma unroll
+            for (int kb = 0; kb < NJ; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(TD, smem_desc(ab + kb * 16384 + ks * 32, 16, 1024, kLayoutSW128),
+                            smem_desc(u16 + kb * 8192 + ks * 32, 16, 1024, kLayoutSW128), idesc_d,
+                            (kb | ks) != 0);
+            mma_commit(&bar_mma);
+        }
+        mma_pending = 1;
+        ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        mma_phase ^= 1;
+        mma_pending = 0;
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        tc_fence_after();
+
+        // dK^ and dP (rows 0..63) out; dgamma
+        if (lane_row < 64) {
+#pragma unroll 1
+            for (int cb = wg; cb < DK / 32; cb += 2) {
+                float v[32];
+                tmem_ld32_sync(TC + lane_base + 32 * cb, v);
+                float* dst = out + VS::DKH + (size_t)lane_row * DK + 32 * cb;
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            }
+            {
+                float v[32];
+                tmem_ld32_sync(TD + lane_base + 32 * wg, v);
+                float* dst = out + VS::DP + (size_t)lane_row * kChunk + 32 * wg;
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    const int col = 32 * wg + i;
+                    *reinterpret_cast<float4*>(dst + i) =
+                        make_float4(col <= lane_row ? v[i] : 0.f, col + 1 <= lane_row ? v[i + 1] : 0.f,
+                                    col + 2 <= lane_row ? v[i + 2] : 0.f, col + 3 <= lane_row ? v[i + 3] : 0.f);
+                }
+            }
+        }
+        if (tid < DK) out[VS::DGAM + tid] = s_dgam[tid];
+        tc_fence_before();
+        __syncthreads();   // smem and TMEM are free for the next item
+    }
+
+    if (aborted) {
+        if (tid == 0) flag_error(hdr, kStatusTimeout);
+        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        (void)mbar_wait_cycles(&bar_load, load_phase, kWaitCycles / 4);
+    }
+    if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
 // ------------------------------------------------------------- host -----
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1336,6 +1618,29 @@ cudaError_t launch_bwd_inter_tc_t(const ChunkArgs& a) {
     return cudaGetLastError();
 }
 
+template <int DK, int DV>
+cudaError_t launch_bwd_vside_tc_t(const ChunkArgs& a) {
+    if (a.max_chunks == 0) return cudaSuccess;
+    const int ntok = a.cu_seqlens ? a.T : a.B * a.T;
+    CUtensorMap mdo;
+    if (!make_map(&mdo, a.d_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
+    auto kern = bwd_vside_tc_kernel<DK, DV>;
+    const int smem = (int)VsSmem<DK, DV>::END + 1024;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const size_t items = a.max_chunks * (size_t)a.H;   // upper bound; the kernel reads the exact count
+    const unsigned grid = (unsigned)(items < (size_t)sms ? items : (size_t)sms);
+    kern<<<grid, 256, smem, a.stream>>>(mdo, map, static_cast<WsHeader*>(a.ws_header),
+                                        static_cast<const unsigned char*>(a.records), a.states, a.dS_end, a.dU,
+                                        a.vside, a.H, a.max_chunks, a.scale);
+    return cudaGetLastError();
+}
+
 #define KDA_TC_DISPATCH(FN, a)                                                  \
     do {                                                                       \
         if ((a).dk == 128 && (a).dv == 128) return FN<128, 128>(a);            \
@@ -1363,5 +1668,7 @@ cudaError_t launch_chunk_inter_tc(const ChunkArgs& a) {
 }
 
 cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_inter_tc_t, a); }
+
+cudaError_t launch_chunk_bwd_vside_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_vside_tc_t, a); }
 
 }  // namespace kda

@@ -49,6 +49,20 @@ struct F32Rec {
     static constexpr size_t FLOATS = (GC + DK + 63) / 64 * 64;   // 256-byte multiple
 };
 
+// Backward, per (head, chunk), fp32: the products over the value dimension,
+// dQ~ = D S^T, dW = -dU S^T, dK^ = U dS'^T [64][DK] each, dP = D U^T [64][64]
+// (lower with the diagonal), dgamma [DK].  Written by the tensor-core
+// value-side kernel (bf16 inputs), read by the per-chunk gradient kernel.
+template <int DK>
+struct VSide {
+    static constexpr size_t DQT = 0;
+    static constexpr size_t DW = DQT + kChunk * DK;
+    static constexpr size_t DKH = DW + kChunk * DK;
+    static constexpr size_t DP = DKH + kChunk * DK;
+    static constexpr size_t DGAM = DP + kChunk * kChunk;
+    static constexpr size_t FLOATS = (DGAM + DK + 63) / 64 * 64;
+};
+
 // Element loads/stores for the two input dtypes.
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }

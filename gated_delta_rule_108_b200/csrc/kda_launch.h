@@ -49,6 +49,7 @@ struct ChunkArgs {
     float* dS_end;                // [H][max_chunks][dk][dv]: dL/d(state leaving each chunk)
     float* dU;                    // [H][max_chunks][64][dv]: dL/dU of each chunk
     float* scratch;               // per-CTA fp32 scratch of the per-chunk gradient kernel
+    float* vside;                 // bf16: [H][max_chunks] VSide blocks from the value-side kernel (else null)
     int bwd_ctas;                 // CTAs of that kernel (its scratch holds this many)
     // test hook (kda_debug_drop_copy): the tensor-core intra-chunk kernel leaves
     // out one copy and caps its waits at wait_cap cycles (0: the default cap)
@@ -72,6 +73,7 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a); // bf16 inputs: tensor-co
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K2
 cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a);  // backward: serial over chunks, reversed
 cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a); // the same on the tensor cores (bf16 inputs)
+cudaError_t launch_chunk_bwd_vside_tc(const ChunkArgs& a); // backward products over the value dim (bf16 inputs)
 cudaError_t launch_chunk_bwd_intra(const ChunkArgs& a);  // backward: all chunks in parallel
 size_t bwd_scratch_bytes_per_cta(int dk, int dv);
 constexpr int kBwdMaxCtas = 512;   // scratch is sized for at most this many CTAs
