@@ -15,7 +15,7 @@ namespace {
 
 thread_local std::string g_last_error;
 thread_local long long g_debug_drop_cap = 0;   // armed by kda_debug_drop_copy (one call)
-constexpr int kMaxStageEvents = 6;
+constexpr int kMaxStageEvents = 7;
 thread_local cudaEvent_t g_stage_events[kMaxStageEvents] = {};
 thread_local int g_stage_event_count = 0;   // 0: off
 
@@ -348,7 +348,7 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
     // tensor cores for bf16 inputs, which also write their own fp16 records
     // for their inter-chunk kernel), then the reversed pass over chunks, then
     // the per-chunk gradients
-    const bool marks = g_stage_event_count >= 6;   // the backward records all six or none
+    const bool marks = g_stage_event_count >= 7;   // the backward records all seven or none
     auto mark = [&](int i) { return marks ? mark_stage(i, a.stream) : cudaSuccess; };
     if (a.bf16) a.xrecords = reinterpret_cast<float*>(ws + L.xrec_off);
     e = mark(0);
@@ -368,8 +368,9 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
         if (e == cudaSuccess) e = kda::launch_chunk_bwd_vside_tc(a);
         a.records = a.xrecords;
     }
-    if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);
     if (e == cudaSuccess) e = mark(5);
+    if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);
+    if (e == cudaSuccess) e = mark(6);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_chunk_bwd launch failed: %s", cudaGetErrorString(e));
     return ok();
 }

@@ -249,11 +249,11 @@ kda_status kda_chunk_bwd_gated(const void* q, const void* k, const void* v,
  * (cudaEvent_t passed as void*) on its stream at the stage boundaries:
  * events[0] before the first kernel, events[1] after the chunk-table/status
  * kernel, events[2] after the intra-chunk stage, events[3] after the
- * inter-chunk stage.  With `count` >= 6, each later kda_chunk_bwd records
- * events[0] before its first kernel and events[1..5] after the chunk-table,
- * forward intra-chunk, forward inter-chunk and reversed inter-chunk kernels
- * and after the per-chunk gradient kernels (with bf16 inputs: the value-side
- * products and the rest).  `count` must be >= 4 (only the first 6 are used).  Pass
+ * inter-chunk stage.  With `count` >= 7, each later kda_chunk_bwd records
+ * events[0] before its first kernel and events[1..6] after the chunk-table,
+ * forward intra-chunk, forward inter-chunk, reversed inter-chunk, value-side
+ * (bf16 inputs; an empty stage for fp32) and per-chunk gradient kernels.
+ * `count` must be >= 4 (only the first 7 are used).  Pass
  * NULL to stop.  Recording an event costs a few microseconds of stream time
  * and changes no result.
  */
