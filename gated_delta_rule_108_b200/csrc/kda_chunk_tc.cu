@@ -1333,15 +1333,21 @@ bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsH
         if (tid < DK) s_dgam[tid] = 0.f;
         __syncthreads();
         // fp16 operands: S and dS' (rows = key channel), -dU (rows 64..127 of [D; -dU]); dgamma
-#pragma unroll 2
+        // DV / 8 consecutive threads share a key row: their dgamma parts are
+        // summed by shuffles, then added once (DV / 8 divides 32)
+        static_assert(32 % (DV / 8) == 0, "row groups within a warp");
+#pragma unroll 4
         for (int idx = tid; idx < DK * DV / 8; idx += 256) {
             const int ch = idx / (DV / 8), j8 = (idx - ch * (DV / 8)) * 8;
             const float4 s0 = *reinterpret_cast<const float4*>(Sn + (size_t)ch * DV + j8);
             const float4 s1 = *reinterpret_cast<const float4*>(Sn + (size_t)ch * DV + j8 + 4);
             const float4 d0 = *reinterpret_cast<const float4*>(dSe + (size_t)ch * DV + j8);
             const float4 d1 = *reinterpret_cast<const float4*>(dSe + (size_t)ch * DV + j8 + 4);
-            atomicAdd(&s_dgam[ch], s0.x * d0.x + s0.y * d0.y + s0.z * d0.z + s0.w * d0.w +
-                                   s1.x * d1.x + s1.y * d1.y + s1.z * d1.z + s1.w * d1.w);
+            float gpart = s0.x * d0.x + s0.y * d0.y + s0.z * d0.z + s0.w * d0.w +
+                          s1.x * d1.x + s1.y * d1.y + s1.z * d1.z + s1.w * d1.w;
+#pragma unroll
+            for (int off = DV / 16; off; off >>= 1) gpart += __shfl_xor_sync(0xffffffffu, gpart, off);
+            if ((tid & (DV / 8 - 1)) == 0) atomicAdd(&s_dgam[ch], gpart);
             __align__(16) __half2 hs[4] = {__floats2half2_rn(s0.x, s0.y), __floats2half2_rn(s0.z, s0.w),
                                            __floats2half2_rn(s1.x, s1.y), __floats2half2_rn(s1.z, s1.w)};
             __align__(16) __half2 hd[4] = {__floats2half2_rn(d0.x, d0.y), __floats2half2_rn(d0.z, d0.w),
@@ -1354,6 +1360,7 @@ bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsH
             *reinterpret_cast<uint4*>(sm + Sm::S16 + o) = *reinterpret_cast<const uint4*>(hs);
             *reinterpret_cast<uint4*>(sm + Sm::DS16 + o) = *reinterpret_cast<const uint4*>(hd);
         }
+#pragma unroll 4
         for (int idx = tid; idx < kChunk * DV / 8; idx += 256) {
             const int r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
             const float4 u0 = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8);
