@@ -149,3 +149,23 @@ def test_chunk_bwd_gates(cuda_device, dtype, gate):
         check(got["dlog_alpha"], ref["dlog_alpha"].sum(-1), dtype, "head dlog_alpha")
     else:
         assert got["dlog_alpha"] is None
+
+
+def test_chunk_bwd_c4_varlen_sampled(cuda_device):
+    """The packed varlen workload (16 sequences of 1,024..16,384 tokens, H=32,
+    bf16, 10% beta = 1 and 10% beta = 0): the backward of the whole pack on the
+    GPU; the shortest and the longest sequence, one head each, against the oracle."""
+    w = I.workload("C4")
+    x = I.chunk_inputs(w)
+    d_o, dSf = cotangents(x, 570)
+    got = run_bwd(x, d_o, dSf)
+    cu = x["cu_seqlens"].tolist()
+    lens = [cu[i + 1] - cu[i] for i in range(len(cu) - 1)]
+    for s, h in ((lens.index(min(lens)), 3), (lens.index(max(lens)), 29)):
+        a, b = cu[s], cu[s + 1]
+        xs = {k: x[k][:, a:b, h:h + 1].contiguous() for k in ("q", "k", "v", "log_alpha", "beta")}
+        xs["initial_state"] = x["initial_state"][s:s + 1, h:h + 1].contiguous()
+        xs["cu_seqlens"] = None
+        ref = oracle_bwd(xs, d_o[:, a:b, h:h + 1].contiguous(), dSf[s:s + 1, h:h + 1].contiguous())
+        part = {n: (got[n][:, a:b, h:h + 1] if n != "dS0" else got[n][s:s + 1, h:h + 1]) for n in GRADS}
+        check_all(part, ref, torch.bfloat16, f"C4 seq {s} (len {b - a}) head {h}")
