@@ -72,11 +72,10 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
 }
 
 // Backward workspace: [header][chunk_offsets][the forward's records][bf16
-// inputs: fp32 records][T][chunk-start states][dS at chunk ends][dU][per-CTA
-// scratch], each 256-byte aligned.
+// inputs: the value-side products][T][chunk-start states][dS at chunk ends]
+// [dU][per-CTA scratch], each 256-byte aligned.
 struct BwdLayout {
     WsLayout base;   // header, offsets, the forward's records for this dtype
-    size_t xrec_off; // bf16: fp32 records written by the tensor-core K1 (0 for fp32)
     size_t vside_off;// bf16: the value-side products per (head, chunk) (0 for fp32)
     size_t tmat_off, states_off, dS_off, dU_off, scratch_off, total;
     int ctas;        // CTAs the scratch holds
@@ -87,11 +86,8 @@ bool bwd_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, 
     if (!ws_layout(B, T, H, dk, dv, num_seqs, varlen, dtype, L.base)) return false;
     const size_t units = (size_t)H * L.base.max_chunks;   // (head, chunk) pairs
     size_t off = round_up(L.base.total, 256);
-    L.xrec_off = 0;
     L.vside_off = 0;
     if (dtype == KDA_BF16) {
-        L.xrec_off = off;
-        off = round_up(off + kda::simt_record_bytes(dk, dv) * units, 256);
         L.vside_off = off;
         const size_t vs_floats = dk == 128 ? kda::VSide<128>::FLOATS : kda::VSide<64>::FLOATS;
         off = round_up(off + sizeof(float) * vs_floats * units, 256);
@@ -344,13 +340,12 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "device query failed: %s", cudaGetErrorString(e));
     a.bwd_ctas = L.ctas < 2 * sms ? L.ctas : 2 * sms;   // two resident per SM
 
-    // forward recomputation (fp32 records + T + chunk-start states: on the
-    // tensor cores for bf16 inputs, which also write their own fp16 records
-    // for their inter-chunk kernel), then the reversed pass over chunks, then
-    // the per-chunk gradients
+    // forward recomputation (the records, T and the chunk-start states: fp16
+    // records on the tensor cores for bf16 inputs, fp32 ones on CUDA cores for
+    // fp32 inputs), then the reversed pass over chunks, then the per-chunk
+    // gradients
     const bool marks = g_stage_event_count >= 7;   // the backward records all seven or none
     auto mark = [&](int i) { return marks ? mark_stage(i, a.stream) : cudaSuccess; };
-    if (a.bf16) a.xrecords = reinterpret_cast<float*>(ws + L.xrec_off);
     e = mark(0);
     if (e == cudaSuccess) e = kda::launch_chunk_prep(a);
     if (e == cudaSuccess) e = mark(1);
@@ -360,13 +355,12 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
     if (e == cudaSuccess) e = mark(3);
     // the reversed chain reads the fp16 tensor-core records (bf16) or the fp32
     // ones; for bf16 the products over the value dimension are formed on the
-    // tensor cores too; the per-chunk gradient kernel reads the fp32 records
+    // tensor cores too, and the per-chunk gradient kernel reads no record
     if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_bwd_inter_tc(a) : kda::launch_chunk_bwd_inter(a);
     if (e == cudaSuccess) e = mark(4);
     if (a.bf16) {
         a.vside = reinterpret_cast<float*>(ws + L.vside_off);
         if (e == cudaSuccess) e = kda::launch_chunk_bwd_vside_tc(a);
-        a.records = a.xrecords;
     }
     if (e == cudaSuccess) e = mark(5);
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);

@@ -97,8 +97,7 @@ constexpr int kCopyThread = 32;   // the intra-chunk kernel's TMA / bulk-copy th
 // per (r, i) pair, lanes over channels; k and q are the bf16 tiles as loaded.
 template <int DK>
 __device__ __forceinline__ void exact_a_p(const float* g, const unsigned char* ks, const unsigned char* qs,
-                                          const float* s_beta, int L, float* am, unsigned char* prec,
-                                          float* xp)
+                                          const float* s_beta, int L, float* am, unsigned char* prec)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int pr = warp; pr < 64 * 64; pr += 8) {
@@ -126,7 +125,6 @@ __device__ __forceinline__ void exact_a_p(const float* g, const unsigned char* k
         if (lane == 0) {
             am[r * 68 + i] = (i < r) ? s_beta[r] * sa : 0.f;
             *reinterpret_cast<__half*>(prec + sw128_offset(r, i * 2)) = __float2half_rn(sp);
-            if (xp) xp[r * 64 + i] = sp;   // fp32 record (backward mode)
         }
     }
 }
@@ -183,12 +181,10 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                       const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_la,
                       const float* __restrict__ log_alpha_head, const float* __restrict__ beta,
                       ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
-                      size_t max_chunks, long long wait_cap, int drop_first_la,
-                      float* __restrict__ xrecords, float* __restrict__ tmat)
+                      size_t max_chunks, long long wait_cap, int drop_first_la, float* __restrict__ tmat)
 {
     using Sm = K1Smem<DK, DV>;
     using R = TcRec<DK, DV>;
-    using XR = F32Rec<DK, DV>;
     constexpr int NPART = 256 / DK;       // threads per key channel in the cumulative sum
     constexpr int TPP = kChunk / NPART;   // tokens per such thread
     constexpr int NCH8 = DK / 8;          // 8-channel (16-byte bf16) groups per token row
@@ -295,8 +291,6 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         int c, h, tok0, L;
         locate(w, c, h, tok0, L);
         unsigned char* rec = records + ((size_t)h * max_chunks + c) * R::BYTES;
-        // backward mode: the same quantities in fp32 (F32Rec layout) and T itself
-        float* xr = xrecords ? xrecords + ((size_t)h * max_chunks + c) * XR::FLOATS : nullptr;
         if (tid >= 192) {
             s_beta[tid - 192] = beta_next;
             if constexpr (GATE == kGateHead) s_lah[tid - 192] = lah_next;
@@ -338,7 +332,6 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             s_egm[tid] = ex2_approx(gm);
             s_eglm[tid] = ex2_approx(gl - gm);
             reinterpret_cast<float*>(rec + R::GC)[tid] = exp2f(gl);
-            if (xr) xr[XR::GC + tid] = exp2f(gl);
             wide = fmaxf(g[tid] - gm, gm - gl) > kMaxSplitExponent2;
         }
         // Strong decay: the factors e^{+-(g - g_m)} of A and P could overflow, so
@@ -346,7 +339,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         const bool strong = __syncthreads_or(wide);
         if (strong) {
             float* am = reinterpret_cast<float*>(sm + Sm::AM);
-            exact_a_p<DK>(g, st + Sm::KS, st + Sm::QS, s_beta, L, am, rec + R::P, xr ? xr + XR::P : nullptr);
+            exact_a_p<DK>(g, st + Sm::KS, st + Sm::QS, s_beta, L, am, rec + R::P);
             __syncthreads();   // the k, q tiles are converted in place next
         }
 
@@ -412,11 +405,6 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                     k0[e2] = __floats2half2_rn(k0v[0], k0v[1]);
                     q0[e2] = __floats2half2_rn(q0v[0], q0v[1]);
                     kh[e2] = __floats2half2_rn(khv[0], khv[1]);
-                    if (xr) {   // fp32 Q~ and K^ (rows past the chunk are zero)
-                        const size_t o2 = (size_t)r * DK + c8 + 2 * e2;
-                        *reinterpret_cast<float2*>(xr + XR::QT + o2) = make_float2(q0v[0], q0v[1]);
-                        *reinterpret_cast<float2*>(xr + XR::KH + o2) = make_float2(khv[0], khv[1]);
-                    }
                 }
                 // tf32 operands: 8 fp32 = two 16-byte chunks of a 128-byte row
                 const uint32_t fo = (c8 >> 5) * 16384u, fob = (c8 >> 5) * 8192u;
@@ -532,15 +520,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                     *reinterpret_cast<uint4*>(rec + R::P + sw128_offset(r, (32 * wg + 8 * i8) * 2)) =
                         *reinterpret_cast<const uint4*>(hv);
                 }
-                if (xr) {   // fp32 P
-#pragma unroll
-                    for (int i4 = 0; i4 < 8; ++i4) {
-                        const int col = 32 * wg + 4 * i4;
-                        *reinterpret_cast<float4*>(xr + XR::P + r * 64 + col) =
-                            make_float4(col <= r ? v[4 * i4] : 0.f, col + 1 <= r ? v[4 * i4 + 1] : 0.f,
-                                        col + 2 <= r ? v[4 * i4 + 2] : 0.f, col + 3 <= r ? v[4 * i4 + 3] : 0.f);
-                    }
-                }
+
             }
         }
         }   // !strong
@@ -669,13 +649,6 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             for (int cb = wg; cb < (DK + DV) / 32; cb += 2) {
                 float v[32];
                 tmem_ld32_sync(R2 + lane_base + 32 * cb, v);
-                if (xr) {   // fp32 W | U0
-                    float* dst = 32 * cb < DK ? xr + XR::W + (size_t)r * DK + 32 * cb
-                                              : xr + XR::U0 + (size_t)r * DV + (32 * cb - DK);
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                }
 #pragma unroll
                 for (int i8 = 0; i8 < 4; ++i8) {
                     __align__(16) __half hv[8];
@@ -1586,8 +1559,7 @@ cudaError_t launch_intra_tc_t(const ChunkArgs& a) {
     kern<<<grid, 256, smem, a.stream>>>(mk, mv, mq, mla, a.log_alpha, a.beta, map,
                                         static_cast<WsHeader*>(a.ws_header),
                                         static_cast<unsigned char*>(a.records), a.H, a.max_chunks,
-                                        a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy,
-                                        a.xrecords, a.tmat);
+                                        a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy, a.tmat);
     return cudaGetLastError();
 }
 

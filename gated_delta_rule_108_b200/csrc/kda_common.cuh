@@ -35,9 +35,8 @@ static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
 
 // fp32 record of one (head, chunk), row-major: W [64][DK] | U0 [64][DV] |
 // Q~ [64][DK] | K^ [64][DK] | P [64][64] | gamma [DK].  Rows past the chunk's
-// tokens are zero.  Written by the CUDA-core intra-chunk kernel (fp32 inputs)
-// or by the tensor-core one in its backward mode; read by the CUDA-core
-// inter-chunk kernel and the backward kernels.
+// tokens are zero.  Written by the CUDA-core intra-chunk kernel (fp32 inputs);
+// read by the CUDA-core inter-chunk kernel and the fp32 backward kernels.
 template <int DK, int DV>
 struct F32Rec {
     static constexpr size_t W = 0;

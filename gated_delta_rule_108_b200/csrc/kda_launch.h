@@ -39,7 +39,6 @@ struct ChunkArgs {
     cudaStream_t stream;
     // backward pass only (all null in the forward)
     float* tmat;                  // [H][max_chunks][64][64]: K1 also writes T = (I + A)^{-1}
-    float* xrecords;              // bf16 inputs: the tensor-core K1 also writes fp32 records (F32Rec) here
     float* states;                // [H][max_chunks][dk][dv]: K2 also writes the state entering each chunk
     const void* d_o;              // [.., H, dv], input dtype
     const float* d_final_state;   // [N, H, dk, dv], nullable (zeros)

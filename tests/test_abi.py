@@ -144,6 +144,12 @@ def test_chunk_bwd_rejects(lib, over, status):
     assert lib.kda_last_error()
 
 
+def lib_simt_record_bytes(dk, dv):
+    """fp32 record bytes per (chunk, head): W, U0, Q~, K^, P, gamma, 256-byte padded."""
+    floats = 64 * (3 * dk + dv + 64) + dk
+    return (floats + 63) // 64 * 64 * 4
+
+
 def test_bwd_workspace_size(lib):
     f32, bf16 = 0, 1
     fwd = lib.kda_chunk_fwd_workspace_size(4, 4096, 16, 128, 128, 4, 0, f32)
@@ -151,9 +157,11 @@ def test_bwd_workspace_size(lib):
     units = 4 * 64 * 16
     # records + T + two state-sized buffers per (head, chunk) + dU
     assert bwd >= fwd + units * 4 * (64 * 64 + 2 * 128 * 128 + 64 * 128)
-    # bf16 inputs recompute on the tensor cores: their fp16 records (74,240 B per
-    # (chunk, head) at d = 128) on top of the fp32 ones
-    assert lib.kda_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 4, 0, bf16) >= bwd + units * 74240
+    # bf16 inputs: fp16 records (74,240 B per (chunk, head) at d = 128) instead of
+    # fp32 ones, plus the value-side products (3 x 64 x 128 + 64 x 64 + 128 fp32)
+    vs = 4 * (3 * 64 * 128 + 64 * 64 + 128)
+    assert lib.kda_chunk_bwd_workspace_size(4, 4096, 16, 128, 128, 4, 0, bf16) >= (
+        bwd - units * lib_simt_record_bytes(128, 128) + units * (74240 + vs))
     assert lib.kda_chunk_bwd_workspace_size(1, 100, 2, 96, 64, 1, 0, f32) == 0
 
 
