@@ -217,16 +217,20 @@ def bench_chunk(args, dev, world, rank):
 
 def chunk_bwd_simt_flops_per_chunk_head(dk, dv, C=64):
     """FLOPs (2 x multiply-adds) of the CUDA-core per-chunk gradient kernel once
-    the value-side products are formed on the tensor cores: Z (C C dv), Y, M,
-    dKl, dQl (C C dk), dT (C C (dk + dv)), dKr (2 C C dk), dT T^T and T^T X (C^3)."""
-    return 2 * (C * C * (2 * dv + 7 * dk) + 2 * C ** 3)
+    the value-side and T-chain products are formed on the tensor cores: M, dKl,
+    dQl (C C dk each) and dKr (2 C C dk)."""
+    return 2 * 5 * C * C * dk
 
 
-def chunk_bwd_vside_bytes_per_chunk_head(dk, dv, C=64):
-    """Algorithmic bytes of the value-side kernel: reads S, dS' (fp32 dk x dv),
-    dU (fp32 C x dv), d_o (bf16 C x dv), the fp16 W, Q~, U0 tiles; writes dQ~, dW,
-    dK^ (fp32 C x dk), dP (fp32 C x C) and dgamma (fp32 dk)."""
-    return 2 * 4 * dk * dv + 4 * C * dv + 2 * C * dv + 2 * (2 * C * dk + C * dv) + 4 * (3 * C * dk + C * C + dk)
+def chunk_bwd_tc_bytes_per_chunk_head(dk, dv, C=64):
+    """Algorithmic bytes of the two tensor-core product kernels.  Value side:
+    reads S, dS' (fp32 dk x dv), dU (fp32 C x dv), d_o (bf16 C x dv), the fp16 W,
+    Q~, U0 tiles; writes dQ~, dW, dK^ (fp32 C x dk), dP (fp32 C x C), dgamma.
+    T-chain: reads the fp16 T, K~, V tiles, dU (fp32 C x dv), dW (fp32 C x dk),
+    beta; writes dv (bf16 C x dv), dK~ (fp32 C x dk), dA (fp32 C x C), dbeta parts."""
+    vside = 2 * 4 * dk * dv + 4 * C * dv + 2 * C * dv + 2 * (2 * C * dk + C * dv) + 4 * (3 * C * dk + C * C + dk)
+    tchain = 2 * (C * C + C * dk + C * dv) + 4 * C * dv + 4 * C * dk + 4 * C + 2 * C * dv + 4 * (C * dk + C * C + C)
+    return vside + tchain
 
 
 def bench_backward(args, dev, world, rank):
@@ -270,10 +274,10 @@ def bench_backward(args, dev, world, rank):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(start.elapsed_time(end), world, dev) / steps
-    names = ("chunk_prep", "fwd_intra_chunk", "fwd_inter_chunk", "bwd_inter_chunk", "bwd_value_side",
+    names = ("chunk_prep", "fwd_intra_chunk", "fwd_inter_chunk", "bwd_inter_chunk", "bwd_tc_products",
              "bwd_intra_chunk")
     stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i, n in enumerate(names)}
-    return dict(w=w, ms_per_step=ms, stages=stages, launches=(6 if w.dtype == torch.bfloat16 else 5) * steps)
+    return dict(w=w, ms_per_step=ms, stages=stages, launches=(7 if w.dtype == torch.bfloat16 else 5) * steps)
 
 
 def bench_decode(args, dev, world, rank):
@@ -453,8 +457,8 @@ def run_ours(args):
         bw = bwd["w"]
         n_ch = bw.num_seqs * ((bw.T + 63) // 64) * bw.H
         bflops = chunk_bwd_simt_flops_per_chunk_head(bw.dk, bw.dv) * n_ch
-        vbytes = chunk_bwd_vside_bytes_per_chunk_head(bw.dk, bw.dv) * n_ch
-        vms = bwd["stages"]["bwd_value_side"]
+        vbytes = chunk_bwd_tc_bytes_per_chunk_head(bw.dk, bw.dv) * n_ch
+        vms = bwd["stages"]["bwd_tc_products"]
         bms = bwd["stages"]["bwd_intra_chunk"]
         btf = bflops / (bms / 1e3) / 1e12
         alu_peak = FP32_SIMT_TFLOPS
@@ -468,7 +472,7 @@ def run_ours(args):
                          "unit": "TFLOP/s", "frac": btf / alu_peak, "traffic": traffic_for("bwd_intra_chunk"),
                          "peak_source": "derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1.965 GHz",
                          "algorithmic_flops_per_launch": bflops, "ms_per_launch": bms},
-            "value_side_roofline": {"kernel": "bwd_vside_tc", "bound": "hbm",
+            "tc_products_roofline": {"kernel": "bwd_vside_tc + bwd_tchain_tc", "bound": "hbm",
                                     "achieved": vbytes / (vms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
                                     "frac": vbytes / (vms / 1e3) / 1e9 / hbm,
                                     "algorithmic_bytes_per_launch": vbytes, "ms_per_launch": vms},

@@ -72,11 +72,13 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
 }
 
 // Backward workspace: [header][chunk_offsets][the forward's records][bf16
-// inputs: the value-side products][T][chunk-start states][dS at chunk ends]
-// [dU][per-CTA scratch], each 256-byte aligned.
+// inputs: the tensor-core products, fp16 T / K~ / V tiles; fp32 inputs: T]
+// [chunk-start states][dS at chunk ends][dU][per-CTA scratch], each 256-byte
+// aligned.
 struct BwdLayout {
     WsLayout base;   // header, offsets, the forward's records for this dtype
-    size_t vside_off;// bf16: the value-side products per (head, chunk) (0 for fp32)
+    size_t vside_off;// bf16: the tensor-core products per (head, chunk) (0 for fp32)
+    size_t tiles_off;// bf16: fp16 T, K~, V tiles per (head, chunk) (0 for fp32)
     size_t tmat_off, states_off, dS_off, dU_off, scratch_off, total;
     int ctas;        // CTAs the scratch holds
 };
@@ -87,13 +89,20 @@ bool bwd_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, 
     const size_t units = (size_t)H * L.base.max_chunks;   // (head, chunk) pairs
     size_t off = round_up(L.base.total, 256);
     L.vside_off = 0;
+    L.tiles_off = 0;
+    L.tmat_off = 0;
     if (dtype == KDA_BF16) {
         L.vside_off = off;
         const size_t vs_floats = dk == 128 ? kda::VSide<128>::FLOATS : kda::VSide<64>::FLOATS;
         off = round_up(off + sizeof(float) * vs_floats * units, 256);
+        L.tiles_off = off;
+        off = round_up(off + (size_t)8192 * (1 + dk / 64 + dv / 64) * units, 256);   // fp16 T, K~, V tiles
+    } else {
+        L.tmat_off = off;
+        off = round_up(off + sizeof(float) * kda::kChunk * kda::kChunk * units, 256);
     }
-    L.tmat_off = off;
-    L.states_off = round_up(L.tmat_off + sizeof(float) * kda::kChunk * kda::kChunk * units, 256);
+    const size_t after_t = off;
+    L.states_off = after_t;
     L.dS_off = round_up(L.states_off + sizeof(float) * (size_t)dk * dv * units, 256);
     L.dU_off = round_up(L.dS_off + sizeof(float) * (size_t)dk * dv * units, 256);
     L.scratch_off = round_up(L.dU_off + sizeof(float) * kda::kChunk * (size_t)dv * units, 256);
@@ -326,7 +335,8 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
     a.max_chunks = L.base.max_chunks;
     a.fixed_chunks_per_seq = L.base.chunks_per_seq;
     a.stream = static_cast<cudaStream_t>(stream);
-    a.tmat = reinterpret_cast<float*>(ws + L.tmat_off);
+    a.tmat = a.bf16 ? nullptr : reinterpret_cast<float*>(ws + L.tmat_off);
+    a.bwd_tiles = a.bf16 ? static_cast<void*>(ws + L.tiles_off) : nullptr;
     a.states = reinterpret_cast<float*>(ws + L.states_off);
     a.d_o = d_o; a.d_final_state = d_final_state;
     a.dq = dq; a.dk_out = dk_out; a.dv_out = dv_out;
@@ -361,6 +371,7 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
     if (a.bf16) {
         a.vside = reinterpret_cast<float*>(ws + L.vside_off);
         if (e == cudaSuccess) e = kda::launch_chunk_bwd_vside_tc(a);
+        if (e == cudaSuccess) e = kda::launch_chunk_bwd_tchain_tc(a);
     }
     if (e == cudaSuccess) e = mark(5);
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);

@@ -452,7 +452,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         } else if (tid >= 128 && tid < 128 + kChunk) {
             const int r = tid - 128;
             sm.beta[r] = (r < L) ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
-            sm.dbeta[r] = 0.f;
+            sm.dbeta[r] = vs ? vs[VSide<DK>::DBP + r] : 0.f;   // the parts through W, U0 when precomputed
         }
         __syncthreads();
         bool wide = false;
@@ -483,13 +483,13 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                 scr[C::KL + idx] = kk;
                 scr[C::QL + idx] = qq;
             }
-            scr[C::KT + idx] = kk * expf(gg);
+            if (!vs) scr[C::KT + idx] = kk * expf(gg);
         }
 #pragma unroll 4
         for (int idx = tid; idx < kChunk * DV; idx += 256) {
             const int r = idx / DV, j = idx - r * DV;
             const size_t off = (size_t)(tok0 + r) * rowv + (size_t)h * DV + j;
-            scr[C::VV + idx] = (r < L) ? to_f32(v[off]) : 0.f;
+            if (!vs) scr[C::VV + idx] = (r < L) ? to_f32(v[off]) : 0.f;
             if (!vs) scr[C::DO + idx] = (r < L) ? scale * to_f32(d_o[off]) : 0.f;
         }
         // dgamma_c = sum_j dS'_cj S_cj: one warp per key row
@@ -538,6 +538,8 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
         }
         }   // !vs
         // ---- through W = T diag(beta) K~ and U0 = T diag(beta) V -------------
+        // (precomputed on the tensor cores for bf16 inputs: dv, dK~, dA, dbeta parts)
+        if (!vs) {
         {   // Z = T^T dU: dv = beta Z, dbeta += <Z, v>
             float acc[4][DV / 16];
             zero_acc<DV>(acc);
@@ -581,6 +583,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             gemm64<kChunk>(acc, Mat{scr + C::DT, kChunk, false}, Mat{Tm, kChunk, true}, kChunk, sm.st);
             for_acc<kChunk>(acc, [&](int r, int i, float x) { scr[C::X1 + r * kChunk + i] = x; });
         }
+        }   // !vs
         // ---- M = Kl Kr^T (the unweighted A), strictly lower -------------------
         if (!strong) {
             float acc[4][kChunk / 16];
@@ -600,7 +603,21 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                 if (lane == 0) scr[C::M + pr] = acc;
             }
         }
-        {   // dA = -T^T X1 (strictly lower); dbeta += rowsum(dA M); dM = diag(beta) dA
+        if (vs) {   // dA precomputed: dbeta += rowsum(dA M); dM = diag(beta) dA (one warp per row)
+            __syncthreads();   // M complete
+            for (int r = warp; r < kChunk; r += 8) {
+                float part = 0.f;
+#pragma unroll
+                for (int i = lane; i < kChunk; i += 32) {
+                    const float da = vs[VSide<DK>::DA + r * kChunk + i];
+                    part += da * scr[C::M + r * kChunk + i];
+                    scr[C::DM + r * kChunk + i] = sm.beta[r] * da;
+                }
+#pragma unroll
+                for (int off = 16; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+                if (lane == 0) sm.dbeta[r] += part;
+            }
+        } else {   // dA = -T^T X1 (strictly lower); dbeta += rowsum(dA M); dM = diag(beta) dA
             float acc[4][kChunk / 16];
             zero_acc<kChunk>(acc);
             gemm64<kChunk>(acc, Mat{Tm, kChunk, true}, Mat{scr + C::X1, kChunk, false}, kChunk, sm.st);
@@ -679,7 +696,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
             const float gg = sm.g[r][ch];
             const float eg = expf(gg), eh = expf(sm.gl[ch] - gg);
             const float dkl = scr[C::DKL + idx], dkr = scr[C::DKR + idx], dql = scr[C::DQL + idx];
-            const float dkt = scr[C::DKT + idx], dkh = pDKH[idx], dqt = pDQT[idx];
+            const float dkt = vs ? vs[VSide<DK>::DKT + idx] : scr[C::DKT + idx], dkh = pDKH[idx], dqt = pDQT[idx];
             if (r < L) {
                 dk[off] = from_f32<T>(dkl + dkr + dkt * eg + dkh * eh);
                 dq[off] = from_f32<T>(dql + dqt * eg);

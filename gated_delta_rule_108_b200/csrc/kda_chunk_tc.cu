@@ -83,12 +83,24 @@ struct TcRec {
 };
 
 
+// Backward mode of the intra-chunk kernel, per (head, chunk): T = (I + A)^{-1},
+// K~ = k e^{g} and V as fp16 128-byte-swizzled tiles of 64 rows (token) by 64
+// columns, the operands of the backward's T-chain products.
+template <int DK, int DV>
+struct BwdTiles {
+    static constexpr uint32_t T = 0;
+    static constexpr uint32_t KT = T + 8192;
+    static constexpr uint32_t V = KT + (DK / 64) * 8192;
+    static constexpr uint32_t BYTES = V + (DV / 64) * 8192;
+};
+
 constexpr float kMaxSplitExponent = 60.f;   // e^60 ~ 1e26: far inside the fp32 range
 // The intra-chunk kernel keeps the cumulative log-decay in base 2 (g log2(e)),
 // so each factor e^{x} is one hardware 2^{x}.
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kMaxSplitExponent2 = kMaxSplitExponent * kLog2e;
-constexpr int kCopyThread = 32;   // the intra-chunk kernel's TMA / bulk-copy thread (warp 1)
+constexpr int kCopyThread = 32;     // the intra-chunk kernel's TMA / bulk-copy thread (warp 1)
+constexpr int kTileThread = 128;    // its backward-mode tile stores (warp 4, idle in the diagonal solve)
 
 // Exact A and P of one chunk, used when its decay is too strong for the split
 // factors (g in base 2): A_ri = beta_r sum_c k_rc k_ic e^{g_rc - g_ic} (i < r) into am
@@ -181,7 +193,8 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                       const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_la,
                       const float* __restrict__ log_alpha_head, const float* __restrict__ beta,
                       ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
-                      size_t max_chunks, long long wait_cap, int drop_first_la, float* __restrict__ tmat)
+                      size_t max_chunks, long long wait_cap, int drop_first_la,
+                      unsigned char* __restrict__ bwd_tiles)
 {
     using Sm = K1Smem<DK, DV>;
     using R = TcRec<DK, DV>;
@@ -282,6 +295,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
     uint32_t mma_phase = 0;
     int mma_pending = 0;      // commits issued on bar_mma not yet waited for
     bool stored = false;      // the copy thread has bulk stores in flight
+    bool tstored = false;     // kTileThread has bulk stores in flight (backward mode)
     float range_max = 0.f;
 
     int it = 0;
@@ -525,6 +539,15 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         }
         }   // !strong
         __syncthreads();
+        unsigned char* btile = bwd_tiles ? bwd_tiles + ((size_t)h * max_chunks + c) * BwdTiles<DK, DV>::BYTES : nullptr;
+        if (btile && tid == kTileThread) {   // backward mode: K~ and fp16 V are final
+#pragma unroll
+            for (int b = 0; b < DK / 64; ++b) bulk_store(btile + BwdTiles<DK, DV>::KT + b * 8192, st + Sm::KS + b * Sm::TILE, 8192);
+#pragma unroll
+            for (int b = 0; b < DV / 64; ++b) bulk_store(btile + BwdTiles<DK, DV>::V + b * 8192, st + Sm::VS + b * Sm::TILE, 8192);
+            bulk_store_commit();
+            tstored = true;
+        }
 
         // ---- T = (I + A)^{-1} in 16 x 16 blocks, written as fp16 T diag(beta)
         //      (K-major, rows 0..63) as soon as each block is final.
@@ -627,12 +650,18 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             mma_commit(&bar_mma);
         }
         mma_pending = 1;
-        if (tmat) {   // backward mode: T = (I + A)^{-1} (zero above the diagonal blocks)
-            float* tm = tmat + ((size_t)h * max_chunks + c) * kChunk * kChunk;
-            for (int idx = tid; idx < kChunk * kChunk; idx += 256) {
-                const int r = idx >> 6, cc = idx & 63;
-                tm[idx] = ((cc >> 4) > (r >> 4)) ? 0.f : tmx[r * 68 + cc];
+        if (btile) {   // backward mode: T = (I + A)^{-1} as an fp16 tile (zero above the diagonal blocks)
+            for (int idx = tid; idx < kChunk * 8; idx += 256) {
+                const int r = idx >> 3, c8 = (idx & 7) * 8;
+                __align__(16) __half hv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    hv[e] = __float2half_rn(((c8 + e) >> 4) > (r >> 4) ? 0.f : tmx[r * 68 + c8 + e]);
+                *reinterpret_cast<uint4*>(btile + BwdTiles<DK, DV>::T + sw128_offset(r, c8 * 2)) =
+                    *reinterpret_cast<const uint4*>(hv);
             }
+            // the K~ / V tile stores must have read the stage before W, U0 are staged there
+            if (tid == kTileThread) bulk_store_wait_read();
         }
         ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
@@ -682,7 +711,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         if constexpr (channel_gate) (void)mbar_wait_cycles(&bar_la, 0, wait_cap / 4);
         if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
     }
-    if (stored) bulk_store_wait_all();
+    if (stored || tstored) bulk_store_wait_all();
     if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
     tc_fence_before();
     __syncthreads();
@@ -1505,6 +1534,290 @@ bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsH
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// ------------------------------------------------ backward T-chain (bf16) ----
+// The products of the backward through W = T diag(beta) K~, U0 = T diag(beta) V
+// and T = (I + A)^{-1} on the tensor cores (bf16 inputs), one (chunk, head) at
+// a time per CTA:
+//     [Z | Y] = T^T [dU | dW]          -> dv = beta Z, dK~ = beta Y, dbeta parts <Z, v> + <Y, K~>
+//     dT = (dW K~^T + dU V^T) diag(beta) -> X1 = dT T^T -> dA = -T^T X1 (strictly lower)
+// T, K~, V are the forward kernel's fp16 tiles (backward mode), dU and dW
+// (fp32) are converted to fp16; products accumulate in fp32 in TMEM.
+template <int DK, int DV>
+struct TchSmem {
+    // fp16 128-byte-swizzled tiles of 64 rows x 64 columns (8 KB); an operand read
+    // as a 128-row MMA operand is followed by another valid tile
+    static constexpr uint32_t T = 0;                        // T [i][r]
+    static constexpr uint32_t X1 = T + 8192;                // X1 [j][i]
+    static constexpr uint32_t DU = X1 + 8192;               // dU [r][j]: DV / 64 tiles
+    static constexpr uint32_t DW = DU + (DV / 64) * 8192;   // dW [r][c]: DK / 64 tiles
+    static constexpr uint32_t DT = DW + (DK / 64) * 8192;   // dT diag(beta) [r][i], then a spare tile
+    static constexpr uint32_t KT = DT + 16384;              // K~ [i][c]: DK / 64 tiles
+    static constexpr uint32_t V = KT + (DK / 64) * 8192;    // V [i][j]: DV / 64 tiles
+    static constexpr uint32_t END = V + (DV / 64) * 8192;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(256, 1)
+bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restrict__ tiles,
+                     const float* __restrict__ dU_all, const float* __restrict__ beta,
+                     float* __restrict__ vside, __nv_bfloat16* __restrict__ dv, int H, size_t max_chunks)
+{
+    using Sm = TchSmem<DK, DV>;
+    using BT = BwdTiles<DK, DV>;
+    using VS = VSide<DK>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t bar_load, bar_mma;
+    __shared__ uint32_t s_tmem;
+    __shared__ float s_beta[kChunk], s_dbp[kChunk];
+
+    if (hdr->status != kStatusOk) return;
+    const int total = hdr->num_chunks * H;
+    if ((int)blockIdx.x >= total) return;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int lane_row = (warp & 3) * 32 + (tid & 31);   // TMEM lane = MMA row
+    const int wg = warp >> 2;
+    if (tid == 0) {
+        mbar_init(&bar_load, 1);
+        mbar_init(&bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const uint32_t TZY = tmem;                   // [Z | Y]: DV + DK columns
+    const uint32_t TDT = tmem + DV + DK;         // dT: 64
+    const uint32_t TX1 = TDT + 64;               // X1: 64
+    const uint32_t TDA = TX1 + 64;               // T^T X1: 64
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    float range_max = 0.f;
+    uint32_t load_phase = 0, mma_phase = 0;
+    bool aborted = false;
+    int mma_pending = 0;
+
+    auto mma_wait = [&]() -> bool {
+        mma_pending = 1;
+        const bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        mma_phase ^= 1;
+        mma_pending = 0;
+        return ok;
+    };
+    // fp16 copy of 8 fp32 values into a swizzled tile row
+    auto put8 = [&](uint32_t off, const float4& a, const float4& b, float sgn) {
+        __align__(16) __half2 hv[4] = {__floats2half2_rn(sgn * a.x, sgn * a.y), __floats2half2_rn(sgn * a.z, sgn * a.w),
+                                       __floats2half2_rn(sgn * b.x, sgn * b.y), __floats2half2_rn(sgn * b.z, sgn * b.w)};
+        range_max = fmaxf(range_max, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+        range_max = fmaxf(range_max, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
+        *reinterpret_cast<uint4*>(sm + off) = *reinterpret_cast<const uint4*>(hv);
+    };
+
+    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x) {
+        const int c = w / H, h = w - c * H;
+        int seq, tok0, L;
+        map.locate(c, seq, tok0, L);
+        const size_t it = (size_t)h * max_chunks + c;
+        const unsigned char* tl = tiles + it * BT::BYTES;
+        const float* dUc = dU_all + it * kChunk * DV;
+        float* out = vside + it * VS::FLOATS;
+
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&bar_load, BT::BYTES);
+            bulk_load(sm + Sm::T, tl + BT::T, 8192, &bar_load);
+            bulk_load(sm + Sm::KT, tl + BT::KT, (DK / 64) * 8192, &bar_load);
+            bulk_load(sm + Sm::V, tl + BT::V, (DV / 64) * 8192, &bar_load);
+        }
+        if (tid < kChunk) {
+            s_beta[tid] = tid < L ? beta[(size_t)(tok0 + tid) * H + h] : 0.f;
+            s_dbp[tid] = 0.f;
+        }
+        // dU and dW (rows = token) as fp16 tiles
+#pragma unroll 4
+        for (int idx = tid; idx < kChunk * DV / 8; idx += 256) {
+            const int r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
+            const float4 a = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8);
+            const float4 b = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8 + 4);
+            put8(Sm::DU + (j8 >> 6) * 8192 + sw128_offset(r, (j8 & 63) * 2), a, b, 1.f);
+        }
+#pragma unroll 4
+        for (int idx = tid; idx < kChunk * DK / 8; idx += 256) {
+            const int r = idx / (DK / 8), c8 = (idx - r * (DK / 8)) * 8;
+            const float4 a = *reinterpret_cast<const float4*>(out + VS::DW + (size_t)r * DK + c8);
+            const float4 b = *reinterpret_cast<const float4*>(out + VS::DW + (size_t)r * DK + c8 + 4);
+            put8(Sm::DW + (c8 >> 6) * 8192 + sw128_offset(r, (c8 & 63) * 2), a, b, 1.f);
+        }
+        const bool ok_load = mbar_wait_cycles(&bar_load, load_phase, kWaitCycles);
+        load_phase ^= 1;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(!ok_load)) { aborted = true; break; }
+
+        // [Z | Y] = T^T [dU | dW];  dT_raw = dW K~^T + dU V^T
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc_zy = instr_desc(kFmtF16, 128, DV + DK, true, true);   // A, B MN-major
+            constexpr uint32_t idesc_dt = instr_desc(kFmtF16, 128, 64, false, false);     // both K-major
+            const uint32_t t = smem_u32(sm + Sm::T), du = smem_u32(sm + Sm::DU), dw = smem_u32(sm + Sm::DW);
+            const uint32_t kt = smem_u32(sm + Sm::KT), vv = smem_u32(sm + Sm::V);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(TZY, smem_desc(t + ks * 2048, 8192, 1024, kLayoutSW128),
+                        smem_desc(du + ks * 2048, 8192, 1024, kLayoutSW128), idesc_zy, ks != 0);
+#pragma unroll
+            for (int b = 0; b < DK / 64; ++b)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(TDT, smem_desc(dw + b * 8192 + ks * 32, 16, 1024, kLayoutSW128),
+                            smem_desc(kt + b * 8192 + ks * 32, 16, 1024, kLayoutSW128), idesc_dt, (b | ks) != 0);
+#pragma unroll
+            for (int b = 0; b < DV / 64; ++b)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(TDT, smem_desc(du + b * 8192 + ks * 32, 16, 1024, kLayoutSW128),
+                            smem_desc(vv + b * 8192 + ks * 32, 16, 1024, kLayoutSW128), idesc_dt, true);
+            mma_commit(&bar_mma);
+        }
+        bool ok = mma_wait();
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        tc_fence_after();
+
+        // dT diag(beta) -> fp16 tile (rows 0..63)
+        if (lane_row < 64) {
+            float v[32];
+            tmem_ld32_sync(TDT + lane_base + 32 * wg, v);
+#pragma unroll
+            for (int i8 = 0; i8 < 4; ++i8) {
+                const int col = 32 * wg + 8 * i8;
+                const float4 a = make_float4(v[8 * i8] * s_beta[col], v[8 * i8 + 1] * s_beta[col + 1],
+                                             v[8 * i8 + 2] * s_beta[col + 2], v[8 * i8 + 3] * s_beta[col + 3]);
+                const float4 b = make_float4(v[8 * i8 + 4] * s_beta[col + 4], v[8 * i8 + 5] * s_beta[col + 5],
+                                             v[8 * i8 + 6] * s_beta[col + 6], v[8 * i8 + 7] * s_beta[col + 7]);
+                put8(Sm::DT + sw128_offset(lane_row, col * 2), a, b, 1.f);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // X1 = dT T^T
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc = instr_desc(kFmtF16, 128, 64, false, false);
+            const uint32_t dt = smem_u32(sm + Sm::DT), t = smem_u32(sm + Sm::T);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(TX1, smem_desc(dt + ks * 32, 16, 1024, kLayoutSW128),
+                        smem_desc(t + ks * 32, 16, 1024, kLayoutSW128), idesc, ks != 0);
+            mma_commit(&bar_mma);
+        }
+        // meanwhile: dv = beta Z (out), dK~ = beta Y (out), dbeta parts <Z, v> + <Y, K~>
+        if (lane_row < 64) {
+            const int r = lane_row;
+            const float br = s_beta[r];
+            float part = 0.f;
+#pragma unroll 1
+            for (int cb = wg; cb < (DV + DK) / 32; cb += 2) {
+                float v[32];
+                tmem_ld32_sync(TZY + lane_base + 32 * cb, v);
+                const bool zpart = 32 * cb < DV;
+                const int col0 = zpart ? 32 * cb : 32 * cb - DV;
+                const uint32_t base = zpart ? Sm::V : Sm::KT;
+#pragma unroll
+                for (int i8 = 0; i8 < 4; ++i8) {
+                    const int col = col0 + 8 * i8;
+                    const uint4 raw = *reinterpret_cast<const uint4*>(sm + base + (col >> 6) * 8192 + sw128_offset(r, (col & 63) * 2));
+                    const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __half22float2(hp[e]);
+                        part += v[8 * i8 + 2 * e] * f.x + v[8 * i8 + 2 * e + 1] * f.y;
+                    }
+                }
+                if (zpart) {
+                    if (r < L) {
+                        __nv_bfloat16* dst = dv + ((size_t)(tok0 + r) * H + h) * DV + col0;
+#pragma unroll
+                        for (int i8 = 0; i8 < 4; ++i8) {
+                            __align__(16) __nv_bfloat162 bv[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                bv[e] = __floats2bfloat162_rn(br * v[8 * i8 + 2 * e], br * v[8 * i8 + 2 * e + 1]);
+                            *reinterpret_cast<uint4*>(dst + 8 * i8) = *reinterpret_cast<const uint4*>(bv);
+                        }
+                    }
+                } else {
+                    float* dst = out + VS::DKT + (size_t)r * DK + col0;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(dst + i) = make_float4(br * v[i], br * v[i + 1], br * v[i + 2], br * v[i + 3]);
+                }
+            }
+            atomicAdd(&s_dbp[r], part);
+        }
+        ok = mma_wait();
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        tc_fence_after();
+
+        // X1 (rows j) -> fp16 tile [j][i]
+        if (lane_row < 64) {
+            float v[32];
+            tmem_ld32_sync(TX1 + lane_base + 32 * wg, v);
+#pragma unroll
+            for (int i8 = 0; i8 < 4; ++i8) {
+                const float4 a = make_float4(v[8 * i8], v[8 * i8 + 1], v[8 * i8 + 2], v[8 * i8 + 3]);
+                const float4 b = make_float4(v[8 * i8 + 4], v[8 * i8 + 5], v[8 * i8 + 6], v[8 * i8 + 7]);
+                put8(Sm::X1 + sw128_offset(lane_row, (32 * wg + 8 * i8) * 2), a, b, 1.f);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // T^T X1
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc = instr_desc(kFmtF16, 128, 64, true, true);
+            const uint32_t t = smem_u32(sm + Sm::T), x1 = smem_u32(sm + Sm::X1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(TDA, smem_desc(t + ks * 2048, 8192, 1024, kLayoutSW128),
+                        smem_desc(x1 + ks * 2048, 8192, 1024, kLayoutSW128), idesc, ks != 0);
+            mma_commit(&bar_mma);
+        }
+        ok = mma_wait();
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        tc_fence_after();
+        // dA = -T^T X1, strictly lower (rows 0..63); dbeta parts
+        if (lane_row < 64) {
+            float v[32];
+            tmem_ld32_sync(TDA + lane_base + 32 * wg, v);
+            float* dst = out + VS::DA + (size_t)lane_row * kChunk + 32 * wg;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const int col = 32 * wg + i;
+                *reinterpret_cast<float4*>(dst + i) =
+                    make_float4(col < lane_row ? -v[i] : 0.f, col + 1 < lane_row ? -v[i + 1] : 0.f,
+                                col + 2 < lane_row ? -v[i + 2] : 0.f, col + 3 < lane_row ? -v[i + 3] : 0.f);
+            }
+        }
+        if (tid < kChunk) out[VS::DBP + tid] = s_dbp[tid];
+        tc_fence_before();
+        __syncthreads();   // smem and TMEM are free for the next item
+    }
+
+    if (aborted) {
+        if (tid == 0) flag_error(hdr, kStatusTimeout);
+        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        (void)mbar_wait_cycles(&bar_load, load_phase, kWaitCycles / 4);
+    }
+    if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
 // ------------------------------------------------------------- host -----
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1559,7 +1872,8 @@ cudaError_t launch_intra_tc_t(const ChunkArgs& a) {
     kern<<<grid, 256, smem, a.stream>>>(mk, mv, mq, mla, a.log_alpha, a.beta, map,
                                         static_cast<WsHeader*>(a.ws_header),
                                         static_cast<unsigned char*>(a.records), a.H, a.max_chunks,
-                                        a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy, a.tmat);
+                                        a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy,
+                                        static_cast<unsigned char*>(a.bwd_tiles));
     return cudaGetLastError();
 }
 
@@ -1620,6 +1934,25 @@ cudaError_t launch_bwd_vside_tc_t(const ChunkArgs& a) {
     return cudaGetLastError();
 }
 
+template <int DK, int DV>
+cudaError_t launch_bwd_tchain_tc_t(const ChunkArgs& a) {
+    if (a.max_chunks == 0) return cudaSuccess;
+    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
+    auto kern = bwd_tchain_tc_kernel<DK, DV>;
+    const int smem = (int)TchSmem<DK, DV>::END + 1024;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const size_t items = a.max_chunks * (size_t)a.H;
+    const unsigned grid = (unsigned)(items < (size_t)sms ? items : (size_t)sms);
+    kern<<<grid, 256, smem, a.stream>>>(map, static_cast<WsHeader*>(a.ws_header),
+                                        static_cast<const unsigned char*>(a.bwd_tiles), a.dU, a.beta, a.vside,
+                                        static_cast<__nv_bfloat16*>(a.dv_out), a.H, a.max_chunks);
+    return cudaGetLastError();
+}
+
 #define KDA_TC_DISPATCH(FN, a)                                                  \
     do {                                                                       \
         if ((a).dk == 128 && (a).dv == 128) return FN<128, 128>(a);            \
@@ -1649,5 +1982,7 @@ cudaError_t launch_chunk_inter_tc(const ChunkArgs& a) {
 cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_inter_tc_t, a); }
 
 cudaError_t launch_chunk_bwd_vside_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_vside_tc_t, a); }
+
+cudaError_t launch_chunk_bwd_tchain_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_tchain_tc_t, a); }
 
 }  // namespace kda

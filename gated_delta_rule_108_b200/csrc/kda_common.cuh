@@ -52,6 +52,9 @@ struct F32Rec {
 // dQ~ = D S^T, dW = -dU S^T, dK^ = U dS'^T [64][DK] each, dP = D U^T [64][64]
 // (lower with the diagonal), dgamma [DK].  Written by the tensor-core
 // value-side kernel (bf16 inputs), read by the per-chunk gradient kernel.
+// Then the T-chain products (tensor-core T-chain kernel): dK~ = beta T^T dW
+// [64][DK], dA = -T^T dT T^T [64][64] (strictly lower) and the parts of dbeta
+// that come through W and U0 [64].
 template <int DK>
 struct VSide {
     static constexpr size_t DQT = 0;
@@ -59,7 +62,10 @@ struct VSide {
     static constexpr size_t DKH = DW + kChunk * DK;
     static constexpr size_t DP = DKH + kChunk * DK;
     static constexpr size_t DGAM = DP + kChunk * kChunk;
-    static constexpr size_t FLOATS = (DGAM + DK + 63) / 64 * 64;
+    static constexpr size_t DKT = DGAM + DK;
+    static constexpr size_t DA = DKT + kChunk * DK;
+    static constexpr size_t DBP = DA + kChunk * kChunk;
+    static constexpr size_t FLOATS = (DBP + kChunk + 63) / 64 * 64;
 };
 
 // Element loads/stores for the two input dtypes.

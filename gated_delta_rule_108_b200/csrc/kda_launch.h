@@ -38,7 +38,8 @@ struct ChunkArgs {
     int fixed_chunks_per_seq;     // ceil(T / 64) for fixed length
     cudaStream_t stream;
     // backward pass only (all null in the forward)
-    float* tmat;                  // [H][max_chunks][64][64]: K1 also writes T = (I + A)^{-1}
+    float* tmat;                  // [H][max_chunks][64][64]: the fp32 K1 also writes T = (I + A)^{-1}
+    void* bwd_tiles;              // bf16: [H][max_chunks] fp16 T, K~, V tiles from the tensor-core K1
     float* states;                // [H][max_chunks][dk][dv]: K2 also writes the state entering each chunk
     const void* d_o;              // [.., H, dv], input dtype
     const float* d_final_state;   // [N, H, dk, dv], nullable (zeros)
@@ -73,6 +74,7 @@ cudaError_t launch_chunk_inter_tc(const ChunkArgs& a); // bf16 inputs: tensor-co
 cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a);  // backward: serial over chunks, reversed
 cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a); // the same on the tensor cores (bf16 inputs)
 cudaError_t launch_chunk_bwd_vside_tc(const ChunkArgs& a); // backward products over the value dim (bf16 inputs)
+cudaError_t launch_chunk_bwd_tchain_tc(const ChunkArgs& a); // backward products through T, W, U0 (bf16 inputs)
 cudaError_t launch_chunk_bwd_intra(const ChunkArgs& a);  // backward: all chunks in parallel
 size_t bwd_scratch_bytes_per_cta(int dk, int dv);
 constexpr int kBwdMaxCtas = 512;   // scratch is sized for at most this many CTAs
