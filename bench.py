@@ -44,9 +44,6 @@ if ROOT not in sys.path:
 import torch  # noqa: E402
 
 METRIC = "KDA tokens/s (chunk fwd & decode) at 1 B200; % bf16 TC peak / % HBM BW"
-# fp32 CUDA-core peak of one B200 from its unit counts and clock: 148 SMs x 128
-# fp32 lanes x 2 flops per FMA x 1.965 GHz (clocks.max.sm)
-FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # FLOPs per token and head of the chunk forward at MMA tile granularity
 # (d_k = d_v = d, chunk C = 64): 2C(3d_k + 2d_v) + 6 d_k d_v.
@@ -215,22 +212,19 @@ def bench_chunk(args, dev, world, rank):
                 x=x, o=o, S=S, ws=ws)
 
 
-def chunk_bwd_simt_flops_per_chunk_head(dk, dv, C=64):
-    """FLOPs (2 x multiply-adds) of the CUDA-core per-chunk gradient kernel once
-    the value-side and T-chain products are formed on the tensor cores: M, dKl,
-    dQl (C C dk each) and dKr (2 C C dk)."""
-    return 2 * 5 * C * C * dk
-
-
 def chunk_bwd_tc_bytes_per_chunk_head(dk, dv, C=64):
-    """Algorithmic bytes of the two tensor-core product kernels.  Value side:
-    reads S, dS' (fp32 dk x dv), dU (fp32 C x dv), d_o (bf16 C x dv), the fp16 W,
-    Q~, U0 tiles; writes dQ~, dW, dK^ (fp32 C x dk), dP (fp32 C x C), dgamma.
-    T-chain: reads the fp16 T, K~, V tiles, dU (fp32 C x dv), dW (fp32 C x dk),
-    beta; writes dv (bf16 C x dv), dK~ (fp32 C x dk), dA (fp32 C x C), dbeta parts."""
+    """Algorithmic bytes of the backward's three tensor-core product kernels per
+    (chunk, head).  Value side: reads S, dS' (fp32 dk x dv), dU (fp32 C x dv), d_o
+    (bf16 C x dv), the fp16 W, Q~, U0 tiles; writes dQ~, dW, dK^ (fp32 C x dk), dP
+    (fp32 C x C), dgamma.  T-chain: reads the fp16 T, K~, V tiles, dU, dW, beta;
+    writes dv (bf16), dK~ (fp32 C x dk), dA (fp32 C x C), dbeta parts.  Split
+    factors: reads q, k (bf16), log_alpha, beta, dA, dP, M (fp32 C x C), dQ~, dK^,
+    dK~, dgamma, dbeta parts; writes dq, dk (bf16), dlog_alpha (fp32), dbeta."""
     vside = 2 * 4 * dk * dv + 4 * C * dv + 2 * C * dv + 2 * (2 * C * dk + C * dv) + 4 * (3 * C * dk + C * C + dk)
     tchain = 2 * (C * C + C * dk + C * dv) + 4 * C * dv + 4 * C * dk + 4 * C + 2 * C * dv + 4 * (C * dk + C * C + C)
-    return vside + tchain
+    split = (2 * 2 * C * dk + 4 * C * dk + 4 * C + 4 * 3 * C * C + 4 * (3 * C * dk + dk + C)
+             + 2 * 2 * C * dk + 4 * C * dk + 4 * C)
+    return vside + tchain + split
 
 
 def bench_backward(args, dev, world, rank):
@@ -456,26 +450,21 @@ def run_ours(args):
     if bwd is not None:
         bw = bwd["w"]
         n_ch = bw.num_seqs * ((bw.T + 63) // 64) * bw.H
-        bflops = chunk_bwd_simt_flops_per_chunk_head(bw.dk, bw.dv) * n_ch
         vbytes = chunk_bwd_tc_bytes_per_chunk_head(bw.dk, bw.dv) * n_ch
         vms = bwd["stages"]["bwd_tc_products"]
-        bms = bwd["stages"]["bwd_intra_chunk"]
-        btf = bflops / (bms / 1e3) / 1e12
-        alu_peak = FP32_SIMT_TFLOPS
+        vgbs = vbytes / (vms / 1e3) / 1e9
         line["chunk_bwd"] = {
             "workload": f"{bw.name}: kda_chunk_bwd (dq, dk, dv, dlog_alpha, dbeta, dS0), B={bw.B}, T={bw.T}, "
-                        f"H={bw.H}, d_k=d_v={bw.dk}, bf16 q/k/v/d_o, fp32 arithmetic on CUDA cores",
+                        f"H={bw.H}, d_k=d_v={bw.dk}, bf16 q/k/v/d_o; tensor-core products (fp16 / tf32 operands, "
+                        "fp32 accumulation), strong-decay chunks on CUDA cores in fp32",
             "value": bw.tokens * world / (bwd["ms_per_step"] / 1e3), "unit": "tokens/s",
             "ms_per_step": bwd["ms_per_step"], "steps": args.bwd_steps, "kernels_ms": bwd["stages"],
             "gpu_launches": bwd["launches"],
-            "roofline": {"kernel": "bwd_intra_chunk", "bound": "alu", "achieved": btf, "peak": alu_peak,
-                         "unit": "TFLOP/s", "frac": btf / alu_peak, "traffic": traffic_for("bwd_intra_chunk"),
-                         "peak_source": "derived: 148 SMs x 128 fp32 FMA/clk x 2 x 1.965 GHz",
-                         "algorithmic_flops_per_launch": bflops, "ms_per_launch": bms},
-            "tc_products_roofline": {"kernel": "bwd_vside_tc + bwd_tchain_tc", "bound": "hbm",
-                                    "achieved": vbytes / (vms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
-                                    "frac": vbytes / (vms / 1e3) / 1e9 / hbm,
-                                    "algorithmic_bytes_per_launch": vbytes, "ms_per_launch": vms},
+            "roofline": {"kernel": "bwd_vside_tc + bwd_tchain_tc + bwd_split_tc (the dominant stage)",
+                         "bound": "hbm", "achieved": vgbs, "peak": hbm, "unit": "GB/s", "frac": vgbs / hbm,
+                         "traffic": traffic_for("bwd_tc_products"), "peak_source": f"{peak_kind} hbm_gbs",
+                         "algorithmic_bytes_per_launch": vbytes, "ms_per_launch": vms},
+            "strong_decay_chunks_ms": bwd["stages"]["bwd_intra_chunk"],
         }
     if e2e is not None:
         ms_e, h2d, d2h = e2e

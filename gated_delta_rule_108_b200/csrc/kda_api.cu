@@ -78,7 +78,8 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
 struct BwdLayout {
     WsLayout base;   // header, offsets, the forward's records for this dtype
     size_t vside_off;// bf16: the tensor-core products per (head, chunk) (0 for fp32)
-    size_t tiles_off;// bf16: fp16 T, K~, V tiles per (head, chunk) (0 for fp32)
+    size_t tiles_off;// bf16: fp16 T, K~, V tiles, fp32 M per (head, chunk) (0 for fp32)
+    size_t flags_off;// bf16: strong-decay flag per (head, chunk) (0 for fp32)
     size_t tmat_off, states_off, dS_off, dU_off, scratch_off, total;
     int ctas;        // CTAs the scratch holds
 };
@@ -90,13 +91,16 @@ bool bwd_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, 
     size_t off = round_up(L.base.total, 256);
     L.vside_off = 0;
     L.tiles_off = 0;
+    L.flags_off = 0;
     L.tmat_off = 0;
     if (dtype == KDA_BF16) {
         L.vside_off = off;
         const size_t vs_floats = dk == 128 ? kda::VSide<128>::FLOATS : kda::VSide<64>::FLOATS;
         off = round_up(off + sizeof(float) * vs_floats * units, 256);
         L.tiles_off = off;
-        off = round_up(off + (size_t)8192 * (1 + dk / 64 + dv / 64) * units, 256);   // fp16 T, K~, V tiles
+        off = round_up(off + kda::bwd_tiles_bytes(dk, dv) * units, 256);   // fp16 T, K~, V tiles, fp32 M
+        L.flags_off = off;
+        off = round_up(off + sizeof(int) * units, 256);
     } else {
         L.tmat_off = off;
         off = round_up(off + sizeof(float) * kda::kChunk * kda::kChunk * units, 256);
@@ -337,6 +341,7 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
     a.stream = static_cast<cudaStream_t>(stream);
     a.tmat = a.bf16 ? nullptr : reinterpret_cast<float*>(ws + L.tmat_off);
     a.bwd_tiles = a.bf16 ? static_cast<void*>(ws + L.tiles_off) : nullptr;
+    a.bwd_flags = a.bf16 ? reinterpret_cast<int*>(ws + L.flags_off) : nullptr;
     a.states = reinterpret_cast<float*>(ws + L.states_off);
     a.d_o = d_o; a.d_final_state = d_final_state;
     a.dq = dq; a.dk_out = dk_out; a.dv_out = dv_out;
@@ -372,6 +377,7 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
         a.vside = reinterpret_cast<float*>(ws + L.vside_off);
         if (e == cudaSuccess) e = kda::launch_chunk_bwd_vside_tc(a);
         if (e == cudaSuccess) e = kda::launch_chunk_bwd_tchain_tc(a);
+        if (e == cudaSuccess) e = kda::launch_chunk_bwd_split_tc(a);
     }
     if (e == cudaSuccess) e = mark(5);
     if (e == cudaSuccess) e = kda::launch_chunk_bwd_intra(a);

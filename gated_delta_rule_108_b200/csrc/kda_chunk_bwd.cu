@@ -399,7 +399,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                  const float* __restrict__ dS_end, const float* __restrict__ dU_all, float* scratch,
                  T* __restrict__ dq, T* __restrict__ dk, T* __restrict__ dv, float* __restrict__ dla,
                  float* __restrict__ dbeta, int H, size_t max_chunks, float scale, int gate,
-                 const float* __restrict__ vside)
+                 const float* __restrict__ vside, const int* __restrict__ only_flagged)
 {
     using R = Rec<DK, DV>;
     using C = Scr<DK, DV>;
@@ -415,6 +415,9 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
 
     for (long item = blockIdx.x; item < total; item += gridDim.x) {
         const int c = (int)(item / H), h = (int)(item % H);
+        // with the split-factor products on the tensor cores, only the chunks that
+        // took the strong-decay (exact) path are left to this kernel
+        if (only_flagged && !only_flagged[(size_t)h * max_chunks + c]) continue;
         int s, tok0, L;
         map.locate(c, s, tok0, L);
         const size_t it = (size_t)h * max_chunks + c;
@@ -759,7 +762,7 @@ cudaError_t launch_bwd_intra_t(const ChunkArgs& a) {
         static_cast<const T*>(a.d_o), map, static_cast<const WsHeader*>(a.ws_header),
         static_cast<const float*>(a.records), a.tmat, a.states, a.dS_end, a.dU, a.scratch,
         static_cast<T*>(a.dq), static_cast<T*>(a.dk_out), static_cast<T*>(a.dv_out), a.dlog_alpha, a.dbeta,
-        a.H, a.max_chunks, a.scale, a.gate, a.vside);
+        a.H, a.max_chunks, a.scale, a.gate, a.vside, a.bwd_flags);
     return cudaGetLastError();
 }
 

@@ -91,7 +91,9 @@ struct BwdTiles {
     static constexpr uint32_t T = 0;
     static constexpr uint32_t KT = T + 8192;
     static constexpr uint32_t V = KT + (DK / 64) * 8192;
-    static constexpr uint32_t BYTES = V + (DV / 64) * 8192;
+    static constexpr uint32_t TILE_BYTES = V + (DV / 64) * 8192;   // the fp16 tiles
+    static constexpr uint32_t M = TILE_BYTES;                       // fp32 M = K_l K_r^T [64][64], strictly lower
+    static constexpr uint32_t BYTES = M + 64 * 64 * 4;
 };
 
 constexpr float kMaxSplitExponent = 60.f;   // e^60 ~ 1e26: far inside the fp32 range
@@ -194,7 +196,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                       const float* __restrict__ log_alpha_head, const float* __restrict__ beta,
                       ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
                       size_t max_chunks, long long wait_cap, int drop_first_la,
-                      unsigned char* __restrict__ bwd_tiles)
+                      unsigned char* __restrict__ bwd_tiles, int* __restrict__ bwd_flags)
 {
     using Sm = K1Smem<DK, DV>;
     using R = TcRec<DK, DV>;
@@ -305,6 +307,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         int c, h, tok0, L;
         locate(w, c, h, tok0, L);
         unsigned char* rec = records + ((size_t)h * max_chunks + c) * R::BYTES;
+        unsigned char* btile = bwd_tiles ? bwd_tiles + ((size_t)h * max_chunks + c) * BwdTiles<DK, DV>::BYTES : nullptr;
         if (tid >= 192) {
             s_beta[tid - 192] = beta_next;
             if constexpr (GATE == kGateHead) s_lah[tid - 192] = lah_next;
@@ -520,6 +523,10 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                     a4.z = (col + 2 < row) ? b * v[4 * i4 + 2] : 0.f;
                     a4.w = (col + 3 < row) ? b * v[4 * i4 + 3] : 0.f;
                     *reinterpret_cast<float4*>(am + row * 68 + col) = a4;
+                    if (btile)   // backward mode: the unweighted M = K_l K_r^T
+                        *reinterpret_cast<float4*>(btile + BwdTiles<DK, DV>::M + (row * 64 + col) * 4) =
+                            make_float4((col + 0 < row) ? v[4 * i4 + 0] : 0.f, (col + 1 < row) ? v[4 * i4 + 1] : 0.f,
+                                        (col + 2 < row) ? v[4 * i4 + 2] : 0.f, (col + 3 < row) ? v[4 * i4 + 3] : 0.f);
                 }
             } else {
                 const int r = row - 64;
@@ -539,7 +546,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         }
         }   // !strong
         __syncthreads();
-        unsigned char* btile = bwd_tiles ? bwd_tiles + ((size_t)h * max_chunks + c) * BwdTiles<DK, DV>::BYTES : nullptr;
+        if (bwd_flags && tid == 0) bwd_flags[(size_t)h * max_chunks + c] = strong ? 1 : 0;   // strong-decay path taken
         if (btile && tid == kTileThread) {   // backward mode: K~ and fp16 V are final
 #pragma unroll
             for (int b = 0; b < DK / 64; ++b) bulk_store(btile + BwdTiles<DK, DV>::KT + b * 8192, st + Sm::KS + b * Sm::TILE, 8192);
@@ -1626,7 +1633,7 @@ bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restric
         float* out = vside + it * VS::FLOATS;
 
         if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_load, BT::BYTES);
+            mbar_arrive_expect_tx(&bar_load, BT::TILE_BYTES);
             bulk_load(sm + Sm::T, tl + BT::T, 8192, &bar_load);
             bulk_load(sm + Sm::KT, tl + BT::KT, (DK / 64) * 8192, &bar_load);
             bulk_load(sm + Sm::V, tl + BT::V, (DV / 64) * 8192, &bar_load);
@@ -1818,6 +1825,257 @@ bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restric
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// --------------------------------------- backward split-factor part (bf16) ----
+// The rest of the backward for chunks without strong decay, on the tensor
+// cores in tf32 (bf16 inputs): with K_l = k e^{g - g_m}, K_r = k e^{g_m - g},
+// Q_l = q e^{g - g_m} (fp32 range, hence tf32) and dM = diag(beta) dA,
+//     [dK_l^T | dQ_l^T] = K_r^T [dM; dP]^T        dK_r^T = [K_l^T | Q_l^T] [dM^T | dP^T]^T
+// so that TMEM lane = key channel; then the decay factors and the suffix sums
+// of dlog_alpha per channel, and dbeta = (parts through W, U0) + rowsum(dA M)
+// with M from the forward kernel.  Every operand is K-major.
+template <int DK, int DV>
+struct SpSmem {
+    static constexpr uint32_t G = 0;                        // g (natural log) [64][DK] fp32, later dg
+    static constexpr uint32_t KRT = G + 64 * DK * 4;        // K_r^T [c][i]: 2 tiles (32 i) of DK rows x 128 B
+    static constexpr uint32_t KLQT = KRT + 2 * DK * 128;    // [K_l^T | Q_l^T] [c][r]: 4 tiles
+    static constexpr uint32_t DMP = KLQT + 4 * DK * 128;    // [dM; dP] [r][i]: 2 tiles of 128 rows x 128 B
+    static constexpr uint32_t DMPT = DMP + 2 * 16384;       // [dM^T | dP^T] [i][r]: 4 tiles of 64 rows x 128 B
+    static constexpr uint32_t END = DMPT + 4 * 8192 + 8192; // + a spare tile (128-row reads of the last one)
+    static_assert(END + 1024 <= 232448, "shared memory");
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(256, 1)
+bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                    const float* __restrict__ log_alpha, const float* __restrict__ beta, ChunkMap map,
+                    WsHeader* hdr, const unsigned char* __restrict__ tiles, const int* __restrict__ flags,
+                    const float* __restrict__ vside, __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
+                    float* __restrict__ dla, float* __restrict__ dbeta, int H, size_t max_chunks, int gate)
+{
+    using Sm = SpSmem<DK, DV>;
+    using BT = BwdTiles<DK, DV>;
+    using VS = VSide<DK>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t bar_mma;
+    __shared__ uint32_t s_tmem;
+    __shared__ float s_gm[DK], s_gl[DK], s_dgl[DK], s_beta[kChunk];
+
+    if (hdr->status != kStatusOk) return;
+    const int total = hdr->num_chunks * H;
+    if ((int)blockIdx.x >= total) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int lane_row = (warp & 3) * 32 + (tid & 31);   // TMEM lane = key channel
+    const int wg = warp >> 2;                            // tokens [32 wg, 32 wg + 32)
+    const size_t rowk = (size_t)H * DK;
+    if (tid == 0) {
+        mbar_init(&bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const uint32_t T1 = tmem;          // [dK_l^T | dQ_l^T]: 128 columns (token r)
+    const uint32_t T2 = tmem + 128;    // dK_r^T: 64 columns (token i)
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    uint32_t mma_phase = 0;
+    bool aborted = false;
+    int mma_pending = 0;
+    float* g = reinterpret_cast<float*>(sm + Sm::G);
+
+    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x) {
+        const int c = w / H, h = w - c * H;
+        const size_t it = (size_t)h * max_chunks + c;
+        if (flags[it]) continue;   // strong decay: the exact CUDA-core path handles this chunk
+        int seq, tok0, L;
+        map.locate(c, seq, tok0, L);
+        const float* vs = vside + it * VS::FLOATS;
+        const float* Mg = reinterpret_cast<const float*>(tiles + it * BT::BYTES + BT::M);
+
+        // cumulative log-decay (natural log) per channel; beta
+        if (tid < DK) {
+            float acc = 0.f;
+            if (gate == kGateNone) {
+                for (int r = 0; r < kChunk; ++r) g[r * DK + tid] = 0.f;
+            } else {
+                const bool chan = gate == kGateChannel;
+                const size_t rstride = chan ? rowk : (size_t)H;
+                const float* la = chan ? log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid
+                                       : log_alpha + (size_t)tok0 * H + h;
+                for (int r = 0; r < kChunk; ++r) {
+                    acc += (r < L) ? la[(size_t)r * rstride] : 0.f;
+                    g[r * DK + tid] = acc;
+                }
+            }
+            s_dgl[tid] = 0.f;
+        } else if (tid >= 128 && tid < 128 + kChunk) {
+            const int r = tid - 128;
+            s_beta[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
+        }
+        __syncthreads();
+        if (tid < DK) {
+            s_gm[tid] = g[((L - 1) >> 1) * DK + tid];
+            s_gl[tid] = g[(L - 1) * DK + tid];
+        }
+        __syncthreads();
+
+        // tf32 operands.  K_r^T, K_l^T, Q_l^T: (channel, 4 tokens) per step
+#pragma unroll 2
+        for (int idx = tid; idx < DK * (kChunk / 4); idx += 256) {
+            const int ch = idx % DK, r4 = (idx / DK) * 4;
+            float kr[4], kl[4], ql[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int r = r4 + t;
+                float kk = 0.f, qq = 0.f;
+                if (r < L) {
+                    const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
+                    kk = __bfloat162float(k[off]);
+                    qq = __bfloat162float(q[off]);
+                }
+                const float d = g[r * DK + ch] - s_gm[ch];
+                const float fl = __expf(d), fr = __expf(-d);
+                kr[t] = round_tf32_alu(kk * fr);
+                kl[t] = round_tf32_alu(kk * fl);
+                ql[t] = round_tf32_alu(qq * fl);
+            }
+            *reinterpret_cast<float4*>(sm + Sm::KRT + f_off(ch, r4, DK * 128)) = make_float4(kr[0], kr[1], kr[2], kr[3]);
+            *reinterpret_cast<float4*>(sm + Sm::KLQT + f_off(ch, r4, DK * 128)) = make_float4(kl[0], kl[1], kl[2], kl[3]);
+            *reinterpret_cast<float4*>(sm + Sm::KLQT + f_off(ch, 64 + r4, DK * 128)) = make_float4(ql[0], ql[1], ql[2], ql[3]);
+        }
+        // [dM; dP] and their transposes: (row r, 4 columns i) per step
+#pragma unroll 2
+        for (int idx = tid; idx < kChunk * (kChunk / 4); idx += 256) {
+            const int r = idx >> 4, i4 = (idx & 15) * 4;
+            const float4 da = *reinterpret_cast<const float4*>(vs + VS::DA + r * kChunk + i4);
+            const float4 dp = *reinterpret_cast<const float4*>(vs + VS::DP + r * kChunk + i4);
+            const float br = s_beta[r];
+            const float dm[4] = {round_tf32_alu(br * da.x), round_tf32_alu(br * da.y),
+                                 round_tf32_alu(br * da.z), round_tf32_alu(br * da.w)};
+            const float pp[4] = {round_tf32_alu(dp.x), round_tf32_alu(dp.y), round_tf32_alu(dp.z), round_tf32_alu(dp.w)};
+            *reinterpret_cast<float4*>(sm + Sm::DMP + f_off(r, i4, 16384)) = make_float4(dm[0], dm[1], dm[2], dm[3]);
+            *reinterpret_cast<float4*>(sm + Sm::DMP + f_off(64 + r, i4, 16384)) = make_float4(pp[0], pp[1], pp[2], pp[3]);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                *reinterpret_cast<float*>(sm + Sm::DMPT + f_off(i4 + t, r, 8192)) = dm[t];
+                *reinterpret_cast<float*>(sm + Sm::DMPT + f_off(i4 + t, 64 + r, 8192)) = pp[t];
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idesc1 = instr_desc(kFmtTF32, 128, 128);
+            constexpr uint32_t idesc2 = instr_desc(kFmtTF32, 128, 64);
+            const uint32_t krt = smem_u32(sm + Sm::KRT), klqt = smem_u32(sm + Sm::KLQT);
+            const uint32_t dmp = smem_u32(sm + Sm::DMP), dmpt = smem_u32(sm + Sm::DMPT);
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_tf32(T1, smem_desc(krt + kb * (DK * 128) + ks * 32, 16, 1024, kLayoutSW128),
+                             smem_desc(dmp + kb * 16384 + ks * 32, 16, 1024, kLayoutSW128), idesc1, (kb | ks) != 0);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_tf32(T2, smem_desc(klqt + kb * (DK * 128) + ks * 32, 16, 1024, kLayoutSW128),
+                             smem_desc(dmpt + kb * 8192 + ks * 32, 16, 1024, kLayoutSW128), idesc2, (kb | ks) != 0);
+            mma_commit(&bar_mma);
+        }
+        // meanwhile: dbeta = (parts through W, U0) + rowsum(dA M), one warp per token
+        for (int r = warp; r < L; r += 8) {
+            float part = 0.f;
+            for (int i = lane; i < kChunk; i += 32) part += vs[VS::DA + r * kChunk + i] * Mg[r * kChunk + i];
+#pragma unroll
+            for (int off = 16; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+            if (lane == 0) dbeta[(size_t)(tok0 + r) * H + h] = vs[VS::DBP + r] + part;
+        }
+        mma_pending = 1;
+        const bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        mma_phase ^= 1;
+        mma_pending = 0;
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        tc_fence_after();
+
+        // dq, dk and dg for channel lane_row, tokens [32 wg, 32 wg + 32)
+        if (lane_row < DK) {
+            const int ch = lane_row;
+            const float gm = s_gm[ch], gl = s_gl[ch];
+            const float egm = __expf(gm), eglm = __expf(gl - gm);
+            float dgl = 0.f;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {   // 16 tokens at a time
+                float dkl[16], dql[16], dkr[16];
+                const uint32_t col = 32 * wg + 16 * half;
+                tmem_ld16(T1 + lane_base + col, dkl);
+                tmem_ld16(T1 + lane_base + 64 + col, dql);
+                tmem_ld16(T2 + lane_base + col, dkr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int r = (int)col + t;
+                    const float gg = g[r * DK + ch];
+                    float kk = 0.f, qq = 0.f;
+                    const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
+                    if (r < L) {
+                        kk = __bfloat162float(k[off]);
+                        qq = __bfloat162float(q[off]);
+                    }
+                    const float d = gg - gm;
+                    const float fl = __expf(d), fr = __expf(-d);
+                    const float eg = egm * fl, eh = eglm * fr;   // e^{g}, e^{g_{L-1} - g}
+                    const float a = dkl[t] * fl, b = dql[t] * fl, cr = dkr[t] * fr;
+                    const float dkt = vs[VS::DKT + r * DK + ch], dkh = vs[VS::DKH + r * DK + ch], dqt = vs[VS::DQT + r * DK + ch];
+                    if (r < L) {
+                        dk[off] = __float2bfloat16_rn(a + cr + dkt * eg + dkh * eh);
+                        dq[off] = __float2bfloat16_rn(b + dqt * eg);
+                    }
+                    const float kh = kk * eh;
+                    dgl += dkh * kh;
+                    g[r * DK + ch] = kk * (a - cr + dkt * eg) - dkh * kh + qq * (b + dqt * eg);   // dg
+                }
+            }
+            atomicAdd(&s_dgl[ch], dgl);
+        }
+        __syncthreads();
+        // dlog_alpha_s = sum_{r >= s} dg_r (+ g_{L-1}'s own cotangent), per channel
+        if (gate != kGateNone && tid < DK) {
+            float run = s_dgl[tid] + vs[VS::DGAM + tid] * __expf(s_gl[tid]);
+            for (int r = L - 1; r >= 0; --r) {
+                run += g[r * DK + tid];
+                if (gate == kGateChannel) dla[(size_t)(tok0 + r) * rowk + (size_t)h * DK + tid] = run;
+                else g[r * DK + tid] = run;
+            }
+        }
+        if (gate == kGateHead) {
+            __syncthreads();
+            if (tid < L) {
+                float acc = 0.f;
+                for (int cc = 0; cc < DK; ++cc) acc += g[tid * DK + (cc + tid) % DK];
+                dla[(size_t)(tok0 + tid) * H + h] = acc;
+            }
+        }
+        tc_fence_before();
+        __syncthreads();   // smem and TMEM are free for the next item
+    }
+
+    if (aborted) {
+        if (tid == 0) flag_error(hdr, kStatusTimeout);
+        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
 // ------------------------------------------------------------- host -----
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1873,7 +2131,7 @@ cudaError_t launch_intra_tc_t(const ChunkArgs& a) {
                                         static_cast<WsHeader*>(a.ws_header),
                                         static_cast<unsigned char*>(a.records), a.H, a.max_chunks,
                                         a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy,
-                                        static_cast<unsigned char*>(a.bwd_tiles));
+                                        static_cast<unsigned char*>(a.bwd_tiles), a.bwd_flags);
     return cudaGetLastError();
 }
 
@@ -1953,6 +2211,27 @@ cudaError_t launch_bwd_tchain_tc_t(const ChunkArgs& a) {
     return cudaGetLastError();
 }
 
+template <int DK, int DV>
+cudaError_t launch_bwd_split_tc_t(const ChunkArgs& a) {
+    if (a.max_chunks == 0) return cudaSuccess;
+    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
+    auto kern = bwd_split_tc_kernel<DK, DV>;
+    const int smem = (int)SpSmem<DK, DV>::END + 1024;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const size_t items = a.max_chunks * (size_t)a.H;
+    const unsigned grid = (unsigned)(items < (size_t)sms ? items : (size_t)sms);
+    kern<<<grid, 256, smem, a.stream>>>(
+        static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k), a.log_alpha, a.beta, map,
+        static_cast<WsHeader*>(a.ws_header), static_cast<const unsigned char*>(a.bwd_tiles), a.bwd_flags, a.vside,
+        static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dk_out), a.dlog_alpha, a.dbeta, a.H,
+        a.max_chunks, a.gate);
+    return cudaGetLastError();
+}
+
 #define KDA_TC_DISPATCH(FN, a)                                                  \
     do {                                                                       \
         if ((a).dk == 128 && (a).dv == 128) return FN<128, 128>(a);            \
@@ -1963,6 +2242,14 @@ cudaError_t launch_bwd_tchain_tc_t(const ChunkArgs& a) {
     } while (0)
 
 }  // namespace
+
+size_t bwd_tiles_bytes(int dk, int dv) {
+    if (dk == 128 && dv == 128) return BwdTiles<128, 128>::BYTES;
+    if (dk == 128 && dv == 64) return BwdTiles<128, 64>::BYTES;
+    if (dk == 64 && dv == 128) return BwdTiles<64, 128>::BYTES;
+    if (dk == 64 && dv == 64) return BwdTiles<64, 64>::BYTES;
+    return 0;
+}
 
 size_t tc_record_bytes(int dk, int dv) {
     if (dk == 128 && dv == 128) return TcRec<128, 128>::BYTES;
@@ -1984,5 +2271,7 @@ cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(laun
 cudaError_t launch_chunk_bwd_vside_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_vside_tc_t, a); }
 
 cudaError_t launch_chunk_bwd_tchain_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_tchain_tc_t, a); }
+
+cudaError_t launch_chunk_bwd_split_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_split_tc_t, a); }
 
 }  // namespace kda

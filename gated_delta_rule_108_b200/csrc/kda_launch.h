@@ -39,7 +39,8 @@ struct ChunkArgs {
     cudaStream_t stream;
     // backward pass only (all null in the forward)
     float* tmat;                  // [H][max_chunks][64][64]: the fp32 K1 also writes T = (I + A)^{-1}
-    void* bwd_tiles;              // bf16: [H][max_chunks] fp16 T, K~, V tiles from the tensor-core K1
+    void* bwd_tiles;              // bf16: [H][max_chunks] fp16 T, K~, V tiles and fp32 M from the tensor-core K1
+    int* bwd_flags;               // bf16: [H][max_chunks] 1 where the chunk took the strong-decay path
     float* states;                // [H][max_chunks][dk][dv]: K2 also writes the state entering each chunk
     const void* d_o;              // [.., H, dv], input dtype
     const float* d_final_state;   // [N, H, dk, dv], nullable (zeros)
@@ -60,6 +61,7 @@ struct ChunkArgs {
 // Bytes of per-(head, chunk) intermediates: fp32 CUDA-core path / bf16 tensor-core path.
 size_t simt_record_bytes(int dk, int dv);
 size_t tc_record_bytes(int dk, int dv);
+size_t bwd_tiles_bytes(int dk, int dv);   // the tensor-core K1's backward-mode block per (head, chunk)
 
 // Sets the calling thread's kda_last_error() message and returns `status`
 // (status is a kda_status value).
@@ -75,6 +77,7 @@ cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a);  // backward: serial ove
 cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a); // the same on the tensor cores (bf16 inputs)
 cudaError_t launch_chunk_bwd_vside_tc(const ChunkArgs& a); // backward products over the value dim (bf16 inputs)
 cudaError_t launch_chunk_bwd_tchain_tc(const ChunkArgs& a); // backward products through T, W, U0 (bf16 inputs)
+cudaError_t launch_chunk_bwd_split_tc(const ChunkArgs& a);  // backward split-factor products and gradients (bf16)
 cudaError_t launch_chunk_bwd_intra(const ChunkArgs& a);  // backward: all chunks in parallel
 size_t bwd_scratch_bytes_per_cta(int dk, int dv);
 constexpr int kBwdMaxCtas = 512;   // scratch is sized for at most this many CTAs

@@ -252,7 +252,8 @@ kda_status kda_chunk_bwd_gated(const void* q, const void* k, const void* v,
  * inter-chunk stage.  With `count` >= 7, each later kda_chunk_bwd records
  * events[0] before its first kernel and events[1..6] after the chunk-table,
  * forward intra-chunk, forward inter-chunk, reversed inter-chunk, tensor-core
- * product (bf16 inputs; an empty stage for fp32) and per-chunk gradient kernels.
+ * product kernels (bf16 inputs: every chunk without strong decay is finished
+ * there; an empty stage for fp32) and the CUDA-core per-chunk gradient kernel.
  * `count` must be >= 4 (only the first 7 are used).  Pass
  * NULL to stop.  Recording an event costs a few microseconds of stream time
  * and changes no result.
