@@ -446,6 +446,7 @@ bwd_intra_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __re
                 const size_t rstride = chan ? rowk : (size_t)H;
                 const float* la = chan ? log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid
                                        : log_alpha + (size_t)tok0 * H + h;
+#pragma unroll 16   // the loads are independent: keep 16 in flight
                 for (int r = 0; r < kChunk; ++r) {
                     acc += (r < L) ? la[(size_t)r * rstride] : 0.f;
                     sm.g[r][tid] = acc;

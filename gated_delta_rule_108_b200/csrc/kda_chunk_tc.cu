@@ -1907,6 +1907,7 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
                 const size_t rstride = chan ? rowk : (size_t)H;
                 const float* la = chan ? log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid
                                        : log_alpha + (size_t)tok0 * H + h;
+#pragma unroll 16   // the loads are independent: keep 16 in flight
                 for (int r = 0; r < kChunk; ++r) {
                     acc += (r < L) ? la[(size_t)r * rstride] : 0.f;
                     g[r * DK + tid] = acc;
