@@ -1926,7 +1926,7 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
         __syncthreads();
 
         // tf32 operands.  K_r^T, K_l^T, Q_l^T: (channel, 4 tokens) per step
-#pragma unroll 2
+#pragma unroll
         for (int idx = tid; idx < DK * (kChunk / 4); idx += 256) {
             const int ch = idx % DK, r4 = (idx / DK) * 4;
             float kr[4], kl[4], ql[4];
@@ -1950,7 +1950,7 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
             *reinterpret_cast<float4*>(sm + Sm::KLQT + f_off(ch, 64 + r4, DK * 128)) = make_float4(ql[0], ql[1], ql[2], ql[3]);
         }
         // [dM; dP] and their transposes: (row r, 4 columns i) per step
-#pragma unroll 2
+#pragma unroll
         for (int idx = tid; idx < kChunk * (kChunk / 4); idx += 256) {
             const int r = idx >> 4, i4 = (idx & 15) * 4;
             const float4 da = *reinterpret_cast<const float4*>(vs + VS::DA + r * kChunk + i4);
@@ -1991,13 +1991,26 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
                              smem_desc(dmpt + kb * 8192 + ks * 32, 16, 1024, kLayoutSW128), idesc2, (kb | ks) != 0);
             mma_commit(&bar_mma);
         }
-        // meanwhile: dbeta = (parts through W, U0) + rowsum(dA M), one warp per token
-        for (int r = warp; r < L; r += 8) {
-            float part = 0.f;
-            for (int i = lane; i < kChunk; i += 32) part += vs[VS::DA + r * kChunk + i] * Mg[r * kChunk + i];
+        // meanwhile: dbeta = (parts through W, U0) + rowsum(dA M); warp w takes the
+        // tokens w + 8 j, all its loads issued before the sums
+        {
+            float da[16], mm[16];
 #pragma unroll
-            for (int off = 16; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-            if (lane == 0) dbeta[(size_t)(tok0 + r) * H + h] = vs[VS::DBP + r] + part;
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int r = warp + 8 * j, i = lane + 32 * e;
+                    da[2 * j + e] = vs[VS::DA + r * kChunk + i];
+                    mm[2 * j + e] = Mg[r * kChunk + i];
+                }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float part = da[2 * j] * mm[2 * j] + da[2 * j + 1] * mm[2 * j + 1];
+#pragma unroll
+                for (int off = 16; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+                const int r = warp + 8 * j;
+                if (lane == 0 && r < L) dbeta[(size_t)(tok0 + r) * H + h] = vs[VS::DBP + r] + part;
+            }
         }
         mma_pending = 1;
         const bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
@@ -2019,22 +2032,30 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
                 tmem_ld16(T1 + lane_base + col, dkl);
                 tmem_ld16(T1 + lane_base + 64 + col, dql);
                 tmem_ld16(T2 + lane_base + col, dkr);
+                // this half's global operands, all in flight before the arithmetic
+                float kv[16], qv[16], dktv[16], dkhv[16], dqtv[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int r = (int)col + t;
+                    const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
+                    kv[t] = r < L ? __bfloat162float(k[off]) : 0.f;
+                    qv[t] = r < L ? __bfloat162float(q[off]) : 0.f;
+                    dktv[t] = vs[VS::DKT + r * DK + ch];
+                    dkhv[t] = vs[VS::DKH + r * DK + ch];
+                    dqtv[t] = vs[VS::DQT + r * DK + ch];
+                }
                 tmem_wait_ld();
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int r = (int)col + t;
                     const float gg = g[r * DK + ch];
-                    float kk = 0.f, qq = 0.f;
+                    const float kk = kv[t], qq = qv[t];
                     const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
-                    if (r < L) {
-                        kk = __bfloat162float(k[off]);
-                        qq = __bfloat162float(q[off]);
-                    }
                     const float d = gg - gm;
                     const float fl = __expf(d), fr = __expf(-d);
                     const float eg = egm * fl, eh = eglm * fr;   // e^{g}, e^{g_{L-1} - g}
                     const float a = dkl[t] * fl, b = dql[t] * fl, cr = dkr[t] * fr;
-                    const float dkt = vs[VS::DKT + r * DK + ch], dkh = vs[VS::DKH + r * DK + ch], dqt = vs[VS::DQT + r * DK + ch];
+                    const float dkt = dktv[t], dkh = dkhv[t], dqt = dqtv[t];
                     if (r < L) {
                         dk[off] = __float2bfloat16_rn(a + cr + dkt * eg + dkh * eh);
                         dq[off] = __float2bfloat16_rn(b + dqt * eg);
