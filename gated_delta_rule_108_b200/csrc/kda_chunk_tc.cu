@@ -1833,6 +1833,11 @@ bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restric
 // so that TMEM lane = key channel; then the decay factors and the suffix sums
 // of dlog_alpha per channel, and dbeta = (parts through W, U0) + rowsum(dA M)
 // with M from the forward kernel.  Every operand is K-major.
+// A CTA takes its items in turn.  The operand buffers are dead from the end of
+// an item's MMAs, so the next item's k, q, log_alpha (TMA) and dA, dP (bulk
+// copies) are fetched into them then, behind this item's element pass, and an
+// item builds its operands from shared memory.  The item's own dK~ and dK^
+// are bulk-copied into [K_l^T | Q_l^T]'s buffer for its element pass.
 template <int DK, int DV>
 struct SpSmem {
     static constexpr uint32_t G = 0;                        // g (natural log) [64][DK] fp32, later dg
@@ -1841,14 +1846,27 @@ struct SpSmem {
     static constexpr uint32_t DMP = KLQT + 4 * DK * 128;    // [dM; dP] [r][i]: 2 tiles of 128 rows x 128 B
     static constexpr uint32_t DMPT = DMP + 2 * 16384;       // [dM^T | dP^T] [i][r]: 4 tiles of 64 rows x 128 B
     static constexpr uint32_t END = DMPT + 4 * 8192 + 8192; // + a spare tile (128-row reads of the last one)
+    // the next item's inputs, each in a buffer that is written only after it has been read
+    static constexpr uint32_t PF_LA = KRT;                  // log_alpha [64][DK] fp32
+    static constexpr uint32_t PF_K = DMP;                   // k [64][DK] bf16
+    static constexpr uint32_t PF_Q = DMP + 64 * DK * 2;     // q [64][DK] bf16
+    static constexpr uint32_t PF_DA = DMPT;                 // dA [64][64] fp32
+    static constexpr uint32_t PF_DP = DMPT + 64 * 64 * 4;   // dP [64][64] fp32
+    // this item's dK~ and dK^ [64][DK] fp32 for its element pass, under [K_l^T | Q_l^T]
+    static constexpr uint32_t CUR_DKT = KLQT;
+    static constexpr uint32_t CUR_DKH = KLQT + 64 * DK * 4;
+    static_assert(64 * DK * 4 <= KLQT - KRT && 2 * 64 * DK * 2 <= DMPT - DMP && 2 * 64 * 64 * 4 <= END - DMPT &&
+                  2 * 64 * DK * 4 <= DMP - KLQT, "prefetch buffers");
     static_assert(END + 1024 <= 232448, "shared memory");
 };
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(256, 1)
-bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                    const float* __restrict__ log_alpha, const float* __restrict__ beta, ChunkMap map,
-                    WsHeader* hdr, const unsigned char* __restrict__ tiles, const int* __restrict__ flags,
+bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_la, const __nv_bfloat16* __restrict__ q,
+                    const __nv_bfloat16* __restrict__ k, const float* __restrict__ log_alpha,
+                    const float* __restrict__ beta, ChunkMap map, WsHeader* hdr,
+                    const unsigned char* __restrict__ tiles, const int* __restrict__ flags,
                     const float* __restrict__ vside, __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
                     float* __restrict__ dla, float* __restrict__ dbeta, int H, size_t max_chunks, int gate)
 {
@@ -1857,20 +1875,56 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
     using VS = VSide<DK>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar_mma;
+    __shared__ __align__(8) uint64_t bar_mma, bar_load, bar_cur;
     __shared__ uint32_t s_tmem;
     __shared__ float s_gm[DK], s_gl[DK], s_dgl[DK], s_beta[kChunk];
 
     if (hdr->status != kStatusOk) return;
     const int total = hdr->num_chunks * H;
-    if ((int)blockIdx.x >= total) return;
+    // this CTA's items are blockIdx.x + j gridDim.x, less the strong-decay chunks
+    // (the exact CUDA-core path takes those)
+    auto next_item = [&](int x) {
+        while (x < total) {
+            const int c = x / H;
+            if (!flags[(size_t)(x - c * H) * max_chunks + c]) break;
+            x += gridDim.x;
+        }
+        return x;
+    };
+    int w = next_item(blockIdx.x);
+    if (w >= total) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int lane_row = (warp & 3) * 32 + (tid & 31);   // TMEM lane = key channel
     const int wg = warp >> 2;                            // tokens [32 wg, 32 wg + 32)
     const size_t rowk = (size_t)H * DK;
+    const uint32_t load_bytes = 2 * 64 * DK * 2 + 2 * 64 * 64 * 4 + (gate == kGateChannel ? 64 * DK * 4 : 0);
+    auto prefetch = [&](int x) {   // one thread: item x's k, q, log_alpha, dA, dP
+        const int c = x / H, hh = x - c * H;
+        int s_, t0, l_;
+        map.locate(c, s_, t0, l_);
+        const float* xv = vside + ((size_t)hh * max_chunks + c) * VS::FLOATS;
+        mbar_arrive_expect_tx(&bar_load, load_bytes);
+        tma_load_3d(sm + Sm::PF_K, &tm_k, &bar_load, 0, hh, t0);
+        tma_load_3d(sm + Sm::PF_Q, &tm_q, &bar_load, 0, hh, t0);
+        if (gate == kGateChannel) tma_load_3d(sm + Sm::PF_LA, &tm_la, &bar_load, 0, hh, t0);
+        bulk_load(sm + Sm::PF_DA, xv + VS::DA, 64 * 64 * 4, &bar_load);
+        bulk_load(sm + Sm::PF_DP, xv + VS::DP, 64 * 64 * 4, &bar_load);
+    };
+    auto load_beta = [&](int x) {   // threads 128 .. 191: item x's beta of token tid - 128
+        const int c = x / H, hh = x - c * H, r = tid - 128;
+        int s_, t0, l_;
+        map.locate(c, s_, t0, l_);
+        return r < l_ ? beta[(size_t)(t0 + r) * H + hh] : 0.f;
+    };
+    const bool beta_thread = tid >= 128 && tid < 128 + kChunk;
     if (tid == 0) {
         mbar_init(&bar_mma, 1);
+        mbar_init(&bar_load, 1);
+        mbar_init(&bar_cur, 1);
         fence_mbar_init();
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_q);
+        if (gate == kGateChannel) tma_prefetch_desc(&tm_la);
     }
     if (warp == 0) {
         tmem_alloc(&s_tmem, 256);
@@ -1883,82 +1937,103 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
     const uint32_t T1 = tmem;          // [dK_l^T | dQ_l^T]: 128 columns (token r)
     const uint32_t T2 = tmem + 128;    // dK_r^T: 64 columns (token i)
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    uint32_t mma_phase = 0;
-    bool aborted = false;
-    int mma_pending = 0;
+    if (tid == 0) prefetch(w);
+    float bnext = beta_thread ? load_beta(w) : 0.f;
+    uint32_t mma_phase = 0, load_phase = 0, cur_phase = 0;
+    bool aborted = false, load_pending = true, mma_pending = false, cur_pending = false;
     float* g = reinterpret_cast<float*>(sm + Sm::G);
 
-    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x) {
+    while (w < total) {
         const int c = w / H, h = w - c * H;
         const size_t it = (size_t)h * max_chunks + c;
-        if (flags[it]) continue;   // strong decay: the exact CUDA-core path handles this chunk
         int seq, tok0, L;
         map.locate(c, seq, tok0, L);
+        const int nw = next_item(w + gridDim.x);
         const float* vs = vside + it * VS::FLOATS;
         const float* Mg = reinterpret_cast<const float*>(tiles + it * BT::BYTES + BT::M);
+        if (beta_thread) s_beta[tid - 128] = bnext;
+        // this thread's rows of M and dbeta parts through W, U0 (used once the MMAs are issued):
+        // step j covers row r = (tid + 256 j) / 16, columns 4 ((tid + 256 j) % 16) + [0, 4)
+        float4 mm[4];
+        float dbp[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int idx = tid + 256 * j, r = idx >> 4, i4 = (idx & 15) * 4;
+            mm[j] = *reinterpret_cast<const float4*>(Mg + r * kChunk + i4);
+            dbp[j] = vs[VS::DBP + r];
+        }
+        const bool got = mbar_wait_cycles(&bar_load, load_phase, kWaitCycles);
+        if (__syncthreads_or(!got)) { aborted = true; break; }
+        load_phase ^= 1;
+        load_pending = false;
 
-        // cumulative log-decay (natural log) per channel; beta
+        // cumulative log-decay (natural log) per channel; g_m, g_{L-1}
         if (tid < DK) {
             float acc = 0.f;
-            if (gate == kGateNone) {
-                for (int r = 0; r < kChunk; ++r) g[r * DK + tid] = 0.f;
-            } else {
-                const bool chan = gate == kGateChannel;
-                const size_t rstride = chan ? rowk : (size_t)H;
-                const float* la = chan ? log_alpha + (size_t)tok0 * rowk + (size_t)h * DK + tid
-                                       : log_alpha + (size_t)tok0 * H + h;
-#pragma unroll 16   // the loads are independent: keep 16 in flight
+            if (gate == kGateChannel) {
+                const float* la = reinterpret_cast<const float*>(sm + Sm::PF_LA) + tid;
+#pragma unroll 16
                 for (int r = 0; r < kChunk; ++r) {
-                    acc += (r < L) ? la[(size_t)r * rstride] : 0.f;
+                    acc += (r < L) ? la[r * DK] : 0.f;
                     g[r * DK + tid] = acc;
                 }
+            } else if (gate == kGateHead) {
+                const float* la = log_alpha + (size_t)tok0 * H + h;
+#pragma unroll 16   // the loads are independent: keep 16 in flight
+                for (int r = 0; r < kChunk; ++r) {
+                    acc += (r < L) ? la[(size_t)r * H] : 0.f;
+                    g[r * DK + tid] = acc;
+                }
+            } else {
+                for (int r = 0; r < kChunk; ++r) g[r * DK + tid] = 0.f;
             }
-            s_dgl[tid] = 0.f;
-        } else if (tid >= 128 && tid < 128 + kChunk) {
-            const int r = tid - 128;
-            s_beta[r] = r < L ? beta[(size_t)(tok0 + r) * H + h] : 0.f;
-        }
-        __syncthreads();
-        if (tid < DK) {
             s_gm[tid] = g[((L - 1) >> 1) * DK + tid];
             s_gl[tid] = g[(L - 1) * DK + tid];
+            s_dgl[tid] = 0.f;
+        }
+        float4 da[4], dp[4];   // same (row, 4 columns) steps as mm
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int idx = tid + 256 * j;
+            da[j] = reinterpret_cast<const float4*>(sm + Sm::PF_DA)[idx];   // row idx / 16, columns 4 (idx % 16) + [0, 4)
+            dp[j] = reinterpret_cast<const float4*>(sm + Sm::PF_DP)[idx];
         }
         __syncthreads();
 
         // tf32 operands.  K_r^T, K_l^T, Q_l^T: (channel, 4 tokens) per step
+        {
+            const __nv_bfloat16* pk = reinterpret_cast<const __nv_bfloat16*>(sm + Sm::PF_K);
+            const __nv_bfloat16* pq = reinterpret_cast<const __nv_bfloat16*>(sm + Sm::PF_Q);
 #pragma unroll
-        for (int idx = tid; idx < DK * (kChunk / 4); idx += 256) {
-            const int ch = idx % DK, r4 = (idx / DK) * 4;
-            float kr[4], kl[4], ql[4];
+            for (int idx = tid; idx < DK * (kChunk / 4); idx += 256) {
+                const int ch = idx % DK, r4 = (idx / DK) * 4;
+                float kr[4], kl[4], ql[4];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int r = r4 + t;
-                float kk = 0.f, qq = 0.f;
-                if (r < L) {
-                    const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
-                    kk = __bfloat162float(k[off]);
-                    qq = __bfloat162float(q[off]);
+                for (int t = 0; t < 4; ++t) {
+                    const int r = r4 + t;
+                    const float kk = r < L ? __bfloat162float(pk[r * DK + ch]) : 0.f;
+                    const float qq = r < L ? __bfloat162float(pq[r * DK + ch]) : 0.f;
+                    const float d = g[r * DK + ch] - s_gm[ch];
+                    const float fl = __expf(d), fr = __expf(-d);
+                    kr[t] = round_tf32_alu(kk * fr);
+                    kl[t] = round_tf32_alu(kk * fl);
+                    ql[t] = round_tf32_alu(qq * fl);
                 }
-                const float d = g[r * DK + ch] - s_gm[ch];
-                const float fl = __expf(d), fr = __expf(-d);
-                kr[t] = round_tf32_alu(kk * fr);
-                kl[t] = round_tf32_alu(kk * fl);
-                ql[t] = round_tf32_alu(qq * fl);
+                *reinterpret_cast<float4*>(sm + Sm::KRT + f_off(ch, r4, DK * 128)) = make_float4(kr[0], kr[1], kr[2], kr[3]);
+                *reinterpret_cast<float4*>(sm + Sm::KLQT + f_off(ch, r4, DK * 128)) = make_float4(kl[0], kl[1], kl[2], kl[3]);
+                *reinterpret_cast<float4*>(sm + Sm::KLQT + f_off(ch, 64 + r4, DK * 128)) = make_float4(ql[0], ql[1], ql[2], ql[3]);
             }
-            *reinterpret_cast<float4*>(sm + Sm::KRT + f_off(ch, r4, DK * 128)) = make_float4(kr[0], kr[1], kr[2], kr[3]);
-            *reinterpret_cast<float4*>(sm + Sm::KLQT + f_off(ch, r4, DK * 128)) = make_float4(kl[0], kl[1], kl[2], kl[3]);
-            *reinterpret_cast<float4*>(sm + Sm::KLQT + f_off(ch, 64 + r4, DK * 128)) = make_float4(ql[0], ql[1], ql[2], ql[3]);
         }
-        // [dM; dP] and their transposes: (row r, 4 columns i) per step
+        __syncthreads();   // k, q (under [dM; dP]) and dA, dP (under its transpose) are read
+        // [dM; dP] and their transposes
 #pragma unroll
-        for (int idx = tid; idx < kChunk * (kChunk / 4); idx += 256) {
-            const int r = idx >> 4, i4 = (idx & 15) * 4;
-            const float4 da = *reinterpret_cast<const float4*>(vs + VS::DA + r * kChunk + i4);
-            const float4 dp = *reinterpret_cast<const float4*>(vs + VS::DP + r * kChunk + i4);
+        for (int j = 0; j < 4; ++j) {
+            const int idx = tid + 256 * j, r = idx >> 4, i4 = (idx & 15) * 4;
             const float br = s_beta[r];
-            const float dm[4] = {round_tf32_alu(br * da.x), round_tf32_alu(br * da.y),
-                                 round_tf32_alu(br * da.z), round_tf32_alu(br * da.w)};
-            const float pp[4] = {round_tf32_alu(dp.x), round_tf32_alu(dp.y), round_tf32_alu(dp.z), round_tf32_alu(dp.w)};
+            const float dm[4] = {round_tf32_alu(br * da[j].x), round_tf32_alu(br * da[j].y),
+                                 round_tf32_alu(br * da[j].z), round_tf32_alu(br * da[j].w)};
+            const float pp[4] = {round_tf32_alu(dp[j].x), round_tf32_alu(dp[j].y), round_tf32_alu(dp[j].z),
+                                 round_tf32_alu(dp[j].w)};
             *reinterpret_cast<float4*>(sm + Sm::DMP + f_off(r, i4, 16384)) = make_float4(dm[0], dm[1], dm[2], dm[3]);
             *reinterpret_cast<float4*>(sm + Sm::DMP + f_off(64 + r, i4, 16384)) = make_float4(pp[0], pp[1], pp[2], pp[3]);
 #pragma unroll
@@ -1991,71 +2066,79 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
                              smem_desc(dmpt + kb * 8192 + ks * 32, 16, 1024, kLayoutSW128), idesc2, (kb | ks) != 0);
             mma_commit(&bar_mma);
         }
-        // meanwhile: dbeta = (parts through W, U0) + rowsum(dA M); warp w takes the
-        // tokens w + 8 j, all its loads issued before the sums
-        {
-            float da[16], mm[16];
+        mma_pending = true;
+        // this thread's element-pass operands from global memory (channel lane_row,
+        // tokens [32 wg, 32 wg + 32)), in flight across the MMAs
+        __nv_bfloat16 kv[32], qv[32];
+        float dqtv[32];
+        if (lane_row < DK) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int r = warp + 8 * j, i = lane + 32 * e;
-                    da[2 * j + e] = vs[VS::DA + r * kChunk + i];
-                    mm[2 * j + e] = Mg[r * kChunk + i];
-                }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float part = da[2 * j] * mm[2 * j] + da[2 * j + 1] * mm[2 * j + 1];
-#pragma unroll
-                for (int off = 16; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-                const int r = warp + 8 * j;
-                if (lane == 0 && r < L) dbeta[(size_t)(tok0 + r) * H + h] = vs[VS::DBP + r] + part;
+            for (int t = 0; t < 32; ++t) {
+                const int r = 32 * wg + t;
+                const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + lane_row;
+                kv[t] = r < L ? k[off] : __float2bfloat16_rn(0.f);
+                qv[t] = r < L ? q[off] : __float2bfloat16_rn(0.f);
+                dqtv[t] = vs[VS::DQT + r * DK + lane_row];
             }
         }
-        mma_pending = 1;
+        // meanwhile: dbeta = (parts through W, U0) + rowsum(dA M); a row's 16 steps
+        // sit in one half-warp
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float part = da[j].x * mm[j].x + da[j].y * mm[j].y + da[j].z * mm[j].z + da[j].w * mm[j].w;
+#pragma unroll
+            for (int off = 8; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+            const int r = (tid + 256 * j) >> 4;
+            if ((lane & 15) == 0 && r < L) dbeta[(size_t)(tok0 + r) * H + h] = dbp[j] + part;
+        }
         const bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        mma_phase ^= 1;
-        mma_pending = 0;
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        mma_phase ^= 1;
+        mma_pending = false;
         tc_fence_after();
+        // the operand buffers are free: this item's dK~, dK^ and the next item's
+        // inputs land behind the element pass
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&bar_cur, 2 * 64 * DK * 4);
+            bulk_load(sm + Sm::CUR_DKT, vs + VS::DKT, 64 * DK * 4, &bar_cur);
+            bulk_load(sm + Sm::CUR_DKH, vs + VS::DKH, 64 * DK * 4, &bar_cur);
+        }
+        cur_pending = true;
+        if (nw < total) {
+            if (tid == 0) prefetch(nw);
+            load_pending = true;
+            if (beta_thread) bnext = load_beta(nw);
+        }
 
         // dq, dk and dg for channel lane_row, tokens [32 wg, 32 wg + 32)
+        bool cur_ok = true;
+        const float* s_dkt = reinterpret_cast<const float*>(sm + Sm::CUR_DKT);
+        const float* s_dkh = reinterpret_cast<const float*>(sm + Sm::CUR_DKH);
         if (lane_row < DK) {
             const int ch = lane_row;
             const float gm = s_gm[ch], gl = s_gl[ch];
             const float egm = __expf(gm), eglm = __expf(gl - gm);
             float dgl = 0.f;
-#pragma unroll 1
+#pragma unroll
             for (int half = 0; half < 2; ++half) {   // 16 tokens at a time
                 float dkl[16], dql[16], dkr[16];
                 const uint32_t col = 32 * wg + 16 * half;
                 tmem_ld16(T1 + lane_base + col, dkl);
                 tmem_ld16(T1 + lane_base + 64 + col, dql);
                 tmem_ld16(T2 + lane_base + col, dkr);
-                // this half's global operands, all in flight before the arithmetic
-                float kv[16], qv[16], dktv[16], dkhv[16], dqtv[16];
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const int r = (int)col + t;
-                    const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
-                    kv[t] = r < L ? __bfloat162float(k[off]) : 0.f;
-                    qv[t] = r < L ? __bfloat162float(q[off]) : 0.f;
-                    dktv[t] = vs[VS::DKT + r * DK + ch];
-                    dkhv[t] = vs[VS::DKH + r * DK + ch];
-                    dqtv[t] = vs[VS::DQT + r * DK + ch];
-                }
                 tmem_wait_ld();
+                if (half == 0 && !mbar_wait_cycles(&bar_cur, cur_phase, kWaitCycles)) cur_ok = false;
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int r = (int)col + t;
                     const float gg = g[r * DK + ch];
-                    const float kk = kv[t], qq = qv[t];
+                    const float kk = __bfloat162float(kv[16 * half + t]), qq = __bfloat162float(qv[16 * half + t]);
                     const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
                     const float d = gg - gm;
                     const float fl = __expf(d), fr = __expf(-d);
                     const float eg = egm * fl, eh = eglm * fr;   // e^{g}, e^{g_{L-1} - g}
                     const float a = dkl[t] * fl, b = dql[t] * fl, cr = dkr[t] * fr;
-                    const float dkt = dktv[t], dkh = dkhv[t], dqt = dqtv[t];
+                    const float dkt = s_dkt[r * DK + ch], dkh = s_dkh[r * DK + ch], dqt = dqtv[16 * half + t];
                     if (r < L) {
                         dk[off] = __float2bfloat16_rn(a + cr + dkt * eg + dkh * eh);
                         dq[off] = __float2bfloat16_rn(b + dqt * eg);
@@ -2067,7 +2150,9 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
             }
             atomicAdd(&s_dgl[ch], dgl);
         }
-        __syncthreads();
+        if (__syncthreads_or(!cur_ok)) { aborted = true; break; }
+        cur_phase ^= 1;
+        cur_pending = false;
         // dlog_alpha_s = sum_{r >= s} dg_r (+ g_{L-1}'s own cotangent), per channel
         if (gate != kGateNone && tid < DK) {
             float run = s_dgl[tid] + vs[VS::DGAM + tid] * __expf(s_gl[tid]);
@@ -2086,12 +2171,15 @@ bwd_split_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
             }
         }
         tc_fence_before();
-        __syncthreads();   // smem and TMEM are free for the next item
+        __syncthreads();   // g, s_beta and TMEM are free for the next item
+        w = nw;
     }
 
     if (aborted) {
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        if (load_pending) (void)mbar_wait_cycles(&bar_load, load_phase, kWaitCycles / 4);
+        if (cur_pending) (void)mbar_wait_cycles(&bar_cur, cur_phase, kWaitCycles / 4);
     }
     tc_fence_before();
     __syncthreads();
@@ -2236,6 +2324,14 @@ cudaError_t launch_bwd_tchain_tc_t(const ChunkArgs& a) {
 template <int DK, int DV>
 cudaError_t launch_bwd_split_tc_t(const ChunkArgs& a) {
     if (a.max_chunks == 0) return cudaSuccess;
+    const int ntok = a.cu_seqlens ? a.T : a.B * a.T;
+    CUtensorMap mk, mq, mla;
+    if (!make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, DK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, DK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        (a.gate == kGateChannel &&
+         !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, ntok, DK, CU_TENSOR_MAP_SWIZZLE_NONE)))
+        return cudaErrorInvalidValue;
+    if (a.gate != kGateChannel) memset(&mla, 0, sizeof(mla));   // unused
     ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
     auto kern = bwd_split_tc_kernel<DK, DV>;
     const int smem = (int)SpSmem<DK, DV>::END + 1024;
@@ -2247,10 +2343,10 @@ cudaError_t launch_bwd_split_tc_t(const ChunkArgs& a) {
     const size_t items = a.max_chunks * (size_t)a.H;
     const unsigned grid = (unsigned)(items < (size_t)sms ? items : (size_t)sms);
     kern<<<grid, 256, smem, a.stream>>>(
-        static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k), a.log_alpha, a.beta, map,
-        static_cast<WsHeader*>(a.ws_header), static_cast<const unsigned char*>(a.bwd_tiles), a.bwd_flags, a.vside,
-        static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dk_out), a.dlog_alpha, a.dbeta, a.H,
-        a.max_chunks, a.gate);
+        mq, mk, mla, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k), a.log_alpha,
+        a.beta, map, static_cast<WsHeader*>(a.ws_header), static_cast<const unsigned char*>(a.bwd_tiles),
+        a.bwd_flags, a.vside, static_cast<__nv_bfloat16*>(a.dq), static_cast<__nv_bfloat16*>(a.dk_out),
+        a.dlog_alpha, a.dbeta, a.H, a.max_chunks, a.gate);
     return cudaGetLastError();
 }
 
