@@ -1321,37 +1321,67 @@ bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsH
     bool aborted = false;
     int mma_pending = 0;
 
-    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x) {
+    // an item's S, dS' (DK x DV) and dU (64 x DV) in fp32, 8 columns per thread and
+    // step; the next item's are loaded into registers while this item's last
+    // products and write-out run
+    constexpr int NSD = DK * DV / 8 / 256, NU = kChunk * DV / 8 / 256;
+    static_assert(DK * DV / 8 % 256 == 0 && kChunk * DV / 8 % 256 == 0, "whole steps");
+    float4 rs[2 * NSD], rd[2 * NSD], ru[2 * NU];
+    auto load_item = [&](int x) {
+        const int c = x / H, hh = x - c * H;
+        const size_t it = (size_t)hh * max_chunks + c;
+        const float* Sn = states + it * DK * DV;
+        const float* dSe = dS_end + it * DK * DV;
+        const float* dUc = dU_all + it * kChunk * DV;
+#pragma unroll
+        for (int j = 0; j < NSD; ++j) {
+            const int idx = tid + 256 * j, ch = idx / (DV / 8), j8 = (idx - ch * (DV / 8)) * 8;
+            rs[2 * j] = *reinterpret_cast<const float4*>(Sn + (size_t)ch * DV + j8);
+            rs[2 * j + 1] = *reinterpret_cast<const float4*>(Sn + (size_t)ch * DV + j8 + 4);
+            rd[2 * j] = *reinterpret_cast<const float4*>(dSe + (size_t)ch * DV + j8);
+            rd[2 * j + 1] = *reinterpret_cast<const float4*>(dSe + (size_t)ch * DV + j8 + 4);
+        }
+#pragma unroll
+        for (int j = 0; j < NU; ++j) {
+            const int idx = tid + 256 * j, r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
+            ru[2 * j] = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8);
+            ru[2 * j + 1] = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8 + 4);
+        }
+    };
+    auto issue_tiles = [&](int x) {   // one thread: item x's record tiles and d_o
+        const int c = x / H, hh = x - c * H;
+        int s_, t0, l_;
+        map.locate(c, s_, t0, l_);
+        const unsigned char* rec = records + ((size_t)hh * max_chunks + c) * R::BYTES;
+        mbar_arrive_expect_tx(&bar_load, Sm::TX_BYTES);
+        bulk_load(sm + Sm::WQ, rec + R::WQ, R::WQ_BYTES, &bar_load);
+        bulk_load(sm + Sm::U0, rec + R::U0, R::U0_BYTES, &bar_load);
+#pragma unroll
+        for (int b = 0; b < NJ; ++b) tma_load_3d(sm + Sm::AB + b * 16384, &tm_do, &bar_load, b * 64, hh, t0);
+    };
+    int w = blockIdx.x;
+    if (tid == 0) issue_tiles(w);
+    bool load_pending = true;
+    load_item(w);
+
+    while (w < total) {
         const int c = w / H, h = w - c * H;
         int seq, tok0, L;
         map.locate(c, seq, tok0, L);
         const size_t it = (size_t)h * max_chunks + c;
-        const unsigned char* rec = records + it * R::BYTES;
-        const float* Sn = states + it * DK * DV;
-        const float* dSe = dS_end + it * DK * DV;
-        const float* dUc = dU_all + it * kChunk * DV;
         float* out = vside + it * VS::FLOATS;
+        const int nw = w + gridDim.x;
 
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_load, Sm::TX_BYTES);
-            bulk_load(sm + Sm::WQ, rec + R::WQ, R::WQ_BYTES, &bar_load);
-            bulk_load(sm + Sm::U0, rec + R::U0, R::U0_BYTES, &bar_load);
-#pragma unroll
-            for (int b = 0; b < NJ; ++b) tma_load_3d(sm + Sm::AB + b * 16384, &tm_do, &bar_load, b * 64, h, tok0);
-        }
         if (tid < DK) s_dgam[tid] = 0.f;
         __syncthreads();
         // fp16 operands: S and dS' (rows = key channel), -dU (rows 64..127 of [D; -dU]); dgamma
         // DV / 8 consecutive threads share a key row: their dgamma parts are
         // summed by shuffles, then added once (DV / 8 divides 32)
         static_assert(32 % (DV / 8) == 0, "row groups within a warp");
-#pragma unroll 4
-        for (int idx = tid; idx < DK * DV / 8; idx += 256) {
-            const int ch = idx / (DV / 8), j8 = (idx - ch * (DV / 8)) * 8;
-            const float4 s0 = *reinterpret_cast<const float4*>(Sn + (size_t)ch * DV + j8);
-            const float4 s1 = *reinterpret_cast<const float4*>(Sn + (size_t)ch * DV + j8 + 4);
-            const float4 d0 = *reinterpret_cast<const float4*>(dSe + (size_t)ch * DV + j8);
-            const float4 d1 = *reinterpret_cast<const float4*>(dSe + (size_t)ch * DV + j8 + 4);
+#pragma unroll
+        for (int j = 0; j < NSD; ++j) {
+            const int idx = tid + 256 * j, ch = idx / (DV / 8), j8 = (idx - ch * (DV / 8)) * 8;
+            const float4 s0 = rs[2 * j], s1 = rs[2 * j + 1], d0 = rd[2 * j], d1 = rd[2 * j + 1];
             float gpart = s0.x * d0.x + s0.y * d0.y + s0.z * d0.z + s0.w * d0.w +
                           s1.x * d1.x + s1.y * d1.y + s1.z * d1.z + s1.w * d1.w;
 #pragma unroll
@@ -1369,11 +1399,10 @@ bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsH
             *reinterpret_cast<uint4*>(sm + Sm::S16 + o) = *reinterpret_cast<const uint4*>(hs);
             *reinterpret_cast<uint4*>(sm + Sm::DS16 + o) = *reinterpret_cast<const uint4*>(hd);
         }
-#pragma unroll 4
-        for (int idx = tid; idx < kChunk * DV / 8; idx += 256) {
-            const int r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
-            const float4 u0 = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8);
-            const float4 u1 = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8 + 4);
+#pragma unroll
+        for (int j = 0; j < NU; ++j) {
+            const int idx = tid + 256 * j, r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
+            const float4 u0 = ru[2 * j], u1 = ru[2 * j + 1];
             __align__(16) __half2 hu[4] = {__floats2half2_rn(-u0.x, -u0.y), __floats2half2_rn(-u0.z, -u0.w),
                                            __floats2half2_rn(-u1.x, -u1.y), __floats2half2_rn(-u1.z, -u1.w)};
             range_max = fmaxf(range_max, fmaxf(fmaxf(fabsf(u0.x), fabsf(u0.y)), fmaxf(fabsf(u0.z), fabsf(u0.w))));
@@ -1383,8 +1412,9 @@ bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsH
         }
         // D = c dO: bf16 -> fp16 in place (rows 0..63 of [D; -dU]); rows past the chunk are zero
         const bool ok_load = mbar_wait_cycles(&bar_load, load_phase, kWaitCycles);
-        load_phase ^= 1;
         if (__syncthreads_or(!ok_load)) { aborted = true; break; }
+        load_phase ^= 1;
+        load_pending = false;
         for (int idx = tid; idx < kChunk * DV / 8; idx += 256) {
             const int r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
             const uint32_t o = Sm::AB + (j8 >> 6) * 16384 + sw128_offset(r, (j8 & 63) * 2);
@@ -1428,9 +1458,9 @@ bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsH
         }
         mma_pending = 1;
         bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
         mma_phase ^= 1;
         mma_pending = 0;
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
         tc_fence_after();
 
         // U = U0 - W S (rows 0..63) -> fp16 U tiles
@@ -1495,11 +1525,17 @@ bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsH
             mma_commit(&bar_mma);
         }
         mma_pending = 1;
+        if (nw < total) load_item(nw);   // in flight across these MMAs and the write-out below
         ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
         mma_phase ^= 1;
         mma_pending = 0;
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
         tc_fence_after();
+        // every operand buffer is read: the next item's record tiles and d_o come in
+        if (nw < total) {
+            if (tid == 0) issue_tiles(nw);
+            load_pending = true;
+        }
 
         // dK^ and dP (rows 0..63) out; dgamma
         if (lane_row < 64) {
@@ -1528,12 +1564,13 @@ bwd_vside_tc_kernel(const __grid_constant__ CUtensorMap tm_do, ChunkMap map, WsH
         if (tid < DK) out[VS::DGAM + tid] = s_dgam[tid];
         tc_fence_before();
         __syncthreads();   // smem and TMEM are free for the next item
+        w = nw;
     }
 
     if (aborted) {
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        (void)mbar_wait_cycles(&bar_load, load_phase, kWaitCycles / 4);
+        if (load_pending) (void)mbar_wait_cycles(&bar_load, load_phase, kWaitCycles / 4);
     }
     if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
     tc_fence_before();
