@@ -1647,8 +1647,10 @@ bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restric
     auto mma_wait = [&]() -> bool {
         mma_pending = 1;
         const bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        mma_phase ^= 1;
-        mma_pending = 0;
+        if (ok) {
+            mma_phase ^= 1;
+            mma_pending = 0;
+        }
         return ok;
     };
     // fp16 copy of 8 fp32 values into a swizzled tile row
@@ -1660,45 +1662,72 @@ bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restric
         *reinterpret_cast<uint4*>(sm + off) = *reinterpret_cast<const uint4*>(hv);
     };
 
-    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x) {
+    // an item's dU (64 x DV) and dW (64 x DK) in fp32, 8 columns per thread and
+    // step; the next item's are loaded into registers while this item's
+    // write-out and last products run
+    constexpr int NUJ = kChunk * DV / 8 / 256, NWJ = kChunk * DK / 8 / 256;
+    static_assert(kChunk * DV / 8 % 256 == 0 && kChunk * DK / 8 % 256 == 0, "whole steps");
+    float4 ru[2 * NUJ], rw[2 * NWJ];
+    auto load_item = [&](int x) {
+        const int c = x / H, hh = x - c * H;
+        const size_t it = (size_t)hh * max_chunks + c;
+        const float* dUc = dU_all + it * kChunk * DV;
+        const float* dWc = vside + it * VS::FLOATS + VS::DW;
+#pragma unroll
+        for (int j = 0; j < NUJ; ++j) {
+            const int idx = tid + 256 * j, r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
+            ru[2 * j] = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8);
+            ru[2 * j + 1] = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8 + 4);
+        }
+#pragma unroll
+        for (int j = 0; j < NWJ; ++j) {
+            const int idx = tid + 256 * j, r = idx / (DK / 8), c8 = (idx - r * (DK / 8)) * 8;
+            rw[2 * j] = *reinterpret_cast<const float4*>(dWc + (size_t)r * DK + c8);
+            rw[2 * j + 1] = *reinterpret_cast<const float4*>(dWc + (size_t)r * DK + c8 + 4);
+        }
+    };
+    auto issue_tiles = [&](int x) {   // one thread: item x's fp16 T, K~, V tiles
+        const int c = x / H, hh = x - c * H;
+        const unsigned char* tl = tiles + ((size_t)hh * max_chunks + c) * BT::BYTES;
+        mbar_arrive_expect_tx(&bar_load, BT::TILE_BYTES);
+        bulk_load(sm + Sm::T, tl + BT::T, 8192, &bar_load);
+        bulk_load(sm + Sm::KT, tl + BT::KT, (DK / 64) * 8192, &bar_load);
+        bulk_load(sm + Sm::V, tl + BT::V, (DV / 64) * 8192, &bar_load);
+    };
+    int w = blockIdx.x;
+    if (tid == 0) issue_tiles(w);
+    bool load_pending = true;
+    load_item(w);
+
+    while (w < total) {
         const int c = w / H, h = w - c * H;
         int seq, tok0, L;
         map.locate(c, seq, tok0, L);
         const size_t it = (size_t)h * max_chunks + c;
-        const unsigned char* tl = tiles + it * BT::BYTES;
-        const float* dUc = dU_all + it * kChunk * DV;
         float* out = vside + it * VS::FLOATS;
+        const int nw = w + gridDim.x;
 
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_load, BT::TILE_BYTES);
-            bulk_load(sm + Sm::T, tl + BT::T, 8192, &bar_load);
-            bulk_load(sm + Sm::KT, tl + BT::KT, (DK / 64) * 8192, &bar_load);
-            bulk_load(sm + Sm::V, tl + BT::V, (DV / 64) * 8192, &bar_load);
-        }
         if (tid < kChunk) {
             s_beta[tid] = tid < L ? beta[(size_t)(tok0 + tid) * H + h] : 0.f;
             s_dbp[tid] = 0.f;
         }
         // dU and dW (rows = token) as fp16 tiles
-#pragma unroll 4
-        for (int idx = tid; idx < kChunk * DV / 8; idx += 256) {
-            const int r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
-            const float4 a = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8);
-            const float4 b = *reinterpret_cast<const float4*>(dUc + (size_t)r * DV + j8 + 4);
-            put8(Sm::DU + (j8 >> 6) * 8192 + sw128_offset(r, (j8 & 63) * 2), a, b, 1.f);
+#pragma unroll
+        for (int j = 0; j < NUJ; ++j) {
+            const int idx = tid + 256 * j, r = idx / (DV / 8), j8 = (idx - r * (DV / 8)) * 8;
+            put8(Sm::DU + (j8 >> 6) * 8192 + sw128_offset(r, (j8 & 63) * 2), ru[2 * j], ru[2 * j + 1], 1.f);
         }
-#pragma unroll 4
-        for (int idx = tid; idx < kChunk * DK / 8; idx += 256) {
-            const int r = idx / (DK / 8), c8 = (idx - r * (DK / 8)) * 8;
-            const float4 a = *reinterpret_cast<const float4*>(out + VS::DW + (size_t)r * DK + c8);
-            const float4 b = *reinterpret_cast<const float4*>(out + VS::DW + (size_t)r * DK + c8 + 4);
-            put8(Sm::DW + (c8 >> 6) * 8192 + sw128_offset(r, (c8 & 63) * 2), a, b, 1.f);
+#pragma unroll
+        for (int j = 0; j < NWJ; ++j) {
+            const int idx = tid + 256 * j, r = idx / (DK / 8), c8 = (idx - r * (DK / 8)) * 8;
+            put8(Sm::DW + (c8 >> 6) * 8192 + sw128_offset(r, (c8 & 63) * 2), rw[2 * j], rw[2 * j + 1], 1.f);
         }
         const bool ok_load = mbar_wait_cycles(&bar_load, load_phase, kWaitCycles);
-        load_phase ^= 1;
         fence_proxy_async_smem();
         tc_fence_before();
         if (__syncthreads_or(!ok_load)) { aborted = true; break; }
+        load_phase ^= 1;
+        load_pending = false;
 
         // [Z | Y] = T^T [dU | dW];  dT_raw = dW K~^T + dU V^T
         if (tid == 0) {
@@ -1757,6 +1786,7 @@ bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restric
                         smem_desc(t + ks * 32, 16, 1024, kLayoutSW128), idesc, ks != 0);
             mma_commit(&bar_mma);
         }
+        if (nw < total) load_item(nw);   // in flight across the rest of this item
         // meanwhile: dv = beta Z (out), dK~ = beta Y (out), dbeta parts <Z, v> + <Y, K~>
         if (lane_row < 64) {
             const int r = lane_row;
@@ -1833,6 +1863,11 @@ bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restric
         ok = mma_wait();
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         tc_fence_after();
+        // every tile is read: the next item's come in
+        if (nw < total) {
+            if (tid == 0) issue_tiles(nw);
+            load_pending = true;
+        }
         // dA = -T^T X1, strictly lower (rows 0..63); dbeta parts
         if (lane_row < 64) {
             float v[32];
@@ -1849,12 +1884,13 @@ bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restric
         if (tid < kChunk) out[VS::DBP + tid] = s_dbp[tid];
         tc_fence_before();
         __syncthreads();   // smem and TMEM are free for the next item
+        w = nw;
     }
 
     if (aborted) {
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        (void)mbar_wait_cycles(&bar_load, load_phase, kWaitCycles / 4);
+        if (load_pending) (void)mbar_wait_cycles(&bar_load, load_phase, kWaitCycles / 4);
     }
     if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
     tc_fence_before();
