@@ -1909,8 +1909,9 @@ bwd_tchain_tc_kernel(ChunkMap map, WsHeader* hdr, const unsigned char* __restric
 // A CTA takes its items in turn.  The operand buffers are dead from the end of
 // an item's MMAs, so the next item's k, q, log_alpha (TMA) and dA, dP (bulk
 // copies) are fetched into them then, behind this item's element pass, and an
-// item builds its operands from shared memory.  The item's own dK~ and dK^
-// are bulk-copied into [K_l^T | Q_l^T]'s buffer for its element pass.
+// item builds its operands from shared memory.  The operand build keeps a copy
+// of the item's k and q for its element pass, whose other operands (dK~, dK^,
+// dQ~) load into registers while the MMAs run.
 template <int DK, int DV>
 struct SpSmem {
     static constexpr uint32_t G = 0;                        // g (natural log) [64][DK] fp32, later dg
@@ -1918,18 +1919,16 @@ struct SpSmem {
     static constexpr uint32_t KLQT = KRT + 2 * DK * 128;    // [K_l^T | Q_l^T] [c][r]: 4 tiles
     static constexpr uint32_t DMP = KLQT + 4 * DK * 128;    // [dM; dP] [r][i]: 2 tiles of 128 rows x 128 B
     static constexpr uint32_t DMPT = DMP + 2 * 16384;       // [dM^T | dP^T] [i][r]: 4 tiles of 64 rows x 128 B
-    static constexpr uint32_t END = DMPT + 4 * 8192 + 8192; // + a spare tile (128-row reads of the last one)
+    static constexpr uint32_t KQ = DMPT + 4 * 8192;         // this item's k, q [64][DK] bf16, for its element pass
+    static constexpr uint32_t END = KQ + 2 * 64 * DK * 2;
     // the next item's inputs, each in a buffer that is written only after it has been read
     static constexpr uint32_t PF_LA = KRT;                  // log_alpha [64][DK] fp32
     static constexpr uint32_t PF_K = DMP;                   // k [64][DK] bf16
     static constexpr uint32_t PF_Q = DMP + 64 * DK * 2;     // q [64][DK] bf16
     static constexpr uint32_t PF_DA = DMPT;                 // dA [64][64] fp32
     static constexpr uint32_t PF_DP = DMPT + 64 * 64 * 4;   // dP [64][64] fp32
-    // this item's dK~ and dK^ [64][DK] fp32 for its element pass, under [K_l^T | Q_l^T]
-    static constexpr uint32_t CUR_DKT = KLQT;
-    static constexpr uint32_t CUR_DKH = KLQT + 64 * DK * 4;
-    static_assert(64 * DK * 4 <= KLQT - KRT && 2 * 64 * DK * 2 <= DMPT - DMP && 2 * 64 * 64 * 4 <= END - DMPT &&
-                  2 * 64 * DK * 4 <= DMP - KLQT, "prefetch buffers");
+    static_assert(64 * DK * 4 <= KLQT - KRT && 2 * 64 * DK * 2 <= DMPT - DMP && 2 * 64 * 64 * 4 <= KQ - DMPT,
+                  "prefetch buffers");
     static_assert(END + 1024 <= 232448, "shared memory");
 };
 
@@ -1948,7 +1947,7 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     using VS = VSide<DK>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar_mma, bar_load, bar_cur;
+    __shared__ __align__(8) uint64_t bar_mma, bar_load;
     __shared__ uint32_t s_tmem;
     __shared__ float s_gm[DK], s_gl[DK], s_dgl[DK], s_beta[kChunk];
 
@@ -1993,7 +1992,6 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (tid == 0) {
         mbar_init(&bar_mma, 1);
         mbar_init(&bar_load, 1);
-        mbar_init(&bar_cur, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_q);
@@ -2012,8 +2010,8 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     if (tid == 0) prefetch(w);
     float bnext = beta_thread ? load_beta(w) : 0.f;
-    uint32_t mma_phase = 0, load_phase = 0, cur_phase = 0;
-    bool aborted = false, load_pending = true, mma_pending = false, cur_pending = false;
+    uint32_t mma_phase = 0, load_phase = 0;
+    bool aborted = false, load_pending = true, mma_pending = false;
     float* g = reinterpret_cast<float*>(sm + Sm::G);
 
     while (w < total) {
@@ -2077,6 +2075,8 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         {
             const __nv_bfloat16* pk = reinterpret_cast<const __nv_bfloat16*>(sm + Sm::PF_K);
             const __nv_bfloat16* pq = reinterpret_cast<const __nv_bfloat16*>(sm + Sm::PF_Q);
+            __nv_bfloat16* kq = reinterpret_cast<__nv_bfloat16*>(sm + Sm::KQ);   // k rows, then q rows
+            const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
 #pragma unroll
             for (int idx = tid; idx < DK * (kChunk / 4); idx += 256) {
                 const int ch = idx % DK, r4 = (idx / DK) * 4;
@@ -2084,8 +2084,10 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
                     const int r = r4 + t;
-                    const float kk = r < L ? __bfloat162float(pk[r * DK + ch]) : 0.f;
-                    const float qq = r < L ? __bfloat162float(pq[r * DK + ch]) : 0.f;
+                    const __nv_bfloat16 kb = r < L ? pk[r * DK + ch] : zero, qb = r < L ? pq[r * DK + ch] : zero;
+                    kq[r * DK + ch] = kb;
+                    kq[(kChunk + r) * DK + ch] = qb;
+                    const float kk = __bfloat162float(kb), qq = __bfloat162float(qb);
                     const float d = g[r * DK + ch] - s_gm[ch];
                     const float fl = __expf(d), fr = __expf(-d);
                     kr[t] = round_tf32_alu(kk * fr);
@@ -2142,16 +2144,14 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mma_pending = true;
         // this thread's element-pass operands from global memory (channel lane_row,
         // tokens [32 wg, 32 wg + 32)), in flight across the MMAs
-        __nv_bfloat16 kv[32], qv[32];
-        float dqtv[32];
+        float dqtv[32], dktv[32], dkhv[32];
         if (lane_row < DK) {
 #pragma unroll
             for (int t = 0; t < 32; ++t) {
                 const int r = 32 * wg + t;
-                const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + lane_row;
-                kv[t] = r < L ? k[off] : __float2bfloat16_rn(0.f);
-                qv[t] = r < L ? q[off] : __float2bfloat16_rn(0.f);
                 dqtv[t] = vs[VS::DQT + r * DK + lane_row];
+                dktv[t] = vs[VS::DKT + r * DK + lane_row];
+                dkhv[t] = vs[VS::DKH + r * DK + lane_row];
             }
         }
         // meanwhile: dbeta = (parts through W, U0) + rowsum(dA M); a row's 16 steps
@@ -2169,14 +2169,7 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mma_phase ^= 1;
         mma_pending = false;
         tc_fence_after();
-        // the operand buffers are free: this item's dK~, dK^ and the next item's
-        // inputs land behind the element pass
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_cur, 2 * 64 * DK * 4);
-            bulk_load(sm + Sm::CUR_DKT, vs + VS::DKT, 64 * DK * 4, &bar_cur);
-            bulk_load(sm + Sm::CUR_DKH, vs + VS::DKH, 64 * DK * 4, &bar_cur);
-        }
-        cur_pending = true;
+        // the operand buffers are free: the next item's inputs land behind the element pass
         if (nw < total) {
             if (tid == 0) prefetch(nw);
             load_pending = true;
@@ -2184,9 +2177,7 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
 
         // dq, dk and dg for channel lane_row, tokens [32 wg, 32 wg + 32)
-        bool cur_ok = true;
-        const float* s_dkt = reinterpret_cast<const float*>(sm + Sm::CUR_DKT);
-        const float* s_dkh = reinterpret_cast<const float*>(sm + Sm::CUR_DKH);
+        const __nv_bfloat16* kq = reinterpret_cast<const __nv_bfloat16*>(sm + Sm::KQ);
         if (lane_row < DK) {
             const int ch = lane_row;
             const float gm = s_gm[ch], gl = s_gl[ch];
@@ -2200,18 +2191,17 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tmem_ld16(T1 + lane_base + 64 + col, dql);
                 tmem_ld16(T2 + lane_base + col, dkr);
                 tmem_wait_ld();
-                if (half == 0 && !mbar_wait_cycles(&bar_cur, cur_phase, kWaitCycles)) cur_ok = false;
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int r = (int)col + t;
                     const float gg = g[r * DK + ch];
-                    const float kk = __bfloat162float(kv[16 * half + t]), qq = __bfloat162float(qv[16 * half + t]);
+                    const float kk = __bfloat162float(kq[r * DK + ch]), qq = __bfloat162float(kq[(kChunk + r) * DK + ch]);
                     const size_t off = (size_t)(tok0 + r) * rowk + (size_t)h * DK + ch;
                     const float d = gg - gm;
                     const float fl = __expf(d), fr = __expf(-d);
                     const float eg = egm * fl, eh = eglm * fr;   // e^{g}, e^{g_{L-1} - g}
                     const float a = dkl[t] * fl, b = dql[t] * fl, cr = dkr[t] * fr;
-                    const float dkt = s_dkt[r * DK + ch], dkh = s_dkh[r * DK + ch], dqt = dqtv[16 * half + t];
+                    const float dkt = dktv[16 * half + t], dkh = dkhv[16 * half + t], dqt = dqtv[16 * half + t];
                     if (r < L) {
                         dk[off] = __float2bfloat16_rn(a + cr + dkt * eg + dkh * eh);
                         dq[off] = __float2bfloat16_rn(b + dqt * eg);
@@ -2223,16 +2213,17 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             atomicAdd(&s_dgl[ch], dgl);
         }
-        if (__syncthreads_or(!cur_ok)) { aborted = true; break; }
-        cur_phase ^= 1;
-        cur_pending = false;
+        __syncthreads();
         // dlog_alpha_s = sum_{r >= s} dg_r (+ g_{L-1}'s own cotangent), per channel
         if (gate != kGateNone && tid < DK) {
             float run = s_dgl[tid] + vs[VS::DGAM + tid] * __expf(s_gl[tid]);
-            for (int r = L - 1; r >= 0; --r) {
-                run += g[r * DK + tid];
-                if (gate == kGateChannel) dla[(size_t)(tok0 + r) * rowk + (size_t)h * DK + tid] = run;
-                else g[r * DK + tid] = run;
+#pragma unroll 16
+            for (int r = kChunk - 1; r >= 0; --r) {
+                if (r < L) {
+                    run += g[r * DK + tid];
+                    if (gate == kGateChannel) dla[(size_t)(tok0 + r) * rowk + (size_t)h * DK + tid] = run;
+                    else g[r * DK + tid] = run;
+                }
             }
         }
         if (gate == kGateHead) {
@@ -2252,7 +2243,6 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
         if (load_pending) (void)mbar_wait_cycles(&bar_load, load_phase, kWaitCycles / 4);
-        if (cur_pending) (void)mbar_wait_cycles(&bar_cur, cur_phase, kWaitCycles / 4);
     }
     tc_fence_before();
     __syncthreads();
