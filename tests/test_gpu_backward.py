@@ -169,3 +169,30 @@ def test_chunk_bwd_c4_varlen_sampled(cuda_device):
         ref = oracle_bwd(xs, d_o[:, a:b, h:h + 1].contiguous(), dSf[s:s + 1, h:h + 1].contiguous())
         part = {n: (got[n][:, a:b, h:h + 1] if n != "dS0" else got[n][s:s + 1, h:h + 1]) for n in GRADS}
         check_all(part, ref, torch.bfloat16, f"C4 seq {s} (len {b - a}) head {h}")
+
+
+def test_chunk_bwd_mixed_strong_chunks_many_items(cuda_device):
+    """About eight (chunk, head) items per CTA, with strong-decay chunks among the ordinary ones:
+    every third chunk of head 0 and every other chunk of head 2 (B=1, T=300 chunks, H=4, bf16).
+    The per-item kernels walk their items in turn, skip the flagged chunks and fetch the next
+    unflagged one ahead; heads 0 and 2 go against the oracle whole."""
+    nch = 300
+    w = I.ChunkWorkload("bmix", B=1, T=64 * nch, H=4, dk=128, dv=64, dtype=torch.bfloat16, s0_std=0.05,
+                        seed=59)
+    x = I.chunk_inputs(w)
+    la = x["log_alpha"].clone()
+    gen = torch.Generator().manual_seed(591)
+    chunk = torch.arange(w.T) // 64
+    # per-token log-decay down to -8 on four channels: |g - g_m| far above the split limit
+    for h, strong in ((0, chunk % 3 == 1), (2, chunk % 2 == 0)):
+        la[0, strong, h, :4] = -8.0 * torch.rand(int(strong.sum()), 4, generator=gen)
+    x["log_alpha"] = la.contiguous()
+    d_o, dSf = cotangents(x, 592)
+    got = run_bwd(x, d_o, dSf)
+    for h in (0, 2):
+        xs = {k: x[k][:, :, h:h + 1].contiguous() for k in ("q", "k", "v", "log_alpha", "beta")}
+        xs["initial_state"] = x["initial_state"][:, h:h + 1].contiguous()
+        xs["cu_seqlens"] = None
+        ref = oracle_bwd(xs, d_o[:, :, h:h + 1].contiguous(), dSf[:, h:h + 1].contiguous())
+        part = {n: (got[n][:, :, h:h + 1] if n != "dS0" else got[n][:, h:h + 1]) for n in GRADS}
+        check_all(part, ref, torch.bfloat16, f"mixed head {h}")
