@@ -2033,6 +2033,7 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mm[j] = *reinterpret_cast<const float4*>(Mg + r * kChunk + i4);
             dbp[j] = vs[VS::DBP + r];
         }
+        const float dgam = tid < DK ? vs[VS::DGAM + tid] : 0.f;   // for the dlog_alpha scan
         const bool got = mbar_wait_cycles(&bar_load, load_phase, kWaitCycles);
         if (__syncthreads_or(!got)) { aborted = true; break; }
         load_phase ^= 1;
@@ -2216,7 +2217,7 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         __syncthreads();
         // dlog_alpha_s = sum_{r >= s} dg_r (+ g_{L-1}'s own cotangent), per channel
         if (gate != kGateNone && tid < DK) {
-            float run = s_dgl[tid] + vs[VS::DGAM + tid] * __expf(s_gl[tid]);
+            float run = s_dgl[tid] + dgam * __expf(s_gl[tid]);
 #pragma unroll 16
             for (int r = kChunk - 1; r >= 0; --r) {
                 if (r < L) {
