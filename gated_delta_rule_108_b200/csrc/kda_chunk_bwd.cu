@@ -33,6 +33,11 @@
 //
 // The forward quantities come from the forward kernels run again with two
 // extra outputs: T from K1 and the state entering every chunk from K2.
+//
+// These two kernels are the whole backward for fp32 inputs.  For bf16 inputs
+// the tensor-core kernels (kda_chunk_tc.cu) compute the same quantities, and
+// KB4 here reads their products and takes only the chunks that the forward
+// kernel flagged as too strongly decayed for the split factors.
 #include "kda_common.cuh"
 #include "kda_launch.h"
 #include "ptx.cuh"
