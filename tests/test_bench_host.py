@@ -1,0 +1,51 @@
+"""Host-side helpers of bench.py on CPU: the timed oracle sample and the
+DRAM-traffic lookup that only answers while the captured source is unchanged."""
+import hashlib
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from gated_delta_rule_108_b200 import inputs as I  # noqa: E402
+
+
+def test_cpu_oracle_rate_repeats_whole_passes():
+    w = I.workload("C0")
+    x = I.chunk_inputs(w)
+    rate, dt, passes, threads = bench.cpu_oracle_rate(w, x, slice(0, w.B), 128, min_seconds=0.2)
+    assert dt >= 0.2 and passes >= 1
+    assert threads >= 1
+    assert rate == pytest.approx(passes * w.B * 128 / dt)
+    # with no minimum, exactly one pass
+    _, _, one, _ = bench.cpu_oracle_rate(w, x, slice(0, w.B), 128)
+    assert one == 1
+
+
+def test_traffic_lookup_follows_the_source_hash(tmp_path, monkeypatch):
+    src = tmp_path / "kernel.cu"
+    src.write_text("__global__ void k() {}\n")
+    (tmp_path / "profiles").mkdir()
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    table = {"k": {"source": "kernel.cu", "source_sha": sha, "bytes_per_launch_full": 1234}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(table))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_for("k") == 1234
+    assert bench.traffic_for("other") is None
+    src.write_text("__global__ void k() { /* changed */ }\n")   # counters no longer describe it
+    assert bench.traffic_for("k") is None
+
+
+def test_committed_traffic_table_covers_the_reported_kernels():
+    """Each kernel whose roofline the bench line reports has a committed capture,
+    naming a source file that exists and a positive byte count."""
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        table = json.load(f)
+    for name in ("intra_chunk", "inter_chunk", "decode_step", "bwd_tc_products"):
+        ent = table[name]
+        assert os.path.exists(os.path.join(ROOT, ent["source"])), name
+        assert len(ent["source_sha"]) == 16 and ent["bytes_per_launch_full"] > 0, name
