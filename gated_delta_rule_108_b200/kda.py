@@ -114,13 +114,38 @@ def _stream_ptr(stream: Optional[torch.cuda.Stream], device) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _need(t: torch.Tensor, name: str, dtype=None):
+def _need(t: torch.Tensor, name: str, dtype=None, device=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _dims(t: torch.Tensor, name: str, n: int):
+    if t.dim() != n:
+        raise ValueError(f"{name} must have {n} dimensions, got shape {tuple(t.shape)}")
+
+
+def _shape(t: Optional[torch.Tensor], name: str, shape):
+    """The kernels take every size from q (and v, cu_seqlens): a tensor of any
+    other shape would be read or written out of bounds, so it is refused here."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _num_seqs(B: int, cu_seqlens) -> int:
+    if cu_seqlens is None:
+        return B
+    _dims(cu_seqlens, "cu_seqlens", 1)
+    if B != 1:
+        raise ValueError(f"cu_seqlens requires B == 1 (sequences packed along T), got B={B}")
+    if cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must hold N + 1 >= 1 offsets")
+    return cu_seqlens.numel() - 1
 
 
 def chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
@@ -131,18 +156,20 @@ def chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
                                                   int(bool(varlen)), code))
 
 
-def _gate_of(log_alpha, channel_ndim: int, shape_channel, shape_head) -> int:
+def _gate_of(log_alpha, channel_ndim: int, shape_channel, shape_head, device=None) -> int:
     """Gate kind from log_alpha's shape: None -> no gate (DeltaNet), one value
     per head -> Gated DeltaNet, one value per key channel -> KDA."""
     if log_alpha is None:
         return KDA_GATE_NONE
-    _need(log_alpha, "log_alpha", torch.float32)
     if tuple(log_alpha.shape) == tuple(shape_channel):
-        return KDA_GATE_CHANNEL
-    if tuple(log_alpha.shape) == tuple(shape_head):
-        return KDA_GATE_HEAD
-    raise ValueError(f"log_alpha must be {tuple(shape_channel)} (per channel), {tuple(shape_head)} "
-                     f"(per head) or None, got {tuple(log_alpha.shape)}")
+        gate = KDA_GATE_CHANNEL
+    elif tuple(log_alpha.shape) == tuple(shape_head):
+        gate = KDA_GATE_HEAD
+    else:
+        raise ValueError(f"log_alpha must be {tuple(shape_channel)} (per channel), {tuple(shape_head)} "
+                         f"(per head) or None, got {tuple(log_alpha.shape)}")
+    _need(log_alpha, "log_alpha", torch.float32, device)
+    return gate
 
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
@@ -155,19 +182,26 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
     initial_state [N, H, dk, dv] fp32 or None; cu_seqlens int32 [N+1] or None.
     Returns (o [B, T, H, dv], final_state [N, H, dk, dv] or None).
     """
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n, q.dtype)
-    _need(beta, "beta", torch.float32)
+    _dims(q, "q", 4)
+    _dims(v, "v", 4)
     B, T, H, dk = q.shape
-    gate = _gate_of(log_alpha, 4, (B, T, H, dk), (B, T, H))
     dv = v.shape[-1]
+    N = _num_seqs(B, cu_seqlens)
+    for t, n, shape in ((k, "k", (B, T, H, dk)), (v, "v", (B, T, H, dv)), (beta, "beta", (B, T, H)),
+                        (initial_state, "initial_state", (N, H, dk, dv)), (o, "o", (B, T, H, dv)),
+                        (final_state, "final_state", (N, H, dk, dv))):
+        _shape(t, n, shape)
+    dev = q.device
+    gate = _gate_of(log_alpha, 4, (B, T, H, dk), (B, T, H), dev)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, dev)
+    _need(beta, "beta", torch.float32, dev)
     if cu_seqlens is not None:
-        _need(cu_seqlens, "cu_seqlens", torch.int32)
-        N = cu_seqlens.numel() - 1
-    else:
-        N = B
-    if initial_state is not None:
-        _need(initial_state, "initial_state", torch.float32)
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    for t, n, dt in ((initial_state, "initial_state", torch.float32), (o, "o", q.dtype),
+                     (final_state, "final_state", torch.float32)):
+        if t is not None:
+            _need(t, n, dt, dev)
     if o is None:
         o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
     if final_state is None and output_final_state:
@@ -202,20 +236,25 @@ def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=N
     like log_alpha, None without a gate), dbeta (fp32) and dS0 [N, H, dk, dv]
     (fp32, or None when ``output_d_initial_state`` is false).
     """
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o")):
-        _need(t, n, q.dtype)
-    _need(beta, "beta", torch.float32)
+    _dims(q, "q", 4)
+    _dims(v, "v", 4)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    gate = _gate_of(log_alpha, 4, (B, T, H, dk), (B, T, H))
+    N = _num_seqs(B, cu_seqlens)
+    for t, n, shape in ((k, "k", (B, T, H, dk)), (v, "v", (B, T, H, dv)), (beta, "beta", (B, T, H)),
+                        (d_o, "d_o", (B, T, H, dv)), (initial_state, "initial_state", (N, H, dk, dv)),
+                        (d_final_state, "d_final_state", (N, H, dk, dv))):
+        _shape(t, n, shape)
+    dev = q.device
+    gate = _gate_of(log_alpha, 4, (B, T, H, dk), (B, T, H), dev)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o")):
+        _need(t, n, q.dtype, dev)
+    _need(beta, "beta", torch.float32, dev)
     if cu_seqlens is not None:
-        _need(cu_seqlens, "cu_seqlens", torch.int32)
-        N = cu_seqlens.numel() - 1
-    else:
-        N = B
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
     for t, n in ((initial_state, "initial_state"), (d_final_state, "d_final_state")):
         if t is not None:
-            _need(t, n, torch.float32)
+            _need(t, n, torch.float32, dev)
     g = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
          "dlog_alpha": None if log_alpha is None else torch.empty_like(log_alpha),
          "dbeta": torch.empty_like(beta),
@@ -261,13 +300,21 @@ def recurrent_step(q, k, v, log_alpha, beta, state, o=None, stream=None) -> torc
     log_alpha [B, H, dk] (KDA), [B, H] (Gated DeltaNet) or None (DeltaNet).
     Returns o [B, H, dv] in q's dtype.
     """
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n, q.dtype)
-    _need(beta, "beta", torch.float32)
-    _need(state, "state", torch.float32)
+    _dims(q, "q", 3)
+    _dims(v, "v", 3)
     B, H, dk = q.shape
     dv = v.shape[-1]
-    gate = _gate_of(log_alpha, 3, (B, H, dk), (B, H))
+    for t, n, shape in ((k, "k", (B, H, dk)), (v, "v", (B, H, dv)), (beta, "beta", (B, H)),
+                        (state, "state", (B, H, dk, dv)), (o, "o", (B, H, dv))):
+        _shape(t, n, shape)
+    dev = q.device
+    gate = _gate_of(log_alpha, 3, (B, H, dk), (B, H), dev)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(state, "state", torch.float32, dev)
+    if o is not None:
+        _need(o, "o", q.dtype, dev)
     if o is None:
         o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
     _check(lib().kda_recurrent_step_gated(
