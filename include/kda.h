@@ -201,7 +201,12 @@ size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv,
  * of the kda_chunk_fwd call with the same inputs, it writes dL/dq, dL/dk,
  * dL/dv, dL/dlog_alpha, dL/dbeta and dL/dinitial_state.  The forward
  * quantities are recomputed from the inputs (no forward output is needed).
- * All arithmetic is fp32 on CUDA cores for both dtypes.
+ * fp32 inputs: every product in fp32 on CUDA cores (max-relative error 1e-4
+ * against an fp64 reference).  bf16 inputs: the products on the tensor cores
+ * with fp16 operands (tf32 for the split-factor products) and fp32
+ * accumulation (relative L2 error 5e-3); chunks whose decay is too strong for
+ * the split factors on CUDA cores in fp32.  As in the forward, a bf16-path
+ * value beyond the fp16 range sets KDA_ERR_RANGE in the workspace status.
  *
  *  q, k, v, log_alpha, beta, initial_state, cu_seqlens, sizes, dtype:
  *              as kda_chunk_fwd (per-channel gate)
