@@ -76,9 +76,10 @@ def inv_blocked(A, rnd, bs=16):
     return T
 
 
-def bf16_path_head(q, k, v, la, beta, S0, inv=inv_exact, inv_rnd=ident, C=64):
-    """The bf16-input plan: tf32 split factors for A and P, fp16 T diag(beta),
-    W, U0, Q~, K^, state and U operands, bf16 output."""
+def bf16_path_head(q, k, v, la, beta, S0, inv=inv_exact, inv_rnd=ident, C=64, ops=tf32, mid=fp16):
+    """The bf16-input plan: ``ops`` (tf32) for the split factors of A and P,
+    ``mid`` (fp16) for T diag(beta), W, U0, P, Q~, K^, the state and U
+    operands, bf16 output.  ops = mid = bf16 is the all-bf16 plan."""
     T_, dk = q.shape
     scale = dk ** -0.5
     S = S0.copy()
@@ -88,16 +89,16 @@ def bf16_path_head(q, k, v, la, beta, S0, inv=inv_exact, inv_rnd=ident, C=64):
         L = e - s
         g = np.cumsum(la[s:e], axis=0)
         gm = g[(L - 1) // 2]
-        Kl, Kr, Ql = tf32(k[s:e] * np.exp(g - gm)), tf32(k[s:e] * np.exp(gm - g)), tf32(q[s:e] * np.exp(g - gm))
+        Kl, Kr, Ql = ops(k[s:e] * np.exp(g - gm)), ops(k[s:e] * np.exp(gm - g)), ops(q[s:e] * np.exp(g - gm))
         b = beta[s:e]
         A = np.tril(b[:, None] * (Kl @ Kr.T), -1)
-        Tb = fp16(inv(A, inv_rnd) * b[None, :])
-        W = fp16(Tb @ fp16(k[s:e] * np.exp(g)))
-        U0 = fp16(Tb @ v[s:e])
-        P = fp16(np.tril(Ql @ Kr.T, 0))
-        Qt, Kh = fp16(q[s:e] * np.exp(g)), fp16(k[s:e] * np.exp(g[-1] - g))
-        Sop = fp16(S)
-        Uop = fp16(U0 - W @ Sop)
+        Tb = mid(inv(A, inv_rnd) * b[None, :])
+        W = mid(Tb @ mid(k[s:e] * np.exp(g)))
+        U0 = mid(Tb @ v[s:e])
+        P = mid(np.tril(Ql @ Kr.T, 0))
+        Qt, Kh = mid(q[s:e] * np.exp(g)), mid(k[s:e] * np.exp(g[-1] - g))
+        Sop = mid(S)
+        Uop = mid(U0 - W @ Sop)
         out[s:e] = bf16(scale * (Qt @ Sop + P @ Uop))
         S = np.exp(g[-1])[:, None] * S + Kh.T @ Uop
     return out, S

@@ -34,6 +34,9 @@ def test_bf16_plan_costs_only_the_output_rounding():
     for args, o_ref in _heads(w, 2):
         o, _ = pm.bf16_path_head(*args)
         assert _rel_l2(o, o_ref) < 2.5e-3
+        # bf16 everywhere would sit close to the bar
+        o_b, _ = pm.bf16_path_head(*args, ops=pm.bf16, mid=pm.bf16)
+        assert _rel_l2(o_b, o_ref) > 1.7 * _rel_l2(o, o_ref)
 
 
 def test_product_form_inverse_breaks_where_the_blocked_form_holds():
