@@ -4,34 +4,43 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One JSON line on rank 0.  ``value`` is the chunkwise forward's throughput in
-tokens/s (a token spans all H heads) summed over all ranks, on the training
-shape B=4, T=4096, H=16, d_k=d_v=128, bf16 q/k/v, fp32 log_alpha/beta/state,
-with its inputs resident in HBM; each rank runs its own batch (weak scaling,
-no data-path collective: sequences and heads are independent).  Timing is on
-the device with CUDA events on the launching stream, bracketed by a barrier
-and a synchronize, max over ranks.  The line also carries:
+tokens/s (a token spans all H heads) summed over all ranks, on the largest
+single-GPU workload: 16 packed sequences of 1,024-16,384 tokens (about 147 k
+tokens), H=32, d_k=d_v=128, bf16 q/k/v, fp32 log_alpha/beta/state, with its
+inputs resident in HBM.  Each rank runs its own batch (weak scaling, no
+data-path collective: sequences and heads are independent).  Timing is on the
+device with CUDA events on the launching stream, bracketed by a barrier and a
+synchronize, max over ranks.  The line also carries:
 
 * ``roofline``      -- the dominant kernel, timed live with events that the
-                       library records between its launches (HBM-bound);
+                       library records between its launches, against the HBM
+                       bytes the method itself moves through that kernel;
 * ``path_roofline`` -- the whole forward against the algorithmic minimum
-                       traffic of the method (inputs + outputs + state);
-* ``decode``        -- one recurrent step for B=256, H=32, d=128 (state 512 MiB),
-                       tokens/s and its HBM roofline;
-* ``e2e``           -- the same forward through the public API from pinned
+                       traffic of the method (inputs + outputs + state), and
+                       FLOP-counted against the bf16 tensor-core peak;
+* ``c1``, ``c2``    -- the same figures on the training shape (B=4, T=4096,
+                       H=16) and on one 65,536-token sequence (H=32);
+* ``decode``        -- 1,024 consecutive recurrent steps for B=256, H=32, d=128
+                       (state 512 MiB), tokens/s and the HBM roofline;
+* ``chunk_bwd``     -- the backward on the training shape;
+* ``e2e``           -- the headline forward through the public API from pinned
                        host buffers, copies in and out inside the timed region;
 * ``cpu_baseline``  -- the fp64 CPU oracle on a bounded sample (rank 0, N=1);
 * ``clocks``        -- SM clocks and throttle reasons sampled during timing.
 
 ``--impl reference`` times the fp64 CPU oracle instead (the reference arm), on
-rank 0 only.
+rank 0 only.  ``--gpus N`` without a torchrun environment starts N ranks
+itself under torch.distributed.run.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -45,9 +54,12 @@ import torch  # noqa: E402
 
 METRIC = "KDA tokens/s (chunk fwd & decode) at 1 B200; % bf16 TC peak / % HBM BW"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CHUNK = 64
+
+
 # FLOPs per token and head of the chunk forward at MMA tile granularity
 # (d_k = d_v = d, chunk C = 64): 2C(3d_k + 2d_v) + 6 d_k d_v.
-def chunk_flops_per_token_head(dk, dv, C=64):
+def chunk_flops_per_token_head(dk, dv, C=CHUNK):
     return 2 * C * (3 * dk + 2 * dv) + 6 * dk * dv
 
 
@@ -56,15 +68,33 @@ def log(*a):
 
 
 # ------------------------------------------------------------------ setup --
-def dist_setup():
+def free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch_under_torchrun(gpus: int) -> int:
+    """Run this script as ``gpus`` ranks under torch.distributed.run (same
+    arguments); returns its exit code."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def dist_setup(use_cuda: bool = True):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if use_cuda:
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     return world, rank, local
 
 
@@ -92,8 +122,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def traffic_for(kernel: str):
-    """DRAM bytes per launch from a committed ncu capture, if its source still matches."""
+def traffic_per_unit(kernel: str):
+    """DRAM bytes per unit of work (a (chunk, head) item; a (sequence, head)
+    pair for decode) from a committed ncu capture, if its source still matches."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -108,7 +139,7 @@ def traffic_for(kernel: str):
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     if sha != ent.get("source_sha"):
         return None
-    return ent.get("bytes_per_launch_full")
+    return ent.get("bytes_per_unit")
 
 
 class ClockSampler:
@@ -161,58 +192,157 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+# ---------------------------------------------------- workload arithmetic --
+def seq_lengths(w):
+    return list(w.lengths) if w.lengths is not None else [w.T] * w.B
+
+
+def chunk_units(w) -> int:
+    """(chunk, head) work items of a chunk-forward workload."""
+    return sum((n + CHUNK - 1) // CHUNK for n in seq_lengths(w)) * w.H
+
+
+def method_bytes(w):
+    """Algorithmic HBM bytes of the chunk forward, by the kernel that moves them:
+    the intra-chunk kernel reads q, k, v, log_alpha, beta; the inter-chunk
+    kernel writes o and reads / writes the states.  Per token-head:
+    (2 d_k + d_v) e + 4 d_k + 4 in, d_v e out (e = element bytes)."""
+    eb = 2 if w.dtype == torch.bfloat16 else 4
+    th = w.tokens * w.H
+    reads = th * ((2 * w.dk + w.dv) * eb + 4 * w.dk + 4)
+    o = th * w.dv * eb
+    state = (2 if w.s0_std > 0 else 1) * w.num_seqs * w.H * w.dk * w.dv * 4
+    return {"intra_chunk": reads, "inter_chunk": o + state, "total": reads + o + state}
+
+
+def record_bytes_per_unit(w) -> int:
+    """Chunk intermediates the intra-chunk kernel writes and the inter-chunk
+    kernel reads, per (chunk, head): W, Q~, K^ [64 x dk], P [64 x 64], U0
+    [64 x dv] (fp16 on the bf16 tensor-core path, fp32 on the fp32 path) and
+    gamma_C [dk] fp32."""
+    rec_eb = 2 if w.dtype == torch.bfloat16 else 4
+    return rec_eb * CHUNK * (3 * w.dk + w.dv + CHUNK) + 4 * w.dk
+
+
+def describe(w) -> str:
+    dt = "bf16" if w.dtype == torch.bfloat16 else "fp32"
+    if w.lengths is not None:
+        shape = (f"{len(w.lengths)} packed sequences (cu_seqlens), lengths {min(w.lengths)}-{max(w.lengths)}, "
+                 f"{w.tokens} tokens")
+    else:
+        shape = f"B={w.B}, T={w.T}"
+    return (f"{w.name}: KDA chunk fwd, {shape}, H={w.H}, d_k={w.dk}, d_v={w.dv}, chunk 64, {dt} q/k/v, "
+            f"fp32 log_alpha/beta/state")
+
+
+def data_recipe(w) -> str:
+    s = (f"synthetic (seeded; q,k unit-norm N(0,1), v N(0,1), beta sigmoid(N({w.beta_mu:g},1)), "
+         f"log_alpha -exp(N(0,1))/{w.la_div:g}, S0 " + (f"N(0,{w.s0_std:g}^2)" if w.s0_std > 0 else "0"))
+    if w.beta_edge_frac > 0:
+        s += f"; {w.beta_edge_frac:.0%} of tokens beta=1 and a disjoint {w.beta_edge_frac:.0%} beta=0"
+    return s + ")"
+
+
+def rank_workload(w, rank: int):
+    """Each rank draws its own batch of the same shape (weak scaling)."""
+    if rank == 0:
+        return w
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank, lengths_from=None)
+
+
 # --------------------------------------------------------------- our arm --
-def bench_chunk(args, dev, world, rank):
+def bench_chunk(name, steps, warmup, dev, world, rank):
+    """Time kda_chunk_fwd on one workload; per-stage times from library events."""
     from gated_delta_rule_108_b200 import inputs as I
     from gated_delta_rule_108_b200 import kda
 
-    w = I.workload(args.workload)
-    if w.lengths is not None:
-        raise SystemExit("bench workload must be fixed-length")
-    wr = I.ChunkWorkload(**{**w.__dict__, "seed": w.seed + 1000 * rank})  # own batch per rank
-    x = I.chunk_inputs(wr)
+    w = I.workload(name)
+    x = I.chunk_inputs(rank_workload(w, rank))
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
-    o = torch.empty(B, T, H, dv, dtype=w.dtype, device=dev)
-    S = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
-    ws = torch.empty(kda.chunk_fwd_workspace_size(B, T, H, dk, dv, B, False, w.dtype),
+    varlen = g["cu_seqlens"] is not None
+    o = torch.empty(w.B, w.T, w.H, w.dv, dtype=w.dtype, device=dev)
+    S = torch.empty(w.num_seqs, w.H, w.dk, w.dv, dtype=torch.float32, device=dev)
+    ws = torch.empty(kda.chunk_fwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.num_seqs, varlen, w.dtype),
                      dtype=torch.uint8, device=dev)
 
     def step():
         kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], g["initial_state"],
-                      None, o=o, final_state=S, workspace=ws)
+                      g["cu_seqlens"], o=o, final_state=S, workspace=ws)
 
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     for evs in stage_ev:
         for e in evs:
             e.record()  # creates the event handles
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     status = kda.workspace_status(ws)
     if status != 0:
-        raise RuntimeError(f"device status {status} after warm-up")
+        raise RuntimeError(f"{name}: device status {status} after warm-up")
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     start.record()
-    for i in range(args.steps):
+    for i in range(steps):
         kda.set_stage_events(stage_ev[i])
         step()
     end.record()
     kda.set_stage_events(None)
     torch.cuda.synchronize()
     barrier(world)
-    ms_local = start.elapsed_time(end)
-    ms = max_over_ranks(ms_local, world, dev)
-    stages = {name: statistics.mean(e[a].elapsed_time(e[b]) for e in stage_ev)
-              for name, a, b in (("chunk_prep", 0, 1), ("intra_chunk", 1, 2), ("inter_chunk", 2, 3))}
-    return dict(w=w, ms=ms, stages=stages, tokens=w.tokens, launches=3 * args.steps,
-                x=x, o=o, S=S, ws=ws)
+    ms = max_over_ranks(start.elapsed_time(end), world, dev) / steps
+    if kda.workspace_status(ws) != 0:
+        raise RuntimeError(f"{name}: device status set during timing")
+    stages = {st: statistics.mean(e[a].elapsed_time(e[b]) for e in stage_ev)
+              for st, a, b in (("chunk_prep", 0, 1), ("intra_chunk", 1, 2), ("inter_chunk", 2, 3))}
+    return dict(w=w, ms=ms, stages=stages, launches=3 * steps, x=x, g=g, o=o, S=S, ws=ws)
 
 
-def chunk_bwd_tc_bytes_per_chunk_head(dk, dv, C=64):
+def chunk_summary(res, world, peaks, peak_kind):
+    """Throughput and rooflines of one timed chunk-forward workload."""
+    w, ms = res["w"], res["ms"]
+    units = chunk_units(w)
+    mb = method_bytes(w)
+    rec = record_bytes_per_unit(w) * units
+    hbm = float(peaks["hbm_gbs"])
+    kern = {k: res["stages"][k] for k in ("intra_chunk", "inter_chunk")}
+    dom = max(kern, key=kern.get)
+    dom_ms = kern[dom]
+    achieved = mb[dom] / (dom_ms / 1e3) / 1e9
+    tpu = traffic_per_unit(dom)
+    path_gbs = mb["total"] / (ms / 1e3) / 1e9
+    th = w.tokens * w.H
+    tflops = chunk_flops_per_token_head(w.dk, w.dv) * th / (ms / 1e3) / 1e12
+    # the binding roofline of the whole path: min(tensor peak, HBM bandwidth x arithmetic intensity)
+    ai = chunk_flops_per_token_head(w.dk, w.dv) * th / mb["total"]
+    bound_tflops = min(float(peaks["bf16_tflops"]), hbm * ai / 1e3)
+    return {
+        "workload": describe(w),
+        "value": w.tokens * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+        "token_heads_per_step": th, "chunk_head_items": units,
+        "kernels_ms": res["stages"],
+        "roofline": {
+            "kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": None if tpu is None else tpu * units,
+            "peak_source": f"{peak_kind} hbm_gbs",
+            "algorithmic_bytes_per_launch": mb[dom], "ms_per_launch": dom_ms,
+            "intermediate_bytes_per_launch": rec,
+            "intermediate_note": "chunk records written by intra_chunk and read by inter_chunk "
+                                 "(not method bytes; not counted in achieved)",
+        },
+        "path_roofline": {
+            "bound": "hbm", "achieved": path_gbs, "peak": hbm, "unit": "GB/s", "frac": path_gbs / hbm,
+            "algorithmic_bytes_per_step": mb["total"],
+            "tc_tflops_flop_counted": tflops,
+            "tc_frac_of_bf16_peak": tflops / float(peaks["bf16_tflops"]),
+            "binding_roofline_tflops": bound_tflops,
+            "frac_of_binding_roofline": tflops / bound_tflops,
+        },
+    }
+
+
+def chunk_bwd_tc_bytes_per_chunk_head(dk, dv, C=CHUNK):
     """Algorithmic bytes of the backward's three tensor-core product kernels per
     (chunk, head).  Value side: reads S, dS' (fp32 dk x dv), dU (fp32 C x dv), d_o
     (bf16 C x dv), the fp16 W, Q~, U0 tiles; writes dQ~, dW, dK^ (fp32 C x dk), dP
@@ -227,24 +357,24 @@ def chunk_bwd_tc_bytes_per_chunk_head(dk, dv, C=64):
     return vside + tchain + split
 
 
-def bench_backward(args, dev, world, rank):
-    """kda_chunk_bwd on the forward's workload, a seeded d_o and d_final_state."""
+def bench_backward(args, dev, world, rank, peaks, peak_kind):
+    """kda_chunk_bwd on the training shape, a seeded d_o and d_final_state."""
     from gated_delta_rule_108_b200 import inputs as I
     from gated_delta_rule_108_b200 import kda
 
-    w = I.workload(args.workload)
-    wr = I.ChunkWorkload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
-    x = I.chunk_inputs(wr)
+    w = I.workload(args.bwd_workload)
+    x = I.chunk_inputs(rank_workload(w, rank))
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     gen = torch.Generator().manual_seed(5000 + rank)
     d_o = torch.randn(w.B, w.T, w.H, w.dv, generator=gen).to(w.dtype).to(dev)
-    dSf = torch.randn(w.B, w.H, w.dk, w.dv, generator=gen).to(dev)
-    ws = torch.empty(kda.chunk_bwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.B, False, w.dtype),
+    dSf = torch.randn(w.num_seqs, w.H, w.dk, w.dv, generator=gen).to(dev)
+    varlen = g["cu_seqlens"] is not None
+    ws = torch.empty(kda.chunk_bwd_workspace_size(w.B, w.T, w.H, w.dk, w.dv, w.num_seqs, varlen, w.dtype),
                      dtype=torch.uint8, device=dev)
 
     def step():
         kda.chunk_bwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], d_o, g["initial_state"], dSf,
-                      workspace=ws)
+                      g["cu_seqlens"], workspace=ws)
 
     steps = args.bwd_steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
@@ -271,16 +401,35 @@ def bench_backward(args, dev, world, rank):
     names = ("chunk_prep", "fwd_intra_chunk", "fwd_inter_chunk", "bwd_inter_chunk", "bwd_tc_products",
              "bwd_intra_chunk")
     stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i, n in enumerate(names)}
-    return dict(w=w, ms_per_step=ms, stages=stages, launches=(7 if w.dtype == torch.bfloat16 else 5) * steps)
+    units = chunk_units(w)
+    vbytes = chunk_bwd_tc_bytes_per_chunk_head(w.dk, w.dv) * units
+    vms = stages["bwd_tc_products"]
+    vgbs = vbytes / (vms / 1e3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    tpu = traffic_per_unit("bwd_tc_products")
+    return {
+        "workload": f"{w.name}: kda_chunk_bwd (dq, dk, dv, dlog_alpha, dbeta, dS0), B={w.B}, T={w.T}, "
+                    f"H={w.H}, d_k=d_v={w.dk}, bf16 q/k/v/d_o; tensor-core products (fp16 / tf32 operands, "
+                    "fp32 accumulation), strong-decay chunks on CUDA cores in fp32",
+        "value": w.tokens * world / (ms / 1e3), "unit": "tokens/s",
+        "ms_per_step": ms, "steps": steps, "kernels_ms": stages,
+        "gpu_launches": (7 if w.dtype == torch.bfloat16 else 5) * steps,
+        "roofline": {"kernel": "bwd_vside_tc + bwd_tchain_tc + bwd_split_tc (the dominant stage)",
+                     "bound": "hbm", "achieved": vgbs, "peak": hbm, "unit": "GB/s", "frac": vgbs / hbm,
+                     "traffic": None if tpu is None else tpu * units, "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": vbytes, "ms_per_launch": vms},
+        "strong_decay_chunks_ms": stages["bwd_intra_chunk"],
+    }
 
 
-def bench_decode(args, dev, world, rank):
+def bench_decode(args, dev, world, rank, peaks, peak_kind):
+    """kda_recurrent_step, ``--decode-steps`` consecutive steps on one state."""
     from gated_delta_rule_108_b200 import inputs as I
     from gated_delta_rule_108_b200 import kda
 
     w = I.workload(args.decode_workload)
     P = 8
-    d = I.decode_inputs(I.DecodeWorkload(**{**w.__dict__, "seed": w.seed + 1000 * rank}), pool=P)
+    d = I.decode_inputs(dataclasses.replace(w, seed=w.seed + 1000 * rank), pool=P)
     g = {k: v.to(dev) for k, v in d.items()}
     st = g["state0"].clone()
     o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=dev)
@@ -288,6 +437,7 @@ def bench_decode(args, dev, world, rank):
     for i in range(args.warmup):
         j = i % P
         kda.recurrent_step(g["q"][j], g["k"][j], g["v"][j], g["log_alpha"][j], g["beta"][j], st, o=o)
+    st.copy_(g["state0"])
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -299,15 +449,30 @@ def bench_decode(args, dev, world, rank):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(start.elapsed_time(end), world, dev) / steps
-    return dict(w=w, ms_per_step=ms, launches=steps)
+    dbytes = w.B * w.H * (2 * w.dk * w.dv * 4 + (2 * w.dk + 2 * w.dv) * 2 + 4 * w.dk + 4)
+    dgbs = dbytes / (ms / 1e3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    tpu = traffic_per_unit("decode_step")
+    return {
+        "workload": f"{w.name}: kda_recurrent_step, B={w.B}, H={w.H}, d_k=d_v={w.dk}, bf16 q/k/v, "
+                    f"fp32 state in place, {steps} consecutive steps (inputs cycle through {P} seeded draws)",
+        "value": w.B * world / (ms / 1e3), "unit": "tokens/s",
+        "ms_per_step": ms, "steps": steps, "gpu_launches": steps,
+        "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": dgbs, "peak": hbm,
+                     "unit": "GB/s", "frac": dgbs / hbm, "peak_source": f"{peak_kind} hbm_gbs",
+                     "traffic": None if tpu is None else tpu * w.B * w.H,
+                     "algorithmic_bytes_per_launch": dbytes, "ms_per_launch": ms},
+    }
 
 
 def bench_e2e(args, dev, world, res):
-    """The forward through the public API from pinned host buffers."""
+    """The headline forward through the public API from pinned host buffers:
+    every step copies that step's inputs in and its outputs back."""
     from gated_delta_rule_108_b200 import kda
 
     x = res["x"]
-    names = ("q", "k", "v", "log_alpha", "beta", "initial_state")
+    names = [n for n in ("q", "k", "v", "log_alpha", "beta", "initial_state", "cu_seqlens")
+             if x[n] is not None]
     host = {n: x[n].pin_memory() for n in names}
     devb = {n: torch.empty_like(host[n], device=dev) for n in names}
     o, S, ws = res["o"], res["S"], res["ws"]
@@ -320,7 +485,7 @@ def bench_e2e(args, dev, world, res):
         for n in names:
             devb[n].copy_(host[n], non_blocking=True)
         kda.chunk_fwd(devb["q"], devb["k"], devb["v"], devb["log_alpha"], devb["beta"],
-                      devb["initial_state"], None, o=o, final_state=S, workspace=ws)
+                      devb.get("initial_state"), devb.get("cu_seqlens"), o=o, final_state=S, workspace=ws)
         o_h.copy_(o, non_blocking=True)
         S_h.copy_(S, non_blocking=True)
 
@@ -340,23 +505,31 @@ def bench_e2e(args, dev, world, res):
     return ms, h2d, d2h
 
 
-def cpu_oracle_rate(w, x, seqs, tokens, min_seconds=0.0):
-    """Time the fp64 oracle on sequences ``seqs`` x first ``tokens`` tokens x all heads, in whole
-    passes repeated until ``min_seconds`` have gone by (at least one pass).  Returns
-    (tokens/s, seconds, passes, threads used)."""
+def cpu_oracle_rate(w, x, heads, min_seconds=0.0, tokens=None):
+    """Time the fp64 oracle on every sequence of ``x`` (its first ``tokens``
+    tokens when given, fixed-length only) and the heads ``heads``, in whole
+    passes repeated until ``min_seconds`` have gone by (at least one pass).
+    Returns (tokens/s, seconds, passes, threads used); a token spans all w.H
+    heads, so the sampled token-heads are divided by w.H."""
     from oracle import oracle as orc
-    sl = {n: x[n][seqs, :tokens] for n in ("q", "k", "v", "log_alpha", "beta")}
-    S0 = None if x["initial_state"] is None else x["initial_state"][seqs]
-    n_seq = len(range(*seqs.indices(w.B)))
+    cu = x["cu_seqlens"]
+    T = x["q"].shape[1] if tokens is None else tokens
+    if cu is not None and tokens is not None:
+        raise ValueError("a token prefix is only defined for fixed-length workloads")
+    sl = {n: x[n][:, :T, heads].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")}
+    S0 = None if x["initial_state"] is None else x["initial_state"][:, heads].contiguous()
+    n_heads = sl["q"].shape[2]
+    token_heads = sl["q"].shape[0] * T * n_heads
+    n_pairs = (sl["q"].shape[0] if cu is None else len(cu) - 1) * n_heads
     passes = 0
     t0 = time.perf_counter()
     while True:
-        orc.kda_forward(sl["q"], sl["k"], sl["v"], sl["log_alpha"], sl["beta"], S0)
+        orc.kda_forward(sl["q"], sl["k"], sl["v"], sl["log_alpha"], sl["beta"], S0, cu)
         passes += 1
         dt = time.perf_counter() - t0
         if dt >= min_seconds:
             break
-    return passes * n_seq * tokens / dt, dt, passes, min(orc.num_threads(), n_seq * w.H)
+    return passes * token_heads / w.H / dt, dt, passes, min(orc.num_threads(), n_pairs)
 
 
 def run_ours(args):
@@ -372,121 +545,81 @@ def run_ours(args):
     uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", ""))
     clocks = ClockSampler(uuid)
     clocks.start()
-    res = bench_chunk(args, dev, world, rank)
-    dec = None if args.no_decode else bench_decode(args, dev, world, rank)
-    bwd = None if args.no_bwd else bench_backward(args, dev, world, rank)
+    head = bench_chunk(args.workload, args.steps, args.warmup, dev, world, rank)
+    extras = {}
+    for name in [n for n in args.extra_workloads.split(",") if n and n != args.workload]:
+        r = bench_chunk(name, args.steps, args.warmup, dev, world, rank)
+        extras[name.lower()] = chunk_summary(r, world, peaks, peak_kind)
+        del r
+        torch.cuda.empty_cache()
+    dec = None if args.no_decode else bench_decode(args, dev, world, rank, peaks, peak_kind)
+    bwd = None if args.no_bwd else bench_backward(args, dev, world, rank, peaks, peak_kind)
     clk = clocks.stop()
-    e2e = None if args.no_e2e else bench_e2e(args, dev, world, res)
+    e2e = None if args.no_e2e else bench_e2e(args, dev, world, head)
 
-    w = res["w"]
-    ms_step = res["ms"] / args.steps
-    tokens_per_s = res["tokens"] * world / (ms_step / 1e3)
-    th = w.tokens * w.H  # token-heads per rank per step
-    eb = 2 if w.dtype == torch.bfloat16 else 4
-    # algorithmic bytes (per token-head unless noted)
-    in_bytes = 2 * w.dk * eb + w.dv * eb + 4 * w.dk + 4          # q, k, v, log_alpha, beta
-    out_bytes = w.dv * eb                                          # o
-    state_bytes = 2 * w.num_seqs * w.H * w.dk * w.dv * 4           # S0 read + final write
-    n_chunks = w.num_seqs * ((w.T + 63) // 64) * w.H
-    # chunk intermediates written by the intra-chunk kernel and read by the
-    # inter-chunk kernel, per chunk and head: W, Q~, K^ [64 x dk], P [64 x 64],
-    # U0 [64 x dv] (fp16 on the bf16 tensor-core path, fp32 on the fp32 path)
-    # and gC [dk] fp32
-    rec_eb = 2 if w.dtype == torch.bfloat16 else 4
-    rec_bytes = rec_eb * 64 * (3 * w.dk + w.dv + 64) + 4 * w.dk
-    kernels = {
-        "intra_chunk": (th * in_bytes + n_chunks * rec_bytes, res["stages"]["intra_chunk"]),
-        "inter_chunk": (n_chunks * rec_bytes + th * out_bytes + state_bytes, res["stages"]["inter_chunk"]),
-    }
-    dom = max(kernels, key=lambda k: kernels[k][1])
-    dom_bytes, dom_ms = kernels[dom]
-    hbm = float(peaks["hbm_gbs"])
-    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-    path_bytes = th * (in_bytes + out_bytes) + state_bytes
-    path_gbs = path_bytes / (ms_step / 1e3) / 1e9
-    flops = chunk_flops_per_token_head(w.dk, w.dv) * th
-    tflops = flops / (ms_step / 1e3) / 1e12
+    w = head["w"]
+    summ = chunk_summary(head, world, peaks, peak_kind)
     line = {
         "metric": METRIC,
-        "value": tokens_per_s,
+        "value": summ["value"],
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms_step,
+        "ms_per_step": summ["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
-        "data": "synthetic (seeded; q,k unit-norm N(0,1), v N(0,1), beta sigmoid(N(0,1)), "
-                "log_alpha -exp(N(0,1))/16, S0 N(0,0.01^2))",
+        "data": data_recipe(w),
         "config": {
-            "workload": f"{w.name}: KDA chunk fwd, B={w.B}, T={w.T}, H={w.H}, d_k=d_v={w.dk}, chunk 64, "
-                        "bf16 q/k/v, fp32 log_alpha/beta/state",
-            "global_batch": w.B * world, "seq_len": w.T, "heads": w.H,
+            "workload": describe(w),
+            "global_batch": w.num_seqs * world,
+            "seq_len": (f"{min(seq_lengths(w))}-{max(seq_lengths(w))} (packed, {w.tokens} tokens per rank)"
+                        if w.lengths is not None else w.T),
+            "heads": w.H,
             "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
-            "l2": f"inputs larger than L2 ({th * in_bytes / 1e6:.0f} MB read per step)",
+            "l2": f"inputs larger than L2 ({method_bytes(w)['intra_chunk'] / 1e6:.0f} MB read per step)",
         },
-        "roofline": {
-            "kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-            "frac": achieved / hbm, "traffic": traffic_for(dom), "peak_source": f"{peak_kind} hbm_gbs",
-            "algorithmic_bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms,
-        },
-        "path_roofline": {
-            "bound": "hbm", "achieved": path_gbs, "peak": hbm, "unit": "GB/s", "frac": path_gbs / hbm,
-            "algorithmic_bytes_per_step": path_bytes,
-            "tc_tflops_flop_counted": tflops,
-            "tc_frac_of_bf16_peak": tflops / float(peaks["bf16_tflops"]),
-        },
-        "kernels_ms": res["stages"],
-        "gpu_launches": res["launches"],
+        "roofline": summ["roofline"],
+        "path_roofline": summ["path_roofline"],
+        "kernels_ms": summ["kernels_ms"],
+        "chunk_head_items": summ["chunk_head_items"],
+        "gpu_launches": head["launches"],
     }
+    line.update(extras)
     if dec is not None:
-        dw = dec["w"]
-        dbytes = dw.B * dw.H * (2 * dw.dk * dw.dv * 4 + (2 * dw.dk + 2 * dw.dv) * 2 + 4 * dw.dk + 4)
-        dgbs = dbytes / (dec["ms_per_step"] / 1e3) / 1e9
-        line["decode"] = {
-            "workload": f"{dw.name}: kda_recurrent_step, B={dw.B}, H={dw.H}, d_k=d_v={dw.dk}, "
-                        "bf16 q/k/v, fp32 state in place",
-            "value": dw.B * world / (dec["ms_per_step"] / 1e3), "unit": "tokens/s",
-            "ms_per_step": dec["ms_per_step"], "steps": args.decode_steps,
-            "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": dgbs, "peak": hbm,
-                         "unit": "GB/s", "frac": dgbs / hbm, "traffic": traffic_for("decode_step"),
-                         "algorithmic_bytes_per_launch": dbytes},
-        }
+        line["decode"] = dec
     if bwd is not None:
-        bw = bwd["w"]
-        n_ch = bw.num_seqs * ((bw.T + 63) // 64) * bw.H
-        vbytes = chunk_bwd_tc_bytes_per_chunk_head(bw.dk, bw.dv) * n_ch
-        vms = bwd["stages"]["bwd_tc_products"]
-        vgbs = vbytes / (vms / 1e3) / 1e9
-        line["chunk_bwd"] = {
-            "workload": f"{bw.name}: kda_chunk_bwd (dq, dk, dv, dlog_alpha, dbeta, dS0), B={bw.B}, T={bw.T}, "
-                        f"H={bw.H}, d_k=d_v={bw.dk}, bf16 q/k/v/d_o; tensor-core products (fp16 / tf32 operands, "
-                        "fp32 accumulation), strong-decay chunks on CUDA cores in fp32",
-            "value": bw.tokens * world / (bwd["ms_per_step"] / 1e3), "unit": "tokens/s",
-            "ms_per_step": bwd["ms_per_step"], "steps": args.bwd_steps, "kernels_ms": bwd["stages"],
-            "gpu_launches": bwd["launches"],
-            "roofline": {"kernel": "bwd_vside_tc + bwd_tchain_tc + bwd_split_tc (the dominant stage)",
-                         "bound": "hbm", "achieved": vgbs, "peak": hbm, "unit": "GB/s", "frac": vgbs / hbm,
-                         "traffic": traffic_for("bwd_tc_products"), "peak_source": f"{peak_kind} hbm_gbs",
-                         "algorithmic_bytes_per_launch": vbytes, "ms_per_launch": vms},
-            "strong_decay_chunks_ms": bwd["stages"]["bwd_intra_chunk"],
-        }
+        line["chunk_bwd"] = bwd
     if e2e is not None:
         ms_e, h2d, d2h = e2e
-        line["e2e"] = {"value": res["tokens"] * world / (ms_e / 1e3), "unit": "tokens/s",
+        line["e2e"] = {"value": w.tokens * world / (ms_e / 1e3), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e}
     if clk is not None:
         line["clocks"] = clk
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, dt, passes, cores = cpu_oracle_rate(w, res["x"], slice(0, w.B), w.T, min_seconds=10.0)
+        heads = slice(0, min(w.H, args.cpu_heads))
+        rate, dt, passes, cores = cpu_oracle_rate(w, head["x"], heads, min_seconds=10.0)
+        n_h = len(range(*heads.indices(w.H)))
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": f"the whole workload ({w.B} sequences x {w.H} heads x {w.T} tokens), "
-                                          f"{passes} passes in {dt:.1f} s, fp64 C oracle, OpenMP over "
-                                          "(sequence, head)"}
+                                "sample": f"every sequence of {w.name} ({w.tokens} tokens), heads 0-{n_h - 1} "
+                                          f"of {w.H} ({passes} passes in {dt:.1f} s), fp64 C oracle, OpenMP "
+                                          f"over (sequence, head); tokens/s = token-heads/s / {w.H}"}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_check_launch(args):
+    """The rank set-up alone, on CPU (gloo): rank 0 prints the world size that
+    the line's n_gpus would report."""
+    world, rank, _ = dist_setup(use_cuda=False)
+    t = max_over_ranks(float(rank), world, torch.device("cpu"))
+    if rank == 0:
+        print(json.dumps({"n_gpus": world, "gpus_arg": args.gpus, "max_rank": t}), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -503,13 +636,21 @@ def run_reference(args):
     orc.build_oracle()
     w = I.workload(args.workload)
     x = I.chunk_inputs(w)
-    tokens = args.reference_tokens
+    # each step: sequence 0, all heads, its first --reference-tokens tokens
+    n0 = seq_lengths(w)[0]
+    tokens = min(args.reference_tokens, n0)
+    a = 0 if x["cu_seqlens"] is None else int(x["cu_seqlens"][0])
+    xs = {n: x[n][0:1, a:a + tokens].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")}
+    xs["initial_state"] = None if x["initial_state"] is None else x["initial_state"][0:1]
+    xs["cu_seqlens"] = None
+    del x
+    heads = slice(0, w.H)
     for _ in range(args.warmup):
-        cpu_oracle_rate(w, x, slice(0, 1), tokens)
+        cpu_oracle_rate(w, xs, heads)
     times = []
     cores = 1
     for _ in range(args.steps):
-        _, dt, _, cores = cpu_oracle_rate(w, x, slice(0, 1), tokens)
+        _, dt, _, cores = cpu_oracle_rate(w, xs, heads)
         times.append(dt)
     ms = 1e3 * statistics.mean(times)
     value = tokens / (ms / 1e3)
@@ -518,12 +659,11 @@ def run_reference(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (same seeded inputs as the CUDA arm)",
-        "config": {"workload": f"{w.name}: KDA chunk fwd, B={w.B}, T={w.T}, H={w.H}, d_k=d_v={w.dk}; "
-                               f"each step = sequence 0, all heads, first {tokens} tokens",
-                   "global_batch": w.B, "seq_len": w.T, "heads": w.H},
+        "data": data_recipe(w),
+        "config": {"workload": describe(w) + f"; each step = sequence 0, all heads, first {tokens} tokens",
+                   "global_batch": w.num_seqs, "heads": w.H},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"sequence 0 of {w.B}, {w.H} heads, {tokens} tokens per step"},
+                         "sample": f"sequence 0 of {w.num_seqs}, {w.H} heads, {tokens} tokens per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -536,16 +676,31 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="C1")
+    ap.add_argument("--workload", default="C4", help="headline chunk-forward workload (C0..C4 minus C3)")
+    ap.add_argument("--extra-workloads", default="C1,C2", help="more chunk-forward workloads, comma-separated")
     ap.add_argument("--decode-workload", default="C3")
-    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--bwd-workload", default="C1")
     ap.add_argument("--reference-tokens", type=int, default=1024)
+    ap.add_argument("--cpu-heads", type=int, default=4, help="heads in the CPU-oracle sample")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward (kda_chunk_bwd) measurement")
     ap.add_argument("--bwd-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--check-launch", action="store_true",
+                    help="set up the ranks only (CPU, gloo) and print the world size")
     args = ap.parse_args()
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        raise SystemExit(relaunch_under_torchrun(args.gpus))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch one rank per GPU")
+    if args.check_launch:
+        run_check_launch(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         log("note: fewer than 3 warm-up steps")
     if args.impl == "reference":

@@ -195,7 +195,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                       const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_la,
                       const float* __restrict__ log_alpha_head, const float* __restrict__ beta,
                       ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
-                      size_t max_chunks, long long wait_cap, int drop_first_la,
+                      size_t max_chunks, long long wait_cap, int drop_la,
                       unsigned char* __restrict__ bwd_tiles, int* __restrict__ bwd_flags)
 {
     using Sm = K1Smem<DK, DV>;
@@ -286,16 +286,24 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         }
     };
 
+    // test hook: CTA 0 can leave out the log-decay copy of its third item (of
+    // its last one if it has fewer), so that the bounded wait on it gives up
+    // with the item's tile copies already waited for and the drain after the
+    // abort starting past phase 0
+    const int drop_it = (drop_la && blockIdx.x == 0) ? min(2, (total - 1) / (int)gridDim.x) : -1;
     if (tid == 0) {
         issue_tma(blockIdx.x, 0);
-        // test hook: CTA 0 can leave out its first log-decay copy, so that the
-        // bounded wait on it gives up (nothing else is in flight at that wait)
-        if (!(drop_first_la && blockIdx.x == 0)) issue_la(blockIdx.x);
+        if (drop_it != 0) issue_la(blockIdx.x);
     }
     load_beta(blockIdx.x);
     bool aborted = false;
     uint32_t mma_phase = 0;
     int mma_pending = 0;      // commits issued on bar_mma not yet waited for
+    // This CTA's items are numbered by iteration j; item j's tiles land on
+    // bar_load[j & 1] (phase parity (j >> 1) & 1) and its log-decay tile on
+    // bar_la (parity j & 1).  Items loads_done .. loads_issued - 1 have copies
+    // issued but not yet waited for (drained on abort).
+    int loads_issued = 1, loads_done = 0;
     bool stored = false;      // the copy thread has bulk stores in flight
     bool tstored = false;     // kTileThread has bulk stores in flight (backward mode)
     float range_max = 0.f;
@@ -321,6 +329,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
         const bool ok_la = !channel_gate || mbar_wait_cycles(&bar_la, it & 1, wait_cap);
         const bool ok_load = mbar_wait_cycles(&bar_load[stage], (it >> 1) & 1, wait_cap);
         if (__syncthreads_or(!(ok_la && ok_load))) { aborted = true; break; }
+        loads_done = it + 1;
         {
             float la_cur[TPP];
             float acc = 0.f;
@@ -466,7 +475,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             if (wn < total) {
                 // log_alpha into G (free now); k, v, q tiles into the other
                 // stage once the bulk stores of the item that used it have read it
-                issue_la(wn);
+                if (it + 1 != drop_it) issue_la(wn);
                 if (stored) bulk_store_wait_read();
                 issue_tma(wn, stage ^ 1);
             }
@@ -477,6 +486,7 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             bulk_store_commit();
             stored = true;
         }
+        if (wn < total) loads_issued = it + 2;   // the copy thread's prefetch above
         mma_pending = strong ? 0 : 1;
         // v: bf16 -> fp16 in place, 8 values per thread and step (warps 2..7)
         for (int item = tid - 64; tid >= 64 && item < kChunk * (DV / 8); item += 192) {
@@ -713,9 +723,12 @@ intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
 
     if (aborted) {
         if (tid == 0) flag_error(hdr, kStatusTimeout);
-        // let this CTA's own copies and MMAs finish (bounded) before freeing
-        for (int s2 = 0; s2 < 2; ++s2) (void)mbar_wait_cycles(&bar_load[s2], 0, wait_cap / 4);
-        if constexpr (channel_gate) (void)mbar_wait_cycles(&bar_la, 0, wait_cap / 4);
+        // let this CTA's own copies and MMAs finish (bounded) before freeing:
+        // exactly the phases that were issued and not yet waited for
+        for (int j = loads_done; j < loads_issued; ++j) {
+            (void)mbar_wait_cycles(&bar_load[j & 1], (j >> 1) & 1, wait_cap / 4);
+            if constexpr (channel_gate) (void)mbar_wait_cycles(&bar_la, j & 1, wait_cap / 4);
+        }
         if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
     }
     if (stored || tstored) bulk_store_wait_all();
@@ -858,12 +871,17 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
 
     bool aborted = false;
     uint32_t mma_phase = 0;
+    int mma_pending = 0;   // a commit on bar_mma not yet waited for
+    // chunk j's records land on bar_full[j & 1] (phase parity (j >> 1) & 1);
+    // chunks copies_done .. copies_issued - 1 are in flight (drained on abort)
+    int copies_issued = nch < 2 ? nch : 2, copies_done = 0;
     int n = 0;
     for (; n < nch; ++n) {
         const int b = n & 1;
         unsigned char* st = sm + b * Sm::STAGE;
         bool ok = mbar_wait_cycles(&bar_full[b], (n >> 1) & 1, kWaitCycles);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        copies_done = n + 1;
 
         const uint32_t R3 = r3(n);
         // MMA3: [W; Q~] S -> R3
@@ -897,9 +915,11 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
             tmem_st32_sync(SACC + lane_base + 32 * wg, v);
         }
         if (n > 0 && lane_row >= 64) write_o(n - 1);
+        mma_pending = 1;
         ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        mma_phase ^= 1;
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        mma_phase ^= 1;
+        mma_pending = 0;
         tc_fence_after();
 
         // U = U0 - W S  (rows 0..63 = tokens), fp16 -> U16
@@ -944,14 +964,17 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
                         smem_desc(ub + ks * 2048, 8192, 1024, kLayoutSW128), idesc_t, true);
             mma_commit(&bar_mma);
         }
+        mma_pending = 1;
         ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        mma_phase ^= 1;
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        mma_phase ^= 1;
+        mma_pending = 0;
         tc_fence_after();
         if (tid == 0) {
             fence_proxy_async_smem();
             issue(n + 2);   // this stage is no longer read
         }
+        if (n + 2 < nch) copies_issued = n + 3;
         // next state's fp16 operand copy (the serial path); the output rows of
         // this chunk are written during the next chunk's MMA3
         if (lane_row < DK) {
@@ -968,8 +991,9 @@ inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict
     if (aborted) {
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         // let MMAs and copies this CTA issued finish before its memory goes away
-        (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        for (int b = 0; b < 2; ++b) (void)mbar_wait_cycles(&bar_full[b], 0, kWaitCycles / 8);
+        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        for (int j = copies_done; j < copies_issued; ++j)
+            (void)mbar_wait_cycles(&bar_full[j & 1], (j >> 1) & 1, kWaitCycles / 8);
     } else {
         if (nch > 0 && lane_row >= 64) write_o(nch - 1);
         if (final_state && lane_row < DK) {
@@ -1103,6 +1127,10 @@ bwd_inter_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const float* __re
     bool aborted = false;
     uint32_t mma_phase = 0;
     int mma_pending = 0;
+    // the m-th chunk processed (n = nch - 1 - m) lands on bar_full[n & 1] with
+    // phase parity (m >> 1) & 1; processed indices copies_done .. copies_issued - 1
+    // are in flight (drained on abort)
+    int copies_issued = nch < 2 ? nch : 2, copies_done = 0;
     for (int n = nch - 1; n >= 0; --n) {
         const int b = n & 1, m = nch - 1 - n;   // m-th chunk processed; stage b's (m >> 1)-th use
         unsigned char* st = sm + b * Sm::STAGE;
@@ -1110,6 +1138,7 @@ bwd_inter_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const float* __re
         const int tok0 = tok_begin + n * kChunk;
         bool ok = mbar_wait_cycles(&bar_full[b], (m >> 1) & 1, kWaitCycles);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
+        copies_done = m + 1;
 
         // D = c dO: bf16 -> fp16 in place; rows past the sequence are zero
         for (int it = tid; it < kChunk * 8; it += 256) {
@@ -1167,9 +1196,9 @@ bwd_inter_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const float* __re
         }
         mma_pending = 1;
         ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
         mma_phase ^= 1;
         mma_pending = 0;
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
         tc_fence_after();
 
         // dU (rows 0..63): fp32 out; -dU as the fp16 operand of MMA-b
@@ -1214,14 +1243,15 @@ bwd_inter_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const float* __re
         }
         mma_pending = 1;
         ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
         mma_phase ^= 1;
         mma_pending = 0;
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
         tc_fence_after();
         if (tid == 0) {
             fence_proxy_async_smem();
             issue(n - 2);   // this stage is no longer read
         }
+        if (n - 2 >= 0) copies_issued = m + 3;
         // the fp16 copy of dS for the previous chunk
         if (lane_row < DK) {
             float v[32];
@@ -1238,7 +1268,8 @@ bwd_inter_tc_kernel(const __grid_constant__ CUtensorMap tm_do, const float* __re
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         // let MMAs and copies this CTA issued finish before its memory goes away
         if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        for (int b = 0; b < 2; ++b) (void)mbar_wait_cycles(&bar_full[b], 0, kWaitCycles / 8);
+        for (int j = copies_done; j < copies_issued; ++j)
+            (void)mbar_wait_cycles(&bar_full[(nch - 1 - j) & 1], (j >> 1) & 1, kWaitCycles / 8);
     } else if (d_initial_state && lane_row < DK) {
         float v[32];
         tmem_ld32_sync(SACC + lane_base + 32 * wg, v);

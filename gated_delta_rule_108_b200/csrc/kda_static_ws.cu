@@ -12,12 +12,17 @@
 // library holds it until the process exits.  In host code the name
 // g_static_workspace is only a stand-in for the device array, never a device
 // address, so the address is looked up with cudaGetSymbolAddress on the first
-// call on each device (with that device current) and cached.  All calls share
+// call on each device (with that device current) and cached together with the
+// CUDA context it belongs to.  If that context has been torn down since (e.g.
+// cudaDeviceReset), the module is loaded again at another address, so a call
+// that finds a different current context repeats the look-up.  All calls share
 // the array; kda_chunk_fwd rewrites every part of it that it reads (its status
 // word and chunk table are set by its first kernel, its per-chunk records are
 // written before they are read), so stale contents from an earlier call do
 // not matter -- but calls that overlap on the GPU (different streams or
 // devices' threads racing on one device) race on it.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "../../include/kda.h"
@@ -30,20 +35,45 @@ static __device__ __align__(256) unsigned char g_static_workspace[KDA_STATIC_WOR
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_dev_ptr[kMaxDevices] = {};
+CUcontext g_dev_ctx[kMaxDevices] = {};
 
-// Device address of g_static_workspace on the current device (set up on the
-// first call per device, with that device current).
+// The driver's cuCtxGetCurrent, reached through the runtime (the library links
+// only the CUDA runtime).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+// Device address of g_static_workspace on the current device: set up on the
+// first call per device (with that device current), again if the device's
+// context has changed since.
 cudaError_t static_workspace_ptr(void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    CtxGetCurrentFn get = ctx_get_current();
+    if (!get) return cudaErrorUnknown;
+    // null until this host thread's first runtime call that binds the context
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_dev_ptr[dev]) {
+    if (!g_dev_ptr[dev] || !ctx || g_dev_ctx[dev] != ctx) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_workspace);
+        e = cudaGetSymbolAddress(&p, g_static_workspace);   // binds the device's context
         if (e != cudaSuccess) return e;
+        if (get(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
         g_dev_ptr[dev] = p;
+        g_dev_ctx[dev] = ctx;
     }
     *out = g_dev_ptr[dev];
     return cudaSuccess;

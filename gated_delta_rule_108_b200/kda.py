@@ -97,6 +97,18 @@ def _check(status: int):
         raise KDAError(status, lib().kda_last_error().decode(errors="replace"))
 
 
+def _validate_default() -> bool:
+    """``KDA_VALIDATE=1`` in the environment turns on ``check`` by default."""
+    return os.environ.get("KDA_VALIDATE", "0") not in ("", "0", "false", "False")
+
+
+def _check_device_status(workspace: torch.Tensor, stream) -> None:
+    """Synchronise on the call's stream and raise if a kernel left an error
+    (bad cu_seqlens, a bounded wait that gave up, an fp16-range overflow)."""
+    _check(lib().kda_workspace_status(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream_ptr(stream, workspace.device)))
+
+
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return KDA_F32
@@ -174,13 +186,22 @@ def _gate_of(log_alpha, channel_ndim: int, shape_channel, shape_head, device=Non
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
               output_final_state: bool = True, o=None, final_state=None,
-              workspace=None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              workspace=None, stream=None,
+              check: Optional[bool] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunkwise forward (``kda_chunk_fwd_gated``).
 
     q, k [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H];
     log_alpha [B, T, H, dk] (KDA), [B, T, H] (Gated DeltaNet) or None (DeltaNet);
     initial_state [N, H, dk, dv] fp32 or None; cu_seqlens int32 [N+1] or None.
     Returns (o [B, T, H, dv], final_state [N, H, dk, dv] or None).
+
+    Errors found by the kernels while they run (cu_seqlens rejected on the
+    device, a bounded wait that gave up, a bf16-path value beyond the fp16
+    range) are written to the workspace's status word and are NOT raised by
+    default, since reading them needs a synchronisation.  ``check=True`` (or
+    ``KDA_VALIDATE=1`` in the environment) synchronises after the call and
+    raises :class:`KDAError` for them; otherwise pass a ``workspace`` and read
+    it later with :func:`workspace_status`.
     """
     _dims(q, "q", 4)
     _dims(v, "v", 4)
@@ -214,6 +235,8 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
         _ptr(cu_seqlens), B, T, H, dk, dv, N, _dtype_code(q), gate, _ptr(o), _ptr(final_state),
         _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream_ptr(stream, q.device)))
+    if check if check is not None else _validate_default():
+        _check_device_status(workspace, stream)
     return o, final_state
 
 
@@ -227,14 +250,15 @@ def chunk_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
 
 def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=None,
               cu_seqlens=None, output_d_initial_state: bool = True, workspace=None,
-              stream=None) -> Dict[str, Optional[torch.Tensor]]:
+              stream=None, check: Optional[bool] = None) -> Dict[str, Optional[torch.Tensor]]:
     """Gradients of the chunkwise forward (``kda_chunk_bwd_gated``).
 
     Inputs as ``chunk_fwd``: log_alpha [B, T, H, dk] (KDA), [B, T, H] (Gated
     DeltaNet) or None (DeltaNet); d_o like o; d_final_state [N, H, dk, dv] fp32
     or None.  Returns a dict with dq, dk, dv (input dtype), dlog_alpha (shaped
     like log_alpha, None without a gate), dbeta (fp32) and dS0 [N, H, dk, dv]
-    (fp32, or None when ``output_d_initial_state`` is false).
+    (fp32, or None when ``output_d_initial_state`` is false).  ``check`` as in
+    :func:`chunk_fwd`.
     """
     _dims(q, "q", 4)
     _dims(v, "v", 4)
@@ -269,6 +293,8 @@ def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=N
         _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]),
         _ptr(g["dS0"]), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream_ptr(stream, q.device)))
+    if check if check is not None else _validate_default():
+        _check_device_status(workspace, stream)
     return g
 
 
@@ -279,7 +305,7 @@ def debug_drop_copy(wait_cycles: int) -> None:
 
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise and return the device status code left in ``workspace``."""
-    return int(lib().kda_workspace_status(_ptr(workspace), workspace.numel(),
+    return int(lib().kda_workspace_status(_ptr(workspace), workspace.numel() * workspace.element_size(),
                                           _stream_ptr(stream, workspace.device)))
 
 

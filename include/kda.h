@@ -175,7 +175,9 @@ kda_status kda_recurrent_step_gated(const void* q, const void* k, const void* v,
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Every call uses the same array, so calls that
+ * before any stream capture.  The address is cached with the device's CUDA
+ * context; a call that finds another context current (after cudaDeviceReset,
+ * say) looks it up again.  Every call uses the same array, so calls that
  * overlap on one GPU (e.g. on two streams) race; order them on one stream.
  * kda_workspace_status cannot read this workspace (use kda_chunk_fwd when the
  * device status is needed).
@@ -269,8 +271,9 @@ kda_status kda_set_stage_events(void* const* events, int count);
  * Test hook for the failure path (no counterpart in the pages).  Arms the next
  * kda_chunk_fwd with bf16 inputs and the per-channel gate on this host thread
  * (one call only): its intra-chunk kernel leaves out one asynchronous copy
- * (the log-decay tile of the first work item of its first CTA) and caps each
- * of its waits at `wait_cycles` SM clock cycles.  The wait on the missing copy
+ * (the log-decay tile of the third work item of its first CTA, or of that
+ * CTA's last item if it has fewer) and caps each of its waits at
+ * `wait_cycles` SM clock cycles.  The wait on the missing copy
  * gives up, the kernel records KDA_ERR_TIMEOUT in the workspace status
  * (kda_workspace_status) and returns; that call's outputs are not meaningful.
  * Nothing faults or hangs, and later calls run normally.  0 disarms.

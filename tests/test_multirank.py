@@ -1,4 +1,5 @@
 """Host-side logic of the N-rank benchmark on CPU: gloo, world size 2."""
+import json
 import os
 import subprocess
 import sys
@@ -48,7 +49,27 @@ def test_two_rank_max_and_independent_batches():
 
 def test_reference_arm_runs_on_rank0_only():
     env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
-    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
                         "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True,
                        timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    """bench.py --gpus 2 outside torchrun relaunches itself as two ranks; the
+    line's n_gpus is the world size those ranks see (CPU, gloo)."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--check-launch"],
+                       env=env, capture_output=True, text=True, timeout=180)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    out = json.loads(lines[0])
+    assert out["n_gpus"] == 2 and out["gpus_arg"] == 2 and out["max_rank"] == 1.0
+
+
+def test_gpus_flag_must_match_world_size():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "4", "--check-launch"],
+                       env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "WORLD_SIZE=2" in r.stderr
