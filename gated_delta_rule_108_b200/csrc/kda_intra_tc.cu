@@ -1,0 +1,666 @@
+// kda_intra_tc.cu -- the forward intra-chunk kernel on the sm_100a tensor cores
+// (bf16 inputs), two CTAs per SM.
+//
+// Per (chunk, head) item, with g_r = sum_{i<=r} log alpha_i per key channel
+// and g_m the middle token's (the chunk algebra of the chunk-wise parallel
+// form, kongchang.com "Kimi Delta Attention详解", section "硬件效率的优化策略",
+// obtained by unrolling the daiw.net update equation, section "KDA 的更新式"):
+//
+//   [A; P] = [K~m; Q~m] K-m^T  (tf32, A operand in TMEM, B in shared memory)
+//   T = (I + A)^{-1} in 16 x 16 blocks on CUDA cores (fp32)
+//   W = T diag(beta) K~,  U0 = T diag(beta) V  (fp16 operands)
+//   records: W, Q~ = q e^{g}, K^ = k e^{g_{L-1} - g}, P, U0 (fp16), gamma_C (fp32)
+//
+// The records have the layout the inter-chunk kernel reads (TcRec).  Compared
+// with the intra-chunk kernel of kda_chunk_tc.cu (which also serves the
+// backward's recomputation), this one keeps MMA1's 128-row A operand in tensor
+// memory instead of 64 KB of shared memory, takes the log-decay tile in a
+// 128-byte-swizzled layout that both the per-channel scan and the per-row
+// element pass read without bank conflicts, and loads v only after the element
+// pass.  That brings a CTA to about 99 KB of shared memory, 256 TMEM columns
+// and 128 registers per thread, so two CTAs share each SM and one item's
+// latency-bound phases (the (I + A)^{-1} solve, the TMEM round trips, the
+// copies) overlap the other CTA's work.
+//
+// Every wait is bounded; a CTA that gives up records KDA_ERR_TIMEOUT, drains
+// exactly the copies and MMAs it issued, frees its tensor memory and returns.
+#include <cuda_fp16.h>
+
+#include <cstring>
+#include <type_traits>
+
+#include "kda_common.cuh"
+#include "kda_launch.h"
+#include "kda_tc_common.cuh"
+#include "ptx.cuh"
+
+namespace kda {
+namespace {
+
+using namespace ptx;
+
+// Shared memory of one CTA (byte offsets; tiles of 64 rows x 128 bytes, 128-byte swizzled).
+template <int DK, int DV>
+struct K1fSmem {
+    static constexpr uint32_t TILE = 8192;
+    static constexpr uint32_t KT = 0;                                   // k (bf16) -> K~ (fp16, MMA2 B)
+    static constexpr uint32_t KT_BYTES = (DK / 64) * TILE;
+    static constexpr uint32_t QT = KT + KT_BYTES;                       // q -> Q~ (fp16) -> v -> V (fp16, MMA2 B)
+    static constexpr uint32_t QT_BYTES = ((DK > DV ? DK : DV) / 64) * TILE;
+    static constexpr uint32_t G = QT + QT_BYTES;                        // log_alpha -> g (fp32, 32-channel tiles)
+    static constexpr uint32_t G_BYTES = 64 * DK * 4;
+    static constexpr uint32_t OPB = G + G_BYTES;                        // K-m tf32 (MMA1 B); W | U0 fp16 staging
+    static constexpr uint32_t OPB_BYTES = (DK / 32) * TILE;
+    static constexpr uint32_t STG_BYTES = ((DK + DV) / 64) * TILE;
+    // after the element pass: T diag(beta) fp16 as MMA2's 128-row A operand
+    // (rows 64..127 are never used), the E blocks and T (fp32, 64 x 68); A
+    // (fp32, 64 x 68) outside G, because the strong-decay path writes it while
+    // g is still live
+    static constexpr uint32_t TP = G;
+    static constexpr uint32_t EM = TP + 16384;
+    static constexpr uint32_t TM = EM + 6 * 16 * 17 * 4;
+    static constexpr uint32_t AM = (TM + 64 * 68 * 4) > OPB ? (TM + 64 * 68 * 4) : OPB;
+    static constexpr uint32_t E0 = OPB + (OPB_BYTES > STG_BYTES ? OPB_BYTES : STG_BYTES);
+    static constexpr uint32_t E1 = AM + 64 * 68 * 4;
+    static constexpr uint32_t END = E0 > E1 ? E0 : E1;
+    static constexpr uint32_t BAR = END;                                 // bar_in, bar_v, bar_mma
+    static constexpr uint32_t TMEMADDR = BAR + 24;
+    static constexpr uint32_t BETA = BAR + 32;                           // [64]
+    static constexpr uint32_t GM = BETA + 256;                           // [DK] g_m (base 2)
+    static constexpr uint32_t EGM = GM + DK * 4;                         // [DK] e^{g_m}
+    static constexpr uint32_t EGLM = EGM + DK * 4;                       // [DK] e^{g_{L-1} - g_m}
+    static constexpr uint32_t LAH = EGLM + DK * 4;                       // [64] per-head log-decay
+    static constexpr uint32_t PART = LAH + 256;                          // [256 / DK][DK] scan partials
+    static constexpr uint32_t TOTAL = PART + 256 * 4;
+    static constexpr uint32_t KQ_TX = 2 * (DK / 64) * TILE;              // k and q tiles
+    static constexpr uint32_t LA_TX = 64 * DK * 4;
+    static constexpr uint32_t V_TX = (DV / 64) * TILE;
+    static_assert(TP % 1024 == 0 && OPB % 1024 == 0 && G % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+    static_assert(EM + 6 * 16 * 17 * 4 <= TM && TM % 16 == 0 && AM % 16 == 0, "T-solve scratch");
+    static_assert(TP + 16384 <= OPB + OPB_BYTES, "T diag(beta) operand inside the free region");
+    // two CTAs per SM: 228 KB per SM, 1 KB reserved per CTA
+    static_assert(2 * (TOTAL + 1024) <= 233472, "two CTAs per SM");
+};
+
+// g (base 2) of token r, channel c in the 128-byte-swizzled log-decay tiles
+// (32 channels x 64 tokens each).
+__device__ __forceinline__ uint32_t g_off(int r, int c) {
+    return (uint32_t)(c >> 5) * 8192u + sw128_offset((uint32_t)r, (uint32_t)(c & 31) * 4u);
+}
+
+template <int DK, int DV, int GATE>
+__global__ void __launch_bounds__(256, 2)
+intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_la,
+                          const float* __restrict__ log_alpha_head, const float* __restrict__ beta,
+                          ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
+                          size_t max_chunks, long long wait_cap, int drop_la)
+{
+    using Sm = K1fSmem<DK, DV>;
+    using R = TcRec<DK, DV>;
+    constexpr int NPART = 256 / DK;       // threads per key channel in the scan
+    constexpr int TPP = kChunk / NPART;   // tokens per such thread
+    constexpr int CH = DK / 2;            // channels per thread in the element pass
+    constexpr bool channel_gate = GATE == kGateChannel;
+    extern __shared__ __align__(1024) unsigned char sm[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Sm::BAR);
+    uint64_t& bar_in = bars[0];    // k, q (and log_alpha) of an item
+    uint64_t& bar_v = bars[1];     // v of an item
+    uint64_t& bar_mma = bars[2];
+    uint32_t& s_tmem = *reinterpret_cast<uint32_t*>(sm + Sm::TMEMADDR);
+    float* s_beta = reinterpret_cast<float*>(sm + Sm::BETA);
+    float* s_gm = reinterpret_cast<float*>(sm + Sm::GM);
+    float* s_egm = reinterpret_cast<float*>(sm + Sm::EGM);
+    float* s_eglm = reinterpret_cast<float*>(sm + Sm::EGLM);
+    float* s_lah = reinterpret_cast<float*>(sm + Sm::LAH);
+    float* s_part = reinterpret_cast<float*>(sm + Sm::PART);
+
+    if (hdr->status != kStatusOk) return;
+    const int total = hdr->num_chunks * H;
+    if ((int)blockIdx.x >= total) return;
+    if ((smem_u32(sm) & 1023u) != 0) {   // the swizzled layouts need 1024-byte alignment
+        if (threadIdx.x == 0) flag_error(hdr, kStatusInternal);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ch = tid % DK, part = tid / DK, r0 = part * TPP;   // scan mapping
+    const int row = 32 * (warp & 3) + lane;                      // TMEM lane: 0..63 K rows, 64..127 Q rows
+    const int hc = warp >> 2;                                    // channel half of the element pass
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+
+    if (tid == 0) {
+        mbar_init(&bar_in, 1);
+        mbar_init(&bar_v, 1);
+        mbar_init(&bar_mma, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const uint32_t AOP = tmem;        // [K~m; Q~m] tf32, 128 lanes x DK columns
+    const uint32_t D1 = tmem + DK;    // [A; P], 128 lanes x 64 columns
+    const uint32_t D2 = tmem;         // [W | U0], lanes 0..63 x (DK + DV) columns (after D1 is read)
+
+    auto locate = [&](int w, int& c, int& h, int& tok0, int& L) {
+        c = w / H;
+        h = w - c * H;
+        int seq;
+        map.locate(c, seq, tok0, L);
+    };
+    // test hook: CTA 0 can leave out the log-decay copy of its third item (of
+    // its last if it has fewer), so that the bounded wait on that item's
+    // inputs gives up with earlier phases consumed
+    const int drop_it = (drop_la && blockIdx.x == 0) ? min(2, (total - 1) / (int)gridDim.x) : -1;
+    auto issue_in = [&](int w, int j) {   // k, q (and log_alpha) of item w, this CTA's j-th
+        int c, h, tok0, L;
+        locate(w, c, h, tok0, L);
+        mbar_arrive_expect_tx(&bar_in, Sm::KQ_TX + (channel_gate ? Sm::LA_TX : 0u));
+#pragma unroll
+        for (int b = 0; b < DK / 64; ++b) {
+            tma_load_3d(sm + Sm::KT + b * Sm::TILE, &tm_k, &bar_in, b * 64, h, tok0);
+            tma_load_3d(sm + Sm::QT + b * Sm::TILE, &tm_q, &bar_in, b * 64, h, tok0);
+        }
+        if constexpr (channel_gate) {
+            if (j != drop_it) {
+#pragma unroll
+                for (int b = 0; b < DK / 32; ++b) tma_load_3d(sm + Sm::G + b * Sm::TILE, &tm_la, &bar_in, b * 32, h, tok0);
+            }
+        }
+    };
+    // beta (and a per-head log-decay) of item w into registers, threads 192..255
+    float beta_next = 0.f, lah_next = 0.f;
+    auto load_beta = [&](int w) {
+        if (tid >= 192) {
+            int c, h, tok0, L;
+            locate(w, c, h, tok0, L);
+            const int r = tid - 192;
+            beta_next = (r < L) ? ld_prefetch_f32(beta + (size_t)(tok0 + r) * H + h) : 0.f;
+            lah_next = (GATE == kGateHead && r < L) ? ld_prefetch_f32(log_alpha_head + (size_t)(tok0 + r) * H + h) : 0.f;
+        }
+    };
+
+    if (tid == kCopyThread) issue_in(blockIdx.x, 0);
+    load_beta(blockIdx.x);
+
+    bool aborted = false;
+    uint32_t mma_phase = 0;
+    int mma_pending = 0;          // a commit on bar_mma not yet waited for
+    // this CTA's j-th item lands on bar_in / bar_v with phase parity j & 1;
+    // items [in_done, in_issued) and [v_done, v_issued) are in flight
+    int in_issued = 1, in_done = 0, v_issued = 0, v_done = 0;
+    bool stored = false;          // the copy thread has bulk stores in flight
+    float range_max = 0.f;
+
+    int it = 0;
+    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x, ++it) {
+        int c, h, tok0, L;
+        locate(w, c, h, tok0, L);
+        unsigned char* rec = records + ((size_t)h * max_chunks + c) * R::BYTES;
+        if (tid >= 192) {
+            s_beta[tid - 192] = beta_next;
+            if constexpr (GATE == kGateHead) s_lah[tid - 192] = lah_next;
+        }
+        const int wn = w + gridDim.x;   // this CTA's next item
+        if (wn < total) load_beta(wn);
+        // the previous item's W / U0 staging (OPB) must be read before it is reused
+        if (tid == kCopyThread && stored) bulk_store_wait_read();
+
+        // ---- cumulative log-decay, in place over the log_alpha tile in G -------
+        const bool ok_in = mbar_wait_cycles(&bar_in, it & 1, wait_cap);
+        if (__syncthreads_or(!ok_in)) { aborted = true; break; }
+        in_done = it + 1;
+        {
+            float la_cur[TPP];
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < TPP; ++i) {
+                if constexpr (channel_gate) la_cur[i] = (r0 + i < L) ? *reinterpret_cast<const float*>(sm + Sm::G + g_off(r0 + i, ch)) : 0.f;
+                else if constexpr (GATE == kGateHead) la_cur[i] = (r0 + i < L) ? s_lah[r0 + i] : 0.f;
+                else la_cur[i] = 0.f;   // no gate: alpha = 1
+                acc += la_cur[i];
+            }
+            s_part[part * DK + ch] = acc;
+            __syncthreads();
+            acc = 0.f;
+            for (int p = 0; p < part; ++p) acc += s_part[p * DK + ch];
+#pragma unroll
+            for (int i = 0; i < TPP; ++i) {
+                acc += la_cur[i];
+                *reinterpret_cast<float*>(sm + Sm::G + g_off(r0 + i, ch)) = acc * kLog2e;   // base 2
+            }
+        }
+        __syncthreads();
+        auto gat = [&](int r, int cc) { return *reinterpret_cast<const float*>(sm + Sm::G + g_off(r, cc)); };
+        bool wide = false;   // this channel's decay within the chunk too strong for the split factors
+        if (tid < DK) {
+            const float gm = gat((L - 1) >> 1, tid), gl = gat(L - 1, tid);   // base 2
+            s_gm[tid] = gm;
+            s_egm[tid] = ex2_approx(gm);
+            s_eglm[tid] = ex2_approx(gl - gm);
+            reinterpret_cast<float*>(rec + R::GC)[tid] = exp2f(gl);
+            wide = fmaxf(gat(0, tid) - gm, gm - gl) > kMaxSplitExponent2;
+        }
+        // Strong decay: the factors e^{+-(g - g_m)} of A and P could overflow, so
+        // this chunk forms A and P exactly (slow path, no MMA1).
+        const bool strong = __syncthreads_or(wide);
+        float* am = reinterpret_cast<float*>(sm + Sm::AM);   // [64][68]
+        if (strong) {
+            exact_a_p<DK>(gat, sm + Sm::KT, sm + Sm::QT, s_beta, L, am, rec + R::P);
+            __syncthreads();   // the k, q tiles are converted in place next
+        }
+
+        // ---- element pass, phase 1: thread -> TMEM lane `row`, channels
+        //      [CH hc, CH hc + CH).  K rows (0..63, token r): K~m -> TMEM, K-m -> OPB
+        //      (tf32).  Q rows (64..127, token r): Q~m -> TMEM, Q~ = q e^{g} -> QT
+        //      (fp16, in place), K^ -> record (fp16).  Q rows read k too, so the
+        //      k tile is only overwritten (by K~) in phase 2, after the barrier.
+        const bool is_k = row < 64;
+        const int er = row & 63;
+        const bool live = er < L;
+        auto element_pass = [&](auto strong_tag) {
+            constexpr bool STRONG = decltype(strong_tag)::value;
+            if (STRONG && is_k) return;   // nothing but K~ (phase 2) for K rows
+#pragma unroll 2
+            for (int j = 0; j < CH / 8; ++j) {
+                const int c8 = CH * hc + 8 * j;
+                const uint32_t ho = (uint32_t)(c8 >> 6) * Sm::TILE + sw128_offset(er, (c8 & 63) * 2);
+                uint4 kraw = *reinterpret_cast<const uint4*>(sm + Sm::KT + ho);
+                uint4 qraw = is_k ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(sm + Sm::QT + ho);
+                if (!live) { kraw = make_uint4(0, 0, 0, 0); qraw = kraw; }
+                const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(&kraw);
+                const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(&qraw);
+                const float4 g0 = *reinterpret_cast<const float4*>(sm + Sm::G + g_off(er, c8));
+                const float4 g1 = *reinterpret_cast<const float4*>(sm + Sm::G + g_off(er, c8 + 4));
+                const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                uint32_t top[8];                      // tf32 bits of K~m / Q~m (TMEM)
+                __align__(16) float kbm[8];           // K-m (OPB)
+                __align__(16) __half2 h0[4], h1[4];   // Q~ (smem), K^ (record)
+                if constexpr (!STRONG) {
+                    const float4 m0 = *reinterpret_cast<const float4*>(s_gm + c8);
+                    const float4 m1 = *reinterpret_cast<const float4*>(s_gm + c8 + 4);
+                    const float gmv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                    if (is_k) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float kk = __bfloat162float(kb[e]);
+                            const float d = gv[e] - gmv[e];
+                            top[e] = __float_as_uint(round_tf32_alu(kk * ex2_approx(d)));   // k e^{g_r - g_m}
+                            kbm[e] = round_tf32_alu(kk * ex2_approx(-d));                   // k e^{g_m - g_r}
+                        }
+                        const uint32_t fo = (uint32_t)(c8 >> 5) * Sm::TILE, fb = (c8 & 31) * 4;
+                        *reinterpret_cast<float4*>(sm + Sm::OPB + fo + sw128_offset(er, fb)) = *reinterpret_cast<const float4*>(kbm);
+                        *reinterpret_cast<float4*>(sm + Sm::OPB + fo + sw128_offset(er, fb + 16)) = *reinterpret_cast<const float4*>(kbm + 4);
+                    } else {
+                        const float4 x0 = *reinterpret_cast<const float4*>(s_egm + c8);
+                        const float4 x1 = *reinterpret_cast<const float4*>(s_egm + c8 + 4);
+                        const float4 y0 = *reinterpret_cast<const float4*>(s_eglm + c8);
+                        const float4 y1 = *reinterpret_cast<const float4*>(s_eglm + c8 + 4);
+                        const float egmv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                        const float eglmv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            float t[2], u2[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int e = 2 * e2 + u;
+                                const float kk = __bfloat162float(kb[e]), qq = __bfloat162float(qb[e]);
+                                const float d = gv[e] - gmv[e];
+                                const float qem = qq * ex2_approx(d);           // q e^{g_r - g_m}
+                                top[e] = __float_as_uint(round_tf32_alu(qem));
+                                t[u] = qem * egmv[e];                           // q e^{g_r}
+                                u2[u] = kk * ex2_approx(-d) * eglmv[e];         // k e^{g_{L-1} - g_r}
+                            }
+                            h0[e2] = __floats2half2_rn(t[0], t[1]);
+                            h1[e2] = __floats2half2_rn(u2[0], u2[1]);
+                        }
+                        *reinterpret_cast<uint4*>(sm + Sm::QT + ho) = *reinterpret_cast<const uint4*>(h0);
+                        *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(h1);
+                    }
+                    tmem_st8(AOP + lane_base + c8, top);
+                } else {   // Q rows of a strong-decay chunk: unsplit factors, every exponent <= 0
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        float t[2], u2[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int e = 2 * e2 + u;
+                            t[u] = __bfloat162float(qb[e]) * ex2_approx(gv[e]);
+                            u2[u] = __bfloat162float(kb[e]) * ex2_approx(gat(L - 1, c8 + e) - gv[e]);
+                        }
+                        h0[e2] = __floats2half2_rn(t[0], t[1]);
+                        h1[e2] = __floats2half2_rn(u2[0], u2[1]);
+                    }
+                    *reinterpret_cast<uint4*>(sm + Sm::QT + ho) = *reinterpret_cast<const uint4*>(h0);
+                    *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(h1);
+                }
+            }
+        };
+        if (strong) element_pass(std::true_type{});
+        else element_pass(std::false_type{});
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && !strong) {
+            // ---- MMA1 (tf32, A from TMEM): [K~m; Q~m] K-m^T -> D1
+            tc_fence_after();
+            constexpr uint32_t idesc = instr_desc(kFmtTF32, 128, 64);
+            const uint32_t b0 = smem_u32(sm + Sm::OPB);
+#pragma unroll
+            for (int kb = 0; kb < DK / 32; ++kb)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_tf32_ts(D1, AOP + kb * 32 + ks * 8, smem_desc(b0 + kb * 8192 + ks * 32, 16, 1024, kLayoutSW128),
+                                idesc, (kb | ks) != 0);
+            mma_commit(&bar_mma);
+        }
+        mma_pending = strong ? 0 : 1;
+        // ---- element pass, phase 2 (K rows, while MMA1 runs): K~ = k e^{g} -> KT
+        //      (fp16, in place; MMA2's B operand), every exponent <= 0
+        if (is_k) {
+#pragma unroll 2
+            for (int j = 0; j < CH / 8; ++j) {
+                const int c8 = CH * hc + 8 * j;
+                const uint32_t ho = (uint32_t)(c8 >> 6) * Sm::TILE + sw128_offset(er, (c8 & 63) * 2);
+                uint4 kraw = *reinterpret_cast<const uint4*>(sm + Sm::KT + ho);
+                if (!live) kraw = make_uint4(0, 0, 0, 0);
+                const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(&kraw);
+                const float4 g0 = *reinterpret_cast<const float4*>(sm + Sm::G + g_off(er, c8));
+                const float4 g1 = *reinterpret_cast<const float4*>(sm + Sm::G + g_off(er, c8 + 4));
+                const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                __align__(16) __half2 h0[4];
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2)
+                    h0[e2] = __floats2half2_rn(__bfloat162float(kb[2 * e2]) * ex2_approx(gv[2 * e2]),
+                                               __bfloat162float(kb[2 * e2 + 1]) * ex2_approx(gv[2 * e2 + 1]));
+                *reinterpret_cast<uint4*>(sm + Sm::KT + ho) = *reinterpret_cast<const uint4*>(h0);
+            }
+            fence_proxy_async_smem();   // MMA2 reads K~ after later barriers
+        }
+        if (tid == kCopyThread) {
+            // Q~ tiles are the lower halves (rows 64..127) of the record's WQ
+            // tiles; once they are read, v comes into the same buffer
+#pragma unroll
+            for (int b = 0; b < DK / 64; ++b)
+                bulk_store(rec + R::WQ + b * 16384 + 8192, sm + Sm::QT + b * Sm::TILE, 8192);
+            bulk_store_commit();
+            stored = true;
+            bulk_store_wait_read();
+            mbar_arrive_expect_tx(&bar_v, Sm::V_TX);
+#pragma unroll
+            for (int b = 0; b < DV / 64; ++b) tma_load_3d(sm + Sm::QT + b * Sm::TILE, &tm_v, &bar_v, b * 64, h, tok0);
+        }
+        v_issued = it + 1;
+
+        float* tmx = reinterpret_cast<float*>(sm + Sm::TM);   // [64][68]
+        float* em_ = reinterpret_cast<float*>(sm + Sm::EM);   // E blocks: 6 x 16 x 17
+        bool ok = true;
+        if (!strong) {
+            ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            mma_phase ^= 1;
+            mma_pending = 0;
+            tc_fence_after();
+            // ---- A (rows 0..63, beta-scaled, strictly lower) to smem; P (rows
+            //      64..127, lower incl. diagonal) to the record
+            float v[32];
+            tmem_ld32_sync(D1 + lane_base + 32 * hc, v);
+            if (row < 64) {
+                const float b = s_beta[row];
+#pragma unroll
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    float4 a4;
+                    const int col = 32 * hc + 4 * i4;
+                    a4.x = (col + 0 < row) ? b * v[4 * i4 + 0] : 0.f;
+                    a4.y = (col + 1 < row) ? b * v[4 * i4 + 1] : 0.f;
+                    a4.z = (col + 2 < row) ? b * v[4 * i4 + 2] : 0.f;
+                    a4.w = (col + 3 < row) ? b * v[4 * i4 + 3] : 0.f;
+                    *reinterpret_cast<float4*>(am + row * 68 + col) = a4;
+                }
+            } else {
+                const int r = row - 64;
+#pragma unroll
+                for (int i8 = 0; i8 < 4; ++i8) {
+                    __align__(16) __half hv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int col = 32 * hc + 8 * i8 + e;
+                        hv[e] = __float2half_rn(col <= r ? v[8 * i8 + e] : 0.f);
+                    }
+                    *reinterpret_cast<uint4*>(rec + R::P + sw128_offset(r, (32 * hc + 8 * i8) * 2)) =
+                        *reinterpret_cast<const uint4*>(hv);
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- T = (I + A)^{-1} in 16 x 16 blocks, written as fp16 T diag(beta)
+        //      (K-major, rows 0..63) as soon as each block is final.
+        //      D_b = (I + A_bb)^{-1};  E_im = D_i A_im (i > m);
+        //      T_{b+l,b} = -sum_{m=b}^{b+l-1} E_{b+l,m} T_{m,b}
+        auto put_t = [&](int rr, int col, float t) {
+            *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(rr, col * 2)) = __float2half_rn(t * s_beta[col]);
+        };
+        if (tid < 64) {    // diagonal blocks, one column per thread
+            const int b = tid >> 4, cc = tid & 15, base = 16 * b;
+            float x[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float* arow = am + (base + j) * 68 + base;
+                float av[16];
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(arow + 4 * k4);
+                    av[4 * k4] = t4.x; av[4 * k4 + 1] = t4.y; av[4 * k4 + 2] = t4.z; av[4 * k4 + 3] = t4.w;
+                }
+                float acc4[4] = {(j == cc) ? 1.f : 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int k = 0; k < j; ++k) acc4[k & 3] -= av[k] * x[k];
+                x[j] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+                tmx[(base + j) * 68 + base + cc] = x[j];
+                put_t(base + j, base + cc, x[j]);
+            }
+        } else {           // zeros above the diagonal blocks
+            for (int o = tid - 64; o < 6 * 256; o += 192) {
+                const int pair = o >> 8, p = (o >> 4) & 15, q = o & 15;
+                const int i = pair < 3 ? 0 : (pair < 5 ? 1 : 2);
+                const int j = pair < 3 ? pair + 1 : (pair < 5 ? pair - 1 : 3);
+                *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(16 * i + p, (16 * j + q) * 2)) = __float2half_rn(0.f);
+            }
+        }
+        __syncthreads();
+        // E_im = D_i A_im for the 6 pairs i > m (pair index: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)),
+        // 2 x 2 outputs per thread
+        for (int o = tid; o < 6 * 64; o += 256) {
+            const int pair = o >> 6, p0 = ((o >> 3) & 7) * 2, q0 = (o & 7) * 2;
+            const int i = pair == 0 ? 1 : (pair < 3 ? 2 : 3);
+            const int m = pair == 0 ? 0 : (pair == 1 ? 0 : (pair == 2 ? 1 : pair - 3));
+            const float* d0 = tmx + (16 * i + p0) * 68 + 16 * i;
+            const float* d1 = d0 + 68;
+            float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float2 a = *reinterpret_cast<const float2*>(am + (16 * i + k) * 68 + 16 * m + q0);
+                const float e0 = d0[k], e1 = d1[k];
+                c00 += e0 * a.x; c01 += e0 * a.y; c10 += e1 * a.x; c11 += e1 * a.y;
+            }
+            float* out = em_ + (pair * 16 + p0) * 17 + q0;
+            out[0] = c00; out[1] = c01; out[17] = c10; out[18] = c11;
+        }
+        __syncthreads();
+        // T_{b+l,b} = -sum_{m=b}^{b+l-1} E_{b+l,m} T_{m,b}, 2 x 2 outputs per thread
+#pragma unroll 1
+        for (int l = 1; l < 4; ++l) {
+            for (int o = tid; o < (4 - l) * 64; o += 256) {
+                const int b = o >> 6, p0 = ((o >> 3) & 7) * 2, q0 = (o & 7) * 2;
+                const int i = b + l, j = b;
+                float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
+                for (int m = j; m < i; ++m) {
+                    const int pair = i == 1 ? 0 : (i == 2 ? 1 + m : 3 + m);
+                    const float* e0p = em_ + (pair * 16 + p0) * 17;
+                    const float* e1p = e0p + 17;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const float2 t = *reinterpret_cast<const float2*>(tmx + (16 * m + k) * 68 + 16 * j + q0);
+                        const float e0 = e0p[k], e1 = e1p[k];
+                        c00 += e0 * t.x; c01 += e0 * t.y; c10 += e1 * t.x; c11 += e1 * t.y;
+                    }
+                }
+                const int rr = 16 * i + p0, cidx = 16 * j + q0;
+                tmx[rr * 68 + cidx] = -c00;
+                tmx[rr * 68 + cidx + 1] = -c01;
+                tmx[(rr + 1) * 68 + cidx] = -c10;
+                tmx[(rr + 1) * 68 + cidx + 1] = -c11;
+                put_t(rr, cidx, -c00);
+                put_t(rr, cidx + 1, -c01);
+                put_t(rr + 1, cidx, -c10);
+                put_t(rr + 1, cidx + 1, -c11);
+            }
+            __syncthreads();
+        }
+
+        // ---- v: bf16 -> fp16 in place in QT, 8 values per thread and step
+        ok = mbar_wait_cycles(&bar_v, it & 1, wait_cap);
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        v_done = it + 1;
+        for (int item = tid; item < kChunk * (DV / 8); item += 256) {
+            const int r = item / (DV / 8), j8 = (item - r * (DV / 8)) * 8;
+            const uint32_t o = Sm::QT + (j8 >> 6) * Sm::TILE + sw128_offset(r, (j8 & 63) * 2);
+            uint4 raw = *reinterpret_cast<const uint4*>(sm + o);
+            if (r >= L) raw = make_uint4(0, 0, 0, 0);
+            const __nv_bfloat162* vb = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            __align__(16) __half2 vh[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = __bfloat1622float2(vb[e]);
+                range_max = fmaxf(range_max, fmaxf(fabsf(x.x), fabsf(x.y)));
+                vh[e] = __floats2half2_rn(x.x, x.y);
+            }
+            *reinterpret_cast<uint4*>(sm + o) = *reinterpret_cast<const uint4*>(vh);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- MMA2 (fp16): [T diag(beta); *] K~ -> D2[0, DK), [T diag(beta); *] V -> D2[DK, DK + DV)
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t idw = instr_desc(kFmtF16, 128, DK, false, true);
+            constexpr uint32_t idu = instr_desc(kFmtF16, 128, DV, false, true);
+            const uint32_t a0 = smem_u32(sm + Sm::TP), bk = smem_u32(sm + Sm::KT), bv = smem_u32(sm + Sm::QT);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(D2, smem_desc(a0 + ks * 32, 16, 1024, kLayoutSW128),
+                        smem_desc(bk + ks * 2048, Sm::TILE, 1024, kLayoutSW128), idw, ks != 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(D2 + DK, smem_desc(a0 + ks * 32, 16, 1024, kLayoutSW128),
+                        smem_desc(bv + ks * 2048, Sm::TILE, 1024, kLayoutSW128), idu, ks != 0);
+            mma_commit(&bar_mma);
+        }
+        mma_pending = 1;
+        ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        mma_phase ^= 1;
+        mma_pending = 0;
+        tc_fence_after();
+        // KT, QT and G are free: the next item's inputs come in behind the write-out
+        if (tid == kCopyThread && wn < total) issue_in(wn, it + 1);
+        if (wn < total) in_issued = it + 2;
+
+        // ---- W and U0 (rows 0..63): fp16 into the OPB staging tiles (record
+        //      layout), then one bulk store per tile; warps 0, 1, 4, 5 (TMEM
+        //      lanes 0..63) take alternate 32-column chunks
+        if ((warp & 3) < 2) {
+            const int r = row;
+#pragma unroll
+            for (int cb = hc; cb < (DK + DV) / 32; cb += 2) {
+                float v[32];
+                tmem_ld32_sync(D2 + lane_base + 32 * cb, v);
+#pragma unroll
+                for (int i8 = 0; i8 < 4; ++i8) {
+                    __align__(16) __half hv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        range_max = fmaxf(range_max, fabsf(v[8 * i8 + e]));
+                        hv[e] = __float2half_rn(v[8 * i8 + e]);
+                    }
+                    const int col = 32 * cb + 8 * i8;   // W tiles then U0 tiles, 64 columns each
+                    *reinterpret_cast<uint4*>(sm + Sm::OPB + h_off(r, col, Sm::TILE)) = *reinterpret_cast<const uint4*>(hv);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();   // D2 and the staging tiles are complete
+        if (tid == kCopyThread) {
+#pragma unroll
+            for (int b = 0; b < DK / 64; ++b)   // W: rows 0..63 of each WQ tile
+                bulk_store(rec + R::WQ + b * 16384, sm + Sm::OPB + b * Sm::TILE, Sm::TILE);
+            bulk_store(rec + R::U0, sm + Sm::OPB + (DK / 64) * Sm::TILE, (DV / 64) * Sm::TILE);
+            bulk_store_commit();
+        }
+    }
+
+    if (aborted) {
+        if (tid == 0) flag_error(hdr, kStatusTimeout);
+        // let this CTA's own copies and MMAs finish (bounded) before its memory goes away
+        for (int j = in_done; j < in_issued; ++j) (void)mbar_wait_cycles(&bar_in, j & 1, wait_cap / 4);
+        for (int j = v_done; j < v_issued; ++j) (void)mbar_wait_cycles(&bar_v, j & 1, wait_cap / 4);
+        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+    }
+    if (tid == kCopyThread && stored) bulk_store_wait_all();
+    if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+template <int DK, int DV>
+cudaError_t launch_intra_fwd_tc_t(const ChunkArgs& a) {
+    if (a.max_chunks == 0) return cudaSuccess;
+    const int ntok = a.cu_seqlens ? a.T : a.B * a.T;
+    CUtensorMap mk, mv, mq, mla;
+    if (!make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        (a.gate == kGateChannel &&
+         !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, ntok, 32, CU_TENSOR_MAP_SWIZZLE_128B)))
+        return cudaErrorInvalidValue;
+    if (a.gate != kGateChannel) memset(&mla, 0, sizeof(mla));   // unused
+    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
+    auto kern = a.gate == kGateChannel ? intra_chunk_fwd_tc_kernel<DK, DV, kGateChannel>
+              : a.gate == kGateHead    ? intra_chunk_fwd_tc_kernel<DK, DV, kGateHead>
+                                       : intra_chunk_fwd_tc_kernel<DK, DV, kGateNone>;
+    const int smem = (int)K1fSmem<DK, DV>::TOTAL;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const size_t items = a.max_chunks * (size_t)a.H;   // upper bound; the kernel reads the exact count
+    const size_t ctas = 2 * (size_t)sms;               // two resident per SM
+    const unsigned grid = (unsigned)(items < ctas ? items : ctas);
+    kern<<<grid, 256, smem, a.stream>>>(mk, mv, mq, mla, a.log_alpha, a.beta, map,
+                                        static_cast<WsHeader*>(a.ws_header),
+                                        static_cast<unsigned char*>(a.records), a.H, a.max_chunks,
+                                        a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_intra_fwd_tc(const ChunkArgs& a) {
+    if (a.dk == 128 && a.dv == 128) return launch_intra_fwd_tc_t<128, 128>(a);
+    if (a.dk == 128 && a.dv == 64) return launch_intra_fwd_tc_t<128, 64>(a);
+    if (a.dk == 64 && a.dv == 128) return launch_intra_fwd_tc_t<64, 128>(a);
+    if (a.dk == 64 && a.dv == 64) return launch_intra_fwd_tc_t<64, 64>(a);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

@@ -72,6 +72,7 @@ cudaError_t launch_chunk_prep(const ChunkArgs& a);     // K0: status reset + var
 cudaError_t launch_chunk_intra(const ChunkArgs& a);    // K1: all chunks in parallel
 cudaError_t launch_chunk_inter(const ChunkArgs& a);    // K2: serial over each sequence's chunks
 cudaError_t launch_chunk_intra_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K1
+cudaError_t launch_chunk_intra_fwd_tc(const ChunkArgs& a); // its forward-only form, two CTAs per SM
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K2
 cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a);  // backward: serial over chunks, reversed
 cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a); // the same on the tensor cores (bf16 inputs)
