@@ -7,7 +7,8 @@
 // obtained by unrolling the daiw.net update equation, section "KDA 的更新式"):
 //
 //   [A; P] = [K~m; Q~m] K-m^T  (tf32, A operand in TMEM, B in shared memory)
-//   T = (I + A)^{-1} in 16 x 16 blocks on CUDA cores (fp32)
+//   T = (I + A)^{-1}: 16 x 16 diagonal blocks on CUDA cores (fp32), the rest by
+//       blocked doubling on the tensor cores (fp16 operands)
 //   W = T diag(beta) K~,  U0 = T diag(beta) V  (fp16 operands)
 //   records: W, Q~ = q e^{g}, K^ = k e^{g_{L-1} - g}, P, U0 (fp16), gamma_C (fp32)
 //
@@ -22,8 +23,12 @@
 // latency-bound phases (the (I + A)^{-1} solve, the TMEM round trips, the
 // copies) overlap the other CTA's work.
 //
-// Every wait is bounded; a CTA that gives up records KDA_ERR_TIMEOUT, drains
-// exactly the copies and MMAs it issued, frees its tensor memory and returns.
+// Each wait on an mbarrier is done by one thread (bounded); the others block at
+// the CTA barrier that follows, so a waiting CTA issues no instructions and
+// leaves the SM's issue slots to the other CTA.  The waiting thread's acquire
+// of the phase and the barrier order the copies / MMAs before every thread's
+// later accesses.  A CTA that gives up records KDA_ERR_TIMEOUT, drains exactly
+// the copies and MMAs it issued, frees its tensor memory and returns.
 #include <cuda_fp16.h>
 
 #include <cstring>
@@ -52,17 +57,26 @@ struct K1fSmem {
     static constexpr uint32_t OPB = G + G_BYTES;                        // K-m tf32 (MMA1 B); W | U0 fp16 staging
     static constexpr uint32_t OPB_BYTES = (DK / 32) * TILE;
     static constexpr uint32_t STG_BYTES = ((DK + DV) / 64) * TILE;
-    // after the element pass: T diag(beta) fp16 as MMA2's 128-row A operand
-    // (rows 64..127 are never used), the E blocks and T (fp32, 64 x 68); A
-    // (fp32, 64 x 68) outside G, because the strong-decay path writes it while
-    // g is still live
+    // after MMA1, from G on: T diag(beta) fp16 as MMA2's 128-row A operand
+    // (rows 64..127 never used); the fp16 operands of the blocked (I + A)^{-1}
+    // (A masked to its level-1 blocks and to its level-2 quadrant, the diagonal
+    // inverses D, a product X, and T restricted to its 32 x 32 diagonal blocks);
+    // A's four diagonal 16 x 16 blocks in fp32 (padded).  Each 64 x 64 fp16 tile
+    // is read as a 128-row operand whose rows 64..127 are the next 8 KB.  The
+    // strong-decay path writes the full fp32 A ([64][68]) before the element
+    // pass, while g is live, at G + 32 KB (>= OPB).
     static constexpr uint32_t TP = G;
-    static constexpr uint32_t EM = TP + 16384;
-    static constexpr uint32_t TM = EM + 6 * 16 * 17 * 4;
-    static constexpr uint32_t AM = (TM + 64 * 68 * 4) > OPB ? (TM + 64 * 68 * 4) : OPB;
+    static constexpr uint32_t AH1 = G + 16384;
+    static constexpr uint32_t AH2 = G + 24576;
+    static constexpr uint32_t DH = G + 32768;
+    static constexpr uint32_t XH = G + 40960;
+    static constexpr uint32_t T1H = G + 49152;
+    static constexpr uint32_t AMD = G + 57344;                         // 4 x (16 x 16 + 4) fp32
+    static constexpr uint32_t AMS = G + 32768;                         // strong path: [64][68] fp32
     static constexpr uint32_t E0 = OPB + (OPB_BYTES > STG_BYTES ? OPB_BYTES : STG_BYTES);
-    static constexpr uint32_t E1 = AM + 64 * 68 * 4;
-    static constexpr uint32_t END = E0 > E1 ? E0 : E1;
+    static constexpr uint32_t E1 = G + 65536;                          // T1H's rows 64..127 end here
+    static constexpr uint32_t E2 = AMS + 64 * 68 * 4;
+    static constexpr uint32_t END = E0 > E1 ? (E0 > E2 ? E0 : E2) : (E1 > E2 ? E1 : E2);
     static constexpr uint32_t BAR = END;                                 // bar_in, bar_v, bar_mma
     static constexpr uint32_t TMEMADDR = BAR + 24;
     static constexpr uint32_t BETA = BAR + 32;                           // [64]
@@ -76,8 +90,8 @@ struct K1fSmem {
     static constexpr uint32_t LA_TX = 64 * DK * 4;
     static constexpr uint32_t V_TX = (DV / 64) * TILE;
     static_assert(TP % 1024 == 0 && OPB % 1024 == 0 && G % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-    static_assert(EM + 6 * 16 * 17 * 4 <= TM && TM % 16 == 0 && AM % 16 == 0, "T-solve scratch");
-    static_assert(TP + 16384 <= OPB + OPB_BYTES, "T diag(beta) operand inside the free region");
+    static_assert(AMS >= G + G_BYTES, "the strong path's A lies outside the live log-decay tile");
+    static_assert(AMD + 4 * 260 * 4 <= T1H + 16384 && AMS + 64 * 68 * 4 <= AMD, "T-solve scratch");
     // two CTAs per SM: 228 KB per SM, 1 KB reserved per CTA
     static_assert(2 * (TOTAL + 1024) <= 233472, "two CTAs per SM");
 };
@@ -211,7 +225,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         if (tid == kCopyThread && stored) bulk_store_wait_read();
 
         // ---- cumulative log-decay, in place over the log_alpha tile in G -------
-        const bool ok_in = mbar_wait_cycles(&bar_in, it & 1, wait_cap);
+        const bool ok_in = tid != 0 || mbar_wait_cycles(&bar_in, it & 1, wait_cap);
         if (__syncthreads_or(!ok_in)) { aborted = true; break; }
         in_done = it + 1;
         {
@@ -248,59 +262,47 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         // Strong decay: the factors e^{+-(g - g_m)} of A and P could overflow, so
         // this chunk forms A and P exactly (slow path, no MMA1).
         const bool strong = __syncthreads_or(wide);
-        float* am = reinterpret_cast<float*>(sm + Sm::AM);   // [64][68]
+        float* am = reinterpret_cast<float*>(sm + Sm::AMS);   // strong path: [64][68]
         if (strong) {
             exact_a_p<DK>(gat, sm + Sm::KT, sm + Sm::QT, s_beta, L, am, rec + R::P);
             __syncthreads();   // the k, q tiles are converted in place next
         }
 
-        // ---- element pass, phase 1: thread -> TMEM lane `row`, channels
-        //      [CH hc, CH hc + CH).  K rows (0..63, token r): K~m -> TMEM, K-m -> OPB
-        //      (tf32).  Q rows (64..127, token r): Q~m -> TMEM, Q~ = q e^{g} -> QT
-        //      (fp16, in place), K^ -> record (fp16).  Q rows read k too, so the
-        //      k tile is only overwritten (by K~) in phase 2, after the barrier.
+        // ---- element pass: thread -> TMEM lane `row`, channels [CH hc, CH hc + CH).
+        //      K rows (0..63, token r) form everything that comes from k: K~m ->
+        //      TMEM and K-m -> OPB (tf32), K~ = k e^{g} -> KT in place (fp16),
+        //      K^ = k e^{g_{L-1} - g} -> record (fp16).  Q rows (64..127) form
+        //      Q~m -> TMEM (tf32) and Q~ = q e^{g} -> QT in place (fp16).  Each
+        //      thread overwrites only the tile row it read.
         const bool is_k = row < 64;
         const int er = row & 63;
         const bool live = er < L;
         auto element_pass = [&](auto strong_tag) {
             constexpr bool STRONG = decltype(strong_tag)::value;
-            if (STRONG && is_k) return;   // nothing but K~ (phase 2) for K rows
 #pragma unroll 2
             for (int j = 0; j < CH / 8; ++j) {
                 const int c8 = CH * hc + 8 * j;
                 const uint32_t ho = (uint32_t)(c8 >> 6) * Sm::TILE + sw128_offset(er, (c8 & 63) * 2);
-                uint4 kraw = *reinterpret_cast<const uint4*>(sm + Sm::KT + ho);
-                uint4 qraw = is_k ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(sm + Sm::QT + ho);
-                if (!live) { kraw = make_uint4(0, 0, 0, 0); qraw = kraw; }
-                const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(&kraw);
-                const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(&qraw);
+                unsigned char* xt = sm + (is_k ? Sm::KT : Sm::QT) + ho;   // this row's k or q chunk
+                uint4 raw = *reinterpret_cast<const uint4*>(xt);
+                if (!live) raw = make_uint4(0, 0, 0, 0);
+                const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(&raw);
                 const float4 g0 = *reinterpret_cast<const float4*>(sm + Sm::G + g_off(er, c8));
                 const float4 g1 = *reinterpret_cast<const float4*>(sm + Sm::G + g_off(er, c8 + 4));
                 const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
                 uint32_t top[8];                      // tf32 bits of K~m / Q~m (TMEM)
                 __align__(16) float kbm[8];           // K-m (OPB)
-                __align__(16) __half2 h0[4], h1[4];   // Q~ (smem), K^ (record)
+                __align__(16) __half2 h0[4], h1[4];   // K~ | Q~ (in place), K^ (record)
                 if constexpr (!STRONG) {
                     const float4 m0 = *reinterpret_cast<const float4*>(s_gm + c8);
                     const float4 m1 = *reinterpret_cast<const float4*>(s_gm + c8 + 4);
+                    const float4 x0 = *reinterpret_cast<const float4*>(s_egm + c8);
+                    const float4 x1 = *reinterpret_cast<const float4*>(s_egm + c8 + 4);
                     const float gmv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                    const float egmv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
                     if (is_k) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float kk = __bfloat162float(kb[e]);
-                            const float d = gv[e] - gmv[e];
-                            top[e] = __float_as_uint(round_tf32_alu(kk * ex2_approx(d)));   // k e^{g_r - g_m}
-                            kbm[e] = round_tf32_alu(kk * ex2_approx(-d));                   // k e^{g_m - g_r}
-                        }
-                        const uint32_t fo = (uint32_t)(c8 >> 5) * Sm::TILE, fb = (c8 & 31) * 4;
-                        *reinterpret_cast<float4*>(sm + Sm::OPB + fo + sw128_offset(er, fb)) = *reinterpret_cast<const float4*>(kbm);
-                        *reinterpret_cast<float4*>(sm + Sm::OPB + fo + sw128_offset(er, fb + 16)) = *reinterpret_cast<const float4*>(kbm + 4);
-                    } else {
-                        const float4 x0 = *reinterpret_cast<const float4*>(s_egm + c8);
-                        const float4 x1 = *reinterpret_cast<const float4*>(s_egm + c8 + 4);
                         const float4 y0 = *reinterpret_cast<const float4*>(s_eglm + c8);
                         const float4 y1 = *reinterpret_cast<const float4*>(s_eglm + c8 + 4);
-                        const float egmv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
                         const float eglmv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
                         for (int e2 = 0; e2 < 4; ++e2) {
@@ -308,35 +310,54 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
                                 const int e = 2 * e2 + u;
-                                const float kk = __bfloat162float(kb[e]), qq = __bfloat162float(qb[e]);
+                                const float kk = __bfloat162float(xb[e]);
                                 const float d = gv[e] - gmv[e];
-                                const float qem = qq * ex2_approx(d);           // q e^{g_r - g_m}
-                                top[e] = __float_as_uint(round_tf32_alu(qem));
-                                t[u] = qem * egmv[e];                           // q e^{g_r}
-                                u2[u] = kk * ex2_approx(-d) * eglmv[e];         // k e^{g_{L-1} - g_r}
+                                const float kem = kk * ex2_approx(d);           // k e^{g_r - g_m}
+                                const float keb = kk * ex2_approx(-d);          // k e^{g_m - g_r}
+                                top[e] = __float_as_uint(round_tf32_alu(kem));
+                                kbm[e] = round_tf32_alu(keb);
+                                t[u] = kem * egmv[e];                           // k e^{g_r}
+                                u2[u] = keb * eglmv[e];                         // k e^{g_{L-1} - g_r}
                             }
                             h0[e2] = __floats2half2_rn(t[0], t[1]);
                             h1[e2] = __floats2half2_rn(u2[0], u2[1]);
                         }
-                        *reinterpret_cast<uint4*>(sm + Sm::QT + ho) = *reinterpret_cast<const uint4*>(h0);
+                        const uint32_t fo = (uint32_t)(c8 >> 5) * Sm::TILE, fb = (c8 & 31) * 4;
+                        *reinterpret_cast<float4*>(sm + Sm::OPB + fo + sw128_offset(er, fb)) = *reinterpret_cast<const float4*>(kbm);
+                        *reinterpret_cast<float4*>(sm + Sm::OPB + fo + sw128_offset(er, fb + 16)) = *reinterpret_cast<const float4*>(kbm + 4);
                         *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(h1);
+                    } else {
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            float t[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int e = 2 * e2 + u;
+                                const float qem = __bfloat162float(xb[e]) * ex2_approx(gv[e] - gmv[e]);   // q e^{g_r - g_m}
+                                top[e] = __float_as_uint(round_tf32_alu(qem));
+                                t[u] = qem * egmv[e];                                                   // q e^{g_r}
+                            }
+                            h0[e2] = __floats2half2_rn(t[0], t[1]);
+                        }
                     }
+                    *reinterpret_cast<uint4*>(xt) = *reinterpret_cast<const uint4*>(h0);
                     tmem_st8(AOP + lane_base + c8, top);
-                } else {   // Q rows of a strong-decay chunk: unsplit factors, every exponent <= 0
+                } else {   // strong-decay chunk: unsplit factors, every exponent <= 0; no MMA1 operands
 #pragma unroll
                     for (int e2 = 0; e2 < 4; ++e2) {
                         float t[2], u2[2];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const int e = 2 * e2 + u;
-                            t[u] = __bfloat162float(qb[e]) * ex2_approx(gv[e]);
-                            u2[u] = __bfloat162float(kb[e]) * ex2_approx(gat(L - 1, c8 + e) - gv[e]);
+                            const float x = __bfloat162float(xb[e]);
+                            t[u] = x * ex2_approx(gv[e]);                                          // k e^{g_r} | q e^{g_r}
+                            u2[u] = is_k ? x * ex2_approx(gat(L - 1, c8 + e) - gv[e]) : 0.f;       // k e^{g_{L-1} - g_r}
                         }
                         h0[e2] = __floats2half2_rn(t[0], t[1]);
                         h1[e2] = __floats2half2_rn(u2[0], u2[1]);
                     }
-                    *reinterpret_cast<uint4*>(sm + Sm::QT + ho) = *reinterpret_cast<const uint4*>(h0);
-                    *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(h1);
+                    *reinterpret_cast<uint4*>(xt) = *reinterpret_cast<const uint4*>(h0);
+                    if (is_k) *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(h1);
                 }
             }
         };
@@ -360,28 +381,6 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             mma_commit(&bar_mma);
         }
         mma_pending = strong ? 0 : 1;
-        // ---- element pass, phase 2 (K rows, while MMA1 runs): K~ = k e^{g} -> KT
-        //      (fp16, in place; MMA2's B operand), every exponent <= 0
-        if (is_k) {
-#pragma unroll 2
-            for (int j = 0; j < CH / 8; ++j) {
-                const int c8 = CH * hc + 8 * j;
-                const uint32_t ho = (uint32_t)(c8 >> 6) * Sm::TILE + sw128_offset(er, (c8 & 63) * 2);
-                uint4 kraw = *reinterpret_cast<const uint4*>(sm + Sm::KT + ho);
-                if (!live) kraw = make_uint4(0, 0, 0, 0);
-                const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(&kraw);
-                const float4 g0 = *reinterpret_cast<const float4*>(sm + Sm::G + g_off(er, c8));
-                const float4 g1 = *reinterpret_cast<const float4*>(sm + Sm::G + g_off(er, c8 + 4));
-                const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                __align__(16) __half2 h0[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2)
-                    h0[e2] = __floats2half2_rn(__bfloat162float(kb[2 * e2]) * ex2_approx(gv[2 * e2]),
-                                               __bfloat162float(kb[2 * e2 + 1]) * ex2_approx(gv[2 * e2 + 1]));
-                *reinterpret_cast<uint4*>(sm + Sm::KT + ho) = *reinterpret_cast<const uint4*>(h0);
-            }
-            fence_proxy_async_smem();   // MMA2 reads K~ after later barriers
-        }
         if (tid == kCopyThread) {
             // Q~ tiles are the lower halves (rows 64..127) of the record's WQ
             // tiles; once they are read, v comes into the same buffer
@@ -397,31 +396,56 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         }
         v_issued = it + 1;
 
-        float* tmx = reinterpret_cast<float*>(sm + Sm::TM);   // [64][68]
-        float* em_ = reinterpret_cast<float*>(sm + Sm::EM);   // E blocks: 6 x 16 x 17
+        float* amd = reinterpret_cast<float*>(sm + Sm::AMD);  // A's diagonal blocks, [4][16 x 16 + 4]
+        // A row `row` (< 64), columns [32 hc, 32 hc + 32), beta-scaled and strictly
+        // lower: its diagonal block -> AMD (fp32); blocks (1,0), (3,2) -> AH1 and
+        // rows 32..63 x columns 0..31 -> AH2 (fp16, zero elsewhere)
+        auto put_a_row = [&](const float (&v)[32]) {
+            const int b = row >> 4;
+            if ((b >> 1) == hc) {   // the diagonal block is columns [0, 16) or [16, 32) of v
+                float* dst = amd + b * 260 + (row & 15) * 16;
+                if ((b & 1) == 0) {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        *reinterpret_cast<float4*>(dst + 4 * k4) = make_float4(v[4 * k4], v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
+                } else {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        *reinterpret_cast<float4*>(dst + 4 * k4) =
+                            make_float4(v[16 + 4 * k4], v[16 + 4 * k4 + 1], v[16 + 4 * k4 + 2], v[16 + 4 * k4 + 3]);
+                }
+            }
+#pragma unroll
+            for (int i8 = 0; i8 < 4; ++i8) {
+                const int col = 32 * hc + 8 * i8, cb = col >> 4;
+                const bool l1 = (b == 1 && cb == 0) || (b == 3 && cb == 2);
+                const bool l2 = b >= 2 && cb < 2;
+                __align__(16) __half h1[8], h2[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    h1[e] = __float2half_rn(l1 ? v[8 * i8 + e] : 0.f);
+                    h2[e] = __float2half_rn(l2 ? v[8 * i8 + e] : 0.f);
+                }
+                *reinterpret_cast<uint4*>(sm + Sm::AH1 + sw128_offset(row, col * 2)) = *reinterpret_cast<const uint4*>(h1);
+                *reinterpret_cast<uint4*>(sm + Sm::AH2 + sw128_offset(row, col * 2)) = *reinterpret_cast<const uint4*>(h2);
+            }
+        };
         bool ok = true;
         if (!strong) {
-            ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+            ok = tid != 0 || mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
             if (__syncthreads_or(!ok)) { aborted = true; break; }
             mma_phase ^= 1;
             mma_pending = 0;
             tc_fence_after();
-            // ---- A (rows 0..63, beta-scaled, strictly lower) to smem; P (rows
-            //      64..127, lower incl. diagonal) to the record
+            // ---- A (rows 0..63) to the T-solve operands; P (rows 64..127, lower
+            //      incl. diagonal) to the record
             float v[32];
             tmem_ld32_sync(D1 + lane_base + 32 * hc, v);
             if (row < 64) {
                 const float b = s_beta[row];
 #pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    float4 a4;
-                    const int col = 32 * hc + 4 * i4;
-                    a4.x = (col + 0 < row) ? b * v[4 * i4 + 0] : 0.f;
-                    a4.y = (col + 1 < row) ? b * v[4 * i4 + 1] : 0.f;
-                    a4.z = (col + 2 < row) ? b * v[4 * i4 + 2] : 0.f;
-                    a4.w = (col + 3 < row) ? b * v[4 * i4 + 3] : 0.f;
-                    *reinterpret_cast<float4*>(am + row * 68 + col) = a4;
-                }
+                for (int i = 0; i < 32; ++i) v[i] = (32 * hc + i < row) ? b * v[i] : 0.f;
+                put_a_row(v);
             } else {
                 const int r = row - 64;
 #pragma unroll
@@ -436,13 +460,20 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                         *reinterpret_cast<const uint4*>(hv);
                 }
             }
+        } else if (row < 64) {   // strong decay: the exact A, already beta-scaled and masked
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = am[row * 68 + 32 * hc + i];
+            put_a_row(v);
         }
         __syncthreads();
 
-        // ---- T = (I + A)^{-1} in 16 x 16 blocks, written as fp16 T diag(beta)
-        //      (K-major, rows 0..63) as soon as each block is final.
-        //      D_b = (I + A_bb)^{-1};  E_im = D_i A_im (i > m);
-        //      T_{b+l,b} = -sum_{m=b}^{b+l-1} E_{b+l,m} T_{m,b}
+        // ---- T = (I + A)^{-1}: exact inverses D_b = (I + A_bb)^{-1} of the four
+        //      diagonal 16 x 16 blocks on CUDA cores, then the off-diagonal blocks on
+        //      the tensor cores by doubling the solved block (fp16 operands, fp32
+        //      accumulation):  T21 = -T22 A21 T11,  first for 16 -> 32 rows (the
+        //      pairs (1,0), (3,2)), then 32 -> 64.  T diag(beta) goes to TP in fp16
+        //      (K-major, rows 0..63) block by block.
         auto put_t = [&](int rr, int col, float t) {
             *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(rr, col * 2)) = __float2half_rn(t * s_beta[col]);
         };
@@ -451,7 +482,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             float x[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const float* arow = am + (base + j) * 68 + base;
+                const float* arow = amd + b * 260 + j * 16;
                 float av[16];
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
@@ -462,70 +493,98 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 #pragma unroll
                 for (int k = 0; k < j; ++k) acc4[k & 3] -= av[k] * x[k];
                 x[j] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                tmx[(base + j) * 68 + base + cc] = x[j];
+                *reinterpret_cast<__half*>(sm + Sm::DH + sw128_offset(base + j, (base + cc) * 2)) = __float2half_rn(x[j]);
                 put_t(base + j, base + cc, x[j]);
             }
-        } else {           // zeros above the diagonal blocks
-            for (int o = tid - 64; o < 6 * 256; o += 192) {
-                const int pair = o >> 8, p = (o >> 4) & 15, q = o & 15;
-                const int i = pair < 3 ? 0 : (pair < 5 ? 1 : 2);
-                const int j = pair < 3 ? pair + 1 : (pair < 5 ? pair - 1 : 3);
-                *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(16 * i + p, (16 * j + q) * 2)) = __float2half_rn(0.f);
+        } else {           // zero chunks: D off its diagonal blocks, T diag(beta) above them
+            for (int o = tid - 64; o < 64 * 8; o += 192) {
+                const int rr = o >> 3, c16 = o & 7, blk = c16 >> 1, rb = rr >> 4;
+                if (blk != rb) *reinterpret_cast<uint4*>(sm + Sm::DH + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
+                if (blk > rb) *reinterpret_cast<uint4*>(sm + Sm::TP + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
-        __syncthreads();
-        // E_im = D_i A_im for the 6 pairs i > m (pair index: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)),
-        // 2 x 2 outputs per thread
-        for (int o = tid; o < 6 * 64; o += 256) {
-            const int pair = o >> 6, p0 = ((o >> 3) & 7) * 2, q0 = (o & 7) * 2;
-            const int i = pair == 0 ? 1 : (pair < 3 ? 2 : 3);
-            const int m = pair == 0 ? 0 : (pair == 1 ? 0 : (pair == 2 ? 1 : pair - 3));
-            const float* d0 = tmx + (16 * i + p0) * 68 + 16 * i;
-            const float* d1 = d0 + 68;
-            float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float2 a = *reinterpret_cast<const float2*>(am + (16 * i + k) * 68 + 16 * m + q0);
-                const float e0 = d0[k], e1 = d1[k];
-                c00 += e0 * a.x; c01 += e0 * a.y; c10 += e1 * a.x; c11 += e1 * a.y;
-            }
-            float* out = em_ + (pair * 16 + p0) * 17 + q0;
-            out[0] = c00; out[1] = c01; out[17] = c10; out[18] = c11;
-        }
-        __syncthreads();
-        // T_{b+l,b} = -sum_{m=b}^{b+l-1} E_{b+l,m} T_{m,b}, 2 x 2 outputs per thread
-#pragma unroll 1
-        for (int l = 1; l < 4; ++l) {
-            for (int o = tid; o < (4 - l) * 64; o += 256) {
-                const int b = o >> 6, p0 = ((o >> 3) & 7) * 2, q0 = (o & 7) * 2;
-                const int i = b + l, j = b;
-                float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
-                for (int m = j; m < i; ++m) {
-                    const int pair = i == 1 ? 0 : (i == 2 ? 1 + m : 3 + m);
-                    const float* e0p = em_ + (pair * 16 + p0) * 17;
-                    const float* e1p = e0p + 17;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float2 t = *reinterpret_cast<const float2*>(tmx + (16 * m + k) * 68 + 16 * j + q0);
-                        const float e0 = e0p[k], e1 = e1p[k];
-                        c00 += e0 * t.x; c01 += e0 * t.y; c10 += e1 * t.x; c11 += e1 * t.y;
-                    }
-                }
-                const int rr = 16 * i + p0, cidx = 16 * j + q0;
-                tmx[rr * 68 + cidx] = -c00;
-                tmx[rr * 68 + cidx + 1] = -c01;
-                tmx[(rr + 1) * 68 + cidx] = -c10;
-                tmx[(rr + 1) * 68 + cidx + 1] = -c11;
-                put_t(rr, cidx, -c00);
-                put_t(rr, cidx + 1, -c01);
-                put_t(rr + 1, cidx, -c10);
-                put_t(rr + 1, cidx + 1, -c11);
-            }
+        // one 64 x 64 x 64 product D[0, 64) = A(128-row K-major operand) B(64 x 64, rows = K)
+        auto level_mma = [&](uint32_t a_off, uint32_t b_off) -> bool {
+            fence_proxy_async_smem();
+            tc_fence_before();
             __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                constexpr uint32_t idl = instr_desc(kFmtF16, 128, 64, false, true);
+                const uint32_t a0 = smem_u32(sm + a_off), b0 = smem_u32(sm + b_off);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tmem, smem_desc(a0 + ks * 32, 16, 1024, kLayoutSW128),
+                            smem_desc(b0 + ks * 2048, Sm::TILE, 1024, kLayoutSW128), idl, ks != 0);
+                mma_commit(&bar_mma);
+            }
+            mma_pending = 1;
+            const bool good = tid != 0 || mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+            if (__syncthreads_or(!good)) return false;
+            mma_phase ^= 1;
+            mma_pending = 0;
+            tc_fence_after();
+            return true;
+        };
+        // rows 0..63 of the product (warps 0, 1, 4, 5), as fp16 into a 64 x 64 tile
+        auto store_x = [&](uint32_t dst) {
+            if (row < 64) {
+                float v[32];
+                tmem_ld32_sync(tmem + lane_base + 32 * hc, v);
+#pragma unroll
+                for (int i8 = 0; i8 < 4; ++i8) {
+                    __align__(16) __half hv[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) hv[e] = __float2half_rn(v[8 * i8 + e]);
+                    *reinterpret_cast<uint4*>(sm + dst + sw128_offset(row, (32 * hc + 8 * i8) * 2)) = *reinterpret_cast<const uint4*>(hv);
+                }
+            }
+        };
+        // level 1: X = A_L1 D, Y = D X; T_10 = -Y_10, T_32 = -Y_32; T1 = D + those blocks
+        if (!level_mma(Sm::AH1, Sm::DH)) { aborted = true; break; }
+        store_x(Sm::XH);
+        if (!level_mma(Sm::DH, Sm::XH)) { aborted = true; break; }
+        if (row < 64) {
+            const int b = row >> 4;
+            float v[32];
+            tmem_ld32_sync(tmem + lane_base + 32 * hc, v);
+#pragma unroll
+            for (int i8 = 0; i8 < 4; ++i8) {
+                const int col = 32 * hc + 8 * i8, cb = col >> 4;
+                const bool l1 = (b == 1 && cb == 0) || (b == 3 && cb == 2);
+                const uint32_t off = sw128_offset(row, col * 2);
+                uint4 d = *reinterpret_cast<const uint4*>(sm + Sm::DH + off);
+                if (l1) {
+                    __align__(16) __half t1[8], tb[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        t1[e] = __float2half_rn(-v[8 * i8 + e]);
+                        tb[e] = __float2half_rn(-v[8 * i8 + e] * s_beta[col + e]);
+                    }
+                    d = *reinterpret_cast<const uint4*>(t1);
+                    *reinterpret_cast<uint4*>(sm + Sm::TP + off) = *reinterpret_cast<const uint4*>(tb);
+                }
+                *reinterpret_cast<uint4*>(sm + Sm::T1H + off) = d;
+            }
+        }
+        // level 2: X = A_L2 T1, Y = T1 X; T[32:64, 0:32] = -Y[32:64, 0:32]
+        if (!level_mma(Sm::AH2, Sm::T1H)) { aborted = true; break; }
+        store_x(Sm::XH);
+        if (!level_mma(Sm::T1H, Sm::XH)) { aborted = true; break; }
+        if (row >= 32 && row < 64 && hc == 0) {
+            float v[32];
+            tmem_ld32_sync(tmem + lane_base, v);
+#pragma unroll
+            for (int i8 = 0; i8 < 4; ++i8) {
+                __align__(16) __half tb[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) tb[e] = __float2half_rn(-v[8 * i8 + e] * s_beta[8 * i8 + e]);
+                *reinterpret_cast<uint4*>(sm + Sm::TP + sw128_offset(row, 16 * i8)) = *reinterpret_cast<const uint4*>(tb);
+            }
         }
 
         // ---- v: bf16 -> fp16 in place in QT, 8 values per thread and step
-        ok = mbar_wait_cycles(&bar_v, it & 1, wait_cap);
+        ok = tid != 0 || mbar_wait_cycles(&bar_v, it & 1, wait_cap);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         v_done = it + 1;
         for (int item = tid; item < kChunk * (DV / 8); item += 256) {
@@ -564,7 +623,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             mma_commit(&bar_mma);
         }
         mma_pending = 1;
-        ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+        ok = tid != 0 || mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
         mma_phase ^= 1;
         mma_pending = 0;
@@ -610,9 +669,11 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     if (aborted) {
         if (tid == 0) flag_error(hdr, kStatusTimeout);
         // let this CTA's own copies and MMAs finish (bounded) before its memory goes away
-        for (int j = in_done; j < in_issued; ++j) (void)mbar_wait_cycles(&bar_in, j & 1, wait_cap / 4);
-        for (int j = v_done; j < v_issued; ++j) (void)mbar_wait_cycles(&bar_v, j & 1, wait_cap / 4);
-        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+        if (tid == 0) {
+            for (int j = in_done; j < in_issued; ++j) (void)mbar_wait_cycles(&bar_in, j & 1, wait_cap / 4);
+            for (int j = v_done; j < v_issued; ++j) (void)mbar_wait_cycles(&bar_v, j & 1, wait_cap / 4);
+            if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+        }
     }
     if (tid == kCopyThread && stored) bulk_store_wait_all();
     if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
