@@ -2362,6 +2362,9 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a) {
 
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a) {
     if (a.num_seqs == 0) return cudaSuccess;
+    // the forward alone takes the slice-width-adaptive kernel of kda_inter_tc.cu;
+    // the backward's recomputation (which also writes the chunk-start states) this one
+    if (!a.states) return launch_chunk_inter_fwd_tc(a);
     KDA_TC_DISPATCH(launch_inter_tc_t, a);
 }
 

@@ -183,6 +183,18 @@ def test_c3_decode_full_sampled(cuda_device):
         check(S[b:b + 1, h:h + 1], S_ref, w.dtype, f"C3 state (b {b}, h {h})")
 
 
+@pytest.mark.parametrize("dk", [64, 128])
+def test_many_chains_wide_slices(cuda_device, dk):
+    """Enough (sequence, head) chains that the inter-chunk kernel takes whole
+    128-column value slices (one CTA per chain), with ragged sequences."""
+    w = I.ChunkWorkload("wide", B=40, T=150, H=8, dk=dk, dv=128, dtype=torch.bfloat16, s0_std=0.05, seed=30)
+    x = I.chunk_inputs(w)
+    o, S = run_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    check(o, o_ref, torch.bfloat16, "o")
+    check(S, S_ref, torch.bfloat16, "final_state")
+
+
 # ----------------------------------------------------------- consistency ---
 def test_chunk_equals_decode_steps(cuda_device):
     """The chunkwise and the recurrent modes agree on one sequence set."""
