@@ -20,6 +20,8 @@ synchronize, max over ranks.  The line also carries:
                        FLOP-counted against the bf16 tensor-core peak;
 * ``c1``, ``c2``    -- the same figures on the training shape (B=4, T=4096,
                        H=16) and on one 65,536-token sequence (H=32);
+* ``c4_fused``      -- the headline workload with the fused single pass forced
+                       (kda_chunk_fwd runs the two-kernel form by itself);
 * ``decode``        -- 1,024 consecutive recurrent steps for B=256, H=32, d=128
                        (state 512 MiB), tokens/s and the HBM roofline;
 * ``chunk_bwd``     -- the backward on the training shape;
@@ -552,6 +554,23 @@ def run_ours(args):
         extras[name.lower()] = chunk_summary(r, world, peaks, peak_kind)
         del r
         torch.cuda.empty_cache()
+    # the fused single pass (one CTA per (sequence, head), no intermediates in
+    # memory), forced, beside the form kda_chunk_fwd picks by itself
+    for name in [n for n in args.fused_workloads.split(",") if n]:
+        old_path = os.environ.get("KDA_CHUNK_PATH")
+        os.environ["KDA_CHUNK_PATH"] = "fused"
+        try:
+            r = bench_chunk(name, args.steps, args.warmup, dev, world, rank)
+        finally:
+            if old_path is None:
+                os.environ.pop("KDA_CHUNK_PATH", None)
+            else:
+                os.environ["KDA_CHUNK_PATH"] = old_path
+        summ_f = chunk_summary(r, world, peaks, peak_kind)
+        summ_f["form"] = "fused single pass (forced; kernels_ms.intra_chunk is the whole pass)"
+        extras[name.lower() + "_fused"] = summ_f
+        del r
+        torch.cuda.empty_cache()
     dec = None if args.no_decode else bench_decode(args, dev, world, rank, peaks, peak_kind)
     bwd = None if args.no_bwd else bench_backward(args, dev, world, rank, peaks, peak_kind)
     clk = clocks.stop()
@@ -559,6 +578,8 @@ def run_ours(args):
 
     w = head["w"]
     summ = chunk_summary(head, world, peaks, peak_kind)
+    from gated_delta_rule_108_b200 import kda as _kda
+    plan = _kda.chunk_fwd_plan(w.B, w.T, w.H, w.dk, w.dv, w.num_seqs, w.lengths is not None, w.dtype)
     line = {
         "metric": METRIC,
         "value": summ["value"],
@@ -584,6 +605,7 @@ def run_ours(args):
         "roofline": summ["roofline"],
         "path_roofline": summ["path_roofline"],
         "kernels_ms": summ["kernels_ms"],
+        "form": "fused single pass" if plan == 1 else "two kernels (intra-chunk, inter-chunk)",
         "chunk_head_items": summ["chunk_head_items"],
         "gpu_launches": head["launches"],
     }
@@ -678,6 +700,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="C4", help="headline chunk-forward workload (C0..C4 minus C3)")
     ap.add_argument("--extra-workloads", default="C1,C2", help="more chunk-forward workloads, comma-separated")
+    ap.add_argument("--fused-workloads", default="C4",
+                    help="chunk-forward workloads also timed with the fused single pass forced")
     ap.add_argument("--decode-workload", default="C3")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--bwd-workload", default="C1")

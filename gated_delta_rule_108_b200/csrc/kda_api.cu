@@ -5,6 +5,8 @@
 // synchronises, except kda_workspace_status.
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
+#include <cstring>
 #include <string>
 
 #include "../../include/kda.h"
@@ -115,6 +117,38 @@ bool bwd_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, 
     return true;
 }
 
+// Which form of the bf16 chunk forward runs.  The two-kernel split form (all
+// chunks in parallel at two CTAs per SM, records through the workspace, then
+// the chunk-to-chunk recurrence) is the faster one on B200 at every workload
+// measured, so it runs whenever the workspace holds the records.  The fused
+// single pass (one CTA per (sequence, head) pair, each chunk's intermediates
+// kept on chip) needs only the header, the chunk table and the pair order, and
+// runs when the workspace is smaller than that.  KDA_CHUNK_PATH = "fused" /
+// "split" forces one (tests, measurements); "auto" or unset decides.
+int chunk_path_override() {
+    const char* e = getenv("KDA_CHUNK_PATH");
+    if (!e || !*e || strcmp(e, "auto") == 0) return 0;
+    if (strcmp(e, "fused") == 0) return 1;
+    if (strcmp(e, "split") == 0) return 2;
+    return 0;
+}
+
+// Workspace bytes of the fused single pass: the header, the chunk table and,
+// for packed sequences, the pair order (N ints) where the records would start.
+size_t fused_ws_bytes(int N, bool varlen, const WsLayout& L) {
+    return L.records_off + (varlen ? sizeof(int) * (size_t)N : 0);
+}
+
+// fused (1) or split (0) for a workspace of ws_bytes (SIZE_MAX: as large as needed)
+int chunk_fwd_fused(int N, bool varlen, kda_dtype dtype, const WsLayout& L, size_t ws_bytes) {
+    if (dtype != KDA_BF16) return 0;
+    const size_t fused_need = fused_ws_bytes(N, varlen, L);
+    const int ov = chunk_path_override();
+    if (ov == 1) return ws_bytes >= fused_need ? 1 : 0;
+    if (ov == 2) return 0;
+    return (ws_bytes < L.total && ws_bytes >= fused_need) ? 1 : 0;
+}
+
 }  // namespace
 
 namespace kda {
@@ -179,8 +213,10 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
     if (!workspace) return fail(KDA_ERR_WORKSPACE, "workspace is null (need %zu bytes)", L.total);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(KDA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-    if (workspace_bytes < L.total)
-        return fail(KDA_ERR_WORKSPACE, "workspace has %zu bytes, need %zu", workspace_bytes, L.total);
+    const int fused = chunk_fwd_fused(N, varlen, dtype, L, workspace_bytes);
+    if (workspace_bytes < L.total && !fused)
+        return fail(KDA_ERR_WORKSPACE, "workspace has %zu bytes, need %zu%s", workspace_bytes, L.total,
+                    dtype == KDA_BF16 ? " (or the fused pass's kda_chunk_fwd_fused_workspace_size)" : "");
 
     kda::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
@@ -205,9 +241,14 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
     cudaError_t e = mark_stage(0, a.stream);
     if (e == cudaSuccess) e = kda::launch_chunk_prep(a);
     if (e == cudaSuccess) e = mark_stage(1, a.stream);
-    if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_intra_tc(a) : kda::launch_chunk_intra(a);
-    if (e == cudaSuccess) e = mark_stage(2, a.stream);
-    if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_inter_tc(a) : kda::launch_chunk_inter(a);
+    if (fused) {   // one pass; the inter-chunk stage is empty
+        if (e == cudaSuccess) e = kda::launch_chunk_fused_tc(a);
+        if (e == cudaSuccess) e = mark_stage(2, a.stream);
+    } else {
+        if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_intra_tc(a) : kda::launch_chunk_intra(a);
+        if (e == cudaSuccess) e = mark_stage(2, a.stream);
+        if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_inter_tc(a) : kda::launch_chunk_inter(a);
+    }
     if (e == cudaSuccess) e = mark_stage(3, a.stream);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_chunk_fwd launch failed: %s", cudaGetErrorString(e));
     return ok();
@@ -406,6 +447,23 @@ kda_status kda_chunk_bwd_gated(const void* q, const void* k, const void* v, cons
     return chunk_bwd_impl(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_o, d_final_state, B, T, H, dk,
                           dv, num_seqs, dtype, gate, dq, dk_out, dv_out, dlog_alpha, dbeta, d_initial_state,
                           workspace, workspace_bytes, stream);
+}
+
+int kda_chunk_fwd_plan(int B, int T, int H, int dk, int dv, int num_seqs, int varlen, kda_dtype dtype,
+                       size_t workspace_bytes) {
+    WsLayout L;
+    if (!ws_layout(B, T, H, dk, dv, num_seqs, varlen != 0, dtype, L)) return -1;
+    const int N = varlen ? num_seqs : B;
+    const int fused = chunk_fwd_fused(N, varlen != 0, dtype, L, workspace_bytes);
+    if (workspace_bytes < L.total && !fused) return -1;
+    return fused;
+}
+
+size_t kda_chunk_fwd_fused_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int varlen,
+                                          kda_dtype dtype) {
+    WsLayout L;
+    if (dtype != KDA_BF16 || !ws_layout(B, T, H, dk, dv, num_seqs, varlen != 0, dtype, L)) return 0;
+    return fused_ws_bytes(varlen ? num_seqs : B, varlen != 0, L);
 }
 
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {

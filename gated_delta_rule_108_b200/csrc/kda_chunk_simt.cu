@@ -39,7 +39,7 @@ chunk_prep_kernel(WsHeader* hdr, int32_t* chunk_offsets, const int32_t* __restri
     __shared__ int s_carry, s_bad;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (cu == nullptr) {
-        if (tid == 0) { hdr->status = kStatusOk; hdr->num_chunks = fixed_num_chunks; hdr->runtime_err = 0; }
+        if (tid == 0) { hdr->status = kStatusOk; hdr->num_chunks = fixed_num_chunks; hdr->runtime_err = 0; hdr->next_pair = 0; }
         return;
     }
     if (tid == 0) { s_carry = 0; s_bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0; }
@@ -83,6 +83,7 @@ chunk_prep_kernel(WsHeader* hdr, int32_t* chunk_offsets, const int32_t* __restri
         hdr->status = bad ? kStatusBadSeqlens : kStatusOk;
         hdr->num_chunks = bad ? 0 : s_carry;
         hdr->runtime_err = 0;
+        hdr->next_pair = 0;
     }
 }
 

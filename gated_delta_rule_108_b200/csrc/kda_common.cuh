@@ -29,7 +29,8 @@ struct WsHeader {
     int status;       // argument check of the last call (0 = ok): kernels skip work if set
     int num_chunks;   // chunks per head in this call
     int runtime_err;  // first error a kernel hit while working (0 = none), e.g. a timeout
-    int reserved[61];
+    int next_pair;    // fused forward: next (sequence, head) pair to claim
+    int reserved[60];
 };
 static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
 

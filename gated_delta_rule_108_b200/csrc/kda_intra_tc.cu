@@ -45,7 +45,7 @@ namespace {
 using namespace ptx;
 
 // Shared memory of one CTA (byte offsets; tiles of 64 rows x 128 bytes, 128-byte swizzled).
-template <int DK, int DV>
+template <int DK, int DV, bool FUSED>
 struct K1fSmem {
     static constexpr uint32_t TILE = 8192;
     static constexpr uint32_t KT = 0;                                   // k (bf16) -> K~ (fp16, MMA2 B)
@@ -76,7 +76,21 @@ struct K1fSmem {
     static constexpr uint32_t E0 = OPB + (OPB_BYTES > STG_BYTES ? OPB_BYTES : STG_BYTES);
     static constexpr uint32_t E1 = G + 65536;                          // T1H's rows 64..127 end here
     static constexpr uint32_t E2 = AMS + 64 * 68 * 4;
-    static constexpr uint32_t END = E0 > E1 ? (E0 > E2 ? E0 : E2) : (E1 > E2 ? E1 : E2);
+    static constexpr uint32_t END0 = E0 > E1 ? (E0 > E2 ? E0 : E2) : (E1 > E2 ? E1 : E2);
+    // fused form only: the chunk's operands of the state step, kept on chip ---
+    // [W; Q~] as 128-row K-major tiles per 64 key channels, U0, K^ and P (P
+    // directly after K^, so the 128-row operand [*; P] reads K^'s tail as its
+    // unused rows 0..63), gamma_C, and the fp16 state (rows = key channel) and
+    // U operands of the state step
+    static constexpr int NTV = DV > 64 ? DV / 64 : 1;
+    static constexpr uint32_t FWQ = END0;
+    static constexpr uint32_t FU0 = FWQ + (DK / 64) * 16384;
+    static constexpr uint32_t FKH = FU0 + (DV / 64) * TILE;
+    static constexpr uint32_t FP = FKH + (DK / 64) * TILE;
+    static constexpr uint32_t S16 = FP + TILE;
+    static constexpr uint32_t U16 = S16 + NTV * 16384;
+    static constexpr uint32_t FGC = U16 + NTV * TILE;
+    static constexpr uint32_t END = FUSED ? FGC + DK * 4 : END0;
     static constexpr uint32_t BAR = END;                                 // bar_in, bar_v, bar_mma
     static constexpr uint32_t TMEMADDR = BAR + 24;
     static constexpr uint32_t BETA = BAR + 32;                           // [64]
@@ -85,15 +99,17 @@ struct K1fSmem {
     static constexpr uint32_t EGLM = EGM + DK * 4;                       // [DK] e^{g_{L-1} - g_m}
     static constexpr uint32_t LAH = EGLM + DK * 4;                       // [64] per-head log-decay
     static constexpr uint32_t PART = LAH + 256;                          // [256 / DK][DK] scan partials
-    static constexpr uint32_t TOTAL = PART + 256 * 4;
+    static constexpr uint32_t PAIR = PART + 256 * 4;                     // fused: the claimed pair
+    static constexpr uint32_t TOTAL = PAIR + 16;
     static constexpr uint32_t KQ_TX = 2 * (DK / 64) * TILE;              // k and q tiles
     static constexpr uint32_t LA_TX = 64 * DK * 4;
     static constexpr uint32_t V_TX = (DV / 64) * TILE;
     static_assert(TP % 1024 == 0 && OPB % 1024 == 0 && G % 1024 == 0, "swizzled tiles need 1024-byte alignment");
     static_assert(AMS >= G + G_BYTES, "the strong path's A lies outside the live log-decay tile");
     static_assert(AMD + 4 * 260 * 4 <= T1H + 16384 && AMS + 64 * 68 * 4 <= AMD, "T-solve scratch");
-    // two CTAs per SM: 228 KB per SM, 1 KB reserved per CTA
-    static_assert(2 * (TOTAL + 1024) <= 233472, "two CTAs per SM");
+    // two CTAs per SM (228 KB per SM, 1 KB reserved per CTA); the fused form one
+    static_assert(FUSED ? TOTAL <= 232448 : 2 * (TOTAL + 1024) <= 233472, "CTAs per SM");
+    static_assert(FWQ % 1024 == 0 && S16 % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 };
 
 // g (base 2) of token r, channel c in the 128-byte-swizzled log-decay tiles
@@ -102,15 +118,17 @@ __device__ __forceinline__ uint32_t g_off(int r, int c) {
     return (uint32_t)(c >> 5) * 8192u + sw128_offset((uint32_t)r, (uint32_t)(c & 31) * 4u);
 }
 
-template <int DK, int DV, int GATE>
-__global__ void __launch_bounds__(256, 2)
+template <int DK, int DV, int GATE, bool FUSED>
+__global__ void __launch_bounds__(256, FUSED ? 1 : 2)
 intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_la,
                           const float* __restrict__ log_alpha_head, const float* __restrict__ beta,
                           ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
-                          size_t max_chunks, long long wait_cap, int drop_la)
+                          size_t max_chunks, long long wait_cap, int drop_la,
+                          const float* __restrict__ initial_state, float* __restrict__ final_state,
+                          __nv_bfloat16* __restrict__ o, float scale, const int* __restrict__ seq_order)
 {
-    using Sm = K1fSmem<DK, DV>;
+    using Sm = K1fSmem<DK, DV, FUSED>;
     using R = TcRec<DK, DV>;
     constexpr int NPART = 256 / DK;       // threads per key channel in the scan
     constexpr int TPP = kChunk / NPART;   // tokens per such thread
@@ -131,7 +149,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 
     if (hdr->status != kStatusOk) return;
     const int total = hdr->num_chunks * H;
-    if ((int)blockIdx.x >= total) return;
+    if (!FUSED && (int)blockIdx.x >= total) return;
     if ((smem_u32(sm) & 1023u) != 0) {   // the swizzled layouts need 1024-byte alignment
         if (threadIdx.x == 0) flag_error(hdr, kStatusInternal);
         return;
@@ -148,8 +166,9 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         mbar_init(&bar_mma, 1);
         fence_mbar_init();
     }
+    constexpr uint32_t kTmemCols = FUSED ? 512 : 256;
     if (warp == 0) {
-        tmem_alloc(&s_tmem, 256);
+        tmem_alloc(&s_tmem, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -159,20 +178,16 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     const uint32_t AOP = tmem;        // [K~m; Q~m] tf32, 128 lanes x DK columns
     const uint32_t D1 = tmem + DK;    // [A; P], 128 lanes x 64 columns
     const uint32_t D2 = tmem;         // [W | U0], lanes 0..63 x (DK + DV) columns (after D1 is read)
+    const uint32_t R3 = tmem;         // fused: [W S; Q~ S + P U], 128 lanes x DV (after D2 is read)
+    const uint32_t SACC = tmem + kTmemCols - DV;   // fused: the fp32 state, lanes 0..DK-1 x DV
 
-    auto locate = [&](int w, int& c, int& h, int& tok0, int& L) {
-        c = w / H;
-        h = w - c * H;
-        int seq;
-        map.locate(c, seq, tok0, L);
-    };
     // test hook: CTA 0 can leave out the log-decay copy of its third item (of
     // its last if it has fewer), so that the bounded wait on that item's
     // inputs gives up with earlier phases consumed
-    const int drop_it = (drop_la && blockIdx.x == 0) ? min(2, (total - 1) / (int)gridDim.x) : -1;
-    auto issue_in = [&](int w, int j) {   // k, q (and log_alpha) of item w, this CTA's j-th
-        int c, h, tok0, L;
-        locate(w, c, h, tok0, L);
+    const int drop_it = (!FUSED && drop_la && blockIdx.x == 0) ? min(2, (total - 1) / (int)gridDim.x) : -1;
+    auto issue_in = [&](int c, int h, int j) {   // k, q (and log_alpha) of chunk c, head h: this CTA's j-th item
+        int seq, tok0, L;
+        map.locate(c, seq, tok0, L);
         mbar_arrive_expect_tx(&bar_in, Sm::KQ_TX + (channel_gate ? Sm::LA_TX : 0u));
 #pragma unroll
         for (int b = 0; b < DK / 64; ++b) {
@@ -188,45 +203,47 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     };
     // beta (and a per-head log-decay) of item w into registers, threads 192..255
     float beta_next = 0.f, lah_next = 0.f;
-    auto load_beta = [&](int w) {
+    auto load_beta = [&](int c, int h) {
         if (tid >= 192) {
-            int c, h, tok0, L;
-            locate(w, c, h, tok0, L);
+            int seq, tok0, L;
+            map.locate(c, seq, tok0, L);
             const int r = tid - 192;
             beta_next = (r < L) ? ld_prefetch_f32(beta + (size_t)(tok0 + r) * H + h) : 0.f;
             lah_next = (GATE == kGateHead && r < L) ? ld_prefetch_f32(log_alpha_head + (size_t)(tok0 + r) * H + h) : 0.f;
         }
     };
 
-    if (tid == kCopyThread) issue_in(blockIdx.x, 0);
-    load_beta(blockIdx.x);
-
     bool aborted = false;
     uint32_t mma_phase = 0;
     int mma_pending = 0;          // a commit on bar_mma not yet waited for
     // this CTA's j-th item lands on bar_in / bar_v with phase parity j & 1;
     // items [in_done, in_issued) and [v_done, v_issued) are in flight
-    int in_issued = 1, in_done = 0, v_issued = 0, v_done = 0;
+    int in_issued = 0, in_done = 0, v_issued = 0, v_done = 0;
     bool stored = false;          // the copy thread has bulk stores in flight
     float range_max = 0.f;
 
-    int it = 0;
-    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x, ++it) {
-        int c, h, tok0, L;
-        locate(w, c, h, tok0, L);
+    int it = 0;   // this CTA's item count
+    // One (chunk c, head h) item of L tokens from token tok0; (nc, nh) is this
+    // CTA's next item (nc < 0: none), prefetched once this one's inputs are
+    // consumed.  Returns false if a wait gave up.
+    auto run_item = [&](int c, int h, int tok0, int L, int nc, int nh) -> bool {
         unsigned char* rec = records + ((size_t)h * max_chunks + c) * R::BYTES;
+        // where the chunk's intermediates go: the record (split form) or the
+        // on-chip operands of the state step (fused form)
+        float* gc_dst = FUSED ? reinterpret_cast<float*>(sm + Sm::FGC) : reinterpret_cast<float*>(rec + R::GC);
+        unsigned char* kh_dst = FUSED ? sm + Sm::FKH : rec + R::KH;
+        unsigned char* p_dst = FUSED ? sm + Sm::FP : rec + R::P;
         if (tid >= 192) {
             s_beta[tid - 192] = beta_next;
             if constexpr (GATE == kGateHead) s_lah[tid - 192] = lah_next;
         }
-        const int wn = w + gridDim.x;   // this CTA's next item
-        if (wn < total) load_beta(wn);
+        if (nc >= 0) load_beta(nc, nh);
         // the previous item's W / U0 staging (OPB) must be read before it is reused
         if (tid == kCopyThread && stored) bulk_store_wait_read();
 
         // ---- cumulative log-decay, in place over the log_alpha tile in G -------
-        const bool ok_in = tid != 0 || mbar_wait_cycles(&bar_in, it & 1, wait_cap);
-        if (__syncthreads_or(!ok_in)) { aborted = true; break; }
+        const bool ok_in = (!FUSED && tid != 0) || mbar_wait_cycles(&bar_in, it & 1, wait_cap);
+        if (__syncthreads_or(!ok_in)) return false;
         in_done = it + 1;
         {
             float la_cur[TPP];
@@ -256,7 +273,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             s_gm[tid] = gm;
             s_egm[tid] = ex2_approx(gm);
             s_eglm[tid] = ex2_approx(gl - gm);
-            reinterpret_cast<float*>(rec + R::GC)[tid] = exp2f(gl);
+            gc_dst[tid] = exp2f(gl);
             wide = fmaxf(gat(0, tid) - gm, gm - gl) > kMaxSplitExponent2;
         }
         // Strong decay: the factors e^{+-(g - g_m)} of A and P could overflow, so
@@ -264,7 +281,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         const bool strong = __syncthreads_or(wide);
         float* am = reinterpret_cast<float*>(sm + Sm::AMS);   // strong path: [64][68]
         if (strong) {
-            exact_a_p<DK>(gat, sm + Sm::KT, sm + Sm::QT, s_beta, L, am, rec + R::P);
+            exact_a_p<DK>(gat, sm + Sm::KT, sm + Sm::QT, s_beta, L, am, p_dst);
             __syncthreads();   // the k, q tiles are converted in place next
         }
 
@@ -284,6 +301,10 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                 const int c8 = CH * hc + 8 * j;
                 const uint32_t ho = (uint32_t)(c8 >> 6) * Sm::TILE + sw128_offset(er, (c8 & 63) * 2);
                 unsigned char* xt = sm + (is_k ? Sm::KT : Sm::QT) + ho;   // this row's k or q chunk
+                // K~ goes back in place (MMA2's operand); Q~ in place (split form:
+                // bulk-stored to the record) or into the fused [W; Q~] operand
+                unsigned char* xo = (FUSED && !is_k)
+                    ? sm + Sm::FWQ + (uint32_t)(c8 >> 6) * 16384 + 8192 + sw128_offset(er, (c8 & 63) * 2) : xt;
                 uint4 raw = *reinterpret_cast<const uint4*>(xt);
                 if (!live) raw = make_uint4(0, 0, 0, 0);
                 const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(&raw);
@@ -325,7 +346,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                         const uint32_t fo = (uint32_t)(c8 >> 5) * Sm::TILE, fb = (c8 & 31) * 4;
                         *reinterpret_cast<float4*>(sm + Sm::OPB + fo + sw128_offset(er, fb)) = *reinterpret_cast<const float4*>(kbm);
                         *reinterpret_cast<float4*>(sm + Sm::OPB + fo + sw128_offset(er, fb + 16)) = *reinterpret_cast<const float4*>(kbm + 4);
-                        *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(h1);
+                        *reinterpret_cast<uint4*>(kh_dst + ho) = *reinterpret_cast<const uint4*>(h1);
                     } else {
 #pragma unroll
                         for (int e2 = 0; e2 < 4; ++e2) {
@@ -340,7 +361,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                             h0[e2] = __floats2half2_rn(t[0], t[1]);
                         }
                     }
-                    *reinterpret_cast<uint4*>(xt) = *reinterpret_cast<const uint4*>(h0);
+                    *reinterpret_cast<uint4*>(xo) = *reinterpret_cast<const uint4*>(h0);
                     tmem_st8(AOP + lane_base + c8, top);
                 } else {   // strong-decay chunk: unsplit factors, every exponent <= 0; no MMA1 operands
 #pragma unroll
@@ -356,8 +377,8 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                         h0[e2] = __floats2half2_rn(t[0], t[1]);
                         h1[e2] = __floats2half2_rn(u2[0], u2[1]);
                     }
-                    *reinterpret_cast<uint4*>(xt) = *reinterpret_cast<const uint4*>(h0);
-                    if (is_k) *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(h1);
+                    *reinterpret_cast<uint4*>(xo) = *reinterpret_cast<const uint4*>(h0);
+                    if (is_k) *reinterpret_cast<uint4*>(kh_dst + ho) = *reinterpret_cast<const uint4*>(h1);
                 }
             }
         };
@@ -382,14 +403,16 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         }
         mma_pending = strong ? 0 : 1;
         if (tid == kCopyThread) {
-            // Q~ tiles are the lower halves (rows 64..127) of the record's WQ
-            // tiles; once they are read, v comes into the same buffer
+            if constexpr (!FUSED) {
+                // Q~ tiles are the lower halves (rows 64..127) of the record's WQ
+                // tiles; once they are read, v comes into the same buffer
 #pragma unroll
-            for (int b = 0; b < DK / 64; ++b)
-                bulk_store(rec + R::WQ + b * 16384 + 8192, sm + Sm::QT + b * Sm::TILE, 8192);
-            bulk_store_commit();
-            stored = true;
-            bulk_store_wait_read();
+                for (int b = 0; b < DK / 64; ++b)
+                    bulk_store(rec + R::WQ + b * 16384 + 8192, sm + Sm::QT + b * Sm::TILE, 8192);
+                bulk_store_commit();
+                stored = true;
+                bulk_store_wait_read();
+            }
             mbar_arrive_expect_tx(&bar_v, Sm::V_TX);
 #pragma unroll
             for (int b = 0; b < DV / 64; ++b) tma_load_3d(sm + Sm::QT + b * Sm::TILE, &tm_v, &bar_v, b * 64, h, tok0);
@@ -432,8 +455,8 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         };
         bool ok = true;
         if (!strong) {
-            ok = tid != 0 || mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            ok = (!FUSED && tid != 0) || mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+            if (__syncthreads_or(!ok)) return false;
             mma_phase ^= 1;
             mma_pending = 0;
             tc_fence_after();
@@ -456,7 +479,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                         const int col = 32 * hc + 8 * i8 + e;
                         hv[e] = __float2half_rn(col <= r ? v[8 * i8 + e] : 0.f);
                     }
-                    *reinterpret_cast<uint4*>(rec + R::P + sw128_offset(r, (32 * hc + 8 * i8) * 2)) =
+                    *reinterpret_cast<uint4*>(p_dst + sw128_offset(r, (32 * hc + 8 * i8) * 2)) =
                         *reinterpret_cast<const uint4*>(hv);
                 }
             }
@@ -519,7 +542,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                 mma_commit(&bar_mma);
             }
             mma_pending = 1;
-            const bool good = tid != 0 || mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+            const bool good = (!FUSED && tid != 0) || mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
             if (__syncthreads_or(!good)) return false;
             mma_phase ^= 1;
             mma_pending = 0;
@@ -541,9 +564,9 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             }
         };
         // level 1: X = A_L1 D, Y = D X; T_10 = -Y_10, T_32 = -Y_32; T1 = D + those blocks
-        if (!level_mma(Sm::AH1, Sm::DH)) { aborted = true; break; }
+        if (!level_mma(Sm::AH1, Sm::DH)) return false;
         store_x(Sm::XH);
-        if (!level_mma(Sm::DH, Sm::XH)) { aborted = true; break; }
+        if (!level_mma(Sm::DH, Sm::XH)) return false;
         if (row < 64) {
             const int b = row >> 4;
             float v[32];
@@ -568,9 +591,9 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             }
         }
         // level 2: X = A_L2 T1, Y = T1 X; T[32:64, 0:32] = -Y[32:64, 0:32]
-        if (!level_mma(Sm::AH2, Sm::T1H)) { aborted = true; break; }
+        if (!level_mma(Sm::AH2, Sm::T1H)) return false;
         store_x(Sm::XH);
-        if (!level_mma(Sm::T1H, Sm::XH)) { aborted = true; break; }
+        if (!level_mma(Sm::T1H, Sm::XH)) return false;
         if (row >= 32 && row < 64 && hc == 0) {
             float v[32];
             tmem_ld32_sync(tmem + lane_base, v);
@@ -584,8 +607,8 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         }
 
         // ---- v: bf16 -> fp16 in place in QT, 8 values per thread and step
-        ok = tid != 0 || mbar_wait_cycles(&bar_v, it & 1, wait_cap);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        ok = (!FUSED && tid != 0) || mbar_wait_cycles(&bar_v, it & 1, wait_cap);
+        if (__syncthreads_or(!ok)) return false;
         v_done = it + 1;
         for (int item = tid; item < kChunk * (DV / 8); item += 256) {
             const int r = item / (DV / 8), j8 = (item - r * (DV / 8)) * 8;
@@ -623,14 +646,14 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             mma_commit(&bar_mma);
         }
         mma_pending = 1;
-        ok = tid != 0 || mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
+        ok = (!FUSED && tid != 0) || mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+        if (__syncthreads_or(!ok)) return false;
         mma_phase ^= 1;
         mma_pending = 0;
         tc_fence_after();
         // KT, QT and G are free: the next item's inputs come in behind the write-out
-        if (tid == kCopyThread && wn < total) issue_in(wn, it + 1);
-        if (wn < total) in_issued = it + 2;
+        if (tid == kCopyThread && nc >= 0) issue_in(nc, nh, it + 1);
+        if (nc >= 0) in_issued = it + 2;
 
         // ---- W and U0 (rows 0..63): fp16 into the OPB staging tiles (record
         //      layout), then one bulk store per tile; warps 0, 1, 4, 5 (TMEM
@@ -650,19 +673,239 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                         hv[e] = __float2half_rn(v[8 * i8 + e]);
                     }
                     const int col = 32 * cb + 8 * i8;   // W tiles then U0 tiles, 64 columns each
-                    *reinterpret_cast<uint4*>(sm + Sm::OPB + h_off(r, col, Sm::TILE)) = *reinterpret_cast<const uint4*>(hv);
+                    uint32_t dst;
+                    if constexpr (FUSED)   // W: rows 0..63 of the [W; Q~] operand; U0 on its own
+                        dst = col < DK ? Sm::FWQ + (uint32_t)(col >> 6) * 16384 + sw128_offset(r, (col & 63) * 2)
+                                       : Sm::FU0 + h_off(r, col - DK, Sm::TILE);
+                    else
+                        dst = Sm::OPB + h_off(r, col, Sm::TILE);
+                    *reinterpret_cast<uint4*>(sm + dst) = *reinterpret_cast<const uint4*>(hv);
                 }
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();   // D2 and the staging tiles are complete
-        if (tid == kCopyThread) {
+        __syncthreads();   // D2 is read; the staging tiles (or the state step's operands) are complete
+        if constexpr (!FUSED) {
+            if (tid == kCopyThread) {
 #pragma unroll
-            for (int b = 0; b < DK / 64; ++b)   // W: rows 0..63 of each WQ tile
-                bulk_store(rec + R::WQ + b * 16384, sm + Sm::OPB + b * Sm::TILE, Sm::TILE);
-            bulk_store(rec + R::U0, sm + Sm::OPB + (DK / 64) * Sm::TILE, (DV / 64) * Sm::TILE);
-            bulk_store_commit();
+                for (int b = 0; b < DK / 64; ++b)   // W: rows 0..63 of each WQ tile
+                    bulk_store(rec + R::WQ + b * 16384, sm + Sm::OPB + b * Sm::TILE, Sm::TILE);
+                bulk_store(rec + R::U0, sm + Sm::OPB + (DK / 64) * Sm::TILE, (DV / 64) * Sm::TILE);
+                bulk_store_commit();
+            }
+        }
+        ++it;
+        return true;
+    };
+
+    if constexpr (!FUSED) {
+        // ---- split form: items (chunk, head) w = blockIdx.x + i gridDim.x; the
+        //      records go to the workspace for the inter-chunk kernel
+        if (tid == kCopyThread) issue_in(blockIdx.x / H, blockIdx.x % H, 0);
+        in_issued = 1;
+        load_beta(blockIdx.x / H, blockIdx.x % H);
+        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+            const int c = w / H, h = w - c * H;
+            int seq, tok0, L;
+            map.locate(c, seq, tok0, L);
+            const int wn = w + gridDim.x;
+            if (!run_item(c, h, tok0, L, wn < total ? wn / H : -1, wn < total ? wn % H : 0)) { aborted = true; break; }
+        }
+    } else {
+        // ---- fused form: whole (sequence, head) pairs, claimed longest first;
+        //      after each chunk's intra-chunk phases the state step consumes the
+        //      chunk's operands from shared memory (no records), with the fp32
+        //      state resident in TMEM for the whole sequence
+        constexpr int CPT = DV / 2;                       // state columns per thread
+        const uint32_t cb = (uint32_t)(CPT * hc);
+        int* s_pair = reinterpret_cast<int*>(sm + Sm::PAIR);
+        auto ld_cols = [&](uint32_t taddr, float (&v)[CPT]) {
+#pragma unroll
+            for (int c0 = 0; c0 < CPT; c0 += 32) {
+                float t[32];
+                tmem_ld32_sync(taddr + c0, t);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[c0 + i] = t[i];
+            }
+        };
+        auto st_cols = [&](uint32_t taddr, const float (&v)[CPT]) {
+#pragma unroll
+            for (int c0 = 0; c0 < CPT; c0 += 32) {
+                float t[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) t[i] = v[c0 + i];
+                tmem_st32_sync(taddr + c0, t);
+            }
+        };
+        // fp16 copy of this thread's state columns (row = key channel): MMA3's B operand
+        auto put_s16 = [&](const float (&v)[CPT]) {
+#pragma unroll
+            for (int i8 = 0; i8 < CPT / 8; ++i8) {
+                const uint32_t col = cb + 8 * i8;
+                __align__(16) __half2 hv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = v[8 * i8 + 2 * e], x1 = v[8 * i8 + 2 * e + 1];
+                    range_max = fmaxf(range_max, fmaxf(fabsf(x0), fabsf(x1)));
+                    hv[e] = __floats2half2_rn(x0, x1);
+                }
+                *reinterpret_cast<uint4*>(sm + Sm::S16 + (col >> 6) * 16384 + sw128_offset(row, (col & 63) * 2)) =
+                    *reinterpret_cast<const uint4*>(hv);
+            }
+        };
+        // one chunk of the state recurrence, on the chunk's on-chip operands:
+        //   U = U0 - W S,  O = d_k^{-1/2} (Q~ S + P U),  S <- Diag(gamma_C) S + K^^T U
+        auto state_step = [&](int tok0, int L, int h) -> bool {
+            if (tid == 0) {   // MMA3: [W; Q~] S -> R3
+                tc_fence_after();
+                constexpr uint32_t idesc = instr_desc(kFmtF16, 128, DV, false, true);
+                const uint32_t a0 = smem_u32(sm + Sm::FWQ), b0 = smem_u32(sm + Sm::S16);
+#pragma unroll
+                for (int kb = 0; kb < DK / 64; ++kb)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16(R3, smem_desc(a0 + kb * 16384 + ks * 32, 16, 1024, kLayoutSW128),
+                                smem_desc(b0 + kb * 8192 + ks * 2048, 16384, 1024, kLayoutSW128), idesc, (kb | ks) != 0);
+                mma_commit(&bar_mma);
+            }
+            mma_pending = 1;
+            if (row < DK) {   // S <- Diag(gamma_C) S while MMA3 reads the fp16 copy
+                const float gcv = reinterpret_cast<const float*>(sm + Sm::FGC)[row];
+                float v[CPT];
+                ld_cols(SACC + lane_base + cb, v);
+#pragma unroll
+                for (int i = 0; i < CPT; ++i) v[i] *= gcv;
+                st_cols(SACC + lane_base + cb, v);
+            }
+            bool ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+            if (__syncthreads_or(!ok)) return false;
+            mma_phase ^= 1;
+            mma_pending = 0;
+            tc_fence_after();
+            if (row < 64) {   // U = U0 - W S (rows = tokens) -> U16
+                float v[CPT];
+                ld_cols(R3 + lane_base + cb, v);
+#pragma unroll
+                for (int i8 = 0; i8 < CPT / 8; ++i8) {
+                    const uint32_t off = h_off(row, cb + 8 * i8, Sm::TILE);
+                    const uint4 u0raw = *reinterpret_cast<const uint4*>(sm + Sm::FU0 + off);
+                    const __half2* u0 = reinterpret_cast<const __half2*>(&u0raw);
+                    __align__(16) __half2 hv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 u0f = __half22float2(u0[e]);
+                        const float ua = u0f.x - v[8 * i8 + 2 * e], ub = u0f.y - v[8 * i8 + 2 * e + 1];
+                        range_max = fmaxf(range_max, fmaxf(fabsf(ua), fabsf(ub)));
+                        hv[e] = __floats2half2_rn(ua, ub);
+                    }
+                    *reinterpret_cast<uint4*>(sm + Sm::U16 + off) = *reinterpret_cast<const uint4*>(hv);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {   // MMA4: [*; P] U += R3;  MMA5: K^^T U += S
+                tc_fence_after();
+                constexpr uint32_t idesc = instr_desc(kFmtF16, 128, DV, false, true);
+                constexpr uint32_t idesc_t = instr_desc(kFmtF16, 128, DV, true, true);
+                const uint32_t pa = smem_u32(sm + Sm::FP) - 8192, ub = smem_u32(sm + Sm::U16);
+                const uint32_t ka = smem_u32(sm + Sm::FKH);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(R3, smem_desc(pa + ks * 32, 16, 1024, kLayoutSW128),
+                            smem_desc(ub + ks * 2048, 8192, 1024, kLayoutSW128), idesc, true);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(SACC, smem_desc(ka + ks * 2048, 8192, 1024, kLayoutSW128),
+                            smem_desc(ub + ks * 2048, 8192, 1024, kLayoutSW128), idesc_t, true);
+                mma_commit(&bar_mma);
+            }
+            mma_pending = 1;
+            ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
+            if (__syncthreads_or(!ok)) return false;
+            mma_phase ^= 1;
+            mma_pending = 0;
+            tc_fence_after();
+            if (row >= 64) {   // output rows
+                const int r = row - 64;
+                float v[CPT];
+                ld_cols(R3 + lane_base + cb, v);
+                if (r < L) {
+                    __nv_bfloat16* dst = o + ((size_t)(tok0 + r) * H + h) * DV + cb;
+#pragma unroll
+                    for (int i8 = 0; i8 < CPT / 8; ++i8) {
+                        __align__(16) __nv_bfloat162 bv[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            bv[e] = __floats2bfloat162_rn(scale * v[8 * i8 + 2 * e], scale * v[8 * i8 + 2 * e + 1]);
+                        *reinterpret_cast<uint4*>(dst + 8 * i8) = *reinterpret_cast<const uint4*>(bv);
+                    }
+                }
+            }
+            if (row < DK) {   // the next chunk's fp16 state operand
+                float v[CPT];
+                ld_cols(SACC + lane_base + cb, v);
+                put_s16(v);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            return true;
+        };
+
+        const int num_pairs = map.num_seqs * H;
+        for (;;) {
+            if (tid == 0) *s_pair = atomicAdd(&hdr->next_pair, 1);
+            __syncthreads();
+            const int p = *s_pair;
+            __syncthreads();
+            if (p >= num_pairs) break;
+            const int si = p / H, h = p - si * H;
+            const int s = seq_order ? seq_order[si] : si;
+            const int first = map.seq_first_chunk(s), nch = map.seq_num_chunks(s);
+            const int tb = map.seq_token_begin(s), te = map.seq_token_end(s);
+            const size_t soff = ((size_t)s * H + h) * DK * DV;
+            if (nch <= 0) {   // empty sequence: the state passes through
+                if (final_state)
+                    for (int i = tid; i < DK * DV; i += 256) final_state[soff + i] = initial_state ? initial_state[soff + i] : 0.f;
+                continue;
+            }
+            if (tid == kCopyThread) issue_in(first, h, it);
+            in_issued = it + 1;
+            load_beta(first, h);
+            if (row < DK) {   // initial state -> TMEM (fp32) and its fp16 operand copy
+                float v[CPT];
+#pragma unroll
+                for (int i = 0; i < CPT; i += 4) {
+                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (initial_state) x = *reinterpret_cast<const float4*>(initial_state + soff + (size_t)row * DV + cb + i);
+                    v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+                }
+                st_cols(SACC + lane_base + cb, v);
+                put_s16(v);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            for (int j = 0; j < nch; ++j) {
+                const int tok0 = tb + j * kChunk, L = min(kChunk, te - tok0);
+                if (!run_item(first + j, h, tok0, L, j + 1 < nch ? first + j + 1 : -1, h)) { aborted = true; break; }
+                if (!state_step(tok0, L, h)) { aborted = true; break; }
+            }
+            if (aborted) break;
+            if (final_state && row < DK) {
+                float v[CPT];
+                ld_cols(SACC + lane_base + cb, v);
+                float* dst = final_state + soff + (size_t)row * DV + cb;
+#pragma unroll
+                for (int i = 0; i < CPT; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            }
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
         }
     }
 
@@ -679,48 +922,101 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-template <int DK, int DV>
+// Packed sequences ordered longest first (ties by index) for the fused form's
+// pair queue: order[rank(s)] = s.  One block; beyond 16384 sequences the order
+// is left as given.
+__global__ void __launch_bounds__(1024)
+seq_order_kernel(const WsHeader* hdr, const int32_t* __restrict__ cu, int N, int* __restrict__ order)
+{
+    if (hdr->status != kStatusOk) return;
+    for (int s = threadIdx.x; s < N; s += blockDim.x) {
+        int rank = s;
+        if (N <= 16384) {
+            const int len = cu[s + 1] - cu[s];
+            rank = 0;
+            for (int t = 0; t < N; ++t) {
+                const int lt = cu[t + 1] - cu[t];
+                rank += (lt > len) || (lt == len && t < s);
+            }
+        }
+        order[rank] = s;
+    }
+}
+
+template <int DK, int DV, bool FUSED>
 cudaError_t launch_intra_fwd_tc_t(const ChunkArgs& a) {
-    if (a.max_chunks == 0) return cudaSuccess;
+    if (a.max_chunks == 0 && !FUSED) return cudaSuccess;
     const int ntok = a.cu_seqlens ? a.T : a.B * a.T;
     CUtensorMap mk, mv, mq, mla;
-    if (!make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        (a.gate == kGateChannel &&
-         !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, ntok, 32, CU_TENSOR_MAP_SWIZZLE_128B)))
+    memset(&mk, 0, sizeof(mk));
+    memset(&mv, 0, sizeof(mv));
+    memset(&mq, 0, sizeof(mq));
+    memset(&mla, 0, sizeof(mla));
+    if (ntok > 0 &&
+        (!make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+         !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+         !make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+         (a.gate == kGateChannel &&
+          !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, ntok, 32, CU_TENSOR_MAP_SWIZZLE_128B))))
         return cudaErrorInvalidValue;
-    if (a.gate != kGateChannel) memset(&mla, 0, sizeof(mla));   // unused
     ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
-    auto kern = a.gate == kGateChannel ? intra_chunk_fwd_tc_kernel<DK, DV, kGateChannel>
-              : a.gate == kGateHead    ? intra_chunk_fwd_tc_kernel<DK, DV, kGateHead>
-                                       : intra_chunk_fwd_tc_kernel<DK, DV, kGateNone>;
-    const int smem = (int)K1fSmem<DK, DV>::TOTAL;
+    auto kern = a.gate == kGateChannel ? intra_chunk_fwd_tc_kernel<DK, DV, kGateChannel, FUSED>
+              : a.gate == kGateHead    ? intra_chunk_fwd_tc_kernel<DK, DV, kGateHead, FUSED>
+                                       : intra_chunk_fwd_tc_kernel<DK, DV, kGateNone, FUSED>;
+    const int smem = (int)K1fSmem<DK, DV, FUSED>::TOTAL;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const size_t items = a.max_chunks * (size_t)a.H;   // upper bound; the kernel reads the exact count
-    const size_t ctas = 2 * (size_t)sms;               // two resident per SM
-    const unsigned grid = (unsigned)(items < ctas ? items : ctas);
+    unsigned grid;
+    const int* order = nullptr;
+    if constexpr (FUSED) {
+        // the pair queue: packed sequences longest first, in the records region
+        // (unused by this form; the caller checked it holds N ints)
+        if (a.cu_seqlens && a.num_seqs > 1) {
+            int* ord = static_cast<int*>(a.records);
+            seq_order_kernel<<<1, 1024, 0, a.stream>>>(static_cast<WsHeader*>(a.ws_header), a.cu_seqlens,
+                                                       a.num_seqs, ord);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            order = ord;
+        }
+        const size_t pairs = (size_t)a.num_seqs * a.H;
+        grid = (unsigned)(pairs < (size_t)sms ? pairs : (size_t)sms);   // one resident per SM
+        if (grid == 0) return cudaSuccess;
+    } else {
+        const size_t items = a.max_chunks * (size_t)a.H;   // upper bound; the kernel reads the exact count
+        const size_t ctas = 2 * (size_t)sms;               // two resident per SM
+        grid = (unsigned)(items < ctas ? items : ctas);
+    }
     kern<<<grid, 256, smem, a.stream>>>(mk, mv, mq, mla, a.log_alpha, a.beta, map,
                                         static_cast<WsHeader*>(a.ws_header),
                                         static_cast<unsigned char*>(a.records), a.H, a.max_chunks,
-                                        a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy);
+                                        a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy,
+                                        a.initial_state, a.final_state, static_cast<__nv_bfloat16*>(a.o), a.scale,
+                                        order);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_chunk_intra_fwd_tc(const ChunkArgs& a) {
-    if (a.dk == 128 && a.dv == 128) return launch_intra_fwd_tc_t<128, 128>(a);
-    if (a.dk == 128 && a.dv == 64) return launch_intra_fwd_tc_t<128, 64>(a);
-    if (a.dk == 64 && a.dv == 128) return launch_intra_fwd_tc_t<64, 128>(a);
-    if (a.dk == 64 && a.dv == 64) return launch_intra_fwd_tc_t<64, 64>(a);
+    if (a.dk == 128 && a.dv == 128) return launch_intra_fwd_tc_t<128, 128, false>(a);
+    if (a.dk == 128 && a.dv == 64) return launch_intra_fwd_tc_t<128, 64, false>(a);
+    if (a.dk == 64 && a.dv == 128) return launch_intra_fwd_tc_t<64, 128, false>(a);
+    if (a.dk == 64 && a.dv == 64) return launch_intra_fwd_tc_t<64, 64, false>(a);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_chunk_fused_tc(const ChunkArgs& a) {
+    if (a.num_seqs == 0) return cudaSuccess;
+    if (a.dk == 128 && a.dv == 128) return launch_intra_fwd_tc_t<128, 128, true>(a);
+    if (a.dk == 128 && a.dv == 64) return launch_intra_fwd_tc_t<128, 64, true>(a);
+    if (a.dk == 64 && a.dv == 128) return launch_intra_fwd_tc_t<64, 128, true>(a);
+    if (a.dk == 64 && a.dv == 64) return launch_intra_fwd_tc_t<64, 64, true>(a);
     return cudaErrorInvalidValue;
 }
 

@@ -75,6 +75,7 @@ cudaError_t launch_chunk_intra_tc(const ChunkArgs& a); // bf16 inputs: tensor-co
 cudaError_t launch_chunk_intra_fwd_tc(const ChunkArgs& a); // its forward-only form, two CTAs per SM
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K2
 cudaError_t launch_chunk_inter_fwd_tc(const ChunkArgs& a); // its forward-only form, slice width per call
+cudaError_t launch_chunk_fused_tc(const ChunkArgs& a);     // bf16 forward in one pass, one CTA per (sequence, head)
 cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a);  // backward: serial over chunks, reversed
 cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a); // the same on the tensor cores (bf16 inputs)
 cudaError_t launch_chunk_bwd_vside_tc(const ChunkArgs& a); // backward products over the value dim (bf16 inputs)

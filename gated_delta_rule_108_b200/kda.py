@@ -65,6 +65,10 @@ def _declare(lib):
     lib.kda_chunk_bwd_gated.restype = i
     lib.kda_chunk_bwd_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
                                         vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.kda_chunk_fwd_plan.restype = i
+    lib.kda_chunk_fwd_plan.argtypes = [i, i, i, i, i, i, i, i, sz]
+    lib.kda_chunk_fwd_fused_workspace_size.restype = sz
+    lib.kda_chunk_fwd_fused_workspace_size.argtypes = [i, i, i, i, i, i, i, i]
     lib.kda_workspace_status.restype = i
     lib.kda_workspace_status.argtypes = [vp, sz, vp]
     lib.kda_set_stage_events.restype = i
@@ -166,6 +170,27 @@ def chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
     code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
     return int(lib().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs,
                                                   int(bool(varlen)), code))
+
+
+def chunk_fwd_plan(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int, varlen: bool,
+                   dtype: torch.dtype, workspace_bytes: Optional[int] = None) -> int:
+    """1 if ``chunk_fwd`` with a workspace of ``workspace_bytes`` (default: the
+    full ``chunk_fwd_workspace_size``) runs the fused single pass, 0 for the
+    two-kernel form, -1 if neither fits (``kda_chunk_fwd_plan``)."""
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    if workspace_bytes is None:
+        workspace_bytes = chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, varlen, dtype)
+    return int(lib().kda_chunk_fwd_plan(B, T, H, dk, dv, num_seqs, int(bool(varlen)), code,
+                                        int(workspace_bytes)))
+
+
+def chunk_fwd_fused_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
+                                   num_seqs: int, varlen: bool, dtype: torch.dtype) -> int:
+    """Workspace bytes of the fused single pass (``kda_chunk_fwd_fused_workspace_size``;
+    0 for fp32 inputs)."""
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(lib().kda_chunk_fwd_fused_workspace_size(B, T, H, dk, dv, num_seqs,
+                                                        int(bool(varlen)), code))
 
 
 def _gate_of(log_alpha, channel_ndim: int, shape_channel, shape_head, device=None) -> int:

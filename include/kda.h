@@ -99,8 +99,11 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
  *  final_state [N, H, dk, dv]  fp32, written, or NULL.  May alias
  *              initial_state exactly (each state is read before it is written).
  *  workspace   device scratch of at least kda_chunk_fwd_workspace_size(...)
- *              bytes, 256-byte aligned; its contents on entry do not matter.
- *              Calls that share one workspace must be ordered on one stream.
+ *              bytes (bf16 inputs: or at least
+ *              kda_chunk_fwd_fused_workspace_size(...), which runs the fused
+ *              pass, see kda_chunk_fwd_plan), 256-byte aligned; its contents
+ *              on entry do not matter.  Calls that share one workspace must be
+ *              ordered on one stream.
  */
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          const float* log_alpha, const float* beta,
@@ -123,6 +126,36 @@ kda_status kda_recurrent_step(const void* q, const void* k, const void* v,
                               const float* log_alpha, const float* beta,
                               float* state_inout, int B, int H, int dk, int dv,
                               kda_dtype dtype, void* o, void* stream);
+
+/*
+ * The two forms of the bf16 chunk forward.  Both compute the same result up
+ * to rounding.
+ *  - split (two kernels): all (chunk, head) items in parallel, two CTAs per
+ *    SM, their intermediates through the workspace; then the chunk-to-chunk
+ *    recurrence, one CTA per (sequence, head, value slice).  Needs
+ *    kda_chunk_fwd_workspace_size bytes (about 74 KB per chunk and head at
+ *    d_k = d_v = 128).
+ *  - fused (one pass): one CTA per (sequence, head) pair carries the state
+ *    through the pair's chunks and keeps each chunk's intermediates on chip
+ *    (no intermediate traffic to memory); one CTA per SM.  Needs only
+ *    kda_chunk_fwd_fused_workspace_size bytes (header, chunk table, pair
+ *    order).  Slower than the split form on B200 at the shapes measured (its
+ *    intra-chunk phases cannot overlap a second CTA's), so it runs only when
+ *    the workspace passed to kda_chunk_fwd is too small for the split form,
+ *    or when forced.
+ * The environment variable KDA_CHUNK_PATH=fused or =split (read at every call)
+ * forces one form for bf16 inputs; fp32 inputs always take the split form.
+ *
+ * kda_chunk_fwd_plan returns 1 if kda_chunk_fwd with a workspace of
+ * `workspace_bytes` runs the fused pass, 0 for the split form, -1 for invalid
+ * sizes or a workspace too small for either.  Other arguments as
+ * kda_chunk_fwd_workspace_size.  kda_chunk_fwd_fused_workspace_size returns
+ * the fused pass's workspace bytes (0 for fp32 inputs or invalid sizes).
+ */
+int kda_chunk_fwd_plan(int B, int T, int H, int dk, int dv, int num_seqs, int varlen,
+                       kda_dtype dtype, size_t workspace_bytes);
+size_t kda_chunk_fwd_fused_workspace_size(int B, int T, int H, int dk, int dv,
+                                          int num_seqs, int varlen, kda_dtype dtype);
 
 /*
  * Waits for `stream`, then reads the device status that the last
@@ -255,8 +288,9 @@ kda_status kda_chunk_bwd_gated(const void* q, const void* k, const void* v,
  * kda_chunk_fwd on this host thread records the caller-created CUDA events
  * (cudaEvent_t passed as void*) on its stream at the stage boundaries:
  * events[0] before the first kernel, events[1] after the chunk-table/status
- * kernel, events[2] after the intra-chunk stage, events[3] after the
- * inter-chunk stage.  With `count` >= 7, each later kda_chunk_bwd records
+ * kernel, events[2] after the intra-chunk stage (the whole fused pass, when
+ * kda_chunk_fwd_plan says 1), events[3] after the inter-chunk stage (empty
+ * for the fused pass).  With `count` >= 7, each later kda_chunk_bwd records
  * events[0] before its first kernel and events[1..6] after the chunk-table,
  * forward intra-chunk, forward inter-chunk, reversed inter-chunk, tensor-core
  * product kernels (bf16 inputs: every chunk without strong decay is finished

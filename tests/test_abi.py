@@ -171,3 +171,24 @@ def test_debug_drop_copy_arms_and_disarms(lib):
     assert lib.kda_debug_drop_copy(-1) == 1
     assert lib.kda_debug_drop_copy(1000) == 0
     assert lib.kda_debug_drop_copy(0) == 0
+
+
+def test_chunk_fwd_plan_without_a_device(lib, monkeypatch):
+    bf16, f32 = 1, 0
+    big = 1 << 40
+    monkeypatch.delenv("KDA_CHUNK_PATH", raising=False)
+    assert lib.kda_chunk_fwd_plan(1, 100, 2, 96, 64, 1, 0, bf16, big) == -1    # unsupported dk
+    assert lib.kda_chunk_fwd_plan(4, 64, 8, 128, 128, 4, 0, f32, big) == 0      # fp32: split
+    assert lib.kda_chunk_fwd_plan(4, 64, 8, 128, 128, 4, 0, bf16, big) == 0     # room for the records: split
+    full = lib.kda_chunk_fwd_workspace_size(1, 300, 8, 128, 128, 3, 1, bf16)
+    small = lib.kda_chunk_fwd_fused_workspace_size(1, 300, 8, 128, 128, 3, 1, bf16)
+    assert 0 < small < full and small % 4 == 0
+    assert lib.kda_chunk_fwd_fused_workspace_size(1, 300, 8, 128, 128, 3, 1, f32) == 0
+    assert lib.kda_chunk_fwd_plan(1, 300, 8, 128, 128, 3, 1, bf16, full) == 0
+    assert lib.kda_chunk_fwd_plan(1, 300, 8, 128, 128, 3, 1, bf16, small) == 1   # only the fused pass fits
+    assert lib.kda_chunk_fwd_plan(1, 300, 8, 128, 128, 3, 1, bf16, small - 1) == -1
+    assert lib.kda_chunk_fwd_plan(1, 300, 8, 128, 128, 3, 1, f32, small) == -1
+    monkeypatch.setenv("KDA_CHUNK_PATH", "fused")
+    assert lib.kda_chunk_fwd_plan(1, 300, 8, 128, 128, 3, 1, bf16, full) == 1
+    monkeypatch.setenv("KDA_CHUNK_PATH", "split")
+    assert lib.kda_chunk_fwd_plan(1, 300, 8, 128, 128, 3, 1, bf16, small) == -1

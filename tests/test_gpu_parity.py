@@ -184,9 +184,11 @@ def test_c3_decode_full_sampled(cuda_device):
 
 
 @pytest.mark.parametrize("dk", [64, 128])
-def test_many_chains_wide_slices(cuda_device, dk):
-    """Enough (sequence, head) chains that the inter-chunk kernel takes whole
-    128-column value slices (one CTA per chain), with ragged sequences."""
+def test_many_chains_wide_slices(cuda_device, dk, monkeypatch):
+    """Enough (sequence, head) chains that the two-kernel form's inter-chunk
+    kernel takes whole 128-column value slices (one CTA per chain), with
+    ragged sequences (the fused pass would take this input by itself)."""
+    monkeypatch.setenv("KDA_CHUNK_PATH", "split")
     w = I.ChunkWorkload("wide", B=40, T=150, H=8, dk=dk, dv=128, dtype=torch.bfloat16, s0_std=0.05, seed=30)
     x = I.chunk_inputs(w)
     o, S = run_chunk(x)
