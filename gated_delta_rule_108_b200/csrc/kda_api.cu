@@ -44,9 +44,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool supported_dim(int d) { return d == 64 || d == 128; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace carve-up: [header 256 B][chunk_offsets (N+1) int32, 256-aligned][records].
+// Workspace carve-up: [header 256 B][chunk_offsets (N+1) int32][sequence order
+// N int32 (packed inputs: longest first)][records], each part 256-byte aligned.
 struct WsLayout {
-    size_t offsets_off, records_off, total;
+    size_t offsets_off, order_off, records_off, total;
     size_t max_chunks;
     int chunks_per_seq;
 };
@@ -68,7 +69,8 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
     // CUDA cores with fp32 records.
     const size_t rec = dtype == KDA_BF16 ? kda::tc_record_bytes(dk, dv) : kda::simt_record_bytes(dk, dv);
     L.offsets_off = kda::kHeaderBytes;
-    L.records_off = round_up(L.offsets_off + sizeof(int32_t) * ((size_t)N + 1), 256);
+    L.order_off = round_up(L.offsets_off + sizeof(int32_t) * ((size_t)N + 1), 256);
+    L.records_off = round_up(L.order_off + sizeof(int32_t) * (size_t)N, 256);
     L.total = L.records_off + rec * (size_t)H * L.max_chunks;
     return true;
 }
@@ -133,10 +135,11 @@ int chunk_path_override() {
     return 0;
 }
 
-// Workspace bytes of the fused single pass: the header, the chunk table and,
-// for packed sequences, the pair order (N ints) where the records would start.
+// Workspace bytes of the fused single pass: the header, the chunk table and
+// the sequence order (everything before the records).
 size_t fused_ws_bytes(int N, bool varlen, const WsLayout& L) {
-    return L.records_off + (varlen ? sizeof(int) * (size_t)N : 0);
+    (void)N; (void)varlen;
+    return L.records_off;
 }
 
 // fused (1) or split (0) for a workspace of ws_bytes (SIZE_MAX: as large as needed)
@@ -228,6 +231,8 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
     a.scale = 1.0f / sqrtf((float)dk);
     a.ws_header = workspace;
     a.chunk_offsets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + L.offsets_off);
+    a.seq_order = (a.bf16 && varlen && N > 1) ? reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + L.order_off)
+                                             : nullptr;
     a.records = static_cast<char*>(workspace) + L.records_off;
     a.max_chunks = L.max_chunks;
     a.fixed_chunks_per_seq = L.chunks_per_seq;
@@ -240,6 +245,7 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
 
     cudaError_t e = mark_stage(0, a.stream);
     if (e == cudaSuccess) e = kda::launch_chunk_prep(a);
+    if (e == cudaSuccess && a.bf16 && a.seq_order) e = kda::launch_chunk_seq_order(a);   // longest first
     if (e == cudaSuccess) e = mark_stage(1, a.stream);
     if (fused) {   // one pass; the inter-chunk stage is empty
         if (e == cudaSuccess) e = kda::launch_chunk_fused_tc(a);

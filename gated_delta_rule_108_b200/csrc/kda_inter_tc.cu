@@ -10,7 +10,7 @@
 //   U = U0 - W S,   O = d_k^{-1/2} (Q~ S + P U),   S <- Diag(gamma_C) S + K^^T U
 //
 // One CTA (8 warps) per (sequence, head, value slice), serial over the
-// sequence's chunks.  The fp32 state slice is resident in TMEM for the whole
+// sequence's chunks; packed sequences are started longest first.  The fp32 state slice is resident in TMEM for the whole
 // sequence; its fp16 copy in shared memory is the B operand of [W; Q~] S.
 // Records arrive by bulk copy into a double buffer.  Per chunk: MMA3 [W; Q~] S
 // -> R3, U = U0 - W S (fp16), then MMA4 [*; P] U onto R3 and MMA5 K^^T U onto
@@ -101,7 +101,8 @@ template <int DK, int DV, int NS>
 __global__ void __launch_bounds__(256, 1)
 inter_chunk_fwd_tc_kernel(const float* __restrict__ initial_state, float* __restrict__ final_state,
                           __nv_bfloat16* __restrict__ o, ChunkMap map, WsHeader* hdr,
-                          const unsigned char* __restrict__ records, int H, size_t max_chunks, float scale)
+                          const unsigned char* __restrict__ records, int H, size_t max_chunks, float scale,
+                          const int* __restrict__ seq_order)
 {
     using Sm = K2fSmem<DK, DV, NS>;
     using R = TcRec<DK, DV>;
@@ -113,7 +114,11 @@ inter_chunk_fwd_tc_kernel(const float* __restrict__ initial_state, float* __rest
     __shared__ uint32_t s_tmem;
 
     if (hdr->status != kStatusOk) return;
-    const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * NS;
+    // CTAs are started in blockIdx order: all slices of one (sequence, head)
+    // pair, pairs sequence by sequence, sequences longest first (seq_order)
+    constexpr int NZ = DV / NS;
+    const int pair = (int)blockIdx.x / NZ, si = pair / H;
+    const int s = seq_order ? seq_order[si] : si, h = pair - si * H, j0 = ((int)blockIdx.x - pair * NZ) * NS;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int lane_row = (warp & 3) * 32 + (tid & 31);   // TMEM lane = MMA row
     const int wg = warp >> 2;                            // warpgroup: columns [CPT wg, CPT wg + CPT)
@@ -358,10 +363,11 @@ cudaError_t launch_inter_fwd_tc_ns(const ChunkArgs& a) {
     const int smem = (int)K2fSmem<DK, DV, NS>::END + 1024;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)a.num_seqs, (unsigned)a.H, (unsigned)(DV / NS));
+    const unsigned grid = (unsigned)((size_t)a.num_seqs * a.H * (DV / NS));
     kern<<<grid, 256, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<__nv_bfloat16*>(a.o), map,
                                         static_cast<WsHeader*>(a.ws_header),
-                                        static_cast<const unsigned char*>(a.records), a.H, a.max_chunks, a.scale);
+                                        static_cast<const unsigned char*>(a.records), a.H, a.max_chunks, a.scale,
+                                        a.seq_order);
     return cudaGetLastError();
 }
 

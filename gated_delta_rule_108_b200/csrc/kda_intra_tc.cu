@@ -925,9 +925,11 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-// Packed sequences ordered longest first (ties by index) for the fused form's
-// pair queue: order[rank(s)] = s.  One block; beyond 16384 sequences the order
-// is left as given.
+// Packed sequences ordered longest first (ties by index), the order in which the
+// forward's per-sequence CTAs are started (the fused pass's pair queue, the
+// inter-chunk kernel's grid), so that the longest chains do not start last:
+// order[rank(s)] = s.  One block; beyond 16384 sequences the order is left as
+// given.
 __global__ void __launch_bounds__(1024)
 seq_order_kernel(const WsHeader* hdr, const int32_t* __restrict__ cu, int N, int* __restrict__ order)
 {
@@ -973,17 +975,8 @@ cudaError_t launch_intra_fwd_tc_t(const ChunkArgs& a) {
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     unsigned grid;
-    const int* order = nullptr;
+    const int* order = a.seq_order;   // pairs claimed longest first (null: in order)
     if constexpr (FUSED) {
-        // the pair queue: packed sequences longest first, in the records region
-        // (unused by this form; the caller checked it holds N ints)
-        if (a.cu_seqlens && a.num_seqs > 1) {
-            int* ord = static_cast<int*>(a.records);
-            seq_order_kernel<<<1, 1024, 0, a.stream>>>(static_cast<WsHeader*>(a.ws_header), a.cu_seqlens,
-                                                       a.num_seqs, ord);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            order = ord;
-        }
         const size_t pairs = (size_t)a.num_seqs * a.H;
         grid = (unsigned)(pairs < (size_t)sms ? pairs : (size_t)sms);   // one resident per SM
         if (grid == 0) return cudaSuccess;
@@ -1009,6 +1002,13 @@ cudaError_t launch_chunk_intra_fwd_tc(const ChunkArgs& a) {
     if (a.dk == 64 && a.dv == 128) return launch_intra_fwd_tc_t<64, 128, false>(a);
     if (a.dk == 64 && a.dv == 64) return launch_intra_fwd_tc_t<64, 64, false>(a);
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_chunk_seq_order(const ChunkArgs& a) {
+    if (!a.seq_order || !a.cu_seqlens || a.num_seqs <= 1) return cudaSuccess;
+    seq_order_kernel<<<1, 1024, 0, a.stream>>>(static_cast<WsHeader*>(a.ws_header), a.cu_seqlens, a.num_seqs,
+                                               a.seq_order);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_fused_tc(const ChunkArgs& a) {

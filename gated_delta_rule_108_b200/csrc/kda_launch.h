@@ -33,6 +33,7 @@ struct ChunkArgs {
     // workspace carve-up (computed by the ABI layer)
     void* ws_header;              // WsHeader
     int32_t* chunk_offsets;       // [N+1], varlen only
+    int32_t* seq_order;           // [N] packed sequences longest first (bf16 forward, N > 1), else null
     void* records;                // per (head, chunk) intermediates
     size_t max_chunks;            // chunks per head the records can hold
     int fixed_chunks_per_seq;     // ceil(T / 64) for fixed length
@@ -76,6 +77,7 @@ cudaError_t launch_chunk_intra_fwd_tc(const ChunkArgs& a); // its forward-only f
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K2
 cudaError_t launch_chunk_inter_fwd_tc(const ChunkArgs& a); // its forward-only form, slice width per call
 cudaError_t launch_chunk_fused_tc(const ChunkArgs& a);     // bf16 forward in one pass, one CTA per (sequence, head)
+cudaError_t launch_chunk_seq_order(const ChunkArgs& a);    // packed sequences longest first into a.seq_order
 cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a);  // backward: serial over chunks, reversed
 cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a); // the same on the tensor cores (bf16 inputs)
 cudaError_t launch_chunk_bwd_vside_tc(const ChunkArgs& a); // backward products over the value dim (bf16 inputs)
