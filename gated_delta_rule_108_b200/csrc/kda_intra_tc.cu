@@ -48,44 +48,57 @@ using namespace ptx;
 template <int DK, int DV, bool FUSED>
 struct K1fSmem {
     static constexpr uint32_t TILE = 8192;
-    static constexpr uint32_t KT = 0;                                   // k (bf16) -> K~ (fp16, MMA2 B)
+    // T diag(beta), rows 0..63: MMA2's 128-row A operand, whose unused rows
+    // 64..127 are the first 8 KB of KT right behind it
+    static constexpr uint32_t TPV = 0;
+    static constexpr uint32_t KT = TPV + TILE;                          // k (bf16) -> K~ (fp16, MMA2 B)
     static constexpr uint32_t KT_BYTES = (DK / 64) * TILE;
-    static constexpr uint32_t QT = KT + KT_BYTES;                       // q -> Q~ (fp16) -> v -> V (fp16, MMA2 B)
-    static constexpr uint32_t QT_BYTES = ((DK > DV ? DK : DV) / 64) * TILE;
+    static constexpr uint32_t QT = KT + KT_BYTES;                       // q -> Q~ (fp16); the next item's q
+    static constexpr uint32_t QT_BYTES = (DK / 64) * TILE;
     static constexpr uint32_t G = QT + QT_BYTES;                        // log_alpha -> g (fp32, 32-channel tiles)
     static constexpr uint32_t G_BYTES = 64 * DK * 4;
+    static constexpr uint32_t VT = G;                                   // after the element pass: v -> V (MMA2 B)
+    static constexpr uint32_t VB = (DV / 64) * TILE;
     static constexpr uint32_t OPB = G + G_BYTES;                        // K-m tf32 (MMA1 B); W | U0 fp16 staging
     static constexpr uint32_t OPB_BYTES = (DK / 32) * TILE;
     static constexpr uint32_t STG_BYTES = ((DK + DV) / 64) * TILE;
-    // after MMA1, from G on: T diag(beta) fp16 as MMA2's 128-row A operand
-    // (rows 64..127 never used); the fp16 operands of the blocked (I + A)^{-1}
-    // (A masked to its level-1 blocks and to its level-2 quadrant, the diagonal
-    // inverses D, a product X, and T restricted to its 32 x 32 diagonal blocks);
-    // A's four diagonal 16 x 16 blocks in fp32 (padded).  Each 64 x 64 fp16 tile
-    // is read as a 128-row operand whose rows 64..127 are the next 8 KB.  The
-    // strong-decay path writes the full fp32 A ([64][68]) before the element
-    // pass, while g is live, at G + 32 KB (>= OPB).
-    static constexpr uint32_t TP = G;
-    static constexpr uint32_t AH1 = G + 16384;
-    static constexpr uint32_t AH2 = G + 24576;
-    static constexpr uint32_t DH = G + 32768;
-    static constexpr uint32_t XH = G + 40960;
-    static constexpr uint32_t T1H = G + 49152;
-    static constexpr uint32_t AMD = G + 57344;                         // 4 x (16 x 16 + 4) fp32
-    static constexpr uint32_t AMS = G + 32768;                         // strong path: [64][68] fp32
+    // after MMA1, behind V: the fp16 operands of the blocked (I + A)^{-1} (A
+    // masked to its level-1 blocks and to its level-2 quadrant, the diagonal
+    // inverses D, a product X, T restricted to its 32 x 32 diagonal blocks),
+    // each 64 x 64 tile read as a 128-row operand whose rows 64..127 are the
+    // next 8 KB; then A's four diagonal 16 x 16 blocks in fp32 (padded).  The
+    // strong-decay path writes the full fp32 A ([64][64]) before the element
+    // pass, while g is live, outside G and clear of AH1, AH2 and AMD.
+    static constexpr uint32_t SCR = G + VB;
+    static constexpr uint32_t AH1 = SCR;
+    static constexpr uint32_t AH2 = SCR + 8192;
+    static constexpr uint32_t DH = SCR + 16384;
+    static constexpr uint32_t XH = SCR + 24576;
+    static constexpr uint32_t T1H = SCR + 32768;
+    static constexpr uint32_t AMD = SCR + 40960;                        // 4 x (16 x 16 + 4) fp32
+    static constexpr uint32_t AMD_END = AMD + 4 * 260 * 4;
+    static constexpr uint32_t AMS0 = (G + G_BYTES) > (AH2 + 8192) ? (G + G_BYTES) : (AH2 + 8192);
+    static constexpr uint32_t AMS = AMS0 + 64 * 64 * 4 <= AMD ? AMS0 : (AMD_END + 15) / 16 * 16;   // [64][64]
+    // log-decay boxes (32 channels, 8 KB) past V overlap only AH1, AH2 and DH,
+    // which are dead once the second blocked-inverse level has read AH2: the
+    // next item's boxes there are fetched then, the others after MMA2
+    static constexpr int LA_EARLY_BOX = (int)(VB / TILE);
     static constexpr uint32_t E0 = OPB + (OPB_BYTES > STG_BYTES ? OPB_BYTES : STG_BYTES);
-    static constexpr uint32_t E1 = G + 65536;                          // T1H's rows 64..127 end here
-    static constexpr uint32_t E2 = AMS + 64 * 68 * 4;
-    static constexpr uint32_t END0 = E0 > E1 ? (E0 > E2 ? E0 : E2) : (E1 > E2 ? E1 : E2);
+    static constexpr uint32_t E1 = T1H + 16384;                          // T1H's rows 64..127 end here
+    static constexpr uint32_t E2 = AMS + 64 * 64 * 4;
+    static constexpr uint32_t E3 = AMD_END;
+    static constexpr uint32_t E01 = E0 > E1 ? E0 : E1;
+    static constexpr uint32_t E23 = E2 > E3 ? E2 : E3;
+    static constexpr uint32_t END0 = ((E01 > E23 ? E01 : E23) + 1023) / 1024 * 1024;
     // fused form only: the chunk's operands of the state step, kept on chip ---
-    // [W; Q~] as 128-row K-major tiles per 64 key channels, U0, K^ and P (P
+    // [W; Q~] as 128-row K-major tiles per 64 key channels, K^ and P (P
     // directly after K^, so the 128-row operand [*; P] reads K^'s tail as its
-    // unused rows 0..63), gamma_C, and the fp16 state (rows = key channel) and
-    // U operands of the state step
+    // unused rows 0..63), gamma_C, the fp16 state (rows = key channel) and U
+    // operands of the state step; U0 where K-m was
     static constexpr int NTV = DV > 64 ? DV / 64 : 1;
     static constexpr uint32_t FWQ = END0;
-    static constexpr uint32_t FU0 = FWQ + (DK / 64) * 16384;
-    static constexpr uint32_t FKH = FU0 + (DV / 64) * TILE;
+    static constexpr uint32_t FU0 = OPB;   // written after MMA2, when OPB (K-m, the solve's scratch) is dead
+    static constexpr uint32_t FKH = FWQ + (DK / 64) * 16384;
     static constexpr uint32_t FP = FKH + (DK / 64) * TILE;
     static constexpr uint32_t S16 = FP + TILE;
     static constexpr uint32_t U16 = S16 + NTV * 16384;
@@ -104,12 +117,15 @@ struct K1fSmem {
     static constexpr uint32_t KQ_TX = 2 * (DK / 64) * TILE;              // k and q tiles
     static constexpr uint32_t LA_TX = 64 * DK * 4;
     static constexpr uint32_t V_TX = (DV / 64) * TILE;
-    static_assert(TP % 1024 == 0 && OPB % 1024 == 0 && G % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-    static_assert(AMS >= G + G_BYTES, "the strong path's A lies outside the live log-decay tile");
-    static_assert(AMD + 4 * 260 * 4 <= T1H + 16384 && AMS + 64 * 68 * 4 <= AMD, "T-solve scratch");
+    static_assert(KT == TPV + 8192 && TPV % 1024 == 0 && OPB % 1024 == 0 && G % 1024 == 0 && SCR % 1024 == 0,
+                  "swizzled tiles need 1024-byte alignment; MMA2's A operand runs into KT");
+    static_assert(AMS >= G + G_BYTES && AMS >= AH2 + 8192 && (AMS + 64 * 64 * 4 <= AMD || AMS >= AMD_END),
+                  "the strong path's A lies outside the live log-decay tile and the converted operands");
+    static_assert(G + G_BYTES <= SCR + 24576, "early log-decay boxes overlap only AH1, AH2, DH");
     // two CTAs per SM (228 KB per SM, 1 KB reserved per CTA); the fused form one
     static_assert(FUSED ? TOTAL <= 232448 : 2 * (TOTAL + 1024) <= 233472, "CTAs per SM");
     static_assert(FWQ % 1024 == 0 && S16 % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+    static_assert((DV / 64) * TILE <= OPB_BYTES, "the fused U0 fits where K-m was");
 };
 
 // g (base 2) of token r, channel c in the 128-byte-swizzled log-decay tiles
@@ -185,21 +201,37 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
     // its last if it has fewer), so that the bounded wait on that item's
     // inputs gives up with earlier phases consumed
     const int drop_it = (!FUSED && drop_la && blockIdx.x == 0) ? min(2, (total - 1) / (int)gridDim.x) : -1;
-    auto issue_in = [&](int c, int h, int j) {   // k, q (and log_alpha) of chunk c, head h: this CTA's j-th item
-        int seq, tok0, L;
-        map.locate(c, seq, tok0, L);
+    // An item's inputs arrive in three parts as their buffers free up: q (QT is
+    // free once the previous item's Q~ has left it), the log-decay boxes past V
+    // (free after the second blocked-inverse level), then k and the other boxes
+    // (after MMA2).  All land on bar_in, armed with the whole byte count by the
+    // first part.  (h, tok0): the item's head and first token; j: this CTA's
+    // item count at that item.
+    auto issue_q = [&](int h, int tok0) {
         mbar_arrive_expect_tx(&bar_in, Sm::KQ_TX + (channel_gate ? Sm::LA_TX : 0u));
 #pragma unroll
-        for (int b = 0; b < DK / 64; ++b) {
-            tma_load_3d(sm + Sm::KT + b * Sm::TILE, &tm_k, &bar_in, b * 64, h, tok0);
-            tma_load_3d(sm + Sm::QT + b * Sm::TILE, &tm_q, &bar_in, b * 64, h, tok0);
-        }
+        for (int b = 0; b < DK / 64; ++b) tma_load_3d(sm + Sm::QT + b * Sm::TILE, &tm_q, &bar_in, b * 64, h, tok0);
+    };
+    auto issue_la = [&](int h, int tok0, int j, bool early) {
         if constexpr (channel_gate) {
-            if (j != drop_it) {
+            if (j == drop_it) return;   // test hook: this item's log-decay copy is left out
 #pragma unroll
-                for (int b = 0; b < DK / 32; ++b) tma_load_3d(sm + Sm::G + b * Sm::TILE, &tm_la, &bar_in, b * 32, h, tok0);
-            }
+            for (int b = 0; b < DK / 32; ++b)
+                if ((b >= Sm::LA_EARLY_BOX) == early)
+                    tma_load_3d(sm + Sm::G + b * Sm::TILE, &tm_la, &bar_in, b * 32, h, tok0);
         }
+    };
+    auto issue_k = [&](int h, int tok0) {
+#pragma unroll
+        for (int b = 0; b < DK / 64; ++b) tma_load_3d(sm + Sm::KT + b * Sm::TILE, &tm_k, &bar_in, b * 64, h, tok0);
+    };
+    auto issue_in = [&](int c, int h, int j) {   // all of chunk c, head h at once
+        int seq, tok0, L;
+        map.locate(c, seq, tok0, L);
+        issue_q(h, tok0);
+        issue_la(h, tok0, j, true);
+        issue_la(h, tok0, j, false);
+        issue_k(h, tok0);
     };
     // beta (and a per-head log-decay) of item w into registers, threads 192..255
     float beta_next = 0.f, lah_next = 0.f;
@@ -238,6 +270,11 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             if constexpr (GATE == kGateHead) s_lah[tid - 192] = lah_next;
         }
         if (nc >= 0) load_beta(nc, nh);
+        int ntok0 = 0;   // the next item's first token (copy thread)
+        if (tid == kCopyThread && nc >= 0) {
+            int sq, nl;
+            map.locate(nc, sq, ntok0, nl);
+        }
         // the previous item's W / U0 staging (OPB) must be read before it is reused
         if (tid == kCopyThread && stored) bulk_store_wait_read();
 
@@ -279,9 +316,9 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         // Strong decay: the factors e^{+-(g - g_m)} of A and P could overflow, so
         // this chunk forms A and P exactly (slow path, no MMA1).
         const bool strong = __syncthreads_or(wide);
-        float* am = reinterpret_cast<float*>(sm + Sm::AMS);   // strong path: [64][68]
+        float* am = reinterpret_cast<float*>(sm + Sm::AMS);   // strong path: [64][64]
         if (strong) {
-            exact_a_p<DK>(gat, sm + Sm::KT, sm + Sm::QT, s_beta, L, am, p_dst);
+            exact_a_p<DK>(gat, sm + Sm::KT, sm + Sm::QT, s_beta, L, am, p_dst, 64);
             __syncthreads();   // the k, q tiles are converted in place next
         }
 
@@ -413,11 +450,14 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                 stored = true;
                 bulk_store_wait_read();
             }
+            // v into the log-decay tile's place (g is dead after the element pass)
             mbar_arrive_expect_tx(&bar_v, Sm::V_TX);
 #pragma unroll
-            for (int b = 0; b < DV / 64; ++b) tma_load_3d(sm + Sm::QT + b * Sm::TILE, &tm_v, &bar_v, b * 64, h, tok0);
+            for (int b = 0; b < DV / 64; ++b) tma_load_3d(sm + Sm::VT + b * Sm::TILE, &tm_v, &bar_v, b * 64, h, tok0);
+            if (nc >= 0) issue_q(nh, ntok0);   // QT is free: the next item's q
         }
         v_issued = it + 1;
+        if (nc >= 0) in_issued = it + 2;
 
         float* amd = reinterpret_cast<float*>(sm + Sm::AMD);  // A's diagonal blocks, [4][16 x 16 + 4]
         // A row `row` (< 64), columns [32 hc, 32 hc + 32), beta-scaled and strictly
@@ -486,7 +526,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         } else if (row < 64) {   // strong decay: the exact A, already beta-scaled and masked
             float v[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = am[row * 68 + 32 * hc + i];
+            for (int i = 0; i < 32; ++i) v[i] = am[row * 64 + 32 * hc + i];
             put_a_row(v);
         }
         __syncthreads();
@@ -495,10 +535,10 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         //      diagonal 16 x 16 blocks on CUDA cores, then the off-diagonal blocks on
         //      the tensor cores by doubling the solved block (fp16 operands, fp32
         //      accumulation):  T21 = -T22 A21 T11,  first for 16 -> 32 rows (the
-        //      pairs (1,0), (3,2)), then 32 -> 64.  T diag(beta) goes to TP in fp16
+        //      pairs (1,0), (3,2)), then 32 -> 64.  T diag(beta) goes to TPV in fp16
         //      (K-major, rows 0..63) block by block.
         auto put_t = [&](int rr, int col, float t) {
-            *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(rr, col * 2)) = __float2half_rn(t * s_beta[col]);
+            *reinterpret_cast<__half*>(sm + Sm::TPV + sw128_offset(rr, col * 2)) = __float2half_rn(t * s_beta[col]);
         };
         if (tid < 64) {    // diagonal blocks, one column per thread
             const int b = tid >> 4, cc = tid & 15, base = 16 * b;
@@ -523,7 +563,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             for (int o = tid - 64; o < 64 * 8; o += 192) {
                 const int rr = o >> 3, c16 = o & 7, blk = c16 >> 1, rb = rr >> 4;
                 if (blk != rb) *reinterpret_cast<uint4*>(sm + Sm::DH + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
-                if (blk > rb) *reinterpret_cast<uint4*>(sm + Sm::TP + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
+                if (blk > rb) *reinterpret_cast<uint4*>(sm + Sm::TPV + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
         // one 64 x 64 x 64 product D[0, 64) = A(128-row K-major operand) B(64 x 64, rows = K)
@@ -585,13 +625,15 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                         tb[e] = __float2half_rn(-v[8 * i8 + e] * s_beta[col + e]);
                     }
                     d = *reinterpret_cast<const uint4*>(t1);
-                    *reinterpret_cast<uint4*>(sm + Sm::TP + off) = *reinterpret_cast<const uint4*>(tb);
+                    *reinterpret_cast<uint4*>(sm + Sm::TPV + off) = *reinterpret_cast<const uint4*>(tb);
                 }
                 *reinterpret_cast<uint4*>(sm + Sm::T1H + off) = d;
             }
         }
         // level 2: X = A_L2 T1, Y = T1 X; T[32:64, 0:32] = -Y[32:64, 0:32]
         if (!level_mma(Sm::AH2, Sm::T1H)) return false;
+        // AH1, AH2 and DH are dead: the next item's log-decay boxes past V come in
+        if (tid == kCopyThread && nc >= 0) issue_la(nh, ntok0, it + 1, true);
         store_x(Sm::XH);
         if (!level_mma(Sm::T1H, Sm::XH)) return false;
         if (row >= 32 && row < 64 && hc == 0) {
@@ -602,17 +644,17 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                 __align__(16) __half tb[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) tb[e] = __float2half_rn(-v[8 * i8 + e] * s_beta[8 * i8 + e]);
-                *reinterpret_cast<uint4*>(sm + Sm::TP + sw128_offset(row, 16 * i8)) = *reinterpret_cast<const uint4*>(tb);
+                *reinterpret_cast<uint4*>(sm + Sm::TPV + sw128_offset(row, 16 * i8)) = *reinterpret_cast<const uint4*>(tb);
             }
         }
 
-        // ---- v: bf16 -> fp16 in place in QT, 8 values per thread and step
+        // ---- v: bf16 -> fp16 in place in VT, 8 values per thread and step
         ok = (!FUSED && tid != 0) || mbar_wait_cycles(&bar_v, it & 1, wait_cap);
         if (__syncthreads_or(!ok)) return false;
         v_done = it + 1;
         for (int item = tid; item < kChunk * (DV / 8); item += 256) {
             const int r = item / (DV / 8), j8 = (item - r * (DV / 8)) * 8;
-            const uint32_t o = Sm::QT + (j8 >> 6) * Sm::TILE + sw128_offset(r, (j8 & 63) * 2);
+            const uint32_t o = Sm::VT + (j8 >> 6) * Sm::TILE + sw128_offset(r, (j8 & 63) * 2);
             uint4 raw = *reinterpret_cast<const uint4*>(sm + o);
             if (r >= L) raw = make_uint4(0, 0, 0, 0);
             const __nv_bfloat162* vb = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -630,11 +672,12 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         __syncthreads();
 
         // ---- MMA2 (fp16): [T diag(beta); *] K~ -> D2[0, DK), [T diag(beta); *] V -> D2[DK, DK + DV)
+        //      (the operand's rows 64..127 are KT's first 8 KB; their products are never read)
         if (tid == 0) {
             tc_fence_after();
             constexpr uint32_t idw = instr_desc(kFmtF16, 128, DK, false, true);
             constexpr uint32_t idu = instr_desc(kFmtF16, 128, DV, false, true);
-            const uint32_t a0 = smem_u32(sm + Sm::TP), bk = smem_u32(sm + Sm::KT), bv = smem_u32(sm + Sm::QT);
+            const uint32_t a0 = smem_u32(sm + Sm::TPV), bk = smem_u32(sm + Sm::KT), bv = smem_u32(sm + Sm::VT);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_f16(D2, smem_desc(a0 + ks * 32, 16, 1024, kLayoutSW128),
@@ -651,9 +694,11 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         mma_phase ^= 1;
         mma_pending = 0;
         tc_fence_after();
-        // KT, QT and G are free: the next item's inputs come in behind the write-out
-        if (tid == kCopyThread && nc >= 0) issue_in(nc, nh, it + 1);
-        if (nc >= 0) in_issued = it + 2;
+        // KT and V are free: the rest of the next item's inputs come in behind the write-out
+        if (tid == kCopyThread && nc >= 0) {
+            issue_k(nh, ntok0);
+            issue_la(nh, ntok0, it + 1, false);
+        }
 
         // ---- W and U0 (rows 0..63): fp16 into the OPB staging tiles (record
         //      layout), then one bulk store per tile; warps 0, 1, 4, 5 (TMEM

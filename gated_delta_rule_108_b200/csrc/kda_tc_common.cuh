@@ -75,13 +75,14 @@ constexpr int kTileThread = 128;    // its backward-mode tile stores (warp 4, id
 
 // Exact A and P of one chunk, used when its decay is too strong for the split
 // factors (g in base 2, read through gat(token, channel)): A_ri = beta_r sum_c
-// k_rc k_ic e^{g_rc - g_ic} (i < r) into am [64][68] (zero on and above the
+// k_rc k_ic e^{g_rc - g_ic} (i < r) into am [64][lda] (zero on and above the
 // diagonal) and P_ri = sum_c q_rc k_ic e^{g_rc - g_ic} (i <= r) as fp16 into the
 // record's P tile.  Every exponent is <= 0.  One warp per (r, i) pair, lanes
 // over channels; k and q are the bf16 tiles as loaded.
 template <int DK, class GAt>
 __device__ __forceinline__ void exact_a_p(GAt gat, const unsigned char* ks, const unsigned char* qs,
-                                          const float* s_beta, int L, float* am, unsigned char* prec)
+                                          const float* s_beta, int L, float* am, unsigned char* prec,
+                                          int lda = 68)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int pr = warp; pr < 64 * 64; pr += 8) {
@@ -107,7 +108,7 @@ __device__ __forceinline__ void exact_a_p(GAt gat, const unsigned char* ks, cons
             }
         }
         if (lane == 0) {
-            am[r * 68 + i] = (i < r) ? s_beta[r] * sa : 0.f;
+            am[r * lda + i] = (i < r) ? s_beta[r] * sa : 0.f;
             *reinterpret_cast<__half*>(prec + sw128_offset(r, i * 2)) = __float2half_rn(sp);
         }
     }
