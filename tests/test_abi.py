@@ -171,3 +171,25 @@ def test_debug_drop_copy_arms_and_disarms(lib):
     assert lib.kda_debug_drop_copy(-1) == 1
     assert lib.kda_debug_drop_copy(1000) == 0
     assert lib.kda_debug_drop_copy(0) == 0
+
+
+def test_saved_forward_entry_points_validate(lib):
+    """kda_chunk_fwd_save needs the backward-sized workspace; kda_chunk_bwd_saved
+    validates like kda_chunk_bwd.  (Every case fails before any launch.)"""
+    p = 1 << 20
+    f32 = 0
+    fwd_bytes = lib.kda_chunk_fwd_workspace_size(1, 64, 1, 64, 64, 1, 0, f32)
+    bwd_bytes = lib.kda_chunk_bwd_workspace_size(1, 64, 1, 64, 64, 1, 0, f32)
+    assert bwd_bytes > fwd_bytes
+    f = lib.kda_chunk_fwd_save
+    # a forward-sized workspace is too small to keep what the backward needs
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 64, 64, 1, f32, 0, p, None, p, fwd_bytes, None) == 5
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 64, 64, 1, f32, 0, p, None, None, 0, None) == 5
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 64, 64, 1, f32, 9, p, None, p, bwd_bytes, None) == 1
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 96, 64, 1, f32, 0, p, None, p, bwd_bytes, None) == 2
+    b = lib.kda_chunk_bwd_saved
+    # null cotangent; workspace too small
+    assert b(p, p, p, p, p, None, None, None, None, 1, 64, 1, 64, 64, 1, f32, 0,
+             p, p, p, p, p, None, p, bwd_bytes, None) == 1
+    assert b(p, p, p, p, p, None, None, p, None, 1, 64, 1, 64, 64, 1, f32, 0,
+             p, p, p, p, p, None, p, 16, None) == 5
