@@ -274,6 +274,44 @@ def bench_backward(args, dev, world, rank):
     return dict(w=w, ms_per_step=ms, stages=stages, launches=(7 if w.dtype == torch.bfloat16 else 5) * steps)
 
 
+def bench_train(args, dev, world, rank):
+    """One training step on the forward's workload: kda_chunk_fwd_save, then
+    kda_chunk_bwd_saved on what it kept (no forward recomputation)."""
+    from gated_delta_rule_108_b200 import inputs as I
+    from gated_delta_rule_108_b200 import kda
+
+    w = I.workload(args.workload)
+    wr = I.ChunkWorkload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+    x = I.chunk_inputs(wr)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    gen = torch.Generator().manual_seed(6000 + rank)
+    d_o = torch.randn(w.B, w.T, w.H, w.dv, generator=gen).to(w.dtype).to(dev)
+    dSf = torch.randn(w.B, w.H, w.dk, w.dv, generator=gen).to(dev)
+
+    def step():
+        _, _, saved = kda.chunk_fwd_train(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], g["initial_state"])
+        kda.chunk_bwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], d_o, g["initial_state"], dSf,
+                      saved=saved)
+        return saved
+
+    for _ in range(args.warmup):
+        saved = step()
+    torch.cuda.synchronize()
+    if kda.workspace_status(saved) != 0:
+        raise RuntimeError("device status set after the training-step warm-up")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(args.bwd_steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end), world, dev) / args.bwd_steps
+    return dict(w=w, ms_per_step=ms)
+
+
 def bench_decode(args, dev, world, rank):
     from gated_delta_rule_108_b200 import inputs as I
     from gated_delta_rule_108_b200 import kda
@@ -375,6 +413,7 @@ def run_ours(args):
     res = bench_chunk(args, dev, world, rank)
     dec = None if args.no_decode else bench_decode(args, dev, world, rank)
     bwd = None if args.no_bwd else bench_backward(args, dev, world, rank)
+    train = None if (args.no_bwd or args.no_train) else bench_train(args, dev, world, rank)
     clk = clocks.stop()
     e2e = None if args.no_e2e else bench_e2e(args, dev, world, res)
 
@@ -473,6 +512,14 @@ def run_ours(args):
                          "algorithmic_bytes_per_launch": vbytes, "ms_per_launch": vms},
             "strong_decay_chunks_ms": bwd["stages"]["bwd_intra_chunk"],
         }
+    if train is not None:
+        tw = train["w"]
+        line["train_step"] = {
+            "workload": f"{tw.name}: kda_chunk_fwd_save then kda_chunk_bwd_saved (forward kept for the "
+                        f"backward), B={tw.B}, T={tw.T}, H={tw.H}, d_k=d_v={tw.dk}, bf16 q/k/v/d_o",
+            "value": tw.tokens * world / (train["ms_per_step"] / 1e3), "unit": "tokens/s",
+            "ms_per_step": train["ms_per_step"], "steps": args.bwd_steps,
+        }
     if e2e is not None:
         ms_e, h2d, d2h = e2e
         line["e2e"] = {"value": res["tokens"] * world / (ms_e / 1e3), "unit": "tokens/s",
@@ -543,6 +590,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward (kda_chunk_bwd) measurement")
     ap.add_argument("--bwd-steps", type=int, default=10)
+    ap.add_argument("--no-train", action="store_true", help="skip the training-step (saved forward) measurement")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
