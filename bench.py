@@ -415,12 +415,59 @@ def bench_backward(args, dev, world, rank, peaks, peak_kind):
                     "fp32 accumulation), strong-decay chunks on CUDA cores in fp32",
         "value": w.tokens * world / (ms / 1e3), "unit": "tokens/s",
         "ms_per_step": ms, "steps": steps, "kernels_ms": stages,
-        "gpu_launches": (7 if w.dtype == torch.bfloat16 else 5) * steps,
+        "gpu_launches": (8 if w.dtype == torch.bfloat16 else 5) * steps,
         "roofline": {"kernel": "bwd_vside_tc + bwd_tchain_tc + bwd_split_tc (the dominant stage)",
                      "bound": "hbm", "achieved": vgbs, "peak": hbm, "unit": "GB/s", "frac": vgbs / hbm,
                      "traffic": None if tpu is None else tpu * units, "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": vbytes, "ms_per_launch": vms},
         "strong_decay_chunks_ms": stages["bwd_intra_chunk"],
+    }
+
+
+def bench_train(args, dev, world, rank):
+    """One training step on the backward's workload: kda_chunk_fwd_save (the
+    forward that keeps T, the tiles and the chunk-start states), then
+    kda_chunk_bwd_saved on what it kept, so the backward recomputes nothing."""
+    from gated_delta_rule_108_b200 import inputs as I
+    from gated_delta_rule_108_b200 import kda
+
+    w = I.workload(args.bwd_workload)
+    x = I.chunk_inputs(rank_workload(w, rank))
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    gen = torch.Generator().manual_seed(6000 + rank)
+    d_o = torch.randn(w.B, w.T, w.H, w.dv, generator=gen).to(w.dtype).to(dev)
+    dSf = torch.randn(w.num_seqs, w.H, w.dk, w.dv, generator=gen).to(dev)
+
+    def step():
+        _, _, saved = kda.chunk_fwd_train(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"],
+                                          g["initial_state"], g["cu_seqlens"])
+        kda.chunk_bwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], d_o, g["initial_state"], dSf,
+                      g["cu_seqlens"], saved=saved)
+        return saved
+
+    saved = None
+    for _ in range(args.warmup):
+        saved = step()
+    torch.cuda.synchronize()
+    if saved is not None and kda.workspace_status(saved) != 0:
+        raise RuntimeError("device status set after the training-step warm-up")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(args.bwd_steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end), world, dev) / args.bwd_steps
+    launches = 3 + (5 if w.dtype == torch.bfloat16 else 2)   # prep, K1, K2; the backward without its recompute
+    return {
+        "workload": f"{w.name}: kda_chunk_fwd_save then kda_chunk_bwd_saved (what the forward keeps "
+                    f"feeds the backward; nothing recomputed), B={w.B}, T={w.T}, H={w.H}, d_k=d_v={w.dk}, "
+                    "bf16 q/k/v/d_o",
+        "value": w.tokens * world / (ms / 1e3), "unit": "tokens/s",
+        "ms_per_step": ms, "steps": args.bwd_steps, "gpu_launches": launches * args.bwd_steps,
     }
 
 
@@ -573,6 +620,7 @@ def run_ours(args):
         torch.cuda.empty_cache()
     dec = None if args.no_decode else bench_decode(args, dev, world, rank, peaks, peak_kind)
     bwd = None if args.no_bwd else bench_backward(args, dev, world, rank, peaks, peak_kind)
+    train = None if (args.no_bwd or args.no_train) else bench_train(args, dev, world, rank)
     clk = clocks.stop()
     e2e = None if args.no_e2e else bench_e2e(args, dev, world, head)
 
@@ -614,6 +662,8 @@ def run_ours(args):
         line["decode"] = dec
     if bwd is not None:
         line["chunk_bwd"] = bwd
+    if train is not None:
+        line["train_step"] = train
     if e2e is not None:
         ms_e, h2d, d2h = e2e
         line["e2e"] = {"value": w.tokens * world / (ms_e / 1e3), "unit": "tokens/s",
@@ -710,6 +760,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward (kda_chunk_bwd) measurement")
     ap.add_argument("--bwd-steps", type=int, default=10)
+    ap.add_argument("--no-train", action="store_true", help="skip the training-step (saved forward) measurement")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--check-launch", action="store_true",

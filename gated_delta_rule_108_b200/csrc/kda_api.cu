@@ -175,11 +175,13 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
     return L.total;
 }
 
+// save: the workspace has the backward's layout, and the forward kernels run in
+// backward mode, so that it also holds what kda_chunk_bwd would recompute.
 static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const float* log_alpha,
                                  const float* beta, const float* initial_state, const int32_t* cu_seqlens,
                                  int B, int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype,
                                  kda_gate gate, void* o, float* final_state, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
+                                 size_t workspace_bytes, void* stream, bool save = false) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
     if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE)
         return fail(KDA_ERR_INVALID_ARG, "unknown gate kind %d", (int)gate);
@@ -210,16 +212,19 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
         if (a0 < b0 + bytes && b0 < a0 + bytes)
             return fail(KDA_ERR_INVALID_ARG, "initial_state and final_state overlap without being equal");
     }
-    WsLayout L;
-    if (!ws_layout(B, T, H, dk, dv, num_seqs, varlen, dtype, L))
+    BwdLayout LB;
+    if (!bwd_layout(B, T, H, dk, dv, num_seqs, varlen, dtype, LB))
         return fail(KDA_ERR_INVALID_ARG, "invalid sizes for the workspace layout");
-    if (!workspace) return fail(KDA_ERR_WORKSPACE, "workspace is null (need %zu bytes)", L.total);
+    const WsLayout& L = LB.base;   // the backward layout starts with the forward's
+    const size_t need = save ? LB.total : L.total;
+    if (!workspace) return fail(KDA_ERR_WORKSPACE, "workspace is null (need %zu bytes)", need);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(KDA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-    const int fused = chunk_fwd_fused(N, varlen, dtype, L, workspace_bytes);
-    if (workspace_bytes < L.total && !fused)
-        return fail(KDA_ERR_WORKSPACE, "workspace has %zu bytes, need %zu%s", workspace_bytes, L.total,
-                    dtype == KDA_BF16 ? " (or the fused pass's kda_chunk_fwd_fused_workspace_size)" : "");
+    // a training forward (save) runs the two-kernel form in backward mode
+    const int fused = save ? 0 : chunk_fwd_fused(N, varlen, dtype, L, workspace_bytes);
+    if (workspace_bytes < need && !fused)
+        return fail(KDA_ERR_WORKSPACE, "workspace has %zu bytes, need %zu%s", workspace_bytes, need,
+                    dtype == KDA_BF16 && !save ? " (or the fused pass's kda_chunk_fwd_fused_workspace_size)" : "");
 
     kda::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
@@ -231,12 +236,19 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
     a.scale = 1.0f / sqrtf((float)dk);
     a.ws_header = workspace;
     a.chunk_offsets = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + L.offsets_off);
-    a.seq_order = (a.bf16 && varlen && N > 1) ? reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + L.order_off)
+    a.seq_order = (a.bf16 && varlen && N > 1 && !save) ? reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + L.order_off)
                                              : nullptr;
     a.records = static_cast<char*>(workspace) + L.records_off;
     a.max_chunks = L.max_chunks;
     a.fixed_chunks_per_seq = L.chunks_per_seq;
     a.stream = static_cast<cudaStream_t>(stream);
+    if (save) {   // backward mode: T (and for bf16 the K~, V tiles, M, strong-decay flags), chunk-start states
+        char* ws = static_cast<char*>(workspace);
+        a.tmat = a.bf16 ? nullptr : reinterpret_cast<float*>(ws + LB.tmat_off);
+        a.bwd_tiles = a.bf16 ? static_cast<void*>(ws + LB.tiles_off) : nullptr;
+        a.bwd_flags = a.bf16 ? reinterpret_cast<int*>(ws + LB.flags_off) : nullptr;
+        a.states = reinterpret_cast<float*>(ws + LB.states_off);
+    }
     if (g_debug_drop_cap > 0 && a.bf16 && gate == KDA_GATE_CHANNEL) {   // one-shot test hook
         a.debug_drop_copy = 1;
         a.wait_cap = g_debug_drop_cap;
@@ -340,7 +352,7 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
                                  const void* d_o, const float* d_final_state, int B, int T, int H, int dk,
                                  int dv, int num_seqs, kda_dtype dtype, kda_gate gate, void* dq, void* dk_out,
                                  void* dv_out, float* dlog_alpha, float* dbeta, float* d_initial_state,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+                                 void* workspace, size_t workspace_bytes, void* stream, bool saved = false) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
     if (gate != KDA_GATE_CHANNEL && gate != KDA_GATE_HEAD && gate != KDA_GATE_NONE)
         return fail(KDA_ERR_INVALID_ARG, "unknown gate kind %d", (int)gate);
@@ -404,16 +416,16 @@ static kda_status chunk_bwd_impl(const void* q, const void* k, const void* v, co
 
     // forward recomputation (the records, T and the chunk-start states: fp16
     // records on the tensor cores for bf16 inputs, fp32 ones on CUDA cores for
-    // fp32 inputs), then the reversed pass over chunks, then the per-chunk
-    // gradients
+    // fp32 inputs) unless kda_chunk_fwd_save left them in this workspace, then
+    // the reversed pass over chunks, then the per-chunk gradients
     const bool marks = g_stage_event_count >= 7;   // the backward records all seven or none
     auto mark = [&](int i) { return marks ? mark_stage(i, a.stream) : cudaSuccess; };
     e = mark(0);
-    if (e == cudaSuccess) e = kda::launch_chunk_prep(a);
+    if (e == cudaSuccess && !saved) e = kda::launch_chunk_prep(a);
     if (e == cudaSuccess) e = mark(1);
-    if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_intra_tc(a) : kda::launch_chunk_intra(a);
+    if (e == cudaSuccess && !saved) e = a.bf16 ? kda::launch_chunk_intra_tc(a) : kda::launch_chunk_intra(a);
     if (e == cudaSuccess) e = mark(2);
-    if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_inter_tc(a) : kda::launch_chunk_inter(a);
+    if (e == cudaSuccess && !saved) e = a.bf16 ? kda::launch_chunk_inter_tc(a) : kda::launch_chunk_inter(a);
     if (e == cudaSuccess) e = mark(3);
     // the reversed chain reads the fp16 tensor-core records (bf16) or the fp32
     // ones; for bf16 the products over the value dimension are formed on the
@@ -470,6 +482,26 @@ size_t kda_chunk_fwd_fused_workspace_size(int B, int T, int H, int dk, int dv, i
     WsLayout L;
     if (dtype != KDA_BF16 || !ws_layout(B, T, H, dk, dv, num_seqs, varlen != 0, dtype, L)) return 0;
     return fused_ws_bytes(varlen ? num_seqs : B, varlen != 0, L);
+}
+
+kda_status kda_chunk_fwd_save(const void* q, const void* k, const void* v, const float* log_alpha,
+                              const float* beta, const float* initial_state, const int32_t* cu_seqlens, int B,
+                              int T, int H, int dk, int dv, int num_seqs, kda_dtype dtype, kda_gate gate,
+                              void* o, float* final_state, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, initial_state, cu_seqlens, B, T, H, dk, dv, num_seqs,
+                          dtype, gate, o, final_state, workspace, workspace_bytes, stream, /*save=*/true);
+}
+
+kda_status kda_chunk_bwd_saved(const void* q, const void* k, const void* v, const float* log_alpha,
+                               const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                               const void* d_o, const float* d_final_state, int B, int T, int H, int dk,
+                               int dv, int num_seqs, kda_dtype dtype, kda_gate gate, void* dq, void* dk_out,
+                               void* dv_out, float* dlog_alpha, float* dbeta, float* d_initial_state,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+    return chunk_bwd_impl(q, k, v, log_alpha, beta, initial_state, cu_seqlens, d_o, d_final_state, B, T, H, dk,
+                          dv, num_seqs, dtype, gate, dq, dk_out, dv_out, dlog_alpha, dbeta, d_initial_state,
+                          workspace, workspace_bytes, stream, /*saved=*/true);
 }
 
 kda_status kda_workspace_status(const void* workspace, size_t workspace_bytes, void* stream) {

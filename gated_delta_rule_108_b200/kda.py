@@ -69,6 +69,12 @@ def _declare(lib):
     lib.kda_chunk_fwd_plan.argtypes = [i, i, i, i, i, i, i, i, sz]
     lib.kda_chunk_fwd_fused_workspace_size.restype = sz
     lib.kda_chunk_fwd_fused_workspace_size.argtypes = [i, i, i, i, i, i, i, i]
+    lib.kda_chunk_fwd_save.restype = i
+    lib.kda_chunk_fwd_save.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
+                                       vp, vp, vp, sz, vp]
+    lib.kda_chunk_bwd_saved.restype = i
+    lib.kda_chunk_bwd_saved.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
+                                        vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.kda_workspace_status.restype = i
     lib.kda_workspace_status.argtypes = [vp, sz, vp]
     lib.kda_set_stage_events.restype = i
@@ -211,8 +217,8 @@ def _gate_of(log_alpha, channel_ndim: int, shape_channel, shape_head, device=Non
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
               output_final_state: bool = True, o=None, final_state=None,
-              workspace=None, stream=None,
-              check: Optional[bool] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              workspace=None, stream=None, check: Optional[bool] = None,
+              _save: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunkwise forward (``kda_chunk_fwd_gated``).
 
     q, k [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H];
@@ -252,17 +258,32 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
         o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
     if final_state is None and output_final_state:
         final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
-    ws_bytes = chunk_fwd_workspace_size(B, T, H, dk, dv, N, cu_seqlens is not None, q.dtype)
+    size_fn = chunk_bwd_workspace_size if _save else chunk_fwd_workspace_size
+    ws_bytes = size_fn(B, T, H, dk, dv, N, cu_seqlens is not None, q.dtype)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
-    _check(lib().kda_chunk_fwd_gated(
+    call = lib().kda_chunk_fwd_save if _save else lib().kda_chunk_fwd_gated
+    _check(call(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
         _ptr(cu_seqlens), B, T, H, dk, dv, N, _dtype_code(q), gate, _ptr(o), _ptr(final_state),
         _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream_ptr(stream, q.device)))
     if check if check is not None else _validate_default():
         _check_device_status(workspace, stream)
+    if _save:
+        return o, final_state, workspace
     return o, final_state
+
+
+def chunk_fwd_train(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
+                    output_final_state: bool = True, o=None, final_state=None, stream=None,
+                    check: Optional[bool] = None):
+    """``chunk_fwd`` for training (``kda_chunk_fwd_save``): returns (o, final_state,
+    saved), where ``saved`` is a backward-sized workspace that also holds what
+    ``chunk_bwd`` would recompute.  Pass it as ``chunk_bwd(..., saved=saved)`` with
+    the same inputs, unchanged, to skip the recomputation."""
+    return chunk_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, output_final_state, o,
+                     final_state, None, stream, check, _save=True)
 
 
 def chunk_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
@@ -275,15 +296,17 @@ def chunk_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int,
 
 def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=None,
               cu_seqlens=None, output_d_initial_state: bool = True, workspace=None,
-              stream=None, check: Optional[bool] = None) -> Dict[str, Optional[torch.Tensor]]:
+              stream=None, saved=None, check: Optional[bool] = None) -> Dict[str, Optional[torch.Tensor]]:
     """Gradients of the chunkwise forward (``kda_chunk_bwd_gated``).
 
     Inputs as ``chunk_fwd``: log_alpha [B, T, H, dk] (KDA), [B, T, H] (Gated
     DeltaNet) or None (DeltaNet); d_o like o; d_final_state [N, H, dk, dv] fp32
     or None.  Returns a dict with dq, dk, dv (input dtype), dlog_alpha (shaped
     like log_alpha, None without a gate), dbeta (fp32) and dS0 [N, H, dk, dv]
-    (fp32, or None when ``output_d_initial_state`` is false).  ``check`` as in
-    :func:`chunk_fwd`.
+    (fp32, or None when ``output_d_initial_state`` is false).  With ``saved``
+    (the third result of ``chunk_fwd_train`` on the same inputs) the forward is
+    not recomputed (``kda_chunk_bwd_saved``); ``workspace`` must then be None.
+    ``check`` as in :func:`chunk_fwd`.
     """
     _dims(q, "q", 4)
     _dims(v, "v", 4)
@@ -310,9 +333,18 @@ def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=N
          "dS0": (torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
                  if output_d_initial_state else None)}
     ws_bytes = chunk_bwd_workspace_size(B, T, H, dk, dv, N, cu_seqlens is not None, q.dtype)
+    call = lib().kda_chunk_bwd_gated
+    if saved is not None:
+        if workspace is not None:
+            raise ValueError("pass either saved or workspace, not both")
+        _need(saved, "saved", torch.uint8, dev)
+        if saved.numel() < ws_bytes:
+            raise ValueError(f"saved holds {saved.numel()} bytes; these sizes need {ws_bytes} "
+                             "(it must come from chunk_fwd_train on the same inputs)")
+        workspace, call = saved, lib().kda_chunk_bwd_saved
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
-    _check(lib().kda_chunk_bwd_gated(
+    _check(call(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
         _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state), B, T, H, dk, dv, N, _dtype_code(q), gate,
         _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]),

@@ -284,6 +284,42 @@ kda_status kda_chunk_bwd_gated(const void* q, const void* k, const void* v,
                                size_t workspace_bytes, void* stream);
 
 /*
+ * Training forward: kda_chunk_fwd_gated (same arguments and outputs) that
+ * also keeps, in `workspace`, everything kda_chunk_bwd would otherwise
+ * recompute from the inputs: the chunk table, the per-chunk records, T =
+ * (I + A)^-1 (for bf16 inputs with the K~ and V tiles, M and the strong-decay
+ * flags) and the state entering every chunk.  `workspace` must have at least
+ * kda_chunk_bwd_workspace_size(...) bytes (256-byte aligned); pass it, with
+ * the same inputs and sizes, to kda_chunk_bwd_saved.  It always runs the
+ * two-kernel form (never the fused pass; KDA_CHUNK_PATH does not apply), with
+ * the kernels that also write what the backward reads.  The chunkwise mode is
+ * the training mode of news.bugfactory.tech/news/3610 (KDA paragraph).
+ */
+kda_status kda_chunk_fwd_save(const void* q, const void* k, const void* v,
+                              const float* log_alpha, const float* beta,
+                              const float* initial_state, const int32_t* cu_seqlens,
+                              int B, int T, int H, int dk, int dv, int num_seqs,
+                              kda_dtype dtype, kda_gate gate, void* o, float* final_state,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * kda_chunk_bwd_gated after kda_chunk_fwd_save: the same arguments, but the
+ * forward is not recomputed.  `workspace` must be the one kda_chunk_fwd_save
+ * filled for exactly these inputs and sizes, unchanged since; its contents are
+ * not checked (a different workspace gives wrong gradients, not an error).
+ * Its status word keeps what the forward recorded (kda_workspace_status).
+ */
+kda_status kda_chunk_bwd_saved(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta,
+                               const float* initial_state, const int32_t* cu_seqlens,
+                               const void* d_o, const float* d_final_state,
+                               int B, int T, int H, int dk, int dv, int num_seqs,
+                               kda_dtype dtype, kda_gate gate, void* dq, void* dk_out,
+                               void* dv_out, float* dlog_alpha, float* dbeta,
+                               float* d_initial_state, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
  * Measurement hook for benchmarks.  When `events` is non-NULL, each later
  * kda_chunk_fwd on this host thread records the caller-created CUDA events
  * (cudaEvent_t passed as void*) on its stream at the stage boundaries:

@@ -192,3 +192,30 @@ def test_chunk_fwd_plan_without_a_device(lib, monkeypatch):
     assert lib.kda_chunk_fwd_plan(1, 300, 8, 128, 128, 3, 1, bf16, full) == 1
     monkeypatch.setenv("KDA_CHUNK_PATH", "split")
     assert lib.kda_chunk_fwd_plan(1, 300, 8, 128, 128, 3, 1, bf16, small) == -1
+
+
+def test_saved_forward_entry_points_validate(lib):
+    """kda_chunk_fwd_save needs the backward-sized workspace; kda_chunk_bwd_saved
+    validates like kda_chunk_bwd.  (Every case fails before any launch.)"""
+    p = 1 << 20
+    f32 = 0
+    fwd_bytes = lib.kda_chunk_fwd_workspace_size(1, 64, 1, 64, 64, 1, 0, f32)
+    bwd_bytes = lib.kda_chunk_bwd_workspace_size(1, 64, 1, 64, 64, 1, 0, f32)
+    assert bwd_bytes > fwd_bytes
+    f = lib.kda_chunk_fwd_save
+    # a forward-sized workspace is too small to keep what the backward needs
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 64, 64, 1, f32, 0, p, None, p, fwd_bytes, None) == 5
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 64, 64, 1, f32, 0, p, None, None, 0, None) == 5
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 64, 64, 1, f32, 9, p, None, p, bwd_bytes, None) == 1
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 96, 64, 1, f32, 0, p, None, p, bwd_bytes, None) == 2
+    b = lib.kda_chunk_bwd_saved
+    # null cotangent; workspace too small
+    assert b(p, p, p, p, p, None, None, None, None, 1, 64, 1, 64, 64, 1, f32, 0,
+             p, p, p, p, p, None, p, bwd_bytes, None) == 1
+    assert b(p, p, p, p, p, None, None, p, None, 1, 64, 1, 64, 64, 1, f32, 0,
+             p, p, p, p, p, None, p, 16, None) == 5
+    # bf16: a workspace that would run the fused forward is still too small to save
+    bf16 = 1
+    fused_bytes = lib.kda_chunk_fwd_fused_workspace_size(1, 64, 1, 64, 64, 1, 0, bf16)
+    assert fused_bytes > 0
+    assert f(p, p, p, p, p, None, None, 1, 64, 1, 64, 64, 1, bf16, 0, p, None, p, fused_bytes, None) == 5
