@@ -263,9 +263,14 @@ static kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, co
         if (e == cudaSuccess) e = kda::launch_chunk_fused_tc(a);
         if (e == cudaSuccess) e = mark_stage(2, a.stream);
     } else {
-        if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_intra_tc(a) : kda::launch_chunk_intra(a);
+        // fp32: the split-tf32 tensor-core K1, or in backward mode (T kept) the CUDA-core one
+        if (e == cudaSuccess)
+            e = a.bf16 ? kda::launch_chunk_intra_tc(a)
+                       : (a.tmat ? kda::launch_chunk_intra(a) : kda::launch_chunk_intra_f32_tc(a));
         if (e == cudaSuccess) e = mark_stage(2, a.stream);
-        if (e == cudaSuccess) e = a.bf16 ? kda::launch_chunk_inter_tc(a) : kda::launch_chunk_inter(a);
+        if (e == cudaSuccess)
+            e = a.bf16 ? kda::launch_chunk_inter_tc(a)
+                       : (a.tmat ? kda::launch_chunk_inter(a) : kda::launch_chunk_inter_f32_tc(a));
     }
     if (e == cudaSuccess) e = mark_stage(3, a.stream);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "kda_chunk_fwd launch failed: %s", cudaGetErrorString(e));

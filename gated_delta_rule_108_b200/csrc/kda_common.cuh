@@ -49,6 +49,25 @@ struct F32Rec {
     static constexpr size_t FLOATS = (GC + DK + 63) / 64 * 64;   // 256-byte multiple
 };
 
+// The same quantities for the fp32 tensor-core kernels, laid out for them:
+//   WQ  [128][DK]  rows 0..63 W, 64..127 Q~ (row-major; one thread loads a row)
+//   KHT [DK][64]   K^ transposed (row = key channel, one thread loads a row)
+//   P   [2][64][32] the two 32-token halves of P, each row's 16-byte chunks
+//                  XOR-swizzled by (row mod 8) (the 128-byte swizzle of an MMA tile)
+//   U0  [DV/32][64][32] 32-column slices of U0, swizzled the same way
+//   GC  [DK]
+// Rows past the chunk's tokens are zero.  Same size as F32Rec.
+template <int DK, int DV>
+struct F32TcRec {
+    static constexpr size_t WQ = 0;
+    static constexpr size_t KHT = WQ + 2 * kChunk * DK;
+    static constexpr size_t P = KHT + DK * kChunk;
+    static constexpr size_t U0 = P + kChunk * kChunk;
+    static constexpr size_t GC = U0 + kChunk * DV;
+    static constexpr size_t FLOATS = (GC + DK + 63) / 64 * 64;
+    static_assert(FLOATS == F32Rec<DK, DV>::FLOATS, "the workspace is sized by F32Rec");
+};
+
 // Backward, per (head, chunk), fp32: the products over the value dimension,
 // dQ~ = D S^T, dW = -dU S^T, dK^ = U dS'^T [64][DK] each, dP = D U^T [64][64]
 // (lower with the diagonal), dgamma [DK].  Written by the tensor-core

@@ -73,9 +73,11 @@ cudaError_t launch_chunk_prep(const ChunkArgs& a);     // K0: status reset + var
 cudaError_t launch_chunk_intra(const ChunkArgs& a);    // K1: all chunks in parallel
 cudaError_t launch_chunk_inter(const ChunkArgs& a);    // K2: serial over each sequence's chunks
 cudaError_t launch_chunk_intra_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K1
+cudaError_t launch_chunk_intra_f32_tc(const ChunkArgs& a); // fp32 inputs, forward: tensor-core K1 (split tf32)
 cudaError_t launch_chunk_intra_fwd_tc(const ChunkArgs& a); // its forward-only form, two CTAs per SM
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a); // bf16 inputs: tensor-core K2
 cudaError_t launch_chunk_inter_fwd_tc(const ChunkArgs& a); // its forward-only form, slice width per call
+cudaError_t launch_chunk_inter_f32_tc(const ChunkArgs& a); // fp32 inputs, forward: tensor-core K2 (split tf32)
 cudaError_t launch_chunk_fused_tc(const ChunkArgs& a);     // bf16 forward in one pass, one CTA per (sequence, head)
 cudaError_t launch_chunk_seq_order(const ChunkArgs& a);    // packed sequences longest first into a.seq_order
 cudaError_t launch_chunk_bwd_inter(const ChunkArgs& a);  // backward: serial over chunks, reversed

@@ -333,6 +333,58 @@ def test_strong_decay(cuda_device, dtype, where):
     check(S, S_ref, dtype, f"{where} final_state")
 
 
+@pytest.mark.parametrize("gate", ["channel", "head", "none"])
+def test_f32_many_items_mixed_strong(cuda_device, gate):
+    """fp32 inputs, persistent intra-chunk kernel with several (chunk, head) items per CTA:
+    five packed sequences of ragged lengths (73 chunks) x H=12 = 876 items, d_k=128, d_v=64.
+    With the per-channel gate, every third chunk of heads 0 and 5 decays strongly enough for
+    the exact path; the per-head gate and no gate go to the oracle broadcast over the key
+    channels.  Every (sequence, head) pair is checked."""
+    lens = (1300, 1, 700, 64, 2477)
+    w = I.ChunkWorkload("f32mix", B=1, T=sum(lens), H=12, dk=128, dv=64, dtype=torch.float32,
+                        s0_std=0.05, lengths=lens, beta_edge_frac=0.1, seed=61)
+    x = I.chunk_inputs(w)
+    if gate == "channel":
+        la = x["log_alpha"].clone()
+        gen = torch.Generator().manual_seed(611)
+        strong = (torch.arange(w.T) // 64) % 3 == 1
+        for h in (0, 5):
+            la[0, strong, h, :4] = -8.0 * torch.rand(int(strong.sum()), 4, generator=gen)
+        x["log_alpha"] = la.contiguous()
+    la_oracle = x["log_alpha"]
+    if gate == "head":
+        x["log_alpha"] = x["log_alpha"][..., 0].contiguous()
+        la_oracle = x["log_alpha"][..., None].expand(la_oracle.shape).contiguous()
+    elif gate == "none":
+        x["log_alpha"] = None
+        la_oracle = torch.zeros_like(la_oracle)
+    o, S = run_chunk(x)
+    o_ref, S_ref = oracle_chunk(dict(x, log_alpha=la_oracle))
+    cu = x["cu_seqlens"].tolist()
+    for s in range(len(lens)):
+        for h in range(w.H):
+            a, b = cu[s], cu[s + 1]
+            if b > a:
+                check(o[:, a:b, h], o_ref[:, a:b, h], torch.float32, f"{gate} seq {s} head {h} o")
+            check(S[s, h], S_ref[s, h], torch.float32, f"{gate} seq {s} head {h} final_state")
+
+
+@pytest.mark.parametrize("dk", [128, 64])
+def test_f32_wide_slices(cuda_device, dk):
+    """fp32 inputs with more (sequence, head) chains than 32-column slices fit in one wave
+    (B=2, H=40, d_v=128: 80 chains x 4 > 148 SMs), so the inter-chunk kernel takes
+    64-column slices (with d_k=128 one R3 buffer in tensor memory).  Every pair is checked."""
+    w = I.ChunkWorkload("f32wide", B=2, T=300, H=40, dk=dk, dv=128, dtype=torch.float32, s0_std=0.05,
+                        seed=62)
+    x = I.chunk_inputs(w)
+    o, S = run_chunk(x)
+    o_ref, S_ref = oracle_chunk(x)
+    for b in range(w.B):
+        for h in range(w.H):
+            check(o[b, :, h], o_ref[b, :, h], torch.float32, f"seq {b} head {h} o")
+            check(S[b, h], S_ref[b, h], torch.float32, f"seq {b} head {h} final_state")
+
+
 def test_value_range_reported(cuda_device):
     """bf16 path: a value beyond the fp16 range of the intermediates is reported."""
     w = I.ChunkWorkload("range", B=1, T=70, H=1, dk=64, dv=64, dtype=torch.bfloat16, seed=29)
