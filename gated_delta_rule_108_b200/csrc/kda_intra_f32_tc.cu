@@ -11,7 +11,7 @@
 // head) item, with g the cumulative log-decay (base 2) and g_m the middle token's:
 //
 //   [A; P] = [K~m; Q~m] K-m^T     A operand (hi, lo) in TMEM, K-m (hi, lo) in smem
-//   T = (I + A)^{-1}              forward substitution on CUDA cores, fp32
+//   T = (I + A)^{-1}              16 x 16 blocks on CUDA cores, fp32
 //   [W | U0] = T diag(beta) [K~ | V]   T diag(beta) (hi, lo) in TMEM, K~^T, V^T in smem
 //
 // and writes the fp32 record (F32TcRec) that the fp32 tensor-core inter-chunk
@@ -56,7 +56,8 @@ struct F32K1Smem {
     //   element pass .. MMA1: K-m (hi | lo) at KB, token-major, K = channel, DK/32 tiles of
     //     64 rows x 128 B (strong-decay chunks: raw k and q [64][DK] there instead), and
     //     K~^T (hi | lo) at KTT, channel-major, 2 tiles (tokens 0..31, 32..63) of DK rows x 128 B
-    //   MMA1 .. MMA2: V^T (hi | lo) at KB, 2 tiles of DV rows x 128 B
+    //   after MMA1: T and its partial products, then V^T (hi | lo) at KB, 2 tiles of
+    //     DV rows x 128 B, until MMA2
     //   after MMA2: the next item's k and q
     static constexpr uint32_t KB = 0;
     static constexpr uint32_t KB_BYTES = (DK > DV ? DK : DV) * 512u;
@@ -65,8 +66,8 @@ struct F32K1Smem {
     static constexpr uint32_t BIG_BYTES = KB_BYTES + KTT_BYTES;
     static constexpr uint32_t KQ_Q = 64u * LDK * 4u;     // q staging, after k's
     static constexpr uint32_t G = BIG_BYTES;             // log-decay (copied in early), then g (base 2): [64][LDK]
-    static constexpr uint32_t AM = G + 64u * LDK * 4u;   // A (beta-scaled, strictly lower), then T diag(beta)
-    static constexpr uint32_t VS = AM + 64u * LDA * 4u;  // v [64][LDV] (copied in at the item's start); then P [64][LDA]
+    static constexpr uint32_t AM = G + 64u * LDK * 4u;   // A (beta-scaled, strictly lower), then P [64][LDA]
+    static constexpr uint32_t VS = AM + 64u * LDA * 4u;  // v [64][LDV] (copied in at the item's start)
     // after MMA2, over G, AM and VS: W [64][LDK] and U0 [64][LDV], staged for coalesced stores
     static constexpr uint32_t WS = G, US = G + 64u * LDK * 4u;
     static constexpr uint32_t BETA = VS + 64u * LDV * 4u;
@@ -75,7 +76,7 @@ struct F32K1Smem {
     static_assert(KB % 1024 == 0 && KTT % 1024 == 0, "operand tiles are 1024-byte aligned");
     static_assert(2u * 64u * LDK * 4u <= BIG_BYTES, "k, q staging fits");
     static_assert(US + 64u * LDV * 4u <= VS + 64u * LDV * 4u, "W, U0 staging fits");
-    static_assert(LDA <= LDV, "P staging fits in VS");
+    static_assert(64u * LDA * 4u + 3u * 16u * 17u * 4u <= KB_BYTES, "T and its partial products fit in K-m's space");
     static_assert(END + 1024 <= 232448, "shared memory");
 };
 
@@ -385,78 +386,112 @@ intra_chunk_f32_tc_kernel(const float* __restrict__ q, const float* __restrict__
         cp_async_wait<0>();   // v
         __syncthreads();      // A complete; K-m (or raw k, q) is dead; v has landed
 
-        // ---- T = (I + A)^{-1} by forward substitution (warps 0-1, one column
-        //      each).  Meanwhile warps 2-7: V^T (hi | lo) over K-m, then P through
-        //      shared memory (coalesced record stores).
-        if (tid < 64) {
-            float x[kChunk];
+        // ---- T = (I + A)^{-1}, blocked over 16 x 16 blocks (all threads, fp32, in
+        //      the free K-m space): the diagonal blocks by forward substitution,
+        //      then T_ij = -T_ii sum_{j <= m < i} A_im T_mj level by level
+        {
+            float* tt = reinterpret_cast<float*>(sm + Sm::KB);   // T [64][LDA]
+            float* xs = tt + 64 * LDA;                            // [3][16][17] partial products
+            if (tid < 64) {
+                const int kb = tid >> 4, j = tid & 15, o0 = 16 * kb;
+                float x[16];
 #pragma unroll
-            for (int r = 0; r < kChunk; ++r) {
-                float a0 = (r == tid) ? 1.f : 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                for (int r = 0; r < 16; ++r) {
+                    float acc = (r == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int i = 0; i + 3 < r; i += 4) {
-                    a0 = fmaf(-am[r * LDA + i], x[i], a0);
-                    a1 = fmaf(-am[r * LDA + i + 1], x[i + 1], a1);
-                    a2 = fmaf(-am[r * LDA + i + 2], x[i + 2], a2);
-                    a3 = fmaf(-am[r * LDA + i + 3], x[i + 3], a3);
+                    for (int i = 0; i < r; ++i) acc = fmaf(-am[(o0 + r) * LDA + o0 + i], x[i], acc);
+                    x[r] = acc;
+                    tt[(o0 + r) * LDA + o0 + j] = acc;
                 }
-#pragma unroll
-                for (int i = r & ~3; i < r; ++i) a0 = fmaf(-am[r * LDA + i], x[i], a0);
-                x[r] = (a0 + a1) + (a2 + a3);
+            } else {   // zero above the diagonal blocks
+                for (int idx = tid - 64; idx < 6 * 256; idx += 192) {
+                    const int blk = idx >> 8, e2 = idx & 255, i = e2 >> 4, j = e2 & 15;
+                    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                    const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                    tt[(16 * bi + i) * LDA + 16 * bj + j] = 0.f;
+                }
             }
-            asm volatile("bar.sync 1, 64;" ::: "memory");   // every solver thread has read all of A
-            const float bt = s_beta[tid];
+            __syncthreads();
+            const int bi = tid >> 4, bj = tid & 15;   // element of a 16 x 16 block
+            // X = sum_{m = mj}^{mi - 1} A_{mi, m} T_{m, mj};  T_{mi, mj} = -T_{mi, mi} X
+            auto x_part = [&](int mi, int mj, float* xo) {
+                float acc = 0.f;
+                for (int m = mj; m < mi; ++m)
 #pragma unroll
-            for (int r = 0; r < kChunk; ++r) am[r * LDA + tid] = x[r] * bt;   // T diag(beta)
-        } else {
-            const int t = tid - 64;   // 0..191
-            {
-                const float* vs = reinterpret_cast<const float*>(sm + Sm::VS);
-                const uint32_t vt_lo = 2u * DV * 128u;
-                for (int idx = t; idx < 64 * (DV / 4); idx += 192) {
-                    const int r = idx & 63, c4 = (idx >> 6) * 4;
-                    const float4 x4 = *reinterpret_cast<const float4*>(vs + r * LDV + c4);
-                    const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
+                    for (int q = 0; q < 16; ++q)
+                        acc = fmaf(am[(16 * mi + bi) * LDA + 16 * m + q], tt[(16 * m + q) * LDA + 16 * mj + bj], acc);
+                xo[bi * 17 + bj] = acc;
+            };
+            auto t_part = [&](int mi, int mj, const float* xi) {
+                float acc = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float hi, lo;
-                        split_tf32(xs[e], hi, lo);
-                        const uint32_t off = (uint32_t)(r >> 5) * (DV * 128u) + sw128_offset(c4 + e, (r & 31) * 4);
-                        *reinterpret_cast<float*>(sm + Sm::KB + off) = hi;
-                        *reinterpret_cast<float*>(sm + Sm::KB + vt_lo + off) = lo;
-                    }
+                for (int q = 0; q < 16; ++q) acc = fmaf(tt[(16 * mi + bi) * LDA + 16 * mi + q], xi[q * 17 + bj], acc);
+                tt[(16 * mi + bi) * LDA + 16 * mj + bj] = -acc;
+            };
+            x_part(1, 0, xs);
+            x_part(2, 1, xs + 272);
+            x_part(3, 2, xs + 544);
+            __syncthreads();
+            t_part(1, 0, xs);
+            t_part(2, 1, xs + 272);
+            t_part(3, 2, xs + 544);
+            __syncthreads();
+            x_part(2, 0, xs);
+            x_part(3, 1, xs + 272);
+            __syncthreads();
+            t_part(2, 0, xs);
+            t_part(3, 1, xs + 272);
+            __syncthreads();
+            x_part(3, 0, xs);
+            __syncthreads();
+            t_part(3, 0, xs);   // A is no longer read: P may use its space
+            if (!strong && !is_k) {   // P (lanes 64..127), lower with the diagonal -> AM
+                float vv[32];
+                tmem_ld32_sync(D1 + lane_base + 32 * hc, vv);
+                const int r = r_el;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = 32 * hc + e;
+                    am[r * LDA + i] = i <= r ? vv[e] : 0.f;
+                }
+            }
+            __syncthreads();
+            // T diag(beta) -> TMEM (hi | lo), MMA2's A operand (lanes 0..63)
+            if (is_k) {
+                float th[32], tl[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    split_tf32(tt[row * LDA + 32 * hc + e] * s_beta[32 * hc + e], th[e], tl[e]);
+                tmem_st32_sync(A2 + lane_base + 32 * hc, th);
+                tmem_st32_sync(A2 + 64 + lane_base + 32 * hc, tl);
+            }
+            __syncthreads();   // T is read: V^T may take its space
+        }
+        // ---- V^T (hi | lo) over K-m (MMA2's B operand); the P record from AM
+        {
+            const float* vs = reinterpret_cast<const float*>(sm + Sm::VS);
+            const uint32_t vt_lo = 2u * DV * 128u;
+            for (int idx = tid; idx < 64 * (DV / 4); idx += 256) {
+                const int r = idx & 63, c4 = (idx >> 6) * 4;
+                const float4 x4 = *reinterpret_cast<const float4*>(vs + r * LDV + c4);
+                const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float hi, lo;
+                    split_tf32(xv[e], hi, lo);
+                    const uint32_t off = (uint32_t)(r >> 5) * (DV * 128u) + sw128_offset(c4 + e, (r & 31) * 4);
+                    *reinterpret_cast<float*>(sm + Sm::KB + off) = hi;
+                    *reinterpret_cast<float*>(sm + Sm::KB + vt_lo + off) = lo;
                 }
             }
             if (!strong) {
-                float* ps = reinterpret_cast<float*>(sm + Sm::VS);   // v is dead once every V^T is written
-                asm volatile("bar.sync 2, 192;" ::: "memory");
-                if (!is_k) {   // P (lanes 64..127), lower with the diagonal
-                    float vv[32];
-                    tmem_ld32_sync(D1 + lane_base + 32 * hc, vv);
-                    const int r = r_el;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = 32 * hc + e;
-                        ps[r * LDA + i] = i <= r ? vv[e] : 0.f;
-                    }
-                }
-                asm volatile("bar.sync 2, 192;" ::: "memory");
                 // record tiles: [half t][row][32 floats], 16-byte chunks swizzled by row
-                for (int idx = t; idx < 1024; idx += 192) {
+                for (int idx = tid; idx < 1024; idx += 256) {
                     const int th = idx >> 9, rr = (idx >> 3) & 63, lc = (idx & 7) ^ (rr & 7);
-                    const float* src = ps + rr * LDA + 32 * th + 4 * lc;
+                    const float* src = am + rr * LDA + 32 * th + 4 * lc;
                     *reinterpret_cast<float4*>(rec + R::P + (size_t)idx * 4) = make_float4(src[0], src[1], src[2], src[3]);
                 }
             }
-        }
-        __syncthreads();
-        // ---- T diag(beta) -> TMEM (hi | lo), MMA2's A operand (lanes 0..63)
-        if (is_k) {
-            float th[32], tl[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) split_tf32(am[row * LDA + 32 * hc + e], th[e], tl[e]);
-            tmem_st32_sync(A2 + lane_base + 32 * hc, th);
-            tmem_st32_sync(A2 + 64 + lane_base + 32 * hc, tl);
         }
         fence_proxy_async_smem();
         tc_fence_before();
