@@ -253,12 +253,15 @@ def rank_workload(w, rank: int):
 
 
 # --------------------------------------------------------------- our arm --
-def bench_chunk(name, steps, warmup, dev, world, rank):
-    """Time kda_chunk_fwd on one workload; per-stage times from library events."""
+def bench_chunk(name, steps, warmup, dev, world, rank, dtype=None):
+    """Time kda_chunk_fwd on one workload (its shape in another input dtype if
+    given); per-stage times from library events."""
     from gated_delta_rule_108_b200 import inputs as I
     from gated_delta_rule_108_b200 import kda
 
     w = I.workload(name)
+    if dtype is not None and dtype != w.dtype:
+        w = dataclasses.replace(w, dtype=dtype, name=f"{w.name} ({'fp32' if dtype == torch.float32 else 'bf16'})")
     x = I.chunk_inputs(rank_workload(w, rank))
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     varlen = g["cu_seqlens"] is not None
@@ -312,7 +315,8 @@ def chunk_summary(res, world, peaks, peak_kind):
     dom = max(kern, key=kern.get)
     dom_ms = kern[dom]
     achieved = mb[dom] / (dom_ms / 1e3) / 1e9
-    tpu = traffic_per_unit(dom)
+    # the committed captures are of the bf16 kernels
+    tpu = traffic_per_unit(dom) if w.dtype == torch.bfloat16 else None
     path_gbs = mb["total"] / (ms / 1e3) / 1e9
     th = w.tokens * w.H
     tflops = chunk_flops_per_token_head(w.dk, w.dv) * th / (ms / 1e3) / 1e12
@@ -618,6 +622,14 @@ def run_ours(args):
         extras[name.lower() + "_fused"] = summ_f
         del r
         torch.cuda.empty_cache()
+    # fp32 inputs on the same shapes (split-tf32 tensor-core kernels)
+    for name in [n for n in args.f32_workloads.split(",") if n]:
+        r = bench_chunk(name, args.steps, args.warmup, dev, world, rank, dtype=torch.float32)
+        summ_f = chunk_summary(r, world, peaks, peak_kind)
+        summ_f["form"] = "two kernels, fp32 inputs: split-tf32 tensor-core products (3 MMAs each)"
+        extras[name.lower() + "_f32"] = summ_f
+        del r
+        torch.cuda.empty_cache()
     dec = None if args.no_decode else bench_decode(args, dev, world, rank, peaks, peak_kind)
     bwd = None if args.no_bwd else bench_backward(args, dev, world, rank, peaks, peak_kind)
     train = None if (args.no_bwd or args.no_train) else bench_train(args, dev, world, rank)
@@ -750,6 +762,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="C4", help="headline chunk-forward workload (C0..C4 minus C3)")
     ap.add_argument("--extra-workloads", default="C1,C2", help="more chunk-forward workloads, comma-separated")
+    ap.add_argument("--f32-workloads", default="C1",
+                    help="chunk-forward workloads also timed with fp32 inputs (key <name>_f32)")
     ap.add_argument("--fused-workloads", default="C4",
                     help="chunk-forward workloads also timed with the fused single pass forced")
     ap.add_argument("--decode-workload", default="C3")
