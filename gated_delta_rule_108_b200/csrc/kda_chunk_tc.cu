@@ -1961,16 +1961,16 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const float* vs = vside + it * VS::FLOATS;
         const float* Mg = reinterpret_cast<const float*>(tiles + it * BT::BYTES + BT::M);
         if (beta_thread) s_beta[tid - 128] = bnext;
-        // this thread's rows of M and dbeta parts through W, U0 (used once the MMAs are issued):
-        // step j covers row r = (tid + 256 j) / 16, columns 4 ((tid + 256 j) % 16) + [0, 4)
-        float4 mm[4];
-        float dbp[4];
+        // this thread's entries of M (used once the MMAs are issued): step j covers
+        // column (tid + 256 j) % 64, rows 4 ((tid + 256 j) / 64) + [0, 4), as dA below
+        float mm[4][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int idx = tid + 256 * j, r = idx >> 4, i4 = (idx & 15) * 4;
-            mm[j] = *reinterpret_cast<const float4*>(Mg + r * kChunk + i4);
-            dbp[j] = vs[VS::DBP + r];
+            const int idx = tid + 256 * j, i = idx & 63, r4 = (idx >> 6) * 4;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mm[j][t] = Mg[(r4 + t) * kChunk + i];
         }
+        const float dbp = tid < kChunk ? vs[VS::DBP + tid] : 0.f;   // dbeta parts through W, U0
         const float dgam = tid < DK ? vs[VS::DGAM + tid] : 0.f;   // for the dlog_alpha scan
         const bool got = mbar_wait_cycles(&bar_load, load_phase, kWaitCycles);
         if (__syncthreads_or(!got)) { aborted = true; break; }
@@ -2001,12 +2001,19 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             s_gl[tid] = g[(L - 1) * DK + tid];
             s_dgl[tid] = 0.f;
         }
-        float4 da[4], dp[4];   // same (row, 4 columns) steps as mm
+        // dA, dP by column: step j holds column idx % 64, rows 4 (idx / 64) + [0, 4)
+        // (idx = tid + 256 j), so that both [dM; dP] (row-major: a warp fills one
+        // row segment) and its transpose (a warp fills one 16-byte chunk of 32
+        // rows) are stored without bank conflicts
+        float da[4][4], dp[4][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int idx = tid + 256 * j;
-            da[j] = reinterpret_cast<const float4*>(sm + Sm::PF_DA)[idx];   // row idx / 16, columns 4 (idx % 16) + [0, 4)
-            dp[j] = reinterpret_cast<const float4*>(sm + Sm::PF_DP)[idx];
+            const int idx = tid + 256 * j, i = idx & 63, r4 = (idx >> 6) * 4;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                da[j][t] = reinterpret_cast<const float*>(sm + Sm::PF_DA)[(r4 + t) * 64 + i];
+                dp[j][t] = reinterpret_cast<const float*>(sm + Sm::PF_DP)[(r4 + t) * 64 + i];
+            }
         }
         __syncthreads();
 
@@ -2042,19 +2049,17 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // [dM; dP] and their transposes
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int idx = tid + 256 * j, r = idx >> 4, i4 = (idx & 15) * 4;
-            const float br = s_beta[r];
-            const float dm[4] = {round_tf32_alu(br * da[j].x), round_tf32_alu(br * da[j].y),
-                                 round_tf32_alu(br * da[j].z), round_tf32_alu(br * da[j].w)};
-            const float pp[4] = {round_tf32_alu(dp[j].x), round_tf32_alu(dp[j].y), round_tf32_alu(dp[j].z),
-                                 round_tf32_alu(dp[j].w)};
-            *reinterpret_cast<float4*>(sm + Sm::DMP + f_off(r, i4, 16384)) = make_float4(dm[0], dm[1], dm[2], dm[3]);
-            *reinterpret_cast<float4*>(sm + Sm::DMP + f_off(64 + r, i4, 16384)) = make_float4(pp[0], pp[1], pp[2], pp[3]);
+            const int idx = tid + 256 * j, i = idx & 63, r4 = (idx >> 6) * 4;
+            float dm[4], pp[4];
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-                *reinterpret_cast<float*>(sm + Sm::DMPT + f_off(i4 + t, r, 8192)) = dm[t];
-                *reinterpret_cast<float*>(sm + Sm::DMPT + f_off(i4 + t, 64 + r, 8192)) = pp[t];
+                dm[t] = round_tf32_alu(s_beta[r4 + t] * da[j][t]);
+                pp[t] = round_tf32_alu(dp[j][t]);
+                *reinterpret_cast<float*>(sm + Sm::DMP + f_off(r4 + t, i, 16384)) = dm[t];
+                *reinterpret_cast<float*>(sm + Sm::DMP + f_off(64 + r4 + t, i, 16384)) = pp[t];
             }
+            *reinterpret_cast<float4*>(sm + Sm::DMPT + f_off(i, r4, 8192)) = make_float4(dm[0], dm[1], dm[2], dm[3]);
+            *reinterpret_cast<float4*>(sm + Sm::DMPT + f_off(i, 64 + r4, 8192)) = make_float4(pp[0], pp[1], pp[2], pp[3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -2093,15 +2098,17 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 dkhv[t] = vs[VS::DKH + r * DK + lane_row];
             }
         }
-        // meanwhile: dbeta = (parts through W, U0) + rowsum(dA M); a row's 16 steps
-        // sit in one half-warp
+        // meanwhile: rowsum(dA M) for dbeta over this warp's 32 columns of 4 rows per
+        // step (the other 32 columns are in the neighbouring warp)
+        float rs[4][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            float part = da[j].x * mm[j].x + da[j].y * mm[j].y + da[j].z * mm[j].z + da[j].w * mm[j].w;
 #pragma unroll
-            for (int off = 8; off; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-            const int r = (tid + 256 * j) >> 4;
-            if ((lane & 15) == 0 && r < L) dbeta[(size_t)(tok0 + r) * H + h] = dbp[j] + part;
+            for (int t = 0; t < 4; ++t) rs[j][t] = da[j][t] * mm[j][t];
+#pragma unroll
+            for (int off = 16; off; off >>= 1)
+#pragma unroll
+                for (int t = 0; t < 4; ++t) rs[j][t] += __shfl_xor_sync(0xffffffffu, rs[j][t], off);
         }
         const bool ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
         if (__syncthreads_or(!ok)) { aborted = true; break; }
@@ -2113,6 +2120,15 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (tid == 0) prefetch(nw);
             load_pending = true;
             if (beta_thread) bnext = load_beta(nw);
+        }
+        // the row sums' two column halves, in [K_l^T | Q_l^T]'s space (read by the
+        // MMAs, not a prefetch target): [2][64]
+        float* rowsum = reinterpret_cast<float*>(sm + Sm::KLQT);
+        if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int t = 0; t < 4; ++t) rowsum[(warp & 1) * kChunk + ((tid + 256 * j) >> 6) * 4 + t] = rs[j][t];
         }
 
         // dq, dk and dg for channel lane_row, tokens [32 wg, 32 wg + 32)
@@ -2153,6 +2169,8 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             atomicAdd(&s_dgl[ch], dgl);
         }
         __syncthreads();
+        // dbeta = (parts through W, U0) + rowsum(dA M)
+        if (tid < L) dbeta[(size_t)(tok0 + tid) * H + h] = dbp + rowsum[tid] + rowsum[kChunk + tid];
         // dlog_alpha_s = sum_{r >= s} dg_r (+ g_{L-1}'s own cotangent), per channel
         if (gate != kGateNone && tid < DK) {
             float run = s_dgl[tid] + dgam * __expf(s_gl[tid]);
