@@ -62,24 +62,26 @@ struct K1fSmem {
     static constexpr uint32_t OPB = G + G_BYTES;                        // K-m tf32 (MMA1 B); W | U0 fp16 staging
     static constexpr uint32_t OPB_BYTES = (DK / 32) * TILE;
     static constexpr uint32_t STG_BYTES = ((DK + DV) / 64) * TILE;
-    // after MMA1, behind V: the fp16 operands of the blocked (I + A)^{-1} (A
-    // masked to its level-1 blocks and to its level-2 quadrant, the diagonal
-    // inverses D, a product X, T restricted to its 32 x 32 diagonal blocks),
-    // each 64 x 64 tile read as a 128-row operand whose rows 64..127 are the
-    // next 8 KB; then A's four diagonal 16 x 16 blocks in fp32 (padded).  The
-    // strong-decay path writes the full fp32 A ([64][64]) before the element
-    // pass, while g is live, outside G and clear of AH1, AH2 and AMD.
+    // after MMA1, behind V: fp32 scratch of the first (CUDA-core) level of the
+    // blocked (I + A)^{-1} (A's blocks (1,0) and (3,2), their products, the
+    // diagonal inverses D), then the fp16 operands of its tensor-core level (A
+    // masked to its lower-left quadrant, a product X, T restricted to its 32 x 32
+    // diagonal blocks), each 64 x 64 tile read as a 128-row operand whose rows
+    // 64..127 are the next 8 KB; then A's four diagonal 16 x 16 blocks in fp32
+    // (padded).  The strong-decay path writes the full fp32 A ([64][64]) before
+    // the element pass, while g is live, outside G and clear of AF, AH2 and AMD.
     static constexpr uint32_t SCR = G + VB;
-    static constexpr uint32_t AH1 = SCR;
+    static constexpr uint32_t AF = SCR;                                 // [2][16][17] fp32 A_10, A_32
+    static constexpr uint32_t XF = SCR + 2304;                          // [2][16][17] fp32 A_10 D_0, A_32 D_2
     static constexpr uint32_t AH2 = SCR + 8192;
-    static constexpr uint32_t DH = SCR + 16384;
+    static constexpr uint32_t DF = SCR + 16384;                         // [4][16][17] fp32 D_0..D_3
     static constexpr uint32_t XH = SCR + 24576;
     static constexpr uint32_t T1H = SCR + 32768;
     static constexpr uint32_t AMD = SCR + 40960;                        // 4 x (16 x 16 + 4) fp32
     static constexpr uint32_t AMD_END = AMD + 4 * 260 * 4;
     static constexpr uint32_t AMS0 = (G + G_BYTES) > (AH2 + 8192) ? (G + G_BYTES) : (AH2 + 8192);
     static constexpr uint32_t AMS = AMS0 + 64 * 64 * 4 <= AMD ? AMS0 : (AMD_END + 15) / 16 * 16;   // [64][64]
-    // log-decay boxes (32 channels, 8 KB) past V overlap only AH1, AH2 and DH,
+    // log-decay boxes (32 channels, 8 KB) past V overlap only AF, XF, AH2 and DF,
     // which are dead once the second blocked-inverse level has read AH2: the
     // next item's boxes there are fetched then, the others after MMA2
     static constexpr int LA_EARLY_BOX = (int)(VB / TILE);
@@ -121,7 +123,8 @@ struct K1fSmem {
                   "swizzled tiles need 1024-byte alignment; MMA2's A operand runs into KT");
     static_assert(AMS >= G + G_BYTES && AMS >= AH2 + 8192 && (AMS + 64 * 64 * 4 <= AMD || AMS >= AMD_END),
                   "the strong path's A lies outside the live log-decay tile and the converted operands");
-    static_assert(G + G_BYTES <= SCR + 24576, "early log-decay boxes overlap only AH1, AH2, DH");
+    static_assert(XF + 2 * 16 * 17 * 4 <= AH2 && DF + 4 * 16 * 17 * 4 <= XH, "level-1 scratch");
+    static_assert(G + G_BYTES <= SCR + 24576, "early log-decay boxes overlap only AF, XF, AH2, DF");
     // two CTAs per SM (228 KB per SM, 1 KB reserved per CTA); the fused form one
     static_assert(FUSED ? TOTAL <= 232448 : 2 * (TOTAL + 1024) <= 233472, "CTAs per SM");
     static_assert(FWQ % 1024 == 0 && S16 % 1024 == 0, "swizzled tiles need 1024-byte alignment");
@@ -461,7 +464,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 
         float* amd = reinterpret_cast<float*>(sm + Sm::AMD);  // A's diagonal blocks, [4][16 x 16 + 4]
         // A row `row` (< 64), columns [32 hc, 32 hc + 32), beta-scaled and strictly
-        // lower: its diagonal block -> AMD (fp32); blocks (1,0), (3,2) -> AH1 and
+        // lower: its diagonal block -> AMD and blocks (1,0), (3,2) -> AF (fp32);
         // rows 32..63 x columns 0..31 -> AH2 (fp16, zero elsewhere)
         auto put_a_row = [&](const float (&v)[32]) {
             const int b = row >> 4;
@@ -483,14 +486,15 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                 const int col = 32 * hc + 8 * i8, cb = col >> 4;
                 const bool l1 = (b == 1 && cb == 0) || (b == 3 && cb == 2);
                 const bool l2 = b >= 2 && cb < 2;
-                __align__(16) __half h1[8], h2[8];
+                __align__(16) __half h2[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    h1[e] = __float2half_rn(l1 ? v[8 * i8 + e] : 0.f);
-                    h2[e] = __float2half_rn(l2 ? v[8 * i8 + e] : 0.f);
-                }
-                *reinterpret_cast<uint4*>(sm + Sm::AH1 + sw128_offset(row, col * 2)) = *reinterpret_cast<const uint4*>(h1);
+                for (int e = 0; e < 8; ++e) h2[e] = __float2half_rn(l2 ? v[8 * i8 + e] : 0.f);
                 *reinterpret_cast<uint4*>(sm + Sm::AH2 + sw128_offset(row, col * 2)) = *reinterpret_cast<const uint4*>(h2);
+                if (l1) {
+                    float* af = reinterpret_cast<float*>(sm + Sm::AF) + (b >> 1) * 272 + (row & 15) * 17 + (col & 15);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) af[e] = v[8 * i8 + e];
+                }
             }
         };
         bool ok = true;
@@ -532,11 +536,11 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         __syncthreads();
 
         // ---- T = (I + A)^{-1}: exact inverses D_b = (I + A_bb)^{-1} of the four
-        //      diagonal 16 x 16 blocks on CUDA cores, then the off-diagonal blocks on
-        //      the tensor cores by doubling the solved block (fp16 operands, fp32
-        //      accumulation):  T21 = -T22 A21 T11,  first for 16 -> 32 rows (the
-        //      pairs (1,0), (3,2)), then 32 -> 64.  T diag(beta) goes to TPV in fp16
-        //      (K-major, rows 0..63) block by block.
+        //      diagonal 16 x 16 blocks on CUDA cores, then the off-diagonal blocks by
+        //      doubling the solved block, T21 = -T22 A21 T11: for 16 -> 32 rows (the
+        //      pairs (1,0), (3,2)) on CUDA cores in fp32, for 32 -> 64 on the tensor
+        //      cores (fp16 operands, fp32 accumulation).  T diag(beta) goes to TPV in
+        //      fp16 (K-major, rows 0..63) block by block.
         auto put_t = [&](int rr, int col, float t) {
             *reinterpret_cast<__half*>(sm + Sm::TPV + sw128_offset(rr, col * 2)) = __float2half_rn(t * s_beta[col]);
         };
@@ -556,13 +560,15 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 #pragma unroll
                 for (int k = 0; k < j; ++k) acc4[k & 3] -= av[k] * x[k];
                 x[j] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                *reinterpret_cast<__half*>(sm + Sm::DH + sw128_offset(base + j, (base + cc) * 2)) = __float2half_rn(x[j]);
+                reinterpret_cast<float*>(sm + Sm::DF)[b * 272 + j * 17 + cc] = x[j];
+                *reinterpret_cast<__half*>(sm + Sm::T1H + sw128_offset(base + j, (base + cc) * 2)) = __float2half_rn(x[j]);
                 put_t(base + j, base + cc, x[j]);
             }
-        } else {           // zero chunks: D off its diagonal blocks, T diag(beta) above them
+        } else {           // zero chunks: T1 off its diagonal and level-1 blocks, T diag(beta) above the diagonal
             for (int o = tid - 64; o < 64 * 8; o += 192) {
                 const int rr = o >> 3, c16 = o & 7, blk = c16 >> 1, rb = rr >> 4;
-                if (blk != rb) *reinterpret_cast<uint4*>(sm + Sm::DH + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
+                const bool l1 = (rb == 1 && blk == 0) || (rb == 3 && blk == 2);
+                if (blk != rb && !l1) *reinterpret_cast<uint4*>(sm + Sm::T1H + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
                 if (blk > rb) *reinterpret_cast<uint4*>(sm + Sm::TPV + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
@@ -603,36 +609,39 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                 }
             }
         };
-        // level 1: X = A_L1 D, Y = D X; T_10 = -Y_10, T_32 = -Y_32; T1 = D + those blocks
-        if (!level_mma(Sm::AH1, Sm::DH)) return false;
-        store_x(Sm::XH);
-        if (!level_mma(Sm::DH, Sm::XH)) return false;
-        if (row < 64) {
-            const int b = row >> 4;
-            float v[32];
-            tmem_ld32_sync(tmem + lane_base + 32 * hc, v);
+        // level 1 (CUDA cores, fp32): X_p = A_{2p+1,2p} D_{2p}, T_{2p+1,2p} = -D_{2p+1} X_p
+        //      for p = 0, 1; two entries of one row per thread
+        __syncthreads();   // D and A's level-1 blocks are complete
+        {
+            const int pp = tid >> 7, i = (tid & 127) >> 3, j0 = (tid & 7) * 2;
+            const float* af = reinterpret_cast<const float*>(sm + Sm::AF) + pp * 272 + i * 17;
+            const float* d0 = reinterpret_cast<const float*>(sm + Sm::DF) + (2 * pp) * 272 + j0;
+            float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-            for (int i8 = 0; i8 < 4; ++i8) {
-                const int col = 32 * hc + 8 * i8, cb = col >> 4;
-                const bool l1 = (b == 1 && cb == 0) || (b == 3 && cb == 2);
-                const uint32_t off = sw128_offset(row, col * 2);
-                uint4 d = *reinterpret_cast<const uint4*>(sm + Sm::DH + off);
-                if (l1) {
-                    __align__(16) __half t1[8], tb[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        t1[e] = __float2half_rn(-v[8 * i8 + e]);
-                        tb[e] = __float2half_rn(-v[8 * i8 + e] * s_beta[col + e]);
-                    }
-                    d = *reinterpret_cast<const uint4*>(t1);
-                    *reinterpret_cast<uint4*>(sm + Sm::TPV + off) = *reinterpret_cast<const uint4*>(tb);
-                }
-                *reinterpret_cast<uint4*>(sm + Sm::T1H + off) = d;
+            for (int m = 0; m < 16; ++m) {
+                x0 = fmaf(af[m], d0[m * 17], x0);
+                x1 = fmaf(af[m], d0[m * 17 + 1], x1);
             }
+            float* xf = reinterpret_cast<float*>(sm + Sm::XF) + pp * 272 + i * 17 + j0;
+            xf[0] = x0;
+            xf[1] = x1;
+            __syncthreads();
+            const float* d1 = reinterpret_cast<const float*>(sm + Sm::DF) + (2 * pp + 1) * 272 + i * 17;
+            const float* xc = reinterpret_cast<const float*>(sm + Sm::XF) + pp * 272 + j0;
+            float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                t0 = fmaf(d1[m], xc[m * 17], t0);
+                t1 = fmaf(d1[m], xc[m * 17 + 1], t1);
+            }
+            const int rr = 16 * (2 * pp + 1) + i, cc = 16 * (2 * pp) + j0;
+            *reinterpret_cast<__half2*>(sm + Sm::T1H + sw128_offset(rr, cc * 2)) = __floats2half2_rn(-t0, -t1);
+            put_t(rr, cc, -t0);
+            put_t(rr, cc + 1, -t1);
         }
         // level 2: X = A_L2 T1, Y = T1 X; T[32:64, 0:32] = -Y[32:64, 0:32]
         if (!level_mma(Sm::AH2, Sm::T1H)) return false;
-        // AH1, AH2 and DH are dead: the next item's log-decay boxes past V come in
+        // AF, XF, AH2 and DF are dead: the next item's log-decay boxes past V come in
         if (tid == kCopyThread && nc >= 0) issue_la(nh, ntok0, it + 1, true);
         store_x(Sm::XH);
         if (!level_mma(Sm::T1H, Sm::XH)) return false;
