@@ -104,6 +104,12 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
  *              pass, see kda_chunk_fwd_plan), 256-byte aligned; its contents
  *              on entry do not matter.  Calls that share one workspace must be
  *              ordered on one stream.
+ *
+ * Numerics: every product runs on the tensor cores with fp32 accumulation.
+ * bf16 inputs use fp16 operands (tf32 where a factor can leave the fp16
+ * range); fp32 inputs use split tf32 (each operand as a tf32 high part plus an
+ * fp32 remainder, three products), about 2e-6 max-relative error against the
+ * fp64 recurrence on the documented workloads.
  */
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
                          const float* log_alpha, const float* beta,
