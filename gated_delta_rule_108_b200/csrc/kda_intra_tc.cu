@@ -18,8 +18,8 @@
 // memory instead of 64 KB of shared memory, takes the log-decay tile in a
 // 128-byte-swizzled layout that both the per-channel scan and the per-row
 // element pass read without bank conflicts, and loads v only after the element
-// pass.  That brings a CTA to about 99 KB of shared memory, 256 TMEM columns
-// and 128 registers per thread, so two CTAs share each SM and one item's
+// pass.  That brings a CTA to about 108 KB of shared memory, 256 TMEM columns
+// and at most 128 registers per thread, so two CTAs share each SM and one item's
 // latency-bound phases (the (I + A)^{-1} solve, the TMEM round trips, the
 // copies) overlap the other CTA's work.
 //
