@@ -644,6 +644,7 @@ def run_ours(args):
                 os.environ["KDA_CHUNK_PATH"] = old_path
         summ_f = chunk_summary(r, world, peaks, peak_kind)
         summ_f["form"] = "fused single pass (forced; kernels_ms.intra_chunk is the whole pass)"
+        summ_f["roofline"]["traffic"] = None   # the committed capture is of the split form's kernel
         extras[name.lower() + "_fused"] = summ_f
         del r
         torch.cuda.empty_cache()
