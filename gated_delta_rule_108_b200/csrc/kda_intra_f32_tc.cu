@@ -52,7 +52,8 @@ struct F32K1Smem {
     static constexpr int LDV = DV + 4;                  // 16-byte accesses by one thread per row
     static constexpr int LDA = kChunk + 1;              // and scalar ones along a column
     // BIG, reused through an item:
-    //   item start: this item's k and q rows ([64][LDK] each), copied in at the end of the previous item
+    //   item start: this item's k and q rows ([64][DK] each, 16-byte chunks XOR-swizzled by row
+    //     within 128 bytes), copied in at the end of the previous item
     //   element pass .. MMA1: K-m (hi | lo) at KB, token-major, K = channel, DK/32 tiles of
     //     64 rows x 128 B (strong-decay chunks: raw k and q [64][DK] there instead), and
     //     K~^T (hi | lo) at KTT, channel-major, 2 tiles (tokens 0..31, 32..63) of DK rows x 128 B
@@ -64,7 +65,7 @@ struct F32K1Smem {
     static constexpr uint32_t KTT = KB + KB_BYTES;
     static constexpr uint32_t KTT_BYTES = DK * 512u;
     static constexpr uint32_t BIG_BYTES = KB_BYTES + KTT_BYTES;
-    static constexpr uint32_t KQ_Q = 64u * LDK * 4u;     // q staging, after k's
+    static constexpr uint32_t KQ_Q = 64u * DK * 4u;      // q staging, after k's
     static constexpr uint32_t G = BIG_BYTES;             // log-decay (copied in early), then g (base 2): [64][LDK]
     static constexpr uint32_t AM = G + 64u * LDK * 4u;   // A (beta-scaled, strictly lower), then P [64][LDA]
     static constexpr uint32_t VS = AM + 64u * LDA * 4u;  // v [64][LDV] (copied in at the item's start)
@@ -74,7 +75,7 @@ struct F32K1Smem {
     static constexpr uint32_t LAH = BETA + 256u;         // per-head log-decay [64]
     static constexpr uint32_t END = LAH + 256u;
     static_assert(KB % 1024 == 0 && KTT % 1024 == 0, "operand tiles are 1024-byte aligned");
-    static_assert(2u * 64u * LDK * 4u <= BIG_BYTES, "k, q staging fits");
+    static_assert(2u * 64u * DK * 4u <= KB_BYTES, "k, q staging lies clear of K~^T");
     static_assert(US + 64u * LDV * 4u <= VS + 64u * LDV * 4u, "W, U0 staging fits");
     static_assert(64u * LDA * 4u + 3u * 16u * 17u * 4u <= KB_BYTES, "T and its partial products fit in K-m's space");
     static_assert(END + 1024 <= 232448, "shared memory");
@@ -145,6 +146,9 @@ intra_chunk_f32_tc_kernel(const float* __restrict__ q, const float* __restrict__
             cp_async16(dst + r * ld + c4, src + (size_t)(tok0 + (r < L ? r : 0)) * stride + c4, r < L ? 16u : 0u);
         }
     };
+    // float offset of the 16-byte chunk holding channels [4 lc, 4 lc + 4) of row r in the
+    // staged k / q (chunks XOR-swizzled by r mod 8 within each 128-byte group)
+    auto kq_off = [](int r, int lc) { return r * DK + (((lc & ~7) | ((lc & 7) ^ (r & 7))) << 2); };
     auto locate = [&](int w, int& h, int& tok0, int& L) {
         const int c = w / H;
         h = w - c * H;
@@ -168,8 +172,13 @@ intra_chunk_f32_tc_kernel(const float* __restrict__ q, const float* __restrict__
     auto prefetch_kq = [&](int w) {
         int h, tok0, L;
         locate(w, h, tok0, L);
-        copy_rows(reinterpret_cast<float*>(sm), LDK, k + (size_t)h * DK, rowk, DK / 4, tok0, L);
-        copy_rows(reinterpret_cast<float*>(sm + Sm::KQ_Q), LDK, q + (size_t)h * DK, rowk, DK / 4, tok0, L);
+        for (int idx = tid; idx < 64 * (DK / 4); idx += 256) {
+            const int r = idx / (DK / 4), lc = idx - r * (DK / 4);
+            const size_t so = (size_t)(tok0 + (r < L ? r : 0)) * rowk + (size_t)h * DK + 4 * lc;
+            const uint32_t nb = r < L ? 16u : 0u;
+            cp_async16(reinterpret_cast<float*>(sm) + kq_off(r, lc), k + so, nb);
+            cp_async16(reinterpret_cast<float*>(sm + Sm::KQ_Q) + kq_off(r, lc), q + so, nb);
+        }
         cp_async_commit();
     };
     if ((int)blockIdx.x < total) {
@@ -201,10 +210,10 @@ intra_chunk_f32_tc_kernel(const float* __restrict__ q, const float* __restrict__
         __syncthreads();
         float xa[DK / 2];
         {
-            const float* src = reinterpret_cast<const float*>(sm + (is_k ? 0u : Sm::KQ_Q)) + r_el * LDK + hc * (DK / 2);
+            const float* src = reinterpret_cast<const float*>(sm + (is_k ? 0u : Sm::KQ_Q));
 #pragma unroll
             for (int j = 0; j < DK / 2; j += 4) {
-                const float4 a = *reinterpret_cast<const float4*>(src + j);
+                const float4 a = *reinterpret_cast<const float4*>(src + kq_off(r_el, (hc * (DK / 2) + j) >> 2));
                 xa[j] = a.x; xa[j + 1] = a.y; xa[j + 2] = a.z; xa[j + 3] = a.w;
             }
         }
@@ -244,7 +253,7 @@ intra_chunk_f32_tc_kernel(const float* __restrict__ q, const float* __restrict__
 #pragma unroll 4
             for (int idx = tid; idx < 64 * (DK / 4); idx += 256) {
                 const int r = idx / (DK / 4), c4 = (idx - r * (DK / 4)) * 4;
-                const float4 qq = *reinterpret_cast<const float4*>(qs + r * LDK + c4);
+                const float4 qq = *reinterpret_cast<const float4*>(qs + kq_off(r, c4 >> 2));
                 const float4 gg = *reinterpret_cast<const float4*>(g + r * LDK + c4);
                 *reinterpret_cast<float4*>(rec + R::WQ + (size_t)(64 + r) * DK + c4) =
                     make_float4(qq.x * ex2_approx(gg.x), qq.y * ex2_approx(gg.y), qq.z * ex2_approx(gg.z),
@@ -252,7 +261,33 @@ intra_chunk_f32_tc_kernel(const float* __restrict__ q, const float* __restrict__
             }
             if (tid < DK) rec[R::GC + tid] = ex2_approx(gend[tid]);
         }
-        const bool strong = __syncthreads_or(wide);   // k and q are read: BIG is free
+        // ---- from the staged k, by all threads (warp = 32 consecutive tokens of one
+        //      quarter of the channels): the record K^ = k e^{g_{L-1} - g} transposed
+        //      and K~ = k e^{g} -> K~^T (hi | lo), MMA2's B operand; a warp fills 128
+        //      contiguous bytes of a channel row in both
+        {
+            const float* ks = reinterpret_cast<const float*>(sm);
+            const int r = 32 * (warp & 1) + lane, cq = warp >> 1;
+            const uint32_t ktt_lo = 2u * DK * 128u;
+#pragma unroll 2
+            for (int c4 = cq * (DK / 4); c4 < (cq + 1) * (DK / 4); c4 += 4) {
+                const float4 kk = *reinterpret_cast<const float4*>(ks + kq_off(r, c4 >> 2));
+                const float4 gg = *reinterpret_cast<const float4*>(g + r * LDK + c4);
+                const float4 ge = *reinterpret_cast<const float4*>(gend + c4);
+                const float kv[4] = {kk.x, kk.y, kk.z, kk.w}, gv[4] = {gg.x, gg.y, gg.z, gg.w};
+                const float gev[4] = {ge.x, ge.y, ge.z, ge.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    rec[R::KHT + (size_t)(c4 + e) * kChunk + r] = kv[e] * ex2_approx(gev[e] - gv[e]);
+                    float hi, lo;
+                    split_tf32(kv[e] * ex2_approx(gv[e]), hi, lo);
+                    const uint32_t off = (uint32_t)(r >> 5) * (DK * 128u) + sw128_offset(c4 + e, (r & 31) * 4);
+                    *reinterpret_cast<float*>(sm + Sm::KTT + off) = hi;
+                    *reinterpret_cast<float*>(sm + Sm::KTT + ktt_lo + off) = lo;
+                }
+            }
+        }
+        const bool strong = __syncthreads_or(wide);   // k and q are read: their space is free
 
         // ---- element pass: thread = token row (K rows on lanes 0..63, Q rows on
         //      64..127), channels [hc DK/2, hc DK/2 + DK/2) in groups of 8
@@ -260,7 +295,6 @@ intra_chunk_f32_tc_kernel(const float* __restrict__ q, const float* __restrict__
             const int r = r_el;
             float* kraw = reinterpret_cast<float*>(sm + Sm::KB);   // strong: raw k, then raw q
             const uint32_t kb_lo = (DK / 32) * 8192u;
-            const uint32_t ktt_lo = 2u * DK * 128u;
 #pragma unroll
             for (int j = 0; j < DK / 2; j += 8) {
                 const int c8 = hc * (DK / 2) + j;
@@ -270,22 +304,6 @@ intra_chunk_f32_tc_kernel(const float* __restrict__ q, const float* __restrict__
                     x[e] = xa[j + e];
                     gr[e] = g[r * LDK + c8 + e];
                     gm[e] = gmid[c8 + e];
-                }
-                if (is_k) {
-                    // record K^ = k e^{g_{L-1} - g}, transposed: a warp's 32 tokens
-                    // fill 128 contiguous bytes of each channel row
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        rec[R::KHT + (size_t)(c8 + e) * kChunk + r] = x[e] * ex2_approx(gend[c8 + e] - gr[e]);
-                    // K~ = k e^{g} -> K~^T (hi | lo), MMA2's B operand
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        float hi, lo;
-                        split_tf32(x[e] * ex2_approx(gr[e]), hi, lo);
-                        const uint32_t off = (uint32_t)(r >> 5) * (DK * 128u) + sw128_offset(c8 + e, (r & 31) * 4);
-                        *reinterpret_cast<float*>(sm + Sm::KTT + off) = hi;
-                        *reinterpret_cast<float*>(sm + Sm::KTT + ktt_lo + off) = lo;
-                    }
                 }
                 if (!strong) {
                     // K~m = k e^{g - g_m} | Q~m = q e^{g - g_m} -> TMEM (hi | lo), MMA1's A operand
