@@ -1,9 +1,10 @@
-// kda_chunk_tc.cu -- chunkwise KDA forward on the sm_100a tensor cores
-// (tcgen05 + TMEM, TMA / bulk-copy fed) for bf16 inputs.
+// kda_chunk_tc.cu -- the backward of the chunkwise KDA forward on the sm_100a
+// tensor cores (tcgen05 + TMEM, TMA / bulk-copy fed) for bf16 inputs, and the
+// host side of the bf16 chunk kernels.
 //
-// The chunk algebra is the one of kda_chunk_simt.cu (unrolling the daiw.net
-// update equation, section "KDA 的更新式", over chunks of 64 tokens; chunk-wise
-// parallel form of the kongchang.com page, section "硬件效率的优化策略"):
+// The forward's chunk algebra (unrolling the daiw.net update equation, section
+// "KDA 的更新式", over chunks of 64 tokens; chunk-wise parallel form of the
+// kongchang.com page, section "硬件效率的优化策略"):
 //
 //   A_{ri} = beta_r <k_r e^{g_r-g_m}, k_i e^{g_m-g_i}>  (i < r),  T = (I + A)^{-1}
 //   P_{ri} =        <q_r e^{g_r-g_m}, k_i e^{g_m-g_i}>  (i <= r)
@@ -11,23 +12,16 @@
 //   K^ = k e^{g_{L-1} - g},        gC = e^{g_{L-1}}
 //   U = U0 - W S,   O = dk^{-1/2} (Q~ S + P U),   S' = Diag(gC) S + K^^T U
 //
-// K1 intra_chunk_tc (one CTA per (chunk, head), all chunks in parallel):
-//   TMA loads q, k, v (bf16, 128-byte swizzled) and log_alpha (fp32) of the
-//   chunk; one thread per key channel forms the cumulative decay and the
-//   decayed operands; a tf32 MMA gives [A; P] = [K~m; Q~m] K-m^T in TMEM; T is
-//   formed by forward substitution (one column per thread); an fp16 MMA gives
-//   [W | U0] = T diag(beta) [K~ | V].  The chunk's intermediates go to the
-//   workspace in fp16, already laid out as the operand tiles K2's MMAs read.
-// K2 inter_chunk_tc (one CTA per (sequence, head, 64-wide value slice),
-//   serial over the sequence's chunks): the fp32 state slice lives in TMEM
-//   for the whole sequence; each chunk's intermediates arrive by bulk copy into
-//   a double buffer; per chunk three MMA groups: [W; Q~] S, then
-//   [*; P] U and K^^T U accumulated onto the TMEM accumulators.
+// The forward kernels are in kda_intra_tc.cu and kda_inter_tc.cu; in backward
+// mode they also write what the kernels here read: fp16 tiles of T, K~ and V,
+// the fp32 M = K_l K_r^T and a strong-decay flag per (head, chunk) (BwdTiles),
+// and the fp32 state entering each chunk.  Here: the reversed chunk chain
+// (KB3), then per (chunk, head) the products over the value dimension, the
+// products through T, W and U0, and the split-factor products with the
+// per-channel gradients (see each section).
 //
-// Precision: tf32 operands (rounded to nearest) for A and P, whose factors can
-// exceed the fp16 range; fp16 (10-bit mantissa, like tf32) for every other
-// operand and intermediate, all accumulation in fp32.  fp16 values above 65000
-// in magnitude set KDA_ERR_RANGE in the workspace status.
+// Precision: fp16 operands (10-bit mantissa) where the values stay in its range,
+// tf32 where a factor e^{+-(g - g_m)} can leave it; fp32 accumulation.
 //
 // All waits are bounded (about one second of SM clock); a CTA that gives up
 // records KDA_ERR_TIMEOUT, waits (bounded) for its own outstanding MMAs and
@@ -49,873 +43,21 @@ namespace {
 
 using namespace ptx;
 
-// ---------------------------------------------------------------- K1 ----
-// Persistent: one CTA per SM walks the (chunk, head) work items.  The k, v, q
-// tiles of the next item are TMA-loaded into the other half of a double
-// buffer, and its log_alpha / beta are loaded into registers, while the
-// current item is being computed.
-template <int DK, int DV>
-struct K1Smem {
-    static constexpr uint32_t TILE = 8192;                          // 64 tokens x 128 bytes
-    static constexpr uint32_t STAGE = (2 * (DK / 64) + DV / 64) * TILE;
-    static constexpr uint32_t KS = 0;                               // + stage * STAGE: k tiles (-> fp16 K~)
-    static constexpr uint32_t VS = (DK / 64) * TILE;                //                  v tiles (-> fp16 V)
-    static constexpr uint32_t QS = VS + (DV / 64) * TILE;           //                  q tiles (-> fp16 Q~)
-    static constexpr uint32_t G = 2 * STAGE;                        // cumulative log-decay [64][DK] fp32
-    static constexpr uint32_t OPA = G + 64 * DK * 4;                // tf32 [K~m; Q~m]: DK/32 tiles of 16 KB
-    static constexpr uint32_t OPB = OPA + (DK / 32) * 16384;        // tf32 K-m: DK/32 tiles of 8 KB
-    static constexpr uint32_t OPB_END = OPB + (DK / 32) * 8192;
-    // after MMA1 (OPA/OPB dead): A, T (fp32, 64 x 68) and the E blocks (6 x 16 x 17)
-    // in OPA when it is large enough, else in an extra region
-    static constexpr uint32_t SCR_BYTES = 2 * 64 * 68 * 4 + 6 * 16 * 17 * 4;
-    static constexpr bool SCR_IN_OPA = (DK / 32) * 16384 >= SCR_BYTES;
-    static constexpr uint32_t AM = SCR_IN_OPA ? OPA : OPB_END;
-    static constexpr uint32_t TM = AM + 64 * 68 * 4;
-    static constexpr uint32_t YM = TM + 64 * 68 * 4;
-    static constexpr uint32_t END = SCR_IN_OPA ? OPB_END : OPB_END + SCR_BYTES;
-    // after MMA1: T diag(beta) fp16, K-major 128 rows x 64 tokens, in OPB
-    static constexpr uint32_t TP = OPB;
-    static constexpr uint32_t TX_BYTES = STAGE;
-    static constexpr uint32_t LA_BYTES = 64 * DK * 4;               // log_alpha tile into G
-    // small per-item arrays after END (no static shared memory, so the
-    // dynamic window starts 1024-byte aligned)
-    static constexpr uint32_t BAR = END;                            // 4 mbarriers
-    static constexpr uint32_t TMEMADDR = BAR + 32;   // after bar_load[2], bar_mma, bar_la
-    static constexpr uint32_t BETA = TMEMADDR + 16;                 // [64]
-    static constexpr uint32_t GM = BETA + 256;                      // [DK] g_m, e^{g_m}, e^{g_{L-1}-g_m}
-    static constexpr uint32_t EGM = GM + DK * 4;
-    static constexpr uint32_t EGLM = EGM + DK * 4;
-    static constexpr uint32_t LAH = EGLM + DK * 4;                  // [64] per-head log-decay
-    static constexpr uint32_t TOTAL = LAH + 256;
-    // cumulative-sum partials live in the (then unused) T-solve scratch
-    static constexpr uint32_t PART = YM;
-    static_assert(YM + 6 * 16 * 17 * 4 <= END, "T-solve scratch");
-    static_assert(PART + (256 / DK) * DK * 4 <= END, "partials alias");
-    static_assert((DK / 32) * 8192 >= 16384, "T diag(beta) in OPB");
-    static_assert(TOTAL <= 232448, "shared memory");
-};
-
-template <int DK, int DV, int GATE>
-__global__ void __launch_bounds__(256, 1)
-intra_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_la,
-                      const float* __restrict__ log_alpha_head, const float* __restrict__ beta,
-                      ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
-                      size_t max_chunks, long long wait_cap, int drop_la,
-                      unsigned char* __restrict__ bwd_tiles, int* __restrict__ bwd_flags)
-{
-    using Sm = K1Smem<DK, DV>;
-    using R = TcRec<DK, DV>;
-    constexpr int NPART = 256 / DK;       // threads per key channel in the cumulative sum
-    constexpr int TPP = kChunk / NPART;   // tokens per such thread
-    constexpr int NCH8 = DK / 8;          // 8-channel (16-byte bf16) groups per token row
-    extern __shared__ __align__(1024) unsigned char sm[];
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + Sm::BAR);   // [2]
-    uint64_t& bar_mma = bar_load[2];
-    uint64_t& bar_la = bar_load[3];
-    uint32_t& s_tmem = *reinterpret_cast<uint32_t*>(sm + Sm::TMEMADDR);
-    float* s_beta = reinterpret_cast<float*>(sm + Sm::BETA);
-    float* s_gm = reinterpret_cast<float*>(sm + Sm::GM);
-    float* s_egm = reinterpret_cast<float*>(sm + Sm::EGM);
-    float* s_eglm = reinterpret_cast<float*>(sm + Sm::EGLM);
-    float* s_lah = reinterpret_cast<float*>(sm + Sm::LAH);
-    float* s_part = reinterpret_cast<float*>(sm + Sm::PART);        // [NPART][DK]
-
-    if (hdr->status != kStatusOk) return;
-    const int total = hdr->num_chunks * H;
-    if ((int)blockIdx.x >= total) return;
-    if ((smem_u32(sm) & 1023u) != 0) {   // the swizzled layouts need 1024-byte alignment
-        if (threadIdx.x == 0) flag_error(hdr, kStatusInternal);
-        return;
-    }
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int ch = tid % DK, part = tid / DK, r0 = part * TPP;   // cumulative-sum mapping
-
-    if (tid == 0) {
-        mbar_init(&bar_load[0], 1);
-        mbar_init(&bar_load[1], 1);
-        mbar_init(&bar_mma, 1);
-        mbar_init(&bar_la, 1);
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&s_tmem, 256);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    const uint32_t R1 = tmem;   // [A; P] 128 lanes x 64 columns, then [W | U0] 128 x (DK + DV)
-    const uint32_t R2 = tmem;
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const int wg = warp >> 2;
-
-    // work item w -> (chunk, head); consecutive items are heads of one chunk
-    auto locate = [&](int w, int& c, int& h, int& tok0, int& L) {
-        c = w / H;
-        h = w - c * H;
-        int seq;
-        map.locate(c, seq, tok0, L);
-    };
-    auto issue_tma = [&](int w, int stage) {
-        int c, h, tok0, L;
-        locate(w, c, h, tok0, L);
-        unsigned char* st = sm + stage * Sm::STAGE;
-        mbar_arrive_expect_tx(&bar_load[stage], Sm::TX_BYTES);
-#pragma unroll
-        for (int b = 0; b < DK / 64; ++b) tma_load_3d(st + Sm::KS + b * Sm::TILE, &tm_k, &bar_load[stage], b * 64, h, tok0);
-#pragma unroll
-        for (int b = 0; b < DV / 64; ++b) tma_load_3d(st + Sm::VS + b * Sm::TILE, &tm_v, &bar_load[stage], b * 64, h, tok0);
-#pragma unroll
-        for (int b = 0; b < DK / 64; ++b) tma_load_3d(st + Sm::QS + b * Sm::TILE, &tm_q, &bar_load[stage], b * 64, h, tok0);
-    };
-    // per-channel gate: log_alpha tile of item w into G (when G is free), by TMA
-    constexpr bool channel_gate = GATE == kGateChannel;
-    auto issue_la = [&](int w) {
-        if constexpr (!channel_gate) return;
-        int c, h, tok0, L;
-        locate(w, c, h, tok0, L);
-        mbar_arrive_expect_tx(&bar_la, Sm::LA_BYTES);
-        tma_load_3d(sm + Sm::G, &tm_la, &bar_la, 0, h, tok0);
-    };
-    // beta (and a per-head log-decay) of item w into registers, threads
-    // 192..255, one token each
-    float beta_next = 0.f, lah_next = 0.f;
-    auto load_beta = [&](int w) {
-        if (tid >= 192) {
-            int c, h, tok0, L;
-            locate(w, c, h, tok0, L);
-            const int r = tid - 192;
-            beta_next = (r < L) ? ld_prefetch_f32(beta + (size_t)(tok0 + r) * H + h) : 0.f;
-            lah_next = (GATE == kGateHead && r < L) ? ld_prefetch_f32(log_alpha_head + (size_t)(tok0 + r) * H + h) : 0.f;
-        }
-    };
-
-    // test hook: CTA 0 can leave out the log-decay copy of its third item (of
-    // its last one if it has fewer), so that the bounded wait on it gives up
-    // with the item's tile copies already waited for and the drain after the
-    // abort starting past phase 0
-    const int drop_it = (drop_la && blockIdx.x == 0) ? min(2, (total - 1) / (int)gridDim.x) : -1;
-    if (tid == 0) {
-        issue_tma(blockIdx.x, 0);
-        if (drop_it != 0) issue_la(blockIdx.x);
-    }
-    load_beta(blockIdx.x);
-    bool aborted = false;
-    uint32_t mma_phase = 0;
-    int mma_pending = 0;      // commits issued on bar_mma not yet waited for
-    // This CTA's items are numbered by iteration j; item j's tiles land on
-    // bar_load[j & 1] (phase parity (j >> 1) & 1) and its log-decay tile on
-    // bar_la (parity j & 1).  Items loads_done .. loads_issued - 1 have copies
-    // issued but not yet waited for (drained on abort).
-    int loads_issued = 1, loads_done = 0;
-    bool stored = false;      // the copy thread has bulk stores in flight
-    bool tstored = false;     // kTileThread has bulk stores in flight (backward mode)
-    float range_max = 0.f;
-
-    int it = 0;
-    for (int w = blockIdx.x; w < total && !aborted; w += gridDim.x, ++it) {
-        const int stage = it & 1;
-        unsigned char* st = sm + stage * Sm::STAGE;
-        int c, h, tok0, L;
-        locate(w, c, h, tok0, L);
-        unsigned char* rec = records + ((size_t)h * max_chunks + c) * R::BYTES;
-        unsigned char* btile = bwd_tiles ? bwd_tiles + ((size_t)h * max_chunks + c) * BwdTiles<DK, DV>::BYTES : nullptr;
-        if (tid >= 192) {
-            s_beta[tid - 192] = beta_next;
-            if constexpr (GATE == kGateHead) s_lah[tid - 192] = lah_next;
-        }
-
-        const int wn = w + gridDim.x;   // this CTA's next item
-        if (wn < total) load_beta(wn);
-
-        // ---- cumulative log-decay, in place over the log_alpha tile in G -------
-        float* g = reinterpret_cast<float*>(sm + Sm::G);   // [64][DK]
-        const bool ok_la = !channel_gate || mbar_wait_cycles(&bar_la, it & 1, wait_cap);
-        const bool ok_load = mbar_wait_cycles(&bar_load[stage], (it >> 1) & 1, wait_cap);
-        if (__syncthreads_or(!(ok_la && ok_load))) { aborted = true; break; }
-        loads_done = it + 1;
-        {
-            float la_cur[TPP];
-            float acc = 0.f;
-#pragma unroll
-            for (int i = 0; i < TPP; ++i) {
-                if constexpr (channel_gate) la_cur[i] = (r0 + i < L) ? g[(r0 + i) * DK + ch] : 0.f;
-                else if constexpr (GATE == kGateHead) la_cur[i] = (r0 + i < L) ? s_lah[r0 + i] : 0.f;
-                else la_cur[i] = 0.f;   // no gate: alpha = 1
-                acc += la_cur[i];
-            }
-            s_part[part * DK + ch] = acc;
-            __syncthreads();
-            acc = 0.f;
-            for (int p = 0; p < part; ++p) acc += s_part[p * DK + ch];
-#pragma unroll
-            for (int i = 0; i < TPP; ++i) {
-                acc += la_cur[i];
-                g[(r0 + i) * DK + ch] = acc * kLog2e;   // base 2
-            }
-        }
-        __syncthreads();
-        bool wide = false;   // this channel's decay within the chunk too strong for the split factors
-        if (tid < DK) {
-            const float gm = g[((L - 1) >> 1) * DK + tid], gl = g[(L - 1) * DK + tid];   // base 2
-            s_gm[tid] = gm;
-            s_egm[tid] = ex2_approx(gm);
-            s_eglm[tid] = ex2_approx(gl - gm);
-            reinterpret_cast<float*>(rec + R::GC)[tid] = exp2f(gl);
-            wide = fmaxf(g[tid] - gm, gm - gl) > kMaxSplitExponent2;
-        }
-        // Strong decay: the factors e^{+-(g - g_m)} of A and P could overflow, so
-        // this chunk forms A and P exactly (slow path, no MMA1).
-        const bool strong = __syncthreads_or(wide);
-        if (strong) {
-            float* am = reinterpret_cast<float*>(sm + Sm::AM);
-            exact_a_p<DK>([&](int r, int c) { return g[r * DK + c]; }, st + Sm::KS, st + Sm::QS, s_beta, L, am,
-                          rec + R::P);
-            __syncthreads();   // the k, q tiles are converted in place next
-        }
-
-        // ---- decayed operands: thread -> token row r = tid / 4, 8-channel groups
-        //      c8 = 8 (tid % 4) + 32 k; two neighbouring rows share an 8-thread
-        //      store phase and their swizzles differ, so the fp32 stores are
-        //      bank-conflict free
-        auto element_pass = [&](auto strong_tag) {
-            constexpr bool STRONG = decltype(strong_tag)::value;
-        {
-            const int r = tid >> 2;
-            const bool live = r < L;
-            constexpr int KUNROLL = STRONG ? 1 : DK / 32;   // keep the rare path small
-#pragma unroll KUNROLL
-            for (int k = 0; k < DK / 32; ++k) {
-                const int c8 = 8 * (tid & 3) + 32 * k;
-                const uint32_t ho = (c8 >> 6) * Sm::TILE + sw128_offset(r, (c8 & 63) * 2);   // 16-byte chunk
-                uint4 kraw = *reinterpret_cast<const uint4*>(st + Sm::KS + ho);
-                uint4 qraw = *reinterpret_cast<const uint4*>(st + Sm::QS + ho);
-                if (!live) { kraw = make_uint4(0, 0, 0, 0); qraw = kraw; }
-                const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(&kraw);
-                const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(&qraw);
-                const float4 g0 = *reinterpret_cast<const float4*>(g + r * DK + c8);
-                const float4 g1 = *reinterpret_cast<const float4*>(g + r * DK + c8 + 4);
-                const float4 m0 = *reinterpret_cast<const float4*>(s_gm + c8);
-                const float4 m1 = *reinterpret_cast<const float4*>(s_gm + c8 + 4);
-                const float4 x0 = *reinterpret_cast<const float4*>(s_egm + c8);
-                const float4 x1 = *reinterpret_cast<const float4*>(s_egm + c8 + 4);
-                const float4 y0 = *reinterpret_cast<const float4*>(s_eglm + c8);
-                const float4 y1 = *reinterpret_cast<const float4*>(s_eglm + c8 + 4);
-                const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                const float gmv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-                const float egmv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                const float eglmv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-                __align__(16) float ka[8], qa[8], kbm[8];
-                __align__(16) __half2 k0[4], q0[4], kh[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    float k0v[2], q0v[2], khv[2];
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const int e = 2 * e2 + h2;
-                        const float kk = __bfloat162float(kb[e]), qq = __bfloat162float(qb[e]);
-                        if constexpr (!STRONG) {
-                            const float d = gv[e] - gmv[e];
-                            const float em = ex2_approx(d);          // e^{g_r - g_m}
-                            const float kem = kk * em, qem = qq * em;
-                            const float keb = kk * ex2_approx(-d);   // k e^{g_m - g_r}
-                            ka[e] = round_tf32_alu(kem);
-                            qa[e] = round_tf32_alu(qem);
-                            kbm[e] = round_tf32_alu(keb);
-                            k0v[h2] = kem * egmv[e];                 // k e^{g_r}
-                            q0v[h2] = qem * egmv[e];                 // q e^{g_r}
-                            khv[h2] = keb * eglmv[e];                // k e^{g_{L-1} - g_r}
-                        } else {                                     // unsplit, every exponent <= 0
-                            const float e0 = ex2_approx(gv[e]);
-                            k0v[h2] = kk * e0;
-                            q0v[h2] = qq * e0;
-                            khv[h2] = kk * ex2_approx(g[(L - 1) * DK + c8 + e] - gv[e]);
-                            ka[e] = qa[e] = kbm[e] = 0.f;
-                        }
-                    }
-                    k0[e2] = __floats2half2_rn(k0v[0], k0v[1]);
-                    q0[e2] = __floats2half2_rn(q0v[0], q0v[1]);
-                    kh[e2] = __floats2half2_rn(khv[0], khv[1]);
-                }
-                // tf32 operands: 8 fp32 = two 16-byte chunks of a 128-byte row
-                const uint32_t fo = (c8 >> 5) * 16384u, fob = (c8 >> 5) * 8192u;
-                const uint32_t fb = (c8 & 31) * 4;
-                if constexpr (!STRONG) {
-                *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(r, fb)) = *reinterpret_cast<const float4*>(ka);
-                *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(r, fb + 16)) = *reinterpret_cast<const float4*>(ka + 4);
-                *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(64 + r, fb)) = *reinterpret_cast<const float4*>(qa);
-                *reinterpret_cast<float4*>(sm + Sm::OPA + fo + sw128_offset(64 + r, fb + 16)) = *reinterpret_cast<const float4*>(qa + 4);
-                *reinterpret_cast<float4*>(sm + Sm::OPB + fob + sw128_offset(r, fb)) = *reinterpret_cast<const float4*>(kbm);
-                *reinterpret_cast<float4*>(sm + Sm::OPB + fob + sw128_offset(r, fb + 16)) = *reinterpret_cast<const float4*>(kbm + 4);
-                }
-                *reinterpret_cast<uint4*>(st + Sm::KS + ho) = *reinterpret_cast<const uint4*>(k0);   // K~ (MMA2 operand)
-                *reinterpret_cast<uint4*>(st + Sm::QS + ho) = *reinterpret_cast<const uint4*>(q0);   // Q~ (record)
-                *reinterpret_cast<uint4*>(rec + R::KH + ho) = *reinterpret_cast<const uint4*>(kh);  // K^ (record)
-            }
-        }
-        };
-        if (strong) element_pass(std::true_type{});
-        else element_pass(std::false_type{});
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && !strong) {
-            // ---- MMA1 (tf32): [K~m; Q~m] K-m^T -> R1 (overlaps the v conversion)
-            tc_fence_after();
-            constexpr uint32_t idesc = instr_desc(kFmtTF32, 128, 64);
-            const uint32_t a0 = smem_u32(sm + Sm::OPA), b0 = smem_u32(sm + Sm::OPB);
-#pragma unroll
-            for (int kb = 0; kb < DK / 32; ++kb)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_tf32(R1, smem_desc(a0 + kb * 16384 + ks * 32, 16, 1024, kLayoutSW128),
-                             smem_desc(b0 + kb * 8192 + ks * 32, 16, 1024, kLayoutSW128), idesc,
-                             (kb | ks) != 0);
-            mma_commit(&bar_mma);
-        }
-        // The copy thread (warp 1) prefetches the next item and stores this
-        // item's Q~ while warp 0 issues MMA1 and warps 2..7 convert v.  It
-        // issues every bulk store of the kernel, so its wait covers them all.
-        if (tid == kCopyThread) {
-            if (wn < total) {
-                // log_alpha into G (free now); k, v, q tiles into the other
-                // stage once the bulk stores of the item that used it have read it
-                if (it + 1 != drop_it) issue_la(wn);
-                if (stored) bulk_store_wait_read();
-                issue_tma(wn, stage ^ 1);
-            }
-            // Q~ tiles are the lower halves (rows 64..127) of the record's WQ tiles
-#pragma unroll
-            for (int b = 0; b < DK / 64; ++b)
-                bulk_store(rec + R::WQ + b * 16384 + 8192, st + Sm::QS + b * Sm::TILE, 8192);
-            bulk_store_commit();
-            stored = true;
-        }
-        if (wn < total) loads_issued = it + 2;   // the copy thread's prefetch above
-        mma_pending = strong ? 0 : 1;
-        // v: bf16 -> fp16 in place, 8 values per thread and step (warps 2..7)
-        for (int item = tid - 64; tid >= 64 && item < kChunk * (DV / 8); item += 192) {
-            const int r = item / (DV / 8), j8 = (item - r * (DV / 8)) * 8;
-            const uint32_t o = Sm::VS + (j8 >> 6) * Sm::TILE + sw128_offset(r, (j8 & 63) * 2);
-            uint4 raw = *reinterpret_cast<const uint4*>(st + o);
-            if (r >= L) raw = make_uint4(0, 0, 0, 0);
-            const __nv_bfloat162* vb = reinterpret_cast<const __nv_bfloat162*>(&raw);
-            __align__(16) __half2 vh[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 x = __bfloat1622float2(vb[e]);
-                range_max = fmaxf(range_max, fmaxf(fabsf(x.x), fabsf(x.y)));
-                vh[e] = __floats2half2_rn(x.x, x.y);
-            }
-            *reinterpret_cast<uint4*>(st + o) = *reinterpret_cast<const uint4*>(vh);
-        }
-        fence_proxy_async_smem();   // fp16 v (MMA2 operand)
-        float* am = reinterpret_cast<float*>(sm + Sm::AM);   // [64][68]
-        float* tmx = reinterpret_cast<float*>(sm + Sm::TM);  // [64][68]
-        float* ym = reinterpret_cast<float*>(sm + Sm::YM);   // [6][16][17]
-        bool ok = true;
-        if (!strong) {
-        ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        mma_phase ^= 1;
-        mma_pending = 0;
-        tc_fence_after();
-
-        // ---- A (rows 0..63, beta-scaled, strictly lower) to smem; P (rows
-        //      64..127, lower incl. diagonal) to the record
-        {
-            float v[32];
-            const int row = (warp & 3) * 32 + (tid & 31);
-            tmem_ld32_sync(R1 + lane_base + 32 * wg, v);
-            if (row < 64) {
-                const float b = s_beta[row];
-#pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    float4 a4;
-                    const int col = 32 * wg + 4 * i4;
-                    a4.x = (col + 0 < row) ? b * v[4 * i4 + 0] : 0.f;
-                    a4.y = (col + 1 < row) ? b * v[4 * i4 + 1] : 0.f;
-                    a4.z = (col + 2 < row) ? b * v[4 * i4 + 2] : 0.f;
-                    a4.w = (col + 3 < row) ? b * v[4 * i4 + 3] : 0.f;
-                    *reinterpret_cast<float4*>(am + row * 68 + col) = a4;
-                    if (btile)   // backward mode: the unweighted M = K_l K_r^T
-                        *reinterpret_cast<float4*>(btile + BwdTiles<DK, DV>::M + (row * 64 + col) * 4) =
-                            make_float4((col + 0 < row) ? v[4 * i4 + 0] : 0.f, (col + 1 < row) ? v[4 * i4 + 1] : 0.f,
-                                        (col + 2 < row) ? v[4 * i4 + 2] : 0.f, (col + 3 < row) ? v[4 * i4 + 3] : 0.f);
-                }
-            } else {
-                const int r = row - 64;
-#pragma unroll
-                for (int i8 = 0; i8 < 4; ++i8) {
-                    __align__(16) __half hv[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int col = 32 * wg + 8 * i8 + e;
-                        hv[e] = __float2half_rn(col <= r ? v[8 * i8 + e] : 0.f);
-                    }
-                    *reinterpret_cast<uint4*>(rec + R::P + sw128_offset(r, (32 * wg + 8 * i8) * 2)) =
-                        *reinterpret_cast<const uint4*>(hv);
-                }
-
-            }
-        }
-        }   // !strong
-        __syncthreads();
-        if (bwd_flags && tid == 0) bwd_flags[(size_t)h * max_chunks + c] = strong ? 1 : 0;   // strong-decay path taken
-        if (btile && tid == kTileThread) {   // backward mode: K~ and fp16 V are final
-#pragma unroll
-            for (int b = 0; b < DK / 64; ++b) bulk_store(btile + BwdTiles<DK, DV>::KT + b * 8192, st + Sm::KS + b * Sm::TILE, 8192);
-#pragma unroll
-            for (int b = 0; b < DV / 64; ++b) bulk_store(btile + BwdTiles<DK, DV>::V + b * 8192, st + Sm::VS + b * Sm::TILE, 8192);
-            bulk_store_commit();
-            tstored = true;
-        }
-
-        // ---- T = (I + A)^{-1} in 16 x 16 blocks, written as fp16 T diag(beta)
-        //      (K-major, rows 0..63) as soon as each block is final.
-        //      D_b = (I + A_bb)^{-1};  E_im = D_i A_im (i > m);
-        //      T_{b+l,b} = -sum_{m=b}^{b+l-1} E_{b+l,m} T_{m,b}
-        auto put_t = [&](int row, int col, float t) {
-            *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(row, col * 2)) = __float2half_rn(t * s_beta[col]);
-        };
-        float* em_ = ym;   // E blocks: 6 x 16 x 17 fp32
-        if (tid < 64) {    // diagonal blocks, one column per thread
-            const int b = tid >> 4, cc = tid & 15, base = 16 * b;
-            float x[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float* arow = am + (base + j) * 68 + base;
-                float av[16];
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(arow + 4 * k4);
-                    av[4 * k4] = t4.x; av[4 * k4 + 1] = t4.y; av[4 * k4 + 2] = t4.z; av[4 * k4 + 3] = t4.w;
-                }
-                float acc4[4] = {(j == cc) ? 1.f : 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int k = 0; k < j; ++k) acc4[k & 3] -= av[k] * x[k];
-                x[j] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                tmx[(base + j) * 68 + base + cc] = x[j];
-                put_t(base + j, base + cc, x[j]);
-            }
-        } else {           // zeros above the diagonal blocks
-            for (int o = tid - 64; o < 6 * 256; o += 192) {
-                const int pair = o >> 8, p = (o >> 4) & 15, q = o & 15;
-                const int i = pair < 3 ? 0 : (pair < 5 ? 1 : 2);
-                const int j = pair < 3 ? pair + 1 : (pair < 5 ? pair - 1 : 3);
-                *reinterpret_cast<__half*>(sm + Sm::TP + sw128_offset(16 * i + p, (16 * j + q) * 2)) = __float2half_rn(0.f);
-            }
-        }
-        __syncthreads();
-        // E_im = D_i A_im for the 6 pairs i > m (pair index: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)),
-        // 2 x 2 outputs per thread
-        for (int o = tid; o < 6 * 64; o += 256) {
-            const int pair = o >> 6, p0 = ((o >> 3) & 7) * 2, q0 = (o & 7) * 2;
-            const int i = pair == 0 ? 1 : (pair < 3 ? 2 : 3);
-            const int m = pair == 0 ? 0 : (pair == 1 ? 0 : (pair == 2 ? 1 : pair - 3));
-            const float* d0 = tmx + (16 * i + p0) * 68 + 16 * i;
-            const float* d1 = d0 + 68;
-            float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float2 a = *reinterpret_cast<const float2*>(am + (16 * i + k) * 68 + 16 * m + q0);
-                const float e0 = d0[k], e1 = d1[k];
-                c00 += e0 * a.x; c01 += e0 * a.y; c10 += e1 * a.x; c11 += e1 * a.y;
-            }
-            float* out = em_ + (pair * 16 + p0) * 17 + q0;
-            out[0] = c00; out[1] = c01; out[17] = c10; out[18] = c11;
-        }
-        __syncthreads();
-        // T_{b+l,b} = -sum_{m=b}^{b+l-1} E_{b+l,m} T_{m,b}, 2 x 2 outputs per thread
-#pragma unroll 1
-        for (int l = 1; l < 4; ++l) {
-            for (int o = tid; o < (4 - l) * 64; o += 256) {
-                const int b = o >> 6, p0 = ((o >> 3) & 7) * 2, q0 = (o & 7) * 2;
-                const int i = b + l, j = b;
-                float c00 = 0.f, c01 = 0.f, c10 = 0.f, c11 = 0.f;
-                for (int m = j; m < i; ++m) {
-                    const int pair = i == 1 ? 0 : (i == 2 ? 1 + m : 3 + m);
-                    const float* e0p = em_ + (pair * 16 + p0) * 17;
-                    const float* e1p = e0p + 17;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float2 t = *reinterpret_cast<const float2*>(tmx + (16 * m + k) * 68 + 16 * j + q0);
-                        const float e0 = e0p[k], e1 = e1p[k];
-                        c00 += e0 * t.x; c01 += e0 * t.y; c10 += e1 * t.x; c11 += e1 * t.y;
-                    }
-                }
-                const int r = 16 * i + p0, cidx = 16 * j + q0;
-                tmx[r * 68 + cidx] = -c00;
-                tmx[r * 68 + cidx + 1] = -c01;
-                tmx[(r + 1) * 68 + cidx] = -c10;
-                tmx[(r + 1) * 68 + cidx + 1] = -c11;
-                put_t(r, cidx, -c00);
-                put_t(r, cidx + 1, -c01);
-                put_t(r + 1, cidx, -c10);
-                put_t(r + 1, cidx + 1, -c11);
-            }
-            __syncthreads();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- MMA2 (fp16): [T diag(beta); *] [K~ | V] -> R2 -----------------
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t idesc = instr_desc(kFmtF16, 128, DK + DV, false, true);
-            const uint32_t a0 = smem_u32(sm + Sm::TP), b0 = smem_u32(st + Sm::KS);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_f16(R2, smem_desc(a0 + ks * 32, 16, 1024, kLayoutSW128),
-                        smem_desc(b0 + ks * 2048, Sm::TILE, 1024, kLayoutSW128), idesc, ks != 0);
-            mma_commit(&bar_mma);
-        }
-        mma_pending = 1;
-        if (btile) {   // backward mode: T = (I + A)^{-1} as an fp16 tile (zero above the diagonal blocks)
-            for (int idx = tid; idx < kChunk * 8; idx += 256) {
-                const int r = idx >> 3, c8 = (idx & 7) * 8;
-                __align__(16) __half hv[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    hv[e] = __float2half_rn(((c8 + e) >> 4) > (r >> 4) ? 0.f : tmx[r * 68 + c8 + e]);
-                *reinterpret_cast<uint4*>(btile + BwdTiles<DK, DV>::T + sw128_offset(r, c8 * 2)) =
-                    *reinterpret_cast<const uint4*>(hv);
-            }
-            // the K~ / V tile stores must have read the stage before W, U0 are staged there
-            if (tid == kTileThread) bulk_store_wait_read();
-        }
-        ok = mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        mma_phase ^= 1;
-        mma_pending = 0;
-        tc_fence_after();
-
-        // ---- W and U0 (rows 0..63): fp16 into the stage's k/v tiles (free after
-        //      MMA2; same 64-row swizzled tile layout as the record), then one
-        //      bulk store per tile.  The two warpgroups take alternate 32-column chunks.
-        if ((warp & 3) < 2) {
-            const int r = (warp & 3) * 32 + (tid & 31);
-#pragma unroll
-            for (int cb = wg; cb < (DK + DV) / 32; cb += 2) {
-                float v[32];
-                tmem_ld32_sync(R2 + lane_base + 32 * cb, v);
-#pragma unroll
-                for (int i8 = 0; i8 < 4; ++i8) {
-                    __align__(16) __half hv[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        range_max = fmaxf(range_max, fabsf(v[8 * i8 + e]));
-                        hv[e] = __float2half_rn(v[8 * i8 + e]);
-                    }
-                    const int col = 32 * cb + 8 * i8;   // k tiles then v tiles, 64 columns each
-                    *reinterpret_cast<uint4*>(st + Sm::KS + h_off(r, col, Sm::TILE)) = *reinterpret_cast<const uint4*>(hv);
-                }
-            }
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == kCopyThread) {
-#pragma unroll
-            for (int b = 0; b < DK / 64; ++b)   // W: rows 0..63 of each WQ tile
-                bulk_store(rec + R::WQ + b * 16384, st + Sm::KS + b * Sm::TILE, Sm::TILE);
-            bulk_store(rec + R::U0, st + Sm::VS, (DV / 64) * Sm::TILE);
-            bulk_store_commit();
-        }
-        tc_fence_before();
-        __syncthreads();   // R1/R2, TP and the stage are free for the next item
-    }
-
-    if (aborted) {
-        if (tid == 0) flag_error(hdr, kStatusTimeout);
-        // let this CTA's own copies and MMAs finish (bounded) before freeing:
-        // exactly the phases that were issued and not yet waited for
-        for (int j = loads_done; j < loads_issued; ++j) {
-            (void)mbar_wait_cycles(&bar_load[j & 1], (j >> 1) & 1, wait_cap / 4);
-            if constexpr (channel_gate) (void)mbar_wait_cycles(&bar_la, j & 1, wait_cap / 4);
-        }
-        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, wait_cap);
-    }
-    if (stored || tstored) bulk_store_wait_all();
-    if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
-}
-
-// ---------------------------------------------------------------- K2 ----
-constexpr int kSliceTc = 64;   // value columns per inter-chunk CTA
+// ------------------------------------------- record stage (reversed chain) ----
+constexpr int kSliceTc = 64;   // value columns per reversed-chain CTA
 
 template <int DK, int DV>
 struct K2Smem {
     using R = TcRec<DK, DV>;
-    // one stage: [WQ][KH][P][U0 slice][GC]; P directly after KH, so the
-    // 128-row A operand [*; P] reads the tail of KH as its (unused) rows 0..63
+    // one stage of a chunk's record: [WQ][KH][P][U0 slice][GC]; P directly after
+    // KH, so a 128-row A operand [*; P] reads the tail of KH as its (unused) rows 0..63
     static constexpr uint32_t WQ = 0;
     static constexpr uint32_t KH = WQ + R::WQ_BYTES;
     static constexpr uint32_t P = KH + R::KH_BYTES;
     static constexpr uint32_t U0 = P + 8192;
     static constexpr uint32_t GC = U0 + 8192;
     static constexpr uint32_t STAGE = (GC + DK * 4 + 1023) / 1024 * 1024;
-    static constexpr uint32_t S16 = 2 * STAGE;              // fp16 state slice, rows = key channel
-    static constexpr uint32_t U16 = S16 + 128 * 128;        // fp16 U, rows = token
-    static constexpr uint32_t END = U16 + 8192;
-    static constexpr uint32_t TX_BYTES = R::WQ_BYTES + R::KH_BYTES + 8192 + 8192 + DK * 4;
 };
-
-template <int DK, int DV>
-__global__ void __launch_bounds__(256, 1)
-inter_chunk_tc_kernel(const float* __restrict__ initial_state, float* __restrict__ final_state,
-                      __nv_bfloat16* __restrict__ o, ChunkMap map, WsHeader* hdr,
-                      const unsigned char* __restrict__ records, int H, size_t max_chunks, float scale,
-                      float* __restrict__ states)
-{
-    using Sm = K2Smem<DK, DV>;
-    using R = TcRec<DK, DV>;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar_full[2], bar_mma;
-    __shared__ uint32_t s_tmem;
-
-    if (hdr->status != kStatusOk) return;
-    const int s = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSliceTc;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int lane_row = (warp & 3) * 32 + (tid & 31);   // TMEM lane = MMA row
-    const int wg = warp >> 2;                            // warpgroup: columns [32 wg, 32 wg + 32)
-    const int first = map.seq_first_chunk(s), nch = map.seq_num_chunks(s);
-    const int tok_begin = map.seq_token_begin(s), tok_end = map.seq_token_end(s);
-    const size_t state_off = ((size_t)s * H + h) * DK * DV;
-
-    if (tid == 0) {
-        mbar_init(&bar_full[0], 1);
-        mbar_init(&bar_full[1], 1);
-        mbar_init(&bar_mma, 1);
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&s_tmem, 256);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
-    // [W S; Q~ S + P U] of chunk n at columns 64 (n & 1) (128 lanes x 64), then the state slice
-    auto r3 = [&](int n) -> uint32_t { return tmem + 64u * (uint32_t)(n & 1); };
-    const uint32_t SACC = tmem + 128;
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    float range_max = 0.f;
-
-    auto issue = [&](int n) {   // bulk-copy chunk n's intermediates into stage n & 1
-        if (n >= nch) return;
-        unsigned char* st = sm + (n & 1) * Sm::STAGE;
-        const unsigned char* rec = records + ((size_t)h * max_chunks + first + n) * R::BYTES;
-        uint64_t* bar = &bar_full[n & 1];
-        mbar_arrive_expect_tx(bar, Sm::TX_BYTES);
-        bulk_load(st + Sm::WQ, rec + R::WQ, R::WQ_BYTES, bar);
-        bulk_load(st + Sm::KH, rec + R::KH, R::KH_BYTES, bar);
-        bulk_load(st + Sm::P, rec + R::P, 8192, bar);
-        bulk_load(st + Sm::U0, rec + R::U0 + (j0 / 64) * 8192, 8192, bar);
-        bulk_load(st + Sm::GC, rec + R::GC, DK * 4, bar);
-    };
-    // fp16 copy of 32 state columns of this thread's key channel (row of S16)
-    auto put_s16 = [&](const float (&v)[32]) {
-#pragma unroll
-        for (int i8 = 0; i8 < 4; ++i8) {
-            __align__(16) __half2 hv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float a = v[8 * i8 + 2 * e], b = v[8 * i8 + 2 * e + 1];
-                range_max = fmaxf(range_max, fmaxf(fabsf(a), fabsf(b)));
-                hv[e] = __floats2half2_rn(a, b);
-            }
-            *reinterpret_cast<uint4*>(sm + Sm::S16 + sw128_offset(lane_row, (32 * wg + 8 * i8) * 2)) =
-                *reinterpret_cast<const uint4*>(hv);
-        }
-    };
-    // output rows (lanes 64..127) of chunk n from R3[n & 1]: warps 2, 3, 6, 7
-    auto write_o = [&](int n) {
-        const int r = lane_row - 64;
-        const int tok = tok_begin + n * kChunk + r;
-        float v[32];
-        tmem_ld32_sync(r3(n) + lane_base + 32 * wg, v);
-        if (o && tok < tok_end) {
-            __nv_bfloat16* dst = o + ((size_t)tok * H + h) * DV + j0 + 32 * wg;
-#pragma unroll
-            for (int i8 = 0; i8 < 4; ++i8) {
-                __align__(16) __nv_bfloat162 bv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    bv[e] = __floats2bfloat162_rn(scale * v[8 * i8 + 2 * e], scale * v[8 * i8 + 2 * e + 1]);
-                *reinterpret_cast<uint4*>(dst + 8 * i8) = *reinterpret_cast<const uint4*>(bv);
-            }
-        }
-    };
-
-    // initial state slice -> TMEM accumulator and fp16 operand copy
-    if (lane_row < DK) {
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (initial_state)
-                x = *reinterpret_cast<const float4*>(initial_state + state_off + (size_t)lane_row * DV + j0 + 32 * wg + i);
-            v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
-        }
-        tmem_st32_sync(SACC + lane_base + 32 * wg, v);
-        put_s16(v);
-    }
-    if (tid == 0) {
-        issue(0);
-        issue(1);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    bool aborted = false;
-    uint32_t mma_phase = 0;
-    int mma_pending = 0;   // a commit on bar_mma not yet waited for
-    // chunk j's records land on bar_full[j & 1] (phase parity (j >> 1) & 1);
-    // chunks copies_done .. copies_issued - 1 are in flight (drained on abort)
-    int copies_issued = nch < 2 ? nch : 2, copies_done = 0;
-    int n = 0;
-    for (; n < nch; ++n) {
-        const int b = n & 1;
-        unsigned char* st = sm + b * Sm::STAGE;
-        bool ok = mbar_wait_cycles(&bar_full[b], (n >> 1) & 1, kWaitCycles);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        copies_done = n + 1;
-
-        const uint32_t R3 = r3(n);
-        // MMA3: [W; Q~] S -> R3
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t idesc = instr_desc(kFmtF16, 128, kSliceTc, false, true);
-            const uint32_t a0 = smem_u32(st + Sm::WQ), b0 = smem_u32(sm + Sm::S16);
-#pragma unroll
-            for (int kb = 0; kb < DK / 64; ++kb)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(R3, smem_desc(a0 + kb * 16384 + ks * 32, 16, 1024, kLayoutSW128),
-                            smem_desc(b0 + kb * 8192 + ks * 2048, 8192, 1024, kLayoutSW128), idesc,
-                            (kb | ks) != 0);
-            mma_commit(&bar_mma);
-        }
-        // meanwhile: S_acc <- Diag(gC) S_acc (MMA3 reads the fp16 copy, not S_acc),
-        // and the previous chunk's output rows
-        if (lane_row < DK) {
-            const float gc = reinterpret_cast<const float*>(st + Sm::GC)[lane_row];
-            float v[32];
-            tmem_ld32_sync(SACC + lane_base + 32 * wg, v);
-            if (states) {   // backward mode: the state entering this chunk
-                float* dst = states + (((size_t)h * max_chunks + first + n) * DK + lane_row) * DV + j0 + 32 * wg;
-#pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= gc;
-            tmem_st32_sync(SACC + lane_base + 32 * wg, v);
-        }
-        if (n > 0 && lane_row >= 64) write_o(n - 1);
-        mma_pending = 1;
-        ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        mma_phase ^= 1;
-        mma_pending = 0;
-        tc_fence_after();
-
-        // U = U0 - W S  (rows 0..63 = tokens), fp16 -> U16
-        if (lane_row < 64) {
-            const int r = lane_row;
-            float v[32];
-            tmem_ld32_sync(R3 + lane_base + 32 * wg, v);
-#pragma unroll
-            for (int i8 = 0; i8 < 4; ++i8) {
-                const uint32_t off = sw128_offset(r, (32 * wg + 8 * i8) * 2);
-                const uint4 u0raw = *reinterpret_cast<const uint4*>(st + Sm::U0 + off);
-                const __half2* u0 = reinterpret_cast<const __half2*>(&u0raw);
-                __align__(16) __half2 hv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 u0f = __half22float2(u0[e]);
-                    const float ua = u0f.x - v[8 * i8 + 2 * e], ub = u0f.y - v[8 * i8 + 2 * e + 1];
-                    range_max = fmaxf(range_max, fmaxf(fabsf(ua), fabsf(ub)));
-                    hv[e] = __floats2half2_rn(ua, ub);
-                }
-                *reinterpret_cast<uint4*>(sm + Sm::U16 + off) = *reinterpret_cast<const uint4*>(hv);
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // MMA4: [*; P] U += R3 ; MMA5: K^^T U += S_acc
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t idesc = instr_desc(kFmtF16, 128, kSliceTc, false, true);
-            constexpr uint32_t idesc_t = instr_desc(kFmtF16, 128, kSliceTc, true, true);
-            const uint32_t pa = smem_u32(st + Sm::P) - 8192, ub = smem_u32(sm + Sm::U16);
-            const uint32_t ka = smem_u32(st + Sm::KH);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_f16(R3, smem_desc(pa + ks * 32, 16, 1024, kLayoutSW128),
-                        smem_desc(ub + ks * 2048, 8192, 1024, kLayoutSW128), idesc, true);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_f16(SACC, smem_desc(ka + ks * 2048, 8192, 1024, kLayoutSW128),
-                        smem_desc(ub + ks * 2048, 8192, 1024, kLayoutSW128), idesc_t, true);
-            mma_commit(&bar_mma);
-        }
-        mma_pending = 1;
-        ok = mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        mma_phase ^= 1;
-        mma_pending = 0;
-        tc_fence_after();
-        if (tid == 0) {
-            fence_proxy_async_smem();
-            issue(n + 2);   // this stage is no longer read
-        }
-        if (n + 2 < nch) copies_issued = n + 3;
-        // next state's fp16 operand copy (the serial path); the output rows of
-        // this chunk are written during the next chunk's MMA3
-        if (lane_row < DK) {
-            float v[32];
-            tmem_ld32_sync(SACC + lane_base + 32 * wg, v);
-            put_s16(v);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-    }
-
-    if (aborted) {
-        if (tid == 0) flag_error(hdr, kStatusTimeout);
-        // let MMAs and copies this CTA issued finish before its memory goes away
-        if (mma_pending) (void)mbar_wait_cycles(&bar_mma, mma_phase, kWaitCycles);
-        for (int j = copies_done; j < copies_issued; ++j)
-            (void)mbar_wait_cycles(&bar_full[j & 1], (j >> 1) & 1, kWaitCycles / 8);
-    } else {
-        if (nch > 0 && lane_row >= 64) write_o(nch - 1);
-        if (final_state && lane_row < DK) {
-            float v[32];
-            tmem_ld32_sync(SACC + lane_base + 32 * wg, v);
-            float* dst = final_state + state_off + (size_t)lane_row * DV + j0 + 32 * wg;
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-        }
-    }
-    if (range_max > kF16Limit) flag_error(hdr, kStatusRange);
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
-}
 
 // --------------------------------------------------- backward KB3 (bf16) ----
 // The backward's reversed chunk chain on the tensor cores (bf16 inputs), one
@@ -2208,53 +1350,6 @@ bwd_split_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
 // ------------------------------------------------------------- host -----
 template <int DK, int DV>
-cudaError_t launch_intra_tc_t(const ChunkArgs& a) {
-    if (a.max_chunks == 0) return cudaSuccess;
-    const int ntok = a.cu_seqlens ? a.T : a.B * a.T;
-    CUtensorMap mk, mv, mq, mla;
-    if (!make_map(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, a.H, ntok, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        (a.gate == kGateChannel &&
-         !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, ntok, DK, CU_TENSOR_MAP_SWIZZLE_NONE)))
-        return cudaErrorInvalidValue;
-    if (a.gate != kGateChannel) memset(&mla, 0, sizeof(mla));   // unused
-    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
-    auto kern = a.gate == kGateChannel ? intra_chunk_tc_kernel<DK, DV, kGateChannel>
-              : a.gate == kGateHead    ? intra_chunk_tc_kernel<DK, DV, kGateHead>
-                                       : intra_chunk_tc_kernel<DK, DV, kGateNone>;
-    const int smem = (int)K1Smem<DK, DV>::TOTAL;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const size_t items = a.max_chunks * (size_t)a.H;   // upper bound; the kernel reads the exact count
-    const unsigned grid = (unsigned)(items < (size_t)sms ? items : (size_t)sms);
-    kern<<<grid, 256, smem, a.stream>>>(mk, mv, mq, mla, a.log_alpha, a.beta, map,
-                                        static_cast<WsHeader*>(a.ws_header),
-                                        static_cast<unsigned char*>(a.records), a.H, a.max_chunks,
-                                        a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy,
-                                        static_cast<unsigned char*>(a.bwd_tiles), a.bwd_flags);
-    return cudaGetLastError();
-}
-
-template <int DK, int DV>
-cudaError_t launch_inter_tc_t(const ChunkArgs& a) {
-    ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
-    auto kern = inter_chunk_tc_kernel<DK, DV>;
-    const int smem = (int)K2Smem<DK, DV>::END + 1024;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)a.num_seqs, (unsigned)a.H, (unsigned)(DV / kSliceTc));
-    kern<<<grid, 256, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<__nv_bfloat16*>(a.o), map,
-                                        static_cast<WsHeader*>(a.ws_header),
-                                        static_cast<const unsigned char*>(a.records), a.H, a.max_chunks, a.scale,
-                                        a.states);
-    return cudaGetLastError();
-}
-
-template <int DK, int DV>
 cudaError_t launch_bwd_inter_tc_t(const ChunkArgs& a) {
     if (a.num_seqs == 0) return cudaSuccess;
     const int ntok = a.cu_seqlens ? a.T : a.B * a.T;
@@ -2372,18 +1467,16 @@ size_t tc_record_bytes(int dk, int dv) {
 }
 
 cudaError_t launch_chunk_intra_tc(const ChunkArgs& a) {
-    // the forward alone takes the two-CTA-per-SM kernel of kda_intra_tc.cu; the
-    // backward's recomputation (which also writes the backward tiles) this one
-    if (!a.bwd_tiles) return launch_chunk_intra_fwd_tc(a);
-    KDA_TC_DISPATCH(launch_intra_tc_t, a);
+    // the two-CTA-per-SM kernel of kda_intra_tc.cu, which also writes the
+    // backward tiles when a.bwd_tiles is set
+    return launch_chunk_intra_fwd_tc(a);
 }
 
 cudaError_t launch_chunk_inter_tc(const ChunkArgs& a) {
     if (a.num_seqs == 0) return cudaSuccess;
-    // the forward alone takes the slice-width-adaptive kernel of kda_inter_tc.cu;
-    // the backward's recomputation (which also writes the chunk-start states) this one
-    if (!a.states) return launch_chunk_inter_fwd_tc(a);
-    KDA_TC_DISPATCH(launch_inter_tc_t, a);
+    // the slice-width-adaptive kernel of kda_inter_tc.cu, which also writes the
+    // chunk-start states when a.states is set
+    return launch_chunk_inter_fwd_tc(a);
 }
 
 cudaError_t launch_chunk_bwd_inter_tc(const ChunkArgs& a) { KDA_TC_DISPATCH(launch_bwd_inter_tc_t, a); }

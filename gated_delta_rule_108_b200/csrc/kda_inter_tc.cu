@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(256, 1)
 inter_chunk_fwd_tc_kernel(const float* __restrict__ initial_state, float* __restrict__ final_state,
                           __nv_bfloat16* __restrict__ o, ChunkMap map, WsHeader* hdr,
                           const unsigned char* __restrict__ records, int H, size_t max_chunks, float scale,
-                          const int* __restrict__ seq_order)
+                          const int* __restrict__ seq_order, float* __restrict__ states)
 {
     using Sm = K2fSmem<DK, DV, NS>;
     using R = TcRec<DK, DV>;
@@ -248,11 +248,17 @@ inter_chunk_fwd_tc_kernel(const float* __restrict__ initial_state, float* __rest
         }
         mma_pending = 1;
         // meanwhile: S_acc <- Diag(gC) S_acc (MMA3 reads the fp16 copy, not S_acc),
-        // and the previous chunk's output rows
+        // and the previous chunk's output rows; backward mode: the state entering
+        // this chunk
         if (lane_row < DK) {
             const float gc = reinterpret_cast<const float*>(st + Sm::GC)[lane_row];
             float v[CPT];
             tmem_ld_cols<CPT>(SACC + lane_base + cb, v);
+            if (states) {
+                float* dst = states + (((size_t)h * max_chunks + first + n) * DK + lane_row) * DV + j0 + cb;
+#pragma unroll
+                for (int i = 0; i < CPT; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            }
 #pragma unroll
             for (int i = 0; i < CPT; ++i) v[i] *= gc;
             tmem_st_cols<CPT>(SACC + lane_base + cb, v);
@@ -367,7 +373,7 @@ cudaError_t launch_inter_fwd_tc_ns(const ChunkArgs& a) {
     kern<<<grid, 256, smem, a.stream>>>(a.initial_state, a.final_state, static_cast<__nv_bfloat16*>(a.o), map,
                                         static_cast<WsHeader*>(a.ws_header),
                                         static_cast<const unsigned char*>(a.records), a.H, a.max_chunks, a.scale,
-                                        a.seq_order);
+                                        a.seq_order, a.states);
     return cudaGetLastError();
 }
 

@@ -137,7 +137,7 @@ __device__ __forceinline__ uint32_t g_off(int r, int c) {
     return (uint32_t)(c >> 5) * 8192u + sw128_offset((uint32_t)r, (uint32_t)(c & 31) * 4u);
 }
 
-template <int DK, int DV, int GATE, bool FUSED>
+template <int DK, int DV, int GATE, bool FUSED, bool BWD>
 __global__ void __launch_bounds__(256, FUSED ? 1 : 2)
 intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_la,
@@ -145,10 +145,12 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                           ChunkMap map, WsHeader* hdr, unsigned char* __restrict__ records, int H,
                           size_t max_chunks, long long wait_cap, int drop_la,
                           const float* __restrict__ initial_state, float* __restrict__ final_state,
-                          __nv_bfloat16* __restrict__ o, float scale, const int* __restrict__ seq_order)
+                          __nv_bfloat16* __restrict__ o, float scale, const int* __restrict__ seq_order,
+                          unsigned char* __restrict__ bwd_tiles, int* __restrict__ bwd_flags)
 {
     using Sm = K1fSmem<DK, DV, FUSED>;
     using R = TcRec<DK, DV>;
+    using BT = BwdTiles<DK, DV>;
     constexpr int NPART = 256 / DK;       // threads per key channel in the scan
     constexpr int TPP = kChunk / NPART;   // tokens per such thread
     constexpr int CH = DK / 2;            // channels per thread in the element pass
@@ -268,6 +270,9 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         float* gc_dst = FUSED ? reinterpret_cast<float*>(sm + Sm::FGC) : reinterpret_cast<float*>(rec + R::GC);
         unsigned char* kh_dst = FUSED ? sm + Sm::FKH : rec + R::KH;
         unsigned char* p_dst = FUSED ? sm + Sm::FP : rec + R::P;
+        // backward mode (split form): T = (I + A)^{-1}, K~ and V as fp16 tiles and the
+        // unweighted M = K_l K_r^T for the backward's T-chain and split-factor kernels
+        unsigned char* btile = (BWD && !FUSED) ? bwd_tiles + ((size_t)h * max_chunks + c) * BT::BYTES : nullptr;
         if (tid >= 192) {
             s_beta[tid - 192] = beta_next;
             if constexpr (GATE == kGateHead) s_lah[tid - 192] = lah_next;
@@ -319,6 +324,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         // Strong decay: the factors e^{+-(g - g_m)} of A and P could overflow, so
         // this chunk forms A and P exactly (slow path, no MMA1).
         const bool strong = __syncthreads_or(wide);
+        if (BWD && !FUSED && tid == 0) bwd_flags[(size_t)h * max_chunks + c] = strong ? 1 : 0;
         float* am = reinterpret_cast<float*>(sm + Sm::AMS);   // strong path: [64][64]
         if (strong) {
             exact_a_p<DK>(gat, sm + Sm::KT, sm + Sm::QT, s_beta, L, am, p_dst, 64);
@@ -449,6 +455,8 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 #pragma unroll
                 for (int b = 0; b < DK / 64; ++b)
                     bulk_store(rec + R::WQ + b * 16384 + 8192, sm + Sm::QT + b * Sm::TILE, 8192);
+                if (btile)   // backward mode: K~ is final in KT
+                    bulk_store(btile + BT::KT, sm + Sm::KT, (DK / 64) * Sm::TILE);
                 bulk_store_commit();
                 stored = true;
                 bulk_store_wait_read();
@@ -509,6 +517,15 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             float v[32];
             tmem_ld32_sync(D1 + lane_base + 32 * hc, v);
             if (row < 64) {
+                if (btile) {   // backward mode: the unweighted, strictly lower M
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const int col = 32 * hc + 4 * i4;
+                        *reinterpret_cast<float4*>(btile + BT::M + (row * 64 + col) * 4) =
+                            make_float4(col < row ? v[4 * i4] : 0.f, col + 1 < row ? v[4 * i4 + 1] : 0.f,
+                                        col + 2 < row ? v[4 * i4 + 2] : 0.f, col + 3 < row ? v[4 * i4 + 3] : 0.f);
+                    }
+                }
                 const float b = s_beta[row];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = (32 * hc + i < row) ? b * v[i] : 0.f;
@@ -563,13 +580,17 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
                 reinterpret_cast<float*>(sm + Sm::DF)[b * 272 + j * 17 + cc] = x[j];
                 *reinterpret_cast<__half*>(sm + Sm::T1H + sw128_offset(base + j, (base + cc) * 2)) = __float2half_rn(x[j]);
                 put_t(base + j, base + cc, x[j]);
+                if (btile) *reinterpret_cast<__half*>(btile + BT::T + sw128_offset(base + j, (base + cc) * 2)) = __float2half_rn(x[j]);
             }
         } else {           // zero chunks: T1 off its diagonal and level-1 blocks, T diag(beta) above the diagonal
             for (int o = tid - 64; o < 64 * 8; o += 192) {
                 const int rr = o >> 3, c16 = o & 7, blk = c16 >> 1, rb = rr >> 4;
                 const bool l1 = (rb == 1 && blk == 0) || (rb == 3 && blk == 2);
                 if (blk != rb && !l1) *reinterpret_cast<uint4*>(sm + Sm::T1H + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
-                if (blk > rb) *reinterpret_cast<uint4*>(sm + Sm::TPV + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
+                if (blk > rb) {
+                    *reinterpret_cast<uint4*>(sm + Sm::TPV + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
+                    if (btile) *reinterpret_cast<uint4*>(btile + BT::T + sw128_offset(rr, c16 * 16)) = make_uint4(0u, 0u, 0u, 0u);
+                }
             }
         }
         // one 64 x 64 x 64 product D[0, 64) = A(128-row K-major operand) B(64 x 64, rows = K)
@@ -636,6 +657,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
             }
             const int rr = 16 * (2 * pp + 1) + i, cc = 16 * (2 * pp) + j0;
             *reinterpret_cast<__half2*>(sm + Sm::T1H + sw128_offset(rr, cc * 2)) = __floats2half2_rn(-t0, -t1);
+            if (btile) *reinterpret_cast<__half2*>(btile + BT::T + sw128_offset(rr, cc * 2)) = __floats2half2_rn(-t0, -t1);
             put_t(rr, cc, -t0);
             put_t(rr, cc + 1, -t1);
         }
@@ -654,6 +676,12 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
 #pragma unroll
                 for (int e = 0; e < 8; ++e) tb[e] = __float2half_rn(-v[8 * i8 + e] * s_beta[8 * i8 + e]);
                 *reinterpret_cast<uint4*>(sm + Sm::TPV + sw128_offset(row, 16 * i8)) = *reinterpret_cast<const uint4*>(tb);
+                if (btile) {
+                    __align__(16) __half tt[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) tt[e] = __float2half_rn(-v[8 * i8 + e]);
+                    *reinterpret_cast<uint4*>(btile + BT::T + sw128_offset(row, 16 * i8)) = *reinterpret_cast<const uint4*>(tt);
+                }
             }
         }
 
@@ -680,6 +708,11 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         tc_fence_before();
         __syncthreads();
 
+        if (btile && tid == kCopyThread) {   // backward mode: the fp16 V is final in VT
+            bulk_store(btile + BT::V, sm + Sm::VT, (DV / 64) * Sm::TILE);
+            bulk_store_commit();
+            stored = true;
+        }
         // ---- MMA2 (fp16): [T diag(beta); *] K~ -> D2[0, DK), [T diag(beta); *] V -> D2[DK, DK + DV)
         //      (the operand's rows 64..127 are KT's first 8 KB; their products are never read)
         if (tid == 0) {
@@ -705,6 +738,7 @@ intra_chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid
         tc_fence_after();
         // KT and V are free: the rest of the next item's inputs come in behind the write-out
         if (tid == kCopyThread && nc >= 0) {
+            if (btile) bulk_store_wait_read();   // the K~ / V tile stores have read KT and VT
             issue_k(nh, ntok0);
             issue_la(nh, ntok0, it + 1, false);
         }
@@ -1019,9 +1053,18 @@ cudaError_t launch_intra_fwd_tc_t(const ChunkArgs& a) {
           !make_map(&mla, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, a.H, ntok, 32, CU_TENSOR_MAP_SWIZZLE_128B))))
         return cudaErrorInvalidValue;
     ChunkMap map{a.cu_seqlens, a.chunk_offsets, a.num_seqs, a.T, a.fixed_chunks_per_seq};
-    auto kern = a.gate == kGateChannel ? intra_chunk_fwd_tc_kernel<DK, DV, kGateChannel, FUSED>
-              : a.gate == kGateHead    ? intra_chunk_fwd_tc_kernel<DK, DV, kGateHead, FUSED>
-                                       : intra_chunk_fwd_tc_kernel<DK, DV, kGateNone, FUSED>;
+    // backward mode (the split form with backward tiles) is its own instance, so
+    // the plain forward carries none of its stores
+    const bool bwd = !FUSED && a.bwd_tiles != nullptr;
+    auto kern = a.gate == kGateChannel ? intra_chunk_fwd_tc_kernel<DK, DV, kGateChannel, FUSED, false>
+              : a.gate == kGateHead    ? intra_chunk_fwd_tc_kernel<DK, DV, kGateHead, FUSED, false>
+                                       : intra_chunk_fwd_tc_kernel<DK, DV, kGateNone, FUSED, false>;
+    if constexpr (!FUSED) {
+        if (bwd)
+            kern = a.gate == kGateChannel ? intra_chunk_fwd_tc_kernel<DK, DV, kGateChannel, false, true>
+                 : a.gate == kGateHead    ? intra_chunk_fwd_tc_kernel<DK, DV, kGateHead, false, true>
+                                          : intra_chunk_fwd_tc_kernel<DK, DV, kGateNone, false, true>;
+    }
     const int smem = (int)K1fSmem<DK, DV, FUSED>::TOTAL;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -1044,7 +1087,8 @@ cudaError_t launch_intra_fwd_tc_t(const ChunkArgs& a) {
                                         static_cast<unsigned char*>(a.records), a.H, a.max_chunks,
                                         a.wait_cap > 0 ? a.wait_cap : kWaitCycles, a.debug_drop_copy,
                                         a.initial_state, a.final_state, static_cast<__nv_bfloat16*>(a.o), a.scale,
-                                        order);
+                                        order, bwd ? static_cast<unsigned char*>(a.bwd_tiles) : nullptr,
+                                        bwd ? a.bwd_flags : nullptr);
     return cudaGetLastError();
 }
 
