@@ -12,13 +12,14 @@
 //   W = T diag(beta) K~,  U0 = T diag(beta) V  (fp16 operands)
 //   records: W, Q~ = q e^{g}, K^ = k e^{g_{L-1} - g}, P, U0 (fp16), gamma_C (fp32)
 //
-// The records have the layout the inter-chunk kernel reads (TcRec).  Compared
-// with the intra-chunk kernel of kda_chunk_tc.cu (which also serves the
-// backward's recomputation), this one keeps MMA1's 128-row A operand in tensor
-// memory instead of 64 KB of shared memory, takes the log-decay tile in a
-// 128-byte-swizzled layout that both the per-channel scan and the per-row
-// element pass read without bank conflicts, and loads v only after the element
-// pass.  That brings a CTA to about 108 KB of shared memory, 256 TMEM columns
+// The records have the layout the inter-chunk kernel reads (TcRec).  In
+// backward mode (a separate instance) the kernel also writes what the backward
+// kernels read (BwdTiles: fp16 T, K~ and V tiles, the fp32 M = K_l K_r^T, a
+// strong-decay flag).  MMA1's 128-row A operand stays in tensor memory instead
+// of 64 KB of shared memory, the log-decay tile comes in a 128-byte-swizzled
+// layout that both the per-channel scan and the per-row element pass read
+// without bank conflicts, and v is loaded only after the element pass.  That
+// brings a CTA to about 108 KB of shared memory, 256 TMEM columns
 // and at most 128 registers per thread, so two CTAs share each SM and one item's
 // latency-bound phases (the (I + A)^{-1} solve, the TMEM round trips, the
 // copies) overlap the other CTA's work.
