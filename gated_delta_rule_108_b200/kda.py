@@ -136,6 +136,18 @@ def _stream_ptr(stream: Optional[torch.cuda.Stream], device) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _used_on(stream: Optional[torch.cuda.Stream], device, *tensors) -> None:
+    """Buffers the binding allocates come from the caching allocator on the
+    current stream.  When the call runs on another stream, mark them as used
+    there, so that their memory is not handed out again (after the caller, or
+    this function's return, drops them) before that stream's work is done."""
+    if stream is None or stream.cuda_stream == torch.cuda.current_stream(device).cuda_stream:
+        return
+    for t in tensors:
+        if t is not None:
+            t.record_stream(stream)
+
+
 def _need(t: torch.Tensor, name: str, dtype=None, device=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -254,14 +266,19 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
                      (final_state, "final_state", torch.float32)):
         if t is not None:
             _need(t, n, dt, dev)
+    made = []
     if o is None:
         o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
+        made.append(o)
     if final_state is None and output_final_state:
         final_state = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+        made.append(final_state)
     size_fn = chunk_bwd_workspace_size if _save else chunk_fwd_workspace_size
     ws_bytes = size_fn(B, T, H, dk, dv, N, cu_seqlens is not None, q.dtype)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+        made.append(workspace)
+    _used_on(stream, q.device, *made)
     call = lib().kda_chunk_fwd_save if _save else lib().kda_chunk_fwd_gated
     _check(call(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
@@ -342,8 +359,11 @@ def chunk_bwd(q, k, v, log_alpha, beta, d_o, initial_state=None, d_final_state=N
             raise ValueError(f"saved holds {saved.numel()} bytes; these sizes need {ws_bytes} "
                              "(it must come from chunk_fwd_train on the same inputs)")
         workspace, call = saved, lib().kda_chunk_bwd_saved
+    made = list(g.values())
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+        made.append(workspace)
+    _used_on(stream, q.device, *made)
     _check(call(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
         _ptr(cu_seqlens), _ptr(d_o), _ptr(d_final_state), B, T, H, dk, dv, N, _dtype_code(q), gate,
@@ -400,6 +420,7 @@ def recurrent_step(q, k, v, log_alpha, beta, state, o=None, stream=None) -> torc
         _need(o, "o", q.dtype, dev)
     if o is None:
         o = torch.empty(B, H, dv, dtype=q.dtype, device=q.device)
+        _used_on(stream, q.device, o)
     _check(lib().kda_recurrent_step_gated(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state),
         B, H, dk, dv, _dtype_code(q), gate, _ptr(o), _stream_ptr(stream, q.device)))

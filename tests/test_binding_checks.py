@@ -92,3 +92,29 @@ def test_recurrent_step_refuses_mismatched_tensors(name, bad):
         a[name] = bad
     with pytest.raises(ValueError, match=name):
         kda.recurrent_step(**a, o=o)
+
+
+def test_buffers_made_for_another_stream_are_marked_used_there(monkeypatch):
+    """A buffer the binding allocates (on the current stream) for a call that
+    runs on another stream is recorded on that stream, so the caching allocator
+    does not hand its memory out again while the call may still use it."""
+    class FakeStream:
+        def __init__(self, handle):
+            self.cuda_stream = handle
+
+    class FakeTensor:
+        def __init__(self):
+            self.recorded = []
+
+        def record_stream(self, s):
+            self.recorded.append(s)
+
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: FakeStream(1))
+    side, same = FakeStream(2), FakeStream(1)
+    a, b = FakeTensor(), FakeTensor()
+    kda._used_on(side, "cuda:0", a, None, b)
+    assert a.recorded == [side] and b.recorded == [side]
+    c = FakeTensor()
+    kda._used_on(same, "cuda:0", c)
+    kda._used_on(None, "cuda:0", c)
+    assert c.recorded == []

@@ -219,6 +219,47 @@ def test_chunk_equals_decode_steps(cuda_device):
     check(od, o_ref, torch.bfloat16, "decode loop o")
 
 
+def test_calls_on_a_side_stream(cuda_device):
+    """Every call can run on a stream other than the current one; the buffers
+    the binding allocates for it (o, states, gradients, workspace) stay
+    reserved for that stream until its work is done."""
+    w = I.ChunkWorkload("side", B=2, T=150, H=2, dk=128, dv=128, dtype=torch.bfloat16,
+                        s0_std=0.05, seed=25)
+    x = I.chunk_inputs(w)
+    g = to_dev(x)
+    cur, side = torch.cuda.current_stream(), torch.cuda.Stream()
+    side.wait_stream(cur)   # the inputs were written on the current stream
+    o, S = kda.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], g["initial_state"],
+                         stream=side)
+    cur.wait_stream(side)
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle_chunk(x)
+    check(o, o_ref, torch.bfloat16, "o")
+    check(S, S_ref, torch.bfloat16, "final_state")
+
+    d_o = torch.randn(o.shape, generator=torch.Generator().manual_seed(9)).to(o.dtype).cuda()
+    side.wait_stream(cur)
+    gs = kda.chunk_bwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], d_o,
+                       initial_state=g["initial_state"], stream=side)
+    cur.wait_stream(side)
+    gc = kda.chunk_bwd(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], d_o,
+                       initial_state=g["initial_state"])
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"):
+        assert rel_l2(gs[n].float().cpu(), gc[n].float().cpu()) < 1e-5, n
+
+    st_side, st_cur = S.clone(), S.clone()
+    t = lambda a: a[:, 0].contiguous()
+    side.wait_stream(cur)
+    o_side = kda.recurrent_step(t(g["q"]), t(g["k"]), t(g["v"]), t(g["log_alpha"]), t(g["beta"]),
+                                st_side, stream=side)
+    cur.wait_stream(side)
+    o_cur = kda.recurrent_step(t(g["q"]), t(g["k"]), t(g["v"]), t(g["log_alpha"]), t(g["beta"]), st_cur)
+    torch.cuda.synchronize()
+    assert rel_l2(o_side.float().cpu(), o_cur.float().cpu()) < 1e-6
+    assert rel_l2(st_side.cpu(), st_cur.cpu()) < 1e-6
+
+
 def test_split_sequence_carries_state(cuda_device):
     w = I.ChunkWorkload("split", B=2, T=300, H=2, dk=64, dv=128, dtype=torch.float32,
                         s0_std=0.05, seed=23)
