@@ -65,8 +65,9 @@ bool ws_layout(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, k
     } else {
         L.max_chunks = (size_t)B * L.chunks_per_seq;
     }
-    // bf16 inputs run on the tensor cores with fp16 records; fp32 inputs on
-    // CUDA cores with fp32 records.
+    // bf16 inputs: fp16 records; fp32 inputs: fp32 records, of one size for
+    // the split-tf32 tensor-core forward and for the CUDA-core kernels of the
+    // backward's recomputation.
     const size_t rec = dtype == KDA_BF16 ? kda::tc_record_bytes(dk, dv) : kda::simt_record_bytes(dk, dv);
     L.offsets_off = kda::kHeaderBytes;
     L.order_off = round_up(L.offsets_off + sizeof(int32_t) * ((size_t)N + 1), 256);
