@@ -199,8 +199,8 @@ kda_status kda_recurrent_step_gated(const void* q, const void* k, const void* v,
                                     kda_dtype dtype, kda_gate gate, void* o, void* stream);
 
 /*
- * kda_chunk_fwd without a caller-provided workspace.  The paper has no
- * counterpart to this call; it exists for callers that cannot allocate device
+ * kda_chunk_fwd without a caller-provided workspace.  The method itself has
+ * no counterpart to this call; it exists for callers that cannot allocate device
  * memory -- a plugin whose host framework owns all device memory and forbids
  * other allocations, a latency-critical loop that cannot afford cudaMalloc's
  * implicit synchronisation, or a tool with a fixed memory budget.
